@@ -1,0 +1,236 @@
+"""Python binding of the B200 hybrid GQA attention library (libhyb_attn.so).
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels behind the C ABI declared in include/hyb_attn.h.  PyTorch supplies
+device memory and streams.  There is no fallback: if the shared library is
+missing or the device is not a B200, calls raise.
+
+Functions keep the C names:
+    hyb_kv_cache_init, hyb_kv_append, hyb_attn_prefill, hyb_attn_decode,
+    hyb_attn_prefill_workspace_size, hyb_attn_decode_workspace_size,
+    hyb_device_error, hyb_launch_count
+plus the KVCache helper that allocates a layer's cache with torch.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+SLIDING = 0
+FULL = 1
+N_Q_HEADS = 16
+N_KV_HEADS = 4
+HEAD_DIM = 256
+WINDOW = 512
+N_LAYERS = 36
+
+DEV_ERR_CAPACITY = 1
+DEV_ERR_TIMEOUT = 2
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "_lib", "libhyb_attn.so")
+
+EXPORTED = (
+    "hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill_workspace_size", "hyb_attn_prefill",
+    "hyb_attn_decode_workspace_size", "hyb_attn_decode", "hyb_device_error", "hyb_last_error",
+    "hyb_launch_count",
+)
+
+
+def layer_type(i: int) -> int:
+    """Layer i is full attention iff i % 4 == 3 (3 sliding + 1 full, x9); past the schedule: full."""
+    if i >= N_LAYERS:
+        return FULL
+    return FULL if i % 4 == 3 else SLIDING
+
+
+class HybError(RuntimeError):
+    def __init__(self, status: int, msg: str):
+        super().__init__(f"hyb status {status}: {msg}")
+        self.status = status
+
+
+class _Cache(ctypes.Structure):
+    _fields_ = [
+        ("type", ctypes.c_int32), ("batch", ctypes.c_int32), ("capacity", ctypes.c_int64),
+        ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_void_p),
+        ("head", ctypes.c_void_p), ("tag", ctypes.c_void_p),
+    ]
+
+
+_lib = None
+
+
+def load(path: str = LIB_PATH):
+    """Loads the shared library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with __graft_entry__.build() "
+                           "or python full_gqa_attention_partial_b200/build.py")
+    lib = ctypes.CDLL(path)
+    vp, i32, i64, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_size_t
+    pc = ctypes.POINTER(_Cache)
+    lib.hyb_kv_cache_init.argtypes = [pc, vp, vp]
+    lib.hyb_kv_append.argtypes = [pc, vp, vp, i64, vp, i32, vp]
+    lib.hyb_attn_prefill_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.hyb_attn_prefill_workspace_size.restype = sz
+    lib.hyb_attn_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, i64, i64, vp, pc, vp, sz, vp]
+    lib.hyb_attn_decode_workspace_size.argtypes = [i32, i32, i64]
+    lib.hyb_attn_decode_workspace_size.restype = sz
+    lib.hyb_attn_decode.argtypes = [vp, vp, vp, pc, i32, i64, vp, vp, sz, vp]
+    lib.hyb_device_error.argtypes = [ctypes.POINTER(i32), i32, vp]
+    lib.hyb_last_error.restype = ctypes.c_char_p
+    lib.hyb_launch_count.restype = ctypes.c_uint64
+    for name in ("hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill", "hyb_attn_decode",
+                 "hyb_device_error"):
+        getattr(lib, name).restype = ctypes.c_int
+    _lib = lib
+    return lib
+
+
+def _check(status: int):
+    if status != 0:
+        raise HybError(status, load().hyb_last_error().decode())
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _row_stride(t: torch.Tensor, heads: int, name: str) -> int:
+    """Token stride (elements) of a [B, T, heads, 256] bf16 view whose rows are laid out densely per token."""
+    if t.dtype != torch.bfloat16 or t.dim() != 4 or t.shape[2] != heads or t.shape[3] != HEAD_DIM:
+        raise ValueError(f"{name} must be bf16 [B, T, {heads}, 256], got {tuple(t.shape)} {t.dtype}")
+    B, T = t.shape[:2]
+    if t.stride(3) != 1 or t.stride(2) != HEAD_DIM:
+        raise ValueError(f"{name}: heads must be dense 256-element rows")
+    rs = t.stride(1) if T > 1 else max(t.stride(1), heads * HEAD_DIM)
+    if B > 1 and t.stride(0) != T * rs:
+        raise ValueError(f"{name}: batch stride must equal T * token stride")
+    return rs
+
+
+# ---------------------------------------------------------------------------
+# KV cache
+# ---------------------------------------------------------------------------
+class KVCache:
+    """One layer's KV cache for `batch` sequences (memory from torch).
+
+    Full layers: linear cache of `capacity` tokens.  Sliding layers: 512-slot
+    ring; `head0` gives each sequence's starting write slot.
+    """
+
+    def __init__(self, layer_type: int, batch: int, capacity: int = WINDOW, device="cuda", head0=None,
+                 stream=None):
+        cap = WINDOW if layer_type == SLIDING else int(capacity)
+        self.layer_type = layer_type
+        self.batch = batch
+        self.capacity = cap
+        bf = torch.bfloat16
+        self.k = torch.empty(batch, N_KV_HEADS, cap, HEAD_DIM, dtype=bf, device=device)
+        self.v = torch.empty(batch, N_KV_HEADS, cap, HEAD_DIM, dtype=bf, device=device)
+        self.len = torch.empty(batch, dtype=torch.int32, device=device)
+        self.head = torch.empty(batch, dtype=torch.int32, device=device)
+        self.tag = torch.empty(batch, WINDOW, dtype=torch.int32, device=device)
+        self.c = _Cache(layer_type, batch, cap, self.k.data_ptr(), self.v.data_ptr(), self.len.data_ptr(),
+                        self.head.data_ptr(), self.tag.data_ptr())
+        hyb_kv_cache_init(self, head0, stream)
+
+    @property
+    def ref(self):
+        return ctypes.byref(self.c)
+
+
+def hyb_kv_cache_init(cache: KVCache, head0=None, stream=None):
+    h0 = None
+    if head0 is not None:
+        arr = (ctypes.c_int32 * cache.batch)(*[int(x) for x in head0])
+        h0 = ctypes.cast(arr, ctypes.c_void_p)
+    _check(load().hyb_kv_cache_init(cache.ref, h0, _stream(stream)))
+
+
+def hyb_kv_append(cache: KVCache, k: torch.Tensor, v: torch.Tensor, pos=None, stream=None):
+    """Appends k/v [B, T, 4, 256] (views into fused qkv rows allowed) to the cache."""
+    rs = _row_stride(k, N_KV_HEADS, "k")
+    if _row_stride(v, N_KV_HEADS, "v") != rs:
+        raise ValueError("k and v must share the token stride")
+    T = k.shape[1]
+    _check(load().hyb_kv_append(cache.ref, _ptr(k), _ptr(v), rs, _ptr(pos), T, _stream(stream)))
+
+
+def hyb_attn_prefill_workspace_size(layer_type: int, B: int, T: int, with_cache: bool) -> int:
+    return int(load().hyb_attn_prefill_workspace_size(layer_type, B, T, 1 if with_cache else 0))
+
+
+def hyb_attn_decode_workspace_size(layer_type: int, B: int, max_len: int) -> int:
+    return int(load().hyb_attn_decode_workspace_size(layer_type, B, max_len))
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    return torch.empty(max(int(nbytes), 256), dtype=torch.uint8, device=device)
+
+
+def hyb_attn_prefill(q, k, v, gate, pos, layer_type: int, out=None, cache: KVCache | None = None,
+                     workspace=None, stream=None):
+    """Prefill attention.  q [B,T,16,256], k/v [B,T,4,256], gate [B,T,16] or None,
+    pos [B,T] int32 or None.  Returns out [B,T,16,256] bf16."""
+    qs = _row_stride(q, N_Q_HEADS, "q")
+    ks = _row_stride(k, N_KV_HEADS, "k")
+    if _row_stride(v, N_KV_HEADS, "v") != ks:
+        raise ValueError("k and v must share the token stride")
+    B, T = q.shape[:2]
+    if gate is not None and (gate.dtype != torch.bfloat16 or not gate.is_contiguous()
+                             or tuple(gate.shape) != (B, T, N_Q_HEADS)):
+        raise ValueError("gate must be contiguous bf16 [B, T, 16]")
+    if pos is not None and (pos.dtype != torch.int32 or not pos.is_contiguous() or tuple(pos.shape) != (B, T)):
+        raise ValueError("pos must be contiguous int32 [B, T]")
+    if out is None:
+        out = torch.empty(B, T, N_Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
+    need = hyb_attn_prefill_workspace_size(layer_type, B, T, cache is not None)
+    if workspace is None and need > 0:
+        workspace = alloc_workspace(need, q.device)
+    wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    _check(load().hyb_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(pos), layer_type, B, T, qs, ks,
+                                   _ptr(out), None if cache is None else cache.ref, _ptr(workspace), wsz,
+                                   _stream(stream)))
+    return out
+
+
+def hyb_attn_decode(q, gate, cache: KVCache, pos=None, max_len: int = 0, out=None, workspace=None,
+                    stream=None):
+    """One decode step.  q [B,16,256] contiguous, gate [B,16] or None.  Returns out [B,16,256]."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous() or tuple(q.shape[1:]) != (N_Q_HEADS, HEAD_DIM):
+        raise ValueError("q must be contiguous bf16 [B, 16, 256]")
+    B = q.shape[0]
+    if gate is not None and (gate.dtype != torch.bfloat16 or not gate.is_contiguous()
+                             or tuple(gate.shape) != (B, N_Q_HEADS)):
+        raise ValueError("gate must be contiguous bf16 [B, 16]")
+    if out is None:
+        out = torch.empty_like(q)
+    ml = max_len if max_len else cache.capacity
+    if workspace is None:
+        workspace = alloc_workspace(hyb_attn_decode_workspace_size(cache.layer_type, cache.batch, ml), q.device)
+    wsz = workspace.numel() * workspace.element_size()
+    _check(load().hyb_attn_decode(_ptr(q), _ptr(gate), _ptr(pos), cache.ref, cache.layer_type, max_len,
+                                  _ptr(out), _ptr(workspace), wsz, _stream(stream)))
+    return out
+
+
+def hyb_device_error(clear: bool = True, stream=None) -> int:
+    flags = ctypes.c_int32(0)
+    _check(load().hyb_device_error(ctypes.byref(flags), 1 if clear else 0, _stream(stream)))
+    return int(flags.value)
+
+
+def hyb_launch_count() -> int:
+    return int(load().hyb_launch_count())

@@ -1,0 +1,412 @@
+// C-ABI layer (include/hyb_attn.h): argument checks, tensor-map encoding,
+// launch sequencing.  Host code only; every step of the computation runs in
+// the kernels of rope_kv.cu, prefill.cu and decode.cu.
+#include <cudaTypedefs.h>
+
+#include <atomic>
+#include <cstdarg>
+#include <cstdio>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "hyb_attn.h"
+#include "common.cuh"
+#include "launch.h"
+
+namespace hyb {
+
+static std::atomic<uint64_t> g_launches{0};
+void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
+
+cudaError_t decode_set_smem_attr();
+cudaError_t prefill_set_smem_attr();
+
+}  // namespace hyb
+
+using namespace hyb;
+
+namespace {
+
+thread_local std::string t_err;
+
+hyb_status fail(hyb_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  t_err = buf;
+  return s;
+}
+
+hyb_status cuda_fail(cudaError_t e, const char* what) {
+  return fail(HYB_ECUDA, "%s: %s", what, cudaGetErrorString(e));
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Per-device one-time set-up: architecture check and the dynamic shared
+// memory opt-in of the two large kernels.
+std::mutex g_mu;
+int g_dev_state[128];  // 0 unknown, 1 ready, -1 unsupported
+
+hyb_status ensure_device() {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= 128) return fail(HYB_EUNSUPPORTED, "device index %d out of range", dev);
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (g_dev_state[dev] == 1) return HYB_OK;
+  if (g_dev_state[dev] == -1) return fail(HYB_EUNSUPPORTED, "device %d is not an sm_100 (B200) GPU", dev);
+  int major = 0, minor = 0;
+  cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+  cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+  if (major != 10 || minor != 0) {
+    g_dev_state[dev] = -1;
+    return fail(HYB_EUNSUPPORTED, "device %d has compute capability %d.%d; this library is built for sm_100a",
+                dev, major, minor);
+  }
+  if ((e = prefill_set_smem_attr()) != cudaSuccess) return cuda_fail(e, "prefill smem attribute");
+  if ((e = decode_set_smem_attr()) != cudaSuccess) return cuda_fail(e, "decode smem attribute");
+  g_dev_state[dev] = 1;
+  return HYB_OK;
+}
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 4-D map {256 dims, rows, 4 KV heads, batch} of bf16 with 64 x 64 boxes and
+// 128-byte swizzle (one box = 64 rows of 128 bytes).
+hyb_status make_kv_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t batch, uint64_t row_bytes,
+                       uint64_t head_bytes, uint64_t batch_bytes, const char* what) {
+  auto enc = encode_fn();
+  if (!enc) return fail(HYB_EUNSUPPORTED, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[4] = {(cuuint64_t)kD, rows, (cuuint64_t)kHkv, batch};
+  cuuint64_t strides[3] = {row_bytes, head_bytes, batch_bytes};
+  cuuint32_t box[4] = {64, 64, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HYB_ECUDA, "cuTensorMapEncodeTiled(%s) failed with CUresult %d", what, (int)r);
+  return HYB_OK;
+}
+
+hyb_status check_cache(const hyb_kv_cache* c) {
+  if (!c) return fail(HYB_EINVAL, "cache is NULL");
+  if (c->type != HYB_SLIDING && c->type != HYB_FULL) return fail(HYB_EINVAL, "cache type %d invalid", c->type);
+  if (c->batch <= 0) return fail(HYB_EINVAL, "cache batch %d must be positive", c->batch);
+  if (!c->k || !c->v || !c->len) return fail(HYB_EINVAL, "cache k, v and len must be non-NULL");
+  if (!aligned16(c->k) || !aligned16(c->v)) return fail(HYB_EALIGN, "cache k/v must be 16-byte aligned");
+  if ((reinterpret_cast<uintptr_t>(c->len) & 3u) != 0) return fail(HYB_EALIGN, "cache len must be 4-byte aligned");
+  if (c->type == HYB_SLIDING) {
+    if (c->capacity != kWindow) return fail(HYB_ESHAPE, "sliding cache capacity must be 512, got %lld",
+                                            (long long)c->capacity);
+    if (!c->head || !c->tag) return fail(HYB_EINVAL, "sliding cache needs head and tag buffers");
+  } else {
+    if (c->capacity <= 0 || c->capacity > (int64_t)0x7fffffff)
+      return fail(HYB_ESHAPE, "full cache capacity %lld out of range [1, 2^31)", (long long)c->capacity);
+  }
+  return HYB_OK;
+}
+
+hyb_status cache_maps(const hyb_kv_cache* c, CUtensorMap* mk, CUtensorMap* mv) {
+  const uint64_t row = kD * 2, head = (uint64_t)c->capacity * row, batch = head * kHkv;
+  hyb_status s = make_kv_map(mk, c->k, (uint64_t)c->capacity, (uint64_t)c->batch, row, head, batch, "cache K");
+  if (s != HYB_OK) return s;
+  return make_kv_map(mv, c->v, (uint64_t)c->capacity, (uint64_t)c->batch, row, head, batch, "cache V");
+}
+
+cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
+
+size_t ctx_rows(int32_t T) { return (size_t)(kWindow - 1) + (size_t)T; }
+
+}  // namespace
+
+extern "C" {
+
+const char* hyb_last_error(void) { return t_err.c_str(); }
+
+uint64_t hyb_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+hyb_status hyb_device_error(int32_t* flags, int32_t clear, void* stream) {
+  if (!flags) return fail(HYB_EINVAL, "flags is NULL");
+  cudaError_t e = cudaStreamSynchronize(as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int v = 0;
+  if ((e = cudaMemcpyFromSymbol(&v, g_dev_err, sizeof(int))) != cudaSuccess) return cuda_fail(e, "read error word");
+  *flags = v;
+  if (clear) {
+    const int zero = 0;
+    if ((e = cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int))) != cudaSuccess)
+      return cuda_fail(e, "clear error word");
+  }
+  return HYB_OK;
+}
+
+hyb_status hyb_kv_cache_init(const hyb_kv_cache* c, const int32_t* head0, void* stream) {
+  hyb_status s = check_cache(c);
+  if (s != HYB_OK) return s;
+  if ((s = ensure_device()) != HYB_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  const size_t kv_bytes = (size_t)c->batch * kHkv * (size_t)c->capacity * kD * 2;
+  cudaError_t e;
+  if ((e = cudaMemsetAsync(c->k, 0, kv_bytes, st)) != cudaSuccess) return cuda_fail(e, "zero cache K");
+  if ((e = cudaMemsetAsync(c->v, 0, kv_bytes, st)) != cudaSuccess) return cuda_fail(e, "zero cache V");
+  if ((e = cudaMemsetAsync(c->len, 0, sizeof(int32_t) * c->batch, st)) != cudaSuccess) return cuda_fail(e, "len");
+  if (c->type == HYB_SLIDING) {
+    if ((e = launch_fill_i32(c->tag, (int64_t)c->batch * kWindow, -1, st)) != cudaSuccess)
+      return cuda_fail(e, "tag fill");
+    if (head0) {
+      for (int b = 0; b < c->batch; ++b)
+        if (head0[b] < 0 || head0[b] >= kWindow) return fail(HYB_ESHAPE, "head0[%d] = %d outside [0,512)", b, head0[b]);
+      if ((e = cudaMemcpyAsync(c->head, head0, sizeof(int32_t) * c->batch, cudaMemcpyHostToDevice, st)) !=
+          cudaSuccess)
+        return cuda_fail(e, "head upload");
+      // head0 is pageable host memory: make sure it has been read before returning
+      if ((e = cudaStreamSynchronize(st)) != cudaSuccess) return cuda_fail(e, "head upload sync");
+    } else if ((e = cudaMemsetAsync(c->head, 0, sizeof(int32_t) * c->batch, st)) != cudaSuccess) {
+      return cuda_fail(e, "head");
+    }
+  }
+  return HYB_OK;
+}
+
+hyb_status hyb_kv_append(const hyb_kv_cache* c, const void* k, const void* v, int64_t kv_row_stride,
+                         const int32_t* pos, int32_t T, void* stream) {
+  hyb_status s = check_cache(c);
+  if (s != HYB_OK) return s;
+  if (!k || !v) return fail(HYB_EINVAL, "k and v must be non-NULL");
+  if (T <= 0) return fail(HYB_EINVAL, "T = %d must be positive", T);
+  if (!aligned16(k) || !aligned16(v)) return fail(HYB_EALIGN, "k/v must be 16-byte aligned");
+  if (kv_row_stride < kHkv * kD || kv_row_stride % 8 != 0)
+    return fail(HYB_EALIGN, "kv_row_stride %lld must be >= 1024 and a multiple of 8 elements",
+                (long long)kv_row_stride);
+  if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u)) return fail(HYB_EALIGN, "pos must be 4-byte aligned");
+  if ((s = ensure_device()) != HYB_OK) return s;
+  cudaStream_t st = as_stream(stream);
+  const bool full = c->type == HYB_FULL;
+  RopeStoreHost r;
+  r.k = k;
+  r.v = v;
+  r.src_bstride = (int64_t)T * kv_row_stride;
+  r.src_tstride = kv_row_stride;
+  r.src_hstride = kD;
+  r.pos = pos;
+  r.dk = c->k;
+  r.dv = c->v;
+  r.dst_rows = c->capacity;
+  r.mode = full ? 0 : 1;
+  r.len = c->len;
+  r.head = c->head;
+  r.tag = c->tag;
+  r.B = c->batch;
+  r.T = T;
+  r.t_first = full ? 0 : (T > kWindow ? T - kWindow : 0);
+  cudaError_t e = launch_rope_store(full, r, st);
+  if (e != cudaSuccess) return cuda_fail(e, "append launch");
+  if ((e = launch_kv_commit(c->len, c->head, c->capacity, !full, c->batch, T, st)) != cudaSuccess)
+    return cuda_fail(e, "commit launch");
+  return HYB_OK;
+}
+
+size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache) {
+  if (B <= 0 || T <= 0) return 0;
+  const size_t row = (size_t)kHkv * kD * 2;  // one token of K (or V), 4 heads
+  if (!with_cache) return (size_t)B * (size_t)T * row;                  // rotated K
+  if (layer_type == HYB_FULL) return 0;                                  // reads the cache in place
+  return 2 * (size_t)B * ctx_rows(T) * row;                              // context K and V
+}
+
+hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const void* gate, const int32_t* pos,
+                            int32_t layer_type, int32_t B, int32_t T, int64_t q_row_stride,
+                            int64_t kv_row_stride, void* out, const hyb_kv_cache* cache, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  if (!q || !k || !v || !out) return fail(HYB_EINVAL, "q, k, v and out must be non-NULL");
+  if (layer_type != HYB_SLIDING && layer_type != HYB_FULL) return fail(HYB_EINVAL, "layer_type %d invalid", layer_type);
+  if (B <= 0 || T <= 0) return fail(HYB_EINVAL, "B = %d and T = %d must be positive", B, T);
+  if ((int64_t)T + kWindow > (int64_t)0x7fffffff) return fail(HYB_EOVERFLOW, "T = %d too large", T);
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(out))
+    return fail(HYB_EALIGN, "q, k, v and out must be 16-byte aligned");
+  if (q_row_stride < kHq * kD || q_row_stride % 8 != 0)
+    return fail(HYB_EALIGN, "q_row_stride %lld must be >= 4096 and a multiple of 8 elements", (long long)q_row_stride);
+  if (kv_row_stride < kHkv * kD || kv_row_stride % 8 != 0)
+    return fail(HYB_EALIGN, "kv_row_stride %lld must be >= 1024 and a multiple of 8 elements",
+                (long long)kv_row_stride);
+  if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
+  if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u)) return fail(HYB_EALIGN, "pos must be 4-byte aligned");
+  hyb_status s;
+  if (cache) {
+    if ((s = check_cache(cache)) != HYB_OK) return s;
+    if (cache->type != layer_type)
+      return fail(HYB_ESHAPE, "cache type %d differs from layer_type %d", cache->type, layer_type);
+    if (cache->batch != B) return fail(HYB_ESHAPE, "cache batch %d differs from B = %d", cache->batch, B);
+    if (layer_type == HYB_FULL && (int64_t)T > cache->capacity)
+      return fail(HYB_ESHAPE, "T = %d exceeds the cache capacity %lld", T, (long long)cache->capacity);
+  }
+  const size_t need = hyb_attn_prefill_workspace_size(layer_type, B, T, cache != nullptr);
+  if (need > 0) {
+    if (!workspace) return fail(HYB_EINVAL, "workspace of %zu bytes required", need);
+    if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(HYB_EALIGN, "workspace must be 256-byte aligned");
+    if (workspace_bytes < need)
+      return fail(HYB_EOVERFLOW, "workspace of %zu bytes given, %zu required", workspace_bytes, need);
+  }
+  if ((s = ensure_device()) != HYB_OK) return s;
+
+  cudaStream_t st = as_stream(stream);
+  const bool full = layer_type == HYB_FULL;
+  const uint64_t row_bytes = kD * 2;
+  PrefillHost ph;
+  ph.q = q;
+  ph.q_stride = q_row_stride;
+  ph.gate = gate;
+  ph.pos = pos;
+  ph.out = out;
+  ph.B = B;
+  ph.T = T;
+  cudaError_t e;
+
+  RopeStoreHost r;  // new tokens, token-major input rows
+  r.k = k;
+  r.src_bstride = (int64_t)T * kv_row_stride;
+  r.src_tstride = kv_row_stride;
+  r.src_hstride = kD;
+  r.pos = pos;
+  r.B = B;
+  r.T = T;
+
+  if (!cache) {
+    // rotated K into the workspace [B][4][T][256]; V is read in place
+    r.dk = workspace;
+    r.dst_rows = T;
+    r.mode = 2;
+    if ((e = launch_rope_store(full, r, st)) != cudaSuccess) return cuda_fail(e, "rope K launch");
+    const uint64_t hb = (uint64_t)T * row_bytes;
+    if ((s = make_kv_map(&ph.tm_k, workspace, T, B, row_bytes, hb, hb * kHkv, "rotated K")) != HYB_OK) return s;
+    if ((s = make_kv_map(&ph.tm_v, v, T, B, (uint64_t)kv_row_stride * 2, row_bytes,
+                         (uint64_t)T * kv_row_stride * 2, "V")) != HYB_OK)
+      return s;
+    if ((e = launch_prefill(full, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
+    return HYB_OK;
+  }
+
+  if (full) {
+    // append first (rows len .. len+T-1), attend over [0, len+T), then advance len
+    r.v = v;
+    r.dk = cache->k;
+    r.dv = cache->v;
+    r.dst_rows = cache->capacity;
+    r.mode = 0;
+    r.len = cache->len;
+    if ((e = launch_rope_store(true, r, st)) != cudaSuccess) return cuda_fail(e, "append launch");
+    if ((s = cache_maps(cache, &ph.tm_k, &ph.tm_v)) != HYB_OK) return s;
+    ph.qbase = cache->len;
+    ph.ctx_mode = 0;
+    if ((e = launch_prefill(true, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
+    if ((e = launch_kv_commit(cache->len, cache->head, cache->capacity, false, B, T, st)) != cudaSuccess)
+      return cuda_fail(e, "commit launch");
+    return HYB_OK;
+  }
+
+  // sliding layer with a ring: context = ring's last 511 tokens + the chunk,
+  // attend, then write the chunk's last 512 tokens into the ring.
+  const size_t rows = ctx_rows(T);
+  uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
+  void* ck = ws;
+  void* cv = ws + (size_t)B * rows * kHkv * row_bytes;
+  if ((e = launch_ring_gather(cache->k, cache->v, cache->len, cache->head, cache->tag, ck, cv, (int64_t)rows, B,
+                              st)) != cudaSuccess)
+    return cuda_fail(e, "ring gather launch");
+  r.v = v;
+  r.dk = ck;
+  r.dv = cv;
+  r.dst_rows = (int64_t)rows;
+  r.dst_row_offset = kWindow - 1;
+  r.mode = 2;
+  r.len = cache->len;  // default positions: len + t
+  if ((e = launch_rope_store(false, r, st)) != cudaSuccess) return cuda_fail(e, "context rope launch");
+  const uint64_t hb = (uint64_t)rows * row_bytes;
+  if ((s = make_kv_map(&ph.tm_k, ck, rows, B, row_bytes, hb, hb * kHkv, "context K")) != HYB_OK) return s;
+  if ((s = make_kv_map(&ph.tm_v, cv, rows, B, row_bytes, hb, hb * kHkv, "context V")) != HYB_OK) return s;
+  ph.qbase = cache->len;
+  ph.ctx_mode = 1;
+  if ((e = launch_prefill(false, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
+
+  RopeStoreHost w;  // ring append from the context rows (already rotated)
+  w.k = reinterpret_cast<const uint8_t*>(ck) + (size_t)(kWindow - 1) * row_bytes;
+  w.v = reinterpret_cast<const uint8_t*>(cv) + (size_t)(kWindow - 1) * row_bytes;
+  w.src_bstride = (int64_t)kHkv * (int64_t)rows * kD;
+  w.src_tstride = kD;
+  w.src_hstride = (int64_t)rows * kD;
+  w.src_rotated = 1;
+  w.dk = cache->k;
+  w.dv = cache->v;
+  w.dst_rows = kWindow;
+  w.mode = 1;
+  w.len = cache->len;
+  w.head = cache->head;
+  w.tag = cache->tag;
+  w.B = B;
+  w.T = T;
+  w.t_first = T > kWindow ? T - kWindow : 0;
+  if ((e = launch_rope_store(false, w, st)) != cudaSuccess) return cuda_fail(e, "ring append launch");
+  if ((e = launch_kv_commit(cache->len, cache->head, cache->capacity, true, B, T, st)) != cudaSuccess)
+    return cuda_fail(e, "commit launch");
+  return HYB_OK;
+}
+
+size_t hyb_attn_decode_workspace_size(int32_t layer_type, int32_t B, int64_t max_len) {
+  if (B <= 0) return 0;
+  const int S = decode_num_splits(layer_type == HYB_FULL, B, max_len);
+  const size_t rows = (size_t)B * kHq * (size_t)S;
+  return rows * kD * sizeof(float) + ((rows * sizeof(float) + 255) & ~size_t(255));
+}
+
+hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos, const hyb_kv_cache* c,
+                           int32_t layer_type, int64_t max_len, void* out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  hyb_status s = check_cache(c);
+  if (s != HYB_OK) return s;
+  if (!q || !out) return fail(HYB_EINVAL, "q and out must be non-NULL");
+  if (layer_type != c->type) return fail(HYB_ESHAPE, "layer_type %d differs from the cache type %d", layer_type, c->type);
+  if (!aligned16(q) || !aligned16(out)) return fail(HYB_EALIGN, "q and out must be 16-byte aligned");
+  if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
+  if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u)) return fail(HYB_EALIGN, "pos must be 4-byte aligned");
+  if (max_len < 0 || max_len > c->capacity)
+    return fail(HYB_ESHAPE, "max_len %lld outside [0, capacity %lld]", (long long)max_len, (long long)c->capacity);
+  if (max_len == 0) max_len = c->capacity;
+  const size_t need = hyb_attn_decode_workspace_size(layer_type, c->batch, max_len);
+  if (!workspace) return fail(HYB_EINVAL, "workspace of %zu bytes required", need);
+  if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(HYB_EALIGN, "workspace must be 256-byte aligned");
+  if (workspace_bytes < need) return fail(HYB_EOVERFLOW, "workspace of %zu bytes given, %zu required", workspace_bytes, need);
+  if ((s = ensure_device()) != HYB_OK) return s;
+
+  DecodeHost d;
+  if ((s = cache_maps(c, &d.tm_k, &d.tm_v)) != HYB_OK) return s;
+  d.q = q;
+  d.gate = gate;
+  d.pos = pos;
+  d.len = c->len;
+  d.tag = c->type == HYB_SLIDING ? c->tag : nullptr;
+  d.out = out;
+  d.B = c->batch;
+  d.n_splits = decode_num_splits(layer_type == HYB_FULL, c->batch, max_len);
+  d.part_o = reinterpret_cast<float*>(workspace);
+  d.part_lse = d.part_o + (size_t)c->batch * kHq * d.n_splits * kD;
+  cudaError_t e = launch_decode(layer_type == HYB_FULL, d, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return HYB_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,69 @@
+// Host-side interface between the C-ABI layer (api.cu) and the kernel files.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace hyb {
+
+void count_launch();
+
+// ---- KV side (rope_kv.cu) --------------------------------------------------
+struct RopeStoreHost {
+  const void* k = nullptr;
+  const void* v = nullptr;
+  int64_t src_bstride = 0, src_tstride = 0, src_hstride = 0;  // elements
+  int src_rotated = 0;
+  const int32_t* pos = nullptr;
+  void* dk = nullptr;
+  void* dv = nullptr;
+  int64_t dst_rows = 0;
+  int dst_row_offset = 0;
+  int mode = 0;  // 0 linear cache, 1 ring, 2 plain rows
+  const int32_t* len = nullptr;
+  const int32_t* head = nullptr;
+  int32_t* tag = nullptr;
+  int B = 0, T = 0, t_first = 0;
+};
+cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st);
+cudaError_t launch_ring_gather(const void* rk, const void* rv, const int32_t* len, const int32_t* head,
+                               const int32_t* tag, void* ck, void* cv, int64_t ctx_rows, int B,
+                               cudaStream_t st);
+cudaError_t launch_kv_commit(int32_t* len, int32_t* head, int64_t capacity, bool ring, int B, int T,
+                             cudaStream_t st);
+cudaError_t launch_fill_i32(int32_t* p, int64_t n, int32_t v, cudaStream_t st);
+
+// ---- prefill attention (prefill.cu) -----------------------------------------
+struct PrefillHost {
+  CUtensorMap tm_k, tm_v;      // 4-D maps {256, rows, 4, B}, 64x64 boxes, 128B swizzle
+  const void* q = nullptr;     // raw queries
+  int64_t q_stride = 0;        // elements between tokens
+  const void* gate = nullptr;  // [B][T][16] or null
+  const int32_t* pos = nullptr;
+  void* out = nullptr;         // [B][T][16][256]
+  const int32_t* qbase = nullptr;  // [B] sequence index of token 0, or null (0)
+  int ctx_mode = 0;            // 1: key row j holds sequence index qbase - 511 + j
+  int B = 0, T = 0;
+};
+cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st);
+size_t prefill_smem_bytes();
+
+// ---- decode (decode.cu) -------------------------------------------------------
+struct DecodeHost {
+  CUtensorMap tm_k, tm_v;      // 4-D maps over the cache {256, capacity, 4, B}
+  const void* q = nullptr;     // [B][16][256]
+  const void* gate = nullptr;  // [B][16] or null
+  const int32_t* pos = nullptr;
+  const int32_t* len = nullptr;
+  const int32_t* tag = nullptr;  // ring tags (sliding) or null
+  void* out = nullptr;
+  float* part_o = nullptr;     // [B][16][S][256]
+  float* part_lse = nullptr;   // [B][16][S]
+  int B = 0, n_splits = 1;
+};
+cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st);
+int decode_num_splits(bool full, int B, int64_t max_len);
+size_t decode_smem_bytes();
+
+}  // namespace hyb

@@ -1,0 +1,232 @@
+// KV-side kernels: rotate keys and place them (with the values) where the
+// attention kernels read them, plus the KV-cache bookkeeping.
+//
+//   * linear append (full layers): token i of a sequence -> slot i;
+//   * ring append (sliding layers): token i -> slot (head0 + i) % 512, only the
+//     last 512 tokens of a call are written, each slot tagged with the
+//     sequence index it holds ("keep only the most recent 512 tokens":
+//     "不用高显存卡也能跑！..." §"百万上下文的真正瓶颈");
+//   * rotated-key scratch for a cache-less prefill;
+//   * the sliding-layer context buffer of a chunked prefill: the ring's last
+//     511 tokens in sequence order followed by the chunk's own keys;
+//   * the commit step that advances len / head once all writes are done.
+//
+// Keys are rotated with rotate-half RoPE ("百万 Token 塞进 4B ..." §"滑动窗口
+// 的补救：分层 RoPE 与局部/全局分工"): sliding layers theta 1e4 over all 256
+// dims, full layers theta 5e6 over the first 64 dims.
+#include "common.cuh"
+#include "launch.h"
+
+namespace hyb {
+
+// Where a key row goes.
+enum DstMode : int {
+  kDstLinear = 0,   // cache slot len[b] + t, capacity checked
+  kDstRing = 1,     // cache slot (head[b] + t) % 512 for the last 512 tokens, tag written
+  kDstRows = 2,     // dst row t (+ row offset) of a [B][4][rows][256] buffer
+};
+
+struct RopeStoreArgs {
+  const __nv_bfloat16* k;   // source: token t, KV head h of sequence b at
+  const __nv_bfloat16* v;   //   b*src_bstride + t*src_tstride + h*src_hstride (elements)
+  int64_t src_bstride, src_tstride, src_hstride;   // v may be null: values not copied
+  int src_rotated;          // 1: k is already rotated (copy as is)
+  const int32_t* pos;       // [B][T] RoPE positions or null (sequence index)
+  __nv_bfloat16* dk;        // destination [B][4][dst_rows][256]
+  __nv_bfloat16* dv;
+  int64_t dst_rows;
+  int dst_row_offset;       // kDstRows: first destination row
+  int mode;
+  const int32_t* len;       // cache bookkeeping (linear / ring) and default positions
+  const int32_t* head;
+  int32_t* tag;
+  int B, T;
+  int t_first;              // first token index written (ring: max(0, T - 512))
+};
+
+// One block = one token of one sequence, 128 threads; thread i handles
+// 8 consecutive dims (16 bytes) of KV head i / 32.  Rotation partners
+// (k, k + R/2) sit in lanes i and i ^ 16 (R = 256) or i ^ 4 (R = 64).
+template <bool FULL>
+__global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
+  constexpr int R = RopeCfg<FULL>::R;
+  __shared__ double inv_freq[R / 2];
+  for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq(RopeCfg<FULL>::theta, i, R);
+  __syncthreads();
+
+  const int n_tok = a.T - a.t_first;
+  const int lane32 = threadIdx.x & 31;
+  const int kvh = threadIdx.x >> 5;
+  const int d0 = lane32 * 8;
+  for (int job = blockIdx.x; job < a.B * n_tok; job += gridDim.x) {
+    const int b = job / n_tok;
+    const int t = a.t_first + job % n_tok;
+    const int64_t src = (int64_t)b * a.src_bstride + (int64_t)t * a.src_tstride + (int64_t)kvh * a.src_hstride + d0;
+    int64_t dst_row;
+    const int L = (a.len != nullptr) ? a.len[b] : 0;
+    if (a.mode == kDstLinear) {
+      if ((int64_t)L + a.T > a.dst_rows) {  // capacity exceeded: leave the sequence unchanged
+        if (t == a.t_first && threadIdx.x == 0) raise_err(kErrCapacity);
+        continue;
+      }
+      dst_row = L + t;
+    } else if (a.mode == kDstRing) {
+      const int slot = (a.head[b] + t) % kWindow;
+      dst_row = slot;
+      if (threadIdx.x == 0) a.tag[(int64_t)b * kWindow + slot] = L + t;
+    } else {
+      dst_row = a.dst_row_offset + t;
+    }
+    const int64_t dst = (((int64_t)b * kHkv + kvh) * a.dst_rows + dst_row) * kD + d0;
+
+    uint4 kx = *reinterpret_cast<const uint4*>(a.k + src);
+    if (!a.src_rotated) {
+      const int p = a.pos ? a.pos[(int64_t)b * a.T + t] : L + t;
+      const uint32_t xs[4] = {kx.x, kx.y, kx.z, kx.w};
+      uint32_t ys[4];
+      constexpr int xor_mask = (R == 256) ? 16 : 4;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) ys[w] = __shfl_xor_sync(0xffffffffu, xs[w], xor_mask);
+      if (d0 < R) {
+        const bool first_half = d0 < R / 2;
+        const int kbase = first_half ? d0 : d0 - R / 2;
+        uint32_t os[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          float o2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float x = e ? bf16hi(xs[w]) : bf16lo(xs[w]);
+            const float y = e ? bf16hi(ys[w]) : bf16lo(ys[w]);
+            float s, c;
+            rope_sincos(p, inv_freq[kbase + 2 * w + e], &s, &c);
+            // first half: x cos - y sin (y = x[k + R/2]); second half: x cos + y sin (y = x[k])
+            o2[e] = first_half ? fmaf(x, c, -y * s) : fmaf(x, c, y * s);
+          }
+          os[w] = pack_bf16(o2[0], o2[1]);
+        }
+        kx = make_uint4(os[0], os[1], os[2], os[3]);
+      }
+    }
+    *reinterpret_cast<uint4*>(a.dk + dst) = kx;
+    if (a.v != nullptr) {
+      *reinterpret_cast<uint4*>(a.dv + dst) = *reinterpret_cast<const uint4*>(a.v + src);
+    }
+  }
+}
+
+// Context rows [0, 511) of a chunked sliding prefill: row r holds sequence
+// index len - 511 + r, read from the ring; rows before the start of the
+// sequence (or a slot whose tag does not match) are zero-filled so that the
+// masked products stay finite.
+__global__ void __launch_bounds__(128) ring_gather_kernel(const __nv_bfloat16* rk, const __nv_bfloat16* rv,
+                                                          const int32_t* len, const int32_t* head,
+                                                          const int32_t* tag, __nv_bfloat16* ck,
+                                                          __nv_bfloat16* cv, int64_t ctx_rows, int B) {
+  const int lane32 = threadIdx.x & 31;
+  const int kvh = threadIdx.x >> 5;
+  const int d0 = lane32 * 8;
+  constexpr int P = kWindow - 1;
+  for (int job = blockIdx.x; job < B * P; job += gridDim.x) {
+    const int b = job / P;
+    const int r = job % P;
+    const int L = len[b];
+    const int seq = L - P + r;
+    const int slot = ((head[b] - L + seq) % kWindow + kWindow) % kWindow;
+    const bool ok = seq >= 0 && tag[(int64_t)b * kWindow + slot] == seq;
+    const int64_t dst = (((int64_t)b * kHkv + kvh) * ctx_rows + r) * kD + d0;
+    uint4 kx = make_uint4(0, 0, 0, 0), vx = make_uint4(0, 0, 0, 0);
+    if (ok) {
+      const int64_t src = (((int64_t)b * kHkv + kvh) * kWindow + slot) * kD + d0;
+      kx = *reinterpret_cast<const uint4*>(rk + src);
+      vx = *reinterpret_cast<const uint4*>(rv + src);
+    }
+    *reinterpret_cast<uint4*>(ck + dst) = kx;
+    *reinterpret_cast<uint4*>(cv + dst) = vx;
+  }
+}
+
+// Advances the cache state after an append of T tokens.  A full-layer
+// sequence that would overflow its capacity is not advanced (its rows were
+// not written either).
+__global__ void kv_commit_kernel(int32_t* len, int32_t* head, int64_t capacity, int is_ring, int B, int T) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b >= B) return;
+  if (is_ring) {
+    head[b] = (head[b] + T) % kWindow;
+    len[b] += T;
+  } else if ((int64_t)len[b] + T <= capacity) {
+    len[b] += T;
+  }
+}
+
+__global__ void fill_i32_kernel(int32_t* p, int64_t n, int32_t v) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n; i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = v;
+}
+
+// ---------------------------------------------------------------------------
+// Host launchers
+// ---------------------------------------------------------------------------
+static int rope_grid(int jobs) {
+  int g = jobs;
+  const int cap = 148 * 16;
+  return g < cap ? (g > 0 ? g : 1) : cap;
+}
+
+cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st) {
+  RopeStoreArgs a;
+  a.k = reinterpret_cast<const __nv_bfloat16*>(h.k);
+  a.v = reinterpret_cast<const __nv_bfloat16*>(h.v);
+  a.src_bstride = h.src_bstride;
+  a.src_tstride = h.src_tstride;
+  a.src_hstride = h.src_hstride;
+  a.src_rotated = h.src_rotated;
+  a.pos = h.pos;
+  a.dk = reinterpret_cast<__nv_bfloat16*>(h.dk);
+  a.dv = reinterpret_cast<__nv_bfloat16*>(h.dv);
+  a.dst_rows = h.dst_rows;
+  a.dst_row_offset = h.dst_row_offset;
+  a.mode = h.mode;
+  a.len = h.len;
+  a.head = h.head;
+  a.tag = h.tag;
+  a.B = h.B;
+  a.T = h.T;
+  a.t_first = h.t_first;
+  const int grid = rope_grid(h.B * (h.T - h.t_first));
+  if (full)
+    rope_store_kernel<true><<<grid, 128, 0, st>>>(a);
+  else
+    rope_store_kernel<false><<<grid, 128, 0, st>>>(a);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_ring_gather(const void* rk, const void* rv, const int32_t* len, const int32_t* head,
+                               const int32_t* tag, void* ck, void* cv, int64_t ctx_rows, int B,
+                               cudaStream_t st) {
+  ring_gather_kernel<<<rope_grid(B * (kWindow - 1)), 128, 0, st>>>(
+      reinterpret_cast<const __nv_bfloat16*>(rk), reinterpret_cast<const __nv_bfloat16*>(rv), len, head, tag,
+      reinterpret_cast<__nv_bfloat16*>(ck), reinterpret_cast<__nv_bfloat16*>(cv), ctx_rows, B);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_kv_commit(int32_t* len, int32_t* head, int64_t capacity, bool ring, int B, int T,
+                             cudaStream_t st) {
+  kv_commit_kernel<<<(B + 127) / 128, 128, 0, st>>>(len, head, capacity, ring ? 1 : 0, B, T);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fill_i32(int32_t* p, int64_t n, int32_t v, cudaStream_t st) {
+  if (n <= 0) return cudaSuccess;
+  int64_t blocks = (n + 255) / 256;
+  if (blocks > 4096) blocks = 4096;
+  fill_i32_kernel<<<(int)blocks, 256, 0, st>>>(p, n, v);
+  count_launch();
+  return cudaGetLastError();
+}
+
+}  // namespace hyb

@@ -1,0 +1,186 @@
+/*
+ * hyb_attn.h -- C ABI of the B200 (sm_100a) hybrid GQA attention core.
+ *
+ * The operation is the per-layer attention of the Spark-X2.5 / X2.6-4B
+ * decoder as the following pages describe it (titles abbreviated):
+ *
+ *  [TEARDOWN] "百万 Token 塞进 4B 是怎么做到的？星火 X2.5 的长上下文架构拆解与显存博弈"
+ *  [LAPTOP]   "不用高显存卡也能跑！4B参数挑战百万上下文，笔记本就能玩"
+ *  [X26BASE]  the Spark-X2.6-4B-Base config walkthrough (lqnn.cn)
+ *
+ *  - 16 query heads share 4 KV heads (query head h reads KV head h / 4),
+ *    head_dim 256: [TEARDOWN] §"省显存的第二板斧：GQA、融合投影与输出门控",
+ *    [LAPTOP] §"分组查询注意力".
+ *  - Layer types: sliding layers attend to the last 512 tokens (the query
+ *    and the 511 before it) and rotate all 256 dims with RoPE theta 1e4;
+ *    full layers attend causally to the whole prefix and rotate only the
+ *    first 64 dims with theta 5e6: [TEARDOWN] §"混合注意力：每 4 层只给一层
+ *    全量视野" and §"滑动窗口的补救：分层 RoPE 与局部/全局分工";
+ *    [X26BASE] §"全局注意力 + 5M 基频 RoPE".  Layer i is full iff i % 4 == 3.
+ *  - RoPE is rotate-half: for k < R/2, pair (k, k + R/2) rotates by
+ *    pos * theta^(-2k/R); dims >= R are unchanged.
+ *  - Softmax scale 1/16; the normalised output of head h is multiplied by
+ *    sigmoid(gate[h]) ([TEARDOWN] §"省显存的第二板斧", the head-wise output gate).
+ *  - KV cache: a full layer keeps every token (4096 bytes per token per
+ *    layer, [TEARDOWN] §"先算一笔账"); a sliding layer keeps the most recent
+ *    512 tokens in a ring ([LAPTOP] §"百万上下文的真正瓶颈").
+ *
+ * Conventions for every call
+ *  - All tensors are bfloat16 unless stated; all pointers are DEVICE
+ *    pointers owned by the caller, except where a parameter says "host".
+ *    The library never allocates or frees device memory.
+ *  - Every pointer and every row stride (in bytes) must be 16-byte aligned.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t passed as void*;
+ *    NULL = the legacy default stream).  Host-side argument checks run
+ *    before any launch; on a non-OK status nothing was enqueued and
+ *    hyb_last_error() describes the problem.
+ *  - Conditions only the device can see (a full-layer cache running out of
+ *    capacity, a pipeline wait that exceeded its time limit) set sticky
+ *    bits in a per-device error word read by hyb_device_error(); kernels
+ *    never trap.
+ *  - Token positions: a token's sequence index is its position in its
+ *    sequence (0-based, counting cached tokens).  Masks always use sequence
+ *    indices; RoPE uses `pos` when given, else the sequence index.
+ */
+#ifndef HYB_ATTN_H
+#define HYB_ATTN_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define HYB_N_Q_HEADS 16
+#define HYB_N_KV_HEADS 4
+#define HYB_HEAD_DIM 256
+#define HYB_WINDOW 512
+
+typedef enum { HYB_SLIDING = 0, HYB_FULL = 1 } hyb_layer_type;
+
+typedef enum {
+  HYB_OK = 0,
+  HYB_EINVAL = -1,       /* null pointer, bad enum, non-positive size            */
+  HYB_ESHAPE = -2,       /* sizes inconsistent with each other or the cache      */
+  HYB_EALIGN = -3,       /* pointer or row stride not 16-byte aligned            */
+  HYB_EOVERFLOW = -4,    /* workspace too small / size arithmetic overflow       */
+  HYB_ECUDA = -5,        /* a CUDA runtime or driver call failed                 */
+  HYB_EUNSUPPORTED = -6  /* device is not sm_100 / driver entry point missing    */
+} hyb_status;
+
+/* Bits of the per-device error word (hyb_device_error). */
+#define HYB_DEV_ERR_CAPACITY 1  /* append past a full-layer cache's capacity: skipped */
+#define HYB_DEV_ERR_TIMEOUT 2   /* a pipeline wait exceeded its limit: output invalid */
+
+/*
+ * KV cache of one layer for `batch` sequences.  All buffers are caller-owned
+ * device memory; the struct itself may live on the host stack.
+ *   k, v : bf16 [batch][4][capacity][256] (head-major: one KV head's keys of
+ *          one sequence are contiguous).  Keys are stored already rotated.
+ *   len  : int32 [batch], tokens of each sequence appended so far.
+ *   head : SLIDING only, int32 [batch], next ring slot to write.
+ *   tag  : SLIDING only, int32 [batch][512], sequence index held by each
+ *          slot, -1 = empty.
+ * FULL caches keep token i at slot i (capacity >= longest sequence);
+ * SLIDING caches have capacity 512 and write token i at slot
+ * (head0 + i) % 512, head0 being the head when len was 0.
+ */
+typedef struct hyb_kv_cache {
+  int32_t type;      /* hyb_layer_type */
+  int32_t batch;
+  int64_t capacity;
+  void* k;
+  void* v;
+  int32_t* len;
+  int32_t* head;
+  int32_t* tag;
+} hyb_kv_cache;
+
+/*
+ * Resets a cache: len = 0, head = head0[b] (host array, NULL = all 0),
+ * tag = -1, and zero-fills k and v so that no slot ever holds a non-finite
+ * bit pattern (masked keys are multiplied by a zero weight, and 0 * NaN
+ * would poison the output).  Must run once on fresh memory.
+ * Errors: HYB_EINVAL (null buffer, bad type), HYB_ESHAPE (SLIDING with
+ * capacity != 512, head0 outside [0,512)), HYB_EALIGN, HYB_ECUDA.
+ */
+hyb_status hyb_kv_cache_init(const hyb_kv_cache* cache, const int32_t* head0, void* stream);
+
+/*
+ * Appends T tokens to every sequence of the cache (§ KV cache above).
+ *   k, v : rows of 4 x 256 bf16 per token, token t of sequence b at
+ *          element offset (b*T + t) * kv_row_stride.  kv_row_stride = 1024
+ *          for contiguous [B,T,4,256]; 6144 for k/v views into a fused
+ *          q_k_v_proj row ([TEARDOWN] §"省显存的第二板斧": q = [:4096],
+ *          k = [4096:5120], v = [5120:6144]).
+ *   pos  : device int32 [batch][T] RoPE positions, or NULL (sequence index).
+ * K is rotated with the cache's layer type before it is stored; V is copied
+ * bit for bit.  A full-layer sequence whose len + T exceeds capacity is left
+ * unchanged and HYB_DEV_ERR_CAPACITY is raised.  For a sliding layer only
+ * the last min(T, 512) tokens are written.
+ */
+hyb_status hyb_kv_append(const hyb_kv_cache* cache, const void* k, const void* v,
+                         int64_t kv_row_stride, const int32_t* pos, int32_t T, void* stream);
+
+/*
+ * Prefill attention of T new tokens per sequence, B sequences.
+ *   q    : 16 x 256 per token at element offset (b*T + t) * q_row_stride
+ *          (4096 contiguous, 6144 for a fused q_k_v_proj row).
+ *   k, v : as in hyb_kv_append (kv_row_stride).
+ *   gate : bf16 [B][T][16] gate scores, or NULL for no gate.
+ *   pos  : device int32 [B][T] RoPE positions, or NULL (sequence index).
+ *   out  : bf16 [B][T][16][256].
+ *   cache: NULL -> the T tokens are whole sequences (token t has sequence
+ *          index t).  Non-NULL -> they continue the cached sequences (token
+ *          t has index len[b] + t), attend over the cached keys as well, and
+ *          are appended to the cache.  cache->type must equal layer_type and
+ *          cache->batch must equal B.
+ *   workspace: device scratch of at least
+ *          hyb_attn_prefill_workspace_size(layer_type, B, T, cache != NULL)
+ *          bytes (256-byte aligned); it holds rotated keys between launches.
+ * Errors: HYB_EINVAL, HYB_ESHAPE, HYB_EALIGN, HYB_EOVERFLOW (workspace too
+ * small), HYB_EUNSUPPORTED (not an sm_100 device), HYB_ECUDA.
+ */
+size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache);
+hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const void* gate,
+                            const int32_t* pos, int32_t layer_type, int32_t B, int32_t T,
+                            int64_t q_row_stride, int64_t kv_row_stride, void* out,
+                            const hyb_kv_cache* cache, void* workspace, size_t workspace_bytes,
+                            void* stream);
+
+/*
+ * One decode step: one query token per sequence against its cache, which
+ * must already hold the token itself (call hyb_kv_append first).
+ *   q    : bf16 [B][16][256] contiguous query (not rotated).
+ *   gate : bf16 [B][16] or NULL.
+ *   pos  : device int32 [B] RoPE position of the query, or NULL (len - 1).
+ *   max_len : host-side upper bound of len over the batch (<= capacity), or
+ *          0 for capacity; it sizes the split-KV grid and the workspace.
+ *   out  : bf16 [B][16][256].
+ *   workspace: at least hyb_attn_decode_workspace_size(layer_type, B,
+ *          max_len) bytes of device scratch for the per-split partial
+ *          outputs and log-sum-exps.
+ * Errors: as hyb_attn_prefill.
+ */
+size_t hyb_attn_decode_workspace_size(int32_t layer_type, int32_t B, int64_t max_len);
+hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos,
+                           const hyb_kv_cache* cache, int32_t layer_type, int64_t max_len,
+                           void* out, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, copies the current device's error word to
+ * *flags (host) and, if clear != 0, resets it.
+ */
+hyb_status hyb_device_error(int32_t* flags, int32_t clear, void* stream);
+
+/* Message for the last non-OK status returned on the calling thread. */
+const char* hyb_last_error(void);
+
+/* Number of kernels this library has launched in the process so far. */
+uint64_t hyb_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* HYB_ATTN_H */

@@ -1,0 +1,108 @@
+"""Host-side tests of the C-ABI library that need no GPU.
+
+* the shared library loads and exports every function include/hyb_attn.h
+  declares;
+* argument checks that run before any CUDA call return the documented
+  status codes;
+* workspace-size arithmetic.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "hyb_attn.h")
+
+
+@pytest.fixture(scope="module")
+def hyb():
+    import full_gqa_attention_partial_b200 as hyb
+    from full_gqa_attention_partial_b200 import build
+    build.build()
+    hyb.load()
+    return hyb
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(hyb_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for fn in ("hyb_attn_prefill", "hyb_attn_decode", "hyb_kv_append", "hyb_kv_cache_init"):
+        assert fn in names
+
+
+def test_library_exports_every_declared_symbol(hyb):
+    lib = ctypes.CDLL(hyb.LIB_PATH)
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+    assert set(_declared_functions()) <= set(hyb.EXPORTED) | {"hyb_last_error"}
+
+
+def _cache(hyb, lt=0, batch=1, cap=512, null_k=False):
+    c = hyb._Cache(lt, batch, cap, 0 if null_k else 0x1000, 0x2000, 0x3000, 0x4000, 0x5000)
+    return c
+
+
+def test_argument_checks_before_any_cuda_call(hyb):
+    lib = hyb.load()
+    vp = ctypes.c_void_p
+    A = vp(0x10000)
+    # null q
+    assert lib.hyb_attn_prefill(None, A, A, None, None, 0, 1, 8, 4096, 1024, A, None, None, 0, None) == -1
+    # bad layer type
+    assert lib.hyb_attn_prefill(A, A, A, None, None, 7, 1, 8, 4096, 1024, A, None, None, 0, None) == -1
+    # T = 0
+    assert lib.hyb_attn_prefill(A, A, A, None, None, 0, 1, 0, 4096, 1024, A, None, None, 0, None) == -1
+    # misaligned q
+    assert lib.hyb_attn_prefill(vp(0x10008), A, A, None, None, 0, 1, 8, 4096, 1024, A, None, None, 0,
+                                None) == -3
+    # q row stride not a multiple of 8 / too small
+    assert lib.hyb_attn_prefill(A, A, A, None, None, 0, 1, 8, 4100, 1024, A, None, None, 0, None) == -3
+    assert lib.hyb_attn_prefill(A, A, A, None, None, 0, 1, 8, 1024, 1024, A, None, None, 0, None) == -3
+    # workspace missing / too small
+    assert lib.hyb_attn_prefill(A, A, A, None, None, 0, 1, 8, 4096, 1024, A, None, None, 0, None) == -1
+    assert lib.hyb_attn_prefill(A, A, A, None, None, 0, 1, 8, 4096, 1024, A, None, vp(0x20000), 16,
+                                None) == -4
+    msg = lib.hyb_last_error().decode()
+    assert "workspace" in msg
+    # cache problems
+    c = _cache(hyb, lt=0, cap=100)
+    assert lib.hyb_kv_append(ctypes.byref(c), A, A, 1024, None, 4, None) == -2      # sliding cap != 512
+    c = _cache(hyb, lt=1, cap=1024, null_k=True)
+    assert lib.hyb_kv_append(ctypes.byref(c), A, A, 1024, None, 4, None) == -1      # null k buffer
+    c = _cache(hyb, lt=1, cap=1024)
+    assert lib.hyb_kv_append(ctypes.byref(c), A, A, 1024, None, 0, None) == -1      # T = 0
+    assert lib.hyb_kv_append(ctypes.byref(c), A, A, 1000, None, 4, None) == -3      # stride
+    # cache type vs layer type; batch mismatch; T beyond a full cache's capacity
+    assert lib.hyb_attn_prefill(A, A, A, None, None, 0, 1, 8, 4096, 1024, A, ctypes.byref(c), None, 0,
+                                None) == -2
+    assert lib.hyb_attn_prefill(A, A, A, None, None, 1, 2, 8, 4096, 1024, A, ctypes.byref(c), None, 0,
+                                None) == -2
+    assert lib.hyb_attn_prefill(A, A, A, None, None, 1, 1, 2048, 4096, 1024, A, ctypes.byref(c), None, 0,
+                                None) == -2
+    # decode: max_len beyond capacity, layer type mismatch
+    assert lib.hyb_attn_decode(A, None, None, ctypes.byref(c), 1, 4096, A, A, 1 << 20, None) == -2
+    assert lib.hyb_attn_decode(A, None, None, ctypes.byref(c), 0, 0, A, A, 1 << 20, None) == -2
+
+
+def test_workspace_sizes(hyb):
+    # cache-less prefill holds the rotated keys: B * T * 4 heads * 256 * 2 bytes
+    assert hyb.hyb_attn_prefill_workspace_size(hyb.FULL, 2, 1000, False) == 2 * 1000 * 2048
+    assert hyb.hyb_attn_prefill_workspace_size(hyb.FULL, 2, 1000, True) == 0
+    # sliding chunk: context K and V of 511 + T rows
+    assert hyb.hyb_attn_prefill_workspace_size(hyb.SLIDING, 1, 8192, True) == 2 * (511 + 8192) * 2048
+    # decode: B * 16 * splits * (256 + 1) floats, rounded up
+    for lt, B, L in ((hyb.FULL, 1, 1 << 20), (hyb.FULL, 16, 131073), (hyb.SLIDING, 16, 512)):
+        n = hyb.hyb_attn_decode_workspace_size(lt, B, L)
+        assert n >= B * 16 * 257 * 4 and n % 4 == 0
+
+
+def test_layer_schedule_binding(hyb):
+    types = [hyb.layer_type(i) for i in range(36)]
+    assert types.count(hyb.FULL) == 9 and types[3] == hyb.FULL and types[35] == hyb.FULL
