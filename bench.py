@@ -1,0 +1,562 @@
+#!/usr/bin/env python
+"""Benchmark of the hybrid GQA attention hot path on B200.
+
+Step (the headline workload): prefill of one 4-layer group -- 3 sliding
+layers and 1 full layer, batch 1, 32768 tokens, 16 query / 4 KV heads,
+head_dim 256 -- into fresh KV caches (RoPE, masked GQA attention, sigmoid
+gate, linear-cache and ring appends).  Inputs are seeded N(0,1) bf16 and
+each layer's fused qkv rows (400 MB) are larger than L2, so no flush is
+needed between steps.
+
+The JSON line also carries:
+  roofline      the full-layer prefill attention kernel, timed live with CUDA
+                events around its launches, against the measured bf16 peak;
+  e2e           the same metric through the C ABI from pinned host buffers,
+                copies inside the timed region;
+  decode        decode, batch 16, 131072-token full-layer cache and a full
+                512-slot ring (head at a random offset): KV GB/s, % of HBM,
+                tokens/s;
+  prefill_128k  one full layer, 131072 tokens: TFLOP/s and % of peak;
+  decode_1m     (--decode-1m) 36-layer decode at 1M tokens: tokens/s;
+  cpu_baseline  the fp64 oracle on a bounded sample of the same workload.
+
+`--impl reference` times the oracle as the reference arm instead.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+SLIDING, FULL = 0, 1
+H, KVH, D, W = 16, 4, 256, 512
+GROUP_LAYERS = [SLIDING, SLIDING, SLIDING, FULL]   # layers 0..3 of the 3 + 1 pattern
+T_MAIN = 32768
+B_MAIN = 1
+METRIC = "prefill attn TFLOP/s"
+WORKLOAD = ("prefill of one 4-layer group (3 sliding + 1 full), batch 1, seq 32768, 16 Q / 4 KV heads, "
+            "head_dim 256, bf16 N(0,1) inputs, seed 1")
+
+
+def pairs(n: int, lt: int) -> int:
+    if lt == FULL or n <= W:
+        return n * (n + 1) // 2
+    return W * (W + 1) // 2 + (n - W) * W
+
+
+def flops(n: int, lt: int, heads: int = H) -> int:
+    return pairs(n, lt) * heads * 4 * D
+
+
+def layer_seed(base: int, i: int) -> int:
+    return base + 7919 * i
+
+
+# ---------------------------------------------------------------------------
+# plumbing: ranks, peaks, clocks
+# ---------------------------------------------------------------------------
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend="nccl"):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+        if torch.cuda.is_available():
+            torch.cuda.set_device(self.local)
+
+    def barrier(self):
+        if self.pg:
+            self.pg.barrier()
+
+    def max(self, x: float) -> float:
+        if not self.pg:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        j = json.load(open(p))
+        return {"hbm_gbs": float(j["hbm_gbs"]), "bf16_tflops": float(j["bf16_tflops"]),
+                "bf16_tflops_sustained": float(j.get("bf16_tflops_sustained", j["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+class Clocks:
+    """nvidia-smi sampling (every 200 ms) while the timed regions run."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self):
+        self.proc = None
+        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{os.environ.get('RANK', '0')}.csv")
+
+    def start(self):
+        try:
+            os.makedirs(os.path.dirname(self.path), exist_ok=True)
+            sel = []
+            try:
+                uuid = str(torch.cuda.get_device_properties(torch.cuda.current_device()).uuid)
+                sel = ["-i", uuid if uuid.startswith("GPU-") else "GPU-" + uuid]
+            except Exception:
+                pass
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(["nvidia-smi", *sel, f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "200"],
+                                         stdout=self.f, stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.f.close()
+        rows = []
+        for line in open(self.path):
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), float(parts[3]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        pmax = max(r[2] for r in rows)
+        load = [r for r in rows if r[2] >= 0.4 * pmax] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in load for i, v in enumerate(r[3]) if v.lower().startswith("active")})
+        return {"sm_mhz": statistics.median(r[0] for r in load), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples_under_load": len(load), "power_w_max": pmax}
+
+
+# ---------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------
+def make_layer_inputs(T: int, seed: int):
+    from full_gqa_attention_partial_b200 import synth
+    return synth.prefill_inputs(B_MAIN, T, seed=seed, device="cuda")
+
+
+def bench_main(hyb, args, dist: Dist, peaks):
+    layers = [make_layer_inputs(T_MAIN, layer_seed(1, i)) for i in range(len(GROUP_LAYERS))]
+    n_steps = args.warmup + args.steps
+    caches = [[hyb.KVCache(lt, B_MAIN, capacity=T_MAIN) for lt in GROUP_LAYERS] for _ in range(n_steps)]
+    ws_bytes = max(hyb.hyb_attn_prefill_workspace_size(lt, B_MAIN, T_MAIN, True) for lt in GROUP_LAYERS)
+    ws = hyb.alloc_workspace(ws_bytes)
+    outs = [torch.empty(B_MAIN, T_MAIN, H, D, dtype=torch.bfloat16, device="cuda") for _ in GROUP_LAYERS]
+    step_flops = sum(flops(T_MAIN, lt) for lt in GROUP_LAYERS)
+
+    def step(i):
+        for li, lt in enumerate(GROUP_LAYERS):
+            x = layers[li]
+            hyb.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], None, lt, out=outs[li],
+                                 cache=caches[i][li], workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    assert hyb.hyb_device_error() == 0
+    dist.barrier()
+    torch.cuda.synchronize()
+    l0 = hyb.hyb_launch_count()
+    timer = hyb.KernelTimer(args.steps * len(GROUP_LAYERS))
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with timer:
+        ev0.record()
+        for i in range(args.steps):
+            step(args.warmup + i)
+        ev1.record()
+    torch.cuda.synchronize()
+    dist.barrier()
+    launches = hyb.hyb_launch_count() - l0
+    ms = dist.max(ev0.elapsed_time(ev1))
+    assert hyb.hyb_device_error() == 0
+    kt = timer.times_ms()
+    per_layer = {li: kt[li::len(GROUP_LAYERS)] for li in range(len(GROUP_LAYERS))}
+    full_ms = statistics.mean(per_layer[3])
+    slide_ms = statistics.mean(t for li in range(3) for t in per_layer[li])
+    total_s = ms / 1e3
+    peak = peaks["bf16_tflops_sustained"] if total_s >= 1.0 else peaks["bf16_tflops"]
+    peak_kind = "sustained" if total_s >= 1.0 else "burst"
+    achieved = flops(T_MAIN, FULL) / (full_ms / 1e3) / 1e12
+    kernel_share = sum(kt) / (ms / 1.0) if ms > 0 else None
+    res = {
+        "value": dist.world * args.steps * step_flops / total_s / 1e12,
+        "ms_per_step": ms / args.steps,
+        "gpu_launches": launches,
+        "roofline": {
+            "bound": "tensor", "kernel": "prefill_kernel<FULL> (tcgen05)", "achieved": achieved,
+            "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
+            "peak_source": f"{peaks['source']} bf16 {peak_kind}",
+            "algorithmic_flops_per_launch": flops(T_MAIN, FULL),
+            "avg_launch_ms": full_ms, "launches": len(per_layer[3]),
+            "traffic": args.full_traffic,
+            "sliding_kernel": {"avg_launch_ms": slide_ms,
+                               "achieved": flops(T_MAIN, SLIDING) / (slide_ms / 1e3) / 1e12},
+            "attention_kernels_share_of_step": kernel_share,
+        },
+    }
+    # ---- e2e: pinned host inputs -> device -> library -> host ----
+    host_in = [{k: layers[li][k].cpu().pin_memory() for k in ("qkv", "gate")} for li in range(len(GROUP_LAYERS))]
+    host_out = [torch.empty(B_MAIN, T_MAIN, H, D, dtype=torch.bfloat16).pin_memory() for _ in GROUP_LAYERS]
+    dev_qkv = torch.empty_like(layers[0]["qkv"])
+    dev_gate = torch.empty_like(layers[0]["gate"])
+    e2e_caches = [[hyb.KVCache(lt, B_MAIN, capacity=T_MAIN) for lt in GROUP_LAYERS] for _ in range(n_steps)]
+    q = dev_qkv[..., :4096].unflatten(-1, (H, D))
+    k = dev_qkv[..., 4096:5120].unflatten(-1, (KVH, D))
+    v = dev_qkv[..., 5120:].unflatten(-1, (KVH, D))
+    h2d = sum(t.numel() * t.element_size() for hi in host_in for t in hi.values())
+    d2h = sum(t.numel() * t.element_size() for t in host_out)
+
+    def e2e_step(i):
+        for li, lt in enumerate(GROUP_LAYERS):
+            dev_qkv.copy_(host_in[li]["qkv"], non_blocking=True)
+            dev_gate.copy_(host_in[li]["gate"], non_blocking=True)
+            hyb.hyb_attn_prefill(q, k, v, dev_gate, None, lt, out=outs[li], cache=e2e_caches[i][li], workspace=ws)
+            host_out[li].copy_(outs[li], non_blocking=True)
+
+    for i in range(args.warmup):
+        e2e_step(i)
+    torch.cuda.synchronize()
+    dist.barrier()
+    ev0.record()
+    for i in range(args.steps):
+        e2e_step(args.warmup + i)
+    ev1.record()
+    torch.cuda.synchronize()
+    e2e_ms = dist.max(ev0.elapsed_time(ev1))
+    res["e2e"] = {"value": dist.world * args.steps * step_flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+                  "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
+    del caches, e2e_caches, host_in, host_out
+    return res, layers
+
+
+def bench_prefill_128k(hyb, args, peaks):
+    T = 131072
+    x = make_layer_inputs(T, layer_seed(1, 3))
+    ws = hyb.alloc_workspace(hyb.hyb_attn_prefill_workspace_size(FULL, 1, T, False))
+    out = torch.empty(1, T, H, D, dtype=torch.bfloat16, device="cuda")
+    n = 3
+    hyb.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], x["pos"], FULL, out=out, workspace=ws)
+    torch.cuda.synchronize()
+    timer = hyb.KernelTimer(n)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with timer:
+        ev0.record()
+        for _ in range(n):
+            hyb.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], x["pos"], FULL, out=out, workspace=ws)
+        ev1.record()
+    torch.cuda.synchronize()
+    assert hyb.hyb_device_error() == 0
+    call_ms = ev0.elapsed_time(ev1) / n
+    k_ms = statistics.mean(timer.times_ms())
+    f = flops(T, FULL)
+    peak = peaks["bf16_tflops"]
+    return {"workload": "one full layer, batch 1, seq 131072", "tflop_per_launch": f / 1e12,
+            "kernel_ms": k_ms, "call_ms": call_ms, "kernel_tflops": f / (k_ms / 1e3) / 1e12,
+            "call_tflops": f / (call_ms / 1e3) / 1e12, "frac_of_peak": f / (k_ms / 1e3) / 1e12 / peak,
+            "peak": peak, "peak_source": f"{peaks['source']} bf16 burst", "launches": n}
+
+
+def fill_full_cache(hyb, B: int, L: int, cap: int, seed: int):
+    """Full-layer cache holding L random tokens (keys taken as already rotated)."""
+    from full_gqa_attention_partial_b200 import synth
+    c = hyb.KVCache(FULL, B, capacity=cap)
+    synth.fill_cache_randn_(c.k, c.v, L, seed)
+    c.len.fill_(L)
+    return c
+
+
+def fill_ring_cache(hyb, B: int, L: int, seed: int, head0: int):
+    """A 512-slot ring in the state it has after L tokens: token i at slot (head0 + i) % 512."""
+    from full_gqa_attention_partial_b200 import synth
+    c = hyb.KVCache(SLIDING, B, head0=[head0] * B)
+    synth.fill_cache_randn_(c.k, c.v, W, seed)
+    idx = torch.arange(max(0, L - W), L, dtype=torch.int64, device="cuda")
+    tag = torch.full((W,), -1, dtype=torch.int32, device="cuda")
+    tag[(head0 + idx) % W] = idx.to(torch.int32)
+    c.tag.copy_(tag.expand(B, W))
+    c.len.fill_(L)
+    c.head.fill_((head0 + L) % W)
+    return c
+
+
+def bench_decode(hyb, args, peaks):
+    from full_gqa_attention_partial_b200 import synth
+    B, L = 16, 131072
+    n_steps = args.warmup + args.steps
+    cap = L + n_steps + 1
+    r = synth.ring_offset(2)
+    full = fill_full_cache(hyb, B, L, cap, seed=2)
+    ring = fill_ring_cache(hyb, B, L, seed=3, head0=r)
+    qs = [synth.decode_query(B, seed=1000 + i, device="cuda") for i in range(n_steps)]
+    ws = hyb.alloc_workspace(max(hyb.hyb_attn_decode_workspace_size(FULL, B, cap),
+                                 hyb.hyb_attn_decode_workspace_size(SLIDING, B, W)))
+    out = torch.empty(B, H, D, dtype=torch.bfloat16, device="cuda")
+
+    def step(i):
+        x = qs[i]
+        hyb.hyb_kv_append(full, x["k"], x["v"])
+        hyb.hyb_attn_decode(x["q"], x["gate"], full, max_len=cap, out=out, workspace=ws)
+        hyb.hyb_kv_append(ring, x["k"], x["v"])
+        hyb.hyb_attn_decode(x["q"], x["gate"], ring, max_len=W, out=out, workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    timer = hyb.KernelTimer(2 * args.steps)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with timer:
+        ev0.record()
+        for i in range(args.steps):
+            step(args.warmup + i)
+        ev1.record()
+    torch.cuda.synchronize()
+    assert hyb.hyb_device_error() == 0
+    ms = ev0.elapsed_time(ev1) / args.steps
+    kt = timer.times_ms()
+    full_ms = statistics.mean(kt[0::2])
+    ring_ms = statistics.mean(kt[1::2])
+    # KV bytes read per step: every cached token's K and V of 4 heads (4096 B per token per layer)
+    lens = [L + args.warmup + i + 1 for i in range(args.steps)]
+    full_bytes = statistics.mean(B * n * 4096 for n in lens)
+    ring_bytes = B * W * 4096
+    hbm = peaks["hbm_gbs"]
+    achieved = full_bytes / (full_ms / 1e3) / 1e9
+    return {
+        "workload": "decode, batch 16, full-layer cache 131072 tokens + 512-slot ring (head at random "
+                    f"offset {r}), one full + one sliding layer per step, append + decode, seed 2",
+        "tokens_per_s": B / (ms / 1e3), "ms_per_step": ms,
+        "kv_gb_per_s": (full_bytes + ring_bytes) / (ms / 1e3) / 1e9,
+        "frac_of_hbm": (full_bytes + ring_bytes) / (ms / 1e3) / 1e9 / hbm,
+        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<FULL>", "achieved": achieved, "peak": hbm,
+                     "unit": "GB/s", "frac": achieved / hbm, "peak_source": f"{peaks['source']} HBM copy",
+                     "algorithmic_bytes_per_launch": full_bytes, "avg_launch_ms": full_ms,
+                     "traffic": args.decode_traffic},
+        "sliding_kernel": {"avg_launch_ms": ring_ms, "achieved_gbs": ring_bytes / (ring_ms / 1e3) / 1e9},
+    }
+
+
+def bench_decode_1m(hyb, args, peaks):
+    """36 layers (27 rings, 9 full caches of ~1M tokens), batch 1, 64 steps of append + decode."""
+    from full_gqa_attention_partial_b200 import synth
+    n_steps = 64
+    L0 = (1 << 20) - n_steps
+    cap = 1 << 20
+    r = synth.ring_offset(3)
+    fulls = [fill_full_cache(hyb, 1, L0, cap, seed=3 + 17 * i) for i in range(9)]
+    rings = [fill_ring_cache(hyb, 1, L0, seed=5000 + i, head0=r) for i in range(27)]
+    qs = [synth.decode_query(1, seed=9000 + i, device="cuda") for i in range(n_steps)]
+    ws_full = hyb.alloc_workspace(hyb.hyb_attn_decode_workspace_size(FULL, 1, cap))
+    ws_ring = hyb.alloc_workspace(hyb.hyb_attn_decode_workspace_size(SLIDING, 1, W))
+    out = torch.empty(1, H, D, dtype=torch.bfloat16, device="cuda")
+
+    def step(i):
+        x = qs[i]
+        fi = ri = 0
+        for layer in range(36):
+            lt = FULL if layer % 4 == 3 else SLIDING
+            if lt == FULL:
+                c, ws, ml = fulls[fi], ws_full, cap
+                fi += 1
+            else:
+                c, ws, ml = rings[ri], ws_ring, W
+                ri += 1
+            hyb.hyb_kv_append(c, x["k"], x["v"])
+            hyb.hyb_attn_decode(x["q"], x["gate"], c, max_len=ml, out=out, workspace=ws)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    ev0.record()
+    for i in range(n_steps):
+        step(i)
+    ev1.record()
+    torch.cuda.synchronize()
+    assert hyb.hyb_device_error() == 0
+    ms = ev0.elapsed_time(ev1) / n_steps
+    kv = statistics.mean(9 * 4096 * (L0 + i + 1) + 27 * 4096 * W for i in range(n_steps))
+    return {"workload": "36-layer decode (9 full caches ~1M tokens, 27 rings), batch 1, 64 steps, seed 3",
+            "tokens_per_s": 1e3 / ms, "ms_per_step": ms, "kv_gb_per_s": kv / (ms / 1e3) / 1e9,
+            "frac_of_hbm": kv / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+
+
+# ---------------------------------------------------------------------------
+# the oracle on the host: cpu_baseline and the reference arm
+# ---------------------------------------------------------------------------
+def blas_threads() -> int:
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 0) for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count() or 1
+
+
+def oracle_sample(host_layers, rows_per_layer: int, seed: int):
+    """Times the oracle on `rows_per_layer` query rows of each layer; returns (flops, seconds)."""
+    import oracle as O
+    rng = np.random.default_rng(seed)
+    total_flops, total_s = 0, 0.0
+    for li, lt in enumerate(GROUP_LAYERS):
+        x = host_layers[li]
+        T = x["q"].shape[1]
+        rows = np.sort(rng.choice(T, size=rows_per_layer, replace=False))
+        t0 = time.perf_counter()
+        O.prefill(x["q"], x["k"], x["v"], x["gate"], x["pos"], lt, rows=rows)
+        total_s += time.perf_counter() - t0
+        for t in rows:
+            n_keys = t + 1 if lt == FULL else min(t + 1, W)
+            total_flops += n_keys * H * 4 * D
+    return total_flops, total_s
+
+
+def host_copies(layers):
+    out = []
+    for x in layers:
+        out.append({"q": x["q"].float().cpu().numpy(), "k": x["k"].float().cpu().numpy(),
+                    "v": x["v"].float().cpu().numpy(), "gate": x["gate"].float().cpu().numpy(),
+                    "pos": x["pos"].cpu().numpy()})
+    return out
+
+
+def cpu_baseline(layers, rows_per_layer: int):
+    host = host_copies(layers)
+    f, s = oracle_sample(host, rows_per_layer, seed=0)
+    return {"value": f / s / 1e12, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows_per_layer} random query rows x 16 heads of each of the 4 layers at T=32768 "
+                      f"(oracle recomputes RoPE of all keys per layer); {s:.1f} s of CPU time",
+            "cpu_model": cpu_model()}
+
+
+def cpu_model() -> str:
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                return line.split(":", 1)[1].strip()
+    except Exception:
+        pass
+    return "unknown"
+
+
+def run_reference(args, dist: Dist):
+    if dist.rank != 0:
+        return None
+    from full_gqa_attention_partial_b200 import synth
+    layers = [synth.prefill_inputs(B_MAIN, T_MAIN, seed=layer_seed(1, i)) for i in range(len(GROUP_LAYERS))]
+    host = host_copies(layers)
+    rows = args.ref_rows
+    for i in range(args.warmup):
+        oracle_sample(host, rows, seed=100 + i)
+    f_tot, s_tot = 0, 0.0
+    for i in range(args.steps):
+        f, s = oracle_sample(host, rows, seed=200 + i)
+        f_tot += f
+        s_tot += s
+    value = f_tot / s_tot / 1e12
+    sample = (f"each step: {rows} random query rows x 16 heads of each of the 4 layers at T=32768, "
+              f"fp64 numpy oracle")
+    return {"impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOP/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": s_tot * 1e3 / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic N(0,1) bf16 inputs, seeded", "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"value": value, "unit": "TFLOP/s", "cores": blas_threads(), "kind": "oracle",
+                             "sample": sample, "cpu_model": cpu_model()},
+            "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+# ---------------------------------------------------------------------------
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--decode-1m", action="store_true", help="also run the 36-layer 1M-token decode workload")
+    ap.add_argument("--no-extras", action="store_true", help="only the headline step (no sub-benchmarks)")
+    ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows per layer for cpu_baseline")
+    ap.add_argument("--ref-rows", type=int, default=8, help="oracle rows per layer per reference step")
+    ap.add_argument("--full-traffic", type=float, default=None,
+                    help="DRAM bytes per full-layer prefill launch from an ncu capture (reported as traffic)")
+    ap.add_argument("--decode-traffic", type=float, default=None)
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
+
+    dist = Dist()
+    if args.impl == "reference":
+        res = run_reference(args, dist)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    dist.init()
+    import full_gqa_attention_partial_b200 as hyb
+    hyb.load()
+    peaks = load_peaks()
+    clocks = Clocks()
+    clocks.start()
+    main_res, layers = bench_main(hyb, args, dist, peaks)
+    extras = {}
+    if dist.world == 1 and not args.no_extras:
+        extras["prefill_128k"] = bench_prefill_128k(hyb, args, peaks)
+        extras["decode"] = bench_decode(hyb, args, peaks)
+        if args.decode_1m:
+            extras["decode_1m"] = bench_decode_1m(hyb, args, peaks)
+    clk = clocks.stop()
+    line = {
+        "metric": METRIC, "value": main_res["value"], "unit": "TFLOP/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": main_res["ms_per_step"],
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic N(0,1) bf16, seeded (no dataset on the pages for this path)",
+        "config": {"workload": WORKLOAD, "batch": B_MAIN, "seq_len": T_MAIN,
+                   "layers": "sliding, sliding, sliding, full", "parallelism": f"replicas x{dist.world}",
+                   "l2": "no flush: each layer's inputs (400 MB) exceed the 126 MB L2"},
+        "roofline": main_res["roofline"], "e2e": main_res["e2e"], "gpu_launches": main_res["gpu_launches"],
+        "clocks": clk,
+    }
+    line.update(extras)
+    if dist.rank == 0 and dist.world == 1 and not args.no_extras:
+        line["cpu_baseline"] = cpu_baseline(layers, args.cpu_rows)
+    if dist.rank == 0:
+        print(json.dumps(line), flush=True)
+    dist.close()
+
+
+if __name__ == "__main__":
+    main()

@@ -35,7 +35,7 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libhyb_attn.so")
 EXPORTED = (
     "hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill_workspace_size", "hyb_attn_prefill",
     "hyb_attn_decode_workspace_size", "hyb_attn_decode", "hyb_device_error", "hyb_last_error",
-    "hyb_launch_count",
+    "hyb_launch_count", "hyb_profile_events", "hyb_profile_pairs_used",
 )
 
 
@@ -85,6 +85,9 @@ def load(path: str = LIB_PATH):
     lib.hyb_device_error.argtypes = [ctypes.POINTER(i32), i32, vp]
     lib.hyb_last_error.restype = ctypes.c_char_p
     lib.hyb_launch_count.restype = ctypes.c_uint64
+    lib.hyb_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
+    lib.hyb_profile_events.restype = ctypes.c_int
+    lib.hyb_profile_pairs_used.restype = i32
     for name in ("hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill", "hyb_attn_decode",
                  "hyb_device_error"):
         getattr(lib, name).restype = ctypes.c_int
@@ -234,3 +237,33 @@ def hyb_device_error(clear: bool = True, stream=None) -> int:
 
 def hyb_launch_count() -> int:
     return int(load().hyb_launch_count())
+
+
+class KernelTimer:
+    """Brackets the next `n` attention-kernel launches with CUDA events.
+
+    Uses hyb_profile_events: the library records events[2i] / events[2i+1]
+    on the launch stream right before / after the i-th prefill-attention or
+    decode split-KV kernel launch.
+    """
+
+    def __init__(self, n: int):
+        self.events = [torch.cuda.Event(enable_timing=True) for _ in range(2 * n)]
+        for e in self.events:   # torch creates the CUDA event lazily, on first record
+            e.record()
+        torch.cuda.synchronize()
+        self._arr = (ctypes.c_void_p * (2 * n))(*[e.cuda_event for e in self.events])
+        self.n = n
+
+    def __enter__(self):
+        _check(load().hyb_profile_events(self._arr, self.n))
+        return self
+
+    def __exit__(self, *exc):
+        self.used = int(load().hyb_profile_pairs_used())
+        _check(load().hyb_profile_events(None, 0))
+        return False
+
+    def times_ms(self):
+        torch.cuda.synchronize()
+        return [self.events[2 * i].elapsed_time(self.events[2 * i + 1]) for i in range(self.used)]

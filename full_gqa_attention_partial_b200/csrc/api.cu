@@ -19,6 +19,27 @@ namespace hyb {
 static std::atomic<uint64_t> g_launches{0};
 void count_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
+static void* const* g_prof_events = nullptr;
+static int g_prof_pairs = 0;
+static int g_prof_used = 0;
+// A failed record (e.g. a handle that is not a live event) disables
+// profiling and clears the error, so it never surfaces as a launch failure.
+static void profile_record(int idx, cudaStream_t st) {
+  if (cudaEventRecord(reinterpret_cast<cudaEvent_t>(g_prof_events[idx]), st) != cudaSuccess) {
+    (void)cudaGetLastError();
+    g_prof_events = nullptr;
+  }
+}
+void profile_before(cudaStream_t st) {
+  if (g_prof_events && g_prof_used < g_prof_pairs) profile_record(2 * g_prof_used, st);
+}
+void profile_after(cudaStream_t st) {
+  if (g_prof_events && g_prof_used < g_prof_pairs) {
+    profile_record(2 * g_prof_used + 1, st);
+    ++g_prof_used;
+  }
+}
+
 cudaError_t decode_set_smem_attr();
 cudaError_t prefill_set_smem_attr();
 
@@ -139,6 +160,16 @@ extern "C" {
 const char* hyb_last_error(void) { return t_err.c_str(); }
 
 uint64_t hyb_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+hyb_status hyb_profile_events(void* const* events, int32_t n_pairs) {
+  if (n_pairs < 0) return fail(HYB_EINVAL, "n_pairs %d negative", n_pairs);
+  hyb::g_prof_events = (n_pairs > 0) ? events : nullptr;
+  hyb::g_prof_pairs = (events != nullptr) ? n_pairs : 0;
+  hyb::g_prof_used = 0;
+  return HYB_OK;
+}
+
+int32_t hyb_profile_pairs_used(void) { return hyb::g_prof_used; }
 
 hyb_status hyb_device_error(int32_t* flags, int32_t clear, void* stream) {
   if (!flags) return fail(HYB_EINVAL, "flags is NULL");

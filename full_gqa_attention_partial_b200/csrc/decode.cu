@@ -329,10 +329,12 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
   a.n_splits = h.n_splits;
   const dim3 grid(h.n_splits, kHkv, h.B);
   const size_t smem = decode_smem_bytes();
+  profile_before(st);
   if (full)
     decode_split_kernel<true><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, a);
   else
     decode_split_kernel<false><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, a);
+  profile_after(st);
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;

@@ -9,6 +9,11 @@ namespace hyb {
 
 void count_launch();
 
+// Profiling hook (hyb_profile_events): records a caller-owned event pair
+// around the next attention-kernel launches.
+void profile_before(cudaStream_t st);
+void profile_after(cudaStream_t st);
+
 // ---- KV side (rope_kv.cu) --------------------------------------------------
 struct RopeStoreHost {
   const void* k = nullptr;

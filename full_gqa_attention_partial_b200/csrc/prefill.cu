@@ -391,10 +391,12 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   const long long grid = (long long)a.n_mtiles * h.B * kHq;
   if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   const size_t smem = prefill_smem_bytes();
+  profile_before(st);
   if (full)
     prefill_kernel<true><<<(unsigned)grid, kPfThreads, smem, st>>>(h.tm_k, h.tm_v, a);
   else
     prefill_kernel<false><<<(unsigned)grid, kPfThreads, smem, st>>>(h.tm_k, h.tm_v, a);
+  profile_after(st);
   count_launch();
   return cudaGetLastError();
 }

@@ -180,6 +180,19 @@ const char* hyb_last_error(void);
 /* Number of kernels this library has launched in the process so far. */
 uint64_t hyb_launch_count(void);
 
+/*
+ * Profiling aid.  `events` is a host array of 2 * n_pairs cudaEvent_t handles
+ * (passed as void*) owned by the caller.  The next n_pairs launches of an
+ * attention kernel (the prefill attention kernel or the decode split-KV
+ * kernel) each record events[2i] just before and events[2i+1] just after the
+ * launch, on the launch's stream.  n_pairs = 0 (or events = NULL) disables
+ * it.  The array must stay valid until all pairs are used or profiling is
+ * disabled.  Not thread-safe with concurrent library calls.
+ */
+hyb_status hyb_profile_events(void* const* events, int32_t n_pairs);
+/* Pairs recorded since the last hyb_profile_events call. */
+int32_t hyb_profile_pairs_used(void);
+
 #ifdef __cplusplus
 }
 #endif
