@@ -35,7 +35,7 @@ LIB_PATH = os.path.join(_PKG, "_lib", "libhyb_attn.so")
 EXPORTED = (
     "hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill_workspace_size", "hyb_attn_prefill",
     "hyb_attn_decode_workspace_size", "hyb_attn_decode", "hyb_device_error", "hyb_last_error",
-    "hyb_launch_count", "hyb_profile_events", "hyb_profile_pairs_used",
+    "hyb_launch_count", "hyb_profile_events", "hyb_profile_pairs_used", "hyb_attn_decode_noalloc",
 )
 
 
@@ -82,6 +82,8 @@ def load(path: str = LIB_PATH):
     lib.hyb_attn_decode_workspace_size.argtypes = [i32, i32, i64]
     lib.hyb_attn_decode_workspace_size.restype = sz
     lib.hyb_attn_decode.argtypes = [vp, vp, vp, pc, i32, i64, vp, vp, sz, vp]
+    lib.hyb_attn_decode_noalloc.argtypes = [vp, vp, vp, pc, i32, i64, vp, vp]
+    lib.hyb_attn_decode_noalloc.restype = ctypes.c_int
     lib.hyb_device_error.argtypes = [ctypes.POINTER(i32), i32, vp]
     lib.hyb_last_error.restype = ctypes.c_char_p
     lib.hyb_launch_count.restype = ctypes.c_uint64
@@ -226,6 +228,25 @@ def hyb_attn_decode(q, gate, cache: KVCache, pos=None, max_len: int = 0, out=Non
     wsz = workspace.numel() * workspace.element_size()
     _check(load().hyb_attn_decode(_ptr(q), _ptr(gate), _ptr(pos), cache.ref, cache.layer_type, max_len,
                                   _ptr(out), _ptr(workspace), wsz, _stream(stream)))
+    return out
+
+
+def hyb_attn_decode_noalloc(q, gate, cache: KVCache, pos=None, max_len: int = 0, out=None, stream=None):
+    """hyb_attn_decode without a workspace: for callers that may not allocate
+    device memory while decoding.  The split partials go to a fixed 4 MiB
+    scratch inside the library, shared by all calls (calls that overlap on
+    the GPU race on it).  `out` should be preallocated by such callers; when
+    it is None a tensor is allocated here for convenience."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous() or tuple(q.shape[1:]) != (N_Q_HEADS, HEAD_DIM):
+        raise ValueError("q must be contiguous bf16 [B, 16, 256]")
+    B = q.shape[0]
+    if gate is not None and (gate.dtype != torch.bfloat16 or not gate.is_contiguous()
+                             or tuple(gate.shape) != (B, N_Q_HEADS)):
+        raise ValueError("gate must be contiguous bf16 [B, 16]")
+    if out is None:
+        out = torch.empty_like(q)
+    _check(load().hyb_attn_decode_noalloc(_ptr(q), _ptr(gate), _ptr(pos), cache.ref, cache.layer_type, max_len,
+                                          _ptr(out), _stream(stream)))
     return out
 
 

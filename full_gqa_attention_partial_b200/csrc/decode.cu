@@ -15,6 +15,8 @@
 // the warp-level MMA keeps the instruction count per key low.
 //
 // Warps 0-3 consume (16 keys each per stage), warp 4 issues the TMA loads.
+#include <mutex>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -343,6 +345,46 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
                                                    reinterpret_cast<__nv_bfloat16*>(h.out), h.n_splits);
   count_launch();
   return cudaGetLastError();
+}
+
+// ---------------------------------------------------------------------------
+// Fixed scratch for hyb_attn_decode_noalloc.
+//
+// Some callers may not allocate device memory on their call path -- a plugin
+// running inside a host application that owns every device allocation, or a
+// latency-critical decode loop where cudaMalloc / cudaFree would stall the
+// device.  For them the split partials live in this file-scope array instead
+// of a caller workspace.  Every GPU that loads the library holds it (4 MiB)
+// until the process exits.  All calls share it and it keeps the previous
+// call's contents; nothing in it needs to start at zero, because every split
+// CTA writes its partial output and log-sum-exp before the combine kernel
+// reads them.  Calls whose kernels overlap on the GPU (different streams
+// without ordering between them) race on it.
+// ---------------------------------------------------------------------------
+constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
+static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
+
+// Device address of g_decode_scratch on the current device.  In host code
+// the array's name is only a host-side stand-in, so the address is looked
+// up with cudaGetSymbolAddress, once per device, the first time a device
+// uses it (with that device current), and cached.
+cudaError_t decode_noalloc_scratch(void** ptr, size_t* bytes) {
+  static std::mutex mu;
+  static void* addr[128] = {};
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_decode_scratch);
+    if (e != cudaSuccess) return e;
+    addr[dev] = p;
+  }
+  *ptr = addr[dev];
+  *bytes = kNoAllocScratchBytes;
+  return cudaSuccess;
 }
 
 cudaError_t decode_set_smem_attr() {

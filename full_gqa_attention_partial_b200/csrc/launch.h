@@ -69,6 +69,9 @@ struct DecodeHost {
 };
 cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st);
 int decode_num_splits(bool full, int B, int64_t max_len);
+// Address and size of the library's fixed decode scratch on the current
+// device (looked up on first use per device).
+cudaError_t decode_noalloc_scratch(void** ptr, size_t* bytes);
 size_t decode_smem_bytes();
 
 }  // namespace hyb

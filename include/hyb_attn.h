@@ -169,6 +169,33 @@ hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos,
                            void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * hyb_attn_decode without a workspace.  The pages describe no counterpart:
+ * this entry point exists for callers that may not allocate device memory
+ * on their call path -- for example a plugin inside a host application that
+ * owns every device allocation, or a latency-critical decode loop in which a
+ * cudaMalloc / cudaFree would stall the whole device.  It computes exactly
+ * what hyb_attn_decode computes (same arguments, minus the workspace) and
+ * allocates nothing; the split partials go to a fixed 4 MiB scratch array
+ * inside the library, which every GPU that loads the library holds until
+ * the process exits.
+ *   Limit: batch x 16 heads x splits x 1028 bytes (plus alignment) must fit
+ *   in 4 MiB, i.e. hyb_attn_decode_workspace_size(layer_type, batch,
+ *   max_len) <= 4194304; larger calls return HYB_EOVERFLOW and enqueue
+ *   nothing.
+ *   Set-up: the first call on a device looks up the scratch's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call
+ *   before any stream capture.
+ *   Sharing: every call uses the same scratch, which keeps the previous
+ *   call's contents (nothing in it needs to start at zero).  Calls whose
+ *   kernels can overlap on the GPU -- e.g. on two streams without ordering
+ *   between them -- race on it and give wrong results.
+ * Errors: as hyb_attn_decode, plus HYB_EOVERFLOW above the limit.
+ */
+hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_t* pos,
+                                   const hyb_kv_cache* cache, int32_t layer_type, int64_t max_len,
+                                   void* out, void* stream);
+
+/*
  * Synchronises `stream`, copies the current device's error word to
  * *flags (host) and, if clear != 0, resets it.
  */
