@@ -72,14 +72,16 @@ class Dist:
         self.rank = int(os.environ.get("RANK", "0"))
         self.local = int(os.environ.get("LOCAL_RANK", "0"))
         self.pg = None
+        self.device = "cuda"
 
     def init(self, backend="nccl"):
+        self.device = "cuda" if backend == "nccl" else "cpu"
         if self.world > 1:
             import datetime
             import torch.distributed as dist
             dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
             self.pg = dist
-        if torch.cuda.is_available():
+        if backend == "nccl" and torch.cuda.is_available():
             torch.cuda.set_device(self.local)
 
     def barrier(self):
@@ -89,9 +91,17 @@ class Dist:
     def max(self, x: float) -> float:
         if not self.pg:
             return x
-        t = torch.tensor([x], dtype=torch.float64, device="cuda")
+        t = torch.tensor([x], dtype=torch.float64, device=self.device)
         self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
         return float(t.item())
+
+    def aggregate(self, units_per_rank: float, ms_this_rank: float):
+        """Whole-job throughput: every rank's units over the slowest rank's time.
+
+        Returns (units per second, max ms).  Weak scaling: each rank processes
+        the same per-rank work, so the job processed world * units_per_rank."""
+        ms = self.max(ms_this_rank)
+        return self.world * units_per_rank / (ms / 1e3), ms
 
     def close(self):
         if self.pg:
@@ -204,7 +214,7 @@ def bench_main(hyb, args, dist: Dist, peaks):
     torch.cuda.synchronize()
     dist.barrier()
     launches = hyb.hyb_launch_count() - l0
-    ms = dist.max(ev0.elapsed_time(ev1))
+    rate, ms = dist.aggregate(args.steps * step_flops, ev0.elapsed_time(ev1))
     assert hyb.hyb_device_error() == 0
     kt = timer.times_ms()
     per_layer = {li: kt[li::len(GROUP_LAYERS)] for li in range(len(GROUP_LAYERS))}
@@ -216,7 +226,7 @@ def bench_main(hyb, args, dist: Dist, peaks):
     achieved = flops(T_MAIN, FULL) / (full_ms / 1e3) / 1e12
     kernel_share = sum(kt) / (ms / 1.0) if ms > 0 else None
     res = {
-        "value": dist.world * args.steps * step_flops / total_s / 1e12,
+        "value": rate / 1e12,
         "ms_per_step": ms / args.steps,
         "gpu_launches": launches,
         "roofline": {
@@ -259,8 +269,8 @@ def bench_main(hyb, args, dist: Dist, peaks):
         e2e_step(args.warmup + i)
     ev1.record()
     torch.cuda.synchronize()
-    e2e_ms = dist.max(ev0.elapsed_time(ev1))
-    res["e2e"] = {"value": dist.world * args.steps * step_flops / (e2e_ms / 1e3) / 1e12, "unit": "TFLOP/s",
+    e2e_rate, e2e_ms = dist.aggregate(args.steps * step_flops, ev0.elapsed_time(ev1))
+    res["e2e"] = {"value": e2e_rate / 1e12, "unit": "TFLOP/s",
                   "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps}
     del caches, e2e_caches, host_in, host_out
     return res, layers
@@ -501,6 +511,44 @@ def run_reference(args, dist: Dist):
             "e2e": {"value": value, "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def run_case(hyb, args):
+    """One kernel on a small configuration, for profiler captures: 1 warm-up + args.steps launches."""
+    from full_gqa_attention_partial_b200 import synth
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if args.case.startswith("prefill"):
+        lt = FULL if args.case == "prefill_full" else SLIDING
+        T, B = args.seq, args.batch
+        x = synth.prefill_inputs(B, T, seed=layer_seed(1, 3), device="cuda")
+        ws = hyb.alloc_workspace(hyb.hyb_attn_prefill_workspace_size(lt, B, T, False))
+        out = torch.empty(B, T, H, D, dtype=torch.bfloat16, device="cuda")
+        fn = lambda: hyb.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], x["pos"], lt, out=out, workspace=ws)
+        work = B * flops(T, lt)
+        unit = "TFLOP/s"
+    else:
+        lt = FULL if args.case == "decode_full" else SLIDING
+        B, L = args.batch, args.seq
+        cap = L + args.steps + 2
+        c = fill_full_cache(hyb, B, L, cap, seed=2) if lt == FULL else fill_ring_cache(hyb, B, L, 3, 17)
+        xq = synth.decode_query(B, seed=5, device="cuda")
+        ml = cap if lt == FULL else W
+        ws = hyb.alloc_workspace(hyb.hyb_attn_decode_workspace_size(lt, B, ml))
+        out = torch.empty(B, H, D, dtype=torch.bfloat16, device="cuda")
+        fn = lambda: hyb.hyb_attn_decode(xq["q"], xq["gate"], c, max_len=ml, out=out, workspace=ws)
+        work = B * min(L, cap if lt == FULL else W) * 4096
+        unit = "GB/s"
+    fn()
+    torch.cuda.synchronize()
+    timer = hyb.KernelTimer(args.steps)
+    with timer:
+        for _ in range(args.steps):
+            fn()
+    ms = statistics.mean(timer.times_ms())
+    assert hyb.hyb_device_error() == 0
+    rate = work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
+    print(json.dumps({"case": args.case, "batch": args.batch, "seq": args.seq, "kernel_ms": ms,
+                      "rate": rate, "unit": unit, "work_per_launch": work}), flush=True)
+
+
 # ---------------------------------------------------------------------------
 def main():
     ap = argparse.ArgumentParser()
@@ -515,6 +563,10 @@ def main():
     ap.add_argument("--full-traffic", type=float, default=None,
                     help="DRAM bytes per full-layer prefill launch from an ncu capture (reported as traffic)")
     ap.add_argument("--decode-traffic", type=float, default=None)
+    ap.add_argument("--case", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_sliding"],
+                    default=None, help="time one kernel on a small configuration (profiling)")
+    ap.add_argument("--seq", type=int, default=16384)
+    ap.add_argument("--batch", type=int, default=1)
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
@@ -528,6 +580,9 @@ def main():
     dist.init()
     import full_gqa_attention_partial_b200 as hyb
     hyb.load()
+    if args.case:
+        run_case(hyb, args)
+        return
     peaks = load_peaks()
     clocks = Clocks()
     clocks.start()
