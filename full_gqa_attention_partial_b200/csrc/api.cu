@@ -107,15 +107,15 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 4-D map {256 dims, rows, 4 KV heads, batch} of bf16 with 64 x 64 boxes and
-// 128-byte swizzle (one box = 64 rows of 128 bytes).
+// 4-D map {256 dims, rows, 4 KV heads, batch} of bf16 with boxes of 64 dims x
+// box_rows rows and 128-byte swizzle (one box = box_rows rows of 128 bytes).
 hyb_status make_kv_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t batch, uint64_t row_bytes,
-                       uint64_t head_bytes, uint64_t batch_bytes, const char* what) {
+                       uint64_t head_bytes, uint64_t batch_bytes, uint32_t box_rows, const char* what) {
   auto enc = encode_fn();
   if (!enc) return fail(HYB_EUNSUPPORTED, "cuTensorMapEncodeTiled is not available from the driver");
   cuuint64_t dims[4] = {(cuuint64_t)kD, rows, (cuuint64_t)kHkv, batch};
   cuuint64_t strides[3] = {row_bytes, head_bytes, batch_bytes};
-  cuuint32_t box[4] = {64, 64, 1, 1};
+  cuuint32_t box[4] = {64, box_rows, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -142,11 +142,13 @@ hyb_status check_cache(const hyb_kv_cache* c) {
   return HYB_OK;
 }
 
-hyb_status cache_maps(const hyb_kv_cache* c, CUtensorMap* mk, CUtensorMap* mv) {
+hyb_status cache_maps(const hyb_kv_cache* c, CUtensorMap* mk, CUtensorMap* mv, uint32_t k_box_rows,
+                      uint32_t v_box_rows) {
   const uint64_t row = kD * 2, head = (uint64_t)c->capacity * row, batch = head * kHkv;
-  hyb_status s = make_kv_map(mk, c->k, (uint64_t)c->capacity, (uint64_t)c->batch, row, head, batch, "cache K");
+  hyb_status s =
+      make_kv_map(mk, c->k, (uint64_t)c->capacity, (uint64_t)c->batch, row, head, batch, k_box_rows, "cache K");
   if (s != HYB_OK) return s;
-  return make_kv_map(mv, c->v, (uint64_t)c->capacity, (uint64_t)c->batch, row, head, batch, "cache V");
+  return make_kv_map(mv, c->v, (uint64_t)c->capacity, (uint64_t)c->batch, row, head, batch, v_box_rows, "cache V");
 }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -324,9 +326,11 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
     r.mode = 2;
     if ((e = launch_rope_store(full, r, st)) != cudaSuccess) return cuda_fail(e, "rope K launch");
     const uint64_t hb = (uint64_t)T * row_bytes;
-    if ((s = make_kv_map(&ph.tm_k, workspace, T, B, row_bytes, hb, hb * kHkv, "rotated K")) != HYB_OK) return s;
-    if ((s = make_kv_map(&ph.tm_v, v, T, B, (uint64_t)kv_row_stride * 2, row_bytes,
-                         (uint64_t)T * kv_row_stride * 2, "V")) != HYB_OK)
+    if ((s = make_kv_map(&ph.tm_k, workspace, T, B, row_bytes, hb, hb * kHkv, prefill_k_box_rows(), "rotated K")) !=
+        HYB_OK)
+      return s;
+    if ((s = make_kv_map(&ph.tm_v, v, T, B, (uint64_t)kv_row_stride * 2, row_bytes, (uint64_t)T * kv_row_stride * 2,
+                         prefill_v_box_rows(), "V")) != HYB_OK)
       return s;
     if ((e = launch_prefill(full, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
     return HYB_OK;
@@ -341,7 +345,7 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
     r.mode = 0;
     r.len = cache->len;
     if ((e = launch_rope_store(true, r, st)) != cudaSuccess) return cuda_fail(e, "append launch");
-    if ((s = cache_maps(cache, &ph.tm_k, &ph.tm_v)) != HYB_OK) return s;
+    if ((s = cache_maps(cache, &ph.tm_k, &ph.tm_v, prefill_k_box_rows(), prefill_v_box_rows())) != HYB_OK) return s;
     ph.qbase = cache->len;
     ph.ctx_mode = 0;
     if ((e = launch_prefill(true, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
@@ -368,8 +372,10 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
   r.len = cache->len;  // default positions: len + t
   if ((e = launch_rope_store(false, r, st)) != cudaSuccess) return cuda_fail(e, "context rope launch");
   const uint64_t hb = (uint64_t)rows * row_bytes;
-  if ((s = make_kv_map(&ph.tm_k, ck, rows, B, row_bytes, hb, hb * kHkv, "context K")) != HYB_OK) return s;
-  if ((s = make_kv_map(&ph.tm_v, cv, rows, B, row_bytes, hb, hb * kHkv, "context V")) != HYB_OK) return s;
+  if ((s = make_kv_map(&ph.tm_k, ck, rows, B, row_bytes, hb, hb * kHkv, prefill_k_box_rows(), "context K")) != HYB_OK)
+    return s;
+  if ((s = make_kv_map(&ph.tm_v, cv, rows, B, row_bytes, hb, hb * kHkv, prefill_v_box_rows(), "context V")) != HYB_OK)
+    return s;
   ph.qbase = cache->len;
   ph.ctx_mode = 1;
   if ((e = launch_prefill(false, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
@@ -424,7 +430,7 @@ hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos, 
   if ((s = ensure_device()) != HYB_OK) return s;
 
   DecodeHost d;
-  if ((s = cache_maps(c, &d.tm_k, &d.tm_v)) != HYB_OK) return s;
+  if ((s = cache_maps(c, &d.tm_k, &d.tm_v, 64, 64)) != HYB_OK) return s;
   d.q = q;
   d.gate = gate;
   d.pos = pos;
@@ -469,7 +475,7 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
 
   DecodeHost d;
-  if ((s = cache_maps(c, &d.tm_k, &d.tm_v)) != HYB_OK) return s;
+  if ((s = cache_maps(c, &d.tm_k, &d.tm_v, 64, 64)) != HYB_OK) return s;
   d.q = q;
   d.gate = gate;
   d.pos = pos;

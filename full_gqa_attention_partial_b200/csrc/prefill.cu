@@ -1,26 +1,32 @@
 // Prefill attention on 5th-generation tensor cores (tcgen05, sm_100a).
 //
-// One CTA computes a 128-query tile of one query head:
-//   O[t] = sum_j softmax_j(q_t . k_j / 16) v_j over the keys j that the layer
-//   type lets t see, times sigmoid(gate[t, h]),
-// with query head h reading KV head h / 4 (GQA, 16 / 4 heads, head_dim 256:
-// "百万 Token 塞进 4B ..." §"省显存的第二板斧：GQA、融合投影与输出门控"), the
-// causal mask on full layers and the 512-key band (the query and the 511
-// keys before it) on sliding layers (same page, §"混合注意力").  Key tiles
-// wholly outside the band are never loaded.
+// A cluster of two CTAs (a CTA pair) computes one 128-query tile for two
+// query heads of the same KV group (GQA, 16 query / 4 KV heads, head_dim 256:
+// "百万 Token 塞进 4B ..." §"省显存的第二板斧：GQA、融合投影与输出门控"):
+//   O[t] = sum_j softmax_j(q_t . k_j / 16) v_j, times sigmoid(gate[t, h]),
+// over the keys j the layer type lets t see: causal on full layers, the
+// query and the 511 keys before it on sliding layers (same page, §"混合注意力").
+// Key tiles wholly outside the band are never loaded.
 //
-// Roles (192 threads):
-//   warps 0-3  rotate the query tile (rotate-half RoPE, theta / rotary dim
-//              per layer type) into tensor memory, then run the online
-//              softmax row by row (one TMEM lane = one query row per thread),
-//              and finally the epilogue (1/l, sigmoid gate, bf16 store);
-//   warp 4     TMA producer: K and V tiles (64 keys x 256 dims, four 64x64
-//              boxes with 128-byte swizzle) into a 6-slot shared-memory ring;
-//   warp 5     allocates tensor memory; one lane issues all tcgen05.mma.
-// Tensor memory (512 columns x 128 lanes of 32 bit):
+// The pair shares every K/V tile: each CTA loads half of it (32 of the 64
+// keys of a K tile, 128 of the 256 dims of a V tile) and the pair MMAs
+// (cta_group::2, M = 256: 128 rows per CTA) read both halves, so each SM
+// draws 32 KB from L2 per 64-key tile instead of 64 KB.
+//
+// Roles in each CTA (192 threads):
+//   warps 0-3  rotate this CTA's query head into tensor memory (rotate-half
+//              RoPE, theta / rotary dim per layer type), then the online
+//              softmax (one TMEM lane = one query row per thread) and the
+//              epilogue (1/l, sigmoid gate, bf16 store);
+//   warp 4     TMA producer for this CTA's halves of the K/V tiles, into a
+//              12-slot ring of 16 KB; bytes are counted on CTA 0's barriers;
+//   warp 5     tensor-memory allocation (both CTAs); in CTA 0 the warp runs
+//              the MMA loop convergently and one elected lane issues every
+//              MMA of the pair and commits to both CTAs.
+// Tensor memory, per CTA (512 columns x 128 lanes of 32 bit):
 //   [0,128)   Q as bf16 pairs (A operand of S = Q K^T)
-//   [128,192) S buffer 0, [192,256) S buffer 1 (fp32 64 columns each); P of
-//             a tile (bf16 pairs) overwrites the first 32 columns of its S
+//   [128,192) S buffer 0, [192,256) S buffer 1 (fp32, 64 keys each); P of a
+//             tile (bf16 pairs) overwrites the first 32 columns of its S
 //             buffer and is the A operand of O += P V
 //   [256,512) O accumulator, fp32 128 x 256.
 // Softmax in the log2 domain with a lazily updated row maximum: the running
@@ -31,28 +37,30 @@
 
 namespace hyb {
 
-constexpr int kBM = 128;
-constexpr int kBN = 64;
-constexpr int kSlots = 6;
-constexpr int kSlotBytes = kBN * kD * 2;  // 32 KB
-constexpr int kPfBox = kBN * 128;         // 8 KB: 64 keys x 64 dims
+constexpr int kBM = 128;                  // query rows per CTA
+constexpr int kBN = 64;                   // keys per tile (shared by the pair)
+constexpr int kSlots = 12;
+constexpr int kSlotBytes = 16384;         // one CTA's half of a K or V tile
+constexpr int kKBoxRows = kBN / 2;        // K half: 32 keys x 64 dims per box
+constexpr int kKBox = kKBoxRows * 128;    // 4 KB
+constexpr int kVBox = kBN * 128;          // V half: 64 keys x 64 dims per box, 8 KB
 constexpr int kPfThreads = 192;
 constexpr uint32_t kColQ = 0;
-constexpr uint32_t kColS0 = 128;
-__device__ __forceinline__ uint32_t col_s(int sb) { return sb ? 192u : kColS0; }
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;
+__device__ __forceinline__ uint32_t col_s(int sb) { return sb ? 192u : 128u; }
 
 struct PfSmem {
   uint8_t slot[kSlots][kSlotBytes];  // 1024-byte aligned
   double inv_freq[128];
-  uint64_t full[kSlots];
-  uint64_t empty[kSlots];
-  uint64_t q_ready;
+  uint64_t full[kSlots];   // CTA 0's count both CTAs' bytes
+  uint64_t empty[kSlots];  // per CTA, committed by the MMA issuer
+  uint64_t q_ready;        // CTA 0: one arrival per softmax warp of the pair
   uint64_t s_full[2];
-  uint64_t p_full[2];
-  uint64_t o_done;
-  uint64_t mma_done;   // every MMA issued by this CTA has completed (before TMEM is freed)
+  uint64_t p_full[2];      // CTA 0: one arrival per softmax warp of the pair
+  uint64_t o_done;         // each P.V completed
+  uint64_t o_final;        // the last P.V completed
+  uint64_t mma_done;       // every MMA of the pair completed
   uint32_t tmem_base;
 };
 
@@ -69,7 +77,7 @@ struct PfArgs {
   int B, T, n_mtiles;
 };
 
-// Load order shared by the producer and the MMA issuer:
+// Load order shared by the producers and the MMA issuer:
 //   K0, (K1, V0), (K2, V1), ..., (K_{n-1}, V_{n-2}), V_{n-1}
 __device__ __forceinline__ void load_of(int i, int n, bool& is_k, int& tile) {
   if (i == 0) { is_k = true; tile = 0; return; }
@@ -80,7 +88,6 @@ __device__ __forceinline__ void load_of(int i, int n, bool& is_k, int& tile) {
 
 // Rotates 32 dims [k0, k0+32) against their partners [k0+R/2, ...) for one
 // query row: x1 / x2 hold 16 packed bf16 words each; results replace them.
-template <bool FULL>
 __device__ __forceinline__ void rotate32(uint32_t (&x1)[16], uint32_t (&x2)[16], int k0, int p,
                                          const double* inv_freq) {
 #pragma unroll
@@ -112,22 +119,25 @@ __device__ __forceinline__ void load_words16(const __nv_bfloat16* src, bool vali
 }
 
 template <bool FULL>
-__global__ void __launch_bounds__(kPfThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, PfArgs a) {
   extern __shared__ uint8_t smem_raw[];
   PfSmem& sm = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int R = RopeCfg<FULL>::R;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();   // 0 = the CTA that issues the pair's MMAs
 
-  // ---- work item: longest query tiles first, heads of one tile adjacent ----
-  const int per_tile = a.B * kHq;
-  const int mt = a.n_mtiles - 1 - (int)(blockIdx.x / per_tile);
-  const int rem = blockIdx.x % per_tile;
-  const int h = rem % kHq;
-  const int b = rem / kHq;
-  const int kvh = h / kGroup;
+  // ---- work item: longest query tiles first; the pairs of one tile adjacent ----
+  const int pair = blockIdx.x >> 1;
+  const int per_tile = a.B * (kHq / 2);
+  const int mt = a.n_mtiles - 1 - pair / per_tile;
+  const int rem = pair % per_tile;
+  const int hp = rem % (kHq / 2);
+  const int b = rem / (kHq / 2);
+  const int kvh = hp >> 1;
+  const int h = kvh * kGroup + (hp & 1) * 2 + (int)rank;
   const int m0 = mt * kBM;
-  const int qb = a.qbase ? a.qbase[b] : 0;        // sequence index of token 0
+  const int qb = a.qbase ? a.qbase[b] : 0;             // sequence index of token 0
   const int kb = a.ctx_mode ? qb - (kWindow - 1) : 0;  // sequence index of key row 0
   const int rows_valid = min(kBM, a.T - m0);
   const int q_lo = qb + m0, q_hi = qb + m0 + rows_valid - 1;
@@ -141,27 +151,28 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
-    mbar_init(&sm.q_ready, kBM);
+    mbar_init(&sm.q_ready, 8);
     for (int s = 0; s < 2; ++s) {
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.p_full[s], kBM);
+      mbar_init(&sm.p_full[s], 8);
     }
     mbar_init(&sm.o_done, 1);
+    mbar_init(&sm.o_final, 1);
     mbar_init(&sm.mma_done, 1);
     fence_barrier_init();
   }
   if (warp == 5) {
-    tmem_alloc(&sm.tmem_base, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(&sm.tmem_base, 512);
+    tmem_relinquish_pair();
   }
   if (threadIdx.x < R / 2) sm.inv_freq[threadIdx.x] = rope_inv_freq(RopeCfg<FULL>::theta, threadIdx.x, R);
   tc_fence_before();
-  __syncthreads();
+  cluster_sync();   // barriers of both CTAs initialised before any cross-CTA arrive
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
   if (warp == 4) {
-    // ======================= TMA producer =======================
+    // ======================= TMA producer (both CTAs) =======================
     if (lane == 0) {
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
@@ -172,54 +183,62 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         load_of(i, n, is_k, tile);
         const int slot = i % kSlots;
         if (i >= kSlots && !mbar_wait(&sm.empty[slot], ((i / kSlots) - 1) & 1)) break;
-        mbar_arrive_expect_tx(&sm.full[slot], kSlotBytes);
+        if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
         const uint32_t dst = smem_u32(sm.slot[slot]);
         const int row = (j_lo + tile) * kBN;
-        const CUtensorMap* tm = is_k ? &tm_k : &tm_v;
+        if (is_k) {
 #pragma unroll
-        for (int box = 0; box < 4; ++box) tma_load_4d(dst + box * kPfBox, tm, &sm.full[slot], box * 64, row, kvh, b);
+          for (int box = 0; box < 4; ++box)
+            tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row + kKBoxRows * (int)rank, kvh, b);
+        } else {
+#pragma unroll
+          for (int box = 0; box < 2; ++box)
+            tma_load_4d_pair(dst + box * kVBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * box, row, kvh, b);
+        }
         issued = i + 1;
       }
-      for (int i = max(0, issued - kSlots); i < issued; ++i) mbar_wait(&sm.full[i % kSlots], (i / kSlots) & 1);
+      if (rank == 0)  // every load of the pair completes on CTA 0's barriers
+        for (int i = max(0, issued - kSlots); i < issued; ++i) mbar_wait(&sm.full[i % kSlots], (i / kSlots) & 1);
     }
   } else if (warp == 5) {
-    // ======================= MMA issuer =======================
-    if (lane == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(kBM, kBN, false);   // S = Q K^T, B K-major
-      constexpr uint32_t idesc_o = idesc_bf16(kBM, kD, true);     // O += P V, B MN-major
-      bool ok = mbar_wait(&sm.q_ready, 0);
+    // ======================= MMA issuer (CTA 0, whole warp, one lane issues) =======================
+    if (rank == 0) {
+      constexpr uint32_t idesc_s = idesc_bf16(2 * kBM, kBN, false);   // S = Q K^T, B K-major
+      constexpr uint32_t idesc_o = idesc_bf16(2 * kBM, kD, true);     // O += P V, B MN-major
+      bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_ready, 0));
       tc_fence_after();
       for (int i = 0; ok && i < 2 * n; ++i) {
         bool is_k;
         int tile;
         load_of(i, n, is_k, tile);
         const int slot = i % kSlots;
-        if (!(ok = mbar_wait(&sm.full[slot], (i / kSlots) & 1))) break;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (i / kSlots) & 1)))) break;
         tc_fence_after();
         const uint32_t saddr = smem_u32(sm.slot[slot]);
         const int sb = tile & 1;
         if (is_k) {
 #pragma unroll
           for (int s = 0; s < kD / 16; ++s) {
-            const uint64_t bdesc = smem_desc_sw128(saddr + (s >> 2) * kPfBox + (s & 3) * 32, 16, 1024);
-            mma_ts(tmem + col_s(sb), tmem + kColQ + 8 * s, bdesc, idesc_s, s > 0 ? 1u : 0u);
+            const uint64_t bdesc = smem_desc_sw128(saddr + (s >> 2) * kKBox + (s & 3) * 32, 16, 1024);
+            mma_ts_pair_warp(tmem + col_s(sb), tmem + kColQ + 8 * s, bdesc, idesc_s, s > 0 ? 1u : 0u);
           }
-          mma_commit(&sm.empty[slot]);
-          mma_commit(&sm.s_full[sb]);
+          mma_commit_pair_warp(&sm.empty[slot]);
+          mma_commit_pair_warp(&sm.s_full[sb]);
         } else {
-          if (!(ok = mbar_wait(&sm.p_full[sb], (tile >> 1) & 1))) break;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[sb], (tile >> 1) & 1)))) break;
           tc_fence_after();
 #pragma unroll
           for (int s = 0; s < kBN / 16; ++s) {
-            const uint64_t bdesc = smem_desc_sw128(saddr + s * 16 * 128, kPfBox, 1024);
-            mma_ts(tmem + kColO, tmem + col_s(sb) + 8 * s, bdesc, idesc_o, (tile > 0 || s > 0) ? 1u : 0u);
+            const uint64_t bdesc = smem_desc_sw128(saddr + s * 16 * 128, kVBox, 1024);
+            mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 8 * s, bdesc, idesc_o, (tile > 0 || s > 0) ? 1u : 0u);
           }
-          mma_commit(&sm.empty[slot]);
-          mma_commit(&sm.o_done);
+          mma_commit_pair_warp(&sm.empty[slot]);
+          mma_commit_pair_warp(&sm.o_done);
+          if (tile == n - 1) mma_commit_pair_warp(&sm.o_final);
         }
       }
-      // also on an early exit: wait until nothing this thread issued is in flight
-      mma_commit(&sm.mma_done);
+      // also on an early exit: wait until nothing the pair issued is in flight
+      mma_commit_pair_warp(&sm.mma_done);
       mbar_wait(&sm.mma_done, 0);
     }
   } else {
@@ -237,7 +256,7 @@ __global__ void __launch_bounds__(kPfThreads, 1)
       uint32_t x1[16], x2[16];
       load_words16(qrow, valid, x1);
       load_words16(qrow + 32, valid, x2);
-      rotate32<FULL>(x1, x2, 0, p, sm.inv_freq);
+      rotate32(x1, x2, 0, p, sm.inv_freq);
       tmem_st16(trow + kColQ + 0, x1);
       tmem_st16(trow + kColQ + 16, x2);
 #pragma unroll
@@ -252,14 +271,18 @@ __global__ void __launch_bounds__(kPfThreads, 1)
         uint32_t x1[16], x2[16];
         load_words16(qrow + 32 * c, valid, x1);
         load_words16(qrow + 128 + 32 * c, valid, x2);
-        rotate32<FULL>(x1, x2, 32 * c, p, sm.inv_freq);
+        rotate32(x1, x2, 32 * c, p, sm.inv_freq);
         tmem_st16(trow + kColQ + 16 * c, x1);
         tmem_st16(trow + kColQ + 64 + 16 * c, x2);
       }
     }
     tmem_wait_st();
     tc_fence_before();
-    mbar_arrive(&sm.q_ready);
+    __syncwarp();
+    if (lane == 0) {
+      if (rank == 0) mbar_arrive(&sm.q_ready);
+      else mbar_arrive_remote(&sm.q_ready, 0);
+    }
 
     // ---- online softmax over the key tiles ----
     const float scale_log2 = 0.0625f * 1.4426950408889634f;
@@ -292,52 +315,62 @@ __global__ void __launch_bounds__(kPfThreads, 1)
           if (!vis) s[c] = -INFINITY;
         }
       }
-      float mx = s[0];
+      // row maximum: pairwise tree (short dependency chains)
+      float mx[32];
 #pragma unroll
-      for (int c = 1; c < 64; ++c) mx = fmaxf(mx, s[c]);
-      const float m_tile = mx * scale_log2;
+      for (int c = 0; c < 32; ++c) mx[c] = fmaxf(s[c], s[c + 32]);
+#pragma unroll
+      for (int w = 16; w >= 1; w >>= 1)
+#pragma unroll
+        for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
+      const float m_tile = mx[0] * scale_log2;
       const float m_new = fmaxf(m_run, m_tile);
       const bool rescale = m_new > m_run + kRescaleThreshold;
       const float m_use = rescale ? m_new : m_run;
       const float base = (m_use == -INFINITY) ? 0.f : m_use;
-      const float alpha = rescale ? exp2f(m_run - m_use) : 1.f;
-      float sum = 0.f;
+      const float alpha = rescale ? ex2(m_run - m_use) : 1.f;
       uint32_t pw[32];
+      float ps[8];
+#pragma unroll
+      for (int c = 0; c < 8; ++c) ps[c] = 0.f;
 #pragma unroll
       for (int w = 0; w < 32; ++w) {
-        const float p0 = exp2f(fmaf(s[2 * w], scale_log2, -base));
-        const float p1 = exp2f(fmaf(s[2 * w + 1], scale_log2, -base));
-        sum += p0 + p1;
+        const float p0 = ex2(fmaf(s[2 * w], scale_log2, -base));
+        const float p1 = ex2(fmaf(s[2 * w + 1], scale_log2, -base));
+        ps[w & 7] += p0 + p1;
         pw[w] = pack_bf16(p0, p1);
       }
+      const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       l_run = l_run * alpha + sum;
       m_run = m_use;
       tmem_st32(trow + col_s(sb), pw);
       tmem_wait_st();
-      if (j > 0) {
+      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
         // O may only be touched once the previous tile's P.V has landed
         ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done, (j - 1) & 1));
         if (!ok) break;
-        if (__any_sync(0xffffffffu, rescale)) {
-          tc_fence_after();
+        tc_fence_after();
 #pragma unroll 1
-          for (int c8 = 0; c8 < 8; ++c8) {
-            uint32_t ov[32];
-            tmem_ld32(trow + kColO + 32 * c8, ov);
-            tmem_wait_ld();
+        for (int c8 = 0; c8 < 8; ++c8) {
+          uint32_t ov[32];
+          tmem_ld32(trow + kColO + 32 * c8, ov);
+          tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(trow + kColO + 32 * c8, ov);
-          }
-          tmem_wait_st();
+          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+          tmem_st32(trow + kColO + 32 * c8, ov);
         }
+        tmem_wait_st();
       }
       tc_fence_before();
-      mbar_arrive(&sm.p_full[sb]);
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(&sm.p_full[sb]);
+        else mbar_arrive_remote(&sm.p_full[sb], 0);
+      }
     }
 
     // ---- epilogue: O / l * sigmoid(gate) -> bf16 ----
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done, (n - 1) & 1));
+    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, 0));
     if (ok) {
       tc_fence_after();
       float f = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -368,11 +401,13 @@ __global__ void __launch_bounds__(kPfThreads, 1)
     }
   }
 
+  // the peer's shared memory and tensor memory stay alive until both CTAs are done
   tc_fence_before();
   __syncthreads();
+  cluster_sync();
   if (warp == 5) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -388,7 +423,7 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   a.B = h.B;
   a.T = h.T;
   a.n_mtiles = (h.T + kBM - 1) / kBM;
-  const long long grid = (long long)a.n_mtiles * h.B * kHq;
+  const long long grid = (long long)a.n_mtiles * h.B * kHq;   // one CTA per (tile, head), in pairs
   if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidValue;
   const size_t smem = prefill_smem_bytes();
   profile_before(st);
@@ -400,6 +435,10 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   count_launch();
   return cudaGetLastError();
 }
+
+// Box rows of the K and V tensor maps this kernel expects (per-CTA halves).
+int prefill_k_box_rows() { return kKBoxRows; }
+int prefill_v_box_rows() { return kBN; }
 
 cudaError_t prefill_set_smem_attr() {
   const int smem = (int)prefill_smem_bytes();
