@@ -124,6 +124,23 @@ hyb_status make_kv_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t
   return HYB_OK;
 }
 
+// 4-D map {256 dims, 16 heads, T tokens, batch} over query-shaped rows (the
+// raw queries, or the output) with boxes of 64 dims x 1 head x box_rows tokens.
+hyb_status make_q_map(CUtensorMap* m, const void* base, uint64_t T, uint64_t batch, uint64_t token_bytes,
+                      uint32_t box_rows, const char* what) {
+  auto enc = encode_fn();
+  if (!enc) return fail(HYB_EUNSUPPORTED, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)kHq, T, batch};
+  cuuint64_t strides[3] = {(cuuint64_t)kD * 2, token_bytes, T * token_bytes};
+  cuuint32_t box[4] = {64, 1, box_rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HYB_ECUDA, "cuTensorMapEncodeTiled(%s) failed with CUresult %d", what, (int)r);
+  return HYB_OK;
+}
+
 hyb_status check_cache(const hyb_kv_cache* c) {
   if (!c) return fail(HYB_EINVAL, "cache is NULL");
   if (c->type != HYB_SLIDING && c->type != HYB_FULL) return fail(HYB_EINVAL, "cache type %d invalid", c->type);
@@ -301,6 +318,8 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
   const bool full = layer_type == HYB_FULL;
   const uint64_t row_bytes = kD * 2;
   PrefillHost ph;
+  if ((s = make_q_map(&ph.tm_q, q, T, B, (uint64_t)q_row_stride * 2, prefill_q_box_rows(), "Q")) != HYB_OK) return s;
+  if ((s = make_q_map(&ph.tm_o, out, T, B, (uint64_t)kHq * kD * 2, prefill_q_box_rows(), "out")) != HYB_OK) return s;
   ph.q = q;
   ph.q_stride = q_row_stride;
   ph.gate = gate;

@@ -32,8 +32,10 @@ __device__ __forceinline__ void raise_err(int bit) { atomicOr(&g_dev_err, bit); 
 
 // ---------------------------------------------------------------------------
 // RoPE angle: phi = pos * inv_freq in fp64, reduced to [-pi, pi] with a
-// two-term 2*pi (Cody-Waite style reduction), then sin/cos in fp32.  fp32
-// pos * inv_freq alone would be off by ~0.06 rad at pos ~ 2^20.
+// two-term 2*pi (Cody-Waite style reduction), then sin/cos of the reduced
+// angle on the special-function unit (__sincosf: absolute error ~5e-7 on
+// [-pi, pi], far below bf16 resolution).  fp32 pos * inv_freq alone would be
+// off by ~0.06 rad at pos ~ 2^20.
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ double rope_inv_freq(double theta, int k, int R) {
   return pow(theta, -2.0 * (double)k / (double)R);
@@ -47,7 +49,7 @@ __device__ __forceinline__ void rope_sincos(int pos, double inv_freq, float* s, 
   double n = rint(phi * inv_two_pi);
   double r = fma(-n, two_pi_hi, phi);
   r = fma(-n, two_pi_lo, r);
-  sincosf((float)r, s, c);
+  __sincosf((float)r, s, c);
 }
 
 // 2^x on the special-function unit (flush-to-zero; x <= 8 here)
@@ -55,6 +57,16 @@ __device__ __forceinline__ float ex2(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// sin / cos of x = delta * inv_freq for a small integer delta (|x| <~ 2^8):
+// fp32 product, reduction with a two-term fp32 2*pi, then the SFU.
+__device__ __forceinline__ void small_angle_sincos(int delta, float inv_freq_f, float* s, float* c) {
+  const float x = (float)delta * inv_freq_f;
+  const float n = rintf(x * 0.159154943f);
+  float r = fmaf(-n, 6.28318548f, x);     // 2*pi rounded to fp32 ...
+  r = fmaf(-n, -1.74845553e-7f, r);       // ... and the rest of 2*pi
+  __sincosf(r, s, c);
 }
 
 // ---------------------------------------------------------------------------
@@ -141,6 +153,16 @@ __device__ __forceinline__ void tma_load_4d(uint32_t smem_dst, const void* tmap,
       " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_dst),
       "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_u32(bar))
       : "memory");
+}
+// TMA: 4-D tiled store from shared memory (bulk group); rows outside the
+// tensor are not written.
+__device__ __forceinline__ void tma_store_4d(const void* tmap, uint32_t smem_src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%1, %2, %3, %4}], [%5];" ::"l"(tmap),
+               "r"(c0), "r"(c1), "r"(c2), "r"(c3), "r"(smem_src)
+               : "memory");
+}
+__device__ __forceinline__ void tma_store_commit_and_wait() {
+  asm volatile("cp.async.bulk.commit_group;\n\tcp.async.bulk.wait_group 0;" ::: "memory");
 }
 __device__ __forceinline__ void prefetch_tmap(const void* tmap) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(tmap) : "memory");

@@ -42,6 +42,7 @@ cudaError_t launch_fill_i32(int32_t* p, int64_t n, int32_t v, cudaStream_t st);
 // ---- prefill attention (prefill.cu) -----------------------------------------
 struct PrefillHost {
   CUtensorMap tm_k, tm_v;      // 4-D maps {256, rows, 4, B}, 64-dim boxes, 128B swizzle
+  CUtensorMap tm_q, tm_o;      // 4-D maps {256, 16, T, B} over q and out, 64-dim x 128-row boxes
   const void* q = nullptr;     // raw queries
   int64_t q_stride = 0;        // elements between tokens
   const void* gate = nullptr;  // [B][T][16] or null
@@ -54,6 +55,7 @@ struct PrefillHost {
 cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st);
 int prefill_k_box_rows();   // rows (keys) per TMA box of the K map
 int prefill_v_box_rows();   // rows (keys) per TMA box of the V map
+int prefill_q_box_rows();   // rows (tokens) per TMA box of the Q and O maps
 size_t prefill_smem_bytes();
 
 // ---- decode (decode.cu) -------------------------------------------------------

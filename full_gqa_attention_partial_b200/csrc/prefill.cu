@@ -53,6 +53,11 @@ __device__ __forceinline__ uint32_t col_s(int sb) { return sb ? 192u : 128u; }
 struct PfSmem {
   uint8_t slot[kSlots][kSlotBytes];  // 1024-byte aligned
   double inv_freq[128];
+  // rotation tables for the tile's rows (positions p_base + 16 i + j):
+  //   rot_lo[k][j] = (cos, sin)(j * inv_freq_k),               j < 16
+  //   rot_hi[k][i] = (cos, sin)((p_base + 16 i) * inv_freq_k),  i < 8
+  float2 rot_lo[128][16];
+  float2 rot_hi[128][8];
   uint64_t full[kSlots];   // CTA 0's count both CTAs' bytes
   uint64_t empty[kSlots];  // per CTA, committed by the MMA issuer
   uint64_t q_ready;        // CTA 0: one arrival per softmax warp of the pair
@@ -61,8 +66,14 @@ struct PfSmem {
   uint64_t o_done;         // each P.V completed
   uint64_t o_final;        // the last P.V completed
   uint64_t mma_done;       // every MMA of the pair completed
+  uint64_t q_full;         // this CTA's query tile landed (ring slots 8..11)
+  uint64_t q_free;         // the softmax warps have read it
   uint32_t tmem_base;
 };
+// The query tile (4 boxes of 64 dims x 128 rows = 64 KB) arrives in ring slots
+// 8..11 before the K/V stream first reaches them; the output tile leaves
+// through slots 0..3 once every MMA is done.
+constexpr int kQSlot = 8;
 
 size_t prefill_smem_bytes() { return sizeof(PfSmem) + 1024; }
 
@@ -88,9 +99,34 @@ __device__ __forceinline__ void load_of(int i, int n, bool& is_k, int& tile) {
 
 // Rotates 32 dims [k0, k0+32) against their partners [k0+R/2, ...) for one
 // query row: x1 / x2 hold 16 packed bf16 words each; results replace them.
-__device__ __forceinline__ void rotate32(uint32_t (&x1)[16], uint32_t (&x2)[16], int k0, int p,
-                                         const double* inv_freq) {
+// Pair k turns by p * inv_freq_k.  Table form, for a row at p_base + 16 i + j
+// (the rows of a tile are consecutive positions): the turn is the product of
+// two precomputed unit complex numbers, rot_hi[k][i] * rot_lo[k][j].  General
+// form (any other position): the fp64-reduced full angle.
+__device__ __forceinline__ void rotate32_table(uint32_t (&x1)[16], uint32_t (&x2)[16], int k0, int i_hi,
+                                               int j_lo, const float2 (*rot_lo)[16], const float2 (*rot_hi)[8]) {
 #pragma unroll
+  for (int w = 0; w < 16; ++w) {
+    float a[2], bb[2];
+#pragma unroll
+    for (int e = 0; e < 2; ++e) {
+      const int k = k0 + 2 * w + e;
+      const float x = e ? bf16hi(x1[w]) : bf16lo(x1[w]);
+      const float y = e ? bf16hi(x2[w]) : bf16lo(x2[w]);
+      const float2 u = rot_hi[k][i_hi];
+      const float2 v = rot_lo[k][j_lo];
+      const float c = fmaf(u.x, v.x, -u.y * v.y);
+      const float s = fmaf(u.y, v.x, u.x * v.y);
+      a[e] = fmaf(x, c, -y * s);
+      bb[e] = fmaf(y, c, x * s);
+    }
+    x1[w] = pack_bf16(a[0], a[1]);
+    x2[w] = pack_bf16(bb[0], bb[1]);
+  }
+}
+__device__ __noinline__ void rotate32_general(uint32_t (&x1)[16], uint32_t (&x2)[16], int k0, int p,
+                                              const double* inv_freq) {
+#pragma unroll 4
   for (int w = 0; w < 16; ++w) {
     float a[2], bb[2];
 #pragma unroll
@@ -106,21 +142,19 @@ __device__ __forceinline__ void rotate32(uint32_t (&x1)[16], uint32_t (&x2)[16],
     x2[w] = pack_bf16(bb[0], bb[1]);
   }
 }
-
-__device__ __forceinline__ void load_words16(const __nv_bfloat16* src, bool valid, uint32_t (&w)[16]) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    uint4 v = valid ? *reinterpret_cast<const uint4*>(src + 8 * i) : make_uint4(0, 0, 0, 0);
-    w[4 * i + 0] = v.x;
-    w[4 * i + 1] = v.y;
-    w[4 * i + 2] = v.z;
-    w[4 * i + 3] = v.w;
-  }
+// in_table: warp-uniform (every row of the warp at p_base + [0, 128))
+__device__ __forceinline__ void rotate32(uint32_t (&x1)[16], uint32_t (&x2)[16], int k0, int p, int delta,
+                                         bool in_table, const PfSmem& sm) {
+  if (in_table)
+    rotate32_table(x1, x2, k0, delta >> 4, delta & 15, sm.rot_lo, sm.rot_hi);
+  else
+    rotate32_general(x1, x2, k0, p, sm.inv_freq);
 }
 
 template <bool FULL>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
-    prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v, PfArgs a) {
+    prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, PfArgs a) {
   extern __shared__ uint8_t smem_raw[];
   PfSmem& sm = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int R = RopeCfg<FULL>::R;
@@ -145,6 +179,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   const int j_lo = (k_lo - kb) / kBN;
   const int j_hi = (q_hi - kb) / kBN;
   const int n = j_hi - j_lo + 1;
+  // RoPE positions (the tile's first row and this thread's row), loaded early
+  // so their latency hides behind the set-up
+  const int p_base = a.pos ? a.pos[(int64_t)b * a.T + m0] : qb + m0;
+  int p_row = 0;
+  if (warp < 4) {
+    const int row = m0 + (int)threadIdx.x;
+    p_row = a.pos ? (row < a.T ? a.pos[(int64_t)b * a.T + row] : 0) : qb + row;
+  }
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
@@ -159,13 +201,32 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     mbar_init(&sm.o_done, 1);
     mbar_init(&sm.o_final, 1);
     mbar_init(&sm.mma_done, 1);
+    mbar_init(&sm.q_full, 1);
+    mbar_init(&sm.q_free, 4);
     fence_barrier_init();
   }
   if (warp == 5) {
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
   }
+  // rotation tables: pair k = t % (R/2) of entry group t / (R/2); 24 entries per pair
   if (threadIdx.x < R / 2) sm.inv_freq[threadIdx.x] = rope_inv_freq(RopeCfg<FULL>::theta, threadIdx.x, R);
+  __syncthreads();
+  {
+    for (int t = threadIdx.x; t < (R / 2) * 24; t += kPfThreads) {
+      const int k = t % (R / 2);
+      const int e = t / (R / 2);
+      const double f = sm.inv_freq[k];
+      float sn, cs;
+      if (e < 16) {
+        small_angle_sincos(e, (float)f, &sn, &cs);
+        sm.rot_lo[k][e] = make_float2(cs, sn);
+      } else {
+        rope_sincos(p_base + 16 * (e - 16), f, &sn, &cs);
+        sm.rot_hi[k][e - 16] = make_float2(cs, sn);
+      }
+    }
+  }
   tc_fence_before();
   cluster_sync();   // barriers of both CTAs initialised before any cross-CTA arrive
   tc_fence_after();
@@ -174,6 +235,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   if (warp == 4) {
     // ======================= TMA producer (both CTAs) =======================
     if (lane == 0) {
+      // this CTA's query tile first: 4 boxes of 64 dims x 128 rows of head h
+      mbar_arrive_expect_tx(&sm.q_full, 4 * kSlotBytes);
+#pragma unroll
+      for (int box = 0; box < 4; ++box)
+        tma_load_4d(smem_u32(sm.slot[kQSlot + box]), &tm_q, &sm.q_full, box * 64, h, m0, b);
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
       int issued = 0;
@@ -183,6 +249,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         load_of(i, n, is_k, tile);
         const int slot = i % kSlots;
         if (i >= kSlots && !mbar_wait(&sm.empty[slot], ((i / kSlots) - 1) & 1)) break;
+        if (i == kQSlot && !mbar_wait(&sm.q_free, 0)) break;   // the query tile has been read
         if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
         const uint32_t dst = smem_u32(sm.slot[slot]);
         const int row = (j_lo + tile) * kBN;
@@ -244,34 +311,56 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   } else {
     // ======================= softmax / epilogue (warps 0-3) =======================
     const int r = threadIdx.x;          // query row in the tile = TMEM lane
+    bool ok_q = true;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     const int row = m0 + r;
     const bool valid = row < a.T;
     const int qseq = qb + row;
-    const int p = a.pos ? (valid ? a.pos[(int64_t)b * a.T + row] : 0) : qseq;
-    const __nv_bfloat16* qrow = a.q + ((int64_t)b * a.T + (valid ? row : 0)) * a.q_stride + (int64_t)h * kD;
+    const int p = p_row;
+    const int delta = p - p_base;
+    const bool small = __all_sync(0xffffffffu, delta >= 0 && delta < kBM);
 
-    // ---- rotate the query row into TMEM columns [0,128) ----
+    // ---- this row of the query tile: shared memory (128-byte swizzled boxes) -> registers ----
+    uint4 qv[kD / 8];
+    ok_q = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0));
+#pragma unroll
+    for (int i = 0; i < kD / 8; ++i) {
+      const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(i & 7) * 16);
+      qv[i] = *reinterpret_cast<const uint4*>(sm.slot[kQSlot + (i >> 3)] + off);
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&sm.q_free);
+    // ---- rotate it into TMEM columns [0,128) ----
+    auto words16 = [&](int dim0, uint32_t (&w)[16]) {   // 16 packed words = dims [dim0, dim0 + 32)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint4 v = qv[dim0 / 8 + i];
+        w[4 * i + 0] = v.x;
+        w[4 * i + 1] = v.y;
+        w[4 * i + 2] = v.z;
+        w[4 * i + 3] = v.w;
+      }
+    };
     if (FULL) {
       uint32_t x1[16], x2[16];
-      load_words16(qrow, valid, x1);
-      load_words16(qrow + 32, valid, x2);
-      rotate32(x1, x2, 0, p, sm.inv_freq);
+      words16(0, x1);
+      words16(32, x2);
+      rotate32(x1, x2, 0, p, delta, small, sm);
       tmem_st16(trow + kColQ + 0, x1);
       tmem_st16(trow + kColQ + 16, x2);
 #pragma unroll
       for (int c = 0; c < 6; ++c) {  // dims 64..255 unchanged
         uint32_t w[16];
-        load_words16(qrow + 64 + 32 * c, valid, w);
+        words16(64 + 32 * c, w);
         tmem_st16(trow + kColQ + 32 + 16 * c, w);
       }
     } else {
-#pragma unroll 1
+#pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t x1[16], x2[16];
-        load_words16(qrow + 32 * c, valid, x1);
-        load_words16(qrow + 128 + 32 * c, valid, x2);
-        rotate32(x1, x2, 32 * c, p, sm.inv_freq);
+        words16(32 * c, x1);
+        words16(128 + 32 * c, x2);
+        rotate32(x1, x2, 32 * c, p, delta, small, sm);
         tmem_st16(trow + kColQ + 16 * c, x1);
         tmem_st16(trow + kColQ + 64 + 16 * c, x2);
       }
@@ -287,8 +376,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     // ---- online softmax over the key tiles ----
     const float scale_log2 = 0.0625f * 1.4426950408889634f;
     float m_run = -INFINITY, l_run = 0.f;
-    bool ok = true;
-    for (int j = 0; j < n; ++j) {
+    bool ok = ok_q;
+    for (int j = 0; ok && j < n; ++j) {
       const int sb = j & 1;
       ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (j >> 1) & 1));
       if (!ok) break;
@@ -378,26 +467,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         const float gs = __bfloat162float(a.gate[((int64_t)b * a.T + row) * kHq + h]);
         f *= 1.f / (1.f + __expf(-gs));
       }
-      __nv_bfloat16* orow = a.out + (((int64_t)b * a.T + (valid ? row : 0)) * kHq + h) * kD;
+      // O / l * gate -> bf16 -> ring slots 0..3 in the 128-byte swizzled box
+      // layout of the output map; then one thread stores the tile with TMA
+      // (rows past T are clipped by the tensor map).
 #pragma unroll 1
       for (int c8 = 0; c8 < 8; ++c8) {
         uint32_t ov[32];
         tmem_ld32(trow + kColO + 32 * c8, ov);
         tmem_wait_ld();
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + 32 * c8);
+        uint8_t* box = sm.slot[c8 >> 1];
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t w4[4];
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t w4[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 8 * q4 + 2 * e;
-              w4[e] = pack_bf16(__uint_as_float(ov[c]) * f, __uint_as_float(ov[c + 1]) * f);
-            }
-            dst[q4] = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int e = 0; e < 4; ++e) {
+            const int c = 8 * q4 + 2 * e;
+            w4[e] = pack_bf16(__uint_as_float(ov[c]) * f, __uint_as_float(ov[c + 1]) * f);
           }
+          const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(((c8 & 1) * 4 + q4) * 16));
+          *reinterpret_cast<uint4*>(box + off) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
       }
+      fence_proxy_async();
+    }
+    asm volatile("bar.sync 1, 128;" ::: "memory");
+    if (ok && r == 0) {
+#pragma unroll
+      for (int box = 0; box < 4; ++box) tma_store_4d(&tm_o, smem_u32(sm.slot[box]), box * 64, h, m0, b);
+      tma_store_commit_and_wait();
     }
   }
 
@@ -428,9 +525,9 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   const size_t smem = prefill_smem_bytes();
   profile_before(st);
   if (full)
-    prefill_kernel<true><<<(unsigned)grid, kPfThreads, smem, st>>>(h.tm_k, h.tm_v, a);
+    prefill_kernel<true><<<(unsigned)grid, kPfThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_q, h.tm_o, a);
   else
-    prefill_kernel<false><<<(unsigned)grid, kPfThreads, smem, st>>>(h.tm_k, h.tm_v, a);
+    prefill_kernel<false><<<(unsigned)grid, kPfThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_q, h.tm_o, a);
   profile_after(st);
   count_launch();
   return cudaGetLastError();
@@ -439,6 +536,7 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
 // Box rows of the K and V tensor maps this kernel expects (per-CTA halves).
 int prefill_k_box_rows() { return kKBoxRows; }
 int prefill_v_box_rows() { return kBN; }
+int prefill_q_box_rows() { return kBM; }
 
 cudaError_t prefill_set_smem_attr() {
   const int smem = (int)prefill_smem_bytes();
