@@ -163,14 +163,16 @@ def gqa_attention(q, k, v, q_idx, k_idx, window, gate=None, scale=None):
     if scale is None:
         scale = 1.0 / np.sqrt(q.shape[-1])
     mask = dense_mask(q_idx, k_idx, window)                 # [Tq, Tk]
-    s = np.einsum("thd,jhd->htj", q, kr, optimize=True) * scale
+    # scores s[h, t, j] = q[t, h] . k[j, h] as one matrix product per head
+    s = np.matmul(q.transpose(1, 0, 2), kr.transpose(1, 2, 0)) * scale
     s = np.where(mask[None], s, -np.inf)
     m = s.max(axis=-1, keepdims=True)
     m = np.where(np.isfinite(m), m, 0.0)                    # fully masked row -> all zero
     p = np.exp(s - m)
     l = p.sum(axis=-1, keepdims=True)
     p = p / np.where(l > 0, l, 1.0)
-    o = np.einsum("htj,jhd->thd", p, vr, optimize=True)
+    # o[t, h] = sum_j p[h, t, j] v[j, h]
+    o = np.matmul(p, vr.transpose(1, 0, 2)).transpose(1, 0, 2)
     if gate is not None:
         # [TEARDOWN] §"省显存的第二板斧": attn_output * sigmoid(gate_score.float()),
         # one score per head.
