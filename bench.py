@@ -18,6 +18,7 @@ The JSON line also carries:
                 tokens/s;
   prefill_128k  one full layer, 131072 tokens: TFLOP/s and % of peak;
   decode_1m     (--decode-1m) 36-layer decode at 1M tokens: tokens/s;
+  chunked_prefill (--chunked) 262144 tokens in 8192-token chunks, 36 layers;
   cpu_baseline  the fp64 oracle on a bounded sample of the same workload.
 
 `--impl reference` times the oracle as the reference arm instead.
@@ -425,6 +426,48 @@ def bench_decode_1m(hyb, args, peaks):
             "frac_of_hbm": kv / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
 
 
+def bench_chunked(hyb, args, peaks):
+    """262144 tokens in 8192-token chunks through all 36 layers (9 full, 27 sliding), batch 1.
+
+    Each chunk is appended to its layer's cache and attends over the cached
+    context.  The 32 chunk inputs (seed 4 + c) are shared by the layers: the
+    work does not depend on the values.
+    """
+    from full_gqa_attention_partial_b200 import synth
+    total, C = 262144, 8192
+    n_chunks = total // C
+    xs = [synth.prefill_inputs(1, C, seed=4 + c, device="cuda", start=c * C) for c in range(n_chunks)]
+    fulls = [hyb.KVCache(FULL, 1, capacity=total) for _ in range(9)]
+    rings = [hyb.KVCache(SLIDING, 1) for _ in range(27)]
+    ws = hyb.alloc_workspace(hyb.hyb_attn_prefill_workspace_size(SLIDING, 1, C, True))
+    out = torch.empty(1, C, H, D, dtype=torch.bfloat16, device="cuda")
+    work = 9 * flops(total, FULL) + 27 * flops(total, SLIDING)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for c in range(n_chunks):
+        x = xs[c]
+        fi = ri = 0
+        for layer in range(36):
+            if layer % 4 == 3:
+                cache, lt = fulls[fi], FULL
+                fi += 1
+            else:
+                cache, lt = rings[ri], SLIDING
+                ri += 1
+            hyb.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], None, lt, out=out, cache=cache, workspace=ws)
+    ev1.record()
+    torch.cuda.synchronize()
+    assert hyb.hyb_device_error() == 0
+    ms = ev0.elapsed_time(ev1)
+    rate = work / (ms / 1e3) / 1e12
+    return {"workload": "chunked prefill, batch 1, 262144 tokens in 8192-token chunks, 36 layers "
+                        "(9 full, 27 sliding), seed 4", "pflop": work / 1e15, "ms": ms,
+            "tflops": rate, "frac_of_peak": rate / peaks["bf16_tflops_sustained"],
+            "peak_source": f"{peaks['source']} bf16 sustained (seconds-long run)",
+            "prefill_tokens_per_s": total / (ms / 1e3)}
+
+
 # ---------------------------------------------------------------------------
 # the oracle on the host: cpu_baseline and the reference arm
 # ---------------------------------------------------------------------------
@@ -557,6 +600,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--decode-1m", action="store_true", help="also run the 36-layer 1M-token decode workload")
+    ap.add_argument("--chunked", action="store_true",
+                    help="also run the 262144-token chunked prefill through 36 layers")
     ap.add_argument("--no-extras", action="store_true", help="only the headline step (no sub-benchmarks)")
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows per layer for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="oracle rows per layer per reference step")
@@ -593,6 +638,8 @@ def main():
         extras["decode"] = bench_decode(hyb, args, peaks)
         if args.decode_1m:
             extras["decode_1m"] = bench_decode_1m(hyb, args, peaks)
+        if args.chunked:
+            extras["chunked_prefill"] = bench_chunked(hyb, args, peaks)
     clk = clocks.stop()
     line = {
         "metric": METRIC, "value": main_res["value"], "unit": "TFLOP/s", "n_gpus": dist.world,
