@@ -71,6 +71,13 @@ bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) ==
 // memory opt-in of the two large kernels.
 std::mutex g_mu;
 int g_dev_state[128];  // 0 unknown, 1 ready, -1 unsupported
+int g_dev_sms[128];    // multiprocessor count
+
+int device_sms() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 128 || g_dev_sms[dev] <= 0) return 148;
+  return g_dev_sms[dev];
+}
 
 hyb_status ensure_device() {
   int dev = 0;
@@ -89,6 +96,7 @@ hyb_status ensure_device() {
                 dev, major, minor);
   }
   if ((e = prefill_set_smem_attr()) != cudaSuccess) return cuda_fail(e, "prefill smem attribute");
+  cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev);
   if ((e = decode_set_smem_attr()) != cudaSuccess) return cuda_fail(e, "decode smem attribute");
   g_dev_state[dev] = 1;
   return HYB_OK;
@@ -327,6 +335,10 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
   ph.out = out;
   ph.B = B;
   ph.T = T;
+  // sliding layers: many short, equal work items -> persistent CTA pairs (one
+  // per two SMs); full layers: long items of unequal length -> one item per
+  // pair, handed out longest first by the hardware block scheduler.
+  ph.n_pairs = full ? (1 << 29) : device_sms() / 2;
   cudaError_t e;
 
   RopeStoreHost r;  // new tokens, token-major input rows

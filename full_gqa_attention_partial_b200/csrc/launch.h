@@ -51,6 +51,7 @@ struct PrefillHost {
   const int32_t* qbase = nullptr;  // [B] sequence index of token 0, or null (0)
   int ctx_mode = 0;            // 1: key row j holds sequence index qbase - 511 + j
   int B = 0, T = 0;
+  int n_pairs = 74;            // persistent CTA pairs (SMs / 2)
 };
 cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st);
 int prefill_k_box_rows();   // rows (keys) per TMA box of the K map

@@ -39,7 +39,7 @@ namespace hyb {
 
 constexpr int kBM = 128;                  // query rows per CTA
 constexpr int kBN = 64;                   // keys per tile (shared by the pair)
-constexpr int kSlots = 12;
+constexpr int kSlots = 8;                 // K/V ring
 constexpr int kSlotBytes = 16384;         // one CTA's half of a K or V tile
 constexpr int kKBoxRows = kBN / 2;        // K half: 32 keys x 64 dims per box
 constexpr int kKBox = kKBoxRows * 128;    // 4 KB
@@ -47,11 +47,12 @@ constexpr int kVBox = kBN * 128;          // V half: 64 keys x 64 dims per box, 
 constexpr int kPfThreads = 192;
 constexpr uint32_t kColQ = 0;
 constexpr uint32_t kColO = 256;
-constexpr float kRescaleThreshold = 8.0f;
+constexpr float kRescaleThreshold = 8.0f;             // 1 of every 4 exponentials on the FMA pipe
 __device__ __forceinline__ uint32_t col_s(int sb) { return sb ? 192u : 128u; }
 
 struct PfSmem {
   uint8_t slot[kSlots][kSlotBytes];  // 1024-byte aligned
+  uint8_t qo[4][kSlotBytes];         // the query tile in (4 boxes of 64 dims x 128 rows), the output tile out
   double inv_freq[128];
   // rotation tables for the tile's rows (positions p_base + 16 i + j):
   //   rot_lo[k][j] = (cos, sin)(j * inv_freq_k),               j < 16
@@ -66,14 +67,10 @@ struct PfSmem {
   uint64_t o_done;         // each P.V completed
   uint64_t o_final;        // the last P.V completed
   uint64_t mma_done;       // every MMA of the pair completed
-  uint64_t q_full;         // this CTA's query tile landed (ring slots 8..11)
-  uint64_t q_free;         // the softmax warps have read it
+  uint64_t q_full;         // this CTA's query tile landed in qo
+  uint64_t q_free;         // qo is free again (the previous output tile has left)
   uint32_t tmem_base;
 };
-// The query tile (4 boxes of 64 dims x 128 rows = 64 KB) arrives in ring slots
-// 8..11 before the K/V stream first reaches them; the output tile leaves
-// through slots 0..3 once every MMA is done.
-constexpr int kQSlot = 8;
 
 size_t prefill_smem_bytes() { return sizeof(PfSmem) + 1024; }
 
@@ -151,6 +148,50 @@ __device__ __forceinline__ void rotate32(uint32_t (&x1)[16], uint32_t (&x2)[16],
     rotate32_general(x1, x2, k0, p, sm.inv_freq);
 }
 
+// One work item: a 128-query tile of the two query heads (2 hp + {0, 1}) of KV
+// head hp / 2 in sequence b; items are numbered longest first (the query
+// tiles of the end of the sequence first), the 8 head pairs of a tile adjacent.
+struct Item {
+  int b, kvh, h_pair0, m0, qb, kb, q_lo, q_hi, j_lo, n;
+};
+template <bool FULL>
+__device__ __forceinline__ Item item_of(int w, const PfArgs& a) {
+  Item it;
+  const int per_tile = a.B * (kHq / 2);
+  const int mt = a.n_mtiles - 1 - w / per_tile;
+  const int rem = w % per_tile;
+  const int hp = rem % (kHq / 2);
+  it.b = rem / (kHq / 2);
+  it.kvh = hp >> 1;
+  it.h_pair0 = it.kvh * kGroup + (hp & 1) * 2;
+  it.m0 = mt * kBM;
+  it.qb = a.qbase ? a.qbase[it.b] : 0;             // sequence index of token 0
+  it.kb = a.ctx_mode ? it.qb - (kWindow - 1) : 0;  // sequence index of key row 0
+  const int rows_valid = min(kBM, a.T - it.m0);
+  it.q_lo = it.qb + it.m0;
+  it.q_hi = it.qb + it.m0 + rows_valid - 1;
+  const int k_lo = FULL ? 0 : max(0, it.q_lo - (kWindow - 1));
+  it.j_lo = (k_lo - it.kb) / kBN;
+  it.n = (it.q_hi - it.kb) / kBN - it.j_lo + 1;
+  return it;
+}
+
+// Item of CTA pair `pair` in round k: the items of a round are the next
+// n_pairs of the longest-first order, dealt out in alternating direction
+// (pair p gets the p-th of round k when k is even, the p-th from the end
+// when k is odd), which evens out the pairs' total work.  -1: none (this pair
+// sits out the last, partial round); -2: past the last round.
+__device__ __forceinline__ int item_index(int k, int pair, int n_pairs, int n_items) {
+  const int base = k * n_pairs;
+  if (base >= n_items) return -2;
+  const int w = base + ((k & 1) ? n_pairs - 1 - pair : pair);
+  return w < n_items ? w : -1;
+}
+
+// Persistent: each CTA pair walks its items round by round.
+// Barrier phases run on across items: K/V loads by a global load counter,
+// S / P buffers by a global tile counter, query / output / last-P.V barriers
+// by the item counter.
 template <bool FULL>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
@@ -160,33 +201,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   constexpr int R = RopeCfg<FULL>::R;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();   // 0 = the CTA that issues the pair's MMAs
-
-  // ---- work item: longest query tiles first; the pairs of one tile adjacent ----
-  const int pair = blockIdx.x >> 1;
-  const int per_tile = a.B * (kHq / 2);
-  const int mt = a.n_mtiles - 1 - pair / per_tile;
-  const int rem = pair % per_tile;
-  const int hp = rem % (kHq / 2);
-  const int b = rem / (kHq / 2);
-  const int kvh = hp >> 1;
-  const int h = kvh * kGroup + (hp & 1) * 2 + (int)rank;
-  const int m0 = mt * kBM;
-  const int qb = a.qbase ? a.qbase[b] : 0;             // sequence index of token 0
-  const int kb = a.ctx_mode ? qb - (kWindow - 1) : 0;  // sequence index of key row 0
-  const int rows_valid = min(kBM, a.T - m0);
-  const int q_lo = qb + m0, q_hi = qb + m0 + rows_valid - 1;
-  const int k_lo = FULL ? 0 : max(0, q_lo - (kWindow - 1));
-  const int j_lo = (k_lo - kb) / kBN;
-  const int j_hi = (q_hi - kb) / kBN;
-  const int n = j_hi - j_lo + 1;
-  // RoPE positions (the tile's first row and this thread's row), loaded early
-  // so their latency hides behind the set-up
-  const int p_base = a.pos ? a.pos[(int64_t)b * a.T + m0] : qb + m0;
-  int p_row = 0;
-  if (warp < 4) {
-    const int row = m0 + (int)threadIdx.x;
-    p_row = a.pos ? (row < a.T ? a.pos[(int64_t)b * a.T + row] : 0) : qb + row;
-  }
+  const int pair0 = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int n_items = a.n_mtiles * a.B * (kHq / 2);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kSlots; ++s) {
@@ -202,30 +219,21 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     mbar_init(&sm.o_final, 1);
     mbar_init(&sm.mma_done, 1);
     mbar_init(&sm.q_full, 1);
-    mbar_init(&sm.q_free, 4);
+    mbar_init(&sm.q_free, 1);
     fence_barrier_init();
   }
   if (warp == 5) {
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
   }
-  // rotation tables: pair k = t % (R/2) of entry group t / (R/2); 24 entries per pair
+  // frequencies and the position-independent rotation table
   if (threadIdx.x < R / 2) sm.inv_freq[threadIdx.x] = rope_inv_freq(RopeCfg<FULL>::theta, threadIdx.x, R);
   __syncthreads();
-  {
-    for (int t = threadIdx.x; t < (R / 2) * 24; t += kPfThreads) {
-      const int k = t % (R / 2);
-      const int e = t / (R / 2);
-      const double f = sm.inv_freq[k];
-      float sn, cs;
-      if (e < 16) {
-        small_angle_sincos(e, (float)f, &sn, &cs);
-        sm.rot_lo[k][e] = make_float2(cs, sn);
-      } else {
-        rope_sincos(p_base + 16 * (e - 16), f, &sn, &cs);
-        sm.rot_hi[k][e - 16] = make_float2(cs, sn);
-      }
-    }
+  for (int t = threadIdx.x; t < (R / 2) * 16; t += kPfThreads) {
+    const int k = t % (R / 2), e = t / (R / 2);
+    float sn, cs;
+    small_angle_sincos(e, (float)sm.inv_freq[k], &sn, &cs);
+    sm.rot_lo[k][e] = make_float2(cs, sn);
   }
   tc_fence_before();
   cluster_sync();   // barriers of both CTAs initialised before any cross-CTA arrive
@@ -233,76 +241,108 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   const uint32_t tmem = sm.tmem_base;
 
   if (warp == 4) {
-    // ======================= TMA producer (both CTAs) =======================
     if (lane == 0) {
-      // this CTA's query tile first: 4 boxes of 64 dims x 128 rows of head h
-      mbar_arrive_expect_tx(&sm.q_full, 4 * kSlotBytes);
-#pragma unroll
-      for (int box = 0; box < 4; ++box)
-        tma_load_4d(smem_u32(sm.slot[kQSlot + box]), &tm_q, &sm.q_full, box * 64, h, m0, b);
+      // ======================= K/V producer (both CTAs) =======================
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      int issued = 0;
-      for (int i = 0; i < 2 * n; ++i) {
-        bool is_k;
-        int tile;
-        load_of(i, n, is_k, tile);
-        const int slot = i % kSlots;
-        if (i >= kSlots && !mbar_wait(&sm.empty[slot], ((i / kSlots) - 1) & 1)) break;
-        if (i == kQSlot && !mbar_wait(&sm.q_free, 0)) break;   // the query tile has been read
-        if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
-        const uint32_t dst = smem_u32(sm.slot[slot]);
-        const int row = (j_lo + tile) * kBN;
-        if (is_k) {
+      uint32_t g = 0;   // loads issued so far by this CTA
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int w = item_index(k, pair0, n_pairs, n_items);
+        if (w == -2) break;
+        if (w < 0) continue;
+        const Item it = item_of<FULL>(w, a);
+        for (int i = 0; i < 2 * it.n; ++i, ++g) {
+          bool is_k;
+          int tile;
+          load_of(i, it.n, is_k, tile);
+          const int slot = g % kSlots;
+          if (g >= kSlots && !(ok = mbar_wait(&sm.empty[slot], ((g / kSlots) - 1) & 1))) break;
+          if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
+          const uint32_t dst = smem_u32(sm.slot[slot]);
+          const int row = (it.j_lo + tile) * kBN;
+          if (is_k) {
 #pragma unroll
-          for (int box = 0; box < 4; ++box)
-            tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row + kKBoxRows * (int)rank, kvh, b);
-        } else {
+            for (int box = 0; box < 4; ++box)
+              tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row + kKBoxRows * (int)rank,
+                               it.kvh, it.b);
+          } else {
 #pragma unroll
-          for (int box = 0; box < 2; ++box)
-            tma_load_4d_pair(dst + box * kVBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * box, row, kvh, b);
+            for (int box = 0; box < 2; ++box)
+              tma_load_4d_pair(dst + box * kVBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * box, row, it.kvh,
+                               it.b);
+          }
         }
-        issued = i + 1;
       }
       if (rank == 0)  // every load of the pair completes on CTA 0's barriers
-        for (int i = max(0, issued - kSlots); i < issued; ++i) mbar_wait(&sm.full[i % kSlots], (i / kSlots) & 1);
+        for (uint32_t i = (g > kSlots ? g - kSlots : 0); i < g; ++i) mbar_wait(&sm.full[i % kSlots], (i / kSlots) & 1);
+    } else if (lane == 1) {
+      // ======================= query-tile producer (both CTAs) =======================
+      prefetch_tmap(&tm_q);
+      int item = 0;
+      for (int k = 0;; ++k) {
+        const int w = item_index(k, pair0, n_pairs, n_items);
+        if (w == -2) break;
+        if (w < 0) continue;
+        const Item it = item_of<FULL>(w, a);
+        if (item > 0 && !mbar_wait(&sm.q_free, (item - 1) & 1)) break;
+        mbar_arrive_expect_tx(&sm.q_full, 4 * kSlotBytes);
+#pragma unroll
+        for (int box = 0; box < 4; ++box)
+          tma_load_4d(smem_u32(sm.qo[box]), &tm_q, &sm.q_full, box * 64, it.h_pair0 + (int)rank, it.m0, it.b);
+        ++item;
+      }
+      if (item > 0) mbar_wait(&sm.q_full, (item - 1) & 1);   // no copy left landing at exit
     }
   } else if (warp == 5) {
     // ======================= MMA issuer (CTA 0, whole warp, one lane issues) =======================
     if (rank == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(2 * kBM, kBN, false);   // S = Q K^T, B K-major
       constexpr uint32_t idesc_o = idesc_bf16(2 * kBM, kD, true);     // O += P V, B MN-major
-      bool ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_ready, 0));
-      tc_fence_after();
-      for (int i = 0; ok && i < 2 * n; ++i) {
-        bool is_k;
-        int tile;
-        load_of(i, n, is_k, tile);
-        const int slot = i % kSlots;
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (i / kSlots) & 1)))) break;
+      uint32_t g = 0, J = 0;
+      int item = 0;
+      bool ok = true;
+      for (int k = 0; ok; ++k) {
+        const int w = item_index(k, pair0, n_pairs, n_items);
+        if (w == -2) break;
+        if (w < 0) continue;
+        const Item it = item_of<FULL>(w, a);
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_ready, item & 1)))) break;
         tc_fence_after();
-        const uint32_t saddr = smem_u32(sm.slot[slot]);
-        const int sb = tile & 1;
-        if (is_k) {
-#pragma unroll
-          for (int s = 0; s < kD / 16; ++s) {
-            const uint64_t bdesc = smem_desc_sw128(saddr + (s >> 2) * kKBox + (s & 3) * 32, 16, 1024);
-            mma_ts_pair_warp(tmem + col_s(sb), tmem + kColQ + 8 * s, bdesc, idesc_s, s > 0 ? 1u : 0u);
-          }
-          mma_commit_pair_warp(&sm.empty[slot]);
-          mma_commit_pair_warp(&sm.s_full[sb]);
-        } else {
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[sb], (tile >> 1) & 1)))) break;
+        for (int i = 0; i < 2 * it.n; ++i, ++g) {
+          bool is_k;
+          int tile;
+          load_of(i, it.n, is_k, tile);
+          const int slot = g % kSlots;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (g / kSlots) & 1)))) break;
           tc_fence_after();
+          const uint32_t saddr = smem_u32(sm.slot[slot]);
+          const uint32_t jt = J + tile;   // global tile index
+          const int sb = jt & 1;
+          if (is_k) {
 #pragma unroll
-          for (int s = 0; s < kBN / 16; ++s) {
-            const uint64_t bdesc = smem_desc_sw128(saddr + s * 16 * 128, kVBox, 1024);
-            mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 8 * s, bdesc, idesc_o, (tile > 0 || s > 0) ? 1u : 0u);
+            for (int s = 0; s < kD / 16; ++s) {
+              const uint64_t bdesc = smem_desc_sw128(saddr + (s >> 2) * kKBox + (s & 3) * 32, 16, 1024);
+              mma_ts_pair_warp(tmem + col_s(sb), tmem + kColQ + 8 * s, bdesc, idesc_s, s > 0 ? 1u : 0u);
+            }
+            mma_commit_pair_warp(&sm.empty[slot]);
+            mma_commit_pair_warp(&sm.s_full[sb]);
+          } else {
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[sb], (jt >> 1) & 1)))) break;
+            tc_fence_after();
+#pragma unroll
+            for (int s = 0; s < kBN / 16; ++s) {
+              const uint64_t bdesc = smem_desc_sw128(saddr + s * 16 * 128, kVBox, 1024);
+              mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 8 * s, bdesc, idesc_o,
+                               (tile > 0 || s > 0) ? 1u : 0u);
+            }
+            mma_commit_pair_warp(&sm.empty[slot]);
+            mma_commit_pair_warp(&sm.o_done);
+            if (tile == it.n - 1) mma_commit_pair_warp(&sm.o_final);
           }
-          mma_commit_pair_warp(&sm.empty[slot]);
-          mma_commit_pair_warp(&sm.o_done);
-          if (tile == n - 1) mma_commit_pair_warp(&sm.o_final);
         }
+        J += it.n;
+        ++item;
       }
       // also on an early exit: wait until nothing the pair issued is in flight
       mma_commit_pair_warp(&sm.mma_done);
@@ -311,190 +351,208 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   } else {
     // ======================= softmax / epilogue (warps 0-3) =======================
     const int r = threadIdx.x;          // query row in the tile = TMEM lane
-    bool ok_q = true;
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
-    const int row = m0 + r;
-    const bool valid = row < a.T;
-    const int qseq = qb + row;
-    const int p = p_row;
-    const int delta = p - p_base;
-    const bool small = __all_sync(0xffffffffu, delta >= 0 && delta < kBM);
-
-    // ---- this row of the query tile: shared memory (128-byte swizzled boxes) -> registers ----
-    uint4 qv[kD / 8];
-    ok_q = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, 0));
-#pragma unroll
-    for (int i = 0; i < kD / 8; ++i) {
-      const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(i & 7) * 16);
-      qv[i] = *reinterpret_cast<const uint4*>(sm.slot[kQSlot + (i >> 3)] + off);
-    }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.q_free);
-    // ---- rotate it into TMEM columns [0,128) ----
-    auto words16 = [&](int dim0, uint32_t (&w)[16]) {   // 16 packed words = dims [dim0, dim0 + 32)
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const uint4 v = qv[dim0 / 8 + i];
-        w[4 * i + 0] = v.x;
-        w[4 * i + 1] = v.y;
-        w[4 * i + 2] = v.z;
-        w[4 * i + 3] = v.w;
-      }
-    };
-    if (FULL) {
-      uint32_t x1[16], x2[16];
-      words16(0, x1);
-      words16(32, x2);
-      rotate32(x1, x2, 0, p, delta, small, sm);
-      tmem_st16(trow + kColQ + 0, x1);
-      tmem_st16(trow + kColQ + 16, x2);
-#pragma unroll
-      for (int c = 0; c < 6; ++c) {  // dims 64..255 unchanged
-        uint32_t w[16];
-        words16(64 + 32 * c, w);
-        tmem_st16(trow + kColQ + 32 + 16 * c, w);
-      }
-    } else {
-#pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint32_t x1[16], x2[16];
-        words16(32 * c, x1);
-        words16(128 + 32 * c, x2);
-        rotate32(x1, x2, 32 * c, p, delta, small, sm);
-        tmem_st16(trow + kColQ + 16 * c, x1);
-        tmem_st16(trow + kColQ + 64 + 16 * c, x2);
-      }
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncwarp();
-    if (lane == 0) {
-      if (rank == 0) mbar_arrive(&sm.q_ready);
-      else mbar_arrive_remote(&sm.q_ready, 0);
-    }
-
-    // ---- online softmax over the key tiles ----
     const float scale_log2 = 0.0625f * 1.4426950408889634f;
-    float m_run = -INFINITY, l_run = 0.f;
-    bool ok = ok_q;
-    for (int j = 0; ok && j < n; ++j) {
-      const int sb = j & 1;
-      ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (j >> 1) & 1));
-      if (!ok) break;
-      tc_fence_after();
-      uint32_t sraw[64];
-      {
-        uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]);
-        uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]);
-        tmem_ld32(trow + col_s(sb), lo);
-        tmem_ld32(trow + col_s(sb) + 32, hi);
-      }
-      tmem_wait_ld();
-      float s[64];
-#pragma unroll
-      for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sraw[c]);
+    uint32_t J = 0;
+    int item = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int w = item_index(k, pair0, n_pairs, n_items);
+      if (w == -2) break;
+      if (w < 0) continue;
+      const Item it = item_of<FULL>(w, a);
+      const int h = it.h_pair0 + (int)rank;
+      const int row = it.m0 + r;
+      const bool valid = row < a.T;
+      const int qseq = it.qb + row;
+      const int p_base = a.pos ? a.pos[(int64_t)it.b * a.T + it.m0] : it.qb + it.m0;
+      const int p = a.pos ? (valid ? a.pos[(int64_t)it.b * a.T + row] : 0) : qseq;
+      const int delta = p - p_base;
+      const bool in_table = __all_sync(0xffffffffu, delta >= 0 && delta < kBM);
 
-      const int ks0 = kb + (j_lo + j) * kBN;   // sequence index of the tile's first key
-      const bool whole = ks0 >= 0 && ks0 + kBN - 1 <= q_lo && (FULL || q_hi - ks0 <= kWindow - 1);
-      if (!whole) {
+      // ---- rotation table for this tile's base position ----
+      for (int t = r; t < (R / 2) * 8; t += kBM) {
+        const int k = t % (R / 2), e = t / (R / 2);
+        float sn, cs;
+        rope_sincos(p_base + 16 * e, sm.inv_freq[k], &sn, &cs);
+        sm.rot_hi[k][e] = make_float2(cs, sn);
+      }
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+
+      // ---- this row of the query tile: shared memory (128-byte swizzled boxes) -> registers ----
+      uint4 qv[kD / 8];
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, item & 1)))) break;
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const int ks = ks0 + c;
-          const bool vis = ks >= 0 && ks <= qseq && (FULL || qseq - ks <= kWindow - 1);
-          if (!vis) s[c] = -INFINITY;
+      for (int i = 0; i < kD / 8; ++i) {
+        const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(i & 7) * 16);
+        qv[i] = *reinterpret_cast<const uint4*>(sm.qo[i >> 3] + off);
+      }
+      // ---- rotate it into TMEM columns [0,128) ----
+      auto words16 = [&](int dim0, uint32_t (&wd)[16]) {   // 16 packed words = dims [dim0, dim0 + 32)
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const uint4 v = qv[dim0 / 8 + i];
+          wd[4 * i + 0] = v.x;
+          wd[4 * i + 1] = v.y;
+          wd[4 * i + 2] = v.z;
+          wd[4 * i + 3] = v.w;
+        }
+      };
+      if (FULL) {
+        uint32_t x1[16], x2[16];
+        words16(0, x1);
+        words16(32, x2);
+        rotate32(x1, x2, 0, p, delta, in_table, sm);
+        tmem_st16(trow + kColQ + 0, x1);
+        tmem_st16(trow + kColQ + 16, x2);
+#pragma unroll
+        for (int c = 0; c < 6; ++c) {  // dims 64..255 unchanged
+          uint32_t wd[16];
+          words16(64 + 32 * c, wd);
+          tmem_st16(trow + kColQ + 32 + 16 * c, wd);
+        }
+      } else {
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          uint32_t x1[16], x2[16];
+          words16(32 * c, x1);
+          words16(128 + 32 * c, x2);
+          rotate32(x1, x2, 32 * c, p, delta, in_table, sm);
+          tmem_st16(trow + kColQ + 16 * c, x1);
+          tmem_st16(trow + kColQ + 64 + 16 * c, x2);
         }
       }
-      // row maximum: pairwise tree (short dependency chains)
-      float mx[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) mx[c] = fmaxf(s[c], s[c + 32]);
-#pragma unroll
-      for (int w = 16; w >= 1; w >>= 1)
-#pragma unroll
-        for (int c = 0; c < w; ++c) mx[c] = fmaxf(mx[c], mx[c + w]);
-      const float m_tile = mx[0] * scale_log2;
-      const float m_new = fmaxf(m_run, m_tile);
-      const bool rescale = m_new > m_run + kRescaleThreshold;
-      const float m_use = rescale ? m_new : m_run;
-      const float base = (m_use == -INFINITY) ? 0.f : m_use;
-      const float alpha = rescale ? ex2(m_run - m_use) : 1.f;
-      uint32_t pw[32];
-      float ps[8];
-#pragma unroll
-      for (int c = 0; c < 8; ++c) ps[c] = 0.f;
-#pragma unroll
-      for (int w = 0; w < 32; ++w) {
-        const float p0 = ex2(fmaf(s[2 * w], scale_log2, -base));
-        const float p1 = ex2(fmaf(s[2 * w + 1], scale_log2, -base));
-        ps[w & 7] += p0 + p1;
-        pw[w] = pack_bf16(p0, p1);
-      }
-      const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      l_run = l_run * alpha + sum;
-      m_run = m_use;
-      tmem_st32(trow + col_s(sb), pw);
       tmem_wait_st();
-      if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-        // O may only be touched once the previous tile's P.V has landed
-        ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done, (j - 1) & 1));
-        if (!ok) break;
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(&sm.q_ready);
+        else mbar_arrive_remote(&sm.q_ready, 0);
+      }
+
+      // ---- online softmax over the key tiles ----
+      float m_run = -INFINITY, l_run = 0.f;
+      for (int j = 0; ok && j < it.n; ++j) {
+        const uint32_t jt = J + j;
+        const int sb = jt & 1;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (jt >> 1) & 1)))) break;
         tc_fence_after();
+        uint32_t sraw[64];
+        {
+          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]);
+          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]);
+          tmem_ld32(trow + col_s(sb), lo);
+          tmem_ld32(trow + col_s(sb) + 32, hi);
+        }
+        tmem_wait_ld();
+        float s[64];
+#pragma unroll
+        for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sraw[c]);
+
+        const int ks0 = it.kb + (it.j_lo + j) * kBN;   // sequence index of the tile's first key
+        const bool whole = ks0 >= 0 && ks0 + kBN - 1 <= it.q_lo && (FULL || it.q_hi - ks0 <= kWindow - 1);
+        if (!whole) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c) {
+            const int ks = ks0 + c;
+            const bool vis = ks >= 0 && ks <= qseq && (FULL || qseq - ks <= kWindow - 1);
+            if (!vis) s[c] = -INFINITY;
+          }
+        }
+        // row maximum: pairwise tree (short dependency chains)
+        float mx[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) mx[c] = fmaxf(s[c], s[c + 32]);
+#pragma unroll
+        for (int wd = 16; wd >= 1; wd >>= 1)
+#pragma unroll
+          for (int c = 0; c < wd; ++c) mx[c] = fmaxf(mx[c], mx[c + wd]);
+        const float m_tile = mx[0] * scale_log2;
+        const float m_new = fmaxf(m_run, m_tile);
+        const bool rescale = m_new > m_run + kRescaleThreshold;
+        const float m_use = rescale ? m_new : m_run;
+        const float base = (m_use == -INFINITY) ? 0.f : m_use;
+        const float alpha = rescale ? ex2(m_run - m_use) : 1.f;
+        uint32_t pw[32];
+        float ps[8];
+#pragma unroll
+        for (int c = 0; c < 8; ++c) ps[c] = 0.f;
+#pragma unroll
+        for (int wd = 0; wd < 32; ++wd) {
+          const float p0 = ex2(fmaf(s[2 * wd], scale_log2, -base));
+          const float p1 = ex2(fmaf(s[2 * wd + 1], scale_log2, -base));
+          ps[wd & 7] += p0 + p1;
+          pw[wd] = pack_bf16(p0, p1);
+        }
+        const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
+        l_run = l_run * alpha + sum;
+        m_run = m_use;
+        tmem_st32(trow + col_s(sb), pw);
+        tmem_wait_st();
+        if (j > 0 && __any_sync(0xffffffffu, rescale)) {
+          // O may only be touched once the previous tile's P.V has landed
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done, (jt - 1) & 1)))) break;
+          tc_fence_after();
+#pragma unroll 1
+          for (int c8 = 0; c8 < 8; ++c8) {
+            uint32_t ov[32];
+            tmem_ld32(trow + kColO + 32 * c8, ov);
+            tmem_wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
+            tmem_st32(trow + kColO + 32 * c8, ov);
+          }
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(&sm.p_full[sb]);
+          else mbar_arrive_remote(&sm.p_full[sb], 0);
+        }
+      }
+      J += it.n;
+
+      // ---- epilogue: O / l * sigmoid(gate) -> bf16 -> qo -> TMA store ----
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, item & 1));
+      if (ok) {
+        tc_fence_after();
+        float f = l_run > 0.f ? 1.f / l_run : 0.f;
+        if (a.gate != nullptr && valid) {
+          const float gs = __bfloat162float(a.gate[((int64_t)it.b * a.T + row) * kHq + h]);
+          f *= 1.f / (1.f + __expf(-gs));
+        }
 #pragma unroll 1
         for (int c8 = 0; c8 < 8; ++c8) {
           uint32_t ov[32];
           tmem_ld32(trow + kColO + 32 * c8, ov);
           tmem_wait_ld();
+          uint8_t* box = sm.qo[c8 >> 1];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-          tmem_st32(trow + kColO + 32 * c8, ov);
-        }
-        tmem_wait_st();
-      }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (rank == 0) mbar_arrive(&sm.p_full[sb]);
-        else mbar_arrive_remote(&sm.p_full[sb], 0);
-      }
-    }
-
-    // ---- epilogue: O / l * sigmoid(gate) -> bf16 ----
-    if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, 0));
-    if (ok) {
-      tc_fence_after();
-      float f = l_run > 0.f ? 1.f / l_run : 0.f;
-      if (a.gate != nullptr && valid) {
-        const float gs = __bfloat162float(a.gate[((int64_t)b * a.T + row) * kHq + h]);
-        f *= 1.f / (1.f + __expf(-gs));
-      }
-      // O / l * gate -> bf16 -> ring slots 0..3 in the 128-byte swizzled box
-      // layout of the output map; then one thread stores the tile with TMA
-      // (rows past T are clipped by the tensor map).
-#pragma unroll 1
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint32_t ov[32];
-        tmem_ld32(trow + kColO + 32 * c8, ov);
-        tmem_wait_ld();
-        uint8_t* box = sm.slot[c8 >> 1];
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint32_t w4[4];
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int c = 8 * q4 + 2 * e;
-            w4[e] = pack_bf16(__uint_as_float(ov[c]) * f, __uint_as_float(ov[c + 1]) * f);
+            for (int e = 0; e < 4; ++e) {
+              const int c = 8 * q4 + 2 * e;
+              w4[e] = pack_bf16(__uint_as_float(ov[c]) * f, __uint_as_float(ov[c + 1]) * f);
+            }
+            const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(((c8 & 1) * 4 + q4) * 16));
+            *reinterpret_cast<uint4*>(box + off) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
-          const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(((c8 & 1) * 4 + q4) * 16));
-          *reinterpret_cast<uint4*>(box + off) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
+        fence_proxy_async();
       }
-      fence_proxy_async();
-    }
-    asm volatile("bar.sync 1, 128;" ::: "memory");
-    if (ok && r == 0) {
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (r == 0) {
+        if (ok) {
 #pragma unroll
-      for (int box = 0; box < 4; ++box) tma_store_4d(&tm_o, smem_u32(sm.slot[box]), box * 64, h, m0, b);
-      tma_store_commit_and_wait();
+          for (int box = 0; box < 4; ++box) tma_store_4d(&tm_o, smem_u32(sm.qo[box]), box * 64, h, it.m0, it.b);
+          tma_store_commit_and_wait();
+        }
+        mbar_arrive(&sm.q_free);   // the next query tile may land in qo
+      }
+      ok = __all_sync(0xffffffffu, ok);
+      ++item;
     }
   }
 
@@ -520,8 +578,9 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   a.B = h.B;
   a.T = h.T;
   a.n_mtiles = (h.T + kBM - 1) / kBM;
-  const long long grid = (long long)a.n_mtiles * h.B * kHq;   // one CTA per (tile, head), in pairs
-  if (grid <= 0 || grid > 0x7fffffffLL) return cudaErrorInvalidValue;
+  const long long n_items = (long long)a.n_mtiles * h.B * (kHq / 2);   // (query tile, head pair)
+  if (n_items <= 0 || n_items > 0x3fffffffLL) return cudaErrorInvalidValue;
+  const long long grid = 2 * (n_items < h.n_pairs ? n_items : h.n_pairs);   // persistent CTA pairs
   const size_t smem = prefill_smem_bytes();
   profile_before(st);
   if (full)
