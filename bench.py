@@ -64,6 +64,32 @@ def layer_seed(base: int, i: int) -> int:
     return base + 7919 * i
 
 
+# DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
+# capture of the kernel as it was when its sources hashed to `sha` (profiles/ has
+# the capture's summary).  Reported as roofline.traffic only while the sources are
+# unchanged; otherwise null.
+TRAFFIC = {
+    "prefill_full_T32768": {"bytes": 2.225e9, "sha": "52c4bcaa723ed33b",
+                            "sources": ["prefill.cu", "common.cuh"],
+                            "capture": "profiles/prefill_kernel_full_T32768.md"},
+}
+
+
+def kernel_sources_sha(files) -> str:
+    import hashlib
+    d = hashlib.sha256()
+    for f in files:
+        d.update(open(os.path.join(ROOT, "full_gqa_attention_partial_b200", "csrc", f), "rb").read())
+    return d.hexdigest()[:16]
+
+
+def traffic_of(name: str):
+    t = TRAFFIC.get(name)
+    if t is None or kernel_sources_sha(t["sources"]) != t["sha"]:
+        return None
+    return t["bytes"]
+
+
 # ---------------------------------------------------------------------------
 # plumbing: ranks, peaks, clocks
 # ---------------------------------------------------------------------------
@@ -236,7 +262,7 @@ def bench_main(hyb, args, dist: Dist, peaks):
             "peak_source": f"{peaks['source']} bf16 {peak_kind}",
             "algorithmic_flops_per_launch": flops(T_MAIN, FULL),
             "avg_launch_ms": full_ms, "launches": len(per_layer[3]),
-            "traffic": args.full_traffic,
+            "traffic": traffic_of("prefill_full_T32768"),
             "sliding_kernel": {"avg_launch_ms": slide_ms,
                                "achieved": flops(T_MAIN, SLIDING) / (slide_ms / 1e3) / 1e12},
             "attention_kernels_share_of_step": kernel_share,
@@ -378,7 +404,7 @@ def bench_decode(hyb, args, peaks):
         "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<FULL>", "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm, "peak_source": f"{peaks['source']} HBM copy",
                      "algorithmic_bytes_per_launch": full_bytes, "avg_launch_ms": full_ms,
-                     "traffic": args.decode_traffic},
+                     "traffic": traffic_of("decode_full_B16_L131072")},
         "sliding_kernel": {"avg_launch_ms": ring_ms, "achieved_gbs": ring_bytes / (ring_ms / 1e3) / 1e9},
     }
 
@@ -605,9 +631,6 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="only the headline step (no sub-benchmarks)")
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows per layer for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="oracle rows per layer per reference step")
-    ap.add_argument("--full-traffic", type=float, default=None,
-                    help="DRAM bytes per full-layer prefill launch from an ncu capture (reported as traffic)")
-    ap.add_argument("--decode-traffic", type=float, default=None)
     ap.add_argument("--case", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_sliding"],
                     default=None, help="time one kernel on a small configuration (profiling)")
     ap.add_argument("--seq", type=int, default=16384)

@@ -69,6 +69,7 @@ struct PfSmem {
   uint64_t mma_done;       // every MMA of the pair completed
   uint64_t q_full;         // this CTA's query tile landed in qo
   uint64_t q_free;         // qo is free again (the previous output tile has left)
+  uint64_t sync_sm;        // the 128 softmax threads (bounded waits, unlike bar.sync)
   uint32_t tmem_base;
 };
 
@@ -220,6 +221,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     mbar_init(&sm.mma_done, 1);
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_free, 1);
+    mbar_init(&sm.sync_sm, kBM);
     fence_barrier_init();
   }
   if (warp == 5) {
@@ -353,6 +355,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     const int r = threadIdx.x;          // query row in the tile = TMEM lane
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     const float scale_log2 = 0.0625f * 1.4426950408889634f;
+    // barrier among the softmax threads; each thread counts the phases it has
+    // passed (none can get two phases ahead: every phase needs all arrivals)
+    uint32_t n_sync = 0;
+    auto sync_softmax = [&]() -> bool {
+      mbar_arrive(&sm.sync_sm);
+      return mbar_wait(&sm.sync_sm, (n_sync++) & 1);
+    };
     uint32_t J = 0;
     int item = 0;
     bool ok = true;
@@ -377,7 +386,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         rope_sincos(p_base + 16 * e, sm.inv_freq[k], &sn, &cs);
         sm.rot_hi[k][e] = make_float2(cs, sn);
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (!(ok = __all_sync(0xffffffffu, sync_softmax()))) break;
 
       // ---- this row of the query tile: shared memory (128-byte swizzled boxes) -> registers ----
       uint4 qv[kD / 8];
@@ -542,7 +551,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         }
         fence_proxy_async();
       }
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      ok = __all_sync(0xffffffffu, sync_softmax()) && ok;
       if (r == 0) {
         if (ok) {
 #pragma unroll
