@@ -263,6 +263,21 @@ __device__ __forceinline__ void mma_ts_pair_warp(uint32_t d_tmem, uint32_t a_tme
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// As mma_ts_pair_warp, with A (K-major, 128-byte swizzle) in shared memory:
+// each CTA of the pair supplies its own 128 rows of A from the same offset.
+__device__ __forceinline__ void mma_ss_pair_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                                 uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
+// Orders this thread's earlier memory writes before its later ones for every
+// thread of the cluster.
+__device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
 __device__ __forceinline__ void mma_commit_pair_warp(uint64_t* bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"
@@ -314,6 +329,15 @@ __host__ __device__ constexpr uint32_t idesc_bf16(int M, int N, bool b_mn_major)
 __device__ __forceinline__ uint64_t smem_desc_sw128(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
   return (uint64_t)((saddr >> 4) & 0x3FFFu) | ((uint64_t)((lbo >> 4) & 0x3FFFu) << 16) |
          ((uint64_t)((sbo >> 4) & 0x3FFFu) << 32) | (1ull << 46) | (2ull << 61);
+}
+// The same descriptor `bytes` further on (bytes a multiple of 16, the operand
+// inside shared memory, so the start-address field cannot overflow): one
+// 32-bit add, which keeps the MMA issue loop short -- with N = 64 the issuing
+// warp, not the tensor core, limited the rate when every descriptor was
+// rebuilt from its address.
+__device__ __forceinline__ uint64_t desc_advance(uint64_t desc, uint32_t bytes) {
+  const uint32_t lo = (uint32_t)desc + (bytes >> 4);
+  return ((desc >> 32) << 32) | lo;
 }
 
 // tcgen05.ld / st, 32 lanes x 32 bit: thread i of the warp gets lane

@@ -14,21 +14,28 @@
 // draws 32 KB from L2 per 64-key tile instead of 64 KB.
 //
 // Roles in each CTA (192 threads):
-//   warps 0-3  rotate this CTA's query head into tensor memory (rotate-half
-//              RoPE, theta / rotary dim per layer type), then the online
-//              softmax (one TMEM lane = one query row per thread) and the
-//              epilogue (1/l, sigmoid gate, bf16 store);
-//   warp 4     TMA producer for this CTA's halves of the K/V tiles, into a
-//              12-slot ring of 16 KB; bytes are counted on CTA 0's barriers;
+//   warps 0-3  rotate this CTA's query head in place in the shared-memory
+//              query tile (rotate-half RoPE, theta / rotary dim per layer
+//              type); then the online softmax (one TMEM lane = one query row
+//              per thread) and the epilogue (1/l, sigmoid gate, bf16, TMA
+//              store);
+//   warp 4     lane 0: TMA producer for this CTA's halves of the K/V tiles,
+//              into an 8-slot ring of 16 KB, bytes counted on CTA 0's
+//              barriers; lane 1: TMA producer of the query tile;
 //   warp 5     tensor-memory allocation (both CTAs); in CTA 0 the warp runs
 //              the MMA loop convergently and one elected lane issues every
 //              MMA of the pair and commits to both CTAs.
+// S = Q K^T reads both operands from shared memory: with N = 64 an MMA whose
+// A operand sits in tensor memory ran at ~40 % of the tensor rate on B200,
+// one reading A from shared memory at ~90 %.
 // Tensor memory, per CTA (512 columns x 128 lanes of 32 bit):
-//   [0,128)   Q as bf16 pairs (A operand of S = Q K^T)
-//   [128,192) S buffer 0, [192,256) S buffer 1 (fp32, 64 keys each); P of a
-//             tile (bf16 pairs) overwrites the first 32 columns of its S
-//             buffer and is the A operand of O += P V
+//   [0,256)   kNS S buffers (fp32, 64 keys each); P of a tile (bf16 pairs)
+//             overwrites the first 32 columns of its S buffer and is the A
+//             operand of O += P V
 //   [256,512) O accumulator, fp32 128 x 256.
+// The pair's MMAs run kNS - 1 key tiles ahead of the softmax (S of tile
+// j + kNS - 1 is issued before P.V of tile j), so the time the softmax of a
+// tile takes to hand P over is hidden behind tensor-core work.
 // Softmax in the log2 domain with a lazily updated row maximum: the running
 // maximum only moves (and O is only rescaled) when a tile's maximum exceeds
 // it by more than 8, so P stays <= 256.
@@ -45,14 +52,16 @@ constexpr int kKBoxRows = kBN / 2;        // K half: 32 keys x 64 dims per box
 constexpr int kKBox = kKBoxRows * 128;    // 4 KB
 constexpr int kVBox = kBN * 128;          // V half: 64 keys x 64 dims per box, 8 KB
 constexpr int kPfThreads = 192;
-constexpr uint32_t kColQ = 0;
+constexpr int kNS = 4;                    // S buffers in tensor memory
+constexpr int kAhead = kNS - 1;           // key tiles whose S is issued before the P.V of a tile
 constexpr uint32_t kColO = 256;
-constexpr float kRescaleThreshold = 8.0f;             // 1 of every 4 exponentials on the FMA pipe
-__device__ __forceinline__ uint32_t col_s(int sb) { return sb ? 192u : 128u; }
+constexpr float kRescaleThreshold = 8.0f;
+__device__ __forceinline__ uint32_t col_s(uint32_t sb) { return 64u * sb; }
 
 struct PfSmem {
   uint8_t slot[kSlots][kSlotBytes];  // 1024-byte aligned
-  uint8_t qo[4][kSlotBytes];         // the query tile in (4 boxes of 64 dims x 128 rows), the output tile out
+  uint8_t qo[4][kSlotBytes];         // the query tile in (4 boxes of 64 dims x 128 rows, rotated in place:
+                                     // the A operand of S = Q K^T), the output tile out
   double inv_freq[128];
   // rotation tables for the tile's rows (positions p_base + 16 i + j):
   //   rot_lo[k][j] = (cos, sin)(j * inv_freq_k),               j < 16
@@ -62,9 +71,9 @@ struct PfSmem {
   uint64_t full[kSlots];   // CTA 0's count both CTAs' bytes
   uint64_t empty[kSlots];  // per CTA, committed by the MMA issuer
   uint64_t q_ready;        // CTA 0: one arrival per softmax warp of the pair
-  uint64_t s_full[2];
-  uint64_t p_full[2];      // CTA 0: one arrival per softmax warp of the pair
-  uint64_t o_done;         // each P.V completed
+  uint64_t s_full[kNS];
+  uint64_t p_full[kNS];    // CTA 0: one arrival per softmax warp of the pair
+  uint64_t o_done[kNS];    // P.V of a tile in S buffer i completed (two P.Vs may be in flight)
   uint64_t o_final;        // the last P.V completed
   uint64_t mma_done;       // every MMA of the pair completed
   uint64_t q_full;         // this CTA's query tile landed in qo
@@ -86,14 +95,8 @@ struct PfArgs {
   int B, T, n_mtiles;
 };
 
-// Load order shared by the producers and the MMA issuer:
-//   K0, (K1, V0), (K2, V1), ..., (K_{n-1}, V_{n-2}), V_{n-1}
-__device__ __forceinline__ void load_of(int i, int n, bool& is_k, int& tile) {
-  if (i == 0) { is_k = true; tile = 0; return; }
-  if (i == 2 * n - 1) { is_k = false; tile = n - 1; return; }
-  if (i & 1) { is_k = true; tile = (i + 1) >> 1; }
-  else { is_k = false; tile = (i >> 1) - 1; }
-}
+// Load order shared by the K/V producer and the MMA issuer: step s (0 <= s
+// < n + kAhead) loads K_s if s < n, then V_{s - kAhead} if 0 <= s - kAhead < n.
 
 // Rotates 32 dims [k0, k0+32) against their partners [k0+R/2, ...) for one
 // query row: x1 / x2 hold 16 packed bf16 words each; results replace them.
@@ -212,11 +215,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.empty[s], 1);
     }
     mbar_init(&sm.q_ready, 8);
-    for (int s = 0; s < 2; ++s) {
+    for (int s = 0; s < kNS; ++s) {
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 8);
     }
-    mbar_init(&sm.o_done, 1);
+    for (int s = 0; s < kNS; ++s) mbar_init(&sm.o_done[s], 1);
     mbar_init(&sm.o_final, 1);
     mbar_init(&sm.mma_done, 1);
     mbar_init(&sm.q_full, 1);
@@ -254,25 +257,29 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         if (w == -2) break;
         if (w < 0) continue;
         const Item it = item_of<FULL>(w, a);
-        for (int i = 0; i < 2 * it.n; ++i, ++g) {
-          bool is_k;
-          int tile;
-          load_of(i, it.n, is_k, tile);
-          const int slot = g % kSlots;
-          if (g >= kSlots && !(ok = mbar_wait(&sm.empty[slot], ((g / kSlots) - 1) & 1))) break;
-          if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
-          const uint32_t dst = smem_u32(sm.slot[slot]);
-          const int row = (it.j_lo + tile) * kBN;
-          if (is_k) {
+        for (int st = 0; ok && st < it.n + kAhead; ++st) {
+#pragma unroll 1
+          for (int part = 0; part < 2; ++part) {
+            const bool is_k = part == 0;
+            const int tile = is_k ? st : st - kAhead;
+            if (tile < 0 || tile >= it.n) continue;
+            const int slot = g % kSlots;
+            if (g >= kSlots && !(ok = mbar_wait(&sm.empty[slot], ((g / kSlots) - 1) & 1))) break;
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
+            const uint32_t dst = smem_u32(sm.slot[slot]);
+            const int row = (it.j_lo + tile) * kBN;
+            if (is_k) {
 #pragma unroll
-            for (int box = 0; box < 4; ++box)
-              tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row + kKBoxRows * (int)rank,
-                               it.kvh, it.b);
-          } else {
+              for (int box = 0; box < 4; ++box)
+                tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row + kKBoxRows * (int)rank,
+                                 it.kvh, it.b);
+            } else {
 #pragma unroll
-            for (int box = 0; box < 2; ++box)
-              tma_load_4d_pair(dst + box * kVBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * box, row, it.kvh,
-                               it.b);
+              for (int box = 0; box < 2; ++box)
+                tma_load_4d_pair(dst + box * kVBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * box, row, it.kvh,
+                                 it.b);
+            }
+            ++g;
           }
         }
       }
@@ -301,6 +308,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     if (rank == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(2 * kBM, kBN, false);   // S = Q K^T, B K-major
       constexpr uint32_t idesc_o = idesc_bf16(2 * kBM, kD, true);     // O += P V, B MN-major
+      const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.qo[0]), 16, 1024);         // Q, K-major
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(sm.slot[0]), 16, 1024);      // K in slot 0, K-major
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(sm.slot[0]), kVBox, 1024);   // V in slot 0, MN-major
       uint32_t g = 0, J = 0;
       int item = 0;
       bool ok = true;
@@ -311,36 +321,42 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         const Item it = item_of<FULL>(w, a);
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_ready, item & 1)))) break;
         tc_fence_after();
-        for (int i = 0; i < 2 * it.n; ++i, ++g) {
-          bool is_k;
-          int tile;
-          load_of(i, it.n, is_k, tile);
-          const int slot = g % kSlots;
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (g / kSlots) & 1)))) break;
-          tc_fence_after();
-          const uint32_t saddr = smem_u32(sm.slot[slot]);
-          const uint32_t jt = J + tile;   // global tile index
-          const int sb = jt & 1;
-          if (is_k) {
-#pragma unroll
-            for (int s = 0; s < kD / 16; ++s) {
-              const uint64_t bdesc = smem_desc_sw128(saddr + (s >> 2) * kKBox + (s & 3) * 32, 16, 1024);
-              mma_ts_pair_warp(tmem + col_s(sb), tmem + kColQ + 8 * s, bdesc, idesc_s, s > 0 ? 1u : 0u);
-            }
-            mma_commit_pair_warp(&sm.empty[slot]);
-            mma_commit_pair_warp(&sm.s_full[sb]);
-          } else {
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[sb], (jt >> 1) & 1)))) break;
+        for (int st = 0; ok && st < it.n + kAhead; ++st) {
+#pragma unroll 1
+          for (int part = 0; part < 2; ++part) {
+            const bool is_k = part == 0;
+            const int tile = is_k ? st : st - kAhead;
+            if (tile < 0 || tile >= it.n) continue;
+            const int slot = g % kSlots;
+            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (g / kSlots) & 1)))) break;
             tc_fence_after();
+            const uint32_t jt = J + tile;   // global tile index
+            const uint32_t sb = jt % kNS;
+            if (is_k) {
+              const uint64_t kdesc = desc_advance(kdesc0, slot * kSlotBytes);
 #pragma unroll
-            for (int s = 0; s < kBN / 16; ++s) {
-              const uint64_t bdesc = smem_desc_sw128(saddr + s * 16 * 128, kVBox, 1024);
-              mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 8 * s, bdesc, idesc_o,
-                               (tile > 0 || s > 0) ? 1u : 0u);
+              for (int s = 0; s < kD / 16; ++s) {
+                const uint64_t adesc = desc_advance(qdesc, (s >> 2) * kSlotBytes + (s & 3) * 32);
+                const uint64_t bdesc = desc_advance(kdesc, (s >> 2) * kKBox + (s & 3) * 32);
+                mma_ss_pair_warp(tmem + col_s(sb), adesc, bdesc, idesc_s, s > 0 ? 1u : 0u);
+              }
+              mma_commit_pair_warp(&sm.empty[slot]);
+              mma_commit_pair_warp(&sm.s_full[sb]);
+            } else {
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[sb], (jt / kNS) & 1)))) break;
+              tc_fence_after();
+              const uint64_t vdesc = desc_advance(vdesc0, slot * kSlotBytes);
+#pragma unroll
+              for (int s = 0; s < kBN / 16; ++s) {
+                const uint64_t bdesc = desc_advance(vdesc, s * 16 * 128);
+                mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 8 * s, bdesc, idesc_o,
+                                 (tile > 0 || s > 0) ? 1u : 0u);
+              }
+              mma_commit_pair_warp(&sm.empty[slot]);
+              mma_commit_pair_warp(&sm.o_done[sb]);
+              if (tile == it.n - 1) mma_commit_pair_warp(&sm.o_final);
             }
-            mma_commit_pair_warp(&sm.empty[slot]);
-            mma_commit_pair_warp(&sm.o_done);
-            if (tile == it.n - 1) mma_commit_pair_warp(&sm.o_final);
+            ++g;
           }
         }
         J += it.n;
@@ -396,7 +412,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(i & 7) * 16);
         qv[i] = *reinterpret_cast<const uint4*>(sm.qo[i >> 3] + off);
       }
-      // ---- rotate it into TMEM columns [0,128) ----
+      // ---- rotate it in place (rotated dims go back to where they were read) ----
       auto words16 = [&](int dim0, uint32_t (&wd)[16]) {   // 16 packed words = dims [dim0, dim0 + 32)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -407,32 +423,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
           wd[4 * i + 3] = v.w;
         }
       };
-      if (FULL) {
+      auto store16 = [&](int dim0, const uint32_t (&wd)[16]) {   // inverse of words16, into qo
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int ci = dim0 / 8 + i;
+          const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(ci & 7) * 16);
+          *reinterpret_cast<uint4*>(sm.qo[ci >> 3] + off) = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
+        }
+      };
+#pragma unroll
+      for (int c = 0; c < R / 64; ++c) {   // dims [R, 256) are not rotated and stay as loaded
         uint32_t x1[16], x2[16];
-        words16(0, x1);
-        words16(32, x2);
-        rotate32(x1, x2, 0, p, delta, in_table, sm);
-        tmem_st16(trow + kColQ + 0, x1);
-        tmem_st16(trow + kColQ + 16, x2);
-#pragma unroll
-        for (int c = 0; c < 6; ++c) {  // dims 64..255 unchanged
-          uint32_t wd[16];
-          words16(64 + 32 * c, wd);
-          tmem_st16(trow + kColQ + 32 + 16 * c, wd);
-        }
-      } else {
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t x1[16], x2[16];
-          words16(32 * c, x1);
-          words16(128 + 32 * c, x2);
-          rotate32(x1, x2, 32 * c, p, delta, in_table, sm);
-          tmem_st16(trow + kColQ + 16 * c, x1);
-          tmem_st16(trow + kColQ + 64 + 16 * c, x2);
-        }
+        words16(32 * c, x1);
+        words16(R / 2 + 32 * c, x2);
+        rotate32(x1, x2, 32 * c, p, delta, in_table, sm);
+        store16(32 * c, x1);
+        store16(R / 2 + 32 * c, x2);
       }
-      tmem_wait_st();
-      tc_fence_before();
+      fence_proxy_async();              // qo is read by the tensor core
+      if (rank != 0) fence_cluster();   // ... through MMAs issued from CTA 0
+      tc_fence_before();                // the previous item's reads of O are done
       __syncwarp();
       if (lane == 0) {
         if (rank == 0) mbar_arrive(&sm.q_ready);
@@ -443,16 +453,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       float m_run = -INFINITY, l_run = 0.f;
       for (int j = 0; ok && j < it.n; ++j) {
         const uint32_t jt = J + j;
-        const int sb = jt & 1;
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (jt >> 1) & 1)))) break;
+        const uint32_t sb = jt % kNS;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (jt / kNS) & 1)))) break;
         tc_fence_after();
         uint32_t sraw[64];
-        {
-          uint32_t (&lo)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]);
-          uint32_t (&hi)[32] = *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]);
-          tmem_ld32(trow + col_s(sb), lo);
-          tmem_ld32(trow + col_s(sb) + 32, hi);
-        }
+        tmem_ld32(trow + col_s(sb), *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
+        tmem_ld32(trow + col_s(sb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
         tmem_wait_ld();
         float s[64];
 #pragma unroll
@@ -476,7 +482,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         for (int wd = 16; wd >= 1; wd >>= 1)
 #pragma unroll
           for (int c = 0; c < wd; ++c) mx[c] = fmaxf(mx[c], mx[c + wd]);
-        const float m_tile = mx[0] * scale_log2;
+        const float m_row = mx[0];
+        const float m_tile = m_row * scale_log2;
         const float m_new = fmaxf(m_run, m_tile);
         const bool rescale = m_new > m_run + kRescaleThreshold;
         const float m_use = rescale ? m_new : m_run;
@@ -498,9 +505,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         m_run = m_use;
         tmem_st32(trow + col_s(sb), pw);
         tmem_wait_st();
+        if (!ok) break;
         if (j > 0 && __any_sync(0xffffffffu, rescale)) {
           // O may only be touched once the previous tile's P.V has landed
-          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done, (jt - 1) & 1)))) break;
+          const uint32_t jp = jt - 1;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done[jp % kNS], (jp / kNS) & 1)))) break;
           tc_fence_after();
 #pragma unroll 1
           for (int c8 = 0; c8 < 8; ++c8) {
