@@ -77,7 +77,7 @@ struct PfSmem {
   uint64_t o_final;        // the last P.V completed
   uint64_t mma_done;       // every MMA of the pair completed
   uint64_t q_full;         // this CTA's query tile landed in qo
-  uint64_t q_free;         // qo is free again (the previous output tile has left)
+  uint64_t q_free;         // qo is free again (the item's last S = Q K^T completed)
   uint64_t sync_sm;        // the 128 softmax threads (bounded waits, unlike bar.sync)
   uint32_t tmem_base;
 };
@@ -342,6 +342,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
               }
               mma_commit_pair_warp(&sm.empty[slot]);
               mma_commit_pair_warp(&sm.s_full[sb]);
+              if (tile == it.n - 1) mma_commit_pair_warp(&sm.q_free);   // qo is no longer read
             } else {
               if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[sb], (jt / kNS) & 1)))) break;
               tc_fence_after();
@@ -368,6 +369,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     }
   } else {
     // ======================= softmax / epilogue (warps 0-3) =======================
+    // Per item: the online softmax over its key tiles; then the next item's
+    // query tile is rotated (so the pair's MMAs for it can start), and only
+    // then this item's output leaves, straight from TMEM to global memory.
     const int r = threadIdx.x;          // query row in the tile = TMEM lane
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     const float scale_log2 = 0.0625f * 1.4426950408889634f;
@@ -378,15 +382,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       mbar_arrive(&sm.sync_sm);
       return mbar_wait(&sm.sync_sm, (n_sync++) & 1);
     };
-    uint32_t J = 0;
-    int item = 0;
-    bool ok = true;
-    for (int k = 0; ok; ++k) {
-      const int w = item_index(k, pair0, n_pairs, n_items);
-      if (w == -2) break;
-      if (w < 0) continue;
-      const Item it = item_of<FULL>(w, a);
-      const int h = it.h_pair0 + (int)rank;
+    // rotates the query tile of `it` (the item_no-th of this pair) in qo and
+    // hands it to the MMA issuer
+    auto prepare_q = [&](const Item& it, int item_no) -> bool {
       const int row = it.m0 + r;
       const bool valid = row < a.T;
       const int qseq = it.qb + row;
@@ -402,11 +400,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         rope_sincos(p_base + 16 * e, sm.inv_freq[k], &sn, &cs);
         sm.rot_hi[k][e] = make_float2(cs, sn);
       }
-      if (!(ok = __all_sync(0xffffffffu, sync_softmax()))) break;
+      if (!__all_sync(0xffffffffu, sync_softmax())) return false;
 
       // ---- this row of the query tile: shared memory (128-byte swizzled boxes) -> registers ----
       uint4 qv[kD / 8];
-      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_full, item & 1)))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full, item_no & 1))) return false;
 #pragma unroll
       for (int i = 0; i < kD / 8; ++i) {
         const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(i & 7) * 16);
@@ -442,12 +440,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       }
       fence_proxy_async();              // qo is read by the tensor core
       if (rank != 0) fence_cluster();   // ... through MMAs issued from CTA 0
-      tc_fence_before();                // the previous item's reads of O are done
+      tc_fence_before();                // TMEM accesses so far precede the MMAs q_ready releases
       __syncwarp();
       if (lane == 0) {
         if (rank == 0) mbar_arrive(&sm.q_ready);
         else mbar_arrive_remote(&sm.q_ready, 0);
       }
+      return true;
+    };
+    auto next_item = [&](int& k, Item& it) -> bool {
+      for (;; ++k) {
+        const int w = item_index(k, pair0, n_pairs, n_items);
+        if (w == -2) return false;
+        if (w >= 0) {
+          it = item_of<FULL>(w, a);
+          ++k;
+          return true;
+        }
+      }
+    };
+
+    uint32_t J = 0;
+    int k = 0, item = 0;
+    Item it;
+    bool have = next_item(k, it);
+    bool ok = !have || prepare_q(it, 0);
+    while (ok && have) {
+      const int h = it.h_pair0 + (int)rank;
+      const int row = it.m0 + r;
+      const bool valid = row < a.T;
+      const int qseq = it.qb + row;
 
       // ---- online softmax over the key tiles ----
       float m_run = -INFINITY, l_run = 0.f;
@@ -505,7 +527,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         m_run = m_use;
         tmem_st32(trow + col_s(sb), pw);
         tmem_wait_st();
-        if (!ok) break;
         if (j > 0 && __any_sync(0xffffffffu, rescale)) {
           // O may only be touched once the previous tile's P.V has landed
           const uint32_t jp = jt - 1;
@@ -530,22 +551,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         }
       }
       J += it.n;
+      if (!ok) break;
+      Item nxt{};
+      const bool have_next = next_item(k, nxt);
+      if (have_next && !(ok = prepare_q(nxt, item + 1))) break;
 
-      // ---- epilogue: O / l * sigmoid(gate) -> bf16 -> qo -> TMA store ----
-      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, item & 1));
-      if (ok) {
-        tc_fence_after();
-        float f = l_run > 0.f ? 1.f / l_run : 0.f;
-        if (a.gate != nullptr && valid) {
-          const float gs = __bfloat162float(a.gate[((int64_t)it.b * a.T + row) * kHq + h]);
-          f *= 1.f / (1.f + __expf(-gs));
-        }
+      // ---- epilogue: O / l * sigmoid(gate) -> bf16 -> global ----
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, item & 1)))) break;
+      tc_fence_after();
+      float f = l_run > 0.f ? 1.f / l_run : 0.f;
+      if (a.gate != nullptr && valid) {
+        const float gs = __bfloat162float(a.gate[((int64_t)it.b * a.T + row) * kHq + h]);
+        f *= 1.f / (1.f + __expf(-gs));
+      }
+      __nv_bfloat16* orow = a.out + (((int64_t)it.b * a.T + row) * kHq + h) * kD;
 #pragma unroll 1
-        for (int c8 = 0; c8 < 8; ++c8) {
-          uint32_t ov[32];
-          tmem_ld32(trow + kColO + 32 * c8, ov);
-          tmem_wait_ld();
-          uint8_t* box = sm.qo[c8 >> 1];
+      for (int c8 = 0; c8 < 8; ++c8) {
+        uint32_t ov[32];
+        tmem_ld32(trow + kColO + 32 * c8, ov);
+        tmem_wait_ld();
+        if (valid) {
 #pragma unroll
           for (int q4 = 0; q4 < 4; ++q4) {
             uint32_t w4[4];
@@ -554,22 +579,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
               const int c = 8 * q4 + 2 * e;
               w4[e] = pack_bf16(__uint_as_float(ov[c]) * f, __uint_as_float(ov[c + 1]) * f);
             }
-            const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(((c8 & 1) * 4 + q4) * 16));
-            *reinterpret_cast<uint4*>(box + off) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+            *reinterpret_cast<uint4*>(orow + 32 * c8 + 8 * q4) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
         }
-        fence_proxy_async();
       }
-      ok = __all_sync(0xffffffffu, sync_softmax()) && ok;
-      if (r == 0) {
-        if (ok) {
-#pragma unroll
-          for (int box = 0; box < 4; ++box) tma_store_4d(&tm_o, smem_u32(sm.qo[box]), box * 64, h, it.m0, it.b);
-          tma_store_commit_and_wait();
-        }
-        mbar_arrive(&sm.q_free);   // the next query tile may land in qo
-      }
-      ok = __all_sync(0xffffffffu, ok);
+      it = nxt;
+      have = have_next;
       ++item;
     }
   }
