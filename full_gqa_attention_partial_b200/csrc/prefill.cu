@@ -64,10 +64,12 @@ struct PfSmem {
                                      // the A operand of S = Q K^T), the output tile out
   double inv_freq[128];
   // rotation tables for the tile's rows (positions p_base + 16 i + j):
-  //   rot_lo[k][j] = (cos, sin)(j * inv_freq_k),               j < 16
-  //   rot_hi[k][i] = (cos, sin)((p_base + 16 i) * inv_freq_k),  i < 8
-  float2 rot_lo[128][16];
-  float2 rot_hi[128][8];
+  //   rot_lo[k / 2][j] = (cos, sin)(j * inv_freq_k), k even then odd,             j < 16
+  //   rot_hi[i][k / 2] = (cos, sin)((p_base + 16 i) * inv_freq_k), k even then odd,  i < 8
+  // (two frequencies per 16-byte entry: one shared-memory load per pair of them)
+  float4 rot_lo[64][16];
+  float4 rot_hi[8][64];
+  uint8_t ostage[4][2048];           // per softmax warp: 32 rows x 32 output dims (bf16), transposed on the way out
   uint64_t full[kSlots];   // CTA 0's count both CTAs' bytes
   uint64_t empty[kSlots];  // per CTA, committed by the MMA issuer
   uint64_t q_ready;        // CTA 0: one arrival per softmax warp of the pair
@@ -83,6 +85,7 @@ struct PfSmem {
 };
 
 size_t prefill_smem_bytes() { return sizeof(PfSmem) + 1024; }
+static_assert(sizeof(PfSmem) + 1024 <= 232448, "prefill shared memory exceeds 227 KB");
 
 struct PfArgs {
   const __nv_bfloat16* q;
@@ -102,20 +105,22 @@ struct PfArgs {
 // query row: x1 / x2 hold 16 packed bf16 words each; results replace them.
 // Pair k turns by p * inv_freq_k.  Table form, for a row at p_base + 16 i + j
 // (the rows of a tile are consecutive positions): the turn is the product of
-// two precomputed unit complex numbers, rot_hi[k][i] * rot_lo[k][j].  General
-// form (any other position): the fp64-reduced full angle.
+// two precomputed unit complex numbers (rot_hi for i, rot_lo for j).
+// General form (any other position): the fp64-reduced full angle.
 __device__ __forceinline__ void rotate32_table(uint32_t (&x1)[16], uint32_t (&x2)[16], int k0, int i_hi,
-                                               int j_lo, const float2 (*rot_lo)[16], const float2 (*rot_hi)[8]) {
+                                               int j_lo, const float4 (*rot_lo)[16], const float4 (*rot_hi)[64]) {
 #pragma unroll
   for (int w = 0; w < 16; ++w) {
+    const int kp = k0 / 2 + w;   // frequencies 2 kp and 2 kp + 1
+    const float4 u4 = rot_hi[i_hi][kp];
+    const float4 v4 = rot_lo[kp][j_lo];
     float a[2], bb[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
-      const int k = k0 + 2 * w + e;
       const float x = e ? bf16hi(x1[w]) : bf16lo(x1[w]);
       const float y = e ? bf16hi(x2[w]) : bf16lo(x2[w]);
-      const float2 u = rot_hi[k][i_hi];
-      const float2 v = rot_lo[k][j_lo];
+      const float2 u = e ? make_float2(u4.z, u4.w) : make_float2(u4.x, u4.y);
+      const float2 v = e ? make_float2(v4.z, v4.w) : make_float2(v4.x, v4.y);
       const float c = fmaf(u.x, v.x, -u.y * v.y);
       const float s = fmaf(u.y, v.x, u.x * v.y);
       a[e] = fmaf(x, c, -y * s);
@@ -238,7 +243,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     const int k = t % (R / 2), e = t / (R / 2);
     float sn, cs;
     small_angle_sincos(e, (float)sm.inv_freq[k], &sn, &cs);
-    sm.rot_lo[k][e] = make_float2(cs, sn);
+    reinterpret_cast<float2*>(&sm.rot_lo[k >> 1][e])[k & 1] = make_float2(cs, sn);
   }
   tc_fence_before();
   cluster_sync();   // barriers of both CTAs initialised before any cross-CTA arrive
@@ -398,7 +403,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         const int k = t % (R / 2), e = t / (R / 2);
         float sn, cs;
         rope_sincos(p_base + 16 * e, sm.inv_freq[k], &sn, &cs);
-        sm.rot_hi[k][e] = make_float2(cs, sn);
+        reinterpret_cast<float2*>(&sm.rot_hi[e][k >> 1])[k & 1] = make_float2(cs, sn);
       }
       if (!__all_sync(0xffffffffu, sync_softmax())) return false;
 
@@ -557,6 +562,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       if (have_next && !(ok = prepare_q(nxt, item + 1))) break;
 
       // ---- epilogue: O / l * sigmoid(gate) -> bf16 -> global ----
+      // 32 dims at a time through the warp's staging area: each thread writes
+      // its row (16-byte chunks XOR-swizzled by row, so neither phase has bank
+      // conflicts), then each store instruction covers 8 rows x 64 bytes.
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, item & 1)))) break;
       tc_fence_after();
       float f = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -564,24 +572,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         const float gs = __bfloat162float(a.gate[((int64_t)it.b * a.T + row) * kHq + h]);
         f *= 1.f / (1.f + __expf(-gs));
       }
-      __nv_bfloat16* orow = a.out + (((int64_t)it.b * a.T + row) * kHq + h) * kD;
+      uint8_t* stg = sm.ostage[warp];
+      const int rr = lane >> 2, ch = lane & 3;   // store phase: rows rr + 8 t, chunk ch
 #pragma unroll 1
       for (int c8 = 0; c8 < 8; ++c8) {
         uint32_t ov[32];
         tmem_ld32(trow + kColO + 32 * c8, ov);
         tmem_wait_ld();
-        if (valid) {
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint32_t w4[4];
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t w4[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              const int c = 8 * q4 + 2 * e;
-              w4[e] = pack_bf16(__uint_as_float(ov[c]) * f, __uint_as_float(ov[c + 1]) * f);
-            }
-            *reinterpret_cast<uint4*>(orow + 32 * c8 + 8 * q4) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+          for (int e = 0; e < 4; ++e) {
+            const int c = 8 * q4 + 2 * e;
+            w4[e] = pack_bf16(__uint_as_float(ov[c]) * f, __uint_as_float(ov[c + 1]) * f);
           }
+          *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q4 ^ ((lane >> 1) & 3))) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
+        __syncwarp();
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+          const int rw = rr + 8 * t;                   // row within this warp's 32
+          const int grow = it.m0 + 32 * warp + rw;     // query row in the sequence
+          const uint4 v = *reinterpret_cast<const uint4*>(stg + rw * 64 + 16 * (ch ^ ((rw >> 1) & 3)));
+          if (grow < a.T)
+            *reinterpret_cast<uint4*>(a.out + (((int64_t)it.b * a.T + grow) * kHq + h) * kD + 32 * c8 + 8 * ch) = v;
+        }
+        __syncwarp();
       }
       it = nxt;
       have = have_next;
