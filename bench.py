@@ -69,9 +69,17 @@ def layer_seed(base: int, i: int) -> int:
 # the capture's summary).  Reported as roofline.traffic only while the sources are
 # unchanged; otherwise null.
 TRAFFIC = {
-    "prefill_full_T32768": {"bytes": 2.225e9, "sha": "52c4bcaa723ed33b",
+    "prefill_full_T32768": {"bytes": 2.173e9, "sha": "5f20a5427468bc15",
                             "sources": ["prefill.cu", "common.cuh"],
                             "capture": "profiles/prefill_kernel_full_T32768.md"},
+    "prefill_sliding_T32768": {"bytes": 0.6386e9, "sha": "5f20a5427468bc15",
+                               "sources": ["prefill.cu", "common.cuh"],
+                               "capture": "profiles/prefill_kernel_sliding_T32768.md"},
+    # captured at 16 x 32768 tokens (2.153 GB); decode streams each cached byte
+    # once, so traffic scales with the tokens: x 8590491648 / 2147483648
+    "decode_full_B16_L131072": {"bytes": 2.153e9 * 8590491648 / 2147483648, "sha": "bba9668dc1aff40b",
+                                "sources": ["decode.cu", "common.cuh"],
+                                "capture": "profiles/decode_split_kernel_full_B16_L32768.md"},
 }
 
 
@@ -264,7 +272,8 @@ def bench_main(hyb, args, dist: Dist, peaks):
             "avg_launch_ms": full_ms, "launches": len(per_layer[3]),
             "traffic": traffic_of("prefill_full_T32768"),
             "sliding_kernel": {"avg_launch_ms": slide_ms,
-                               "achieved": flops(T_MAIN, SLIDING) / (slide_ms / 1e3) / 1e12},
+                               "achieved": flops(T_MAIN, SLIDING) / (slide_ms / 1e3) / 1e12,
+                               "traffic": traffic_of("prefill_sliding_T32768")},
             "attention_kernels_share_of_step": kernel_share,
         },
     }
