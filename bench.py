@@ -278,31 +278,66 @@ def bench_main(hyb, args, dist: Dist, peaks):
         },
     }
     # ---- e2e: pinned host inputs -> device -> library -> host ----
+    # Three streams: host-to-device copies of the next layer's inputs and the
+    # device-to-host copy of the previous layer's output overlap the attention
+    # of the current layer (two input buffers, one output buffer per layer).
     host_in = [{k: layers[li][k].cpu().pin_memory() for k in ("qkv", "gate")} for li in range(len(GROUP_LAYERS))]
     host_out = [torch.empty(B_MAIN, T_MAIN, H, D, dtype=torch.bfloat16).pin_memory() for _ in GROUP_LAYERS]
-    dev_qkv = torch.empty_like(layers[0]["qkv"])
-    dev_gate = torch.empty_like(layers[0]["gate"])
+    dev_qkv = [torch.empty_like(layers[0]["qkv"]) for _ in range(2)]
+    dev_gate = [torch.empty_like(layers[0]["gate"]) for _ in range(2)]
     e2e_caches = [[hyb.KVCache(lt, B_MAIN, capacity=T_MAIN) for lt in GROUP_LAYERS] for _ in range(n_steps)]
-    q = dev_qkv[..., :4096].unflatten(-1, (H, D))
-    k = dev_qkv[..., 4096:5120].unflatten(-1, (KVH, D))
-    v = dev_qkv[..., 5120:].unflatten(-1, (KVH, D))
+    qkv_views = [(x[..., :4096].unflatten(-1, (H, D)), x[..., 4096:5120].unflatten(-1, (KVH, D)),
+                  x[..., 5120:].unflatten(-1, (KVH, D))) for x in dev_qkv]
     h2d = sum(t.numel() * t.element_size() for hi in host_in for t in hi.values())
     d2h = sum(t.numel() * t.element_size() for t in host_out)
+    comp = torch.cuda.current_stream()
+    s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]
+    in_free = [torch.cuda.Event() for _ in range(2)]
+    out_ready = [torch.cuda.Event() for _ in GROUP_LAYERS]
+    out_free = [torch.cuda.Event() for _ in GROUP_LAYERS]
+    n_layer_calls = [0]
 
     def e2e_step(i):
         for li, lt in enumerate(GROUP_LAYERS):
-            dev_qkv.copy_(host_in[li]["qkv"], non_blocking=True)
-            dev_gate.copy_(host_in[li]["gate"], non_blocking=True)
-            hyb.hyb_attn_prefill(q, k, v, dev_gate, None, lt, out=outs[li], cache=e2e_caches[i][li], workspace=ws)
-            host_out[li].copy_(outs[li], non_blocking=True)
+            n = n_layer_calls[0]
+            buf = n % 2
+            with torch.cuda.stream(s_in):
+                if n >= 2:
+                    s_in.wait_event(in_free[buf])
+                dev_qkv[buf].copy_(host_in[li]["qkv"], non_blocking=True)
+                dev_gate[buf].copy_(host_in[li]["gate"], non_blocking=True)
+                in_ready[buf].record(s_in)
+            comp.wait_event(in_ready[buf])
+            if n >= len(GROUP_LAYERS):
+                comp.wait_event(out_free[li])
+            q, k, v = qkv_views[buf]
+            hyb.hyb_attn_prefill(q, k, v, dev_gate[buf], None, lt, out=outs[li], cache=e2e_caches[i][li], workspace=ws)
+            in_free[buf].record(comp)
+            out_ready[li].record(comp)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(out_ready[li])
+                host_out[li].copy_(outs[li], non_blocking=True)
+                out_free[li].record(s_out)
+            n_layer_calls[0] += 1
+
+    def drain():   # the compute stream waits for every copy issued so far
+        for li in range(len(GROUP_LAYERS)):
+            comp.wait_event(out_free[li])
+        for b in range(2):
+            ev = torch.cuda.Event()
+            ev.record(s_in)
+            comp.wait_event(ev)
 
     for i in range(args.warmup):
         e2e_step(i)
+    drain()
     torch.cuda.synchronize()
     dist.barrier()
     ev0.record()
     for i in range(args.steps):
         e2e_step(args.warmup + i)
+    drain()
     ev1.record()
     torch.cuda.synchronize()
     e2e_rate, e2e_ms = dist.aggregate(args.steps * step_flops, ev0.elapsed_time(ev1))
