@@ -240,6 +240,31 @@ def decode(q, gate, qpos, cache_k, cache_v, cache_idx, lt):
     return out
 
 
+def decode_group(q_rows, k, v, q_idx, k_idx, lt, gate=None):
+    """One decode query for the query heads of a single KV group.
+
+    The same definition as gqa_attention, written per group (the grouping of
+    [LAPTOP] §"分组查询注意力" applied by indexing instead of repeating K/V),
+    so that a history of ~10^6 keys fits in host memory.
+    q_rows [G, D] the group's query heads, already roped; k / v [L, D] that
+    KV head's keys (roped) and values; k_idx [L] their sequence indices; the
+    query sits at sequence index q_idx.  gate [G] raw gate scores or None.
+    Returns [G, D] float64.
+    """
+    q_rows = np.asarray(q_rows, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    v = np.asarray(v, dtype=np.float64)
+    visible = dense_mask(np.array([q_idx]), np.asarray(k_idx), window_of(lt))[0]
+    s = (q_rows @ k.T) / np.sqrt(q_rows.shape[-1])          # [G, L]
+    s = np.where(visible[None], s, -np.inf)
+    m = s.max(axis=-1, keepdims=True)
+    p = np.exp(s - m)
+    o = (p @ v) / p.sum(axis=-1, keepdims=True)
+    if gate is not None:
+        o = o * sigmoid(gate)[:, None]
+    return o
+
+
 # ---------------------------------------------------------------------------
 # KV caches: linear (full layers) and the 512-slot ring (sliding layers)
 # ---------------------------------------------------------------------------

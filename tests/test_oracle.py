@@ -335,3 +335,21 @@ def test_pair_counts_match_dense_mask(n):
         assert O.attention_pairs(n, lt) == int(O.dense_mask(idx, idx, O.window_of(lt)).sum())
     assert O.prefill_flops(1024, O.FULL) == 524_800 * 16 * 1024
     assert O.attention_pairs(1024, O.SLIDING) == 393_472
+
+
+@pytest.mark.parametrize("lt", [O.SLIDING, O.FULL])
+def test_decode_group_equals_gqa_attention(lt):
+    """The per-group decode form agrees with the dense GQA definition (itself
+    pinned by brute force above) on a history that crosses the window."""
+    rng = np.random.default_rng(11)
+    L = 700
+    k = rng.standard_normal((L, O.N_KV_HEADS, O.HEAD_DIM))
+    v = rng.standard_normal((L, O.N_KV_HEADS, O.HEAD_DIM))
+    q = rng.standard_normal((1, O.N_Q_HEADS, O.HEAD_DIM))
+    g = rng.standard_normal((1, O.N_Q_HEADS))
+    idx = rng.permutation(L)            # any order of the history
+    ref = O.gqa_attention(q, k, v, np.array([L - 1]), idx, O.window_of(lt), g)[0]
+    for kvh in range(O.N_KV_HEADS):
+        hs = slice(O.GROUP * kvh, O.GROUP * (kvh + 1))
+        got = O.decode_group(q[0, hs], k[:, kvh], v[:, kvh], L - 1, idx, lt, g[0, hs])
+        np.testing.assert_allclose(got, ref[hs], rtol=1e-12, atol=1e-12)

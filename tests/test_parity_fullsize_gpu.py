@@ -2,17 +2,19 @@
 
 Each case runs the CUDA path at the workload's full size and compares a
 sample of outputs with the fp64 oracle, which computes those rows (or
-sequences) one by one from the same seeded inputs:
+decode steps) from the same seeded inputs.  Row samples per prefill layer:
+every row within 600 of a band edge (the start of the sequence and the
+point where the 512-key window becomes full), the first and last 256 rows,
+rows around query-tile edges, and 1024 random rows (fixed seeds):
 
-* the 3-sliding + 1-full group prefill at T=32768 into fresh KV caches:
-  first and last 128 rows, rows around the 512-key band edge and tile
-  edges, 64 random rows, per layer;
-* one full layer at T=131072 without a cache: last 64 rows, first 16 rows,
-  tile edges, random rows;
+* the 3-sliding + 1-full group prefill at T=32768 into fresh KV caches;
+* one full layer at T=131072 without a cache (the same sample, without the
+  band-edge block, which the first 256 rows cover for a full layer);
 * decode at batch 16 over a 131072-token full-layer cache and a full ring
-  (write head at a random offset), after an append: 3 sequences of the full
-  layer and all 16 of the sliding layer;
-* decode over a 1,048,576-token full-layer cache;
+  (write head at a random offset), after an append;
+* 64 steps of append + decode on a full-layer cache prefilled with
+  1,048,512 tokens (ending at 1,048,576) and on a full ring, every step and
+  all 16 heads of both layers compared;
 * chunked prefill of 262144 tokens in 8192-token chunks, full and sliding
   layer: rows of the second, a middle and the last chunk.
 """
@@ -42,16 +44,40 @@ def check(got, ref, what):
     assert max_abs <= MAX_ABS and rel <= REL_L2, f"{what}: max_abs {max_abs:.3e} rel_l2 {rel:.3e}"
 
 
-def sample_rows(T, n_random, seed, head=128, tail=128):
+def sample_rows(T, n_random, seed, head=256, tail=256, band_edges=True):
     rng = np.random.default_rng(seed)
-    edges = [e + d for e in (63, 64, 127, 128, 511, 512, 1023, 1024, T // 2) for d in (-1, 0, 1)]
-    rows = set(range(min(head, T))) | set(range(max(0, T - tail), T)) | {e for e in edges if 0 <= e < T}
+    rows = set(range(min(head, T))) | set(range(max(0, T - tail), T))
+    if band_edges:   # within 600 of row 0 and of row 511 (first row with a full window)
+        rows |= set(range(0, min(T, O.WINDOW - 1 + 601)))
+    edges = [e + d for e in (63, 64, 127, 128, 1023, 1024, T // 2) for d in (-1, 0, 1)]
+    rows |= {e for e in edges if 0 <= e < T}
     rows |= set(rng.choice(T, size=min(n_random, T), replace=False).tolist())
     return np.array(sorted(rows))
 
 
 def host_layer(x):
     return {k: f64(x[k]) if k != "pos" else x[k].cpu().numpy() for k in ("q", "k", "v", "gate", "pos")}
+
+
+def oracle_rows(h, lt, rows, max_rows=128, max_span=4096):
+    """The oracle's prefill rows (sorted), a chunk of rows at a time; each chunk
+    passes only the tokens its rows can see (from the first key of the
+    earliest row's band to the last row), positioned by `start`."""
+    rows = np.sort(np.asarray(rows))
+    out = []
+    i = 0
+    while i < len(rows):
+        j = i + 1
+        while j < len(rows) and j - i < max_rows and (lt == O.FULL or rows[j] - rows[i] <= max_span):
+            j += 1
+        chunk = rows[i:j]
+        lo = 0 if lt == O.FULL else max(0, int(chunk[0]) - (O.WINDOW - 1))
+        hi = int(chunk[-1]) + 1
+        sl = slice(lo, hi)
+        out.append(O.prefill(h["q"][:, sl], h["k"][:, sl], h["v"][:, sl], h["gate"][:, sl], h["pos"][:, sl], lt,
+                             rows=chunk - lo, start=[lo]))
+        i = j
+    return np.concatenate(out, axis=1)
 
 
 def test_group_prefill_T32768_into_caches(lib):
@@ -62,10 +88,9 @@ def test_group_prefill_T32768_into_caches(lib):
         out = lib.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], None, lt, cache=cache)
         torch.cuda.synchronize()
         assert lib.hyb_device_error() == 0
-        rows = sample_rows(T, 64, seed=li)
-        h = host_layer(x)
-        ref = O.prefill(h["q"], h["k"], h["v"], h["gate"], h["pos"], lt, rows=rows)
-        check(out[:, rows], ref, f"group layer {li} (type {lt})")
+        rows = sample_rows(T, 1024, seed=li)
+        ref = oracle_rows(host_layer(x), lt, rows)
+        check(out[:, rows], ref, f"group layer {li} (type {lt}), {len(rows)} rows")
         del x, cache, out
 
 
@@ -75,10 +100,9 @@ def test_full_layer_prefill_T131072(lib):
     out = lib.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], x["pos"], lib.FULL)
     torch.cuda.synchronize()
     assert lib.hyb_device_error() == 0
-    rows = sample_rows(T, 32, seed=7, head=16, tail=64)
-    h = host_layer(x)
-    ref = O.prefill(h["q"], h["k"], h["v"], h["gate"], h["pos"], O.FULL, rows=rows)
-    check(out[:, rows], ref, "full layer T=131072")
+    rows = sample_rows(T, 1024, seed=7, band_edges=False)
+    ref = oracle_rows(host_layer(x), O.FULL, rows, max_rows=64)
+    check(out[:, rows], ref, f"full layer T=131072, {len(rows)} rows")
 
 
 def test_decode_batch16_L131072(lib):
@@ -121,31 +145,59 @@ def test_decode_batch16_L131072(lib):
             check(out, ref, "sliding decode, 16 sequences")
 
 
-def test_decode_L1M_full_layer(lib):
-    L0 = (1 << 20) - 64
+def test_decode_1m_64_steps(lib):
+    """The 1M-token decode workload's two layer types: 64 steps of append +
+    decode, each step compared for all 16 heads.  The oracle keeps its own fp64
+    history (the seeded cache content, snapshot before any library call, plus
+    each step's raw token rotated by the oracle)."""
+    n_steps = 64
     cap = 1 << 20
+    L0 = cap - n_steps
+    r = synth.ring_offset(3)
     full = bench.fill_full_cache(lib, 1, L0, cap, seed=3)
-    hist_k = full.k[0, :, :L0].cpu()                     # seeded history, before any library call on it
-    hist_v = full.v[0, :, :L0].cpu()
-    x = synth.decode_query(1, seed=9000, device="cuda")
-    lib.hyb_kv_append(full, x["k"], x["v"])
-    out = lib.hyb_attn_decode(x["q"], x["gate"], full, max_len=cap)
-    torch.cuda.synchronize()
-    assert lib.hyb_device_error() == 0
-    n = L0 + 1
-    q, g = f64(x["q"])[0], f64(x["gate"])[0]
-    qr = O.rope_layer(q[None], np.array([n - 1]), O.FULL)          # [1, 16, 256]
-    kn = O.rope_layer(f64(x["k"])[0], np.array([n - 1]), O.FULL)   # [1, 4, 256]
-    vn = f64(x["v"])[0]
-    ref = np.zeros((16, 256))
-    idx = np.arange(n)
-    for kvh in range(4):    # one KV group at a time keeps the fp64 copies at ~4 GB
-        kc = np.concatenate([f64(hist_k[kvh]), kn[:, kvh]])[:, None]
-        vc = np.concatenate([f64(hist_v[kvh]), vn[:, kvh]])[:, None]
-        hs = slice(4 * kvh, 4 * kvh + 4)
-        ref[hs] = O.gqa_attention(qr[:, hs], kc, vc, np.array([n - 1]), idx, None, g[None, hs])[0]
-        del kc, vc
-    check(out[0], ref, "full decode at 1M tokens")
+    ring = bench.fill_ring_cache(lib, 1, L0, seed=5, head0=r)
+    hk = np.empty((O.N_KV_HEADS, cap, O.HEAD_DIM))
+    hv = np.empty((O.N_KV_HEADS, cap, O.HEAD_DIM))
+    for h in range(O.N_KV_HEADS):
+        hk[h, :L0] = f64(full.k[0, h, :L0])
+        hv[h, :L0] = f64(full.v[0, h, :L0])
+    # ring: token i (L0 - 512 <= i < L0) at slot (r + i) % 512
+    ring_k = f64(ring.k[0]).transpose(1, 0, 2)       # [512 slots, 4, 256]
+    ring_v = f64(ring.v[0]).transpose(1, 0, 2)
+    win_idx = list(range(L0 - O.WINDOW, L0))
+    win_k = [ring_k[(r + i) % O.WINDOW] for i in win_idx]
+    win_v = [ring_v[(r + i) % O.WINDOW] for i in win_idx]
+    for step in range(n_steps):
+        x = synth.decode_query(1, seed=20000 + step, device="cuda")
+        lib.hyb_kv_append(full, x["k"], x["v"])
+        lib.hyb_kv_append(ring, x["k"], x["v"])
+        out_f = lib.hyb_attn_decode(x["q"], x["gate"], full, max_len=cap)
+        out_r = lib.hyb_attn_decode(x["q"], x["gate"], ring, max_len=O.WINDOW)
+        torch.cuda.synchronize()
+        assert lib.hyb_device_error() == 0
+        n = L0 + step + 1                            # tokens after the append; the query is token n - 1
+        q, g = f64(x["q"])[0], f64(x["gate"])[0]
+        knew, vnew = f64(x["k"])[0, 0], f64(x["v"])[0, 0]
+        # full layer
+        hk[:, n - 1] = O.rope_layer(knew[None], np.array([n - 1]), O.FULL)[0]
+        hv[:, n - 1] = vnew
+        qf = O.rope_layer(q[None], np.array([n - 1]), O.FULL)[0]
+        ref = np.empty((O.N_Q_HEADS, O.HEAD_DIM))
+        idx = np.arange(n)
+        for kvh in range(O.N_KV_HEADS):
+            hs = slice(O.GROUP * kvh, O.GROUP * (kvh + 1))
+            ref[hs] = O.decode_group(qf[hs], hk[kvh, :n], hv[kvh, :n], n - 1, idx, O.FULL, g[hs])
+        check(out_f[0], ref, f"1M decode step {step}, full layer")
+        # sliding layer
+        win_idx = win_idx[1:] + [n - 1]
+        win_k = win_k[1:] + [O.rope_layer(knew[None], np.array([n - 1]), O.SLIDING)[0]]
+        win_v = win_v[1:] + [vnew]
+        qs = O.rope_layer(q[None], np.array([n - 1]), O.SLIDING)[0]
+        wk, wv = np.stack(win_k), np.stack(win_v)    # [512, 4, 256]
+        for kvh in range(O.N_KV_HEADS):
+            hs = slice(O.GROUP * kvh, O.GROUP * (kvh + 1))
+            ref[hs] = O.decode_group(qs[hs], wk[:, kvh], wv[:, kvh], n - 1, np.array(win_idx), O.SLIDING, g[hs])
+        check(out_r[0], ref, f"1M decode step {step}, sliding layer")
 
 
 @pytest.mark.parametrize("lt", [O.SLIDING, O.FULL])
@@ -168,7 +220,7 @@ def test_chunked_prefill_262144(lib, lt):
             hk = torch.cat(hist_k[:-1], 1)[0, lo:start] if c > 0 else None
             hv = torch.cat(hist_v[:-1], 1)[0, lo:start] if c > 0 else None
             idx = np.arange(lo, start)
-            rows = sample_rows(C, 32, seed=c, head=48, tail=48)
+            rows = sample_rows(C, 32, seed=c, head=48, tail=48, band_edges=False)
             h = host_layer(x)
             ref = O.prefill(h["q"], h["k"], h["v"], h["gate"], h["pos"], lt, rows=rows, start=[start],
                             hist_k=[O.rope_layer(f64(hk), idx, lt)], hist_v=[f64(hv)], hist_idx=[idx])
