@@ -114,7 +114,9 @@ class Dist:
         if self.world > 1:
             import datetime
             import torch.distributed as dist
-            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            # a short timeout: ranks waiting on one that died end with an error
+            limit_s = float(os.environ.get("HYB_PG_TIMEOUT_S", "120"))
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=limit_s))
             self.pg = dist
         if backend == "nccl" and torch.cuda.is_available():
             torch.cuda.set_device(self.local)

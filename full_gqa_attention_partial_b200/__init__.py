@@ -36,6 +36,7 @@ EXPORTED = (
     "hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill_workspace_size", "hyb_attn_prefill",
     "hyb_attn_decode_workspace_size", "hyb_attn_decode", "hyb_device_error", "hyb_last_error",
     "hyb_launch_count", "hyb_profile_events", "hyb_profile_pairs_used", "hyb_attn_decode_noalloc",
+    "hyb_selftest_wait_timeout",
 )
 
 
@@ -90,6 +91,7 @@ def load(path: str = LIB_PATH):
     lib.hyb_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     lib.hyb_profile_events.restype = ctypes.c_int
     lib.hyb_profile_pairs_used.restype = i32
+    lib.hyb_selftest_wait_timeout.argtypes = [vp]
     for name in ("hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill", "hyb_attn_decode",
                  "hyb_device_error"):
         getattr(lib, name).restype = ctypes.c_int
@@ -254,6 +256,12 @@ def hyb_device_error(clear: bool = True, stream=None) -> int:
     flags = ctypes.c_int32(0)
     _check(load().hyb_device_error(ctypes.byref(flags), 1 if clear else 0, _stream(stream)))
     return int(flags.value)
+
+
+def hyb_selftest_wait_timeout(stream=None) -> None:
+    """Runs the failure-path self-test kernel (a wait that times out); the
+    error word then holds DEV_ERR_TIMEOUT (read it with hyb_device_error)."""
+    _check(load().hyb_selftest_wait_timeout(_stream(stream)))
 
 
 def hyb_launch_count() -> int:

@@ -213,6 +213,14 @@ hyb_status hyb_device_error(int32_t* flags, int32_t clear, void* stream) {
   return HYB_OK;
 }
 
+hyb_status hyb_selftest_wait_timeout(void* stream) {
+  hyb_status s = ensure_device();
+  if (s != HYB_OK) return s;
+  cudaError_t e = launch_selftest_wait(as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "self-test launch");
+  return HYB_OK;
+}
+
 hyb_status hyb_kv_cache_init(const hyb_kv_cache* c, const int32_t* head0, void* stream) {
   hyb_status s = check_cache(c);
   if (s != HYB_OK) return s;

@@ -37,6 +37,7 @@ cudaError_t launch_ring_gather(const void* rk, const void* rv, const int32_t* le
                                cudaStream_t st);
 cudaError_t launch_kv_commit(int32_t* len, int32_t* head, int64_t capacity, bool ring, int B, int T,
                              cudaStream_t st);
+cudaError_t launch_selftest_wait(cudaStream_t st);
 cudaError_t launch_fill_i32(int32_t* p, int64_t n, int32_t v, cudaStream_t st);
 
 // ---- prefill attention (prefill.cu) -----------------------------------------

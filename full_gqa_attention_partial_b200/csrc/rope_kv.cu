@@ -220,6 +220,23 @@ cudaError_t launch_kv_commit(int32_t* len, int32_t* head, int64_t capacity, bool
   return cudaGetLastError();
 }
 
+// One thread waits on a barrier that nothing completes; the bounded wait
+// raises the timeout bit and the kernel ends (failure-path self-test).
+__global__ void selftest_wait_kernel() {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+    (void)mbar_wait(&bar, 0);
+  }
+}
+
+cudaError_t launch_selftest_wait(cudaStream_t st) {
+  selftest_wait_kernel<<<1, 32, 0, st>>>();
+  count_launch();
+  return cudaGetLastError();
+}
+
 cudaError_t launch_fill_i32(int32_t* p, int64_t n, int32_t v, cudaStream_t st) {
   if (n <= 0) return cudaSuccess;
   int64_t blocks = (n + 255) / 256;

@@ -201,6 +201,17 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
  */
 hyb_status hyb_device_error(int32_t* flags, int32_t clear, void* stream);
 
+/*
+ * Failure-path self-test (no counterpart in the pages).  Launches one block
+ * on `stream` whose first thread waits on a shared-memory barrier that
+ * nothing completes.  The wait is bounded like every pipeline wait of the
+ * library: it gives up after its limit (about 2 s of device time; 1 ms once
+ * the error word already holds HYB_DEV_ERR_TIMEOUT), raises
+ * HYB_DEV_ERR_TIMEOUT in the error word and the kernel returns, leaving the
+ * context usable.  Returns HYB_ECUDA if the launch fails.
+ */
+hyb_status hyb_selftest_wait_timeout(void* stream);
+
 /* Message for the last non-OK status returned on the calling thread. */
 const char* hyb_last_error(void);
 

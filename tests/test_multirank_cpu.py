@@ -2,7 +2,9 @@
 
 Each rank reports its own timing; the job's throughput must be all ranks'
 work over the slowest rank's time (weak scaling: every rank runs the same
-per-rank step), and the reference arm must run on rank 0 only.
+per-rank step), and the reference arm must run on rank 0 only.  Failures
+are made on the host: a rank that raises after joining, and a rank that
+never joins; the surviving rank must end with an error, not hang.
 """
 import os
 import socket
@@ -64,3 +66,45 @@ def test_reference_arm_skips_nonzero_ranks(monkeypatch):
         steps = 1
         gpus = 2
     assert bench.run_reference(A(), bench.Dist()) is None
+
+
+def _failing_worker(rank, world, port, q, mode):
+    os.environ.update(RANK=str(rank), WORLD_SIZE=str(world), LOCAL_RANK=str(rank),
+                      MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), HYB_PG_TIMEOUT_S="5")
+    sys.path.insert(0, ROOT)
+    import time
+    import bench
+    if rank == 1 and mode == "never_joins":
+        q.put((rank, "absent", 0.0))
+        return
+    d = bench.Dist()
+    t0 = time.monotonic()
+    try:
+        d.init("gloo")
+        if rank == 1:
+            raise RuntimeError("rank 1 fails between steps")
+        d.barrier()
+        d.max(1.0)
+        q.put((rank, "completed", time.monotonic() - t0))
+    except RuntimeError as e:
+        q.put((rank, "error" if rank == 0 else "raised", time.monotonic() - t0))
+        if rank == 1:   # leave without tearing the group down, as a crashed rank would
+            q.close()
+            q.join_thread()
+            os._exit(3)
+
+
+@pytest.mark.parametrize("mode", ["raises_after_join", "never_joins"])
+def test_surviving_rank_errors_instead_of_hanging(mode):
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_failing_worker, args=(r, 2, port, q, mode)) for r in range(2)]
+    for p in procs:
+        p.start()
+    res = dict((r, (status, t)) for r, status, t in (q.get(timeout=120) for _ in procs))
+    for p in procs:
+        p.join(timeout=60)
+    status0, t0 = res[0]
+    assert status0 == "error", res
+    assert t0 < 60.0, res

@@ -258,3 +258,25 @@ def test_full_cache_overflow_sets_flag_and_keeps_state(lib):
     assert cache.len.tolist() == [80]
     assert torch.equal(cache.k, before)
     assert lib.hyb_device_error() == 0   # cleared by the previous read
+
+
+def test_bounded_wait_times_out_and_context_stays_usable(lib):
+    """A device-side wait that nothing satisfies gives up after its limit and
+    raises the timeout bit instead of hanging; the next calls work."""
+    import time
+    lib.hyb_device_error(clear=True)
+    t0 = time.perf_counter()
+    lib.hyb_selftest_wait_timeout()
+    flags = lib.hyb_device_error(clear=True)
+    elapsed = time.perf_counter() - t0
+    assert flags == lib.DEV_ERR_TIMEOUT
+    assert 0.5 < elapsed < 30.0, elapsed
+    # the context is usable: a small prefill still matches the oracle
+    x = synth.prefill_inputs(1, 300, seed=77, device="cuda")
+    out = lib.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], x["pos"], lib.FULL)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    h = {k: x[k].float().cpu().double().numpy() for k in ("q", "k", "v", "gate")}
+    ref = O.prefill(h["q"], h["k"], h["v"], h["gate"], x["pos"].cpu().numpy(), O.FULL)
+    got = out.float().cpu().double().numpy()
+    assert np.abs(got - ref).max() <= 2e-2
