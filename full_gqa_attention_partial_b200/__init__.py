@@ -36,7 +36,7 @@ EXPORTED = (
     "hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill_workspace_size", "hyb_attn_prefill",
     "hyb_attn_decode_workspace_size", "hyb_attn_decode", "hyb_device_error", "hyb_last_error",
     "hyb_launch_count", "hyb_profile_events", "hyb_profile_pairs_used", "hyb_attn_decode_noalloc",
-    "hyb_selftest_wait_timeout",
+    "hyb_selftest_wait_timeout", "hyb_linear",
 )
 
 
@@ -92,6 +92,7 @@ def load(path: str = LIB_PATH):
     lib.hyb_profile_events.restype = ctypes.c_int
     lib.hyb_profile_pairs_used.restype = i32
     lib.hyb_selftest_wait_timeout.argtypes = [vp]
+    lib.hyb_linear.argtypes = [vp, i64, vp, i64, vp, i64, i32, i32, i32, vp]
     for name in ("hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill", "hyb_attn_decode",
                  "hyb_device_error"):
         getattr(lib, name).restype = ctypes.c_int
@@ -256,6 +257,25 @@ def hyb_device_error(clear: bool = True, stream=None) -> int:
     flags = ctypes.c_int32(0)
     _check(load().hyb_device_error(ctypes.byref(flags), 1 if clear else 0, _stream(stream)))
     return int(flags.value)
+
+
+def hyb_linear(x: torch.Tensor, w: torch.Tensor, out: torch.Tensor = None, stream=None) -> torch.Tensor:
+    """y = x @ w.T on the tensor cores: x bf16 [..., K] (unit stride along K),
+    w bf16 [N, K] (Linear weight layout); returns bf16 [..., N]."""
+    K = x.shape[-1]
+    N = w.shape[0]
+    x2 = x.reshape(-1, K)
+    if x2.stride(-1) != 1:
+        x2 = x2.contiguous()
+    if w.stride(-1) != 1:
+        w = w.contiguous()
+    M = x2.shape[0]
+    if out is None:
+        out = torch.empty(*x.shape[:-1], N, dtype=torch.bfloat16, device=x.device)
+    y2 = out.view(-1, N)
+    _check(load().hyb_linear(_ptr(x2), x2.stride(0), _ptr(w), w.stride(0), _ptr(y2), y2.stride(0), M, N, K,
+                             _stream(stream)))
+    return out
 
 
 def hyb_selftest_wait_timeout(stream=None) -> None:

@@ -98,6 +98,7 @@ hyb_status ensure_device() {
   if ((e = prefill_set_smem_attr()) != cudaSuccess) return cuda_fail(e, "prefill smem attribute");
   cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev);
   if ((e = decode_set_smem_attr()) != cudaSuccess) return cuda_fail(e, "decode smem attribute");
+  if ((e = gemm_set_smem_attr()) != cudaSuccess) return cuda_fail(e, "linear smem attribute");
   g_dev_state[dev] = 1;
   return HYB_OK;
 }
@@ -210,6 +211,48 @@ hyb_status hyb_device_error(int32_t* flags, int32_t clear, void* stream) {
     if ((e = cudaMemcpyToSymbol(g_dev_err, &zero, sizeof(int))) != cudaSuccess)
       return cuda_fail(e, "clear error word");
   }
+  return HYB_OK;
+}
+
+namespace {
+// 2-D map over a row-major bf16 matrix [rows][ld] (K = cols used), 64 x 128 boxes
+hyb_status make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint64_t cols, uint64_t ld,
+                         const char* what) {
+  auto enc = encode_fn();
+  if (!enc) return fail(HYB_EUNSUPPORTED, "cuTensorMapEncodeTiled is not available from the driver");
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {ld * 2};
+  cuuint32_t box[2] = {(cuuint32_t)gemm_box_k(), (cuuint32_t)gemm_box_rows()};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HYB_ECUDA, "cuTensorMapEncodeTiled(%s) failed with CUresult %d", what, (int)r);
+  return HYB_OK;
+}
+}  // namespace
+
+hyb_status hyb_linear(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int32_t M,
+                      int32_t N, int32_t K, void* stream) {
+  if (!x || !w || !y) return fail(HYB_EINVAL, "x, w and y must not be NULL");
+  if (M <= 0 || N <= 0 || K <= 0) return fail(HYB_ESHAPE, "M, N, K must be positive (got %d, %d, %d)", M, N, K);
+  if (N % 8 || K % 8) return fail(HYB_ESHAPE, "N and K must be multiples of 8 (got %d, %d)", N, K);
+  if (ldx < K || ldw < K || ldy < N) return fail(HYB_ESHAPE, "row strides must cover the rows (ldx, ldw >= K; ldy >= N)");
+  if (ldx % 8 || ldw % 8 || ldy % 8) return fail(HYB_EALIGN, "row strides must be multiples of 8 elements");
+  if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return fail(HYB_EALIGN, "x, w and y must be 16-byte aligned");
+  hyb_status s = ensure_device();
+  if (s != HYB_OK) return s;
+  GemmHost gh;
+  if ((s = make_rows_map(&gh.tm_x, x, (uint64_t)M, (uint64_t)K, (uint64_t)ldx, "x")) != HYB_OK) return s;
+  if ((s = make_rows_map(&gh.tm_w, w, (uint64_t)N, (uint64_t)K, (uint64_t)ldw, "w")) != HYB_OK) return s;
+  gh.y = y;
+  gh.ldy = ldy;
+  gh.M = M;
+  gh.N = N;
+  gh.K = K;
+  gh.n_pairs = device_sms() / 2;
+  cudaError_t e = launch_gemm(gh, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "linear launch");
   return HYB_OK;
 }
 

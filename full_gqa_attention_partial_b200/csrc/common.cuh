@@ -201,6 +201,16 @@ __device__ __forceinline__ void tma_load_4d_pair(uint32_t smem_dst, const void* 
       : "memory");
 }
 
+// The same for a 2-D map.
+__device__ __forceinline__ void tma_load_2d_pair(uint32_t smem_dst, const void* tmap, uint64_t* bar, int c0,
+                                                 int c1) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_dst),
+      "l"(tmap), "r"(c0), "r"(c1), "r"(mapa_cluster(smem_u32(bar), 0))
+      : "memory");
+}
+
 // ---------------------------------------------------------------------------
 // tcgen05 (5th-generation tensor cores, accumulators in tensor memory)
 // ---------------------------------------------------------------------------

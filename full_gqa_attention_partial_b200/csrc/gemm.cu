@@ -1,0 +1,219 @@
+// Linear projections around the attention core (q_k_v_proj, the head-wise
+// gate projection and o_proj of "百万 Token 塞进 4B ..." §"省显存的第二板斧"):
+//   Y[M, N] = X[M, K] W[N, K]^T   (bf16 in and out, fp32 accumulation),
+// with W in the usual [out_features, in_features] layout.
+//
+// A cluster of two CTAs owns a 256 x 256 output tile: each CTA TMA-loads its
+// 128 rows of X and 128 rows of W per 64-wide K block into a 6-stage ring
+// (128-byte swizzle), and one warp of CTA 0 issues pair MMAs
+// (tcgen05.mma.cta_group::2, M = 256, N = 256, both operands from shared
+// memory).  The accumulator (128 x 256 fp32 per CTA) is double-buffered in
+// tensor memory, so the 4 epilogue warps drain one tile (TMEM -> bf16 ->
+// per-warp 32 x 32 transpose in shared memory -> 64-byte row segments to
+// global memory) while the next tile accumulates.  Pairs are persistent and
+// walk the tiles row-band first (all column tiles of 256 rows in turn), so
+// W and the current rows of X stay in L2.
+//
+// Roles (192 threads): warps 0-3 epilogue (one TMEM lane = one output row),
+// warp 4 lane 0 TMA producer (both CTAs), warp 5 TMEM allocation and, in
+// CTA 0, the MMA loop.  Every wait is bounded.
+#include "common.cuh"
+#include "launch.h"
+
+namespace hyb {
+
+constexpr int kGM = 128;            // output rows per CTA (256 per pair)
+constexpr int kGN = 256;            // output columns per pair tile
+constexpr int kGK = 64;             // K per stage
+constexpr int kGStages = 6;
+constexpr int kGHalf = 16384;       // one CTA's 128 rows x 64 K of X, or of W
+constexpr int kGThreads = 192;
+
+struct GemmSmem {
+  uint8_t x[kGStages][kGHalf];      // 1024-byte aligned
+  uint8_t w[kGStages][kGHalf];
+  uint8_t ostage[4][2048];          // per epilogue warp: 32 rows x 32 columns (bf16)
+  uint64_t full[kGStages];          // CTA 0's count both CTAs' bytes
+  uint64_t empty[kGStages];
+  uint64_t acc_full[2];             // accumulator buffer complete (MMA commit)
+  uint64_t acc_empty[2];            // drained: one arrival per epilogue warp of the pair
+  uint64_t mma_done;
+  uint32_t tmem_base;
+};
+
+size_t gemm_smem_bytes() { return sizeof(GemmSmem) + 1024; }
+static_assert(sizeof(GemmSmem) + 1024 <= 232448, "GEMM shared memory exceeds 227 KB");
+
+struct GemmArgs {
+  __nv_bfloat16* y;
+  int64_t ldy;
+  int M, N, K;
+  int tiles_n, n_tiles;
+};
+
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, GemmArgs g) {
+  extern __shared__ uint8_t smem_raw[];
+  GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const int pair0 = blockIdx.x >> 1;
+  const int n_pairs = gridDim.x >> 1;
+  const int k_blocks = (g.K + kGK - 1) / kGK;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kGStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&sm.acc_full[b], 1);
+      mbar_init(&sm.acc_empty[b], 8);
+    }
+    mbar_init(&sm.mma_done, 1);
+    fence_barrier_init();
+  }
+  if (warp == 5) {
+    tmem_alloc_pair(&sm.tmem_base, 512);
+    tmem_relinquish_pair();
+  }
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();   // barriers of both CTAs initialised before any cross-CTA arrive
+  tc_fence_after();
+  const uint32_t tmem = sm.tmem_base;
+
+  if (warp == 4) {
+    if (lane == 0) {
+      // ======================= TMA producer (both CTAs) =======================
+      prefetch_tmap(&tm_x);
+      prefetch_tmap(&tm_w);
+      uint32_t it = 0;   // stages filled so far
+      bool ok = true;
+      for (int t = pair0; ok && t < g.n_tiles; t += n_pairs) {
+        const int mt = t / g.tiles_n, nt = t % g.tiles_n;
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % kGStages;
+          if (it >= kGStages && !(ok = mbar_wait(&sm.empty[s], ((it / kGStages) - 1) & 1))) break;
+          if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 4 * kGHalf);
+          tma_load_2d_pair(smem_u32(sm.x[s]), &tm_x, &sm.full[s], kb * kGK, mt * 2 * kGM + (int)rank * kGM);
+          tma_load_2d_pair(smem_u32(sm.w[s]), &tm_w, &sm.full[s], kb * kGK, nt * kGN + (int)rank * (kGN / 2));
+        }
+      }
+      if (rank == 0)   // every load of the pair completes on CTA 0's barriers
+        for (uint32_t i = (it > kGStages ? it - kGStages : 0); i < it; ++i)
+          mbar_wait(&sm.full[i % kGStages], (i / kGStages) & 1);
+    }
+  } else if (warp == 5) {
+    // ======================= MMA issuer (CTA 0, whole warp, one lane issues) =======================
+    if (rank == 0) {
+      constexpr uint32_t idesc = idesc_bf16(2 * kGM, kGN, false);   // both operands K-major
+      const uint64_t xdesc0 = smem_desc_sw128(smem_u32(sm.x[0]), 16, 1024);
+      const uint64_t wdesc0 = smem_desc_sw128(smem_u32(sm.w[0]), 16, 1024);
+      uint32_t it = 0, acc = 0;
+      bool ok = true;
+      for (int t = pair0; ok && t < g.n_tiles; t += n_pairs, ++acc) {
+        const uint32_t b = acc & 1;
+        if (acc >= 2 && !(ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_empty[b], ((acc >> 1) - 1) & 1)))) break;
+        tc_fence_after();
+        for (int kb = 0; kb < k_blocks; ++kb, ++it) {
+          const int s = it % kGStages;
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[s], (it / kGStages) & 1)))) break;
+          tc_fence_after();
+          const uint64_t xd = desc_advance(xdesc0, s * kGHalf), wd = desc_advance(wdesc0, s * kGHalf);
+#pragma unroll
+          for (int k = 0; k < kGK / 16; ++k)
+            mma_ss_pair_warp(tmem + b * kGN, desc_advance(xd, k * 32), desc_advance(wd, k * 32), idesc,
+                             (kb > 0 || k > 0) ? 1u : 0u);
+          mma_commit_pair_warp(&sm.empty[s]);
+        }
+        if (ok) mma_commit_pair_warp(&sm.acc_full[b]);
+      }
+      // also on an early exit: wait until nothing the pair issued is in flight
+      mma_commit_pair_warp(&sm.mma_done);
+      mbar_wait(&sm.mma_done, 0);
+    }
+  } else {
+    // ======================= epilogue (warps 0-3, both CTAs) =======================
+    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    uint8_t* stg = sm.ostage[warp];
+    const int rr = lane >> 2, ch = lane & 3;   // store phase: rows rr + 8 q, 16-byte chunk ch
+    uint32_t acc = 0;
+    bool ok = true;
+    for (int t = pair0; ok && t < g.n_tiles; t += n_pairs, ++acc) {
+      const int mt = t / g.tiles_n, nt = t % g.tiles_n;
+      const uint32_t b = acc & 1;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full[b], (acc >> 1) & 1)))) break;
+      tc_fence_after();
+      const int row0 = mt * 2 * kGM + (int)rank * kGM + warp * 32;   // this warp's first output row
+#pragma unroll 1
+      for (int c = 0; c < kGN / 32; ++c) {
+        const int col0 = nt * kGN + 32 * c;
+        uint32_t v[32];
+        tmem_ld32(trow + b * kGN + 32 * c, v);
+        tmem_wait_ld();
+        // row `lane`: 32 columns -> 4 chunks of 8 bf16, XOR-swizzled by row
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            w4[e] = pack_bf16(__uint_as_float(v[8 * q + 2 * e]), __uint_as_float(v[8 * q + 2 * e + 1]));
+          *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q ^ ((lane >> 1) & 3))) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int rw = rr + 8 * q;
+          const int row = row0 + rw, col = col0 + 8 * ch;
+          const uint4 val = *reinterpret_cast<const uint4*>(stg + rw * 64 + 16 * (ch ^ ((rw >> 1) & 3)));
+          if (row < g.M && col < g.N) *reinterpret_cast<uint4*>(g.y + (int64_t)row * g.ldy + col) = val;
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(&sm.acc_empty[b]);
+        else mbar_arrive_remote(&sm.acc_empty[b], 0);
+      }
+    }
+  }
+
+  // the peer's shared memory and tensor memory stay alive until both CTAs are done
+  tc_fence_before();
+  __syncthreads();
+  cluster_sync();
+  if (warp == 5) {
+    tc_fence_after();
+    tmem_dealloc_pair(tmem, 512);
+  }
+}
+
+int gemm_box_rows() { return kGM; }
+int gemm_box_k() { return kGK; }
+
+cudaError_t launch_gemm(const GemmHost& h, cudaStream_t st) {
+  GemmArgs g;
+  g.y = reinterpret_cast<__nv_bfloat16*>(h.y);
+  g.ldy = h.ldy;
+  g.M = h.M;
+  g.N = h.N;
+  g.K = h.K;
+  const int tiles_m = (h.M + 2 * kGM - 1) / (2 * kGM);
+  g.tiles_n = (h.N + kGN - 1) / kGN;
+  const long long n_tiles = (long long)tiles_m * g.tiles_n;
+  if (n_tiles <= 0 || n_tiles > 0x3fffffffLL) return cudaErrorInvalidValue;
+  g.n_tiles = (int)n_tiles;
+  const long long grid = 2 * (n_tiles < h.n_pairs ? n_tiles : h.n_pairs);
+  gemm_kernel<<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, g);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t gemm_set_smem_attr() {
+  return cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes());
+}
+
+}  // namespace hyb

@@ -3,4 +3,5 @@
 #include "rope_kv.cu"
 #include "decode.cu"
 #include "prefill.cu"
+#include "gemm.cu"
 #include "api.cu"

@@ -40,6 +40,19 @@ cudaError_t launch_kv_commit(int32_t* len, int32_t* head, int64_t capacity, bool
 cudaError_t launch_selftest_wait(cudaStream_t st);
 cudaError_t launch_fill_i32(int32_t* p, int64_t n, int32_t v, cudaStream_t st);
 
+// ---- linear projections (gemm.cu) -------------------------------------------
+struct GemmHost {
+  CUtensorMap tm_x, tm_w;      // 2-D maps {K, rows}, 64 x 128 boxes, 128B swizzle
+  void* y = nullptr;           // bf16 [M][ldy]
+  int64_t ldy = 0;
+  int M = 0, N = 0, K = 0;
+  int n_pairs = 74;            // persistent CTA pairs (SMs / 2)
+};
+cudaError_t launch_gemm(const GemmHost& h, cudaStream_t st);
+cudaError_t gemm_set_smem_attr();
+int gemm_box_rows();   // rows of X or W per TMA box
+int gemm_box_k();      // K elements per TMA box
+
 // ---- prefill attention (prefill.cu) -----------------------------------------
 struct PrefillHost {
   CUtensorMap tm_k, tm_v;      // 4-D maps {256, rows, 4, B}, 64-dim boxes, 128B swizzle

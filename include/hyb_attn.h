@@ -202,6 +202,21 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
 hyb_status hyb_device_error(int32_t* flags, int32_t clear, void* stream);
 
 /*
+ * Linear projection Y = X W^T, the q_k_v_proj / gate / o_proj GEMMs around the
+ * attention core ("百万 Token 塞进 4B ..." §"省显存的第二板斧": the fused
+ * q_k_v_proj output is sliced into q, k and v; the gate has one score per
+ * head; o_proj maps the 16 x 256 attention output back to the residual
+ * width).  Device pointers, caller-owned, row-major bf16:
+ *   x [M][ldx] (K used), w [N][ldw] (K used; PyTorch Linear weight layout
+ *   [out_features][in_features]), y [M][ldy] (N written).
+ * fp32 accumulation; y is rounded to bf16 once.  N, K, ldx, ldw, ldy must be
+ * multiples of 8 and the pointers 16-byte aligned (HYB_ESHAPE / HYB_EALIGN
+ * otherwise, checked before any launch).  Asynchronous on `stream`.
+ */
+hyb_status hyb_linear(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int32_t M,
+                      int32_t N, int32_t K, void* stream);
+
+/*
  * Failure-path self-test (no counterpart in the pages).  Launches one block
  * on `stream` whose first thread waits on a shared-memory barrier that
  * nothing completes.  The wait is bounded like every pipeline wait of the

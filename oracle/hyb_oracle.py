@@ -266,6 +266,15 @@ def decode_group(q_rows, k, v, q_idx, k_idx, lt, gate=None):
 
 
 # ---------------------------------------------------------------------------
+# Projections around the attention core
+# ---------------------------------------------------------------------------
+def linear(x, w):
+    """y = x W^T with W in the [out_features, in_features] layout of the
+    q_k_v_proj / gate / o_proj weights ([TEARDOWN] §"省显存的第二板斧")."""
+    return np.asarray(x, dtype=np.float64) @ np.asarray(w, dtype=np.float64).T
+
+
+# ---------------------------------------------------------------------------
 # KV caches: linear (full layers) and the 512-slot ring (sliding layers)
 # ---------------------------------------------------------------------------
 def linear_slots(length: int, n_new: int) -> np.ndarray:

@@ -353,3 +353,16 @@ def test_decode_group_equals_gqa_attention(lt):
         hs = slice(O.GROUP * kvh, O.GROUP * (kvh + 1))
         got = O.decode_group(q[0, hs], k[:, kvh], v[:, kvh], L - 1, idx, lt, g[0, hs])
         np.testing.assert_allclose(got, ref[hs], rtol=1e-12, atol=1e-12)
+
+
+def test_linear_matches_scalar_loops():
+    """y[m, n] = sum_k x[m, k] w[n, k], written as explicit loops."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((3, 7))
+    w = rng.standard_normal((5, 7))
+    ref = np.zeros((3, 5))
+    for m in range(3):
+        for n in range(5):
+            for k in range(7):
+                ref[m, n] += x[m, k] * w[n, k]
+    np.testing.assert_allclose(O.linear(x, w), ref, rtol=1e-13, atol=1e-13)
