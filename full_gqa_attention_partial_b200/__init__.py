@@ -36,7 +36,7 @@ EXPORTED = (
     "hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill_workspace_size", "hyb_attn_prefill",
     "hyb_attn_decode_workspace_size", "hyb_attn_decode", "hyb_device_error", "hyb_last_error",
     "hyb_launch_count", "hyb_profile_events", "hyb_profile_pairs_used", "hyb_attn_decode_noalloc",
-    "hyb_selftest_wait_timeout", "hyb_linear",
+    "hyb_selftest_wait_timeout", "hyb_linear", "hyb_attn_layer_prefill_workspace_size", "hyb_attn_layer_prefill",
 )
 
 
@@ -93,6 +93,9 @@ def load(path: str = LIB_PATH):
     lib.hyb_profile_pairs_used.restype = i32
     lib.hyb_selftest_wait_timeout.argtypes = [vp]
     lib.hyb_linear.argtypes = [vp, i64, vp, i64, vp, i64, i32, i32, i32, vp]
+    lib.hyb_attn_layer_prefill_workspace_size.argtypes = [i32, i32, i32, i32]
+    lib.hyb_attn_layer_prefill_workspace_size.restype = sz
+    lib.hyb_attn_layer_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, pc, vp, sz, vp]
     for name in ("hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill", "hyb_attn_decode",
                  "hyb_device_error"):
         getattr(lib, name).restype = ctypes.c_int
@@ -211,6 +214,40 @@ def hyb_attn_prefill(q, k, v, gate, pos, layer_type: int, out=None, cache: KVCac
     _check(load().hyb_attn_prefill(_ptr(q), _ptr(k), _ptr(v), _ptr(gate), _ptr(pos), layer_type, B, T, qs, ks,
                                    _ptr(out), None if cache is None else cache.ref, _ptr(workspace), wsz,
                                    _stream(stream)))
+    return out
+
+
+HIDDEN = 2560
+
+
+def hyb_attn_layer_prefill_workspace_size(layer_type: int, B: int, T: int, with_cache: bool) -> int:
+    return int(load().hyb_attn_layer_prefill_workspace_size(layer_type, B, T, 1 if with_cache else 0))
+
+
+def hyb_attn_layer_prefill(hidden, w_qkv, w_gate, w_o, pos, layer_type: int, out=None,
+                           cache: KVCache | None = None, workspace=None, stream=None):
+    """One attention layer for prefill: q_k_v_proj, gate projection, attention,
+    o_proj.  hidden bf16 [B,T,2560] contiguous; w_qkv [6144,2560], w_gate
+    [16,2560] or None, w_o [2560,4096] (Linear weight layout); pos [B,T] int32
+    or None.  Returns out bf16 [B,T,2560]."""
+    if hidden.dtype != torch.bfloat16 or not hidden.is_contiguous() or hidden.shape[-1] != HIDDEN:
+        raise ValueError("hidden must be contiguous bf16 [B, T, 2560]")
+    for name, w, shape in (("w_qkv", w_qkv, (6144, HIDDEN)), ("w_o", w_o, (HIDDEN, N_Q_HEADS * HEAD_DIM)),
+                           ("w_gate", w_gate, (N_Q_HEADS, HIDDEN))):
+        if w is not None and (w.dtype != torch.bfloat16 or not w.is_contiguous() or tuple(w.shape) != shape):
+            raise ValueError(f"{name} must be contiguous bf16 {list(shape)}")
+    B, T = hidden.shape[:2]
+    if pos is not None and (pos.dtype != torch.int32 or not pos.is_contiguous() or tuple(pos.shape) != (B, T)):
+        raise ValueError("pos must be contiguous int32 [B, T]")
+    if out is None:
+        out = torch.empty(B, T, HIDDEN, dtype=torch.bfloat16, device=hidden.device)
+    need = hyb_attn_layer_prefill_workspace_size(layer_type, B, T, cache is not None)
+    if workspace is None:
+        workspace = alloc_workspace(need, hidden.device)
+    wsz = workspace.numel() * workspace.element_size()
+    _check(load().hyb_attn_layer_prefill(_ptr(hidden), _ptr(w_qkv), _ptr(w_gate), _ptr(w_o), _ptr(pos), layer_type,
+                                         B, T, _ptr(out), None if cache is None else cache.ref, _ptr(workspace), wsz,
+                                         _stream(stream)))
     return out
 
 

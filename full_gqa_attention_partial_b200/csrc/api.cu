@@ -574,3 +574,54 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Whole attention layer: q_k_v_proj + gate projection, the attention core,
+// o_proj ("百万 Token 塞进 4B ..." §"省显存的第二板斧").
+// ---------------------------------------------------------------------------
+namespace {
+constexpr int64_t kHidden = 2560;                        // residual width (hidden_size)
+constexpr int64_t kQkv = (int64_t)(kHq + 2 * kHkv) * kD;   // 6144: fused q | k | v row
+size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
+}  // namespace
+
+size_t hyb_attn_layer_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache) {
+  if (B <= 0 || T <= 0) return 0;
+  const size_t n = (size_t)B * (size_t)T;
+  return round256(n * kQkv * 2) + round256(n * kHq * 2) + round256(n * kHq * kD * 2) +
+         hyb_attn_prefill_workspace_size(layer_type, B, T, with_cache);
+}
+
+hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const void* w_gate, const void* w_o,
+                                  const int32_t* pos, int32_t layer_type, int32_t B, int32_t T, void* out,
+                                  const hyb_kv_cache* cache, void* workspace, size_t workspace_bytes,
+                                  void* stream) {
+  if (!hidden || !w_qkv || !w_o || !out) return fail(HYB_EINVAL, "hidden, w_qkv, w_o and out must be non-NULL");
+  if (layer_type != HYB_SLIDING && layer_type != HYB_FULL) return fail(HYB_EINVAL, "layer_type %d invalid", layer_type);
+  if (B <= 0 || T <= 0) return fail(HYB_EINVAL, "B = %d and T = %d must be positive", B, T);
+  if ((int64_t)B * T > 0x7fffffffLL) return fail(HYB_ESHAPE, "B * T = %lld tokens is too many", (long long)B * T);
+  const size_t need = hyb_attn_layer_prefill_workspace_size(layer_type, B, T, cache != nullptr);
+  if (workspace_bytes < need) return fail(HYB_EOVERFLOW, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(HYB_EALIGN, "workspace must be non-NULL and 256-byte aligned");
+  const int32_t M = B * T;
+  const size_t n = (size_t)M;
+  uint8_t* p = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* qkv = reinterpret_cast<__nv_bfloat16*>(p);
+  p += round256(n * kQkv * 2);
+  __nv_bfloat16* gate = reinterpret_cast<__nv_bfloat16*>(p);
+  p += round256(n * kHq * 2);
+  __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(p);
+  p += round256(n * kHq * kD * 2);
+  const size_t attn_ws = hyb_attn_prefill_workspace_size(layer_type, B, T, cache != nullptr);
+  hyb_status s = hyb_linear(hidden, kHidden, w_qkv, kHidden, qkv, kQkv, M, (int32_t)kQkv, (int32_t)kHidden, stream);
+  if (s != HYB_OK) return s;
+  if (w_gate && (s = hyb_linear(hidden, kHidden, w_gate, kHidden, gate, kHq, M, kHq, (int32_t)kHidden, stream)) !=
+                    HYB_OK)
+    return s;
+  s = hyb_attn_prefill(qkv, qkv + (int64_t)kHq * kD, qkv + (int64_t)(kHq + kHkv) * kD, w_gate ? gate : nullptr, pos,
+                       layer_type, B, T, kQkv, kQkv, attn, cache, attn_ws ? p : nullptr, attn_ws, stream);
+  if (s != HYB_OK) return s;
+  return hyb_linear(attn, (int64_t)kHq * kD, w_o, (int64_t)kHq * kD, out, kHidden, M, (int32_t)kHidden,
+                    (int32_t)(kHq * kD), stream);
+}

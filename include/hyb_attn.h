@@ -217,6 +217,29 @@ hyb_status hyb_linear(const void* x, int64_t ldx, const void* w, int64_t ldw, vo
                       int32_t N, int32_t K, void* stream);
 
 /*
+ * One whole attention layer of the model for prefill ("百万 Token 塞进 4B ..."
+ * §"省显存的第二板斧"): the fused q_k_v_proj, the head-wise gate projection,
+ * the attention core of hyb_attn_prefill (RoPE, masked GQA, sigmoid gate,
+ * cache update) and o_proj.
+ *   hidden : bf16 [B][T][2560] contiguous (the layer's input, hidden_size 2560).
+ *   w_qkv  : bf16 [6144][2560], rows q (4096) | k (1024) | v (1024).
+ *   w_gate : bf16 [16][2560], one gate score per head, or NULL (no gate).
+ *   w_o    : bf16 [2560][4096].
+ *   pos, layer_type, B, T, cache: as hyb_attn_prefill.
+ *   out    : bf16 [B][T][2560].
+ *   workspace: at least hyb_attn_layer_prefill_workspace_size(layer_type, B,
+ *          T, cache != NULL) bytes, 256-byte aligned; it holds the fused
+ *          q|k|v rows, the gate scores and the attention output (bf16, as
+ *          the model's tensors are) between the steps.
+ * Errors: as hyb_linear and hyb_attn_prefill.
+ */
+size_t hyb_attn_layer_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache);
+hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const void* w_gate, const void* w_o,
+                                  const int32_t* pos, int32_t layer_type, int32_t B, int32_t T, void* out,
+                                  const hyb_kv_cache* cache, void* workspace, size_t workspace_bytes,
+                                  void* stream);
+
+/*
  * Failure-path self-test (no counterpart in the pages).  Launches one block
  * on `stream` whose first thread waits on a shared-memory barrier that
  * nothing completes.  The wait is bounded like every pipeline wait of the

@@ -274,6 +274,32 @@ def linear(x, w):
     return np.asarray(x, dtype=np.float64) @ np.asarray(w, dtype=np.float64).T
 
 
+def to_bf16(x):
+    """Round to bfloat16 (round to nearest even) and back to float64: the
+    model's activations between the projections and the attention are bf16
+    tensors ([CONFIG] §"模型身份与硬件画像": dtype bfloat16)."""
+    import torch
+    return torch.from_numpy(np.asarray(x, dtype=np.float64)).to(torch.bfloat16).to(torch.float64).numpy()
+
+
+def attention_layer(hidden, w_qkv, w_gate, w_o, pos, lt, rows=None):
+    """One attention layer for prefill ([TEARDOWN] §"省显存的第二板斧"):
+    qkv = hidden W_qkv^T, sliced q | k | v; gate = hidden W_g^T; the attention
+    of prefill() on them; out = attention(rows) W_o^T.  The three intermediate
+    tensors are rounded to bf16, as the model's tensors are.
+    hidden [B, T, 2560]; w_qkv [6144, 2560]; w_gate [16, 2560] or None;
+    w_o [2560, 4096].  Returns [B, len(rows), 2560] float64."""
+    hidden = np.asarray(hidden, dtype=np.float64)
+    B, T = hidden.shape[:2]
+    qkv = to_bf16(linear(hidden, w_qkv))
+    q = qkv[..., :N_Q_HEADS * HEAD_DIM].reshape(B, T, N_Q_HEADS, HEAD_DIM)
+    k = qkv[..., N_Q_HEADS * HEAD_DIM:(N_Q_HEADS + N_KV_HEADS) * HEAD_DIM].reshape(B, T, N_KV_HEADS, HEAD_DIM)
+    v = qkv[..., (N_Q_HEADS + N_KV_HEADS) * HEAD_DIM:].reshape(B, T, N_KV_HEADS, HEAD_DIM)
+    gate = None if w_gate is None else to_bf16(linear(hidden, w_gate))
+    o = to_bf16(prefill(q, k, v, gate, pos, lt, rows=rows))
+    return linear(o.reshape(B, o.shape[1], N_Q_HEADS * HEAD_DIM), w_o)
+
+
 # ---------------------------------------------------------------------------
 # KV caches: linear (full layers) and the 512-slot ring (sliding layers)
 # ---------------------------------------------------------------------------

@@ -1,0 +1,97 @@
+"""A whole attention layer (q_k_v_proj + gate projection -> attention core ->
+o_proj) against the oracle's attention_layer, which rounds the three
+intermediate tensors to bf16 as the model does; synthetic weights
+N(0, 1/fan_in), hidden states N(0, 1)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+
+pytestmark = pytest.mark.gpu
+
+MAX_ABS = 2e-2
+REL_L2 = 5e-3
+
+
+def f64(t):
+    return t.detach().float().cpu().double().numpy()
+
+
+def weights(seed, gate=True):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    w_qkv = (torch.randn(6144, 2560, generator=g, device="cuda") / 2560 ** 0.5).to(torch.bfloat16)
+    w_gate = (torch.randn(16, 2560, generator=g, device="cuda") / 2560 ** 0.5).to(torch.bfloat16) if gate else None
+    w_o = (torch.randn(2560, 4096, generator=g, device="cuda") / 4096 ** 0.5).to(torch.bfloat16)
+    return w_qkv, w_gate, w_o
+
+
+def hidden_states(B, T, seed):
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    return torch.randn(B, T, 2560, generator=g, device="cuda").to(torch.bfloat16)
+
+
+def check(got, ref, what):
+    got = f64(got)
+    assert np.all(np.isfinite(got)), what
+    max_abs = float(np.abs(got - ref).max())
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    assert max_abs <= MAX_ABS and rel <= REL_L2, f"{what}: max_abs {max_abs:.3e} rel_l2 {rel:.3e}"
+
+
+def oracle(h, w_qkv, w_gate, w_o, pos, lt, rows=None):
+    return O.attention_layer(f64(h), f64(w_qkv), None if w_gate is None else f64(w_gate), f64(w_o),
+                             pos.cpu().numpy(), lt, rows=rows)
+
+
+@pytest.mark.parametrize("lt", [O.SLIDING, O.FULL])
+@pytest.mark.parametrize("gate", [True, False])
+def test_layer_prefill_small(lib, lt, gate):
+    B, T = 2, 300
+    h = hidden_states(B, T, seed=1 + lt)
+    w_qkv, w_gate, w_o = weights(10 + lt, gate)
+    pos = torch.arange(T, dtype=torch.int32, device="cuda").repeat(B, 1).contiguous()
+    out = lib.hyb_attn_layer_prefill(h, w_qkv, w_gate, w_o, pos, lt)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    check(out, oracle(h, w_qkv, w_gate, w_o, pos, lt), f"layer B={B} T={T} type {lt} gate {gate}")
+
+
+@pytest.mark.parametrize("lt", [O.SLIDING, O.FULL])
+def test_layer_prefill_into_cache_then_chunk(lib, lt):
+    """Two chunks through a cache: the second chunk's rows see the first's keys."""
+    T1, T2 = 700, 260
+    h = hidden_states(1, T1 + T2, seed=5 + lt)
+    w_qkv, w_gate, w_o = weights(20 + lt)
+    cache = lib.KVCache(lt, 1, capacity=T1 + T2) if lt == O.FULL else lib.KVCache(lt, 1)
+    pos = torch.arange(T1 + T2, dtype=torch.int32, device="cuda")[None].contiguous()
+    out1 = lib.hyb_attn_layer_prefill(h[:, :T1].contiguous(), w_qkv, w_gate, w_o, pos[:, :T1].contiguous(), lt,
+                                      cache=cache)
+    out2 = lib.hyb_attn_layer_prefill(h[:, T1:].contiguous(), w_qkv, w_gate, w_o, pos[:, T1:].contiguous(), lt,
+                                      cache=cache)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    ref = oracle(h, w_qkv, w_gate, w_o, pos, lt)      # one shot over both chunks
+    check(out1, ref[:, :T1], f"layer chunk 1 type {lt}")
+    check(out2, ref[:, T1:], f"layer chunk 2 type {lt}")
+
+
+@pytest.mark.parametrize("lt", [O.SLIDING, O.FULL])
+def test_layer_prefill_T8192_sampled(lib, lt):
+    T = 8192
+    h = hidden_states(1, T, seed=30 + lt)
+    w_qkv, w_gate, w_o = weights(40 + lt)
+    pos = torch.arange(T, dtype=torch.int32, device="cuda")[None].contiguous()
+    out = lib.hyb_attn_layer_prefill(h, w_qkv, w_gate, w_o, pos, lt)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    rng = np.random.default_rng(lt)
+    rows = np.unique(np.concatenate([np.arange(0, 140), np.arange(T - 140, T), rng.choice(T, 200, replace=False)]))
+    check(out[:, rows], oracle(h, w_qkv, w_gate, w_o, pos, lt, rows=rows), f"layer T={T} type {lt}")
+
+
+def test_layer_rejects_bad_weight_shape(lib):
+    h = hidden_states(1, 8, seed=0)
+    w_qkv, w_gate, w_o = weights(0)
+    with pytest.raises(ValueError):
+        lib.hyb_attn_layer_prefill(h, w_qkv[:, :2048].contiguous(), w_gate, w_o, None, O.FULL)

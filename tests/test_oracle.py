@@ -366,3 +366,36 @@ def test_linear_matches_scalar_loops():
             for k in range(7):
                 ref[m, n] += x[m, k] * w[n, k]
     np.testing.assert_allclose(O.linear(x, w), ref, rtol=1e-13, atol=1e-13)
+
+
+def test_attention_layer_slices_q_k_v_from_the_fused_projection():
+    """With one-hot hidden states, column t of W_qkv is token t's fused
+    q | k | v row and column t of W_g its gate scores, so the layer must equal
+    the attention of exactly those q, k, v, g, followed by o_proj.  A swapped
+    slice or a missing transpose fails."""
+    rng = np.random.default_rng(9)
+    B, T, Hd = 1, 6, 2560
+    hidden = np.zeros((B, T, Hd))
+    hidden[0, np.arange(T), np.arange(T)] = 1.0
+    q = O.to_bf16(rng.standard_normal((B, T, 16, 256)))
+    k = O.to_bf16(rng.standard_normal((B, T, 4, 256)))
+    v = O.to_bf16(rng.standard_normal((B, T, 4, 256)))
+    g = O.to_bf16(rng.standard_normal((B, T, 16)))
+    w_qkv = np.zeros((6144, Hd))
+    w_qkv[:, :T] = np.concatenate([q[0].reshape(T, -1), k[0].reshape(T, -1), v[0].reshape(T, -1)], axis=1).T
+    w_gate = np.zeros((16, Hd))
+    w_gate[:, :T] = g[0].T
+    w_o = rng.standard_normal((Hd, 4096)) / 64.0
+    pos = np.arange(T)[None]
+    for lt in (O.SLIDING, O.FULL):
+        got = O.attention_layer(hidden, w_qkv, w_gate, w_o, pos, lt)
+        att = O.to_bf16(O.prefill(q, k, v, g, pos, lt)).reshape(B, T, 4096)
+        np.testing.assert_allclose(got, att @ w_o.T, rtol=1e-12, atol=1e-12)
+
+
+def test_to_bf16_rounds_to_nearest_even():
+    x = np.array([1.0, 1.0 + 2 ** -8, 1.0 + 3 * 2 ** -9, 1.0 + 2 ** -9, -2.5, 3.0e38])
+    got = O.to_bf16(x)
+    # bf16 keeps 8 significant bits: ulp(1) = 2^-7; halfway cases go to even
+    np.testing.assert_array_equal(got[:5], [1.0, 1.0, 1.0 + 2 ** -7, 1.0, -2.5])
+    assert np.isfinite(got[5]) and abs(got[5] / 3.0e38 - 1) < 2 ** -8
