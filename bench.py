@@ -17,6 +17,7 @@ The JSON line also carries:
                 512-slot ring (head at a random offset): KV GB/s, % of HBM,
                 tokens/s;
   prefill_128k  one full layer, 131072 tokens: TFLOP/s and % of peak;
+  layer_prefill the 4-layer group as whole layers (projections + attention);
   decode_1m     (--decode-1m) 36-layer decode at 1M tokens: tokens/s;
   chunked_prefill (--chunked) 262144 tokens in 8192-token chunks, 36 layers;
   cpu_baseline  the fp64 oracle on a bounded sample of the same workload.
@@ -69,15 +70,15 @@ def layer_seed(base: int, i: int) -> int:
 # the capture's summary).  Reported as roofline.traffic only while the sources are
 # unchanged; otherwise null.
 TRAFFIC = {
-    "prefill_full_T32768": {"bytes": 2.173e9, "sha": "5f20a5427468bc15",
+    "prefill_full_T32768": {"bytes": 2.173e9, "sha": "e1af5fc5ed4c8197",
                             "sources": ["prefill.cu", "common.cuh"],
                             "capture": "profiles/prefill_kernel_full_T32768.md"},
-    "prefill_sliding_T32768": {"bytes": 0.6386e9, "sha": "5f20a5427468bc15",
+    "prefill_sliding_T32768": {"bytes": 0.6386e9, "sha": "e1af5fc5ed4c8197",
                                "sources": ["prefill.cu", "common.cuh"],
                                "capture": "profiles/prefill_kernel_sliding_T32768.md"},
     # captured at 16 x 32768 tokens (2.153 GB); decode streams each cached byte
     # once, so traffic scales with the tokens: x 8590491648 / 2147483648
-    "decode_full_B16_L131072": {"bytes": 2.153e9 * 8590491648 / 2147483648, "sha": "bba9668dc1aff40b",
+    "decode_full_B16_L131072": {"bytes": 2.153e9 * 8590491648 / 2147483648, "sha": "724f44ab245c48aa",
                                 "sources": ["decode.cu", "common.cuh"],
                                 "capture": "profiles/decode_split_kernel_full_B16_L32768.md"},
 }
@@ -374,6 +375,45 @@ def bench_prefill_128k(hyb, args, peaks):
             "kernel_ms": k_ms, "call_ms": call_ms, "kernel_tflops": f / (k_ms / 1e3) / 1e12,
             "call_tflops": f / (call_ms / 1e3) / 1e12, "frac_of_peak": f / (k_ms / 1e3) / 1e12 / peak,
             "peak": peak, "peak_source": f"{peaks['source']} bf16 burst", "launches": n}
+
+
+def bench_layer(hyb, args, peaks):
+    """The 3-sliding + 1-full group as whole layers (projections included),
+    T=32768, into fresh caches: hyb_attn_layer_prefill per layer."""
+    T = T_MAIN
+    hidden = make_layer_inputs(T, layer_seed(1, 0))["qkv"][..., :2560].contiguous()
+    g = torch.Generator(device="cuda").manual_seed(77)
+    w = [((torch.randn(6144, 2560, generator=g, device="cuda") / 2560 ** 0.5).to(torch.bfloat16),
+          (torch.randn(16, 2560, generator=g, device="cuda") / 2560 ** 0.5).to(torch.bfloat16),
+          (torch.randn(2560, 4096, generator=g, device="cuda") / 4096 ** 0.5).to(torch.bfloat16))
+         for _ in GROUP_LAYERS]
+    out = torch.empty(1, T, 2560, dtype=torch.bfloat16, device="cuda")
+    ws = hyb.alloc_workspace(max(hyb.hyb_attn_layer_prefill_workspace_size(lt, 1, T, True) for lt in GROUP_LAYERS))
+    n = 3
+    caches = [[hyb.KVCache(lt, 1, capacity=T) for lt in GROUP_LAYERS] for _ in range(n + 1)]
+
+    def step(i):
+        for li, lt in enumerate(GROUP_LAYERS):
+            hyb.hyb_attn_layer_prefill(hidden, *w[li], None, lt, out=out, cache=caches[i][li], workspace=ws)
+
+    step(0)
+    torch.cuda.synchronize()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record()
+    for i in range(n):
+        step(1 + i)
+    ev1.record()
+    torch.cuda.synchronize()
+    assert hyb.hyb_device_error() == 0
+    ms = ev0.elapsed_time(ev1) / n
+    attn = sum(flops(T, lt) for lt in GROUP_LAYERS)
+    proj = len(GROUP_LAYERS) * 2 * T * 2560 * (6144 + 16 + 4096)
+    return {"workload": "3 sliding + 1 full attention layers with q_k_v_proj, gate and o_proj (synthetic weights "
+                        "N(0, 1/fan_in)), batch 1, seq 32768, into fresh caches",
+            "ms_per_step": ms, "tflop_per_step": (attn + proj) / 1e12, "projection_tflop": proj / 1e12,
+            "tflops": (attn + proj) / (ms / 1e3) / 1e12,
+            "frac_of_peak": (attn + proj) / (ms / 1e3) / 1e12 / peaks["bf16_tflops"],
+            "peak_source": f"{peaks['source']} bf16 burst"}
 
 
 def fill_full_cache(hyb, B: int, L: int, cap: int, seed: int):
@@ -704,6 +744,7 @@ def main():
     extras = {}
     if dist.world == 1 and not args.no_extras:
         extras["prefill_128k"] = bench_prefill_128k(hyb, args, peaks)
+        extras["layer_prefill"] = bench_layer(hyb, args, peaks)
         extras["decode"] = bench_decode(hyb, args, peaks)
         if args.decode_1m:
             extras["decode_1m"] = bench_decode_1m(hyb, args, peaks)
