@@ -230,10 +230,12 @@ hyb_status make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint64
   if (r != CUDA_SUCCESS) return fail(HYB_ECUDA, "cuTensorMapEncodeTiled(%s) failed with CUresult %d", what, (int)r);
   return HYB_OK;
 }
-}  // namespace
 
-hyb_status hyb_linear(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int32_t M,
-                      int32_t N, int32_t K, void* stream) {
+// rope: 0 none; 1 / 2 rotate the 256-wide column tiles below rope_cols as a
+// sliding / full layer's heads (see GemmHost)
+hyb_status linear_impl(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int32_t M,
+                       int32_t N, int32_t K, void* stream, int rope = 0, int rope_cols = 0, int32_t T = 0,
+                       const int32_t* pos = nullptr, const int32_t* len = nullptr) {
   if (!x || !w || !y) return fail(HYB_EINVAL, "x, w and y must not be NULL");
   if (M <= 0 || N <= 0 || K <= 0) return fail(HYB_ESHAPE, "M, N, K must be positive (got %d, %d, %d)", M, N, K);
   if (N % 8 || K % 8) return fail(HYB_ESHAPE, "N and K must be multiples of 8 (got %d, %d)", N, K);
@@ -251,9 +253,20 @@ hyb_status hyb_linear(const void* x, int64_t ldx, const void* w, int64_t ldw, vo
   gh.N = N;
   gh.K = K;
   gh.n_pairs = device_sms() / 2;
+  gh.rope = rope;
+  gh.rope_cols = rope_cols;
+  gh.T = T;
+  gh.pos = pos;
+  gh.len = len;
   cudaError_t e = launch_gemm(gh, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "linear launch");
   return HYB_OK;
+}
+}  // namespace
+
+hyb_status hyb_linear(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int32_t M,
+                      int32_t N, int32_t K, void* stream) {
+  return linear_impl(x, ldx, w, ldw, y, ldy, M, N, K, stream);
 }
 
 hyb_status hyb_selftest_wait_timeout(void* stream) {
@@ -338,10 +351,13 @@ size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T,
   return 2 * (size_t)B * ctx_rows(T) * row;                              // context K and V
 }
 
-hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const void* gate, const int32_t* pos,
-                            int32_t layer_type, int32_t B, int32_t T, int64_t q_row_stride,
-                            int64_t kv_row_stride, void* out, const hyb_kv_cache* cache, void* workspace,
-                            size_t workspace_bytes, void* stream) {
+namespace {
+// qk_rotated: q and k arrive rotated (the whole-layer path rotates them in the
+// q_k_v_proj epilogue); the attention kernel and the K store then skip RoPE.
+hyb_status prefill_impl(const void* q, const void* k, const void* v, const void* gate, const int32_t* pos,
+                        int32_t layer_type, int32_t B, int32_t T, int64_t q_row_stride, int64_t kv_row_stride,
+                        void* out, const hyb_kv_cache* cache, void* workspace, size_t workspace_bytes, void* stream,
+                        bool qk_rotated) {
   if (!q || !k || !v || !out) return fail(HYB_EINVAL, "q, k, v and out must be non-NULL");
   if (layer_type != HYB_SLIDING && layer_type != HYB_FULL) return fail(HYB_EINVAL, "layer_type %d invalid", layer_type);
   if (B <= 0 || T <= 0) return fail(HYB_EINVAL, "B = %d and T = %d must be positive", B, T);
@@ -390,6 +406,7 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
   // per two SMs); full layers: long items of unequal length -> one item per
   // pair, handed out longest first by the hardware block scheduler.
   ph.n_pairs = full ? (1 << 29) : device_sms() / 2;
+  ph.q_rotated = qk_rotated ? 1 : 0;
   cudaError_t e;
 
   RopeStoreHost r;  // new tokens, token-major input rows
@@ -400,6 +417,7 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
   r.pos = pos;
   r.B = B;
   r.T = T;
+  r.src_rotated = qk_rotated ? 1 : 0;
 
   if (!cache) {
     // rotated K into the workspace [B][4][T][256]; V is read in place
@@ -483,6 +501,15 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
   if ((e = launch_kv_commit(cache->len, cache->head, cache->capacity, true, B, T, st)) != cudaSuccess)
     return cuda_fail(e, "commit launch");
   return HYB_OK;
+}
+}  // namespace
+
+hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const void* gate, const int32_t* pos,
+                            int32_t layer_type, int32_t B, int32_t T, int64_t q_row_stride,
+                            int64_t kv_row_stride, void* out, const hyb_kv_cache* cache, void* workspace,
+                            size_t workspace_bytes, void* stream) {
+  return prefill_impl(q, k, v, gate, pos, layer_type, B, T, q_row_stride, kv_row_stride, out, cache, workspace,
+                      workspace_bytes, stream, false);
 }
 
 size_t hyb_attn_decode_workspace_size(int32_t layer_type, int32_t B, int64_t max_len) {
@@ -614,13 +641,17 @@ hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const v
   __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(p);
   p += round256(n * kHq * kD * 2);
   const size_t attn_ws = hyb_attn_prefill_workspace_size(layer_type, B, T, cache != nullptr);
-  hyb_status s = hyb_linear(hidden, kHidden, w_qkv, kHidden, qkv, kQkv, M, (int32_t)kQkv, (int32_t)kHidden, stream);
+  // q_k_v_proj with RoPE of the q and k heads in the epilogue (positions as
+  // hyb_attn_prefill: pos, else the cache length + t, else t)
+  const int32_t* len = cache ? cache->len : nullptr;
+  hyb_status s = linear_impl(hidden, kHidden, w_qkv, kHidden, qkv, kQkv, M, (int32_t)kQkv, (int32_t)kHidden, stream,
+                             layer_type == HYB_FULL ? 2 : 1, (kHq + kHkv) * kD, T, pos, len);
   if (s != HYB_OK) return s;
   if (w_gate && (s = hyb_linear(hidden, kHidden, w_gate, kHidden, gate, kHq, M, kHq, (int32_t)kHidden, stream)) !=
                     HYB_OK)
     return s;
-  s = hyb_attn_prefill(qkv, qkv + (int64_t)kHq * kD, qkv + (int64_t)(kHq + kHkv) * kD, w_gate ? gate : nullptr, pos,
-                       layer_type, B, T, kQkv, kQkv, attn, cache, attn_ws ? p : nullptr, attn_ws, stream);
+  s = prefill_impl(qkv, qkv + (int64_t)kHq * kD, qkv + (int64_t)(kHq + kHkv) * kD, w_gate ? gate : nullptr, pos,
+                   layer_type, B, T, kQkv, kQkv, attn, cache, attn_ws ? p : nullptr, attn_ws, stream, true);
   if (s != HYB_OK) return s;
   return hyb_linear(attn, (int64_t)kHq * kD, w_o, (int64_t)kHq * kD, out, kHidden, M, (int32_t)kHidden,
                     (int32_t)(kHq * kD), stream);

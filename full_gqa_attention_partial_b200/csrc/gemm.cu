@@ -17,6 +17,12 @@
 // Roles (192 threads): warps 0-3 epilogue (one TMEM lane = one output row),
 // warp 4 lane 0 TMA producer (both CTAs), warp 5 TMEM allocation and, in
 // CTA 0, the MMA loop.  Every wait is bounded.
+//
+// Optional RoPE epilogue (ROPE = 1 sliding layer, theta 1e4 over all 256
+// dims; ROPE = 2 full layer, theta 5e6 over the first 64 dims; rotate-half,
+// as in the attention core): for q_k_v_proj, output column tiles below
+// rope_cols are 256-wide heads (q and k), rotated in fp32 from the
+// accumulator at the row's position before the single rounding to bf16.
 #include "common.cuh"
 #include "launch.h"
 
@@ -38,6 +44,7 @@ struct GemmSmem {
   uint64_t acc_full[2];             // accumulator buffer complete (MMA commit)
   uint64_t acc_empty[2];            // drained: one arrival per epilogue warp of the pair
   uint64_t mma_done;
+  double inv_freq[128];             // RoPE frequencies of the layer type
   uint32_t tmem_base;
 };
 
@@ -49,8 +56,38 @@ struct GemmArgs {
   int64_t ldy;
   int M, N, K;
   int tiles_n, n_tiles;
+  // RoPE epilogue: row m is token m % T of sequence m / T, at position
+  // pos[m] if pos, else (len ? len[m / T] : 0) + m % T
+  int rope_cols, T;
+  const int32_t* pos;
+  const int32_t* len;
 };
 
+// Stores 32 columns (col0 ..) of this thread's row through the warp's staging
+// area: each thread writes its row (16-byte chunks XOR-swizzled by row), then
+// each store instruction covers 8 rows x 64 bytes.
+__device__ __forceinline__ void store_cols32(const float (&v)[32], uint8_t* stg, int lane, int row0, int col0,
+                                             const GemmArgs& g) {
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint32_t w4[4];
+#pragma unroll
+    for (int e = 0; e < 4; ++e) w4[e] = pack_bf16(v[8 * q + 2 * e], v[8 * q + 2 * e + 1]);
+    *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q ^ ((lane >> 1) & 3))) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+  }
+  __syncwarp();
+  const int rr = lane >> 2, ch = lane & 3;   // rows rr + 8 q, 16-byte chunk ch
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    const int rw = rr + 8 * q;
+    const int row = row0 + rw, col = col0 + 8 * ch;
+    const uint4 val = *reinterpret_cast<const uint4*>(stg + rw * 64 + 16 * (ch ^ ((rw >> 1) & 3)));
+    if (row < g.M && col < g.N) *reinterpret_cast<uint4*>(g.y + (int64_t)row * g.ldy + col) = val;
+  }
+  __syncwarp();
+}
+
+template <int ROPE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
@@ -73,6 +110,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     mbar_init(&sm.mma_done, 1);
     fence_barrier_init();
   }
+  constexpr int R = ROPE == 1 ? 256 : 64;   // rotary dims of the layer type
+  if (ROPE && threadIdx.x < R / 2) sm.inv_freq[threadIdx.x] = rope_inv_freq(ROPE == 1 ? 1.0e4 : 5.0e6, threadIdx.x, R);
   if (warp == 5) {
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
@@ -137,7 +176,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     // ======================= epilogue (warps 0-3, both CTAs) =======================
     const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
     uint8_t* stg = sm.ostage[warp];
-    const int rr = lane >> 2, ch = lane & 3;   // store phase: rows rr + 8 q, 16-byte chunk ch
     uint32_t acc = 0;
     bool ok = true;
     for (int t = pair0; ok && t < g.n_tiles; t += n_pairs, ++acc) {
@@ -146,31 +184,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.acc_full[b], (acc >> 1) & 1)))) break;
       tc_fence_after();
       const int row0 = mt * 2 * kGM + (int)rank * kGM + warp * 32;   // this warp's first output row
+      const bool rotate = ROPE != 0 && nt * kGN < g.rope_cols;      // the tile is one q or k head
+      int first_plain = 0;                                            // chunks below were rotated
+      if (rotate) {
+        const int m = min(row0 + lane, g.M - 1);
+        const int p = g.pos ? g.pos[m] : (g.len ? g.len[m / g.T] : 0) + m % g.T;
 #pragma unroll 1
-      for (int c = 0; c < kGN / 32; ++c) {
-        const int col0 = nt * kGN + 32 * c;
-        uint32_t v[32];
-        tmem_ld32(trow + b * kGN + 32 * c, v);
+        for (int c = 0; c < R / 64; ++c) {   // dims [32c, 32c+32) against [R/2 + 32c, ...)
+          uint32_t u1[32], u2[32];
+          tmem_ld32(trow + b * kGN + 32 * c, u1);
+          tmem_ld32(trow + b * kGN + R / 2 + 32 * c, u2);
+          tmem_wait_ld();
+          float a1[32], a2[32];
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            float sn, cs;
+            rope_sincos(p, sm.inv_freq[32 * c + i], &sn, &cs);
+            const float x = __uint_as_float(u1[i]), y = __uint_as_float(u2[i]);
+            a1[i] = fmaf(x, cs, -y * sn);
+            a2[i] = fmaf(y, cs, x * sn);
+          }
+          store_cols32(a1, stg, lane, row0, nt * kGN + 32 * c, g);
+          store_cols32(a2, stg, lane, row0, nt * kGN + R / 2 + 32 * c, g);
+        }
+        first_plain = R / 32;
+      }
+#pragma unroll 1
+      for (int c = first_plain; c < kGN / 32; ++c) {
+        uint32_t u[32];
+        tmem_ld32(trow + b * kGN + 32 * c, u);
         tmem_wait_ld();
-        // row `lane`: 32 columns -> 4 chunks of 8 bf16, XOR-swizzled by row
+        float a[32];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          uint32_t w4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            w4[e] = pack_bf16(__uint_as_float(v[8 * q + 2 * e]), __uint_as_float(v[8 * q + 2 * e + 1]));
-          *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q ^ ((lane >> 1) & 3))) =
-              make_uint4(w4[0], w4[1], w4[2], w4[3]);
-        }
-        __syncwarp();
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int rw = rr + 8 * q;
-          const int row = row0 + rw, col = col0 + 8 * ch;
-          const uint4 val = *reinterpret_cast<const uint4*>(stg + rw * 64 + 16 * (ch ^ ((rw >> 1) & 3)));
-          if (row < g.M && col < g.N) *reinterpret_cast<uint4*>(g.y + (int64_t)row * g.ldy + col) = val;
-        }
-        __syncwarp();
+        for (int i = 0; i < 32; ++i) a[i] = __uint_as_float(u[i]);
+        store_cols32(a, stg, lane, row0, nt * kGN + 32 * c, g);
       }
       tc_fence_before();
       __syncwarp();
@@ -206,14 +253,27 @@ cudaError_t launch_gemm(const GemmHost& h, cudaStream_t st) {
   const long long n_tiles = (long long)tiles_m * g.tiles_n;
   if (n_tiles <= 0 || n_tiles > 0x3fffffffLL) return cudaErrorInvalidValue;
   g.n_tiles = (int)n_tiles;
+  g.rope_cols = h.rope_cols;
+  g.T = h.T > 0 ? h.T : 1;
+  g.pos = h.pos;
+  g.len = h.len;
   const long long grid = 2 * (n_tiles < h.n_pairs ? n_tiles : h.n_pairs);
-  gemm_kernel<<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, g);
+  if (h.rope == 1)
+    gemm_kernel<1><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, g);
+  else if (h.rope == 2)
+    gemm_kernel<2><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, g);
+  else
+    gemm_kernel<0><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, g);
   count_launch();
   return cudaGetLastError();
 }
 
 cudaError_t gemm_set_smem_attr() {
-  return cudaFuncSetAttribute(gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)gemm_smem_bytes());
+  const int smem = (int)gemm_smem_bytes();
+  cudaError_t e = cudaFuncSetAttribute(gemm_kernel<0>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess) e = cudaFuncSetAttribute(gemm_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
 }
 
 }  // namespace hyb

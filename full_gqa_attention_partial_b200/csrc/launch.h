@@ -47,6 +47,12 @@ struct GemmHost {
   int64_t ldy = 0;
   int M = 0, N = 0, K = 0;
   int n_pairs = 74;            // persistent CTA pairs (SMs / 2)
+  // RoPE epilogue: 0 none, 1 sliding-layer, 2 full-layer rotation of the
+  // 256-wide column tiles below rope_cols; row m is token m % T of sequence
+  // m / T at position pos[m], else (len ? len[m / T] : 0) + m % T
+  int rope = 0, rope_cols = 0, T = 0;
+  const int32_t* pos = nullptr;
+  const int32_t* len = nullptr;
 };
 cudaError_t launch_gemm(const GemmHost& h, cudaStream_t st);
 cudaError_t gemm_set_smem_attr();
@@ -64,6 +70,7 @@ struct PrefillHost {
   void* out = nullptr;         // [B][T][16][256]
   const int32_t* qbase = nullptr;  // [B] sequence index of token 0, or null (0)
   int ctx_mode = 0;            // 1: key row j holds sequence index qbase - 511 + j
+  int q_rotated = 0;           // 1: q is already rotated (the kernel skips RoPE)
   int B = 0, T = 0;
   int n_pairs = 74;            // persistent CTA pairs (SMs / 2)
 };

@@ -95,6 +95,7 @@ struct PfArgs {
   __nv_bfloat16* out;
   const int32_t* qbase;
   int ctx_mode;
+  int q_rotated;   // the queries arrive rotated (by the projection's epilogue)
   int B, T, n_mtiles;
 };
 
@@ -399,13 +400,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       const bool in_table = __all_sync(0xffffffffu, delta >= 0 && delta < kBM);
 
       // ---- rotation table for this tile's base position ----
-      for (int t = r; t < (R / 2) * 8; t += kBM) {
-        const int k = t % (R / 2), e = t / (R / 2);
-        float sn, cs;
-        rope_sincos(p_base + 16 * e, sm.inv_freq[k], &sn, &cs);
-        reinterpret_cast<float2*>(&sm.rot_hi[e][k >> 1])[k & 1] = make_float2(cs, sn);
+      if (!a.q_rotated) {
+        for (int t = r; t < (R / 2) * 8; t += kBM) {
+          const int k = t % (R / 2), e = t / (R / 2);
+          float sn, cs;
+          rope_sincos(p_base + 16 * e, sm.inv_freq[k], &sn, &cs);
+          reinterpret_cast<float2*>(&sm.rot_hi[e][k >> 1])[k & 1] = make_float2(cs, sn);
+        }
+        if (!__all_sync(0xffffffffu, sync_softmax())) return false;
       }
-      if (!__all_sync(0xffffffffu, sync_softmax())) return false;
 
       // ---- this row of the query tile: shared memory (128-byte swizzled boxes) -> registers ----
       uint4 qv[kD / 8];
@@ -434,17 +437,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
           *reinterpret_cast<uint4*>(sm.qo[ci >> 3] + off) = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
         }
       };
+      if (!a.q_rotated) {
 #pragma unroll
-      for (int c = 0; c < R / 64; ++c) {   // dims [R, 256) are not rotated and stay as loaded
-        uint32_t x1[16], x2[16];
-        words16(32 * c, x1);
-        words16(R / 2 + 32 * c, x2);
-        rotate32(x1, x2, 32 * c, p, delta, in_table, sm);
-        store16(32 * c, x1);
-        store16(R / 2 + 32 * c, x2);
+        for (int c = 0; c < R / 64; ++c) {   // dims [R, 256) are not rotated and stay as loaded
+          uint32_t x1[16], x2[16];
+          words16(32 * c, x1);
+          words16(R / 2 + 32 * c, x2);
+          rotate32(x1, x2, 32 * c, p, delta, in_table, sm);
+          store16(32 * c, x1);
+          store16(R / 2 + 32 * c, x2);
+        }
+        fence_proxy_async();              // qo is read by the tensor core
+        if (rank != 0) fence_cluster();   // ... through MMAs issued from CTA 0
       }
-      fence_proxy_async();              // qo is read by the tensor core
-      if (rank != 0) fence_cluster();   // ... through MMAs issued from CTA 0
       tc_fence_before();                // TMEM accesses so far precede the MMAs q_ready releases
       __syncwarp();
       if (lane == 0) {
@@ -626,6 +631,7 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   a.out = reinterpret_cast<__nv_bfloat16*>(h.out);
   a.qbase = h.qbase;
   a.ctx_mode = h.ctx_mode;
+  a.q_rotated = h.q_rotated;
   a.B = h.B;
   a.T = h.T;
   a.n_mtiles = (h.T + kBM - 1) / kBM;
