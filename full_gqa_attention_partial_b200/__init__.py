@@ -37,6 +37,7 @@ EXPORTED = (
     "hyb_attn_decode_workspace_size", "hyb_attn_decode", "hyb_device_error", "hyb_last_error",
     "hyb_launch_count", "hyb_profile_events", "hyb_profile_pairs_used", "hyb_attn_decode_noalloc",
     "hyb_selftest_wait_timeout", "hyb_linear", "hyb_attn_layer_prefill_workspace_size", "hyb_attn_layer_prefill",
+    "hyb_attn_layer_decode_workspace_size", "hyb_attn_layer_decode",
 )
 
 
@@ -96,6 +97,9 @@ def load(path: str = LIB_PATH):
     lib.hyb_attn_layer_prefill_workspace_size.argtypes = [i32, i32, i32, i32]
     lib.hyb_attn_layer_prefill_workspace_size.restype = sz
     lib.hyb_attn_layer_prefill.argtypes = [vp, vp, vp, vp, vp, i32, i32, i32, vp, pc, vp, sz, vp]
+    lib.hyb_attn_layer_decode_workspace_size.argtypes = [i32, i32, i64]
+    lib.hyb_attn_layer_decode_workspace_size.restype = sz
+    lib.hyb_attn_layer_decode.argtypes = [vp, vp, vp, vp, pc, i32, i64, vp, vp, sz, vp]
     for name in ("hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill", "hyb_attn_decode",
                  "hyb_device_error"):
         getattr(lib, name).restype = ctypes.c_int
@@ -248,6 +252,30 @@ def hyb_attn_layer_prefill(hidden, w_qkv, w_gate, w_o, pos, layer_type: int, out
     _check(load().hyb_attn_layer_prefill(_ptr(hidden), _ptr(w_qkv), _ptr(w_gate), _ptr(w_o), _ptr(pos), layer_type,
                                          B, T, _ptr(out), None if cache is None else cache.ref, _ptr(workspace), wsz,
                                          _stream(stream)))
+    return out
+
+
+def hyb_attn_layer_decode(hidden, w_qkv, w_gate, w_o, cache: KVCache, max_len: int = 0, out=None, workspace=None,
+                          stream=None):
+    """One attention layer for a decode step: hidden bf16 [B,2560] (one new token
+    per sequence); appends the token's K/V to `cache` and attends.  Returns
+    out bf16 [B,2560]."""
+    if hidden.dtype != torch.bfloat16 or not hidden.is_contiguous() or tuple(hidden.shape) != (cache.batch, HIDDEN):
+        raise ValueError("hidden must be contiguous bf16 [B, 2560]")
+    for name, w, shape in (("w_qkv", w_qkv, (6144, HIDDEN)), ("w_o", w_o, (HIDDEN, N_Q_HEADS * HEAD_DIM)),
+                           ("w_gate", w_gate, (N_Q_HEADS, HIDDEN))):
+        if w is not None and (w.dtype != torch.bfloat16 or not w.is_contiguous() or tuple(w.shape) != shape):
+            raise ValueError(f"{name} must be contiguous bf16 {list(shape)}")
+    B = cache.batch
+    if out is None:
+        out = torch.empty(B, HIDDEN, dtype=torch.bfloat16, device=hidden.device)
+    lt = cache.layer_type
+    need = int(load().hyb_attn_layer_decode_workspace_size(lt, B, max_len or cache.capacity))
+    if workspace is None:
+        workspace = alloc_workspace(need, hidden.device)
+    wsz = workspace.numel() * workspace.element_size()
+    _check(load().hyb_attn_layer_decode(_ptr(hidden), _ptr(w_qkv), _ptr(w_gate), _ptr(w_o), cache.ref, lt, max_len,
+                                        _ptr(out), _ptr(workspace), wsz, _stream(stream)))
     return out
 
 

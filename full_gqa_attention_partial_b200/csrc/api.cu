@@ -305,8 +305,9 @@ hyb_status hyb_kv_cache_init(const hyb_kv_cache* c, const int32_t* head0, void* 
   return HYB_OK;
 }
 
-hyb_status hyb_kv_append(const hyb_kv_cache* c, const void* k, const void* v, int64_t kv_row_stride,
-                         const int32_t* pos, int32_t T, void* stream) {
+namespace {
+hyb_status append_impl(const hyb_kv_cache* c, const void* k, const void* v, int64_t kv_row_stride, const int32_t* pos,
+                       int32_t T, void* stream, bool k_rotated) {
   hyb_status s = check_cache(c);
   if (s != HYB_OK) return s;
   if (!k || !v) return fail(HYB_EINVAL, "k and v must be non-NULL");
@@ -336,11 +337,18 @@ hyb_status hyb_kv_append(const hyb_kv_cache* c, const void* k, const void* v, in
   r.B = c->batch;
   r.T = T;
   r.t_first = full ? 0 : (T > kWindow ? T - kWindow : 0);
+  r.src_rotated = k_rotated ? 1 : 0;
   cudaError_t e = launch_rope_store(full, r, st);
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
   if ((e = launch_kv_commit(c->len, c->head, c->capacity, !full, c->batch, T, st)) != cudaSuccess)
     return cuda_fail(e, "commit launch");
   return HYB_OK;
+}
+}  // namespace
+
+hyb_status hyb_kv_append(const hyb_kv_cache* c, const void* k, const void* v, int64_t kv_row_stride,
+                         const int32_t* pos, int32_t T, void* stream) {
+  return append_impl(c, k, v, kv_row_stride, pos, T, stream, false);
 }
 
 size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache) {
@@ -519,9 +527,10 @@ size_t hyb_attn_decode_workspace_size(int32_t layer_type, int32_t B, int64_t max
   return rows * kD * sizeof(float) + ((rows * sizeof(float) + 255) & ~size_t(255));
 }
 
-hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos, const hyb_kv_cache* c,
-                           int32_t layer_type, int64_t max_len, void* out, void* workspace,
-                           size_t workspace_bytes, void* stream) {
+namespace {
+hyb_status decode_impl(const void* q, int64_t q_stride, bool q_rotated, const void* gate, const int32_t* pos,
+                       const hyb_kv_cache* c, int32_t layer_type, int64_t max_len, void* out, void* workspace,
+                       size_t workspace_bytes, void* stream) {
   hyb_status s = check_cache(c);
   if (s != HYB_OK) return s;
   if (!q || !out) return fail(HYB_EINVAL, "q and out must be non-NULL");
@@ -541,6 +550,8 @@ hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos, 
   DecodeHost d;
   if ((s = cache_maps(c, &d.tm_k, &d.tm_v, 64, 64)) != HYB_OK) return s;
   d.q = q;
+  d.q_stride = q_stride;
+  d.q_rotated = q_rotated ? 1 : 0;
   d.gate = gate;
   d.pos = pos;
   d.len = c->len;
@@ -553,6 +564,14 @@ hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos, 
   cudaError_t e = launch_decode(layer_type == HYB_FULL, d, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return HYB_OK;
+}
+}  // namespace
+
+hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos, const hyb_kv_cache* c,
+                           int32_t layer_type, int64_t max_len, void* out, void* workspace,
+                           size_t workspace_bytes, void* stream) {
+  return decode_impl(q, (int64_t)kHq * kD, false, gate, pos, c, layer_type, max_len, out, workspace, workspace_bytes,
+                     stream);
 }
 
 // Same computation as hyb_attn_decode, with the split partials kept in the
@@ -655,4 +674,52 @@ hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const v
   if (s != HYB_OK) return s;
   return hyb_linear(attn, (int64_t)kHq * kD, w_o, (int64_t)kHq * kD, out, kHidden, M, (int32_t)kHidden,
                     (int32_t)(kHq * kD), stream);
+}
+
+size_t hyb_attn_layer_decode_workspace_size(int32_t layer_type, int32_t B, int64_t max_len) {
+  if (B <= 0) return 0;
+  const size_t n = (size_t)B;
+  return round256(n * kQkv * 2) + round256(n * kHq * 2) + round256(n * kHq * kD * 2) +
+         hyb_attn_decode_workspace_size(layer_type, B, max_len);
+}
+
+hyb_status hyb_attn_layer_decode(const void* hidden, const void* w_qkv, const void* w_gate, const void* w_o,
+                                 const hyb_kv_cache* cache, int32_t layer_type, int64_t max_len, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream) {
+  hyb_status s = check_cache(cache);
+  if (s != HYB_OK) return s;
+  if (!hidden || !w_qkv || !w_o || !out) return fail(HYB_EINVAL, "hidden, w_qkv, w_o and out must be non-NULL");
+  if (layer_type != cache->type)
+    return fail(HYB_ESHAPE, "layer_type %d differs from the cache type %d", layer_type, cache->type);
+  if (max_len < 0 || max_len > cache->capacity)
+    return fail(HYB_ESHAPE, "max_len %lld outside [0, capacity %lld]", (long long)max_len, (long long)cache->capacity);
+  if (max_len == 0) max_len = cache->capacity;
+  const int32_t B = cache->batch;
+  const size_t need = hyb_attn_layer_decode_workspace_size(layer_type, B, max_len);
+  if (workspace_bytes < need) return fail(HYB_EOVERFLOW, "workspace %zu bytes < %zu needed", workspace_bytes, need);
+  if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return fail(HYB_EALIGN, "workspace must be non-NULL and 256-byte aligned");
+  const size_t n = (size_t)B;
+  uint8_t* p = static_cast<uint8_t*>(workspace);
+  __nv_bfloat16* qkv = reinterpret_cast<__nv_bfloat16*>(p);
+  p += round256(n * kQkv * 2);
+  __nv_bfloat16* gate = reinterpret_cast<__nv_bfloat16*>(p);
+  p += round256(n * kHq * 2);
+  __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(p);
+  p += round256(n * kHq * kD * 2);
+  // q_k_v_proj with RoPE at the new token's position (the cache length)
+  if ((s = linear_impl(hidden, kHidden, w_qkv, kHidden, qkv, kQkv, B, (int32_t)kQkv, (int32_t)kHidden, stream,
+                       layer_type == HYB_FULL ? 2 : 1, (kHq + kHkv) * kD, 1, nullptr, cache->len)) != HYB_OK)
+    return s;
+  if (w_gate && (s = linear_impl(hidden, kHidden, w_gate, kHidden, gate, kHq, B, kHq, (int32_t)kHidden, stream)) !=
+                    HYB_OK)
+    return s;
+  if ((s = append_impl(cache, qkv + (int64_t)kHq * kD, qkv + (int64_t)(kHq + kHkv) * kD, kQkv, nullptr, 1, stream,
+                       true)) != HYB_OK)
+    return s;
+  if ((s = decode_impl(qkv, kQkv, true, w_gate ? gate : nullptr, nullptr, cache, layer_type, max_len, attn, p,
+                       hyb_attn_decode_workspace_size(layer_type, B, max_len), stream)) != HYB_OK)
+    return s;
+  return linear_impl(attn, (int64_t)kHq * kD, w_o, (int64_t)kHq * kD, out, kHidden, B, (int32_t)kHidden,
+                     (int32_t)(kHq * kD), stream);
 }

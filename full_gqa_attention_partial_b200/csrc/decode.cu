@@ -45,6 +45,8 @@ size_t decode_smem_bytes() { return sizeof(DecSmem) + 1024; }
 
 struct DecArgs {
   const __nv_bfloat16* q;
+  int64_t q_stride;   // elements between the query rows of consecutive sequences
+  int q_rotated;      // 1: the queries arrive rotated
   const int32_t* pos;
   const int32_t* len;
   const int32_t* tag;
@@ -116,13 +118,13 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     const int hh = threadIdx.x >> 5;        // 0..3
     const int d0 = lane * 8;
     const int p = a.pos ? a.pos[b] : qseq;
-    uint4 qx = *reinterpret_cast<const uint4*>(a.q + ((int64_t)b * kHq + kvh * kGroup + hh) * kD + d0);
+    uint4 qx = *reinterpret_cast<const uint4*>(a.q + (int64_t)b * a.q_stride + (int64_t)(kvh * kGroup + hh) * kD + d0);
     const uint32_t xs[4] = {qx.x, qx.y, qx.z, qx.w};
     uint32_t ys[4];
     constexpr int xor_mask = (R == 256) ? 16 : 4;
 #pragma unroll
     for (int w = 0; w < 4; ++w) ys[w] = __shfl_xor_sync(0xffffffffu, xs[w], xor_mask);
-    if (d0 < R) {
+    if (!a.q_rotated && d0 < R) {
       const bool first_half = d0 < R / 2;
       const int kb = first_half ? d0 : d0 - R / 2;
       uint32_t os[4];
@@ -323,6 +325,8 @@ int decode_num_splits(bool full, int B, int64_t max_len) {
 cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
   DecArgs a;
   a.q = reinterpret_cast<const __nv_bfloat16*>(h.q);
+  a.q_stride = h.q_stride;
+  a.q_rotated = h.q_rotated;
   a.pos = h.pos;
   a.len = h.len;
   a.tag = h.tag;

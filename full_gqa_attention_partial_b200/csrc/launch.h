@@ -83,7 +83,9 @@ size_t prefill_smem_bytes();
 // ---- decode (decode.cu) -------------------------------------------------------
 struct DecodeHost {
   CUtensorMap tm_k, tm_v;      // 4-D maps over the cache {256, capacity, 4, B}
-  const void* q = nullptr;     // [B][16][256]
+  const void* q = nullptr;     // [B][16][256] rows q_stride elements apart
+  int64_t q_stride = 16 * 256;
+  int q_rotated = 0;           // 1: q is already rotated (the kernel skips RoPE)
   const void* gate = nullptr;  // [B][16] or null
   const int32_t* pos = nullptr;
   const int32_t* len = nullptr;

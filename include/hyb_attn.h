@@ -240,6 +240,24 @@ hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const v
                                   void* stream);
 
 /*
+ * One whole attention layer for a decode step: q_k_v_proj (RoPE of q and k at
+ * the new token's position, the cache length), the gate projection, the KV
+ * append of the new token, the attention of hyb_attn_decode and o_proj.
+ *   hidden : bf16 [B][2560] (one token per sequence, B = cache->batch).
+ *   w_qkv, w_gate (or NULL), w_o : as hyb_attn_layer_prefill.
+ *   cache, layer_type, max_len : as hyb_attn_decode (max_len bounds the length
+ *          after this step's append).
+ *   out    : bf16 [B][2560].
+ *   workspace: at least hyb_attn_layer_decode_workspace_size(layer_type, B,
+ *          max_len) bytes, 256-byte aligned.
+ * Errors: as hyb_linear, hyb_kv_append and hyb_attn_decode.
+ */
+size_t hyb_attn_layer_decode_workspace_size(int32_t layer_type, int32_t B, int64_t max_len);
+hyb_status hyb_attn_layer_decode(const void* hidden, const void* w_qkv, const void* w_gate, const void* w_o,
+                                 const hyb_kv_cache* cache, int32_t layer_type, int64_t max_len, void* out,
+                                 void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Failure-path self-test (no counterpart in the pages).  Launches one block
  * on `stream` whose first thread waits on a shared-memory barrier that
  * nothing completes.  The wait is bounded like every pipeline wait of the

@@ -300,6 +300,31 @@ def attention_layer(hidden, w_qkv, w_gate, w_o, pos, lt, rows=None):
     return linear(o.reshape(B, o.shape[1], N_Q_HEADS * HEAD_DIM), w_o)
 
 
+def attention_layer_decode(hidden, w_qkv, w_gate, w_o, qpos, hist_k, hist_v, hist_idx, lt):
+    """One attention layer for a decode step: the new token of each sequence
+    goes through the projections, its K/V join the history, and the query
+    attends (the decode definition of decode()).
+    hidden [B, 2560] the new tokens, each at sequence index and RoPE position
+    qpos[b]; hist_k / hist_v [B][L_b, 4, 256] the cached history (K roped),
+    hist_idx [B][L_b] its sequence indices.  Intermediates rounded to bf16 as
+    in attention_layer.  Returns [B, 2560] float64."""
+    hidden = np.asarray(hidden, dtype=np.float64)
+    B = hidden.shape[0]
+    qkv = to_bf16(linear(hidden, w_qkv))
+    q = qkv[:, :N_Q_HEADS * HEAD_DIM].reshape(B, N_Q_HEADS, HEAD_DIM)
+    k = qkv[:, N_Q_HEADS * HEAD_DIM:(N_Q_HEADS + N_KV_HEADS) * HEAD_DIM].reshape(B, N_KV_HEADS, HEAD_DIM)
+    v = qkv[:, (N_Q_HEADS + N_KV_HEADS) * HEAD_DIM:].reshape(B, N_KV_HEADS, HEAD_DIM)
+    gate = None if w_gate is None else to_bf16(linear(hidden, w_gate))
+    keys, vals, idx = [], [], []
+    for b in range(B):
+        kn = rope_layer(k[b][None], np.array([qpos[b]]), lt)[0]
+        keys.append(np.concatenate([np.asarray(hist_k[b], np.float64), kn[None]]))
+        vals.append(np.concatenate([np.asarray(hist_v[b], np.float64), v[b][None]]))
+        idx.append(np.append(np.asarray(hist_idx[b]), qpos[b]))
+    o = to_bf16(decode(q, gate, qpos, keys, vals, idx, lt))
+    return linear(o.reshape(B, N_Q_HEADS * HEAD_DIM), w_o)
+
+
 # ---------------------------------------------------------------------------
 # KV caches: linear (full layers) and the 512-slot ring (sliding layers)
 # ---------------------------------------------------------------------------

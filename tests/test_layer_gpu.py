@@ -95,3 +95,51 @@ def test_layer_rejects_bad_weight_shape(lib):
     w_qkv, w_gate, w_o = weights(0)
     with pytest.raises(ValueError):
         lib.hyb_attn_layer_prefill(h, w_qkv[:, :2048].contiguous(), w_gate, w_o, None, O.FULL)
+
+
+@pytest.mark.parametrize("lt", [O.SLIDING, O.FULL])
+def test_layer_decode_steps(lib, lt):
+    """Three decode steps of the layer over a seeded cache (history snapshot
+    taken before any library call on it; the oracle projects and rotates the
+    new tokens itself)."""
+    import bench
+    from full_gqa_attention_partial_b200 import synth
+    B, L, n_steps = 3, 1500, 3
+    w_qkv, w_gate, w_o = weights(50 + lt)
+    if lt == O.FULL:
+        cap = L + n_steps
+        cache = bench.fill_full_cache(lib, B, L, cap, seed=8)
+        hist = [(f64(cache.k[b, :, :L]).transpose(1, 0, 2), f64(cache.v[b, :, :L]).transpose(1, 0, 2),
+                 np.arange(L)) for b in range(B)]
+        max_len = cap
+    else:
+        r = synth.ring_offset(9)
+        cache = bench.fill_ring_cache(lib, B, L, seed=10, head0=r)
+        idx = np.arange(L - O.WINDOW, L)
+        rk, rv = f64(cache.k), f64(cache.v)           # [B, 4, 512, 256], slot-indexed
+        hist = [(rk[b][:, (r + idx) % O.WINDOW].transpose(1, 0, 2), rv[b][:, (r + idx) % O.WINDOW].transpose(1, 0, 2),
+                 idx) for b in range(B)]
+        max_len = O.WINDOW
+    for step in range(n_steps):
+        h = hidden_states(1, B, seed=60 + step)[0]    # [B, 2560]
+        out = lib.hyb_attn_layer_decode(h, w_qkv, w_gate, w_o, cache, max_len=max_len)
+        torch.cuda.synchronize()
+        assert lib.hyb_device_error() == 0
+        n = L + step                                  # sequence index of the new token
+        ref = O.attention_layer_decode(f64(h), f64(w_qkv), f64(w_gate), f64(w_o), [n] * B,
+                                       [x[0] for x in hist], [x[1] for x in hist], [x[2] for x in hist], lt)
+        check(out, ref, f"layer decode step {step} type {lt}")
+        # the oracle's history grows by the token it just computed
+        hf = f64(h)
+        qkv = O.to_bf16(O.linear(hf, f64(w_qkv)))
+        kn = O.rope_layer(qkv[:, 4096:5120].reshape(B, 1, 4, 256), np.full((B, 1), n), lt)[:, 0]
+        vn = qkv[:, 5120:].reshape(B, 4, 256)
+        new_hist = []
+        for b in range(B):
+            k_b = np.concatenate([hist[b][0], kn[b][None]])
+            v_b = np.concatenate([hist[b][1], vn[b][None]])
+            i_b = np.append(hist[b][2], n)
+            if lt == O.SLIDING:                       # the window keeps the last 512
+                k_b, v_b, i_b = k_b[-O.WINDOW:], v_b[-O.WINDOW:], i_b[-O.WINDOW:]
+            new_hist.append((k_b, v_b, i_b))
+        hist = new_hist

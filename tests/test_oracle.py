@@ -399,3 +399,22 @@ def test_to_bf16_rounds_to_nearest_even():
     # bf16 keeps 8 significant bits: ulp(1) = 2^-7; halfway cases go to even
     np.testing.assert_array_equal(got[:5], [1.0, 1.0, 1.0 + 2 ** -7, 1.0, -2.5])
     assert np.isfinite(got[5]) and abs(got[5] / 3.0e38 - 1) < 2 ** -8
+
+
+@pytest.mark.parametrize("lt", [O.SLIDING, O.FULL])
+def test_layer_decode_equals_last_row_of_layer_prefill(lt):
+    """Decoding the last token of a sequence through the layer, with the other
+    tokens' projected K/V as history, gives the layer prefill's last row."""
+    rng = np.random.default_rng(12)
+    T, Hd = 7, 2560
+    hidden = O.to_bf16(rng.standard_normal((1, T, Hd)))
+    w_qkv = O.to_bf16(rng.standard_normal((6144, Hd)) / np.sqrt(Hd))
+    w_gate = O.to_bf16(rng.standard_normal((16, Hd)) / np.sqrt(Hd))
+    w_o = O.to_bf16(rng.standard_normal((Hd, 4096)) / 64.0)
+    pos = np.arange(T)[None]
+    full = O.attention_layer(hidden, w_qkv, w_gate, w_o, pos, lt)
+    qkv = O.to_bf16(hidden[0, :T - 1] @ w_qkv.T)
+    hk = O.rope_layer(qkv[:, 4096:5120].reshape(T - 1, 4, 256), np.arange(T - 1), lt)
+    hv = qkv[:, 5120:].reshape(T - 1, 4, 256)
+    got = O.attention_layer_decode(hidden[:, T - 1], w_qkv, w_gate, w_o, [T - 1], [hk], [hv], [np.arange(T - 1)], lt)
+    np.testing.assert_allclose(got[0], full[0, T - 1], rtol=1e-10, atol=1e-12)
