@@ -670,7 +670,16 @@ def run_case(hyb, args):
     """One kernel on a small configuration, for profiler captures: 1 warm-up + args.steps launches."""
     from full_gqa_attention_partial_b200 import synth
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if args.case.startswith("prefill"):
+    if args.case == "linear_qkv":
+        M, N, K = args.seq * args.batch, 6144, 2560
+        g = torch.Generator(device="cuda").manual_seed(5)
+        x = torch.randn(M, K, generator=g, device="cuda").to(torch.bfloat16)
+        w = (torch.randn(N, K, generator=g, device="cuda") / K ** 0.5).to(torch.bfloat16)
+        y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        fn = lambda: hyb.hyb_linear(x, w, out=y)
+        work = 2 * M * N * K
+        unit = "TFLOP/s"
+    elif args.case.startswith("prefill"):
         lt = FULL if args.case == "prefill_full" else SLIDING
         T, B = args.seq, args.batch
         x = synth.prefill_inputs(B, T, seed=layer_seed(1, 3), device="cuda")
@@ -693,11 +702,19 @@ def run_case(hyb, args):
         unit = "GB/s"
     fn()
     torch.cuda.synchronize()
-    timer = hyb.KernelTimer(args.steps)
-    with timer:
+    if args.case == "linear_qkv":   # one kernel per call: events around the calls
+        ev0.record()
         for _ in range(args.steps):
             fn()
-    ms = statistics.mean(timer.times_ms())
+        ev1.record()
+        torch.cuda.synchronize()
+        ms = ev0.elapsed_time(ev1) / args.steps
+    else:
+        timer = hyb.KernelTimer(args.steps)
+        with timer:
+            for _ in range(args.steps):
+                fn()
+        ms = statistics.mean(timer.times_ms())
     assert hyb.hyb_device_error() == 0
     rate = work / (ms / 1e3) / (1e12 if unit == "TFLOP/s" else 1e9)
     print(json.dumps({"case": args.case, "batch": args.batch, "seq": args.seq, "kernel_ms": ms,
@@ -717,7 +734,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="only the headline step (no sub-benchmarks)")
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows per layer for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="oracle rows per layer per reference step")
-    ap.add_argument("--case", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_sliding"],
+    ap.add_argument("--case", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_sliding", "linear_qkv"],
                     default=None, help="time one kernel on a small configuration (profiling)")
     ap.add_argument("--seq", type=int, default=16384)
     ap.add_argument("--batch", type=int, default=1)
