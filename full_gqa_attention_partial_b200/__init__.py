@@ -26,6 +26,8 @@ HEAD_DIM = 256
 WINDOW = 512
 N_LAYERS = 36
 
+KV_BF16 = 0
+KV_FP8 = 1
 DEV_ERR_CAPACITY = 1
 DEV_ERR_TIMEOUT = 2
 
@@ -59,6 +61,7 @@ class _Cache(ctypes.Structure):
         ("type", ctypes.c_int32), ("batch", ctypes.c_int32), ("capacity", ctypes.c_int64),
         ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_void_p),
         ("head", ctypes.c_void_p), ("tag", ctypes.c_void_p),
+        ("kv_dtype", ctypes.c_int32), ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
     ]
 
 
@@ -142,23 +145,30 @@ class KVCache:
     """One layer's KV cache for `batch` sequences (memory from torch).
 
     Full layers: linear cache of `capacity` tokens.  Sliding layers: 512-slot
-    ring; `head0` gives each sequence's starting write slot.
+    ring; `head0` gives each sequence's starting write slot.  kv_dtype KV_FP8
+    stores e4m3 codes (uint8) with one fp32 scale per (token, KV head) row.
     """
 
     def __init__(self, layer_type: int, batch: int, capacity: int = WINDOW, device="cuda", head0=None,
-                 stream=None):
+                 stream=None, kv_dtype: int = 0):
         cap = WINDOW if layer_type == SLIDING else int(capacity)
         self.layer_type = layer_type
         self.batch = batch
         self.capacity = cap
-        bf = torch.bfloat16
-        self.k = torch.empty(batch, N_KV_HEADS, cap, HEAD_DIM, dtype=bf, device=device)
-        self.v = torch.empty(batch, N_KV_HEADS, cap, HEAD_DIM, dtype=bf, device=device)
+        self.kv_dtype = kv_dtype
+        et = torch.uint8 if kv_dtype == KV_FP8 else torch.bfloat16
+        self.k = torch.empty(batch, N_KV_HEADS, cap, HEAD_DIM, dtype=et, device=device)
+        self.v = torch.empty(batch, N_KV_HEADS, cap, HEAD_DIM, dtype=et, device=device)
         self.len = torch.empty(batch, dtype=torch.int32, device=device)
         self.head = torch.empty(batch, dtype=torch.int32, device=device)
         self.tag = torch.empty(batch, WINDOW, dtype=torch.int32, device=device)
+        self.k_scale = self.v_scale = None
+        if kv_dtype == KV_FP8:
+            self.k_scale = torch.empty(batch, N_KV_HEADS, cap, dtype=torch.float32, device=device)
+            self.v_scale = torch.empty(batch, N_KV_HEADS, cap, dtype=torch.float32, device=device)
         self.c = _Cache(layer_type, batch, cap, self.k.data_ptr(), self.v.data_ptr(), self.len.data_ptr(),
-                        self.head.data_ptr(), self.tag.data_ptr())
+                        self.head.data_ptr(), self.tag.data_ptr(), kv_dtype,
+                        _ptr(self.k_scale), _ptr(self.v_scale))
         hyb_kv_cache_init(self, head0, stream)
 
     @property

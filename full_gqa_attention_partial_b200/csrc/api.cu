@@ -157,6 +157,13 @@ hyb_status check_cache(const hyb_kv_cache* c) {
   if (!c->k || !c->v || !c->len) return fail(HYB_EINVAL, "cache k, v and len must be non-NULL");
   if (!aligned16(c->k) || !aligned16(c->v)) return fail(HYB_EALIGN, "cache k/v must be 16-byte aligned");
   if ((reinterpret_cast<uintptr_t>(c->len) & 3u) != 0) return fail(HYB_EALIGN, "cache len must be 4-byte aligned");
+  if (c->kv_dtype != HYB_KV_BF16 && c->kv_dtype != HYB_KV_FP8)
+    return fail(HYB_EINVAL, "cache kv_dtype %d invalid", c->kv_dtype);
+  if (c->kv_dtype == HYB_KV_FP8) {
+    if (!c->k_scale || !c->v_scale) return fail(HYB_EINVAL, "an FP8 cache needs k_scale and v_scale buffers");
+    if (!aligned16(c->k_scale) || !aligned16(c->v_scale)) return fail(HYB_EALIGN, "cache scales must be 16-byte aligned");
+    if (c->capacity % 4) return fail(HYB_ESHAPE, "an FP8 cache needs capacity % 4 == 0, got %lld", (long long)c->capacity);
+  }
   if (c->type == HYB_SLIDING) {
     if (c->capacity != kWindow) return fail(HYB_ESHAPE, "sliding cache capacity must be 512, got %lld",
                                             (long long)c->capacity);
@@ -282,10 +289,16 @@ hyb_status hyb_kv_cache_init(const hyb_kv_cache* c, const int32_t* head0, void* 
   if (s != HYB_OK) return s;
   if ((s = ensure_device()) != HYB_OK) return s;
   cudaStream_t st = as_stream(stream);
-  const size_t kv_bytes = (size_t)c->batch * kHkv * (size_t)c->capacity * kD * 2;
+  const bool fp8 = c->kv_dtype == HYB_KV_FP8;
+  const size_t rows = (size_t)c->batch * kHkv * (size_t)c->capacity;
+  const size_t kv_bytes = rows * kD * (fp8 ? 1 : 2);
   cudaError_t e;
   if ((e = cudaMemsetAsync(c->k, 0, kv_bytes, st)) != cudaSuccess) return cuda_fail(e, "zero cache K");
   if ((e = cudaMemsetAsync(c->v, 0, kv_bytes, st)) != cudaSuccess) return cuda_fail(e, "zero cache V");
+  if (fp8) {
+    if ((e = cudaMemsetAsync(c->k_scale, 0, rows * sizeof(float), st)) != cudaSuccess) return cuda_fail(e, "k_scale");
+    if ((e = cudaMemsetAsync(c->v_scale, 0, rows * sizeof(float), st)) != cudaSuccess) return cuda_fail(e, "v_scale");
+  }
   if ((e = cudaMemsetAsync(c->len, 0, sizeof(int32_t) * c->batch, st)) != cudaSuccess) return cuda_fail(e, "len");
   if (c->type == HYB_SLIDING) {
     if ((e = launch_fill_i32(c->tag, (int64_t)c->batch * kWindow, -1, st)) != cudaSuccess)
@@ -338,6 +351,9 @@ hyb_status append_impl(const hyb_kv_cache* c, const void* k, const void* v, int6
   r.T = T;
   r.t_first = full ? 0 : (T > kWindow ? T - kWindow : 0);
   r.src_rotated = k_rotated ? 1 : 0;
+  r.fp8 = c->kv_dtype == HYB_KV_FP8 ? 1 : 0;
+  r.dks = c->k_scale;
+  r.dvs = c->v_scale;
   cudaError_t e = launch_rope_store(full, r, st);
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
   if ((e = launch_kv_commit(c->len, c->head, c->capacity, !full, c->batch, T, st)) != cudaSuccess)
@@ -385,6 +401,8 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
     if (cache->type != layer_type)
       return fail(HYB_ESHAPE, "cache type %d differs from layer_type %d", cache->type, layer_type);
     if (cache->batch != B) return fail(HYB_ESHAPE, "cache batch %d differs from B = %d", cache->batch, B);
+    if (cache->kv_dtype != HYB_KV_BF16)
+      return fail(HYB_EUNSUPPORTED, "prefill attends over bf16 caches only (this cache is FP8)");
     if (layer_type == HYB_FULL && (int64_t)T > cache->capacity)
       return fail(HYB_ESHAPE, "T = %d exceeds the cache capacity %lld", T, (long long)cache->capacity);
   }
@@ -535,6 +553,7 @@ hyb_status decode_impl(const void* q, int64_t q_stride, bool q_rotated, const vo
   if (s != HYB_OK) return s;
   if (!q || !out) return fail(HYB_EINVAL, "q and out must be non-NULL");
   if (layer_type != c->type) return fail(HYB_ESHAPE, "layer_type %d differs from the cache type %d", layer_type, c->type);
+  if (c->kv_dtype != HYB_KV_BF16) return fail(HYB_EUNSUPPORTED, "decode of FP8 caches is not built yet");
   if (!aligned16(q) || !aligned16(out)) return fail(HYB_EALIGN, "q and out must be 16-byte aligned");
   if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
   if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u)) return fail(HYB_EALIGN, "pos must be 4-byte aligned");
@@ -583,6 +602,7 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
   if (s != HYB_OK) return s;
   if (!q || !out) return fail(HYB_EINVAL, "q and out must be non-NULL");
   if (layer_type != c->type) return fail(HYB_ESHAPE, "layer_type %d differs from the cache type %d", layer_type, c->type);
+  if (c->kv_dtype != HYB_KV_BF16) return fail(HYB_EUNSUPPORTED, "decode of FP8 caches is not built yet");
   if (!aligned16(q) || !aligned16(out)) return fail(HYB_EALIGN, "q and out must be 16-byte aligned");
   if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
   if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u)) return fail(HYB_EALIGN, "pos must be 4-byte aligned");

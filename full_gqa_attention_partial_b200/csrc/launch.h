@@ -30,6 +30,9 @@ struct RopeStoreHost {
   const int32_t* head = nullptr;
   int32_t* tag = nullptr;
   int B = 0, T = 0, t_first = 0;
+  int fp8 = 0;                 // 1: destination is an FP8 cache (codes + per-row scales)
+  float* dks = nullptr;
+  float* dvs = nullptr;
 };
 cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st);
 cudaError_t launch_ring_gather(const void* rk, const void* rv, const int32_t* len, const int32_t* head,

@@ -42,7 +42,38 @@ struct RopeStoreArgs {
   int32_t* tag;
   int B, T;
   int t_first;              // first token index written (ring: max(0, T - 512))
+  int fp8;                  // 1: dk / dv hold e4m3 codes (1 byte), scales to dks / dvs
+  float* dks;               // [B][4][dst_rows]
+  float* dvs;
 };
+
+// One 256-dim row (one token, one KV head) held by a warp, 8 bf16 values per
+// lane in `x`: e4m3 codes with scale amax / 448, codes = satfinite round to
+// nearest even of value * (448 / amax) (a zero row: scale 0, codes 0).
+__device__ __forceinline__ void store_row_fp8(uint4 x, uint8_t* dst, float* dscale, int lane) {
+  const uint32_t w[4] = {x.x, x.y, x.z, x.w};
+  float f[8];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    f[2 * i] = bf16lo(w[i]);
+    f[2 * i + 1] = bf16hi(w[i]);
+  }
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+  for (int o = 16; o >= 1; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+  const float inv = amax > 0.f ? 448.f / amax : 0.f;
+  uint32_t c[4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {   // element 2i in the low byte
+    uint16_t h;
+    asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(f[2 * i + 1] * inv), "f"(f[2 * i] * inv));
+    c[i] = h;
+  }
+  *reinterpret_cast<uint2*>(dst) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+  if (lane == 0) *dscale = amax / 448.f;
+}
 
 // One block = one token of one sequence, 128 threads; thread i handles
 // 8 consecutive dims (16 bytes) of KV head i / 32.  Rotation partners
@@ -107,6 +138,14 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
         }
         kx = make_uint4(os[0], os[1], os[2], os[3]);
       }
+    }
+    if (a.fp8) {
+      const int64_t row = ((int64_t)b * kHkv + kvh) * a.dst_rows + dst_row;
+      store_row_fp8(kx, reinterpret_cast<uint8_t*>(a.dk) + dst, a.dks + row, lane32);
+      if (a.v != nullptr)
+        store_row_fp8(*reinterpret_cast<const uint4*>(a.v + src), reinterpret_cast<uint8_t*>(a.dv) + dst, a.dvs + row,
+                      lane32);
+      continue;
     }
     *reinterpret_cast<uint4*>(a.dk + dst) = kx;
     if (a.v != nullptr) {
@@ -182,6 +221,9 @@ cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st
   a.src_tstride = h.src_tstride;
   a.src_hstride = h.src_hstride;
   a.src_rotated = h.src_rotated;
+  a.fp8 = h.fp8;
+  a.dks = h.dks;
+  a.dvs = h.dvs;
   a.pos = h.pos;
   a.dk = reinterpret_cast<__nv_bfloat16*>(h.dk);
   a.dv = reinterpret_cast<__nv_bfloat16*>(h.dv);

@@ -95,7 +95,27 @@ typedef struct hyb_kv_cache {
   int32_t* len;
   int32_t* head;
   int32_t* tag;
+  int32_t kv_dtype;  /* HYB_KV_BF16 (0) or HYB_KV_FP8 (1) */
+  float* k_scale;    /* HYB_KV_FP8 only: fp32 [batch][4][capacity], one scale per */
+  float* v_scale;    /*   (token, KV head) row; NULL for HYB_KV_BF16 */
 } hyb_kv_cache;
+
+/*
+ * KV storage types.  HYB_KV_BF16: k / v hold bf16 [batch][4][capacity][256].
+ * HYB_KV_FP8: k / v hold FP8 e4m3 codes (1 byte) [batch][4][capacity][256],
+ * and each 256-dim row (one token, one KV head) has an fp32 scale:
+ *   scale = amax / 448 (amax = largest |value| of the row, the K row after
+ *   RoPE and bf16 rounding as the bf16 cache would hold it),
+ *   code  = e4m3(round to nearest even, saturating at +-448)(value * (448 / amax)),
+ *   stored value = code * scale (a zero row has scale 0 and zero codes).
+ * Halves the cache bytes that decode streams (the pages' deployments keep
+ * the KV cache in 8 bits: "不用高显存卡也能跑！..." q8_0 KV in llama.cpp).
+ * FP8 caches need capacity % 4 == 0.  Supported by hyb_kv_append,
+ * hyb_attn_decode(_noalloc) and hyb_attn_layer_decode; hyb_attn_prefill and
+ * hyb_attn_layer_prefill with an FP8 cache return HYB_EUNSUPPORTED.
+ */
+#define HYB_KV_BF16 0
+#define HYB_KV_FP8 1
 
 /*
  * Resets a cache: len = 0, head = head0[b] (host array, NULL = all 0),

@@ -326,6 +326,39 @@ def attention_layer_decode(hidden, w_qkv, w_gate, w_o, qpos, hist_k, hist_v, his
 
 
 # ---------------------------------------------------------------------------
+# FP8 (e4m3) KV rows
+# ---------------------------------------------------------------------------
+E4M3_MAX = 448.0
+
+
+def quantize_e4m3_rows(x):
+    """Per-row FP8 e4m3 quantization of KV rows (the 8-bit KV cache the pages'
+    deployments use: [LAPTOP] / [12GB] q8_0 KV cache; the e4m3 format and a
+    per-row scale are this library's reading).  x [..., 256].
+    scale = amax / 448 (fp32); code = e4m3 round-to-nearest-even, saturating
+    at +-448, of x * (448 / amax) computed in fp32, as the kernel does (the
+    code is an integer decided by floating point, so both sides decide it in
+    fp32).  A zero row has scale 0 and zero codes.
+    Returns (codes uint8 [..., 256], scale float32 [...])."""
+    import torch
+    x32 = np.asarray(x, dtype=np.float32)
+    amax = np.abs(x32).max(axis=-1)
+    safe = np.where(amax > 0, amax, np.float32(1.0)).astype(np.float32)
+    inv = np.where(amax > 0, np.float32(E4M3_MAX) / safe, np.float32(0.0)).astype(np.float32)
+    scaled = np.clip(x32 * inv[..., None], -E4M3_MAX, E4M3_MAX).astype(np.float32)
+    codes = torch.from_numpy(np.ascontiguousarray(scaled)).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    scale = (amax / np.float32(E4M3_MAX)).astype(np.float32)
+    return codes, scale
+
+
+def dequantize_e4m3_rows(codes, scale):
+    """code value (e4m3) * scale, in float64."""
+    import torch
+    vals = torch.from_numpy(np.ascontiguousarray(codes)).view(torch.float8_e4m3fn).to(torch.float64).numpy()
+    return vals * np.asarray(scale, dtype=np.float64)[..., None]
+
+
+# ---------------------------------------------------------------------------
 # KV caches: linear (full layers) and the 512-slot ring (sliding layers)
 # ---------------------------------------------------------------------------
 def linear_slots(length: int, n_new: int) -> np.ndarray:

@@ -418,3 +418,32 @@ def test_layer_decode_equals_last_row_of_layer_prefill(lt):
     hv = qkv[:, 5120:].reshape(T - 1, 4, 256)
     got = O.attention_layer_decode(hidden[:, T - 1], w_qkv, w_gate, w_o, [T - 1], [hk], [hv], [np.arange(T - 1)], lt)
     np.testing.assert_allclose(got[0], full[0, T - 1], rtol=1e-10, atol=1e-12)
+
+
+def test_e4m3_quantizer_known_values_and_bounds():
+    """e4m3: 1 sign, 4 exponent (bias 7), 3 mantissa bits, max 448, smallest
+    subnormal 2^-9; round to nearest even; saturating at +-448."""
+    # a row whose amax is 448 keeps representable values exactly (scale 1)
+    row = np.zeros(256)
+    row[:8] = [448.0, -448.0, 1.0, 1.125, 0.015625, 2 ** -9, -3.25, 0.0]
+    codes, scale = O.quantize_e4m3_rows(row)
+    assert scale == np.float32(1.0)
+    # bit patterns: 448 = 0 1111 110; 1.0 = 0 0111 000; 1.125 = 0 0111 001;
+    # 2^-6 = 0 0001 000; 2^-9 = 0 0000 001 (subnormal); -3.25 = 1 1000 101
+    assert codes[:8].tolist() == [0x7E, 0xFE, 0x38, 0x39, 0x08, 0x01, 0xC5, 0x00]
+    np.testing.assert_array_equal(O.dequantize_e4m3_rows(codes, scale)[:8], row[:8])
+    # halfway cases go to even: 1.0625 lies between 1.0 (even code) and 1.125
+    c2, _ = O.quantize_e4m3_rows(np.concatenate([[448.0, 1.0625, 1.1875], np.zeros(253)]))
+    assert c2[1] == 0x38 and c2[2] == 0x3A
+    # random rows: relative error of normal values <= 2^-4 (half of a 3-bit ulp); amax exact
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((64, 256)) * rng.uniform(0.01, 100, size=(64, 1))
+    c, s = O.quantize_e4m3_rows(x)
+    d = O.dequantize_e4m3_rows(c, s)
+    x32 = x.astype(np.float32).astype(np.float64)
+    normal = np.abs(x32) >= (2 ** -6) * (np.abs(x32).max(-1, keepdims=True) / 448)
+    assert np.all(np.abs(d - x32)[normal] <= 2 ** -4 * np.abs(x32)[normal] * (1 + 1e-6))
+    np.testing.assert_allclose(np.abs(d).max(-1), np.abs(x32).max(-1), rtol=1e-6)
+    # a zero row: scale 0, codes 0
+    cz, sz = O.quantize_e4m3_rows(np.zeros(256))
+    assert sz == 0 and not cz.any()
