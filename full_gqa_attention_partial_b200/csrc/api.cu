@@ -150,6 +150,40 @@ hyb_status make_q_map(CUtensorMap* m, const void* base, uint64_t T, uint64_t bat
   return HYB_OK;
 }
 
+// FP8 cache maps: codes {256, capacity, 4, B} uint8 with 128-dim x 64-row
+// boxes (128-byte swizzle), scales {capacity, 4, B} fp32 with 64-row boxes.
+hyb_status cache_maps_fp8(const hyb_kv_cache* c, CUtensorMap* mk, CUtensorMap* mv, CUtensorMap* mks,
+                          CUtensorMap* mvs) {
+  auto enc = encode_fn();
+  if (!enc) return fail(HYB_EUNSUPPORTED, "cuTensorMapEncodeTiled is not available from the driver");
+  const uint64_t cap = (uint64_t)c->capacity;
+  cuuint64_t dims[4] = {(cuuint64_t)kD, cap, (cuuint64_t)kHkv, (cuuint64_t)c->batch};
+  cuuint64_t strides[3] = {(cuuint64_t)kD, cap * kD, cap * kD * kHkv};
+  cuuint32_t box[4] = {128, 64, 1, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  void* bases[2] = {c->k, c->v};
+  CUtensorMap* maps[2] = {mk, mv};
+  for (int i = 0; i < 2; ++i) {
+    CUresult r = enc(maps[i], CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, bases[i], dims, strides, box, estr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(HYB_ECUDA, "cuTensorMapEncodeTiled(FP8 cache) failed with CUresult %d", (int)r);
+  }
+  cuuint64_t sdims[3] = {cap, (cuuint64_t)kHkv, (cuuint64_t)c->batch};
+  cuuint64_t sstrides[2] = {cap * 4, cap * 4 * kHkv};
+  cuuint32_t sbox[3] = {64, 1, 1};
+  cuuint32_t sestr[3] = {1, 1, 1};
+  void* sbases[2] = {c->k_scale, c->v_scale};
+  CUtensorMap* smaps[2] = {mks, mvs};
+  for (int i = 0; i < 2; ++i) {
+    CUresult r = enc(smaps[i], CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, sbases[i], sdims, sstrides, sbox, sestr,
+                     CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_NONE,
+                     CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(HYB_ECUDA, "cuTensorMapEncodeTiled(FP8 scales) failed with CUresult %d", (int)r);
+  }
+  return HYB_OK;
+}
+
 hyb_status check_cache(const hyb_kv_cache* c) {
   if (!c) return fail(HYB_EINVAL, "cache is NULL");
   if (c->type != HYB_SLIDING && c->type != HYB_FULL) return fail(HYB_EINVAL, "cache type %d invalid", c->type);
@@ -553,7 +587,6 @@ hyb_status decode_impl(const void* q, int64_t q_stride, bool q_rotated, const vo
   if (s != HYB_OK) return s;
   if (!q || !out) return fail(HYB_EINVAL, "q and out must be non-NULL");
   if (layer_type != c->type) return fail(HYB_ESHAPE, "layer_type %d differs from the cache type %d", layer_type, c->type);
-  if (c->kv_dtype != HYB_KV_BF16) return fail(HYB_EUNSUPPORTED, "decode of FP8 caches is not built yet");
   if (!aligned16(q) || !aligned16(out)) return fail(HYB_EALIGN, "q and out must be 16-byte aligned");
   if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
   if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u)) return fail(HYB_EALIGN, "pos must be 4-byte aligned");
@@ -567,7 +600,10 @@ hyb_status decode_impl(const void* q, int64_t q_stride, bool q_rotated, const vo
   if ((s = ensure_device()) != HYB_OK) return s;
 
   DecodeHost d;
-  if ((s = cache_maps(c, &d.tm_k, &d.tm_v, 64, 64)) != HYB_OK) return s;
+  d.fp8 = c->kv_dtype == HYB_KV_FP8 ? 1 : 0;
+  if ((s = d.fp8 ? cache_maps_fp8(c, &d.tm_k, &d.tm_v, &d.tm_ks, &d.tm_vs) : cache_maps(c, &d.tm_k, &d.tm_v, 64, 64)) !=
+      HYB_OK)
+    return s;
   d.q = q;
   d.q_stride = q_stride;
   d.q_rotated = q_rotated ? 1 : 0;
@@ -602,7 +638,6 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
   if (s != HYB_OK) return s;
   if (!q || !out) return fail(HYB_EINVAL, "q and out must be non-NULL");
   if (layer_type != c->type) return fail(HYB_ESHAPE, "layer_type %d differs from the cache type %d", layer_type, c->type);
-  if (c->kv_dtype != HYB_KV_BF16) return fail(HYB_EUNSUPPORTED, "decode of FP8 caches is not built yet");
   if (!aligned16(q) || !aligned16(out)) return fail(HYB_EALIGN, "q and out must be 16-byte aligned");
   if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
   if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u)) return fail(HYB_EALIGN, "pos must be 4-byte aligned");
@@ -623,7 +658,10 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
 
   DecodeHost d;
-  if ((s = cache_maps(c, &d.tm_k, &d.tm_v, 64, 64)) != HYB_OK) return s;
+  d.fp8 = c->kv_dtype == HYB_KV_FP8 ? 1 : 0;
+  if ((s = d.fp8 ? cache_maps_fp8(c, &d.tm_k, &d.tm_v, &d.tm_ks, &d.tm_vs) : cache_maps(c, &d.tm_k, &d.tm_v, 64, 64)) !=
+      HYB_OK)
+    return s;
   d.q = q;
   d.gate = gate;
   d.pos = pos;

@@ -15,6 +15,13 @@
 // the warp-level MMA keeps the instruction count per key low.
 //
 // Warps 0-3 consume (16 keys each per stage), warp 4 issues the TMA loads.
+//
+// FP8 caches (e4m3 codes + one fp32 scale per key row): a stage holds the
+// codes (half the bytes) and the 64 keys' scales; each consumer warp first
+// widens its own 16 key rows of K and V to bf16 (exact: every e4m3 value is
+// a bf16 value) in the layout the bf16 path reads, releases the stage, and
+// then runs the same MMAs, with the K scale applied to the scores and the V
+// scale folded into P.
 #include <mutex>
 
 #include "common.cuh"
@@ -28,6 +35,12 @@ constexpr int kDecTileBytes = kDecKeys * kD * 2;     // 32 KB (K or V)
 constexpr int kDecStageBytes = 2 * kDecTileBytes;    // K + V
 constexpr int kDecThreads = 160;
 constexpr int kBoxBytes = kDecKeys * 128;            // one 64-dim box of 64 keys
+// FP8 layout inside DecSmem::stage: per stage K codes (2 boxes of 128 dims),
+// V codes, K scales, V scales; then the widened bf16 K and V tiles.
+constexpr int kDec8TileBytes = kDecKeys * kD;        // 16 KB of codes
+constexpr int kDec8Box = kDecKeys * 128;             // 128 dims x 64 keys
+constexpr int kDec8StageBytes = 2 * kDec8TileBytes + 2 * kDecKeys * 4 + 512;   // padded to 1 KB multiples
+constexpr int kDec8Wide = kDecStages * kDec8StageBytes;                         // widened tiles start here
 
 struct DecSmem {
   // stage buffers first (1024-byte aligned base)
@@ -42,6 +55,8 @@ struct DecSmem {
 };
 
 size_t decode_smem_bytes() { return sizeof(DecSmem) + 1024; }
+static_assert(kDec8StageBytes % 1024 == 0, "FP8 stage must keep 1 KB alignment");
+static_assert(kDec8Wide + 2 * kDecTileBytes <= kDecStages * kDecStageBytes, "FP8 stages + widened tiles must fit");
 
 struct DecArgs {
   const __nv_bfloat16* q;
@@ -55,9 +70,10 @@ struct DecArgs {
   int n_splits;
 };
 
-template <bool FULL>
+template <bool FULL, bool FP8>
 __global__ void __launch_bounds__(kDecThreads, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
+                        const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                         DecArgs a) {
   extern __shared__ uint8_t smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -95,10 +111,24 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       for (int i = 0; i < n_stages; ++i) {
         const int slot = i % kDecStages;
         if (i >= kDecStages && !mbar_wait(&sm.empty[slot], ((i / kDecStages) - 1) & 1)) break;
+        const int key = k0 + i * kDecKeys;
+        if (FP8) {
+          mbar_arrive_expect_tx(&sm.full[slot], 2 * kDec8TileBytes + 2 * kDecKeys * 4);
+          const uint32_t kdst = smem_u32(sm.stage[0]) + slot * kDec8StageBytes;
+          const uint32_t vdst = kdst + kDec8TileBytes;
+#pragma unroll
+          for (int box = 0; box < 2; ++box) {
+            tma_load_4d(kdst + box * kDec8Box, &tm_k, &sm.full[slot], box * 128, key, kvh, b);
+            tma_load_4d(vdst + box * kDec8Box, &tm_v, &sm.full[slot], box * 128, key, kvh, b);
+          }
+          tma_load_3d(vdst + kDec8TileBytes, &tm_ks, &sm.full[slot], key, kvh, b);
+          tma_load_3d(vdst + kDec8TileBytes + kDecKeys * 4, &tm_vs, &sm.full[slot], key, kvh, b);
+          issued = i + 1;
+          continue;
+        }
         mbar_arrive_expect_tx(&sm.full[slot], kDecStageBytes);
         const uint32_t kdst = smem_u32(sm.stage[slot]);
         const uint32_t vdst = kdst + kDecTileBytes;
-        const int key = k0 + i * kDecKeys;
 #pragma unroll
         for (int box = 0; box < 4; ++box) {
           tma_load_4d(kdst + box * kBoxBytes, &tm_k, &sm.full[slot], box * 64, key, kvh, b);
@@ -166,8 +196,46 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   for (int i = 0; i < n_stages; ++i) {
     const int slot = i % kDecStages;
     if (!mbar_wait(&sm.full[slot], (i / kDecStages) & 1)) break;
-    const uint32_t kbase = smem_u32(sm.stage[slot]);
-    const uint32_t vbase = kbase + kDecTileBytes;
+    uint32_t kbase = smem_u32(sm.stage[slot]);
+    uint32_t vbase = kbase + kDecTileBytes;
+    float ksc[4] = {1.f, 1.f, 1.f, 1.f}, vsc[4] = {1.f, 1.f, 1.f, 1.f};   // scales of this thread's keys
+    if (FP8) {
+      // widen this warp's 16 key rows of K and V to bf16 (the bf16 path's layout)
+      uint8_t* st8 = sm.stage[0] + slot * kDec8StageBytes;
+      uint8_t* wide = sm.stage[0] + kDec8Wide;
+#pragma unroll
+      for (int kv = 0; kv < 2; ++kv) {
+        const uint8_t* src_t = st8 + kv * kDec8TileBytes;
+        uint8_t* dst_t = wide + kv * kDecTileBytes;
+#pragma unroll
+        for (int it = 0; it < 8; ++it) {
+          const int job = lane + 32 * it;
+          const uint32_t r = warp * 16 + (job >> 4);
+          const int cs = job & 15;                         // 16-dim chunk: dims 16 cs .. 16 cs + 15
+          const uint4 cw = *reinterpret_cast<const uint4*>(src_t + (cs >> 3) * kDec8Box +
+                                                           ((r * 128u) | ((((uint32_t)cs & 7u) ^ (r & 7u)) << 4)));
+          const int d0 = 16 * cs;
+          const uint4 lo = make_uint4(e4m3x2_to_bf16x2(cw.x & 0xFFFFu), e4m3x2_to_bf16x2(cw.x >> 16),
+                                      e4m3x2_to_bf16x2(cw.y & 0xFFFFu), e4m3x2_to_bf16x2(cw.y >> 16));
+          const uint4 hi = make_uint4(e4m3x2_to_bf16x2(cw.z & 0xFFFFu), e4m3x2_to_bf16x2(cw.z >> 16),
+                                      e4m3x2_to_bf16x2(cw.w & 0xFFFFu), e4m3x2_to_bf16x2(cw.w >> 16));
+          *reinterpret_cast<uint4*>(dst_t + (d0 >> 6) * kBoxBytes + sw128_offset(r, (d0 & 63) * 2)) = lo;
+          *reinterpret_cast<uint4*>(dst_t + ((d0 + 8) >> 6) * kBoxBytes + sw128_offset(r, ((d0 + 8) & 63) * 2)) = hi;
+        }
+      }
+      const float* kscale = reinterpret_cast<const float*>(st8 + 2 * kDec8TileBytes);
+      const float* vscale = kscale + kDecKeys;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const int kl = warp * 16 + (e >> 1) * 8 + 2 * c + (e & 1);
+        ksc[e] = kscale[kl];
+        vsc[e] = vscale[kl];
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[slot]);   // the codes have been read
+      kbase = smem_u32(wide);
+      vbase = kbase + kDecTileBytes;
+    }
 
     // ---- scores of 16 keys x 4 heads ----
     float acc[2][4];
@@ -195,7 +263,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const int tg = sm.tags[key];
         ok = tg >= 0 && tg <= qseq && qseq - tg < kWindow;
       }
-      sv[e] = ok ? acc[e >> 1][e & 1] * scale_log2 : -INFINITY;
+      sv[e] = ok ? acc[e >> 1][e & 1] * ksc[e] * scale_log2 : -INFINITY;
     }
     float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
@@ -212,8 +280,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       o[n][0] *= alpha;
       o[n][1] *= alpha;
     }
-    const uint32_t pa0 = pack_bf16(pv[0], pv[1]);
-    const uint32_t pa2 = pack_bf16(pv[2], pv[3]);
+    const uint32_t pa0 = pack_bf16(pv[0] * vsc[0], pv[1] * vsc[1]);
+    const uint32_t pa2 = pack_bf16(pv[2] * vsc[2], pv[3] * vsc[3]);
     // ---- O += P V over 256 dims ----
 #pragma unroll
     for (int i2 = 0; i2 < 16; ++i2) {
@@ -225,7 +293,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       mma_16816(o[2 * i2 + 1], pa0, 0u, pa2, 0u, r2, r3);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&sm.empty[slot]);
+    if (!FP8 && lane == 0) mbar_arrive(&sm.empty[slot]);
   }
 
   // ---------------- merge the 4 warps, write the split's partial ----------------
@@ -336,10 +404,14 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
   const dim3 grid(h.n_splits, kHkv, h.B);
   const size_t smem = decode_smem_bytes();
   profile_before(st);
-  if (full)
-    decode_split_kernel<true><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, a);
+  if (full && h.fp8)
+    decode_split_kernel<true, true><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_ks, h.tm_vs, a);
+  else if (full)
+    decode_split_kernel<true, false><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_k, h.tm_v, a);
+  else if (h.fp8)
+    decode_split_kernel<false, true><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_ks, h.tm_vs, a);
   else
-    decode_split_kernel<false><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, a);
+    decode_split_kernel<false, false><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_k, h.tm_v, a);
   profile_after(st);
   count_launch();
   cudaError_t e = cudaGetLastError();
@@ -393,9 +465,14 @@ cudaError_t decode_noalloc_scratch(void** ptr, size_t* bytes) {
 
 cudaError_t decode_set_smem_attr() {
   const int smem = (int)decode_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(decode_split_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_split_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_split_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(decode_split_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return e;
 }
 
 }  // namespace hyb

@@ -86,6 +86,8 @@ size_t prefill_smem_bytes();
 // ---- decode (decode.cu) -------------------------------------------------------
 struct DecodeHost {
   CUtensorMap tm_k, tm_v;      // 4-D maps over the cache {256, capacity, 4, B}
+  CUtensorMap tm_ks, tm_vs;    // FP8 caches: 3-D maps over the scales {capacity, 4, B}
+  int fp8 = 0;                 // 1: k / v hold e4m3 codes (tm_k / tm_v are uint8 maps, 128-dim boxes)
   const void* q = nullptr;     // [B][16][256] rows q_stride elements apart
   int64_t q_stride = 16 * 256;
   int q_rotated = 0;           // 1: q is already rotated (the kernel skips RoPE)

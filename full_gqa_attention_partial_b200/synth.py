@@ -78,6 +78,27 @@ def fill_cache_randn_(k_cache: torch.Tensor, v_cache: torch.Tensor, n_tokens: in
             v_cache[b, h, :n].copy_(randn_bf16((n, D), g, k_cache.device))
 
 
+def fill_cache_fp8_(k_codes: torch.Tensor, v_codes: torch.Tensor, k_scale: torch.Tensor, v_scale: torch.Tensor,
+                    n_tokens: int, seed: int):
+    """Fills slots [0, n_tokens) of FP8 caches (codes uint8 [B, KVH, cap, D],
+    scales fp32 [B, KVH, cap]) with random e4m3 bit patterns -- random sign,
+    exponent field 5..9, random 3-bit mantissa (values 0.25 .. 7.5) -- and
+    random scales in [0.1, 0.3]: stored values of magnitude ~0.03 .. 2, no
+    NaN codes.  They stand for rows written by earlier appends."""
+    g = generator(seed, k_codes.device)
+    B, KVH, cap, D = k_codes.shape
+    n = int(n_tokens)
+    dev = k_codes.device
+    for b in range(B):
+        for h in range(KVH):
+            for codes, scale in ((k_codes, k_scale), (v_codes, v_scale)):
+                sign = torch.randint(0, 2, (n, D), generator=g, device=dev, dtype=torch.int32) << 7
+                expo = torch.randint(5, 10, (n, D), generator=g, device=dev, dtype=torch.int32) << 3
+                mant = torch.randint(0, 8, (n, D), generator=g, device=dev, dtype=torch.int32)
+                codes[b, h, :n].copy_((sign | expo | mant).to(torch.uint8))
+                scale[b, h, :n].copy_(0.1 + 0.2 * torch.rand(n, generator=g, device=dev))
+
+
 def ring_offset(seed: int) -> int:
     """Random starting slot of a sliding layer's ring write head, in [0, 512)."""
     g = generator(seed, "cpu")

@@ -63,3 +63,74 @@ def test_fp8_cache_rejected_by_prefill(lib):
     cache = lib.KVCache(O.FULL, 1, capacity=128, kv_dtype=lib.KV_FP8)
     with pytest.raises(lib.HybError):
         lib.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], None, O.FULL, cache=cache)
+
+
+def _fp8_full(lib, B, L, cap, seed):
+    c = lib.KVCache(O.FULL, B, capacity=cap, kv_dtype=lib.KV_FP8)
+    synth.fill_cache_fp8_(c.k, c.v, c.k_scale, c.v_scale, L, seed)
+    c.len.fill_(L)
+    return c
+
+
+def _fp8_ring(lib, B, L, seed, head0):
+    c = lib.KVCache(O.SLIDING, B, kv_dtype=lib.KV_FP8, head0=[head0] * B)
+    synth.fill_cache_fp8_(c.k, c.v, c.k_scale, c.v_scale, 512, seed)
+    idx = torch.arange(L - 512, L, dtype=torch.int64, device="cuda")
+    tag = torch.full((512,), -1, dtype=torch.int32, device="cuda")
+    tag[(head0 + idx) % 512] = idx.to(torch.int32)
+    c.tag.copy_(tag.expand(B, 512))
+    c.len.fill_(L)
+    c.head.fill_((head0 + L) % 512)
+    return c
+
+
+def _snapshot(c, rows):
+    """Host copy of the seeded history rows [B][n, 4, 256] (dequantized by the oracle)."""
+    kc = c.k[:, :, rows].cpu().numpy()
+    vc = c.v[:, :, rows].cpu().numpy()
+    ks = c.k_scale[:, :, rows].cpu().numpy()
+    vs = c.v_scale[:, :, rows].cpu().numpy()
+    return (O.dequantize_e4m3_rows(kc, ks).transpose(0, 2, 1, 3), O.dequantize_e4m3_rows(vc, vs).transpose(0, 2, 1, 3))
+
+
+@pytest.mark.parametrize("lt", [O.FULL, O.SLIDING])
+@pytest.mark.parametrize("noalloc", [False, True])
+def test_fp8_decode_matches_oracle_on_dequantized_cache(lib, lt, noalloc):
+    """Decode over an FP8 cache equals the attention of the dequantized keys
+    and values: the seeded history (snapshot before any library call) plus
+    the new token, which the oracle rotates, rounds to bf16 and quantizes."""
+    B = 4
+    L = 3000 if lt == O.FULL else 1200
+    if lt == O.FULL:
+        cap = L + 4
+        c = _fp8_full(lib, B, L, cap, seed=41)
+        hk, hv = _snapshot(c, np.arange(L))
+        hidx = np.arange(L)
+        max_len = cap
+    else:
+        r = synth.ring_offset(42)
+        c = _fp8_ring(lib, B, L, seed=43, head0=r)
+        hidx = np.arange(L - 511, L)                     # the window after one more token
+        hk, hv = _snapshot(c, (r + hidx) % 512)
+        max_len = 512
+    x = synth.decode_query(B, seed=44 + lt, device="cuda")
+    lib.hyb_kv_append(c, x["k"], x["v"])
+    if noalloc:
+        out = lib.hyb_attn_decode_noalloc(x["q"], x["gate"], c, max_len=max_len)
+    else:
+        out = lib.hyb_attn_decode(x["q"], x["gate"], c, max_len=max_len)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    n = L + 1
+    k_rot = O.to_bf16(O.rope_layer(f64(x["k"]), np.full((B, 1), n - 1), lt)[:, 0])      # [B, 4, 256]
+    kq, ksc = O.quantize_e4m3_rows(k_rot)
+    vq, vsc = O.quantize_e4m3_rows(f64(x["v"])[:, 0])
+    kn, vn = O.dequantize_e4m3_rows(kq, ksc), O.dequantize_e4m3_rows(vq, vsc)
+    keys = [np.concatenate([hk[b], kn[b][None]]) for b in range(B)]
+    vals = [np.concatenate([hv[b], vn[b][None]]) for b in range(B)]
+    idx = [np.append(hidx, n - 1)] * B
+    ref = O.decode(f64(x["q"]), f64(x["gate"]), [n - 1] * B, keys, vals, idx, lt)
+    got = f64(out)
+    max_abs = float(np.abs(got - ref).max())
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    assert max_abs <= 2e-2 and rel <= 5e-3, f"max_abs {max_abs:.3e} rel_l2 {rel:.3e}"
