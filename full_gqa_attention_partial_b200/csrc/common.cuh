@@ -164,15 +164,26 @@ __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const void* tmap,
       "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
-// Two e4m3 codes (low byte first) -> two bf16 in one word (low half first);
-// exact: every e4m3 value is a bf16 value.
-__device__ __forceinline__ uint32_t e4m3x2_to_bf16x2(uint32_t two_codes) {
-  uint32_t h;
-  asm("{\n\t.reg .b16 c;\n\tcvt.u16.u32 c, %1;\n\tcvt.rn.f16x2.e4m3x2 %0, c;\n\t}" : "=r"(h) : "r"(two_codes));
-  const float lo = __half2float(__ushort_as_half((unsigned short)(h & 0xFFFFu)));
-  const float hi = __half2float(__ushort_as_half((unsigned short)(h >> 16)));
-  return pack_bf16(lo, hi);
+// e4m3 -> bf16 by integer bit moves, scaled by 2^-120: the e4m3 sign,
+// exponent and mantissa bits land in the bf16 sign, the low four exponent
+// bits and the top three mantissa bits, so the code 2^(e-7) (1 + m/8) becomes
+// the bf16 2^(e-127) (1 + m/8) and the subnormal code m 2^-9 the bf16
+// subnormal m 2^-129, both exact.  A word of four codes (byte 0 lowest)
+// gives two bf16 pairs: bytes 0 and 2 (low half first), and bytes 1 and 3.
+__device__ __forceinline__ uint32_t e4m3_b02_bf16x2(uint32_t w) {
+  return ((w << 8) & 0x80008000u) | ((w << 4) & 0x07F007F0u);
 }
+__device__ __forceinline__ uint32_t e4m3_b13_bf16x2(uint32_t w) {
+  return (w & 0x80008000u) | ((w >> 4) & 0x07F007F0u);
+}
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
+constexpr float kE4m3WideScale = 1.329227995784916e36f;   // 2^120
+constexpr float kE4m3PScale = 18446744073709551616.f;      // 2^64
+constexpr float kE4m3OutScale = 72057594037927936.f;       // 2^56
 
 // TMA: 4-D tiled store from shared memory (bulk group); rows outside the
 // tensor are not written.
@@ -431,14 +442,21 @@ __device__ __forceinline__ void ldsm_x4_t(uint32_t saddr, uint32_t& r0, uint32_t
                : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
                : "r"(saddr));
 }
-// D = A(16x16, rows g and g+8) * B(16x8) + C, bf16 in, fp32 accumulate.
+// D = A(16x16, rows g and g+8) * B(16x8) + C, bf16 in, fp32 accumulate
+// (registers only, so the compiler may schedule it freely).
 __device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                           uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
       "{%0, %1, %2, %3};"
       : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
       : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// Transpose of an 8x8 b16 matrix held one row per 4 lanes (two elements each).
+__device__ __forceinline__ uint32_t movmatrix_t(uint32_t x) {
+  uint32_t d;
+  asm volatile("movmatrix.sync.aligned.m8n8.trans.b16 %0, %1;" : "=r"(d) : "r"(x));
+  return d;
 }
 
 // Byte offset of element (row, col) inside a TMA box of 128-byte rows with

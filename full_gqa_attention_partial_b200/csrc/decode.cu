@@ -10,18 +10,28 @@
 // 第二板斧").
 //
 // The per-key work (4 heads x 256 dims, scores and P.V) runs on mma.sync
-// m16n8k16 with the 4 query heads as the M rows (rows 4..15 zero): at about
-// 4 flop per byte the kernel is bound by HBM, not by the tensor pipe, and
-// the warp-level MMA keeps the instruction count per key low.
+// m16n8k16 in transposed form: S^T[16 keys x 8 heads] = K Q^T puts a warp's
+// 16 keys on the M rows and the group's 4 query heads on half of the N
+// columns, the probabilities are turned into the B operand by movmatrix,
+// and O^T[256 dims x 8 heads] += V^T P^T.  Half the columns idle instead of
+// three quarters of the rows with the heads on M, so a key costs half the
+// MMAs and the output accumulator half the registers.  At about 4 flop per
+// byte the kernel is bound by HBM, not by the tensor pipe.
 //
 // Warps 0-3 consume (16 keys each per stage), warp 4 issues the TMA loads.
 //
 // FP8 caches (e4m3 codes + one fp32 scale per key row): a stage holds the
-// codes (half the bytes) and the 64 keys' scales; each consumer warp first
-// widens its own 16 key rows of K and V to bf16 (exact: every e4m3 value is
-// a bf16 value) in the layout the bf16 path reads, releases the stage, and
-// then runs the same MMAs, with the K scale applied to the scores and the V
-// scale folded into P.
+// codes (half the bytes) and the 64 keys' scales, five stages deep.  Each
+// lane loads its own codes straight into registers (conflict-free chunk
+// orders below), releases the stage, and widens them to bf16 fragments with
+// integer bit moves (the value times 2^-120).  The contraction over dims is
+// free to take the dims in any order as long as Q's fragments follow the
+// same order, which lets a lane pair codes 0/2 and 1/3 of a word.  The K
+// scale is applied to the scores after the softmax scale has taken back the
+// 2^-120; the V scale (times 2^64) is folded into P and the remaining 2^56
+// goes onto the split's output.  P then stays below the bf16 maximum for any
+// V row of amax up to 448 * 2^64, and the products P V stay far above the
+// fp32 subnormal range.
 #include <mutex>
 
 #include "common.cuh"
@@ -30,33 +40,49 @@
 namespace hyb {
 
 constexpr int kDecKeys = 64;                         // keys per stage
-constexpr int kDecStages = 3;
+constexpr int kDecStages = 3;                        // bf16 stages
 constexpr int kDecTileBytes = kDecKeys * kD * 2;     // 32 KB (K or V)
 constexpr int kDecStageBytes = 2 * kDecTileBytes;    // K + V
 constexpr int kDecThreads = 160;
 constexpr int kBoxBytes = kDecKeys * 128;            // one 64-dim box of 64 keys
-// FP8 layout inside DecSmem::stage: per stage K codes (2 boxes of 128 dims),
-// V codes, K scales, V scales; then the widened bf16 K and V tiles.
+// FP8 stage: K codes (2 boxes of 128 dims), V codes, K scales, V scales.
+constexpr int kDec8Stages = 5;
 constexpr int kDec8TileBytes = kDecKeys * kD;        // 16 KB of codes
 constexpr int kDec8Box = kDecKeys * 128;             // 128 dims x 64 keys
 constexpr int kDec8StageBytes = 2 * kDec8TileBytes + 2 * kDecKeys * 4 + 512;   // padded to 1 KB multiples
-constexpr int kDec8Wide = kDecStages * kDec8StageBytes;                         // widened tiles start here
+constexpr int kDecRingBytes = kDecStages * kDecStageBytes;
+constexpr int kDecMaxStages = kDec8Stages;
 
 struct DecSmem {
-  // stage buffers first (1024-byte aligned base)
-  uint8_t stage[kDecStages][kDecStageBytes];
+  // stage ring first (1024-byte aligned base): kDecStages bf16 stages or kDec8Stages FP8 stages
+  uint8_t ring[kDecRingBytes];
   float merge_o[4][4][kD];      // [warp][head][dim]
   float merge_m[4][4];
   float merge_l[4][4];
   __nv_bfloat16 qs[4][kD];      // rotated queries of the group
   int32_t tags[kWindow];
-  uint64_t full[kDecStages];
-  uint64_t empty[kDecStages];
+  uint64_t full[kDecMaxStages];
+  uint64_t empty[kDecMaxStages];
 };
 
 size_t decode_smem_bytes() { return sizeof(DecSmem) + 1024; }
 static_assert(kDec8StageBytes % 1024 == 0, "FP8 stage must keep 1 KB alignment");
-static_assert(kDec8Wide + 2 * kDecTileBytes <= kDecStages * kDecStageBytes, "FP8 stages + widened tiles must fit");
+static_assert(kDec8Stages * kDec8StageBytes <= kDecRingBytes, "FP8 stages must fit the ring");
+
+// Chunk orders of the FP8 loads.  A 16-byte load of lanes 4t..4t+7 (rows
+// 2t, 2t+1; q = 0..3) is conflict-free when the four lanes of a row read
+// 16-byte slots whose indexes differ in their upper two bits (the 128-byte
+// swizzle XORs the slot with the row).  K: lane q covers 64 dims of box
+// q / 2, chunk dec8_kchunk(q, j) at step j.  V: lane r covers chunk r of
+// both boxes (dims 16 r .. 16 r + 15 of each 128), whose parity alternates
+// with the row.
+__device__ __forceinline__ int dec8_kchunk(int q, int j) {
+  return 2 * ((q & 1) + 2 * ((j & 1) ^ (q >> 1))) + (j >> 1);
+}
+// Dim of row m of MMA block i (O^T rows) for the FP8 V fragments.
+__device__ __forceinline__ int dec8_vdim(int i, int m) {
+  return 128 * (i >> 3) + 16 * (m & 7) + 4 * ((i >> 1) & 3) + 2 * (i & 1) + (m >> 3);
+}
 
 struct DecArgs {
   const __nv_bfloat16* q;
@@ -78,6 +104,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int R = RopeCfg<FULL>::R;
+  constexpr int NST = FP8 ? kDec8Stages : kDecStages;
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -91,7 +118,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   const int n_stages = (k1 > k0 && L > 0) ? (k1 - k0 + kDecKeys - 1) / kDecKeys : 0;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kDecStages; ++s) {
+    for (int s = 0; s < NST; ++s) {
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 4);
     }
@@ -109,12 +136,12 @@ __global__ void __launch_bounds__(kDecThreads, 1)
       prefetch_tmap(&tm_v);
       int issued = 0;
       for (int i = 0; i < n_stages; ++i) {
-        const int slot = i % kDecStages;
-        if (i >= kDecStages && !mbar_wait(&sm.empty[slot], ((i / kDecStages) - 1) & 1)) break;
+        const int slot = i % NST;
+        if (i >= NST && !mbar_wait(&sm.empty[slot], ((i / NST) - 1) & 1)) break;
         const int key = k0 + i * kDecKeys;
         if (FP8) {
           mbar_arrive_expect_tx(&sm.full[slot], 2 * kDec8TileBytes + 2 * kDecKeys * 4);
-          const uint32_t kdst = smem_u32(sm.stage[0]) + slot * kDec8StageBytes;
+          const uint32_t kdst = smem_u32(sm.ring) + slot * kDec8StageBytes;
           const uint32_t vdst = kdst + kDec8TileBytes;
 #pragma unroll
           for (int box = 0; box < 2; ++box) {
@@ -127,7 +154,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
           continue;
         }
         mbar_arrive_expect_tx(&sm.full[slot], kDecStageBytes);
-        const uint32_t kdst = smem_u32(sm.stage[slot]);
+        const uint32_t kdst = smem_u32(sm.ring) + slot * kDecStageBytes;
         const uint32_t vdst = kdst + kDecTileBytes;
 #pragma unroll
         for (int box = 0; box < 4; ++box) {
@@ -137,8 +164,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         issued = i + 1;
       }
       // drain: never leave the CTA with copies still landing in shared memory
-      for (int i = max(0, issued - kDecStages); i < issued; ++i)
-        mbar_wait(&sm.full[i % kDecStages], (i / kDecStages) & 1);
+      for (int i = max(0, issued - NST); i < issued; ++i)
+        mbar_wait(&sm.full[i % NST], (i / NST) & 1);
     }
     return;
   }
@@ -177,137 +204,200 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");
 
-  const int g = lane >> 2, c = lane & 3;
-  // A fragments of the rotated queries: row g = head g (g < 4), zero rows otherwise
-  uint32_t qa0[16], qa2[16];
+  // Lane (r, q) = (lane / 4, lane % 4) in the m16n8k16 fragment layouts.
+  const int r = lane >> 2, q = lane & 3;
+  // B fragments of Q^T per 16-dim k-step: column r = head r (zero for r >= 4).
+  // bf16: k-step kk takes dims 16 kk .. 16 kk + 15 in order.  FP8: k-step
+  // 4 j + wd takes, for lane q, the 4 dims at 4 wd of the K chunk the lane
+  // loads at step j, paired 0/2 and 1/3 like the widened codes.
+  uint32_t qb[16][2];
+  {
+    const uint32_t* qrow = reinterpret_cast<const uint32_t*>(&sm.qs[r & 3][0]);
 #pragma unroll
-  for (int s = 0; s < 16; ++s) {
-    qa0[s] = (g < 4) ? *reinterpret_cast<const uint32_t*>(&sm.qs[g & 3][16 * s + 2 * c]) : 0u;
-    qa2[s] = (g < 4) ? *reinterpret_cast<const uint32_t*>(&sm.qs[g & 3][16 * s + 2 * c + 8]) : 0u;
+    for (int kk = 0; kk < 16; ++kk) {
+      uint32_t b0, b1;
+      if (FP8) {
+        const int d = 128 * (q >> 1) + 16 * dec8_kchunk(q, kk >> 2) + 4 * (kk & 3);
+        const uint32_t x = qrow[d >> 1], y = qrow[(d >> 1) + 1];
+        b0 = prmt(x, y, 0x5410u);
+        b1 = prmt(x, y, 0x7632u);
+      } else {
+        b0 = qrow[8 * kk + q];
+        b1 = qrow[8 * kk + q + 4];
+      }
+      qb[kk][0] = (r < 4) ? b0 : 0u;
+      qb[kk][1] = (r < 4) ? b1 : 0u;
+    }
   }
 
   const float scale_log2 = 0.0625f * 1.4426950408889634f;  // 1/sqrt(256) * log2(e)
-  float m_run = -INFINITY, l_part = 0.f;
-  float o[32][4];
+  const float score_scale = FP8 ? scale_log2 * kE4m3WideScale : scale_log2;
+  // running max and (lane-partial) sum for heads 2q and 2q + 1
+  float m_run[2] = {-INFINITY, -INFINITY}, l_part[2] = {0.f, 0.f};
+  float o[16][4];   // O^T block i: rows = dims, columns = heads 2q, 2q + 1
 #pragma unroll
-  for (int n = 0; n < 32; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+  for (int n = 0; n < 16; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
 
-  const int mi = lane >> 3, rr = lane & 7;
+  const int mi = lane >> 3, rr = lane & 7;     // ldmatrix: matrix and row this lane addresses
+  const int krow = warp * 16 + r;              // this lane's key rows: krow, krow + 8
   for (int i = 0; i < n_stages; ++i) {
-    const int slot = i % kDecStages;
-    if (!mbar_wait(&sm.full[slot], (i / kDecStages) & 1)) break;
-    uint32_t kbase = smem_u32(sm.stage[slot]);
-    uint32_t vbase = kbase + kDecTileBytes;
-    float ksc[4] = {1.f, 1.f, 1.f, 1.f}, vsc[4] = {1.f, 1.f, 1.f, 1.f};   // scales of this thread's keys
+    const int slot = i % NST;
+    if (!mbar_wait(&sm.full[slot], (i / NST) & 1)) break;
+    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};   // even / odd k-steps
+    float ksc[2] = {1.f, 1.f}, vsc[2] = {1.f, 1.f};                 // rows krow, krow + 8
+    uint4 vw[4][2];                                                 // FP8 V codes
+    uint32_t vbase = 0;
     if (FP8) {
-      // widen this warp's 16 key rows of K and V to bf16 (the bf16 path's layout)
-      uint8_t* st8 = sm.stage[0] + slot * kDec8StageBytes;
-      uint8_t* wide = sm.stage[0] + kDec8Wide;
+      const uint8_t* st8 = sm.ring + slot * kDec8StageBytes;
+      uint4 kw[2][4];
 #pragma unroll
-      for (int kv = 0; kv < 2; ++kv) {
-        const uint8_t* src_t = st8 + kv * kDec8TileBytes;
-        uint8_t* dst_t = wide + kv * kDecTileBytes;
+      for (int h = 0; h < 2; ++h) {
+        const int row = krow + 8 * h;
 #pragma unroll
-        for (int it = 0; it < 8; ++it) {
-          const int job = lane + 32 * it;
-          const uint32_t r = warp * 16 + (job >> 4);
-          const int cs = job & 15;                         // 16-dim chunk: dims 16 cs .. 16 cs + 15
-          const uint4 cw = *reinterpret_cast<const uint4*>(src_t + (cs >> 3) * kDec8Box +
-                                                           ((r * 128u) | ((((uint32_t)cs & 7u) ^ (r & 7u)) << 4)));
-          const int d0 = 16 * cs;
-          const uint4 lo = make_uint4(e4m3x2_to_bf16x2(cw.x & 0xFFFFu), e4m3x2_to_bf16x2(cw.x >> 16),
-                                      e4m3x2_to_bf16x2(cw.y & 0xFFFFu), e4m3x2_to_bf16x2(cw.y >> 16));
-          const uint4 hi = make_uint4(e4m3x2_to_bf16x2(cw.z & 0xFFFFu), e4m3x2_to_bf16x2(cw.z >> 16),
-                                      e4m3x2_to_bf16x2(cw.w & 0xFFFFu), e4m3x2_to_bf16x2(cw.w >> 16));
-          *reinterpret_cast<uint4*>(dst_t + (d0 >> 6) * kBoxBytes + sw128_offset(r, (d0 & 63) * 2)) = lo;
-          *reinterpret_cast<uint4*>(dst_t + ((d0 + 8) >> 6) * kBoxBytes + sw128_offset(r, ((d0 + 8) & 63) * 2)) = hi;
-        }
+        for (int j = 0; j < 4; ++j)
+          kw[h][j] = *reinterpret_cast<const uint4*>(st8 + (q >> 1) * kDec8Box + row * 128 +
+                                                     ((dec8_kchunk(q, j) ^ (row & 7)) << 4));
+      }
+#pragma unroll
+      for (int t = 0; t < 4; ++t) {
+        const int row = warp * 16 + 2 * q + (t & 1) + 8 * (t >> 1);
+#pragma unroll
+        for (int u = 0; u < 2; ++u)
+          vw[t][u] = *reinterpret_cast<const uint4*>(st8 + kDec8TileBytes + u * kDec8Box + row * 128 +
+                                                     ((r ^ (row & 7)) << 4));
       }
       const float* kscale = reinterpret_cast<const float*>(st8 + 2 * kDec8TileBytes);
       const float* vscale = kscale + kDecKeys;
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const int kl = warp * 16 + (e >> 1) * 8 + 2 * c + (e & 1);
-        ksc[e] = kscale[kl];
-        vsc[e] = vscale[kl];
+      for (int h = 0; h < 2; ++h) {
+        ksc[h] = kscale[krow + 8 * h];
+        vsc[h] = vscale[krow + 8 * h] * kE4m3PScale;
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sm.empty[slot]);   // the codes have been read
-      kbase = smem_u32(wide);
+      if (lane == 0) mbar_arrive(&sm.empty[slot]);   // every code is in registers
+      // ---- scores S^T = K Q^T ----
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const uint32_t w0[4] = {kw[0][j].x, kw[0][j].y, kw[0][j].z, kw[0][j].w};
+        const uint32_t w1[4] = {kw[1][j].x, kw[1][j].y, kw[1][j].z, kw[1][j].w};
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          const int kk = 4 * j + wd;
+          mma_16816(acc[kk & 1], e4m3_b02_bf16x2(w0[wd]), e4m3_b02_bf16x2(w1[wd]), e4m3_b13_bf16x2(w0[wd]),
+                    e4m3_b13_bf16x2(w1[wd]), qb[kk][0], qb[kk][1]);
+        }
+      }
+    } else {
+      const uint32_t kbase = smem_u32(sm.ring) + slot * kDecStageBytes;
       vbase = kbase + kDecTileBytes;
-    }
-
-    // ---- scores of 16 keys x 4 heads ----
-    float acc[2][4];
+      const uint32_t kr = warp * 16 + (mi & 1) * 8 + rr;
 #pragma unroll
-    for (int nb = 0; nb < 2; ++nb) acc[nb][0] = acc[nb][1] = acc[nb][2] = acc[nb][3] = 0.f;
-#pragma unroll
-    for (int s2 = 0; s2 < 8; ++s2) {
-#pragma unroll
-      for (int nb = 0; nb < 2; ++nb) {
-        const uint32_t kr = warp * 16 + nb * 8 + rr;
-        const uint32_t d = 32 * s2 + 8 * mi;
-        uint32_t r0, r1, r2, r3;
-        ldsm_x4(kbase + (d >> 6) * kBoxBytes + sw128_offset(kr, (d & 63) * 2), r0, r1, r2, r3);
-        mma_16816(acc[nb], qa0[2 * s2], 0u, qa2[2 * s2], 0u, r0, r1);
-        mma_16816(acc[nb], qa0[2 * s2 + 1], 0u, qa2[2 * s2 + 1], 0u, r2, r3);
+      for (int kk = 0; kk < 16; ++kk) {
+        const uint32_t d = 16 * kk + (mi >> 1) * 8;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(kbase + (d >> 6) * kBoxBytes + sw128_offset(kr, (d & 63) * 2), a0, a1, a2, a3);
+        mma_16816(acc[kk & 1], a0, a1, a2, a3, qb[kk][0], qb[kk][1]);
       }
     }
-    // ---- mask, online softmax (log2 domain) ----
-    float sv[4];
+    // ---- mask, online softmax (log2 domain) per head ----
+    // sv[h][e]: key row krow + 8 h, head 2 q + e
+    float sv[2][2];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      const int key = k0 + i * kDecKeys + warp * 16 + (e >> 1) * 8 + 2 * c + (e & 1);
+    for (int h = 0; h < 2; ++h) {
+      const int key = k0 + i * kDecKeys + krow + 8 * h;
       bool ok = key < k1;
       if (!FULL && ok) {
         const int tg = sm.tags[key];
         ok = tg >= 0 && tg <= qseq && qseq - tg < kWindow;
       }
-      sv[e] = ok ? acc[e >> 1][e & 1] * ksc[e] * scale_log2 : -INFINITY;
-    }
-    float mx = fmaxf(fmaxf(sv[0], sv[1]), fmaxf(sv[2], sv[3]));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 2));
-    const float m_new = fmaxf(m_run, mx);
-    const float alpha = (m_run == -INFINITY) ? 1.f : exp2f(m_run - m_new);
-    float pv[4];
 #pragma unroll
-    for (int e = 0; e < 4; ++e) pv[e] = (m_new == -INFINITY || g >= 4) ? 0.f : exp2f(sv[e] - m_new);
-    m_run = m_new;
-    l_part = l_part * alpha + (pv[0] + pv[1] + pv[2] + pv[3]);
-#pragma unroll
-    for (int n = 0; n < 32; ++n) {
-      o[n][0] *= alpha;
-      o[n][1] *= alpha;
+      for (int e = 0; e < 2; ++e) {
+        const float sc = acc[0][2 * h + e] + acc[1][2 * h + e];
+        // (score * scale) first: with FP8 it restores the widening's 2^-120 before the row scale
+        sv[h][e] = ok ? sc * score_scale * ksc[h] : -INFINITY;
+      }
     }
-    const uint32_t pa0 = pack_bf16(pv[0] * vsc[0], pv[1] * vsc[1]);
-    const uint32_t pa2 = pack_bf16(pv[2] * vsc[2], pv[3] * vsc[3]);
-    // ---- O += P V over 256 dims ----
+    float pv[2][2], alpha[2];
 #pragma unroll
-    for (int i2 = 0; i2 < 16; ++i2) {
-      const uint32_t kr = warp * 16 + (mi & 1) * 8 + rr;
-      const uint32_t d = 16 * i2 + (mi >> 1) * 8;
-      uint32_t r0, r1, r2, r3;
-      ldsm_x4_t(vbase + (d >> 6) * kBoxBytes + sw128_offset(kr, (d & 63) * 2), r0, r1, r2, r3);
-      mma_16816(o[2 * i2], pa0, 0u, pa2, 0u, r0, r1);
-      mma_16816(o[2 * i2 + 1], pa0, 0u, pa2, 0u, r2, r3);
+    for (int e = 0; e < 2; ++e) {
+      float mx = fmaxf(sv[0][e], sv[1][e]);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 4));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 8));
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+      const float m_new = fmaxf(m_run[e], mx);
+      alpha[e] = (m_run[e] == -INFINITY) ? 1.f : exp2f(m_run[e] - m_new);
+#pragma unroll
+      for (int h = 0; h < 2; ++h) pv[h][e] = (m_new == -INFINITY || q >= 2) ? 0.f : exp2f(sv[h][e] - m_new);
+      m_run[e] = m_new;
+      l_part[e] = l_part[e] * alpha[e] + (pv[0][e] + pv[1][e]);
     }
-    __syncwarp();
-    if (!FP8 && lane == 0) mbar_arrive(&sm.empty[slot]);
+#pragma unroll
+    for (int n = 0; n < 16; ++n) {
+      o[n][0] *= alpha[0];
+      o[n][1] *= alpha[1];
+      o[n][2] *= alpha[0];
+      o[n][3] *= alpha[1];
+    }
+    // P^T (keys x heads, C layout) -> B fragments (k = keys, n = heads)
+    const uint32_t pb0 = movmatrix_t(pack_bf16(pv[0][0] * vsc[0], pv[0][1] * vsc[0]));
+    const uint32_t pb1 = movmatrix_t(pack_bf16(pv[1][0] * vsc[1], pv[1][1] * vsc[1]));
+    // ---- O^T += V^T P^T over 256 dims ----
+    if (FP8) {
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint32_t w[4][4] = {{vw[0][u].x, vw[0][u].y, vw[0][u].z, vw[0][u].w},
+                                  {vw[1][u].x, vw[1][u].y, vw[1][u].z, vw[1][u].w},
+                                  {vw[2][u].x, vw[2][u].y, vw[2][u].z, vw[2][u].w},
+                                  {vw[3][u].x, vw[3][u].y, vw[3][u].z, vw[3][u].w}};
+#pragma unroll
+        for (int wd = 0; wd < 4; ++wd) {
+          // keys (2q, 2q+1) and (2q+8, 2q+9), dims 4 wd .. 4 wd + 3 of the lane's chunk
+          const uint32_t t0 = prmt(w[0][wd], w[1][wd], 0x5410u), t1 = prmt(w[0][wd], w[1][wd], 0x7632u);
+          const uint32_t t2 = prmt(w[2][wd], w[3][wd], 0x5410u), t3 = prmt(w[2][wd], w[3][wd], 0x7632u);
+          const int ib = 8 * u + 2 * wd;
+          mma_16816(o[ib], e4m3_b02_bf16x2(t0), e4m3_b13_bf16x2(t0), e4m3_b02_bf16x2(t2), e4m3_b13_bf16x2(t2), pb0,
+                    pb1);
+          mma_16816(o[ib + 1], e4m3_b02_bf16x2(t1), e4m3_b13_bf16x2(t1), e4m3_b02_bf16x2(t3),
+                    e4m3_b13_bf16x2(t3), pb0, pb1);
+        }
+      }
+    } else {
+      const uint32_t kr = warp * 16 + (mi >> 1) * 8 + rr;
+#pragma unroll
+      for (int ib = 0; ib < 16; ++ib) {
+        const uint32_t d = 16 * ib + (mi & 1) * 8;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4_t(vbase + (d >> 6) * kBoxBytes + sw128_offset(kr, (d & 63) * 2), a0, a1, a2, a3);
+        mma_16816(o[ib], a0, a1, a2, a3, pb0, pb1);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.empty[slot]);
+    }
   }
 
   // ---------------- merge the 4 warps, write the split's partial ----------------
-  float l_sum = l_part + __shfl_xor_sync(0xffffffffu, l_part, 1);
-  l_sum += __shfl_xor_sync(0xffffffffu, l_sum, 2);
-  if (g < 4) {
-    if (c == 0) {
-      sm.merge_m[warp][g] = m_run;
-      sm.merge_l[warp][g] = l_sum;
+#pragma unroll
+  for (int e = 0; e < 2; ++e) {
+    l_part[e] += __shfl_xor_sync(0xffffffffu, l_part[e], 4);
+    l_part[e] += __shfl_xor_sync(0xffffffffu, l_part[e], 8);
+    l_part[e] += __shfl_xor_sync(0xffffffffu, l_part[e], 16);
+  }
+  if (q < 2) {
+    if (r == 0) {
+#pragma unroll
+      for (int e = 0; e < 2; ++e) {
+        sm.merge_m[warp][2 * q + e] = m_run[e];
+        sm.merge_l[warp][2 * q + e] = l_part[e];
+      }
     }
 #pragma unroll
-    for (int n = 0; n < 32; ++n) {
-      sm.merge_o[warp][g][8 * n + 2 * c] = o[n][0];
-      sm.merge_o[warp][g][8 * n + 2 * c + 1] = o[n][1];
+    for (int n = 0; n < 16; ++n) {
+      const int d0 = FP8 ? dec8_vdim(n, r) : 16 * n + r;
+      const int d1 = FP8 ? dec8_vdim(n, r + 8) : 16 * n + 8 + r;
+      sm.merge_o[warp][2 * q][d0] = o[n][0];
+      sm.merge_o[warp][2 * q + 1][d0] = o[n][1];
+      sm.merge_o[warp][2 * q][d1] = o[n][2];
+      sm.merge_o[warp][2 * q + 1][d1] = o[n][3];
     }
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -330,7 +420,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
 #pragma unroll
         for (int e = 0; e < 8; ++e) res[e] += f * sm.merge_o[w][hh][d0 + e];
       }
-      const float inv = den > 0.f ? 1.f / den : 0.f;
+      // with FP8, P carried 2^64 and V 2^-120: the output takes back 2^56
+      const float inv = den > 0.f ? (FP8 ? kE4m3OutScale : 1.f) / den : 0.f;
 #pragma unroll
       for (int e = 0; e < 8; ++e) res[e] *= inv;
       lse = den > 0.f ? M + log2f(den) : -INFINITY;

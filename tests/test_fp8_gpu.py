@@ -134,3 +134,45 @@ def test_fp8_decode_matches_oracle_on_dequantized_cache(lib, lt, noalloc):
     max_abs = float(np.abs(got - ref).max())
     rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
     assert max_abs <= 2e-2 and rel <= 5e-3, f"max_abs {max_abs:.3e} rel_l2 {rel:.3e}"
+
+
+_FINITE = np.array([c for c in range(256) if c & 0x7F != 0x7F], dtype=np.uint8)   # every non-NaN code
+_SUBNORMAL = np.array([c for c in range(256) if c & 0x78 == 0], dtype=np.uint8)   # exponent field 0
+
+
+@pytest.mark.parametrize("case", ["every_code", "subnormal_only"])
+def test_fp8_decode_code_coverage(lib, case):
+    """Decode reads every finite e4m3 code, subnormals included, at row
+    scales from 1e-3 to 1e3 (values past 1e5): the widening keeps each code's
+    value and the scales reach the output without leaving the fp32 or bf16
+    range."""
+    B, L = 2, 700
+    cap = L + 4
+    rng = np.random.default_rng(7 if case == "every_code" else 8)
+    pool = _FINITE if case == "every_code" else _SUBNORMAL
+    c = lib.KVCache(O.FULL, B, capacity=cap, kv_dtype=lib.KV_FP8)
+    kc = rng.choice(pool, size=(B, 4, L, 256))
+    vc = rng.choice(pool, size=(B, 4, L, 256))
+    if case == "every_code":
+        ks = np.full((B, 4, L), 3e-3, np.float32)                        # key values up to 1.3
+        vs = (10.0 ** rng.uniform(-3, 3, size=(B, 4, L))).astype(np.float32)
+    else:
+        ks = np.full((B, 4, L), 100.0, np.float32)                       # subnormal codes are <= 7/512
+        vs = (10.0 ** rng.uniform(-1, 1, size=(B, 4, L))).astype(np.float32)
+    c.k[:, :, :L].copy_(torch.from_numpy(kc))
+    c.v[:, :, :L].copy_(torch.from_numpy(vc))
+    c.k_scale[:, :, :L].copy_(torch.from_numpy(ks))
+    c.v_scale[:, :, :L].copy_(torch.from_numpy(vs))
+    c.len.fill_(L)
+    x = synth.decode_query(B, seed=45, device="cuda")
+    lib.hyb_kv_append(c, x["k"], x["v"])
+    out = lib.hyb_attn_decode(x["q"], x["gate"], c, max_len=cap)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    hk, hv = _snapshot(c, np.arange(L + 1))            # history and the appended row, as stored
+    idx = [np.arange(L + 1)] * B
+    ref = O.decode(f64(x["q"]), f64(x["gate"]), [L] * B, list(hk), list(hv), idx, O.FULL)
+    got = f64(out)
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    assert np.isfinite(got).all()
+    assert rel <= 5e-3, f"rel_l2 {rel:.3e}"
