@@ -21,7 +21,8 @@
 // Warps 0-3 consume (16 keys each per stage), warp 4 issues the TMA loads.
 //
 // FP8 caches (e4m3 codes + one fp32 scale per key row): a stage holds the
-// codes (half the bytes) and the 64 keys' scales, five stages deep.  Each
+// codes (half the bytes) and the 64 keys' scales, three stages deep, and
+// two FP8 CTAs share an SM.  Each
 // lane loads its own codes straight into registers (conflict-free chunk
 // orders below), releases the stage, and widens them to bf16 fragments with
 // integer bit moves (the value times 2^-120).  The contraction over dims is
@@ -46,28 +47,33 @@ constexpr int kDecStageBytes = 2 * kDecTileBytes;    // K + V
 constexpr int kDecThreads = 160;
 constexpr int kBoxBytes = kDecKeys * 128;            // one 64-dim box of 64 keys
 // FP8 stage: K codes (2 boxes of 128 dims), V codes, K scales, V scales.
-constexpr int kDec8Stages = 5;
+// FP8 CTAs take half the shared memory, so two share an SM.
+constexpr int kDec8Stages = 3;
 constexpr int kDec8TileBytes = kDecKeys * kD;        // 16 KB of codes
 constexpr int kDec8Box = kDecKeys * 128;             // 128 dims x 64 keys
 constexpr int kDec8StageBytes = 2 * kDec8TileBytes + 2 * kDecKeys * 4 + 512;   // padded to 1 KB multiples
-constexpr int kDecRingBytes = kDecStages * kDecStageBytes;
-constexpr int kDecMaxStages = kDec8Stages;
 
+template <bool FP8>
 struct DecSmem {
-  // stage ring first (1024-byte aligned base): kDecStages bf16 stages or kDec8Stages FP8 stages
-  uint8_t ring[kDecRingBytes];
-  float merge_o[4][4][kD];      // [warp][head][dim]
+  static constexpr int kStages = FP8 ? kDec8Stages : kDecStages;
+  static constexpr int kRingBytes = FP8 ? kDec8Stages * kDec8StageBytes : kDecStages * kDecStageBytes;
+  // stage ring first (1024-byte aligned base); after the last stage it holds
+  // the warps' partial outputs, float [warp][head][dim]
+  uint8_t ring[kRingBytes];
   float merge_m[4][4];
   float merge_l[4][4];
   __nv_bfloat16 qs[4][kD];      // rotated queries of the group
   int32_t tags[kWindow];
-  uint64_t full[kDecMaxStages];
-  uint64_t empty[kDecMaxStages];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];
+  __device__ float (&merge_o())[4][4][kD] { return *reinterpret_cast<float(*)[4][4][kD]>(ring); }
 };
+static_assert(DecSmem<true>::kRingBytes >= 4 * 4 * kD * 4 && DecSmem<false>::kRingBytes >= 4 * 4 * kD * 4,
+              "the ring must hold the merge buffer");
 
-size_t decode_smem_bytes() { return sizeof(DecSmem) + 1024; }
+size_t decode_smem_bytes(bool fp8) { return (fp8 ? sizeof(DecSmem<true>) : sizeof(DecSmem<false>)) + 1024; }
+static_assert(2 * (sizeof(DecSmem<true>) + 1024 + 1024) <= 228 * 1024, "two FP8 CTAs must share an SM");
 static_assert(kDec8StageBytes % 1024 == 0, "FP8 stage must keep 1 KB alignment");
-static_assert(kDec8Stages * kDec8StageBytes <= kDecRingBytes, "FP8 stages must fit the ring");
 
 // Chunk orders of the FP8 loads.  A 16-byte load of lanes 4t..4t+7 (rows
 // 2t, 2t+1; q = 0..3) is conflict-free when the four lanes of a row read
@@ -97,14 +103,14 @@ struct DecArgs {
 };
 
 template <bool FULL, bool FP8>
-__global__ void __launch_bounds__(kDecThreads, 1)
+__global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                         const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs,
                         DecArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  DecSmem& sm = *reinterpret_cast<DecSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  DecSmem<FP8>& sm = *reinterpret_cast<DecSmem<FP8>*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int R = RopeCfg<FULL>::R;
-  constexpr int NST = FP8 ? kDec8Stages : kDecStages;
+  constexpr int NST = DecSmem<FP8>::kStages;
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
@@ -376,6 +382,8 @@ __global__ void __launch_bounds__(kDecThreads, 1)
   }
 
   // ---------------- merge the 4 warps, write the split's partial ----------------
+  // the merge buffer overlays the ring: every consumer warp must be done with its last stage
+  asm volatile("bar.sync 1, 128;" ::: "memory");
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     l_part[e] += __shfl_xor_sync(0xffffffffu, l_part[e], 4);
@@ -394,10 +402,10 @@ __global__ void __launch_bounds__(kDecThreads, 1)
     for (int n = 0; n < 16; ++n) {
       const int d0 = FP8 ? dec8_vdim(n, r) : 16 * n + r;
       const int d1 = FP8 ? dec8_vdim(n, r + 8) : 16 * n + 8 + r;
-      sm.merge_o[warp][2 * q][d0] = o[n][0];
-      sm.merge_o[warp][2 * q + 1][d0] = o[n][1];
-      sm.merge_o[warp][2 * q][d1] = o[n][2];
-      sm.merge_o[warp][2 * q + 1][d1] = o[n][3];
+      sm.merge_o()[warp][2 * q][d0] = o[n][0];
+      sm.merge_o()[warp][2 * q + 1][d0] = o[n][1];
+      sm.merge_o()[warp][2 * q][d1] = o[n][2];
+      sm.merge_o()[warp][2 * q + 1][d1] = o[n][3];
     }
   }
   asm volatile("bar.sync 1, 128;" ::: "memory");
@@ -418,7 +426,7 @@ __global__ void __launch_bounds__(kDecThreads, 1)
         const float f = exp2f(mw - M);
         den += f * sm.merge_l[w][hh];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) res[e] += f * sm.merge_o[w][hh][d0 + e];
+        for (int e = 0; e < 8; ++e) res[e] += f * sm.merge_o()[w][hh][d0 + e];
       }
       // with FP8, P carried 2^64 and V 2^-120: the output takes back 2^56
       const float inv = den > 0.f ? (FP8 ? kE4m3OutScale : 1.f) / den : 0.f;
@@ -493,7 +501,7 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
   a.part_lse = h.part_lse;
   a.n_splits = h.n_splits;
   const dim3 grid(h.n_splits, kHkv, h.B);
-  const size_t smem = decode_smem_bytes();
+  const size_t smem = decode_smem_bytes(h.fp8);
   profile_before(st);
   if (full && h.fp8)
     decode_split_kernel<true, true><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_ks, h.tm_vs, a);
@@ -555,14 +563,14 @@ cudaError_t decode_noalloc_scratch(void** ptr, size_t* bytes) {
 }
 
 cudaError_t decode_set_smem_attr() {
-  const int smem = (int)decode_smem_bytes();
+  const int smem = (int)decode_smem_bytes(false), smem8 = (int)decode_smem_bytes(true);
   cudaError_t e = cudaFuncSetAttribute(decode_split_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
     e = cudaFuncSetAttribute(decode_split_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(decode_split_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(decode_split_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem8);
   if (e == cudaSuccess)
-    e = cudaFuncSetAttribute(decode_split_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+    e = cudaFuncSetAttribute(decode_split_kernel<false, true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem8);
   return e;
 }
 

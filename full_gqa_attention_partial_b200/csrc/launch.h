@@ -105,6 +105,6 @@ int decode_num_splits(bool full, int B, int64_t max_len);
 // Address and size of the library's fixed decode scratch on the current
 // device (looked up on first use per device).
 cudaError_t decode_noalloc_scratch(void** ptr, size_t* bytes);
-size_t decode_smem_bytes();
+size_t decode_smem_bytes(bool fp8);
 
 }  // namespace hyb
