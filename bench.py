@@ -70,17 +70,20 @@ def layer_seed(base: int, i: int) -> int:
 # the capture's summary).  Reported as roofline.traffic only while the sources are
 # unchanged; otherwise null.
 TRAFFIC = {
-    "prefill_full_T32768": {"bytes": 2.173e9, "sha": "e1af5fc5ed4c8197",
+    "prefill_full_T32768": {"bytes": 2.173e9, "sha": "1a078391b3929273",
                             "sources": ["prefill.cu", "common.cuh"],
                             "capture": "profiles/prefill_kernel_full_T32768.md"},
-    "prefill_sliding_T32768": {"bytes": 0.6386e9, "sha": "e1af5fc5ed4c8197",
+    "prefill_sliding_T32768": {"bytes": 0.6386e9, "sha": "1a078391b3929273",
                                "sources": ["prefill.cu", "common.cuh"],
                                "capture": "profiles/prefill_kernel_sliding_T32768.md"},
-    # captured at 16 x 32768 tokens (2.153 GB); decode streams each cached byte
-    # once, so traffic scales with the tokens: x 8590491648 / 2147483648
-    "decode_full_B16_L131072": {"bytes": 2.153e9 * 8590491648 / 2147483648, "sha": "724f44ab245c48aa",
+    # captured at 16 x 32768 tokens; decode streams each cached byte once, so
+    # traffic scales with the tokens: x 8590491648 / 2147483648
+    "decode_full_B16_L131072": {"bytes": 2.1556e9 * 8590491648 / 2147483648, "sha": "46caad3ef3b376c7",
                                 "sources": ["decode.cu", "common.cuh"],
                                 "capture": "profiles/decode_split_kernel_full_B16_L32768.md"},
+    "decode_fp8_full_B16_L131072": {"bytes": 1.0970e9 * 8590491648 / 2147483648, "sha": "46caad3ef3b376c7",
+                                    "sources": ["decode.cu", "common.cuh"],
+                                    "capture": "profiles/decode_split_kernel_full_fp8_B16_L32768.md"},
 }
 
 
@@ -416,20 +419,26 @@ def bench_layer(hyb, args, peaks):
             "peak_source": f"{peaks['source']} bf16 burst"}
 
 
-def fill_full_cache(hyb, B: int, L: int, cap: int, seed: int):
+def fill_full_cache(hyb, B: int, L: int, cap: int, seed: int, fp8: bool = False):
     """Full-layer cache holding L random tokens (keys taken as already rotated)."""
     from full_gqa_attention_partial_b200 import synth
-    c = hyb.KVCache(FULL, B, capacity=cap)
-    synth.fill_cache_randn_(c.k, c.v, L, seed)
+    c = hyb.KVCache(FULL, B, capacity=cap, kv_dtype=hyb.KV_FP8 if fp8 else hyb.KV_BF16)
+    if fp8:
+        synth.fill_cache_fp8_(c.k, c.v, c.k_scale, c.v_scale, L, seed)
+    else:
+        synth.fill_cache_randn_(c.k, c.v, L, seed)
     c.len.fill_(L)
     return c
 
 
-def fill_ring_cache(hyb, B: int, L: int, seed: int, head0: int):
+def fill_ring_cache(hyb, B: int, L: int, seed: int, head0: int, fp8: bool = False):
     """A 512-slot ring in the state it has after L tokens: token i at slot (head0 + i) % 512."""
     from full_gqa_attention_partial_b200 import synth
-    c = hyb.KVCache(SLIDING, B, head0=[head0] * B)
-    synth.fill_cache_randn_(c.k, c.v, W, seed)
+    c = hyb.KVCache(SLIDING, B, head0=[head0] * B, kv_dtype=hyb.KV_FP8 if fp8 else hyb.KV_BF16)
+    if fp8:
+        synth.fill_cache_fp8_(c.k, c.v, c.k_scale, c.v_scale, W, seed)
+    else:
+        synth.fill_cache_randn_(c.k, c.v, W, seed)
     idx = torch.arange(max(0, L - W), L, dtype=torch.int64, device="cuda")
     tag = torch.full((W,), -1, dtype=torch.int32, device="cuda")
     tag[(head0 + idx) % W] = idx.to(torch.int32)
@@ -439,14 +448,19 @@ def fill_ring_cache(hyb, B: int, L: int, seed: int, head0: int):
     return c
 
 
-def bench_decode(hyb, args, peaks):
+# KV bytes decode streams per cached token per layer: K and V of 4 heads
+KV_TOKEN_BYTES = {False: 4096, True: 2 * 4 * 256 + 2 * 4 * 4}   # bf16; FP8 codes + fp32 row scales
+
+
+def bench_decode(hyb, args, peaks, fp8: bool = False):
     from full_gqa_attention_partial_b200 import synth
     B, L = 16, 131072
     n_steps = args.warmup + args.steps
     cap = L + n_steps + 1
+    cap += (-cap) % 4
     r = synth.ring_offset(2)
-    full = fill_full_cache(hyb, B, L, cap, seed=2)
-    ring = fill_ring_cache(hyb, B, L, seed=3, head0=r)
+    full = fill_full_cache(hyb, B, L, cap, seed=2, fp8=fp8)
+    ring = fill_ring_cache(hyb, B, L, seed=3, head0=r, fp8=fp8)
     qs = [synth.decode_query(B, seed=1000 + i, device="cuda") for i in range(n_steps)]
     ws = hyb.alloc_workspace(max(hyb.hyb_attn_decode_workspace_size(FULL, B, cap),
                                  hyb.hyb_attn_decode_workspace_size(SLIDING, B, W)))
@@ -477,33 +491,35 @@ def bench_decode(hyb, args, peaks):
     ring_ms = statistics.mean(kt[1::2])
     # KV bytes read per step: every cached token's K and V of 4 heads (4096 B per token per layer)
     lens = [L + args.warmup + i + 1 for i in range(args.steps)]
-    full_bytes = statistics.mean(B * n * 4096 for n in lens)
-    ring_bytes = B * W * 4096
+    tb = KV_TOKEN_BYTES[fp8]
+    full_bytes = statistics.mean(B * n * tb for n in lens)
+    ring_bytes = B * W * tb
     hbm = peaks["hbm_gbs"]
     achieved = full_bytes / (full_ms / 1e3) / 1e9
     return {
         "workload": "decode, batch 16, full-layer cache 131072 tokens + 512-slot ring (head at random "
-                    f"offset {r}), one full + one sliding layer per step, append + decode, seed 2",
+                    f"offset {r}), one full + one sliding layer per step, append + decode, seed 2"
+                    + (", FP8 e4m3 KV cache" if fp8 else ""),
         "tokens_per_s": B / (ms / 1e3), "ms_per_step": ms,
         "kv_gb_per_s": (full_bytes + ring_bytes) / (ms / 1e3) / 1e9,
         "frac_of_hbm": (full_bytes + ring_bytes) / (ms / 1e3) / 1e9 / hbm,
-        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<FULL>", "achieved": achieved, "peak": hbm,
+        "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<FULL, FP8>" if fp8 else "decode_split_kernel<FULL>", "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm, "peak_source": f"{peaks['source']} HBM copy",
                      "algorithmic_bytes_per_launch": full_bytes, "avg_launch_ms": full_ms,
-                     "traffic": traffic_of("decode_full_B16_L131072")},
+                     "traffic": traffic_of("decode_fp8_full_B16_L131072" if fp8 else "decode_full_B16_L131072")},
         "sliding_kernel": {"avg_launch_ms": ring_ms, "achieved_gbs": ring_bytes / (ring_ms / 1e3) / 1e9},
     }
 
 
-def bench_decode_1m(hyb, args, peaks):
+def bench_decode_1m(hyb, args, peaks, fp8: bool = False):
     """36 layers (27 rings, 9 full caches of ~1M tokens), batch 1, 64 steps of append + decode."""
     from full_gqa_attention_partial_b200 import synth
     n_steps = 64
     L0 = (1 << 20) - n_steps
     cap = 1 << 20
     r = synth.ring_offset(3)
-    fulls = [fill_full_cache(hyb, 1, L0, cap, seed=3 + 17 * i) for i in range(9)]
-    rings = [fill_ring_cache(hyb, 1, L0, seed=5000 + i, head0=r) for i in range(27)]
+    fulls = [fill_full_cache(hyb, 1, L0, cap, seed=3 + 17 * i, fp8=fp8) for i in range(9)]
+    rings = [fill_ring_cache(hyb, 1, L0, seed=5000 + i, head0=r, fp8=fp8) for i in range(27)]
     qs = [synth.decode_query(1, seed=9000 + i, device="cuda") for i in range(n_steps)]
     ws_full = hyb.alloc_workspace(hyb.hyb_attn_decode_workspace_size(FULL, 1, cap))
     ws_ring = hyb.alloc_workspace(hyb.hyb_attn_decode_workspace_size(SLIDING, 1, W))
@@ -532,8 +548,11 @@ def bench_decode_1m(hyb, args, peaks):
     torch.cuda.synchronize()
     assert hyb.hyb_device_error() == 0
     ms = ev0.elapsed_time(ev1) / n_steps
-    kv = statistics.mean(9 * 4096 * (L0 + i + 1) + 27 * 4096 * W for i in range(n_steps))
-    return {"workload": "36-layer decode (9 full caches ~1M tokens, 27 rings), batch 1, 64 steps, seed 3",
+    tb = KV_TOKEN_BYTES[fp8]
+    kv = statistics.mean(9 * tb * (L0 + i + 1) + 27 * tb * W for i in range(n_steps))
+    del fulls, rings
+    return {"workload": "36-layer decode (9 full caches ~1M tokens, 27 rings), batch 1, 64 steps, seed 3"
+                        + (", FP8 e4m3 KV caches" if fp8 else ""),
             "tokens_per_s": 1e3 / ms, "ms_per_step": ms, "kv_gb_per_s": kv / (ms / 1e3) / 1e9,
             "frac_of_hbm": kv / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
 
@@ -689,16 +708,18 @@ def run_case(hyb, args):
         work = B * flops(T, lt)
         unit = "TFLOP/s"
     else:
-        lt = FULL if args.case == "decode_full" else SLIDING
+        lt = FULL if args.case.startswith("decode_full") else SLIDING
+        fp8 = args.case.endswith("_fp8")
         B, L = args.batch, args.seq
         cap = L + args.steps + 2
-        c = fill_full_cache(hyb, B, L, cap, seed=2) if lt == FULL else fill_ring_cache(hyb, B, L, 3, 17)
+        cap += (-cap) % 4
+        c = fill_full_cache(hyb, B, L, cap, seed=2, fp8=fp8) if lt == FULL else fill_ring_cache(hyb, B, L, 3, 17, fp8=fp8)
         xq = synth.decode_query(B, seed=5, device="cuda")
         ml = cap if lt == FULL else W
         ws = hyb.alloc_workspace(hyb.hyb_attn_decode_workspace_size(lt, B, ml))
         out = torch.empty(B, H, D, dtype=torch.bfloat16, device="cuda")
         fn = lambda: hyb.hyb_attn_decode(xq["q"], xq["gate"], c, max_len=ml, out=out, workspace=ws)
-        work = B * min(L, cap if lt == FULL else W) * 4096
+        work = B * min(L, cap if lt == FULL else W) * KV_TOKEN_BYTES[fp8]
         unit = "GB/s"
     fn()
     torch.cuda.synchronize()
@@ -734,7 +755,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true", help="only the headline step (no sub-benchmarks)")
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows per layer for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="oracle rows per layer per reference step")
-    ap.add_argument("--case", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_sliding", "linear_qkv"],
+    ap.add_argument("--case", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_sliding", "decode_full_fp8",
+                                       "decode_sliding_fp8", "linear_qkv"],
                     default=None, help="time one kernel on a small configuration (profiling)")
     ap.add_argument("--seq", type=int, default=16384)
     ap.add_argument("--batch", type=int, default=1)
@@ -763,8 +785,11 @@ def main():
         extras["prefill_128k"] = bench_prefill_128k(hyb, args, peaks)
         extras["layer_prefill"] = bench_layer(hyb, args, peaks)
         extras["decode"] = bench_decode(hyb, args, peaks)
+        extras["decode_fp8"] = bench_decode(hyb, args, peaks, fp8=True)
         if args.decode_1m:
             extras["decode_1m"] = bench_decode_1m(hyb, args, peaks)
+            torch.cuda.empty_cache()
+            extras["decode_1m_fp8"] = bench_decode_1m(hyb, args, peaks, fp8=True)
         if args.chunked:
             extras["chunked_prefill"] = bench_chunked(hyb, args, peaks)
     clk = clocks.stop()
