@@ -30,6 +30,7 @@ KV_BF16 = 0
 KV_FP8 = 1
 DEV_ERR_CAPACITY = 1
 DEV_ERR_TIMEOUT = 2
+DEV_ERR_PAGE = 4
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_lib", "libhyb_attn.so")
@@ -62,6 +63,8 @@ class _Cache(ctypes.Structure):
         ("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("len", ctypes.c_void_p),
         ("head", ctypes.c_void_p), ("tag", ctypes.c_void_p),
         ("kv_dtype", ctypes.c_int32), ("k_scale", ctypes.c_void_p), ("v_scale", ctypes.c_void_p),
+        ("page_size", ctypes.c_int32), ("max_pages", ctypes.c_int32), ("n_pages", ctypes.c_int64),
+        ("block_table", ctypes.c_void_p),
     ]
 
 
@@ -147,28 +150,46 @@ class KVCache:
     Full layers: linear cache of `capacity` tokens.  Sliding layers: 512-slot
     ring; `head0` gives each sequence's starting write slot.  kv_dtype KV_FP8
     stores e4m3 codes (uint8) with one fp32 scale per (token, KV head) row.
+
+    Paged full layers: `page_size` > 0 (a multiple of 64), a pool of `n_pages`
+    pages (k / v [n_pages, 4, page_size, 256], scales [n_pages, 4, page_size])
+    and `block_table`, a device int32 [batch, max_pages] tensor owned by the
+    caller: token i of sequence b sits in pool page block_table[b, i //
+    page_size], row i % page_size; capacity = max_pages * page_size.
     """
 
     def __init__(self, layer_type: int, batch: int, capacity: int = WINDOW, device="cuda", head0=None,
-                 stream=None, kv_dtype: int = 0):
-        cap = WINDOW if layer_type == SLIDING else int(capacity)
+                 stream=None, kv_dtype: int = 0, page_size: int = 0, n_pages: int = 0, block_table=None):
+        paged = page_size > 0
+        if paged:
+            if block_table is None or block_table.dtype != torch.int32 or block_table.dim() != 2 \
+                    or not block_table.is_contiguous() or block_table.shape[0] != batch:
+                raise ValueError("a paged cache needs a contiguous int32 block_table [batch, max_pages]")
+            cap = int(page_size) * block_table.shape[1]
+        else:
+            cap = WINDOW if layer_type == SLIDING else int(capacity)
         self.layer_type = layer_type
         self.batch = batch
         self.capacity = cap
         self.kv_dtype = kv_dtype
+        self.page_size = int(page_size)
+        self.block_table = block_table
+        lead, rows = (int(n_pages), int(page_size)) if paged else (batch, cap)
         et = torch.uint8 if kv_dtype == KV_FP8 else torch.bfloat16
-        self.k = torch.empty(batch, N_KV_HEADS, cap, HEAD_DIM, dtype=et, device=device)
-        self.v = torch.empty(batch, N_KV_HEADS, cap, HEAD_DIM, dtype=et, device=device)
+        self.k = torch.empty(lead, N_KV_HEADS, rows, HEAD_DIM, dtype=et, device=device)
+        self.v = torch.empty(lead, N_KV_HEADS, rows, HEAD_DIM, dtype=et, device=device)
         self.len = torch.empty(batch, dtype=torch.int32, device=device)
         self.head = torch.empty(batch, dtype=torch.int32, device=device)
         self.tag = torch.empty(batch, WINDOW, dtype=torch.int32, device=device)
         self.k_scale = self.v_scale = None
         if kv_dtype == KV_FP8:
-            self.k_scale = torch.empty(batch, N_KV_HEADS, cap, dtype=torch.float32, device=device)
-            self.v_scale = torch.empty(batch, N_KV_HEADS, cap, dtype=torch.float32, device=device)
+            self.k_scale = torch.empty(lead, N_KV_HEADS, rows, dtype=torch.float32, device=device)
+            self.v_scale = torch.empty(lead, N_KV_HEADS, rows, dtype=torch.float32, device=device)
         self.c = _Cache(layer_type, batch, cap, self.k.data_ptr(), self.v.data_ptr(), self.len.data_ptr(),
                         self.head.data_ptr(), self.tag.data_ptr(), kv_dtype,
-                        _ptr(self.k_scale), _ptr(self.v_scale))
+                        _ptr(self.k_scale), _ptr(self.v_scale),
+                        self.page_size, block_table.shape[1] if paged else 0, int(n_pages) if paged else 0,
+                        _ptr(block_table))
         hyb_kv_cache_init(self, head0, stream)
 
     @property

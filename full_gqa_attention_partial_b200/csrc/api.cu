@@ -150,14 +150,39 @@ hyb_status make_q_map(CUtensorMap* m, const void* base, uint64_t T, uint64_t bat
   return HYB_OK;
 }
 
-// FP8 cache maps: codes {256, capacity, 4, B} uint8 with 128-dim x 64-row
-// boxes (128-byte swizzle), scales {capacity, 4, B} fp32 with 64-row boxes.
+// Rows per (page or sequence) and pages (or sequences) of a cache's storage:
+// a contiguous cache is [batch][4][capacity][256], a paged one
+// [n_pages][4][page_size][256].
+void cache_geom(const hyb_kv_cache* c, uint64_t* rows, uint64_t* batches) {
+  if (c->page_size > 0) {
+    *rows = (uint64_t)c->page_size;
+    *batches = (uint64_t)c->n_pages;
+  } else {
+    *rows = (uint64_t)c->capacity;
+    *batches = (uint64_t)c->batch;
+  }
+}
+
+PageMap page_map(const hyb_kv_cache* c) {
+  PageMap pm;
+  if (c->page_size > 0) {
+    pm.table = c->block_table;
+    pm.page = c->page_size;
+    pm.max_pages = c->max_pages;
+    pm.n_pages = (int)c->n_pages;
+  }
+  return pm;
+}
+
+// FP8 cache maps: codes {256, rows, 4, batches} uint8 with 128-dim x 64-row
+// boxes (128-byte swizzle), scales {rows, 4, batches} fp32 with 64-row boxes.
 hyb_status cache_maps_fp8(const hyb_kv_cache* c, CUtensorMap* mk, CUtensorMap* mv, CUtensorMap* mks,
                           CUtensorMap* mvs) {
   auto enc = encode_fn();
   if (!enc) return fail(HYB_EUNSUPPORTED, "cuTensorMapEncodeTiled is not available from the driver");
-  const uint64_t cap = (uint64_t)c->capacity;
-  cuuint64_t dims[4] = {(cuuint64_t)kD, cap, (cuuint64_t)kHkv, (cuuint64_t)c->batch};
+  uint64_t cap, nb;
+  cache_geom(c, &cap, &nb);
+  cuuint64_t dims[4] = {(cuuint64_t)kD, cap, (cuuint64_t)kHkv, (cuuint64_t)nb};
   cuuint64_t strides[3] = {(cuuint64_t)kD, cap * kD, cap * kD * kHkv};
   cuuint32_t box[4] = {128, 64, 1, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
@@ -169,7 +194,7 @@ hyb_status cache_maps_fp8(const hyb_kv_cache* c, CUtensorMap* mk, CUtensorMap* m
                      CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     if (r != CUDA_SUCCESS) return fail(HYB_ECUDA, "cuTensorMapEncodeTiled(FP8 cache) failed with CUresult %d", (int)r);
   }
-  cuuint64_t sdims[3] = {cap, (cuuint64_t)kHkv, (cuuint64_t)c->batch};
+  cuuint64_t sdims[3] = {cap, (cuuint64_t)kHkv, (cuuint64_t)nb};
   cuuint64_t sstrides[2] = {cap * 4, cap * 4 * kHkv};
   cuuint32_t sbox[3] = {64, 1, 1};
   cuuint32_t sestr[3] = {1, 1, 1};
@@ -198,6 +223,19 @@ hyb_status check_cache(const hyb_kv_cache* c) {
     if (!aligned16(c->k_scale) || !aligned16(c->v_scale)) return fail(HYB_EALIGN, "cache scales must be 16-byte aligned");
     if (c->capacity % 4) return fail(HYB_ESHAPE, "an FP8 cache needs capacity % 4 == 0, got %lld", (long long)c->capacity);
   }
+  if (c->page_size < 0) return fail(HYB_EINVAL, "page_size %d must be >= 0", c->page_size);
+  if (c->page_size > 0) {
+    if (c->type != HYB_FULL) return fail(HYB_EINVAL, "only full-layer caches can be paged");
+    if (c->page_size % 64) return fail(HYB_ESHAPE, "page_size %d must be a multiple of 64", c->page_size);
+    if (c->max_pages <= 0) return fail(HYB_EINVAL, "max_pages %d must be positive", c->max_pages);
+    if (c->n_pages <= 0 || c->n_pages > (int64_t)0x7fffffff)
+      return fail(HYB_EINVAL, "n_pages %lld out of range [1, 2^31)", (long long)c->n_pages);
+    if (c->capacity != (int64_t)c->max_pages * c->page_size)
+      return fail(HYB_ESHAPE, "capacity %lld must equal max_pages %d x page_size %d", (long long)c->capacity,
+                  c->max_pages, c->page_size);
+    if (!c->block_table) return fail(HYB_EINVAL, "a paged cache needs a block_table");
+    if (reinterpret_cast<uintptr_t>(c->block_table) & 3u) return fail(HYB_EALIGN, "block_table must be 4-byte aligned");
+  }
   if (c->type == HYB_SLIDING) {
     if (c->capacity != kWindow) return fail(HYB_ESHAPE, "sliding cache capacity must be 512, got %lld",
                                             (long long)c->capacity);
@@ -211,11 +249,12 @@ hyb_status check_cache(const hyb_kv_cache* c) {
 
 hyb_status cache_maps(const hyb_kv_cache* c, CUtensorMap* mk, CUtensorMap* mv, uint32_t k_box_rows,
                       uint32_t v_box_rows) {
-  const uint64_t row = kD * 2, head = (uint64_t)c->capacity * row, batch = head * kHkv;
-  hyb_status s =
-      make_kv_map(mk, c->k, (uint64_t)c->capacity, (uint64_t)c->batch, row, head, batch, k_box_rows, "cache K");
+  uint64_t rows, nb;
+  cache_geom(c, &rows, &nb);
+  const uint64_t row = kD * 2, head = rows * row, batch = head * kHkv;
+  hyb_status s = make_kv_map(mk, c->k, rows, nb, row, head, batch, k_box_rows, "cache K");
   if (s != HYB_OK) return s;
-  return make_kv_map(mv, c->v, (uint64_t)c->capacity, (uint64_t)c->batch, row, head, batch, v_box_rows, "cache V");
+  return make_kv_map(mv, c->v, rows, nb, row, head, batch, v_box_rows, "cache V");
 }
 
 cudaStream_t as_stream(void* s) { return reinterpret_cast<cudaStream_t>(s); }
@@ -324,7 +363,9 @@ hyb_status hyb_kv_cache_init(const hyb_kv_cache* c, const int32_t* head0, void* 
   if ((s = ensure_device()) != HYB_OK) return s;
   cudaStream_t st = as_stream(stream);
   const bool fp8 = c->kv_dtype == HYB_KV_FP8;
-  const size_t rows = (size_t)c->batch * kHkv * (size_t)c->capacity;
+  uint64_t grows, gbatches;
+  cache_geom(c, &grows, &gbatches);
+  const size_t rows = (size_t)gbatches * kHkv * (size_t)grows;
   const size_t kv_bytes = rows * kD * (fp8 ? 1 : 2);
   cudaError_t e;
   if ((e = cudaMemsetAsync(c->k, 0, kv_bytes, st)) != cudaSuccess) return cuda_fail(e, "zero cache K");
@@ -388,6 +429,7 @@ hyb_status append_impl(const hyb_kv_cache* c, const void* k, const void* v, int6
   r.fp8 = c->kv_dtype == HYB_KV_FP8 ? 1 : 0;
   r.dks = c->k_scale;
   r.dvs = c->v_scale;
+  r.pm = page_map(c);
   cudaError_t e = launch_rope_store(full, r, st);
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
   if ((e = launch_kv_commit(c->len, c->head, c->capacity, !full, c->batch, T, st)) != cudaSuccess)
@@ -504,8 +546,10 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
     r.dst_rows = cache->capacity;
     r.mode = 0;
     r.len = cache->len;
+    r.pm = page_map(cache);
     if ((e = launch_rope_store(true, r, st)) != cudaSuccess) return cuda_fail(e, "append launch");
     if ((s = cache_maps(cache, &ph.tm_k, &ph.tm_v, prefill_k_box_rows(), prefill_v_box_rows())) != HYB_OK) return s;
+    ph.pm = page_map(cache);
     ph.qbase = cache->len;
     ph.ctx_mode = 0;
     if ((e = launch_prefill(true, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
@@ -613,6 +657,7 @@ hyb_status decode_impl(const void* q, int64_t q_stride, bool q_rotated, const vo
   d.tag = c->type == HYB_SLIDING ? c->tag : nullptr;
   d.out = out;
   d.B = c->batch;
+  d.pm = page_map(c);
   d.n_splits = decode_num_splits(layer_type == HYB_FULL, c->batch, max_len);
   d.part_o = reinterpret_cast<float*>(workspace);
   d.part_lse = d.part_o + (size_t)c->batch * kHq * d.n_splits * kD;
@@ -669,6 +714,7 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
   d.tag = c->type == HYB_SLIDING ? c->tag : nullptr;
   d.out = out;
   d.B = c->batch;
+  d.pm = page_map(c);
   d.n_splits = splits;
   d.part_o = reinterpret_cast<float*>(scratch);
   d.part_lse = d.part_o + (size_t)c->batch * kHq * d.n_splits * kD;

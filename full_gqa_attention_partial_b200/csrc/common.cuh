@@ -8,6 +8,8 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "launch.h"
+
 namespace hyb {
 
 constexpr int kHq = 16;      // query heads
@@ -28,8 +30,32 @@ template <> struct RopeCfg<true>  { static constexpr int R = 64;  static constex
 static __device__ int g_dev_err = 0;
 constexpr int kErrCapacity = 1;
 constexpr int kErrTimeout = 2;
+constexpr int kErrPage = 4;
 
 __device__ __forceinline__ void raise_err(int bit) { atomicOr(&g_dev_err, bit); }
+
+// Row and batch coordinates of key row `row` of sequence b in a cache's TMA
+// map: the identity for contiguous caches; for paged caches the row within
+// the page and the pool page from the block table.  A table entry outside
+// the pool (or a row past the table) raises kErrPage and returns the page
+// coordinate -1, where tensor-map loads read zeros.  Rows of one 64-row
+// tile share a page (the page size is a multiple of 64).
+__device__ __forceinline__ void kv_coord(const PageMap& pm, int b, int row, int& crow, int& cpage) {
+  if (pm.page == 0) {
+    crow = row;
+    cpage = b;
+    return;
+  }
+  const int lp = row / pm.page;
+  int pp = -1;
+  if (lp < pm.max_pages) pp = __ldg(pm.table + (int64_t)b * pm.max_pages + lp);
+  if (pp < 0 || pp >= pm.n_pages) {
+    raise_err(kErrPage);
+    pp = -1;
+  }
+  crow = row - lp * pm.page;
+  cpage = pp;
+}
 
 // ---------------------------------------------------------------------------
 // RoPE angle: phi = pos * inv_freq in fp64, reduced to [-pi, pi] with a

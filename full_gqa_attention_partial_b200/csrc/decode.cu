@@ -100,6 +100,7 @@ struct DecArgs {
   float* part_o;
   float* part_lse;
   int n_splits;
+  PageMap pm;         // paged cache: maps over the pool {.., page, 4, n_pages}
 };
 
 template <bool FULL, bool FP8>
@@ -145,17 +146,19 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
         const int slot = i % NST;
         if (i >= NST && !mbar_wait(&sm.empty[slot], ((i / NST) - 1) & 1)) break;
         const int key = k0 + i * kDecKeys;
+        int crow, cpage;   // the stage's 64 keys lie within one page
+        kv_coord(a.pm, b, key, crow, cpage);
         if (FP8) {
           mbar_arrive_expect_tx(&sm.full[slot], 2 * kDec8TileBytes + 2 * kDecKeys * 4);
           const uint32_t kdst = smem_u32(sm.ring) + slot * kDec8StageBytes;
           const uint32_t vdst = kdst + kDec8TileBytes;
 #pragma unroll
           for (int box = 0; box < 2; ++box) {
-            tma_load_4d(kdst + box * kDec8Box, &tm_k, &sm.full[slot], box * 128, key, kvh, b);
-            tma_load_4d(vdst + box * kDec8Box, &tm_v, &sm.full[slot], box * 128, key, kvh, b);
+            tma_load_4d(kdst + box * kDec8Box, &tm_k, &sm.full[slot], box * 128, crow, kvh, cpage);
+            tma_load_4d(vdst + box * kDec8Box, &tm_v, &sm.full[slot], box * 128, crow, kvh, cpage);
           }
-          tma_load_3d(vdst + kDec8TileBytes, &tm_ks, &sm.full[slot], key, kvh, b);
-          tma_load_3d(vdst + kDec8TileBytes + kDecKeys * 4, &tm_vs, &sm.full[slot], key, kvh, b);
+          tma_load_3d(vdst + kDec8TileBytes, &tm_ks, &sm.full[slot], crow, kvh, cpage);
+          tma_load_3d(vdst + kDec8TileBytes + kDecKeys * 4, &tm_vs, &sm.full[slot], crow, kvh, cpage);
           issued = i + 1;
           continue;
         }
@@ -164,8 +167,8 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
         const uint32_t vdst = kdst + kDecTileBytes;
 #pragma unroll
         for (int box = 0; box < 4; ++box) {
-          tma_load_4d(kdst + box * kBoxBytes, &tm_k, &sm.full[slot], box * 64, key, kvh, b);
-          tma_load_4d(vdst + box * kBoxBytes, &tm_v, &sm.full[slot], box * 64, key, kvh, b);
+          tma_load_4d(kdst + box * kBoxBytes, &tm_k, &sm.full[slot], box * 64, crow, kvh, cpage);
+          tma_load_4d(vdst + box * kBoxBytes, &tm_v, &sm.full[slot], box * 64, crow, kvh, cpage);
         }
         issued = i + 1;
       }
@@ -500,6 +503,7 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
   a.part_o = h.part_o;
   a.part_lse = h.part_lse;
   a.n_splits = h.n_splits;
+  a.pm = h.pm;
   const dim3 grid(h.n_splits, kHkv, h.B);
   const size_t smem = decode_smem_bytes(h.fp8);
   profile_before(st);

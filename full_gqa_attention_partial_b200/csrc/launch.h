@@ -14,6 +14,16 @@ void count_launch();
 void profile_before(cudaStream_t st);
 void profile_after(cudaStream_t st);
 
+// Paged full-layer caches: token i of sequence b lives in pool page
+// table[b * max_pages + i / page], row i % page.  page == 0: contiguous
+// cache, token i of sequence b at row i of batch entry b.
+struct PageMap {
+  const int32_t* table = nullptr;   // device [B][max_pages]
+  int page = 0;
+  int max_pages = 0;
+  int n_pages = 0;
+};
+
 // ---- KV side (rope_kv.cu) --------------------------------------------------
 struct RopeStoreHost {
   const void* k = nullptr;
@@ -33,6 +43,7 @@ struct RopeStoreHost {
   int fp8 = 0;                 // 1: destination is an FP8 cache (codes + per-row scales)
   float* dks = nullptr;
   float* dvs = nullptr;
+  PageMap pm;                  // linear mode: paged destination cache
 };
 cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st);
 cudaError_t launch_ring_gather(const void* rk, const void* rv, const int32_t* len, const int32_t* head,
@@ -76,6 +87,7 @@ struct PrefillHost {
   int q_rotated = 0;           // 1: q is already rotated (the kernel skips RoPE)
   int B = 0, T = 0;
   int n_pairs = 74;            // persistent CTA pairs (SMs / 2)
+  PageMap pm;                  // K/V maps over a paged cache's pool
 };
 cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st);
 int prefill_k_box_rows();   // rows (keys) per TMA box of the K map
@@ -99,6 +111,7 @@ struct DecodeHost {
   float* part_o = nullptr;     // [B][16][S][256]
   float* part_lse = nullptr;   // [B][16][S]
   int B = 0, n_splits = 1;
+  PageMap pm;                  // maps over a paged cache's pool {256, page, 4, n_pages}
 };
 cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st);
 int decode_num_splits(bool full, int B, int64_t max_len);

@@ -97,6 +97,7 @@ struct PfArgs {
   int ctx_mode;
   int q_rotated;   // the queries arrive rotated (by the projection's epilogue)
   int B, T, n_mtiles;
+  PageMap pm;      // K/V maps over a paged cache's pool
 };
 
 // Load order shared by the K/V producer and the MMA issuer: step s (0 <= s
@@ -273,17 +274,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             if (g >= kSlots && !(ok = mbar_wait(&sm.empty[slot], ((g / kSlots) - 1) & 1))) break;
             if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
             const uint32_t dst = smem_u32(sm.slot[slot]);
-            const int row = (it.j_lo + tile) * kBN;
+            int row, cpage;   // the tile's 64 keys lie within one page
+            kv_coord(a.pm, it.b, (it.j_lo + tile) * kBN, row, cpage);
             if (is_k) {
 #pragma unroll
               for (int box = 0; box < 4; ++box)
                 tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row + kKBoxRows * (int)rank,
-                                 it.kvh, it.b);
+                                 it.kvh, cpage);
             } else {
 #pragma unroll
               for (int box = 0; box < 2; ++box)
                 tma_load_4d_pair(dst + box * kVBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * box, row, it.kvh,
-                                 it.b);
+                                 cpage);
             }
             ++g;
           }
@@ -631,6 +633,7 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   a.out = reinterpret_cast<__nv_bfloat16*>(h.out);
   a.qbase = h.qbase;
   a.ctx_mode = h.ctx_mode;
+  a.pm = h.pm;
   a.q_rotated = h.q_rotated;
   a.B = h.B;
   a.T = h.T;

@@ -45,6 +45,7 @@ struct RopeStoreArgs {
   int fp8;                  // 1: dk / dv hold e4m3 codes (1 byte), scales to dks / dvs
   float* dks;               // [B][4][dst_rows]
   float* dvs;
+  PageMap pm;               // linear mode, paged cache: destination [n_pages][4][page][256]
 };
 
 // One 256-dim row (one token, one KV head) held by a warp, 8 bf16 values per
@@ -108,7 +109,14 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
     } else {
       dst_row = a.dst_row_offset + t;
     }
-    const int64_t dst = (((int64_t)b * kHkv + kvh) * a.dst_rows + dst_row) * kD + d0;
+    int64_t row_id = ((int64_t)b * kHkv + kvh) * a.dst_rows + dst_row;   // row of the [..][4][rows] layout
+    if (a.mode == kDstLinear && a.pm.page != 0) {
+      int prow, ppage;
+      kv_coord(a.pm, b, (int)dst_row, prow, ppage);
+      if (ppage < 0) continue;   // bad block-table entry: raised, row skipped
+      row_id = ((int64_t)ppage * kHkv + kvh) * a.pm.page + prow;
+    }
+    const int64_t dst = row_id * kD + d0;
 
     uint4 kx = *reinterpret_cast<const uint4*>(a.k + src);
     if (!a.src_rotated) {
@@ -140,11 +148,10 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
       }
     }
     if (a.fp8) {
-      const int64_t row = ((int64_t)b * kHkv + kvh) * a.dst_rows + dst_row;
-      store_row_fp8(kx, reinterpret_cast<uint8_t*>(a.dk) + dst, a.dks + row, lane32);
+      store_row_fp8(kx, reinterpret_cast<uint8_t*>(a.dk) + dst, a.dks + row_id, lane32);
       if (a.v != nullptr)
-        store_row_fp8(*reinterpret_cast<const uint4*>(a.v + src), reinterpret_cast<uint8_t*>(a.dv) + dst, a.dvs + row,
-                      lane32);
+        store_row_fp8(*reinterpret_cast<const uint4*>(a.v + src), reinterpret_cast<uint8_t*>(a.dv) + dst,
+                      a.dvs + row_id, lane32);
       continue;
     }
     *reinterpret_cast<uint4*>(a.dk + dst) = kx;
@@ -224,6 +231,7 @@ cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st
   a.fp8 = h.fp8;
   a.dks = h.dks;
   a.dvs = h.dvs;
+  a.pm = h.pm;
   a.pos = h.pos;
   a.dk = reinterpret_cast<__nv_bfloat16*>(h.dk);
   a.dv = reinterpret_cast<__nv_bfloat16*>(h.dv);

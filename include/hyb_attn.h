@@ -72,6 +72,8 @@ typedef enum {
 /* Bits of the per-device error word (hyb_device_error). */
 #define HYB_DEV_ERR_CAPACITY 1  /* append past a full-layer cache's capacity: skipped */
 #define HYB_DEV_ERR_TIMEOUT 2   /* a pipeline wait exceeded its limit: output invalid */
+#define HYB_DEV_ERR_PAGE 4      /* a block-table entry outside [0, n_pages): the write
+                                   is skipped, the read gives zero keys and values */
 
 /*
  * KV cache of one layer for `batch` sequences.  All buffers are caller-owned
@@ -98,7 +100,31 @@ typedef struct hyb_kv_cache {
   int32_t kv_dtype;  /* HYB_KV_BF16 (0) or HYB_KV_FP8 (1) */
   float* k_scale;    /* HYB_KV_FP8 only: fp32 [batch][4][capacity], one scale per */
   float* v_scale;    /*   (token, KV head) row; NULL for HYB_KV_BF16 */
+  /* Paged storage (FULL caches only; page_size 0 = the contiguous layout above). */
+  int32_t page_size;      /* tokens per page, a positive multiple of 64 */
+  int32_t max_pages;      /* block_table entries per sequence; capacity == max_pages * page_size */
+  int64_t n_pages;        /* pages in the pool that k / v (and the scales) hold */
+  int32_t* block_table;   /* device int32 [batch][max_pages] */
 } hyb_kv_cache;
+
+/*
+ * Paged KV cache (FULL layers): a serving runtime holds one pool of pages for
+ * many sequences of mixed length and hands pages out as sequences grow
+ * ("不用高显存卡也能跑！..." §3.1 names paged KV caches among the serving
+ * engines' means).  With page_size P > 0:
+ *   k, v       : pool [n_pages][4][P][256] (bf16, or e4m3 codes),
+ *   k_scale, v_scale (FP8): [n_pages][4][P],
+ *   block_table: token i of sequence b lives in pool page
+ *                block_table[b * max_pages + i / P], row i % P.
+ * The library reads only the entries that cover [0, len) (and, for an
+ * append of T tokens, [len, len + T)); the others may hold anything, e.g.
+ * -1 for pages not handed out yet.  An entry it reads that lies outside
+ * [0, n_pages) raises HYB_DEV_ERR_PAGE: appends skip that row, attention
+ * reads zero keys and values there.  Pages may be shared by sequences for
+ * reading (a common prefix); two sequences that append into one page race.
+ * hyb_kv_cache_init zero-fills the whole pool.  P is a multiple of 64 so
+ * that every 64-key tile the kernels load lies within one page.
+ */
 
 /*
  * KV storage types.  HYB_KV_BF16: k / v hold bf16 [batch][4][capacity][256].

@@ -106,3 +106,30 @@ def test_workspace_sizes(hyb):
 def test_layer_schedule_binding(hyb):
     types = [hyb.layer_type(i) for i in range(36)]
     assert types.count(hyb.FULL) == 9 and types[3] == hyb.FULL and types[35] == hyb.FULL
+
+
+def test_paged_cache_checks_before_any_cuda_call(hyb):
+    """A paged cache (full layers only) must have a page size that is a
+    multiple of 64, capacity = max_pages x page_size, a pool and an aligned
+    block table; every violation returns before anything is enqueued."""
+    lib = hyb.load()
+    A = ctypes.c_void_p(0x10000)
+
+    def paged(lt=1, page=128, max_pages=8, cap=None, n_pages=16, table=0x6000):
+        cap = page * max_pages if cap is None else cap
+        return hyb._Cache(lt, 2, cap, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0, None, None,
+                          page, max_pages, n_pages, table)
+
+    def append(c):
+        return lib.hyb_kv_append(ctypes.byref(c), A, A, 1024, None, 4, None)
+
+    assert append(paged(lt=0, cap=512, page=64, max_pages=8)) == -1      # a sliding ring cannot be paged
+    assert append(paged(page=96)) == -2                                   # not a multiple of 64
+    assert append(paged(cap=1000)) == -2                                  # capacity != max_pages x page
+    assert append(paged(max_pages=0, cap=0)) == -1                        # no table entries
+    assert append(paged(n_pages=0)) == -1                                 # empty pool
+    assert append(paged(table=0)) == -1                                   # no block table
+    assert append(paged(table=0x6002)) == -3                              # misaligned block table
+    assert append(hyb._Cache(1, 2, 1024, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0, None, None,
+                             -64, 0, 0, None)) == -1                      # negative page size
+    assert "page" in lib.hyb_last_error().decode()
