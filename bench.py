@@ -15,10 +15,14 @@ The JSON line also carries:
                 copies inside the timed region;
   decode        decode, batch 16, 131072-token full-layer cache and a full
                 512-slot ring (head at a random offset): KV GB/s, % of HBM,
-                tokens/s;
+                tokens/s; decode_fp8 the same over e4m3 caches, decode_paged
+                with the full-layer cache in 64-token pages scattered over a pool;
   prefill_128k  one full layer, 131072 tokens: TFLOP/s and % of peak;
   layer_prefill the 4-layer group as whole layers (projections + attention);
-  decode_1m     (--decode-1m) 36-layer decode at 1M tokens: tokens/s;
+  decode_1m     (--decode-1m) 36-layer decode at 1M tokens: tokens/s (and
+                decode_1m_fp8 over e4m3 caches);
+  decode_1m_sharded (--decode-sharded, every rank) the same with the full
+                layers' history spread over the ranks;
   chunked_prefill (--chunked) 262144 tokens in 8192-token chunks, 36 layers;
   cpu_baseline  the fp64 oracle on a bounded sample of the same workload.
 
@@ -452,14 +456,34 @@ def fill_ring_cache(hyb, B: int, L: int, seed: int, head0: int, fp8: bool = Fals
 KV_TOKEN_BYTES = {False: 4096, True: 2 * 4 * 256 + 2 * 4 * 4}   # bf16; FP8 codes + fp32 row scales
 
 
-def bench_decode(hyb, args, peaks, fp8: bool = False):
+def fill_paged_cache(hyb, B: int, L: int, page: int, max_pages: int, seed: int, fp8: bool = False):
+    """Paged full-layer cache: each sequence's pages are scattered over a pool
+    of B x max_pages pages by a seeded permutation, L random tokens each."""
+    from full_gqa_attention_partial_b200 import synth
+    n_pages = B * max_pages
+    g = torch.Generator().manual_seed(seed)
+    table = torch.randperm(n_pages, generator=g).view(B, max_pages).to(torch.int32).cuda()
+    c = hyb.KVCache(FULL, B, kv_dtype=hyb.KV_FP8 if fp8 else hyb.KV_BF16, page_size=page, n_pages=n_pages,
+                    block_table=table)
+    if fp8:
+        synth.fill_cache_fp8_(c.k, c.v, c.k_scale, c.v_scale, page, seed)
+    else:
+        synth.fill_cache_randn_(c.k, c.v, page, seed)
+    c.len.fill_(L)
+    return c
+
+
+def bench_decode(hyb, args, peaks, fp8: bool = False, page: int = 0):
     from full_gqa_attention_partial_b200 import synth
     B, L = 16, 131072
     n_steps = args.warmup + args.steps
     cap = L + n_steps + 1
     cap += (-cap) % 4
+    if page:
+        cap += (-cap) % page
     r = synth.ring_offset(2)
-    full = fill_full_cache(hyb, B, L, cap, seed=2, fp8=fp8)
+    full = fill_paged_cache(hyb, B, L, page, cap // page, seed=2, fp8=fp8) if page else \
+        fill_full_cache(hyb, B, L, cap, seed=2, fp8=fp8)
     ring = fill_ring_cache(hyb, B, L, seed=3, head0=r, fp8=fp8)
     qs = [synth.decode_query(B, seed=1000 + i, device="cuda") for i in range(n_steps)]
     ws = hyb.alloc_workspace(max(hyb.hyb_attn_decode_workspace_size(FULL, B, cap),
@@ -499,14 +523,16 @@ def bench_decode(hyb, args, peaks, fp8: bool = False):
     return {
         "workload": "decode, batch 16, full-layer cache 131072 tokens + 512-slot ring (head at random "
                     f"offset {r}), one full + one sliding layer per step, append + decode, seed 2"
-                    + (", FP8 e4m3 KV cache" if fp8 else ""),
+                    + (", FP8 e4m3 KV cache" if fp8 else "")
+                    + (f", full-layer cache paged ({page}-token pages scattered over the pool)" if page else ""),
         "tokens_per_s": B / (ms / 1e3), "ms_per_step": ms,
         "kv_gb_per_s": (full_bytes + ring_bytes) / (ms / 1e3) / 1e9,
         "frac_of_hbm": (full_bytes + ring_bytes) / (ms / 1e3) / 1e9 / hbm,
         "roofline": {"bound": "hbm", "kernel": "decode_split_kernel<FULL, FP8>" if fp8 else "decode_split_kernel<FULL>", "achieved": achieved, "peak": hbm,
                      "unit": "GB/s", "frac": achieved / hbm, "peak_source": f"{peaks['source']} HBM copy",
                      "algorithmic_bytes_per_launch": full_bytes, "avg_launch_ms": full_ms,
-                     "traffic": traffic_of("decode_fp8_full_B16_L131072" if fp8 else "decode_full_B16_L131072")},
+                     "traffic": None if page else
+                     traffic_of("decode_fp8_full_B16_L131072" if fp8 else "decode_full_B16_L131072")},
         "sliding_kernel": {"avg_launch_ms": ring_ms, "achieved_gbs": ring_bytes / (ring_ms / 1e3) / 1e9},
     }
 
@@ -555,6 +581,61 @@ def bench_decode_1m(hyb, args, peaks, fp8: bool = False):
                         + (", FP8 e4m3 KV caches" if fp8 else ""),
             "tokens_per_s": 1e3 / ms, "ms_per_step": ms, "kv_gb_per_s": kv / (ms / 1e3) / 1e9,
             "frac_of_hbm": kv / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+
+
+def bench_decode_1m_sharded(hyb, args, peaks, d):
+    """The 36-layer 1M-token decode with each full layer's history spread over
+    the ranks (seqshard.py): rank r holds tokens history_range(L0, N, r) of
+    every full layer and the steps' tokens in round-robin blocks of 64; the
+    27 rings are whole on every rank.  A step is 9 x (partial attention, one
+    all-gather of 16 KB, merge) + 27 ring decodes on every rank."""
+    from full_gqa_attention_partial_b200 import seqshard, synth
+    n_steps = 64
+    L0 = (1 << 20) - n_steps
+    lo, hi = seqshard.history_range(L0, d.world, d.rank)
+    own_steps = sum(1 for s in range(n_steps) if (s // 64) % d.world == d.rank)
+    cap = hi - lo + own_steps
+    cap += (-cap) % 64
+    r = synth.ring_offset(3)
+    fulls = [fill_full_cache(hyb, 1, hi - lo, cap, seed=3 + 17 * i + 1000 * d.rank) for i in range(9)]
+    decs = [seqshard.SeqShardedDecoder(c, block=64) for c in fulls]
+    rings = [fill_ring_cache(hyb, 1, L0, seed=5000 + i, head0=r) for i in range(27)]
+    qs = [synth.decode_query(1, seed=9000 + i, device="cuda") for i in range(n_steps)]
+    ws_ring = hyb.alloc_workspace(hyb.hyb_attn_decode_workspace_size(SLIDING, 1, W))
+    out = torch.empty(1, H, D, dtype=torch.bfloat16, device="cuda")
+    pos = [torch.full((1,), L0 + i, dtype=torch.int32, device="cuda") for i in range(n_steps)]
+
+    def step(i):
+        x = qs[i]
+        fi = ri = 0
+        for layer in range(36):
+            if layer % 4 == 3:
+                decs[fi].step(x["q"], x["k"], x["v"], x["gate"], pos[i], i)
+                fi += 1
+            else:
+                c = rings[ri]
+                ri += 1
+                hyb.hyb_kv_append(c, x["k"], x["v"])
+                hyb.hyb_attn_decode(x["q"], x["gate"], c, max_len=W, out=out, workspace=ws_ring)
+
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    d.barrier()
+    torch.cuda.synchronize()
+    ev0.record()
+    for i in range(n_steps):
+        step(i)
+    ev1.record()
+    torch.cuda.synchronize()
+    d.barrier()
+    assert hyb.hyb_device_error() == 0
+    ms = d.max(ev0.elapsed_time(ev1) / n_steps)
+    kv = statistics.mean(9 * 4096 * (L0 + i + 1) + d.world * 27 * 4096 * W for i in range(n_steps))
+    del fulls, rings, decs
+    return {"workload": f"36-layer decode (9 full caches ~1M tokens spread over {d.world} GPU(s), 27 rings on "
+                        "each), batch 1, 64 steps, seed 3",
+            "tokens_per_s": 1e3 / ms, "ms_per_step": ms, "kv_gb_per_s": kv / (ms / 1e3) / 1e9,
+            "frac_of_hbm_per_gpu": kv / (ms / 1e3) / 1e9 / peaks["hbm_gbs"] / d.world}
 
 
 def bench_chunked(hyb, args, peaks):
@@ -753,6 +834,8 @@ def main():
     ap.add_argument("--chunked", action="store_true",
                     help="also run the 262144-token chunked prefill through 36 layers")
     ap.add_argument("--no-extras", action="store_true", help="only the headline step (no sub-benchmarks)")
+    ap.add_argument("--decode-sharded", action="store_true",
+                    help="also run the 1M-token decode with the full layers' history spread over the ranks")
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows per layer for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="oracle rows per layer per reference step")
     ap.add_argument("--case", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_sliding", "decode_full_fp8",
@@ -786,12 +869,16 @@ def main():
         extras["layer_prefill"] = bench_layer(hyb, args, peaks)
         extras["decode"] = bench_decode(hyb, args, peaks)
         extras["decode_fp8"] = bench_decode(hyb, args, peaks, fp8=True)
+        extras["decode_paged"] = bench_decode(hyb, args, peaks, page=64)
         if args.decode_1m:
             extras["decode_1m"] = bench_decode_1m(hyb, args, peaks)
             torch.cuda.empty_cache()
             extras["decode_1m_fp8"] = bench_decode_1m(hyb, args, peaks, fp8=True)
         if args.chunked:
             extras["chunked_prefill"] = bench_chunked(hyb, args, peaks)
+    if args.decode_sharded:   # every rank takes part (collectives)
+        torch.cuda.empty_cache()
+        extras["decode_1m_sharded"] = bench_decode_1m_sharded(hyb, args, peaks, dist)
     clk = clocks.stop()
     line = {
         "metric": METRIC, "value": main_res["value"], "unit": "TFLOP/s", "n_gpus": dist.world,

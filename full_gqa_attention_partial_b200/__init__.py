@@ -40,7 +40,8 @@ EXPORTED = (
     "hyb_attn_decode_workspace_size", "hyb_attn_decode", "hyb_device_error", "hyb_last_error",
     "hyb_launch_count", "hyb_profile_events", "hyb_profile_pairs_used", "hyb_attn_decode_noalloc",
     "hyb_selftest_wait_timeout", "hyb_linear", "hyb_attn_layer_prefill_workspace_size", "hyb_attn_layer_prefill",
-    "hyb_attn_layer_decode_workspace_size", "hyb_attn_layer_decode",
+    "hyb_attn_layer_decode_workspace_size", "hyb_attn_layer_decode", "hyb_attn_decode_partial",
+    "hyb_attn_decode_merge",
 )
 
 
@@ -106,6 +107,8 @@ def load(path: str = LIB_PATH):
     lib.hyb_attn_layer_decode_workspace_size.argtypes = [i32, i32, i64]
     lib.hyb_attn_layer_decode_workspace_size.restype = sz
     lib.hyb_attn_layer_decode.argtypes = [vp, vp, vp, vp, pc, i32, i64, vp, vp, sz, vp]
+    lib.hyb_attn_decode_partial.argtypes = [vp, vp, pc, i32, i64, vp, vp, vp, sz, vp]
+    lib.hyb_attn_decode_merge.argtypes = [vp, vp, i32, i32, vp, vp, vp]
     for name in ("hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill", "hyb_attn_decode",
                  "hyb_device_error"):
         getattr(lib, name).restype = ctypes.c_int
@@ -346,6 +349,46 @@ def hyb_attn_decode_noalloc(q, gate, cache: KVCache, pos=None, max_len: int = 0,
         out = torch.empty_like(q)
     _check(load().hyb_attn_decode_noalloc(_ptr(q), _ptr(gate), _ptr(pos), cache.ref, cache.layer_type, max_len,
                                           _ptr(out), _stream(stream)))
+    return out
+
+
+def hyb_attn_decode_partial(q, cache: KVCache, pos=None, max_len: int = 0, part_o=None, part_lse=None,
+                            workspace=None, stream=None):
+    """Attention of q [B,16,256] over the keys of `cache` only, ungated: returns
+    (part_o fp32 [B,16,256] normalised over these keys, part_lse fp32 [B,16] =
+    log2 sum_j exp(q.k_j / 16)).  pos: int32 [B] query positions in the whole
+    sequence (None: len - 1 of this cache)."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous() or tuple(q.shape[1:]) != (N_Q_HEADS, HEAD_DIM):
+        raise ValueError("q must be contiguous bf16 [B, 16, 256]")
+    B = q.shape[0]
+    if part_o is None:
+        part_o = torch.empty(B, N_Q_HEADS, HEAD_DIM, dtype=torch.float32, device=q.device)
+    if part_lse is None:
+        part_lse = torch.empty(B, N_Q_HEADS, dtype=torch.float32, device=q.device)
+    need = hyb_attn_decode_workspace_size(cache.layer_type, B, max_len or cache.capacity)
+    if workspace is None:
+        workspace = alloc_workspace(need, q.device)
+    _check(load().hyb_attn_decode_partial(_ptr(q), _ptr(pos), cache.ref, cache.layer_type, max_len, _ptr(part_o),
+                                          _ptr(part_lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+    return part_o, part_lse
+
+
+def hyb_attn_decode_merge(part_o, part_lse, gate=None, out=None, stream=None):
+    """Merges partials part_o fp32 [P,B,16,256] / part_lse fp32 [P,B,16]
+    (e.g. all-gathered from P GPUs), applies the gate (bf16 [B,16] or None);
+    returns bf16 [B,16,256]."""
+    if part_o.dtype != torch.float32 or not part_o.is_contiguous() or part_o.dim() != 4 \
+            or tuple(part_o.shape[2:]) != (N_Q_HEADS, HEAD_DIM):
+        raise ValueError("part_o must be contiguous fp32 [P, B, 16, 256]")
+    P, B = part_o.shape[:2]
+    if part_lse.dtype != torch.float32 or not part_lse.is_contiguous() or tuple(part_lse.shape) != (P, B, N_Q_HEADS):
+        raise ValueError("part_lse must be contiguous fp32 [P, B, 16]")
+    if gate is not None and (gate.dtype != torch.bfloat16 or not gate.is_contiguous()
+                             or tuple(gate.shape) != (B, N_Q_HEADS)):
+        raise ValueError("gate must be contiguous bf16 [B, 16]")
+    if out is None:
+        out = torch.empty(B, N_Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=part_o.device)
+    _check(load().hyb_attn_decode_merge(_ptr(part_o), _ptr(part_lse), P, B, _ptr(gate), _ptr(out), _stream(stream)))
     return out
 
 

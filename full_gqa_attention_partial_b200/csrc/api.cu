@@ -624,12 +624,16 @@ size_t hyb_attn_decode_workspace_size(int32_t layer_type, int32_t B, int64_t max
 }
 
 namespace {
+// out: gated bf16 output; or, with out_o / out_lse set (and out NULL), the
+// merged fp32 output and base-2 log-sum-exp over this cache's keys.
 hyb_status decode_impl(const void* q, int64_t q_stride, bool q_rotated, const void* gate, const int32_t* pos,
                        const hyb_kv_cache* c, int32_t layer_type, int64_t max_len, void* out, void* workspace,
-                       size_t workspace_bytes, void* stream) {
+                       size_t workspace_bytes, void* stream, float* out_o = nullptr, float* out_lse = nullptr) {
   hyb_status s = check_cache(c);
   if (s != HYB_OK) return s;
-  if (!q || !out) return fail(HYB_EINVAL, "q and out must be non-NULL");
+  if (!q || (!out && !(out_o && out_lse))) return fail(HYB_EINVAL, "q and the output buffers must be non-NULL");
+  if (out_o && (!aligned16(out_o) || (reinterpret_cast<uintptr_t>(out_lse) & 3u)))
+    return fail(HYB_EALIGN, "part_o must be 16-byte and part_lse 4-byte aligned");
   if (layer_type != c->type) return fail(HYB_ESHAPE, "layer_type %d differs from the cache type %d", layer_type, c->type);
   if (!aligned16(q) || !aligned16(out)) return fail(HYB_EALIGN, "q and out must be 16-byte aligned");
   if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
@@ -661,6 +665,8 @@ hyb_status decode_impl(const void* q, int64_t q_stride, bool q_rotated, const vo
   d.n_splits = decode_num_splits(layer_type == HYB_FULL, c->batch, max_len);
   d.part_o = reinterpret_cast<float*>(workspace);
   d.part_lse = d.part_o + (size_t)c->batch * kHq * d.n_splits * kD;
+  d.out_o = out_o;
+  d.out_lse = out_lse;
   cudaError_t e = launch_decode(layer_type == HYB_FULL, d, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "decode launch");
   return HYB_OK;
@@ -672,6 +678,30 @@ hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos, 
                            size_t workspace_bytes, void* stream) {
   return decode_impl(q, (int64_t)kHq * kD, false, gate, pos, c, layer_type, max_len, out, workspace, workspace_bytes,
                      stream);
+}
+
+hyb_status hyb_attn_decode_partial(const void* q, const int32_t* pos, const hyb_kv_cache* c, int32_t layer_type,
+                                   int64_t max_len, float* part_o, float* part_lse, void* workspace,
+                                   size_t workspace_bytes, void* stream) {
+  if (!part_o || !part_lse) return fail(HYB_EINVAL, "part_o and part_lse must be non-NULL");
+  return decode_impl(q, (int64_t)kHq * kD, false, nullptr, pos, c, layer_type, max_len, nullptr, workspace,
+                     workspace_bytes, stream, part_o, part_lse);
+}
+
+hyb_status hyb_attn_decode_merge(const float* part_o, const float* part_lse, int32_t n_parts, int32_t B,
+                                 const void* gate, void* out, void* stream) {
+  if (!part_o || !part_lse || !out) return fail(HYB_EINVAL, "part_o, part_lse and out must be non-NULL");
+  if (n_parts <= 0 || B <= 0) return fail(HYB_EINVAL, "n_parts = %d and B = %d must be positive", n_parts, B);
+  if ((int64_t)n_parts * B * kHq * kD > (int64_t)0x7fffffff)
+    return fail(HYB_EOVERFLOW, "n_parts x B x 16 x 256 exceeds 2^31 elements");
+  if (!aligned16(part_o) || !aligned16(out) || (reinterpret_cast<uintptr_t>(part_lse) & 3u))
+    return fail(HYB_EALIGN, "part_o and out must be 16-byte aligned, part_lse 4-byte aligned");
+  if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
+  hyb_status s;
+  if ((s = ensure_device()) != HYB_OK) return s;
+  cudaError_t e = launch_decode_merge(part_o, part_lse, n_parts, B * kHq, gate, out, as_stream(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "merge launch");
+  return HYB_OK;
 }
 
 // Same computation as hyb_attn_decode, with the split partials kept in the

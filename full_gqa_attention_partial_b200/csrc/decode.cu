@@ -446,37 +446,79 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
   }
 }
 
-// Merges the splits of one (sequence, query head) and applies the gate.
-__global__ void __launch_bounds__(256) decode_combine_kernel(const float* part_o, const float* part_lse,
-                                                             const __nv_bfloat16* gate, __nv_bfloat16* out,
-                                                             int n_splits) {
+// Merges n partial results of each (sequence, query head) row.  Partial s
+// of row `row` has its normalised output at o + s * o_sstride + row *
+// o_rstride and its base-2 log-sum-exp at lse + s * l_sstride + row *
+// l_rstride: the merge weighs each by 2^lse (the log-sum-exp combination
+// of split softmaxes).  It writes the gated bf16 output, or with out_o set
+// the merged fp32 output and log-sum-exp (a partial over the union of the
+// keys, for a further merge).
+struct CombineArgs {
+  const float* o;
+  const float* lse;
+  int64_t o_sstride, o_rstride, l_sstride, l_rstride;
+  int n;
+  const __nv_bfloat16* gate;   // [rows] or null (bf16 output only)
+  __nv_bfloat16* out;          // [rows][256]
+  float* out_o;                // [rows][256] or null
+  float* out_lse;              // [rows]
+};
+
+__global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
   const int row = blockIdx.x;  // b * 16 + h
   const int d = threadIdx.x;
-  const float* lse = part_lse + (int64_t)row * n_splits;
+  const float* lse = a.lse + (int64_t)row * a.l_rstride;
+  const float* po = a.o + (int64_t)row * a.o_rstride + d;
   float M = -INFINITY;
-  for (int s = 0; s < n_splits; ++s) M = fmaxf(M, lse[s]);
+  for (int s = 0; s < a.n; ++s) M = fmaxf(M, lse[s * a.l_sstride]);
   float acc = 0.f, den = 0.f;
   if (M != -INFINITY) {
-    for (int s = 0; s < n_splits; ++s) {
-      if (lse[s] == -INFINITY) continue;
-      const float w = exp2f(lse[s] - M);
+    for (int s = 0; s < a.n; ++s) {
+      const float ls = lse[s * a.l_sstride];
+      if (ls == -INFINITY) continue;
+      const float w = exp2f(ls - M);
       den += w;
-      acc += w * part_o[((int64_t)row * n_splits + s) * kD + d];
+      acc += w * po[s * a.o_sstride];
     }
   }
   float r = den > 0.f ? acc / den : 0.f;
-  if (gate != nullptr) {
-    const float gs = __bfloat162float(gate[row]);
+  if (a.out_o != nullptr) {
+    a.out_o[(int64_t)row * kD + d] = r;
+    if (d == 0) a.out_lse[row] = den > 0.f ? M + log2f(den) : -INFINITY;
+    return;
+  }
+  if (a.gate != nullptr) {
+    const float gs = __bfloat162float(a.gate[row]);
     r *= 1.f / (1.f + __expf(-gs));
   }
-  out[(int64_t)row * kD + d] = __float2bfloat16_rn(r);
+  a.out[(int64_t)row * kD + d] = __float2bfloat16_rn(r);
+}
+
+cudaError_t launch_decode_merge(const float* part_o, const float* part_lse, int n_parts, int rows,
+                                const void* gate, void* out, cudaStream_t st) {
+  CombineArgs c;
+  c.o = part_o;
+  c.lse = part_lse;
+  c.o_sstride = (int64_t)rows * kD;
+  c.o_rstride = kD;
+  c.l_sstride = rows;
+  c.l_rstride = 1;
+  c.n = n_parts;
+  c.gate = reinterpret_cast<const __nv_bfloat16*>(gate);
+  c.out = reinterpret_cast<__nv_bfloat16*>(out);
+  c.out_o = nullptr;
+  c.out_lse = nullptr;
+  decode_combine_kernel<<<rows, 256, 0, st>>>(c);
+  count_launch();
+  return cudaGetLastError();
 }
 
 int decode_num_splits(bool full, int B, int64_t max_len) {
   const int64_t keys = full ? (max_len > 0 ? max_len : 1) : kWindow;
   const int64_t pairs = (int64_t)B * kHkv;
   const int64_t s_max = keys / 512 > 1 ? keys / 512 : 1;   // >= 8 stages of 64 keys per split
-  const int sms = 148;
+  // whole waves of 296 CTA slots: two FP8 CTAs per SM (bf16: two waves of 148)
+  const int sms = 2 * 148;
   int best = 1;
   double best_eff = 0.0;
   for (int64_t s = 1; s <= s_max && s <= 1024; ++s) {
@@ -519,9 +561,19 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
   count_launch();
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  decode_combine_kernel<<<h.B * kHq, 256, 0, st>>>(h.part_o, h.part_lse,
-                                                   reinterpret_cast<const __nv_bfloat16*>(h.gate),
-                                                   reinterpret_cast<__nv_bfloat16*>(h.out), h.n_splits);
+  CombineArgs c;
+  c.o = h.part_o;
+  c.lse = h.part_lse;
+  c.o_sstride = kD;
+  c.o_rstride = (int64_t)h.n_splits * kD;
+  c.l_sstride = 1;
+  c.l_rstride = h.n_splits;
+  c.n = h.n_splits;
+  c.gate = reinterpret_cast<const __nv_bfloat16*>(h.gate);
+  c.out = reinterpret_cast<__nv_bfloat16*>(h.out);
+  c.out_o = h.out_o;
+  c.out_lse = h.out_lse;
+  decode_combine_kernel<<<h.B * kHq, 256, 0, st>>>(c);
   count_launch();
   return cudaGetLastError();
 }

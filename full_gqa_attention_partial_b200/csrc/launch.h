@@ -112,8 +112,14 @@ struct DecodeHost {
   float* part_lse = nullptr;   // [B][16][S]
   int B = 0, n_splits = 1;
   PageMap pm;                  // maps over a paged cache's pool {256, page, 4, n_pages}
+  float* out_o = nullptr;      // set: write the merged fp32 output [B][16][256] and base-2
+  float* out_lse = nullptr;    //   log-sum-exp [B][16] instead of the gated bf16 out
 };
 cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st);
+// Merges n_parts partials laid out [n_parts][rows][256] (+ lse [n_parts][rows])
+// into gated bf16 out [rows][256].
+cudaError_t launch_decode_merge(const float* part_o, const float* part_lse, int n_parts, int rows,
+                                const void* gate, void* out, cudaStream_t st);
 int decode_num_splits(bool full, int B, int64_t max_len);
 // Address and size of the library's fixed decode scratch on the current
 // device (looked up on first use per device).

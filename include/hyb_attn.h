@@ -215,6 +215,36 @@ hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos,
                            void* out, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * Sequence-sharded decode.  A long full-layer history can be spread over
+ * several caches (one per GPU, each holding any subset of the sequence's
+ * tokens, keys rotated at their own positions); attention over the union is
+ * the log-sum-exp merge of the attention over each part (the split-KV
+ * combination, "百万 Token 塞进 4B ..." §"省显存的第二板斧" for the gate):
+ *
+ * hyb_attn_decode_partial: attention of the B queries over the keys in
+ *   `cache` only, without the gate.
+ *   q, pos, cache, layer_type, max_len, workspace: as hyb_attn_decode; pos
+ *          should hold the query's position in the whole sequence (NULL
+ *          means len - 1 of this cache).
+ *   part_o  : fp32 [B][16][256], the softmax-normalised output over these keys.
+ *   part_lse: fp32 [B][16], log2 of sum_j exp(q . k_j / 16) over these keys
+ *             (-inf for a sequence with no keys here; part_o is then 0).
+ * hyb_attn_decode_merge: merges n_parts such partials, laid out
+ *   part_o [n_parts][B][16][256] and part_lse [n_parts][B][16] (what an
+ *   all-gather of the per-GPU partials gives), weighting part p by
+ *   2^part_lse[p], applies sigmoid(gate) (bf16 [B][16] or NULL) and writes
+ *   bf16 out [B][16][256].  The caller moves the partials between GPUs
+ *   (16 KB per sequence per part).
+ * Errors: as hyb_attn_decode; merge: HYB_EINVAL (null buffer, n_parts or
+ * B <= 0), HYB_EALIGN, HYB_EOVERFLOW (more than 2^31 elements).
+ */
+hyb_status hyb_attn_decode_partial(const void* q, const int32_t* pos, const hyb_kv_cache* cache,
+                                   int32_t layer_type, int64_t max_len, float* part_o, float* part_lse,
+                                   void* workspace, size_t workspace_bytes, void* stream);
+hyb_status hyb_attn_decode_merge(const float* part_o, const float* part_lse, int32_t n_parts, int32_t B,
+                                 const void* gate, void* out, void* stream);
+
+/*
  * hyb_attn_decode without a workspace.  The pages describe no counterpart:
  * this entry point exists for callers that may not allocate device memory
  * on their call path -- for example a plugin inside a host application that

@@ -265,6 +265,59 @@ def decode_group(q_rows, k, v, q_idx, k_idx, lt, gate=None):
     return o
 
 
+def decode_partial(q, qpos, cache_k, cache_v, lt):
+    """One decode query per sequence against a part of its full-layer history
+    (the keys one GPU holds when the history is spread over several), without
+    the gate.
+
+    q [B, 16, 256] raw query, qpos [B] RoPE positions, cache_k / cache_v
+    [B][L_b, 4, 256] this part's keys (roped) and values.  Every key of a
+    full layer precedes the query, so all are visible.
+    Returns (o [B, 16, 256], lse2 [B, 16]) float64: o the softmax-normalised
+    output over these keys, lse2 = log2 sum_j exp(q . k_j / 16).  A sequence
+    with no keys here gives o = 0 and lse2 = -inf.
+    """
+    assert lt == FULL, "only full layers are spread over several GPUs"
+    q = np.asarray(q, dtype=np.float64)
+    B, H, D = q.shape
+    o = np.zeros((B, H, D))
+    lse2 = np.full((B, H), -np.inf)
+    for b in range(B):
+        k = np.asarray(cache_k[b], np.float64)
+        v = np.asarray(cache_v[b], np.float64)
+        if k.shape[0] == 0:
+            continue
+        qr = rope_layer(q[b][None], np.array([qpos[b]]), lt)[0]     # [H, D]
+        for h in range(H):
+            kv = h // (H // k.shape[1])                              # query head h reads KV head h // 4
+            s = (k[:, kv] @ qr[h]) / np.sqrt(D)
+            m = s.max()
+            p = np.exp(s - m)
+            o[b, h] = (p @ v[:, kv]) / p.sum()
+            lse2[b, h] = (m + np.log(p.sum())) / np.log(2.0)
+    return o, lse2
+
+
+def merge_partials(o_parts, lse2_parts, gate=None):
+    """Attention over the union of the parts from each part's normalised
+    output and log-sum-exp: o = sum_p 2^lse2_p o_p / sum_p 2^lse2_p (parts
+    with lse2 = -inf hold no keys), then the head-wise sigmoid gate.
+
+    o_parts [P, B, 16, 256], lse2_parts [P, B, 16], gate [B, 16] or None.
+    Returns [B, 16, 256] float64.
+    """
+    o_parts = np.asarray(o_parts, np.float64)
+    lse2 = np.asarray(lse2_parts, np.float64)
+    m = lse2.max(axis=0)                                             # [B, H]
+    safe = np.where(np.isfinite(m), m, 0.0)
+    w = np.where(np.isfinite(lse2), np.exp2(lse2 - safe[None]), 0.0)  # [P, B, H]
+    den = w.sum(axis=0)
+    o = (w[..., None] * o_parts).sum(axis=0) / np.where(den > 0, den, 1.0)[..., None]
+    if gate is not None:
+        o = o * sigmoid(np.asarray(gate, np.float64))[..., None]
+    return o
+
+
 # ---------------------------------------------------------------------------
 # Projections around the attention core
 # ---------------------------------------------------------------------------

@@ -447,3 +447,44 @@ def test_e4m3_quantizer_known_values_and_bounds():
     # a zero row: scale 0, codes 0
     cz, sz = O.quantize_e4m3_rows(np.zeros(256))
     assert sz == 0 and not cz.any()
+
+
+def test_decode_partial_brute_force_tiny():
+    """lse2 and o of one part written out as scalar loops (position 0: no rotation)."""
+    rng = np.random.default_rng(5)
+    q = rng.standard_normal((1, 16, 256))
+    k = rng.standard_normal((1, 3, 4, 256))
+    v = rng.standard_normal((1, 3, 4, 256))
+    o, lse2 = O.decode_partial(q, [0], list(k), list(v), O.FULL)
+    for h in (0, 5, 15):
+        kv = h // 4
+        s = [sum(q[0, h, d] * k[0, j, kv, d] for d in range(256)) / 16.0 for j in range(3)]
+        z = sum(math.exp(x) for x in s)
+        assert abs(lse2[0, h] - math.log2(z)) < 1e-12
+        for d in (0, 77, 255):
+            ref = sum(math.exp(s[j]) * v[0, j, kv, d] for j in range(3)) / z
+            assert abs(o[0, h, d] - ref) < 1e-12
+
+
+def test_merged_parts_equal_decode_over_the_union():
+    """Spreading a full-layer history over parts (one of them empty, keys in
+    any order) and merging gives decode over all keys, gate included."""
+    rng = np.random.default_rng(6)
+    B, L = 2, 90
+    q = rng.standard_normal((B, 16, 256))
+    gate = rng.standard_normal((B, 16))
+    k = rng.standard_normal((B, L, 4, 256))
+    v = rng.standard_normal((B, L, 4, 256))
+    qpos = [L - 1, L - 1]
+    owner = rng.integers(0, 3, size=L)
+    owner[owner == 2] = 0                   # part 2 holds nothing
+    parts = [O.decode_partial(q, qpos, [k[b][owner == p] for b in range(B)], [v[b][owner == p] for b in range(B)],
+                              O.FULL) for p in range(3)]
+    assert np.all(parts[2][1] == -np.inf) and np.all(parts[2][0] == 0)
+    got = O.merge_partials(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]), gate)
+    ref = O.decode(q, gate, qpos, list(k), list(v), [np.arange(L)] * B, O.FULL)
+    assert np.abs(got - ref).max() < 1e-12
+    # a single part is decode without the gate, and its merge adds the gate
+    o1, l1 = O.decode_partial(q, qpos, list(k), list(v), O.FULL)
+    assert np.abs(o1 - O.decode(q, None, qpos, list(k), list(v), [np.arange(L)] * B, O.FULL)).max() < 1e-12
+    assert np.abs(O.merge_partials(o1[None], l1[None], gate) - ref).max() < 1e-12
