@@ -618,7 +618,9 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
 
 size_t hyb_attn_decode_workspace_size(int32_t layer_type, int32_t B, int64_t max_len) {
   if (B <= 0) return 0;
-  const int S = decode_num_splits(layer_type == HYB_FULL, B, max_len);
+  // room for either storage type's grid
+  const int S = std::max(decode_num_splits(layer_type == HYB_FULL, B, max_len, false),
+                         decode_num_splits(layer_type == HYB_FULL, B, max_len, true));
   const size_t rows = (size_t)B * kHq * (size_t)S;
   return rows * kD * sizeof(float) + ((rows * sizeof(float) + 255) & ~size_t(255));
 }
@@ -662,7 +664,7 @@ hyb_status decode_impl(const void* q, int64_t q_stride, bool q_rotated, const vo
   d.out = out;
   d.B = c->batch;
   d.pm = page_map(c);
-  d.n_splits = decode_num_splits(layer_type == HYB_FULL, c->batch, max_len);
+  d.n_splits = decode_num_splits(layer_type == HYB_FULL, c->batch, max_len, d.fp8 != 0);
   d.part_o = reinterpret_cast<float*>(workspace);
   d.part_lse = d.part_o + (size_t)c->batch * kHq * d.n_splits * kD;
   d.out_o = out_o;
@@ -719,7 +721,7 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
   if (max_len < 0 || max_len > c->capacity)
     return fail(HYB_ESHAPE, "max_len %lld outside [0, capacity %lld]", (long long)max_len, (long long)c->capacity);
   if (max_len == 0) max_len = c->capacity;
-  const int splits = decode_num_splits(layer_type == HYB_FULL, c->batch, max_len);
+  const int splits = decode_num_splits(layer_type == HYB_FULL, c->batch, max_len, c->kv_dtype == HYB_KV_FP8);
   const size_t need = hyb_attn_decode_workspace_size(layer_type, c->batch, max_len);
   if (need > kNoAllocScratchBytes)
     return fail(HYB_EOVERFLOW,

@@ -513,12 +513,12 @@ cudaError_t launch_decode_merge(const float* part_o, const float* part_lse, int 
   return cudaGetLastError();
 }
 
-int decode_num_splits(bool full, int B, int64_t max_len) {
+int decode_num_splits(bool full, int B, int64_t max_len, bool fp8) {
   const int64_t keys = full ? (max_len > 0 ? max_len : 1) : kWindow;
   const int64_t pairs = (int64_t)B * kHkv;
   const int64_t s_max = keys / 512 > 1 ? keys / 512 : 1;   // >= 8 stages of 64 keys per split
-  // whole waves of 296 CTA slots: two FP8 CTAs per SM (bf16: two waves of 148)
-  const int sms = 2 * 148;
+  // whole waves of CTA slots: one bf16 CTA per SM, two FP8 CTAs
+  const int sms = fp8 ? 2 * 148 : 148;
   int best = 1;
   double best_eff = 0.0;
   for (int64_t s = 1; s <= s_max && s <= 1024; ++s) {

@@ -120,7 +120,7 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st);
 // into gated bf16 out [rows][256].
 cudaError_t launch_decode_merge(const float* part_o, const float* part_lse, int n_parts, int rows,
                                 const void* gate, void* out, cudaStream_t st);
-int decode_num_splits(bool full, int B, int64_t max_len);
+int decode_num_splits(bool full, int B, int64_t max_len, bool fp8);
 // Address and size of the library's fixed decode scratch on the current
 // device (looked up on first use per device).
 cudaError_t decode_noalloc_scratch(void** ptr, size_t* bytes);
