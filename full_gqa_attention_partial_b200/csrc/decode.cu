@@ -516,7 +516,9 @@ cudaError_t launch_decode_merge(const float* part_o, const float* part_lse, int 
 int decode_num_splits(bool full, int B, int64_t max_len, bool fp8) {
   const int64_t keys = full ? (max_len > 0 ? max_len : 1) : kWindow;
   const int64_t pairs = (int64_t)B * kHkv;
-  const int64_t s_max = keys / 512 > 1 ? keys / 512 : 1;   // >= 8 stages of 64 keys per split
+  // full layers: >= 8 stages of 64 keys per split; a 512-slot ring may go down to one
+  // stage per split, so that a small batch still spreads its rings over the SMs
+  const int64_t s_max = full ? (keys / 512 > 1 ? keys / 512 : 1) : kWindow / kDecKeys;
   // whole waves of CTA slots: one bf16 CTA per SM, two FP8 CTAs
   const int sms = fp8 ? 2 * 148 : 148;
   int best = 1;
