@@ -430,9 +430,14 @@ hyb_status append_impl(const hyb_kv_cache* c, const void* k, const void* v, int6
   r.dks = c->k_scale;
   r.dvs = c->v_scale;
   r.pm = page_map(c);
+  // a few tokens per sequence (decode steps): one block per sequence writes its rows and
+  // advances the cache state in the same launch; long appends spread over the SMs and
+  // commit in a second launch
+  r.commit = (T - r.t_first) <= 64 ? 1 : 0;
+  r.capacity = c->capacity;
   cudaError_t e = launch_rope_store(full, r, st);
   if (e != cudaSuccess) return cuda_fail(e, "append launch");
-  if ((e = launch_kv_commit(c->len, c->head, c->capacity, !full, c->batch, T, st)) != cudaSuccess)
+  if (!r.commit && (e = launch_kv_commit(c->len, c->head, c->capacity, !full, c->batch, T, st)) != cudaSuccess)
     return cuda_fail(e, "commit launch");
   return HYB_OK;
 }

@@ -36,14 +36,16 @@ struct RopeStoreHost {
   int64_t dst_rows = 0;
   int dst_row_offset = 0;
   int mode = 0;  // 0 linear cache, 1 ring, 2 plain rows
-  const int32_t* len = nullptr;
-  const int32_t* head = nullptr;
+  int32_t* len = nullptr;
+  int32_t* head = nullptr;
   int32_t* tag = nullptr;
   int B = 0, T = 0, t_first = 0;
   int fp8 = 0;                 // 1: destination is an FP8 cache (codes + per-row scales)
   float* dks = nullptr;
   float* dvs = nullptr;
   PageMap pm;                  // linear mode: paged destination cache
+  int commit = 0;              // 1: advance len / head in the same launch (one block per sequence)
+  int64_t capacity = 0;        // commit, linear mode: cache capacity
 };
 cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st);
 cudaError_t launch_ring_gather(const void* rk, const void* rv, const int32_t* len, const int32_t* head,

@@ -37,8 +37,8 @@ struct RopeStoreArgs {
   int64_t dst_rows;
   int dst_row_offset;       // kDstRows: first destination row
   int mode;
-  const int32_t* len;       // cache bookkeeping (linear / ring) and default positions
-  const int32_t* head;
+  int32_t* len;             // cache bookkeeping (linear / ring) and default positions
+  int32_t* head;
   int32_t* tag;
   int B, T;
   int t_first;              // first token index written (ring: max(0, T - 512))
@@ -46,6 +46,9 @@ struct RopeStoreArgs {
   float* dks;               // [B][4][dst_rows]
   float* dvs;
   PageMap pm;               // linear mode, paged cache: destination [n_pages][4][page][256]
+  int commit;               // 1: grid = B, block b owns sequence b and advances its len (and
+                            //    ring head) after its rows, as kv_commit_kernel would
+  int64_t capacity;         // commit, linear mode: the cache capacity
 };
 
 // One 256-dim row (one token, one KV head) held by a warp, 8 bf16 values per
@@ -90,9 +93,10 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
   const int lane32 = threadIdx.x & 31;
   const int kvh = threadIdx.x >> 5;
   const int d0 = lane32 * 8;
+  // jobs token-major: with grid = B (commit) block b takes exactly sequence b's tokens
   for (int job = blockIdx.x; job < a.B * n_tok; job += gridDim.x) {
-    const int b = job / n_tok;
-    const int t = a.t_first + job % n_tok;
+    const int b = job % a.B;
+    const int t = a.t_first + job / a.B;
     const int64_t src = (int64_t)b * a.src_bstride + (int64_t)t * a.src_tstride + (int64_t)kvh * a.src_hstride + d0;
     int64_t dst_row;
     const int L = (a.len != nullptr) ? a.len[b] : 0;
@@ -157,6 +161,18 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
     *reinterpret_cast<uint4*>(a.dk + dst) = kx;
     if (a.v != nullptr) {
       *reinterpret_cast<uint4*>(a.dv + dst) = *reinterpret_cast<const uint4*>(a.v + src);
+    }
+  }
+  if (a.commit) {
+    __syncthreads();   // every row of sequence blockIdx.x has read len / head
+    if (threadIdx.x == 0 && blockIdx.x < a.B) {
+      const int b = blockIdx.x;
+      if (a.mode == kDstRing) {
+        a.head[b] = (a.head[b] + a.T) % kWindow;
+        a.len[b] += a.T;
+      } else if ((int64_t)a.len[b] + a.T <= a.capacity) {
+        a.len[b] += a.T;
+      }
     }
   }
 }
@@ -244,7 +260,9 @@ cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st
   a.B = h.B;
   a.T = h.T;
   a.t_first = h.t_first;
-  const int grid = rope_grid(h.B * (h.T - h.t_first));
+  a.commit = h.commit;
+  a.capacity = h.capacity;
+  const int grid = h.commit ? h.B : rope_grid(h.B * (h.T - h.t_first));
   if (full)
     rope_store_kernel<true><<<grid, 128, 0, st>>>(a);
   else
