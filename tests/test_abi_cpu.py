@@ -133,3 +133,21 @@ def test_paged_cache_checks_before_any_cuda_call(hyb):
     assert append(hyb._Cache(1, 2, 1024, 0x1000, 0x2000, 0x3000, 0x4000, 0x5000, 0, None, None,
                              -64, 0, 0, None)) == -1                      # negative page size
     assert "page" in lib.hyb_last_error().decode()
+
+
+def test_partial_and_merge_checks_before_any_cuda_call(hyb):
+    lib = hyb.load()
+    A = ctypes.c_void_p(0x10000)
+    c = _cache(hyb, lt=1, cap=1024)
+    # partial: output buffers required and aligned
+    assert lib.hyb_attn_decode_partial(A, None, ctypes.byref(c), 1, 0, None, A, A, 1 << 20, None) == -1
+    assert lib.hyb_attn_decode_partial(A, None, ctypes.byref(c), 1, 0, ctypes.c_void_p(0x10004), A, A, 1 << 20,
+                                       None) == -3
+    assert lib.hyb_attn_decode_partial(A, None, ctypes.byref(c), 0, 0, A, A, A, 1 << 20, None) == -2   # type
+    # merge: null buffers, non-positive counts, misalignment
+    assert lib.hyb_attn_decode_merge(None, A, 2, 1, None, A, None) == -1
+    assert lib.hyb_attn_decode_merge(A, A, 0, 1, None, A, None) == -1
+    assert lib.hyb_attn_decode_merge(A, A, 2, -1, None, A, None) == -1
+    assert lib.hyb_attn_decode_merge(A, ctypes.c_void_p(0x10002), 2, 1, None, A, None) == -3
+    assert lib.hyb_attn_decode_merge(A, A, 2, 1, ctypes.c_void_p(0x10001), A, None) == -3
+    assert lib.hyb_attn_decode_merge(A, A, 1 << 20, 1 << 10, None, A, None) == -4            # > 2^31 elements
