@@ -151,3 +151,34 @@ def test_partial_and_merge_checks_before_any_cuda_call(hyb):
     assert lib.hyb_attn_decode_merge(A, ctypes.c_void_p(0x10002), 2, 1, None, A, None) == -3
     assert lib.hyb_attn_decode_merge(A, A, 2, 1, ctypes.c_void_p(0x10001), A, None) == -3
     assert lib.hyb_attn_decode_merge(A, A, 1 << 20, 1 << 10, None, A, None) == -4            # > 2^31 elements
+
+
+def test_header_is_plain_c_and_links(hyb, tmp_path):
+    """A C99 program that includes only the header links against the library
+    and gets the documented status back from a call that fails its checks
+    (no CUDA device is touched)."""
+    import shutil
+    import subprocess
+    if shutil.which("gcc") is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "abi.c"
+    src.write_text(r'''
+#include <stdio.h>
+#include "hyb_attn.h"
+int main(void) {
+  hyb_kv_cache c = {0};
+  c.type = HYB_SLIDING; c.batch = 1; c.capacity = 100;          /* a ring must hold 512 */
+  c.k = (void*)0x1000; c.v = (void*)0x2000; c.len = (int32_t*)0x3000;
+  c.head = (int32_t*)0x4000; c.tag = (int32_t*)0x5000;
+  hyb_status s = hyb_kv_append(&c, (void*)0x10000, (void*)0x10000, 1024, NULL, 4, NULL);
+  printf("%d %s\n", (int)s, hyb_last_error());
+  return s == HYB_ESHAPE ? 0 : 1;
+}
+''')
+    exe = tmp_path / "abi"
+    lib_dir = os.path.dirname(hyb.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", os.path.join(ROOT, "include"),
+                           str(src), "-o", str(exe), "-L", lib_dir, "-lhyb_attn", "-Wl,-rpath," + lib_dir])
+    r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stdout + r.stderr
+    assert "512" in r.stdout
