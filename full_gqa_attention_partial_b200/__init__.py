@@ -41,7 +41,7 @@ EXPORTED = (
     "hyb_launch_count", "hyb_profile_events", "hyb_profile_pairs_used", "hyb_attn_decode_noalloc",
     "hyb_selftest_wait_timeout", "hyb_linear", "hyb_attn_layer_prefill_workspace_size", "hyb_attn_layer_prefill",
     "hyb_attn_layer_decode_workspace_size", "hyb_attn_layer_decode", "hyb_attn_decode_partial",
-    "hyb_attn_decode_merge",
+    "hyb_attn_decode_merge", "hyb_attn_prefill_cache_workspace_size", "hyb_attn_layer_prefill_cache_workspace_size",
 )
 
 
@@ -109,6 +109,10 @@ def load(path: str = LIB_PATH):
     lib.hyb_attn_layer_decode.argtypes = [vp, vp, vp, vp, pc, i32, i64, vp, vp, sz, vp]
     lib.hyb_attn_decode_partial.argtypes = [vp, vp, pc, i32, i64, vp, vp, vp, sz, vp]
     lib.hyb_attn_decode_merge.argtypes = [vp, vp, i32, i32, vp, vp, vp]
+    lib.hyb_attn_prefill_cache_workspace_size.argtypes = [pc, i32]
+    lib.hyb_attn_prefill_cache_workspace_size.restype = sz
+    lib.hyb_attn_layer_prefill_cache_workspace_size.argtypes = [pc, i32]
+    lib.hyb_attn_layer_prefill_cache_workspace_size.restype = sz
     for name in ("hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill", "hyb_attn_decode",
                  "hyb_device_error"):
         getattr(lib, name).restype = ctypes.c_int
@@ -245,7 +249,8 @@ def hyb_attn_prefill(q, k, v, gate, pos, layer_type: int, out=None, cache: KVCac
         raise ValueError("pos must be contiguous int32 [B, T]")
     if out is None:
         out = torch.empty(B, T, N_Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
-    need = hyb_attn_prefill_workspace_size(layer_type, B, T, cache is not None)
+    need = hyb_attn_prefill_workspace_size(layer_type, B, T, False) if cache is None else \
+        int(load().hyb_attn_prefill_cache_workspace_size(cache.ref, T))
     if workspace is None and need > 0:
         workspace = alloc_workspace(need, q.device)
     wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -279,7 +284,8 @@ def hyb_attn_layer_prefill(hidden, w_qkv, w_gate, w_o, pos, layer_type: int, out
         raise ValueError("pos must be contiguous int32 [B, T]")
     if out is None:
         out = torch.empty(B, T, HIDDEN, dtype=torch.bfloat16, device=hidden.device)
-    need = hyb_attn_layer_prefill_workspace_size(layer_type, B, T, cache is not None)
+    need = hyb_attn_layer_prefill_workspace_size(layer_type, B, T, False) if cache is None else \
+        int(load().hyb_attn_layer_prefill_cache_workspace_size(cache.ref, T))
     if workspace is None:
         workspace = alloc_workspace(need, hidden.device)
     wsz = workspace.numel() * workspace.element_size()

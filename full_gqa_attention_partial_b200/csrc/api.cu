@@ -457,6 +457,25 @@ size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T,
 }
 
 namespace {
+// bf16 copy of one of K / V of an FP8 full-layer cache, whole capacity
+size_t fp8_copy_bytes(const hyb_kv_cache* c) {
+  return ((size_t)c->batch * kHkv * (size_t)c->capacity * kD * 2 + 255) & ~(size_t)255;
+}
+
+// Scratch of a prefill with cache `c` (NULL: standalone).  An FP8 full-layer
+// cache is attended through bf16 copies of its K and V.
+size_t prefill_ws(int32_t layer_type, int32_t B, int32_t T, const hyb_kv_cache* c) {
+  if (c && c->type == HYB_FULL && c->kv_dtype == HYB_KV_FP8) return 2 * fp8_copy_bytes(c);
+  return hyb_attn_prefill_workspace_size(layer_type, B, T, c != nullptr);
+}
+}  // namespace
+
+size_t hyb_attn_prefill_cache_workspace_size(const hyb_kv_cache* cache, int32_t T) {
+  if (!cache || T <= 0 || check_cache(cache) != HYB_OK) return 0;
+  return prefill_ws(cache->type, cache->batch, T, cache);
+}
+
+namespace {
 // qk_rotated: q and k arrive rotated (the whole-layer path rotates them in the
 // q_k_v_proj epilogue); the attention kernel and the K store then skip RoPE.
 hyb_status prefill_impl(const void* q, const void* k, const void* v, const void* gate, const int32_t* pos,
@@ -482,12 +501,10 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
     if (cache->type != layer_type)
       return fail(HYB_ESHAPE, "cache type %d differs from layer_type %d", cache->type, layer_type);
     if (cache->batch != B) return fail(HYB_ESHAPE, "cache batch %d differs from B = %d", cache->batch, B);
-    if (cache->kv_dtype != HYB_KV_BF16)
-      return fail(HYB_EUNSUPPORTED, "prefill attends over bf16 caches only (this cache is FP8)");
     if (layer_type == HYB_FULL && (int64_t)T > cache->capacity)
       return fail(HYB_ESHAPE, "T = %d exceeds the cache capacity %lld", T, (long long)cache->capacity);
   }
-  const size_t need = hyb_attn_prefill_workspace_size(layer_type, B, T, cache != nullptr);
+  const size_t need = prefill_ws(layer_type, B, T, cache);
   if (need > 0) {
     if (!workspace) return fail(HYB_EINVAL, "workspace of %zu bytes required", need);
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(HYB_EALIGN, "workspace must be 256-byte aligned");
@@ -543,6 +560,50 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
     return HYB_OK;
   }
 
+  const bool fp8 = cache->kv_dtype == HYB_KV_FP8;
+  if (full && fp8) {
+    // the chunk goes into the cache (quantized) and, at full precision, into
+    // bf16 copies of K and V whose rows [0, len) are the stored history
+    // dequantized; attend over the copies' [0, len + T), then advance len
+    uint8_t* wk = reinterpret_cast<uint8_t*>(workspace);
+    uint8_t* wv = wk + fp8_copy_bytes(cache);
+    const int64_t cap = cache->capacity;
+    r.v = v;
+    r.dk = cache->k;
+    r.dv = cache->v;
+    r.dst_rows = cap;
+    r.mode = 0;
+    r.len = cache->len;
+    r.pm = page_map(cache);
+    r.fp8 = 1;
+    r.dks = cache->k_scale;
+    r.dvs = cache->v_scale;
+    if ((e = launch_rope_store(true, r, st)) != cudaSuccess) return cuda_fail(e, "append launch");
+    RopeStoreHost c2 = r;   // the chunk into the bf16 copies
+    c2.dk = wk;
+    c2.dv = wv;
+    c2.fp8 = 0;
+    c2.dks = c2.dvs = nullptr;
+    c2.pm = PageMap();
+    if ((e = launch_rope_store(true, c2, st)) != cudaSuccess) return cuda_fail(e, "chunk copy launch");
+    if ((e = launch_dequant_rows(cache->k, cache->v, cache->k_scale, cache->v_scale, page_map(cache), cap,
+                                 cache->len, T, B, wk, wv, cap, st)) != cudaSuccess)
+      return cuda_fail(e, "history dequantize launch");
+    const uint64_t hb = (uint64_t)cap * row_bytes;
+    if ((s = make_kv_map(&ph.tm_k, wk, (uint64_t)cap, B, row_bytes, hb, hb * kHkv, prefill_k_box_rows(),
+                         "FP8 history K")) != HYB_OK)
+      return s;
+    if ((s = make_kv_map(&ph.tm_v, wv, (uint64_t)cap, B, row_bytes, hb, hb * kHkv, prefill_v_box_rows(),
+                         "FP8 history V")) != HYB_OK)
+      return s;
+    ph.qbase = cache->len;
+    ph.ctx_mode = 0;
+    if ((e = launch_prefill(true, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
+    if ((e = launch_kv_commit(cache->len, cache->head, cache->capacity, false, B, T, st)) != cudaSuccess)
+      return cuda_fail(e, "commit launch");
+    return HYB_OK;
+  }
+
   if (full) {
     // append first (rows len .. len+T-1), attend over [0, len+T), then advance len
     r.v = v;
@@ -569,8 +630,8 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
   uint8_t* ws = reinterpret_cast<uint8_t*>(workspace);
   void* ck = ws;
   void* cv = ws + (size_t)B * rows * kHkv * row_bytes;
-  if ((e = launch_ring_gather(cache->k, cache->v, cache->len, cache->head, cache->tag, ck, cv, (int64_t)rows, B,
-                              st)) != cudaSuccess)
+  if ((e = launch_ring_gather(cache->k, cache->v, fp8 ? cache->k_scale : nullptr, fp8 ? cache->v_scale : nullptr,
+                              cache->len, cache->head, cache->tag, ck, cv, (int64_t)rows, B, st)) != cudaSuccess)
     return cuda_fail(e, "ring gather launch");
   r.v = v;
   r.dk = ck;
@@ -606,6 +667,9 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
   w.B = B;
   w.T = T;
   w.t_first = T > kWindow ? T - kWindow : 0;
+  w.fp8 = fp8 ? 1 : 0;
+  w.dks = cache->k_scale;
+  w.dvs = cache->v_scale;
   if ((e = launch_rope_store(false, w, st)) != cudaSuccess) return cuda_fail(e, "ring append launch");
   if ((e = launch_kv_commit(cache->len, cache->head, cache->capacity, true, B, T, st)) != cudaSuccess)
     return cuda_fail(e, "commit launch");
@@ -779,6 +843,13 @@ size_t hyb_attn_layer_prefill_workspace_size(int32_t layer_type, int32_t B, int3
          hyb_attn_prefill_workspace_size(layer_type, B, T, with_cache);
 }
 
+size_t hyb_attn_layer_prefill_cache_workspace_size(const hyb_kv_cache* cache, int32_t T) {
+  if (!cache || T <= 0 || check_cache(cache) != HYB_OK) return 0;
+  const size_t n = (size_t)cache->batch * (size_t)T;
+  return round256(n * kQkv * 2) + round256(n * kHq * 2) + round256(n * kHq * kD * 2) +
+         prefill_ws(cache->type, cache->batch, T, cache);
+}
+
 hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const void* w_gate, const void* w_o,
                                   const int32_t* pos, int32_t layer_type, int32_t B, int32_t T, void* out,
                                   const hyb_kv_cache* cache, void* workspace, size_t workspace_bytes,
@@ -787,7 +858,12 @@ hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const v
   if (layer_type != HYB_SLIDING && layer_type != HYB_FULL) return fail(HYB_EINVAL, "layer_type %d invalid", layer_type);
   if (B <= 0 || T <= 0) return fail(HYB_EINVAL, "B = %d and T = %d must be positive", B, T);
   if ((int64_t)B * T > 0x7fffffffLL) return fail(HYB_ESHAPE, "B * T = %lld tokens is too many", (long long)B * T);
-  const size_t need = hyb_attn_layer_prefill_workspace_size(layer_type, B, T, cache != nullptr);
+  const size_t need = cache ? hyb_attn_layer_prefill_cache_workspace_size(cache, T)
+                            : hyb_attn_layer_prefill_workspace_size(layer_type, B, T, 0);
+  if (cache && need == 0) {
+    hyb_status cs = check_cache(cache);
+    return cs != HYB_OK ? cs : fail(HYB_EINVAL, "T = %d must be positive", T);
+  }
   if (workspace_bytes < need) return fail(HYB_EOVERFLOW, "workspace %zu bytes < %zu needed", workspace_bytes, need);
   if (!workspace || (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return fail(HYB_EALIGN, "workspace must be non-NULL and 256-byte aligned");
@@ -800,7 +876,7 @@ hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const v
   p += round256(n * kHq * 2);
   __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(p);
   p += round256(n * kHq * kD * 2);
-  const size_t attn_ws = hyb_attn_prefill_workspace_size(layer_type, B, T, cache != nullptr);
+  const size_t attn_ws = prefill_ws(layer_type, B, T, cache);
   // q_k_v_proj with RoPE of the q and k heads in the epilogue (positions as
   // hyb_attn_prefill: pos, else the cache length + t, else t)
   const int32_t* len = cache ? cache->len : nullptr;

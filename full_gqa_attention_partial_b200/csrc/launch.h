@@ -48,9 +48,15 @@ struct RopeStoreHost {
   int64_t capacity = 0;        // commit, linear mode: cache capacity
 };
 cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st);
-cudaError_t launch_ring_gather(const void* rk, const void* rv, const int32_t* len, const int32_t* head,
-                               const int32_t* tag, void* ck, void* cv, int64_t ctx_rows, int B,
-                               cudaStream_t st);
+// rks / rvs: FP8 rings' scales (rk / rv hold e4m3 codes), or null for bf16 rings
+cudaError_t launch_ring_gather(const void* rk, const void* rv, const float* rks, const float* rvs,
+                               const int32_t* len, const int32_t* head, const int32_t* tag, void* ck, void* cv,
+                               int64_t ctx_rows, int B, cudaStream_t st);
+// bf16 [B][4][dst_rows][256] copies of rows [0, len[b]) of an FP8 full-layer cache,
+// rows [len + T, end of their 64-row tile) zero-filled
+cudaError_t launch_dequant_rows(const void* kc, const void* vc, const float* ks, const float* vs, const PageMap& pm,
+                                int64_t cap, const int32_t* len, int T, int B, void* dk, void* dv, int64_t dst_rows,
+                                cudaStream_t st);
 cudaError_t launch_kv_commit(int32_t* len, int32_t* head, int64_t capacity, bool ring, int B, int T,
                              cudaStream_t st);
 cudaError_t launch_selftest_wait(cudaStream_t st);

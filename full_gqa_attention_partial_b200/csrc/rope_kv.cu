@@ -177,11 +177,76 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
   }
 }
 
+// Eight e4m3 codes (8 bytes, lowest first) times `scale`, rounded to bf16
+// (8 values in 16 bytes, same order).  The codes are widened exactly (value
+// x 2^-120 by bit moves, then x 2^120 in fp32), then scaled in fp32.
+__device__ __forceinline__ uint4 dequant8_bf16(uint2 codes, float scale) {
+  const uint32_t w[2] = {codes.x, codes.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t a = e4m3_b02_bf16x2(w[i]), c = e4m3_b13_bf16x2(w[i]);   // codes (0, 2) and (1, 3)
+    const float v0 = __uint_as_float(a << 16) * kE4m3WideScale * scale;
+    const float v2 = __uint_as_float(a & 0xFFFF0000u) * kE4m3WideScale * scale;
+    const float v1 = __uint_as_float(c << 16) * kE4m3WideScale * scale;
+    const float v3 = __uint_as_float(c & 0xFFFF0000u) * kE4m3WideScale * scale;
+    o[2 * i] = pack_bf16(v0, v1);
+    o[2 * i + 1] = pack_bf16(v2, v3);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
+}
+
+// bf16 copy of rows [0, len[b]) of an FP8 full-layer cache (contiguous or
+// paged) into dst [B][4][dst_rows][256], K and V: the history a prefill over
+// that cache attends to.  Rows [len + T, ...) up to the end of their 64-row
+// tile are zero-filled: the prefill loads whole tiles and multiplies the
+// masked rows by a zero weight, so they must hold finite values (the T
+// chunk rows in between are written by the chunk's own store).  Block
+// (tile, kvh, b) handles 64 rows.
+__global__ void __launch_bounds__(128) dequant_rows_kernel(const uint8_t* kc, const uint8_t* vc, const float* ks,
+                                                           const float* vs, PageMap pm, int64_t cap,
+                                                           const int32_t* len, int T, __nv_bfloat16* dk,
+                                                           __nv_bfloat16* dv, int64_t dst_rows) {
+  const int b = blockIdx.z, kvh = blockIdx.y;
+  const int row0 = blockIdx.x * 64;
+  const int L = len[b];
+  const int64_t tail_end = min(((int64_t)L + T + 63) / 64 * 64, dst_rows);
+  if (row0 >= tail_end) return;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int rr = warp; rr < 64; rr += 4) {
+    const int row = row0 + rr;
+    if (row >= tail_end) break;
+    const int64_t did = (((int64_t)b * kHkv + kvh) * dst_rows + row) * kD + lane * 8;
+    if (row >= L) {
+      if (row >= (int64_t)L + T) {
+        *reinterpret_cast<uint4*>(dk + did) = make_uint4(0, 0, 0, 0);
+        *reinterpret_cast<uint4*>(dv + did) = make_uint4(0, 0, 0, 0);
+      }
+      continue;
+    }
+    int64_t sid;   // source row of the [..][4][rows] layout
+    if (pm.page != 0) {
+      int prow, ppage;
+      kv_coord(pm, b, row, prow, ppage);
+      if (ppage < 0) ppage = 0;   // raised; read a valid page, the output is flagged invalid
+      sid = ((int64_t)ppage * kHkv + kvh) * pm.page + prow;
+    } else {
+      sid = ((int64_t)b * kHkv + kvh) * cap + row;
+    }
+    const uint2 kx = *reinterpret_cast<const uint2*>(kc + sid * kD + lane * 8);
+    const uint2 vx = *reinterpret_cast<const uint2*>(vc + sid * kD + lane * 8);
+    *reinterpret_cast<uint4*>(dk + did) = dequant8_bf16(kx, ks[sid]);
+    *reinterpret_cast<uint4*>(dv + did) = dequant8_bf16(vx, vs[sid]);
+  }
+}
+
 // Context rows [0, 511) of a chunked sliding prefill: row r holds sequence
-// index len - 511 + r, read from the ring; rows before the start of the
-// sequence (or a slot whose tag does not match) are zero-filled so that the
-// masked products stay finite.
+// index len - 511 + r, read from the ring (FP8 rings: dequantized to bf16 when
+// rks / rvs are given); rows before the start of the sequence (or a slot
+// whose tag does not match) are zero-filled so that the masked products stay
+// finite.
 __global__ void __launch_bounds__(128) ring_gather_kernel(const __nv_bfloat16* rk, const __nv_bfloat16* rv,
+                                                          const float* rks, const float* rvs,
                                                           const int32_t* len, const int32_t* head,
                                                           const int32_t* tag, __nv_bfloat16* ck,
                                                           __nv_bfloat16* cv, int64_t ctx_rows, int B) {
@@ -199,9 +264,16 @@ __global__ void __launch_bounds__(128) ring_gather_kernel(const __nv_bfloat16* r
     const int64_t dst = (((int64_t)b * kHkv + kvh) * ctx_rows + r) * kD + d0;
     uint4 kx = make_uint4(0, 0, 0, 0), vx = make_uint4(0, 0, 0, 0);
     if (ok) {
-      const int64_t src = (((int64_t)b * kHkv + kvh) * kWindow + slot) * kD + d0;
-      kx = *reinterpret_cast<const uint4*>(rk + src);
-      vx = *reinterpret_cast<const uint4*>(rv + src);
+      const int64_t sid = ((int64_t)b * kHkv + kvh) * kWindow + slot;
+      if (rks != nullptr) {
+        const uint8_t* k8 = reinterpret_cast<const uint8_t*>(rk);
+        const uint8_t* v8 = reinterpret_cast<const uint8_t*>(rv);
+        kx = dequant8_bf16(*reinterpret_cast<const uint2*>(k8 + sid * kD + d0), rks[sid]);
+        vx = dequant8_bf16(*reinterpret_cast<const uint2*>(v8 + sid * kD + d0), rvs[sid]);
+      } else {
+        kx = *reinterpret_cast<const uint4*>(rk + sid * kD + d0);
+        vx = *reinterpret_cast<const uint4*>(rv + sid * kD + d0);
+      }
     }
     *reinterpret_cast<uint4*>(ck + dst) = kx;
     *reinterpret_cast<uint4*>(cv + dst) = vx;
@@ -271,12 +343,23 @@ cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st
   return cudaGetLastError();
 }
 
-cudaError_t launch_ring_gather(const void* rk, const void* rv, const int32_t* len, const int32_t* head,
-                               const int32_t* tag, void* ck, void* cv, int64_t ctx_rows, int B,
-                               cudaStream_t st) {
+cudaError_t launch_ring_gather(const void* rk, const void* rv, const float* rks, const float* rvs,
+                               const int32_t* len, const int32_t* head, const int32_t* tag, void* ck, void* cv,
+                               int64_t ctx_rows, int B, cudaStream_t st) {
   ring_gather_kernel<<<rope_grid(B * (kWindow - 1)), 128, 0, st>>>(
-      reinterpret_cast<const __nv_bfloat16*>(rk), reinterpret_cast<const __nv_bfloat16*>(rv), len, head, tag,
-      reinterpret_cast<__nv_bfloat16*>(ck), reinterpret_cast<__nv_bfloat16*>(cv), ctx_rows, B);
+      reinterpret_cast<const __nv_bfloat16*>(rk), reinterpret_cast<const __nv_bfloat16*>(rv), rks, rvs, len, head,
+      tag, reinterpret_cast<__nv_bfloat16*>(ck), reinterpret_cast<__nv_bfloat16*>(cv), ctx_rows, B);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_dequant_rows(const void* kc, const void* vc, const float* ks, const float* vs, const PageMap& pm,
+                                int64_t cap, const int32_t* len, int T, int B, void* dk, void* dv, int64_t dst_rows,
+                                cudaStream_t st) {
+  const dim3 grid((unsigned)((dst_rows + 63) / 64), kHkv, B);
+  dequant_rows_kernel<<<grid, 128, 0, st>>>(reinterpret_cast<const uint8_t*>(kc), reinterpret_cast<const uint8_t*>(vc),
+                                            ks, vs, pm, cap, len, T, reinterpret_cast<__nv_bfloat16*>(dk),
+                                            reinterpret_cast<__nv_bfloat16*>(dv), dst_rows);
   count_launch();
   return cudaGetLastError();
 }

@@ -136,9 +136,12 @@ typedef struct hyb_kv_cache {
  *   stored value = code * scale (a zero row has scale 0 and zero codes).
  * Halves the cache bytes that decode streams (the pages' deployments keep
  * the KV cache in 8 bits: "不用高显存卡也能跑！..." q8_0 KV in llama.cpp).
- * FP8 caches need capacity % 4 == 0.  Supported by hyb_kv_append,
- * hyb_attn_decode(_noalloc) and hyb_attn_layer_decode; hyb_attn_prefill and
- * hyb_attn_layer_prefill with an FP8 cache return HYB_EUNSUPPORTED.
+ * FP8 caches need capacity % 4 == 0.  Decode reads every cached row as
+ * stored (code value x scale, the current token included).  A prefill over
+ * an FP8 cache attends to the cached history as stored (dequantized, rounded
+ * to bf16) and to its own chunk at full precision, and appends the chunk
+ * quantized; over a full-layer FP8 cache it needs the larger workspace of
+ * hyb_attn_prefill_cache_workspace_size (bf16 copies of K and V).
  */
 #define HYB_KV_BF16 0
 #define HYB_KV_FP8 1
@@ -189,6 +192,11 @@ hyb_status hyb_kv_append(const hyb_kv_cache* cache, const void* k, const void* v
  * small), HYB_EUNSUPPORTED (not an sm_100 device), HYB_ECUDA.
  */
 size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache);
+/* Workspace of hyb_attn_prefill with this cache and chunk length: the value
+ * above for bf16 caches, and for a full-layer FP8 cache two bf16 copies of
+ * the cache, 2 x batch x 4 x capacity x 512 bytes (each rounded up to 256).
+ * 0 for an invalid cache or T <= 0. */
+size_t hyb_attn_prefill_cache_workspace_size(const hyb_kv_cache* cache, int32_t T);
 hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const void* gate,
                             const int32_t* pos, int32_t layer_type, int32_t B, int32_t T,
                             int64_t q_row_stride, int64_t kv_row_stride, void* out,
@@ -304,12 +312,15 @@ hyb_status hyb_linear(const void* x, int64_t ldx, const void* w, int64_t ldw, vo
  *   pos, layer_type, B, T, cache: as hyb_attn_prefill.
  *   out    : bf16 [B][T][2560].
  *   workspace: at least hyb_attn_layer_prefill_workspace_size(layer_type, B,
- *          T, cache != NULL) bytes, 256-byte aligned; it holds the fused
- *          q|k|v rows, the gate scores and the attention output (bf16, as
- *          the model's tensors are) between the steps.
+ *          T, 0) bytes without a cache, hyb_attn_layer_prefill_cache_
+ *          workspace_size(cache, T) with one (the two agree for bf16 caches),
+ *          256-byte aligned; it holds the fused q|k|v rows, the gate scores
+ *          and the attention output (bf16, as the model's tensors are)
+ *          between the steps, and the attention's own scratch.
  * Errors: as hyb_linear and hyb_attn_prefill.
  */
 size_t hyb_attn_layer_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache);
+size_t hyb_attn_layer_prefill_cache_workspace_size(const hyb_kv_cache* cache, int32_t T);
 hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const void* w_gate, const void* w_o,
                                   const int32_t* pos, int32_t layer_type, int32_t B, int32_t T, void* out,
                                   const hyb_kv_cache* cache, void* workspace, size_t workspace_bytes,

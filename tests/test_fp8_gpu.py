@@ -1,6 +1,7 @@
 """FP8 (e4m3) KV caches: the quantizing append against the oracle's
-quantizer (values bit-exact, rotated keys within one code), and the calls
-that do not support FP8 yet report it."""
+quantizer (values bit-exact, rotated keys within one code), decode over
+every code and scale range, and chunked prefill over the stored history,
+all against the oracle on the dequantized cache."""
 import numpy as np
 import pytest
 import torch
@@ -58,11 +59,51 @@ def test_fp8_append_matches_quantizer(lib, lt):
     _check_rows(lib, cache, x, lt, slots, tokens)
 
 
-def test_fp8_cache_rejected_by_prefill(lib):
-    x = synth.prefill_inputs(1, 64, seed=1, device="cuda")
-    cache = lib.KVCache(O.FULL, 1, capacity=128, kv_dtype=lib.KV_FP8)
-    with pytest.raises(lib.HybError):
-        lib.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], None, O.FULL, cache=cache)
+@pytest.mark.parametrize("lt", [O.FULL, O.SLIDING])
+def test_fp8_chunked_prefill_matches_oracle(lib, lt):
+    """Two prefill chunks through an FP8 cache: each chunk attends to the
+    cached history as stored (the oracle dequantizes the codes) and to its
+    own tokens at full precision; the chunks are appended quantized."""
+    B, T1, T2 = 2, 700, 300
+    r = synth.ring_offset(51)
+    cache = lib.KVCache(lt, B, capacity=1024, kv_dtype=lib.KV_FP8, head0=None if lt == O.FULL else [r, (r + 99) % 512])
+    x1 = synth.prefill_inputs(B, T1, seed=52, device="cuda")
+    out1 = lib.hyb_attn_prefill(x1["q"], x1["k"], x1["v"], x1["gate"], x1["pos"], lt, cache=cache)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    ref1 = O.prefill(f64(x1["q"]), f64(x1["k"]), f64(x1["v"]), f64(x1["gate"]), x1["pos"].cpu().numpy(), lt)
+    assert_close(out1, ref1, f"chunk 1 lt={lt}")
+    # the history chunk 2 sees, as stored
+    if lt == O.FULL:
+        rows = [np.arange(T1)] * B
+        idx = rows
+    else:
+        tag = cache.tag.cpu().numpy()
+        rows = [np.nonzero(tag[b] >= 0)[0] for b in range(B)]
+        idx = [tag[b][rows[b]] for b in range(B)]
+    hk, hv = [], []
+    for b in range(B):
+        kc = cache.k[b][:, rows[b]].cpu().numpy()
+        vc = cache.v[b][:, rows[b]].cpu().numpy()
+        ks = cache.k_scale[b][:, rows[b]].cpu().numpy()
+        vs = cache.v_scale[b][:, rows[b]].cpu().numpy()
+        hk.append(O.dequantize_e4m3_rows(kc, ks).transpose(1, 0, 2))
+        hv.append(O.dequantize_e4m3_rows(vc, vs).transpose(1, 0, 2))
+    x2 = synth.prefill_inputs(B, T2, seed=53, device="cuda", start=T1)
+    out2 = lib.hyb_attn_prefill(x2["q"], x2["k"], x2["v"], x2["gate"], x2["pos"], lt, cache=cache)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    assert cache.len.tolist() == [T1 + T2] * B
+    ref2 = O.prefill(f64(x2["q"]), f64(x2["k"]), f64(x2["v"]), f64(x2["gate"]), x2["pos"].cpu().numpy(), lt,
+                     start=[T1] * B, hist_k=hk, hist_v=hv, hist_idx=idx)
+    assert_close(out2, ref2, f"chunk 2 lt={lt}")
+
+
+def assert_close(got, ref, what):
+    got = f64(got)
+    max_abs = float(np.abs(got - ref).max())
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    assert max_abs <= 2e-2 and rel <= 5e-3, f"{what}: max_abs {max_abs:.3e} rel_l2 {rel:.3e}"
 
 
 def _fp8_full(lib, B, L, cap, seed):
