@@ -126,12 +126,14 @@ def test_paged_decode_noalloc_and_shared_prefix(lib):
     assert torch.equal(a, b) and torch.equal(b, c)
 
 
-def test_paged_chunked_prefill_equals_contiguous(lib):
+@pytest.mark.parametrize("fp8", [False, True])
+def test_paged_chunked_prefill_equals_contiguous(lib, fp8):
     """Two prefill chunks through a paged cache: the outputs and the cached
     rows equal the contiguous cache's bit for bit (pages of 64 keys, so the
-    prefill's 64-key tiles come from scattered pool pages)."""
+    prefill's 64-key tiles come from scattered pool pages; FP8: the history
+    is dequantized through the table)."""
     B, page, max_pages = 2, 64, 16
-    kvd = lib.KV_BF16
+    kvd = lib.KV_FP8 if fp8 else lib.KV_BF16
     flat = lib.KVCache(O.FULL, B, capacity=page * max_pages, kv_dtype=kvd)
     n_pages = B * max_pages + 5
     paged = lib.KVCache(O.FULL, B, kv_dtype=kvd, page_size=page, n_pages=n_pages,
@@ -147,8 +149,12 @@ def test_paged_chunked_prefill_equals_contiguous(lib):
         start += T
     assert paged.len.tolist() == [start] * B
     for b in range(B):
-        k_, v_ = _gather(paged, b, start)
-        assert torch.equal(k_, flat.k[b, :, :start]) and torch.equal(v_, flat.v[b, :, :start])
+        got = _gather(paged, b, start)
+        ref = [flat.k[b, :, :start], flat.v[b, :, :start]]
+        if fp8:
+            ref += [flat.k_scale[b, :, :start], flat.v_scale[b, :, :start]]
+        for g_, r_ in zip(got, ref):
+            assert torch.equal(g_, r_)
 
 
 def test_paged_layer_decode_equals_contiguous(lib):
