@@ -74,18 +74,18 @@ def layer_seed(base: int, i: int) -> int:
 # the capture's summary).  Reported as roofline.traffic only while the sources are
 # unchanged; otherwise null.
 TRAFFIC = {
-    "prefill_full_T32768": {"bytes": 2.173e9, "sha": "1a078391b3929273",
+    "prefill_full_T32768": {"bytes": 2.2349e9, "sha": "f91bf38ce1984b49",
                             "sources": ["prefill.cu", "common.cuh"],
                             "capture": "profiles/prefill_kernel_full_T32768.md"},
-    "prefill_sliding_T32768": {"bytes": 0.6386e9, "sha": "1a078391b3929273",
+    "prefill_sliding_T32768": {"bytes": 0.6391e9, "sha": "f91bf38ce1984b49",
                                "sources": ["prefill.cu", "common.cuh"],
                                "capture": "profiles/prefill_kernel_sliding_T32768.md"},
     # captured at 16 x 32768 tokens; decode streams each cached byte once, so
     # traffic scales with the tokens: x 8590491648 / 2147483648
-    "decode_full_B16_L131072": {"bytes": 2.1556e9 * 8590491648 / 2147483648, "sha": "46caad3ef3b376c7",
+    "decode_full_B16_L131072": {"bytes": 2.1538e9 * 8590491648 / 2147483648, "sha": "f77e250d919c5a80",
                                 "sources": ["decode.cu", "common.cuh"],
                                 "capture": "profiles/decode_split_kernel_full_B16_L32768.md"},
-    "decode_fp8_full_B16_L131072": {"bytes": 1.0970e9 * 8590491648 / 2147483648, "sha": "46caad3ef3b376c7",
+    "decode_fp8_full_B16_L131072": {"bytes": 1.0972e9 * 8590491648 / 2147483648, "sha": "f77e250d919c5a80",
                                     "sources": ["decode.cu", "common.cuh"],
                                     "capture": "profiles/decode_split_kernel_full_fp8_B16_L32768.md"},
 }

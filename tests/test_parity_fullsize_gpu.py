@@ -145,6 +145,55 @@ def test_decode_batch16_L131072(lib):
             check(out, ref, "sliding decode, 16 sequences")
 
 
+def test_decode_batch16_L131072_fp8(lib):
+    """The bench's FP8 decode configuration: the oracle attends over the
+    seeded codes dequantized (snapshot before any library call) and the new
+    token rotated, rounded to bf16 and quantized by the oracle's quantizer."""
+    B, L = 16, 131072
+    cap = L + 4
+    r = synth.ring_offset(2)
+    full = bench.fill_full_cache(lib, B, L, cap, seed=2, fp8=True)
+    ring = bench.fill_ring_cache(lib, B, L, seed=3, head0=r, fp8=True)
+    seqs = (0, 9)
+
+    def deq(c, b, rows):
+        kc, vc = c.k[b][:, rows].cpu().numpy(), c.v[b][:, rows].cpu().numpy()
+        ks, vs = c.k_scale[b][:, rows].cpu().numpy(), c.v_scale[b][:, rows].cpu().numpy()
+        return (O.dequantize_e4m3_rows(kc, ks).transpose(1, 0, 2), O.dequantize_e4m3_rows(vc, vs).transpose(1, 0, 2))
+
+    hist_full = {b: deq(full, b, np.arange(L)) for b in seqs}
+    n = L + 1
+    idx = np.arange(n - 512, n - 1)
+    slots = (r + idx) % 512
+    hist_ring = [deq(ring, b, slots) for b in range(B)]
+    x = synth.decode_query(B, seed=1001, device="cuda")
+    lib.hyb_kv_append(full, x["k"], x["v"])
+    lib.hyb_kv_append(ring, x["k"], x["v"])
+    out_f = lib.hyb_attn_decode(x["q"], x["gate"], full, max_len=cap)
+    out_r = lib.hyb_attn_decode(x["q"], x["gate"], ring, max_len=512)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    q, g = f64(x["q"]), f64(x["gate"])
+    knew, vnew = f64(x["k"])[:, 0], f64(x["v"])[:, 0]
+    vq, vsc = O.quantize_e4m3_rows(vnew)
+    vn = O.dequantize_e4m3_rows(vq, vsc)
+    for lt, out in ((O.FULL, out_f), (O.SLIDING, out_r)):
+        kr = O.to_bf16(O.rope_layer(knew[:, None], np.full((B, 1), n - 1), lt)[:, 0])
+        kq, ksc = O.quantize_e4m3_rows(kr)
+        kn = O.dequantize_e4m3_rows(kq, ksc)
+        if lt == O.FULL:
+            for b in seqs:
+                kc = np.concatenate([hist_full[b][0], kn[b][None]])
+                vc = np.concatenate([hist_full[b][1], vn[b][None]])
+                ref = O.decode(q[b:b + 1], g[b:b + 1], [n - 1], [kc], [vc], [np.arange(n)], lt)
+                check(out[b:b + 1], ref, f"FP8 full decode seq {b}")
+        else:
+            kc = [np.concatenate([hist_ring[b][0], kn[b][None]]) for b in range(B)]
+            vc = [np.concatenate([hist_ring[b][1], vn[b][None]]) for b in range(B)]
+            ref = O.decode(q, g, [n - 1] * B, kc, vc, [np.append(idx, n - 1)] * B, lt)
+            check(out, ref, "FP8 sliding decode, 16 sequences")
+
+
 def test_decode_1m_64_steps(lib):
     """The 1M-token decode workload's two layer types: 64 steps of append +
     decode, each step compared for all 16 heads.  The oracle keeps its own fp64
