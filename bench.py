@@ -19,11 +19,12 @@ The JSON line also carries:
                 with the full-layer cache in 64-token pages scattered over a pool;
   prefill_128k  one full layer, 131072 tokens: TFLOP/s and % of peak;
   layer_prefill the 4-layer group as whole layers (projections + attention);
-  decode_1m     (--decode-1m) 36-layer decode at 1M tokens: tokens/s (and
-                decode_1m_fp8 over e4m3 caches);
+  decode_1m     36-layer decode at 1M tokens: tokens/s (and decode_1m_fp8
+                over e4m3 caches);
   decode_1m_sharded (--decode-sharded, every rank) the same with the full
                 layers' history spread over the ranks;
-  chunked_prefill (--chunked) 262144 tokens in 8192-token chunks, 36 layers;
+  chunked_prefill 262144 tokens in 8192-token chunks, 36 layers (these two
+                are skipped with --quick);
   cpu_baseline  the fp64 oracle on a bounded sample of the same workload.
 
 `--impl reference` times the oracle as the reference arm instead.
@@ -843,9 +844,11 @@ def main():
     ap.add_argument("--steps", type=int, default=10)
     ap.add_argument("--warmup", type=int, default=3)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
-    ap.add_argument("--decode-1m", action="store_true", help="also run the 36-layer 1M-token decode workload")
+    ap.add_argument("--decode-1m", action="store_true", help="(default) run the 36-layer 1M-token decode workload")
     ap.add_argument("--chunked", action="store_true",
-                    help="also run the 262144-token chunked prefill through 36 layers")
+                    help="(default) run the 262144-token chunked prefill through 36 layers")
+    ap.add_argument("--quick", action="store_true",
+                    help="skip the long sub-benchmarks (1M-token decode, chunked prefill)")
     ap.add_argument("--no-extras", action="store_true", help="only the headline step (no sub-benchmarks)")
     ap.add_argument("--decode-sharded", action="store_true",
                     help="also run the 1M-token decode with the full layers' history spread over the ranks")
@@ -857,6 +860,7 @@ def main():
     ap.add_argument("--seq", type=int, default=16384)
     ap.add_argument("--batch", type=int, default=1)
     args = ap.parse_args()
+    args.decode_1m = args.chunked = not args.quick
     args.warmup = max(args.warmup, 3) if args.impl == "ours" else args.warmup
 
     dist = Dist()
