@@ -313,9 +313,11 @@ hyb_status make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint64
 
 // rope: 0 none; 1 / 2 rotate the 256-wide column tiles below rope_cols as a
 // sliding / full layer's heads (see GemmHost)
+// rope != 0: RoPE epilogue on the column tiles below rope_cols, with the
+// (cos, sin) table of the M rows written first into `rot` (float2 [M][R/2])
 hyb_status linear_impl(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int32_t M,
                        int32_t N, int32_t K, void* stream, int rope = 0, int rope_cols = 0, int32_t T = 0,
-                       const int32_t* pos = nullptr, const int32_t* len = nullptr) {
+                       const int32_t* pos = nullptr, const int32_t* len = nullptr, void* rot = nullptr) {
   if (!x || !w || !y) return fail(HYB_EINVAL, "x, w and y must not be NULL");
   if (M <= 0 || N <= 0 || K <= 0) return fail(HYB_ESHAPE, "M, N, K must be positive (got %d, %d, %d)", M, N, K);
   if (N % 8 || K % 8) return fail(HYB_ESHAPE, "N and K must be multiples of 8 (got %d, %d)", N, K);
@@ -336,9 +338,14 @@ hyb_status linear_impl(const void* x, int64_t ldx, const void* w, int64_t ldw, v
   gh.rope = rope;
   gh.rope_cols = rope_cols;
   gh.T = T;
-  gh.pos = pos;
-  gh.len = len;
-  cudaError_t e = launch_gemm(gh, as_stream(stream));
+  gh.rot = rot;
+  cudaError_t e;
+  if (rope != 0) {
+    if (!rot) return fail(HYB_EINVAL, "RoPE epilogue without its table");
+    if ((e = launch_rope_table(rope == 2, pos, len, T, M, rot, as_stream(stream))) != cudaSuccess)
+      return cuda_fail(e, "rope table launch");
+  }
+  e = launch_gemm(gh, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "linear launch");
   return HYB_OK;
 }
@@ -836,18 +843,20 @@ constexpr int64_t kQkv = (int64_t)(kHq + 2 * kHkv) * kD;   // 6144: fused q | k 
 size_t round256(size_t n) { return (n + 255) & ~(size_t)255; }
 }  // namespace
 
+// fused q|k|v rows, gate scores, attention output, RoPE table (up to 128
+// (cos, sin) pairs per row), then the attention's own scratch
+size_t layer_head_bytes(size_t n) {
+  return round256(n * kQkv * 2) + round256(n * kHq * 2) + round256(n * kHq * kD * 2) + round256(n * 128 * 8);
+}
+
 size_t hyb_attn_layer_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache) {
   if (B <= 0 || T <= 0) return 0;
-  const size_t n = (size_t)B * (size_t)T;
-  return round256(n * kQkv * 2) + round256(n * kHq * 2) + round256(n * kHq * kD * 2) +
-         hyb_attn_prefill_workspace_size(layer_type, B, T, with_cache);
+  return layer_head_bytes((size_t)B * (size_t)T) + hyb_attn_prefill_workspace_size(layer_type, B, T, with_cache);
 }
 
 size_t hyb_attn_layer_prefill_cache_workspace_size(const hyb_kv_cache* cache, int32_t T) {
   if (!cache || T <= 0 || check_cache(cache) != HYB_OK) return 0;
-  const size_t n = (size_t)cache->batch * (size_t)T;
-  return round256(n * kQkv * 2) + round256(n * kHq * 2) + round256(n * kHq * kD * 2) +
-         prefill_ws(cache->type, cache->batch, T, cache);
+  return layer_head_bytes((size_t)cache->batch * (size_t)T) + prefill_ws(cache->type, cache->batch, T, cache);
 }
 
 hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const void* w_gate, const void* w_o,
@@ -876,12 +885,14 @@ hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const v
   p += round256(n * kHq * 2);
   __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(p);
   p += round256(n * kHq * kD * 2);
+  void* rot = p;
+  p += round256(n * 128 * 8);
   const size_t attn_ws = prefill_ws(layer_type, B, T, cache);
   // q_k_v_proj with RoPE of the q and k heads in the epilogue (positions as
   // hyb_attn_prefill: pos, else the cache length + t, else t)
   const int32_t* len = cache ? cache->len : nullptr;
   hyb_status s = linear_impl(hidden, kHidden, w_qkv, kHidden, qkv, kQkv, M, (int32_t)kQkv, (int32_t)kHidden, stream,
-                             layer_type == HYB_FULL ? 2 : 1, (kHq + kHkv) * kD, T, pos, len);
+                             layer_type == HYB_FULL ? 2 : 1, (kHq + kHkv) * kD, T, pos, len, rot);
   if (s != HYB_OK) return s;
   if (w_gate && (s = hyb_linear(hidden, kHidden, w_gate, kHidden, gate, kHq, M, kHq, (int32_t)kHidden, stream)) !=
                     HYB_OK)
@@ -895,9 +906,7 @@ hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const v
 
 size_t hyb_attn_layer_decode_workspace_size(int32_t layer_type, int32_t B, int64_t max_len) {
   if (B <= 0) return 0;
-  const size_t n = (size_t)B;
-  return round256(n * kQkv * 2) + round256(n * kHq * 2) + round256(n * kHq * kD * 2) +
-         hyb_attn_decode_workspace_size(layer_type, B, max_len);
+  return layer_head_bytes((size_t)B) + hyb_attn_decode_workspace_size(layer_type, B, max_len);
 }
 
 hyb_status hyb_attn_layer_decode(const void* hidden, const void* w_qkv, const void* w_gate, const void* w_o,
@@ -924,9 +933,11 @@ hyb_status hyb_attn_layer_decode(const void* hidden, const void* w_qkv, const vo
   p += round256(n * kHq * 2);
   __nv_bfloat16* attn = reinterpret_cast<__nv_bfloat16*>(p);
   p += round256(n * kHq * kD * 2);
+  void* rot = p;
+  p += round256(n * 128 * 8);
   // q_k_v_proj with RoPE at the new token's position (the cache length)
   if ((s = linear_impl(hidden, kHidden, w_qkv, kHidden, qkv, kQkv, B, (int32_t)kQkv, (int32_t)kHidden, stream,
-                       layer_type == HYB_FULL ? 2 : 1, (kHq + kHkv) * kD, 1, nullptr, cache->len)) != HYB_OK)
+                       layer_type == HYB_FULL ? 2 : 1, (kHq + kHkv) * kD, 1, nullptr, cache->len, rot)) != HYB_OK)
     return s;
   if (w_gate && (s = linear_impl(hidden, kHidden, w_gate, kHidden, gate, kHq, B, kHq, (int32_t)kHidden, stream)) !=
                     HYB_OK)

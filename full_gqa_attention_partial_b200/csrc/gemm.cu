@@ -23,6 +23,8 @@
 // as in the attention core): for q_k_v_proj, output column tiles below
 // rope_cols are 256-wide heads (q and k), rotated in fp32 from the
 // accumulator at the row's position before the single rounding to bf16.
+// The (cos, sin) of each (row, frequency) come from a table computed once
+// per call (rope_table_kernel), shared by the row's 20 q and k heads.
 #include "common.cuh"
 #include "launch.h"
 
@@ -44,7 +46,6 @@ struct GemmSmem {
   uint64_t acc_full[2];             // accumulator buffer complete (MMA commit)
   uint64_t acc_empty[2];            // drained: one arrival per epilogue warp of the pair
   uint64_t mma_done;
-  double inv_freq[128];             // RoPE frequencies of the layer type
   uint32_t tmem_base;
 };
 
@@ -59,8 +60,7 @@ struct GemmArgs {
   // RoPE epilogue: row m is token m % T of sequence m / T, at position
   // pos[m] if pos, else (len ? len[m / T] : 0) + m % T
   int rope_cols, T;
-  const int32_t* pos;
-  const int32_t* len;
+  const float2* rot;   // [M][R / 2] (cos, sin) of row m's position x frequency k
 };
 
 // Stores 32 columns (col0 ..) of this thread's row through the warp's staging
@@ -111,7 +111,6 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
     fence_barrier_init();
   }
   constexpr int R = ROPE == 1 ? 256 : 64;   // rotary dims of the layer type
-  if (ROPE && threadIdx.x < R / 2) sm.inv_freq[threadIdx.x] = rope_inv_freq(ROPE == 1 ? 1.0e4 : 5.0e6, threadIdx.x, R);
   if (warp == 5) {
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
@@ -188,7 +187,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
       int first_plain = 0;                                            // chunks below were rotated
       if (rotate) {
         const int m = min(row0 + lane, g.M - 1);
-        const int p = g.pos ? g.pos[m] : (g.len ? g.len[m / g.T] : 0) + m % g.T;
+        const float4* rot_row = reinterpret_cast<const float4*>(g.rot + (int64_t)m * (R / 2));
 #pragma unroll 1
         for (int c = 0; c < R / 64; ++c) {   // dims [32c, 32c+32) against [R/2 + 32c, ...)
           uint32_t u1[32], u2[32];
@@ -197,12 +196,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
           tmem_wait_ld();
           float a1[32], a2[32];
 #pragma unroll
-          for (int i = 0; i < 32; ++i) {
-            float sn, cs;
-            rope_sincos(p, sm.inv_freq[32 * c + i], &sn, &cs);
-            const float x = __uint_as_float(u1[i]), y = __uint_as_float(u2[i]);
-            a1[i] = fmaf(x, cs, -y * sn);
-            a2[i] = fmaf(y, cs, x * sn);
+          for (int i2 = 0; i2 < 16; ++i2) {
+            const float4 t = __ldg(rot_row + 16 * c + i2);   // frequencies 32c + 2 i2, + 1
+#pragma unroll
+            for (int e = 0; e < 2; ++e) {
+              const int i = 2 * i2 + e;
+              const float cs = e ? t.z : t.x, sn = e ? t.w : t.y;
+              const float x = __uint_as_float(u1[i]), y = __uint_as_float(u2[i]);
+              a1[i] = fmaf(x, cs, -y * sn);
+              a2[i] = fmaf(y, cs, x * sn);
+            }
           }
           store_cols32(a1, stg, lane, row0, nt * kGN + 32 * c, g);
           store_cols32(a2, stg, lane, row0, nt * kGN + R / 2 + 32 * c, g);
@@ -255,8 +258,8 @@ cudaError_t launch_gemm(const GemmHost& h, cudaStream_t st) {
   g.n_tiles = (int)n_tiles;
   g.rope_cols = h.rope_cols;
   g.T = h.T > 0 ? h.T : 1;
-  g.pos = h.pos;
-  g.len = h.len;
+  g.rot = reinterpret_cast<const float2*>(h.rot);
+  if (h.rope != 0 && h.rot == nullptr) return cudaErrorInvalidValue;
   const long long grid = 2 * (n_tiles < h.n_pairs ? n_tiles : h.n_pairs);
   if (h.rope == 1)
     gemm_kernel<1><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, g);

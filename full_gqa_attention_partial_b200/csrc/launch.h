@@ -60,6 +60,11 @@ cudaError_t launch_dequant_rows(const void* kc, const void* vc, const float* ks,
 cudaError_t launch_kv_commit(int32_t* len, int32_t* head, int64_t capacity, bool ring, int B, int T,
                              cudaStream_t st);
 cudaError_t launch_selftest_wait(cudaStream_t st);
+// (cos, sin) float2 [M][R / 2] of row m's position x frequency k (R = 64 full,
+// 256 sliding): row m is token m % T of sequence m / T at position pos[m], else
+// (len ? len[m / T] : 0) + m % T
+cudaError_t launch_rope_table(bool full, const int32_t* pos, const int32_t* len, int T, int M, void* tab,
+                              cudaStream_t st);
 cudaError_t launch_fill_i32(int32_t* p, int64_t n, int32_t v, cudaStream_t st);
 
 // ---- linear projections (gemm.cu) -------------------------------------------
@@ -70,11 +75,10 @@ struct GemmHost {
   int M = 0, N = 0, K = 0;
   int n_pairs = 74;            // persistent CTA pairs (SMs / 2)
   // RoPE epilogue: 0 none, 1 sliding-layer, 2 full-layer rotation of the
-  // 256-wide column tiles below rope_cols; row m is token m % T of sequence
-  // m / T at position pos[m], else (len ? len[m / T] : 0) + m % T
+  // 256-wide column tiles below rope_cols, with (cos, sin) from `rot`
+  // (launch_rope_table's [M][R / 2] float2 table)
   int rope = 0, rope_cols = 0, T = 0;
-  const int32_t* pos = nullptr;
-  const int32_t* len = nullptr;
+  const void* rot = nullptr;
 };
 cudaError_t launch_gemm(const GemmHost& h, cudaStream_t st);
 cudaError_t gemm_set_smem_attr();

@@ -14,6 +14,8 @@
 // Keys are rotated with rotate-half RoPE ("百万 Token 塞进 4B ..." §"滑动窗口
 // 的补救：分层 RoPE 与局部/全局分工"): sliding layers theta 1e4 over all 256
 // dims, full layers theta 5e6 over the first 64 dims.
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 
@@ -280,6 +282,25 @@ __global__ void __launch_bounds__(128) ring_gather_kernel(const __nv_bfloat16* r
   }
 }
 
+// RoPE (cos, sin) for every (row, frequency) of a projection's output rows,
+// the same fp64-reduced angle as the other rotations.
+template <bool FULL>
+__global__ void __launch_bounds__(256) rope_table_kernel(const int32_t* pos, const int32_t* len, int T, int M,
+                                                         float2* tab) {
+  constexpr int R = RopeCfg<FULL>::R;
+  __shared__ double inv_freq[R / 2];
+  for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq(RopeCfg<FULL>::theta, i, R);
+  __syncthreads();
+  const int64_t n = (int64_t)M * (R / 2);
+  for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
+    const int m = (int)(idx / (R / 2)), k = (int)(idx % (R / 2));
+    const int p = pos ? pos[m] : (len ? len[m / T] : 0) + m % T;
+    float s, c;
+    rope_sincos(p, inv_freq[k], &s, &c);
+    tab[idx] = make_float2(c, s);
+  }
+}
+
 // Advances the cache state after an append of T tokens.  A full-layer
 // sequence that would overflow its capacity is not advanced (its rows were
 // not written either).
@@ -360,6 +381,18 @@ cudaError_t launch_dequant_rows(const void* kc, const void* vc, const float* ks,
   dequant_rows_kernel<<<grid, 128, 0, st>>>(reinterpret_cast<const uint8_t*>(kc), reinterpret_cast<const uint8_t*>(vc),
                                             ks, vs, pm, cap, len, T, reinterpret_cast<__nv_bfloat16*>(dk),
                                             reinterpret_cast<__nv_bfloat16*>(dv), dst_rows);
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_table(bool full, const int32_t* pos, const int32_t* len, int T, int M, void* tab,
+                              cudaStream_t st) {
+  const int64_t n = (int64_t)M * (full ? 32 : 128);
+  const int grid = (int)std::min<int64_t>((n + 255) / 256, 148 * 8);
+  if (full)
+    rope_table_kernel<true><<<grid, 256, 0, st>>>(pos, len, T > 0 ? T : 1, M, reinterpret_cast<float2*>(tab));
+  else
+    rope_table_kernel<false><<<grid, 256, 0, st>>>(pos, len, T > 0 ? T : 1, M, reinterpret_cast<float2*>(tab));
   count_launch();
   return cudaGetLastError();
 }

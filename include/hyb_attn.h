@@ -316,7 +316,9 @@ hyb_status hyb_linear(const void* x, int64_t ldx, const void* w, int64_t ldw, vo
  *          workspace_size(cache, T) with one (the two agree for bf16 caches),
  *          256-byte aligned; it holds the fused q|k|v rows, the gate scores
  *          and the attention output (bf16, as the model's tensors are)
- *          between the steps, and the attention's own scratch.
+ *          between the steps, the (cos, sin) table of the rows' positions
+ *          that the q_k_v_proj epilogue rotates with, and the attention's own
+ *          scratch.
  * Errors: as hyb_linear and hyb_attn_prefill.
  */
 size_t hyb_attn_layer_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache);
