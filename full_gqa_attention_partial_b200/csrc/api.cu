@@ -789,46 +789,24 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
                                    int32_t layer_type, int64_t max_len, void* out, void* stream) {
   hyb_status s = check_cache(c);
   if (s != HYB_OK) return s;
-  if (!q || !out) return fail(HYB_EINVAL, "q and out must be non-NULL");
-  if (layer_type != c->type) return fail(HYB_ESHAPE, "layer_type %d differs from the cache type %d", layer_type, c->type);
-  if (!aligned16(q) || !aligned16(out)) return fail(HYB_EALIGN, "q and out must be 16-byte aligned");
-  if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
-  if (pos && (reinterpret_cast<uintptr_t>(pos) & 3u)) return fail(HYB_EALIGN, "pos must be 4-byte aligned");
   if (max_len < 0 || max_len > c->capacity)
     return fail(HYB_ESHAPE, "max_len %lld outside [0, capacity %lld]", (long long)max_len, (long long)c->capacity);
-  if (max_len == 0) max_len = c->capacity;
-  const int splits = decode_num_splits(layer_type == HYB_FULL, c->batch, max_len, c->kv_dtype == HYB_KV_FP8);
-  const size_t need = hyb_attn_decode_workspace_size(layer_type, c->batch, max_len);
+  const int64_t ml = max_len == 0 ? c->capacity : max_len;
+  const size_t need = hyb_attn_decode_workspace_size(layer_type, c->batch, ml);
   if (need > kNoAllocScratchBytes)
     return fail(HYB_EOVERFLOW,
                 "batch %d x 16 heads x %d splits needs %zu bytes of split scratch, more than the %zu-byte fixed "
                 "scratch of hyb_attn_decode_noalloc; use hyb_attn_decode with a workspace",
-                c->batch, splits, need, kNoAllocScratchBytes);
+                c->batch, decode_num_splits(layer_type == HYB_FULL, c->batch, ml, c->kv_dtype == HYB_KV_FP8), need,
+                kNoAllocScratchBytes);
   if ((s = ensure_device()) != HYB_OK) return s;
   void* scratch = nullptr;
   size_t scratch_bytes = 0;
   cudaError_t e = decode_noalloc_scratch(&scratch, &scratch_bytes);
   if (e != cudaSuccess) return cuda_fail(e, "cudaGetSymbolAddress(decode scratch)");
-
-  DecodeHost d;
-  d.fp8 = c->kv_dtype == HYB_KV_FP8 ? 1 : 0;
-  if ((s = d.fp8 ? cache_maps_fp8(c, &d.tm_k, &d.tm_v, &d.tm_ks, &d.tm_vs) : cache_maps(c, &d.tm_k, &d.tm_v, 64, 64)) !=
-      HYB_OK)
-    return s;
-  d.q = q;
-  d.gate = gate;
-  d.pos = pos;
-  d.len = c->len;
-  d.tag = c->type == HYB_SLIDING ? c->tag : nullptr;
-  d.out = out;
-  d.B = c->batch;
-  d.pm = page_map(c);
-  d.n_splits = splits;
-  d.part_o = reinterpret_cast<float*>(scratch);
-  d.part_lse = d.part_o + (size_t)c->batch * kHq * d.n_splits * kD;
-  e = launch_decode(layer_type == HYB_FULL, d, as_stream(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
-  return HYB_OK;
+  // the same checks and launches as hyb_attn_decode, with the fixed scratch as its workspace
+  return decode_impl(q, (int64_t)kHq * kD, false, gate, pos, c, layer_type, max_len, out, scratch, scratch_bytes,
+                     stream);
 }
 
 }  // extern "C"
