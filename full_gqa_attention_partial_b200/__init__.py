@@ -108,7 +108,7 @@ def load(path: str = LIB_PATH):
     lib.hyb_attn_layer_decode_workspace_size.restype = sz
     lib.hyb_attn_layer_decode.argtypes = [vp, vp, vp, vp, pc, i32, i64, vp, vp, sz, vp]
     lib.hyb_attn_decode_partial.argtypes = [vp, vp, pc, i32, i64, vp, vp, vp, sz, vp]
-    lib.hyb_attn_decode_merge.argtypes = [vp, vp, i32, i32, vp, vp, vp]
+    lib.hyb_attn_decode_merge.argtypes = [vp, vp, i64, i64, i32, i32, vp, vp, vp]
     lib.hyb_attn_prefill_cache_workspace_size.argtypes = [pc, i32]
     lib.hyb_attn_prefill_cache_workspace_size.restype = sz
     lib.hyb_attn_layer_prefill_cache_workspace_size.argtypes = [pc, i32]
@@ -394,7 +394,37 @@ def hyb_attn_decode_merge(part_o, part_lse, gate=None, out=None, stream=None):
         raise ValueError("gate must be contiguous bf16 [B, 16]")
     if out is None:
         out = torch.empty(B, N_Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=part_o.device)
-    _check(load().hyb_attn_decode_merge(_ptr(part_o), _ptr(part_lse), P, B, _ptr(gate), _ptr(out), _stream(stream)))
+    _check(load().hyb_attn_decode_merge(_ptr(part_o), _ptr(part_lse), 0, 0, P, B, _ptr(gate), _ptr(out),
+                                        _stream(stream)))
+    return out
+
+
+def decode_record_floats(B: int) -> int:
+    """Floats in one partial record: output [B,16,256] then lse [B,16]."""
+    return B * N_Q_HEADS * (HEAD_DIM + 1)
+
+
+def record_views(rec: torch.Tensor, B: int):
+    """(part_o [B,16,256], part_lse [B,16]) views into one fp32 partial record."""
+    n = B * N_Q_HEADS * HEAD_DIM
+    return rec[:n].view(B, N_Q_HEADS, HEAD_DIM), rec[n:n + B * N_Q_HEADS].view(B, N_Q_HEADS)
+
+
+def hyb_attn_decode_merge_records(records, B: int, gate=None, out=None, stream=None):
+    """Merges P partial records (fp32 [P, B*16*257]: each part's output, then
+    its lse), e.g. one all-gather of the per-GPU records; returns bf16 [B,16,256]."""
+    rf = decode_record_floats(B)
+    if records.dtype != torch.float32 or not records.is_contiguous() or records.dim() != 2 \
+            or records.shape[1] != rf:
+        raise ValueError(f"records must be contiguous fp32 [P, {rf}]")
+    if gate is not None and (gate.dtype != torch.bfloat16 or not gate.is_contiguous()
+                             or tuple(gate.shape) != (B, N_Q_HEADS)):
+        raise ValueError("gate must be contiguous bf16 [B, 16]")
+    if out is None:
+        out = torch.empty(B, N_Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=records.device)
+    base = records.data_ptr()
+    _check(load().hyb_attn_decode_merge(ctypes.c_void_p(base), ctypes.c_void_p(base + 4 * B * N_Q_HEADS * HEAD_DIM),
+                                        rf, rf, records.shape[0], B, _ptr(gate), _ptr(out), _stream(stream)))
     return out
 
 

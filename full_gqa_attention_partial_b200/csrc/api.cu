@@ -766,18 +766,25 @@ hyb_status hyb_attn_decode_partial(const void* q, const int32_t* pos, const hyb_
                      workspace_bytes, stream, part_o, part_lse);
 }
 
-hyb_status hyb_attn_decode_merge(const float* part_o, const float* part_lse, int32_t n_parts, int32_t B,
-                                 const void* gate, void* out, void* stream) {
+hyb_status hyb_attn_decode_merge(const float* part_o, const float* part_lse, int64_t o_stride, int64_t lse_stride,
+                                 int32_t n_parts, int32_t B, const void* gate, void* out, void* stream) {
   if (!part_o || !part_lse || !out) return fail(HYB_EINVAL, "part_o, part_lse and out must be non-NULL");
   if (n_parts <= 0 || B <= 0) return fail(HYB_EINVAL, "n_parts = %d and B = %d must be positive", n_parts, B);
-  if ((int64_t)n_parts * B * kHq * kD > (int64_t)0x7fffffff)
-    return fail(HYB_EOVERFLOW, "n_parts x B x 16 x 256 exceeds 2^31 elements");
+  const int64_t rows = (int64_t)B * kHq;
+  if (o_stride == 0) o_stride = rows * kD;
+  if (lse_stride == 0) lse_stride = rows;
+  if (o_stride < rows * kD || lse_stride < rows)
+    return fail(HYB_ESHAPE, "part strides (%lld, %lld) below one part (%lld, %lld floats)", (long long)o_stride,
+                (long long)lse_stride, (long long)(rows * kD), (long long)rows);
+  if ((int64_t)n_parts * o_stride > (int64_t)0x7fffffff || (int64_t)n_parts * lse_stride > (int64_t)0x7fffffff)
+    return fail(HYB_EOVERFLOW, "n_parts x part stride exceeds 2^31 elements");
   if (!aligned16(part_o) || !aligned16(out) || (reinterpret_cast<uintptr_t>(part_lse) & 3u))
     return fail(HYB_EALIGN, "part_o and out must be 16-byte aligned, part_lse 4-byte aligned");
   if (gate && (reinterpret_cast<uintptr_t>(gate) & 1u)) return fail(HYB_EALIGN, "gate must be 2-byte aligned");
   hyb_status s;
   if ((s = ensure_device()) != HYB_OK) return s;
-  cudaError_t e = launch_decode_merge(part_o, part_lse, n_parts, B * kHq, gate, out, as_stream(stream));
+  cudaError_t e =
+      launch_decode_merge(part_o, part_lse, o_stride, lse_stride, n_parts, (int)rows, gate, out, as_stream(stream));
   if (e != cudaSuccess) return cuda_fail(e, "merge launch");
   return HYB_OK;
 }

@@ -494,14 +494,14 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
   a.out[(int64_t)row * kD + d] = __float2bfloat16_rn(r);
 }
 
-cudaError_t launch_decode_merge(const float* part_o, const float* part_lse, int n_parts, int rows,
-                                const void* gate, void* out, cudaStream_t st) {
+cudaError_t launch_decode_merge(const float* part_o, const float* part_lse, int64_t o_stride, int64_t lse_stride,
+                                int n_parts, int rows, const void* gate, void* out, cudaStream_t st) {
   CombineArgs c;
   c.o = part_o;
   c.lse = part_lse;
-  c.o_sstride = (int64_t)rows * kD;
+  c.o_sstride = o_stride;
   c.o_rstride = kD;
-  c.l_sstride = rows;
+  c.l_sstride = lse_stride;
   c.l_rstride = 1;
   c.n = n_parts;
   c.gate = reinterpret_cast<const __nv_bfloat16*>(gate);

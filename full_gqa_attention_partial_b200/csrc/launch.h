@@ -128,10 +128,10 @@ struct DecodeHost {
   float* out_lse = nullptr;    //   log-sum-exp [B][16] instead of the gated bf16 out
 };
 cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st);
-// Merges n_parts partials laid out [n_parts][rows][256] (+ lse [n_parts][rows])
-// into gated bf16 out [rows][256].
-cudaError_t launch_decode_merge(const float* part_o, const float* part_lse, int n_parts, int rows,
-                                const void* gate, void* out, cudaStream_t st);
+// Merges n_parts partials (part p: output [rows][256] at part_o + p * o_stride,
+// lse [rows] at part_lse + p * lse_stride, in floats) into gated bf16 out [rows][256].
+cudaError_t launch_decode_merge(const float* part_o, const float* part_lse, int64_t o_stride, int64_t lse_stride,
+                                int n_parts, int rows, const void* gate, void* out, cudaStream_t st);
 int decode_num_splits(bool full, int B, int64_t max_len, bool fp8);
 // Address and size of the library's fixed decode scratch on the current
 // device (looked up on first use per device).

@@ -14,12 +14,13 @@ holds a part of every sequence's history:
 
 A decode step then runs, on every rank, the attention of the (replicated)
 query over the local part (hyb_attn_decode_partial: normalised output and
-base-2 log-sum-exp per head), one all-gather of those partials (16 heads x
-(256 + 1) fp32 = 16 KB per sequence per rank), and hyb_attn_decode_merge,
-which weighs each part by 2^lse and applies the gate.  Attention over the
-union equals this merge exactly (the split-KV identity), so every rank ends
-the step with the full layer's output, as the replicated layers after it
-expect.  Sliding layers keep their 512-slot rings whole on every rank.
+base-2 log-sum-exp per head, written into one record of 16 heads x (256 +
+1) fp32 = 16 KB per sequence), one all-gather of the records, and
+hyb_attn_decode_merge over the gathered records, which weighs each part by
+2^lse and applies the gate.  Attention over the union equals this merge
+exactly (the split-KV identity), so every rank ends the step with the full
+layer's output, as the replicated layers after it expect.  Sliding layers
+keep their 512-slot rings whole on every rank.
 """
 from __future__ import annotations
 
@@ -60,10 +61,13 @@ class SeqShardedDecoder:
             self.world, self.rank, self.backend = 1, 0, None
         B = cache.batch
         dev = cache.k.device
-        self.part_o = torch.empty(B, 16, 256, dtype=torch.float32, device=dev)
-        self.part_lse = torch.empty(B, 16, dtype=torch.float32, device=dev)
-        self.all_o = torch.empty(self.world, B, 16, 256, dtype=torch.float32, device=dev)
-        self.all_lse = torch.empty(self.world, B, 16, dtype=torch.float32, device=dev)
+        n_o = B * 16 * 256
+        # this rank's record (output, then lse) and every rank's, gathered
+        self.rec = torch.empty(n_o + B * 16, dtype=torch.float32, device=dev)
+        self.part_o = self.rec[:n_o].view(B, 16, 256)
+        self.part_lse = self.rec[n_o:].view(B, 16)
+        self.all_rec = self.rec.view(1, -1) if self.world == 1 else \
+            torch.empty(self.world, n_o + B * 16, dtype=torch.float32, device=dev)
         self.workspace = None
         if dev.type == "cuda":
             need = lib.hyb_attn_decode_workspace_size(cache.layer_type, B, cache.capacity)
@@ -83,15 +87,12 @@ class SeqShardedDecoder:
         lib.hyb_attn_decode_partial(q, self.cache, pos=pos, max_len=self.cache.capacity, part_o=self.part_o,
                                     part_lse=self.part_lse, workspace=self.workspace)
         self._gather()
-        return lib.hyb_attn_decode_merge(self.all_o, self.all_lse, gate)
+        return lib.hyb_attn_decode_merge_records(self.all_rec, self.cache.batch, gate)
 
     def _gather(self):
         if self.world == 1:
-            self.all_o[0].copy_(self.part_o)
-            self.all_lse[0].copy_(self.part_lse)
-        elif self.backend == "nccl":
-            dist.all_gather_into_tensor(self.all_o, self.part_o, group=self.group)
-            dist.all_gather_into_tensor(self.all_lse, self.part_lse, group=self.group)
+            return                      # the only record is this rank's
+        if self.backend == "nccl":
+            dist.all_gather_into_tensor(self.all_rec, self.rec, group=self.group)
         else:
-            dist.all_gather(list(self.all_o.unbind(0)), self.part_o, group=self.group)
-            dist.all_gather(list(self.all_lse.unbind(0)), self.part_lse, group=self.group)
+            dist.all_gather(list(self.all_rec.unbind(0)), self.rec, group=self.group)

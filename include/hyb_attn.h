@@ -237,20 +237,23 @@ hyb_status hyb_attn_decode(const void* q, const void* gate, const int32_t* pos,
  *   part_o  : fp32 [B][16][256], the softmax-normalised output over these keys.
  *   part_lse: fp32 [B][16], log2 of sum_j exp(q . k_j / 16) over these keys
  *             (-inf for a sequence with no keys here; part_o is then 0).
- * hyb_attn_decode_merge: merges n_parts such partials, laid out
- *   part_o [n_parts][B][16][256] and part_lse [n_parts][B][16] (what an
- *   all-gather of the per-GPU partials gives), weighting part p by
- *   2^part_lse[p], applies sigmoid(gate) (bf16 [B][16] or NULL) and writes
- *   bf16 out [B][16][256].  The caller moves the partials between GPUs
- *   (16 KB per sequence per part).
+ * hyb_attn_decode_merge: merges n_parts such partials -- part p's output
+ *   [B][16][256] at part_o + p * o_stride and its lse [B][16] at part_lse +
+ *   p * lse_stride (strides in floats; 0 = dense, B x 4096 and B x 16) --
+ *   weighting part p by 2^lse, applies sigmoid(gate) (bf16 [B][16] or NULL)
+ *   and writes bf16 out [B][16][256].  The caller moves the partials between
+ *   GPUs (16 KB per sequence per part); with each part's output and lse in
+ *   one record of B x 16 x 257 floats (lse after the output), one
+ *   all-gather of the records and o_stride = lse_stride = B x 16 x 257 do it.
  * Errors: as hyb_attn_decode; merge: HYB_EINVAL (null buffer, n_parts or
- * B <= 0), HYB_EALIGN, HYB_EOVERFLOW (more than 2^31 elements).
+ * B <= 0), HYB_ESHAPE (a stride below one part), HYB_EALIGN, HYB_EOVERFLOW
+ * (more than 2^31 elements).
  */
 hyb_status hyb_attn_decode_partial(const void* q, const int32_t* pos, const hyb_kv_cache* cache,
                                    int32_t layer_type, int64_t max_len, float* part_o, float* part_lse,
                                    void* workspace, size_t workspace_bytes, void* stream);
-hyb_status hyb_attn_decode_merge(const float* part_o, const float* part_lse, int32_t n_parts, int32_t B,
-                                 const void* gate, void* out, void* stream);
+hyb_status hyb_attn_decode_merge(const float* part_o, const float* part_lse, int64_t o_stride, int64_t lse_stride,
+                                 int32_t n_parts, int32_t B, const void* gate, void* out, void* stream);
 
 /*
  * hyb_attn_decode without a workspace.  The pages describe no counterpart:

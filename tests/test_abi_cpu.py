@@ -145,12 +145,14 @@ def test_partial_and_merge_checks_before_any_cuda_call(hyb):
                                        None) == -3
     assert lib.hyb_attn_decode_partial(A, None, ctypes.byref(c), 0, 0, A, A, A, 1 << 20, None) == -2   # type
     # merge: null buffers, non-positive counts, misalignment
-    assert lib.hyb_attn_decode_merge(None, A, 2, 1, None, A, None) == -1
-    assert lib.hyb_attn_decode_merge(A, A, 0, 1, None, A, None) == -1
-    assert lib.hyb_attn_decode_merge(A, A, 2, -1, None, A, None) == -1
-    assert lib.hyb_attn_decode_merge(A, ctypes.c_void_p(0x10002), 2, 1, None, A, None) == -3
-    assert lib.hyb_attn_decode_merge(A, A, 2, 1, ctypes.c_void_p(0x10001), A, None) == -3
-    assert lib.hyb_attn_decode_merge(A, A, 1 << 20, 1 << 10, None, A, None) == -4            # > 2^31 elements
+    assert lib.hyb_attn_decode_merge(None, A, 0, 0, 2, 1, None, A, None) == -1
+    assert lib.hyb_attn_decode_merge(A, A, 0, 0, 0, 1, None, A, None) == -1
+    assert lib.hyb_attn_decode_merge(A, A, 0, 0, 2, -1, None, A, None) == -1
+    assert lib.hyb_attn_decode_merge(A, A, 4095, 0, 2, 1, None, A, None) == -2               # stride below a part
+    assert lib.hyb_attn_decode_merge(A, A, 0, 15, 2, 1, None, A, None) == -2
+    assert lib.hyb_attn_decode_merge(A, ctypes.c_void_p(0x10002), 0, 0, 2, 1, None, A, None) == -3
+    assert lib.hyb_attn_decode_merge(A, A, 0, 0, 2, 1, ctypes.c_void_p(0x10001), A, None) == -3
+    assert lib.hyb_attn_decode_merge(A, A, 0, 0, 1 << 20, 1 << 10, None, A, None) == -4      # > 2^31 elements
 
 
 def test_header_is_plain_c_and_links(hyb, tmp_path):

@@ -59,10 +59,12 @@ class _OracleLib:
         part_lse.copy_(torch.from_numpy(lse2))
 
     @staticmethod
-    def hyb_attn_decode_merge(all_o, all_lse, gate):
+    def hyb_attn_decode_merge_records(records, B, gate):
         import oracle as O
+        n = B * 16 * 256
+        r = records.double().numpy()
         g = None if gate is None else gate.double().numpy()
-        return torch.from_numpy(O.merge_partials(all_o.double().numpy(), all_lse.double().numpy(), g))
+        return torch.from_numpy(O.merge_partials(r[:, :n].reshape(-1, B, 16, 256), r[:, n:].reshape(-1, B, 16), g))
 
 
 def _inputs(B, n, seed):
