@@ -83,10 +83,10 @@ TRAFFIC = {
                                "capture": "profiles/prefill_kernel_sliding_T32768.md"},
     # captured at 16 x 32768 tokens; decode streams each cached byte once, so
     # traffic scales with the tokens: x 8590491648 / 2147483648
-    "decode_full_B16_L131072": {"bytes": 2.1538e9 * 8590491648 / 2147483648, "sha": "f77e250d919c5a80",
+    "decode_full_B16_L131072": {"bytes": 2.1536e9 * 8590491648 / 2147483648, "sha": "4683e5d0426bd89b",
                                 "sources": ["decode.cu", "common.cuh"],
                                 "capture": "profiles/decode_split_kernel_full_B16_L32768.md"},
-    "decode_fp8_full_B16_L131072": {"bytes": 1.0972e9 * 8590491648 / 2147483648, "sha": "f77e250d919c5a80",
+    "decode_fp8_full_B16_L131072": {"bytes": 1.0961e9 * 8590491648 / 2147483648, "sha": "4683e5d0426bd89b",
                                     "sources": ["decode.cu", "common.cuh"],
                                     "capture": "profiles/decode_split_kernel_full_fp8_B16_L32768.md"},
 }
