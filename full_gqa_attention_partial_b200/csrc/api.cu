@@ -455,12 +455,24 @@ hyb_status hyb_kv_append(const hyb_kv_cache* c, const void* k, const void* v, in
   return append_impl(c, k, v, kv_row_stride, pos, T, stream, false);
 }
 
-size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache) {
+namespace {
+// Attention scratch: rotated K (standalone) or the sliding context K / V (with
+// a cache); rot_q adds the rotated copy of a sliding layer's queries, which
+// the attention kernel then reads instead of rotating each query tile itself.
+size_t attn_ws(int32_t layer_type, int32_t B, int32_t T, bool with_cache, bool rot_q) {
   if (B <= 0 || T <= 0) return 0;
-  const size_t row = (size_t)kHkv * kD * 2;  // one token of K (or V), 4 heads
-  if (!with_cache) return (size_t)B * (size_t)T * row;                  // rotated K
-  if (layer_type == HYB_FULL) return 0;                                  // reads the cache in place
-  return 2 * (size_t)B * ctx_rows(T) * row;                              // context K and V
+  const size_t row = (size_t)kHkv * kD * 2;  // one token of K (or V), 4 heads (2 KB: keeps 256-byte alignment)
+  size_t n;
+  if (!with_cache) n = (size_t)B * (size_t)T * row;                      // rotated K
+  else if (layer_type == HYB_FULL) n = 0;                                // reads the cache in place
+  else n = 2 * (size_t)B * ctx_rows(T) * row;                            // context K and V
+  if (rot_q && layer_type == HYB_SLIDING) n += (size_t)B * (size_t)T * kHq * kD * 2;
+  return n;
+}
+}  // namespace
+
+size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache) {
+  return attn_ws(layer_type, B, T, with_cache != 0, true);
 }
 
 namespace {
@@ -470,16 +482,16 @@ size_t fp8_copy_bytes(const hyb_kv_cache* c) {
 }
 
 // Scratch of a prefill with cache `c` (NULL: standalone).  An FP8 full-layer
-// cache is attended through bf16 copies of its K and V.
-size_t prefill_ws(int32_t layer_type, int32_t B, int32_t T, const hyb_kv_cache* c) {
+// cache is attended through bf16 copies of its K and V.  rot_q: as attn_ws.
+size_t prefill_ws(int32_t layer_type, int32_t B, int32_t T, const hyb_kv_cache* c, bool rot_q) {
   if (c && c->type == HYB_FULL && c->kv_dtype == HYB_KV_FP8) return 2 * fp8_copy_bytes(c);
-  return hyb_attn_prefill_workspace_size(layer_type, B, T, c != nullptr);
+  return attn_ws(layer_type, B, T, c != nullptr, rot_q);
 }
 }  // namespace
 
 size_t hyb_attn_prefill_cache_workspace_size(const hyb_kv_cache* cache, int32_t T) {
   if (!cache || T <= 0 || check_cache(cache) != HYB_OK) return 0;
-  return prefill_ws(cache->type, cache->batch, T, cache);
+  return prefill_ws(cache->type, cache->batch, T, cache, true);
 }
 
 namespace {
@@ -511,7 +523,10 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
     if (layer_type == HYB_FULL && (int64_t)T > cache->capacity)
       return fail(HYB_ESHAPE, "T = %d exceeds the cache capacity %lld", T, (long long)cache->capacity);
   }
-  const size_t need = prefill_ws(layer_type, B, T, cache);
+  // sliding layers read a rotated copy of the queries (one pass over them)
+  // instead of rotating every query tile in the attention kernel
+  const bool rot_q = layer_type == HYB_SLIDING && !qk_rotated;
+  const size_t need = prefill_ws(layer_type, B, T, cache, rot_q);
   if (need > 0) {
     if (!workspace) return fail(HYB_EINVAL, "workspace of %zu bytes required", need);
     if (reinterpret_cast<uintptr_t>(workspace) & 255u) return fail(HYB_EALIGN, "workspace must be 256-byte aligned");
@@ -524,6 +539,16 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
   const bool full = layer_type == HYB_FULL;
   const uint64_t row_bytes = kD * 2;
   PrefillHost ph;
+  cudaError_t e;
+  bool q_rot = qk_rotated;
+  if (rot_q) {
+    void* qr = reinterpret_cast<uint8_t*>(workspace) + prefill_ws(layer_type, B, T, cache, false);
+    if ((e = launch_rope_q(false, q, q_row_stride, pos, cache ? cache->len : nullptr, B, T, qr, st)) != cudaSuccess)
+      return cuda_fail(e, "query rotation launch");
+    q = qr;
+    q_row_stride = (int64_t)kHq * kD;
+    q_rot = true;
+  }
   if ((s = make_q_map(&ph.tm_q, q, T, B, (uint64_t)q_row_stride * 2, prefill_q_box_rows(), "Q")) != HYB_OK) return s;
   if ((s = make_q_map(&ph.tm_o, out, T, B, (uint64_t)kHq * kD * 2, prefill_q_box_rows(), "out")) != HYB_OK) return s;
   ph.q = q;
@@ -537,8 +562,7 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
   // per two SMs); full layers: long items of unequal length -> one item per
   // pair, handed out longest first by the hardware block scheduler.
   ph.n_pairs = full ? (1 << 29) : device_sms() / 2;
-  ph.q_rotated = qk_rotated ? 1 : 0;
-  cudaError_t e;
+  ph.q_rotated = q_rot ? 1 : 0;
 
   RopeStoreHost r;  // new tokens, token-major input rows
   r.k = k;
@@ -834,14 +858,15 @@ size_t layer_head_bytes(size_t n) {
   return round256(n * kQkv * 2) + round256(n * kHq * 2) + round256(n * kHq * kD * 2) + round256(n * 128 * 8);
 }
 
+// (the layer's queries arrive rotated from the q_k_v_proj epilogue: no query copy)
 size_t hyb_attn_layer_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache) {
   if (B <= 0 || T <= 0) return 0;
-  return layer_head_bytes((size_t)B * (size_t)T) + hyb_attn_prefill_workspace_size(layer_type, B, T, with_cache);
+  return layer_head_bytes((size_t)B * (size_t)T) + attn_ws(layer_type, B, T, with_cache != 0, false);
 }
 
 size_t hyb_attn_layer_prefill_cache_workspace_size(const hyb_kv_cache* cache, int32_t T) {
   if (!cache || T <= 0 || check_cache(cache) != HYB_OK) return 0;
-  return layer_head_bytes((size_t)cache->batch * (size_t)T) + prefill_ws(cache->type, cache->batch, T, cache);
+  return layer_head_bytes((size_t)cache->batch * (size_t)T) + prefill_ws(cache->type, cache->batch, T, cache, false);
 }
 
 hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const void* w_gate, const void* w_o,
@@ -872,7 +897,7 @@ hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const v
   p += round256(n * kHq * kD * 2);
   void* rot = p;
   p += round256(n * 128 * 8);
-  const size_t attn_ws = prefill_ws(layer_type, B, T, cache);
+  const size_t attn_ws = prefill_ws(layer_type, B, T, cache, false);
   // q_k_v_proj with RoPE of the q and k heads in the epilogue (positions as
   // hyb_attn_prefill: pos, else the cache length + t, else t)
   const int32_t* len = cache ? cache->len : nullptr;

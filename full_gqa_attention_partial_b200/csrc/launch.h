@@ -60,6 +60,10 @@ cudaError_t launch_dequant_rows(const void* kc, const void* vc, const float* ks,
 cudaError_t launch_kv_commit(int32_t* len, int32_t* head, int64_t capacity, bool ring, int B, int T,
                              cudaStream_t st);
 cudaError_t launch_selftest_wait(cudaStream_t st);
+// Rotated copy [B][T][16][256] of query rows (16 x 256 at src + (b T + t) src_tstride)
+// at position pos[b][t], else (len ? len[b] : 0) + t
+cudaError_t launch_rope_q(bool full, const void* src, int64_t src_tstride, const int32_t* pos, const int32_t* len,
+                          int B, int T, void* dst, cudaStream_t st);
 // (cos, sin) float2 [M][R / 2] of row m's position x frequency k (R = 64 full,
 // 256 sliding): row m is token m % T of sequence m / T at position pos[m], else
 // (len ? len[m / T] : 0) + m % T

@@ -282,6 +282,67 @@ __global__ void __launch_bounds__(128) ring_gather_kernel(const __nv_bfloat16* r
   }
 }
 
+// Rotated copy of the query rows of a prefill: dst [B][T][16][256] from rows
+// of 16 x 256 at src + (b T + t) src_tstride, at position pos[b][t], else
+// (len ? len[b] : 0) + t.  One block per token: its R/2 (cos, sin) pairs once
+// in shared memory (the fp64-reduced angle), then the 16 heads, one warp per
+// head at a time, 8 dims per lane (the partner dims R/2 away in another lane).
+template <bool FULL>
+__global__ void __launch_bounds__(128) rope_q_kernel(const __nv_bfloat16* src, int64_t src_tstride,
+                                                     const int32_t* pos, const int32_t* len, int B, int T,
+                                                     __nv_bfloat16* dst) {
+  constexpr int R = RopeCfg<FULL>::R;
+  __shared__ double inv_freq[R / 2];
+  __shared__ float2 cs[R / 2];
+  for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq(RopeCfg<FULL>::theta, i, R);
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int d0 = lane * 8;
+  constexpr int xor_mask = (R == 256) ? 16 : 4;
+  for (int64_t m = blockIdx.x; m < (int64_t)B * T; m += gridDim.x) {
+    const int b = (int)(m / T), t = (int)(m % T);
+    const int p = pos ? pos[m] : (len ? len[b] : 0) + t;
+    uint4 qv[kHq / 4];   // this warp's 4 heads, loaded before the angles are ready
+#pragma unroll
+    for (int j = 0; j < kHq / 4; ++j) qv[j] = *reinterpret_cast<const uint4*>(src + m * src_tstride + (warp + 4 * j) * kD + d0);
+    __syncthreads();   // inv_freq written / the previous token's pairs consumed
+    for (int k = threadIdx.x; k < R / 2; k += blockDim.x) {
+      float sn, c;
+      rope_sincos(p, inv_freq[k], &sn, &c);
+      cs[k] = make_float2(c, sn);
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < kHq / 4; ++j) {
+      const int h = warp + 4 * j;
+      uint4 qx = qv[j];
+      const uint32_t xs[4] = {qx.x, qx.y, qx.z, qx.w};
+      uint32_t ys[4];
+#pragma unroll
+      for (int w = 0; w < 4; ++w) ys[w] = __shfl_xor_sync(0xffffffffu, xs[w], xor_mask);
+      if (d0 < R) {
+        const bool first_half = d0 < R / 2;
+        const int kb = first_half ? d0 : d0 - R / 2;
+        uint32_t os[4];
+#pragma unroll
+        for (int w = 0; w < 4; ++w) {
+          float o2[2];
+#pragma unroll
+          for (int e = 0; e < 2; ++e) {
+            const float x = e ? bf16hi(xs[w]) : bf16lo(xs[w]);
+            const float y = e ? bf16hi(ys[w]) : bf16lo(ys[w]);
+            const float2 r = cs[kb + 2 * w + e];
+            // first half: x cos - y sin (y = x[k + R/2]); second half: x cos + y sin (y = x[k])
+            o2[e] = first_half ? fmaf(x, r.x, -y * r.y) : fmaf(x, r.x, y * r.y);
+          }
+          os[w] = pack_bf16(o2[0], o2[1]);
+        }
+        qx = make_uint4(os[0], os[1], os[2], os[3]);
+      }
+      *reinterpret_cast<uint4*>(dst + m * (kHq * kD) + h * kD + d0) = qx;
+    }
+  }
+}
+
 // RoPE (cos, sin) for every (row, frequency) of a projection's output rows,
 // the same fp64-reduced angle as the other rotations.
 template <bool FULL>
@@ -393,6 +454,20 @@ cudaError_t launch_rope_table(bool full, const int32_t* pos, const int32_t* len,
     rope_table_kernel<true><<<grid, 256, 0, st>>>(pos, len, T > 0 ? T : 1, M, reinterpret_cast<float2*>(tab));
   else
     rope_table_kernel<false><<<grid, 256, 0, st>>>(pos, len, T > 0 ? T : 1, M, reinterpret_cast<float2*>(tab));
+  count_launch();
+  return cudaGetLastError();
+}
+
+cudaError_t launch_rope_q(bool full, const void* src, int64_t src_tstride, const int32_t* pos, const int32_t* len,
+                          int B, int T, void* dst, cudaStream_t st) {
+  const int64_t n = (int64_t)B * T;
+  const int grid = (int)std::min<int64_t>(n, 148 * 16);
+  if (full)
+    rope_q_kernel<true><<<grid, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(src), src_tstride, pos, len, B,
+                                              T, reinterpret_cast<__nv_bfloat16*>(dst));
+  else
+    rope_q_kernel<false><<<grid, 128, 0, st>>>(reinterpret_cast<const __nv_bfloat16*>(src), src_tstride, pos, len, B,
+                                               T, reinterpret_cast<__nv_bfloat16*>(dst));
   count_launch();
   return cudaGetLastError();
 }

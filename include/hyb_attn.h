@@ -187,7 +187,9 @@ hyb_status hyb_kv_append(const hyb_kv_cache* cache, const void* k, const void* v
  *          cache->batch must equal B.
  *   workspace: device scratch of at least
  *          hyb_attn_prefill_workspace_size(layer_type, B, T, cache != NULL)
- *          bytes (256-byte aligned); it holds rotated keys between launches.
+ *          bytes (256-byte aligned); it holds rotated keys (or a sliding
+ *          layer's context keys and values) and, for sliding layers, a
+ *          rotated copy of the queries between launches.
  * Errors: HYB_EINVAL, HYB_ESHAPE, HYB_EALIGN, HYB_EOVERFLOW (workspace too
  * small), HYB_EUNSUPPORTED (not an sm_100 device), HYB_ECUDA.
  */

@@ -95,8 +95,9 @@ def test_workspace_sizes(hyb):
     # cache-less prefill holds the rotated keys: B * T * 4 heads * 256 * 2 bytes
     assert hyb.hyb_attn_prefill_workspace_size(hyb.FULL, 2, 1000, False) == 2 * 1000 * 2048
     assert hyb.hyb_attn_prefill_workspace_size(hyb.FULL, 2, 1000, True) == 0
-    # sliding chunk: context K and V of 511 + T rows
-    assert hyb.hyb_attn_prefill_workspace_size(hyb.SLIDING, 1, 8192, True) == 2 * (511 + 8192) * 2048
+    # sliding chunk: context K and V of 511 + T rows, plus the rotated copy of the queries
+    assert hyb.hyb_attn_prefill_workspace_size(hyb.SLIDING, 1, 8192, True) == 2 * (511 + 8192) * 2048 + 8192 * 8192
+    assert hyb.hyb_attn_prefill_workspace_size(hyb.SLIDING, 2, 1000, False) == 2 * 1000 * (2048 + 8192)
     # decode: B * 16 * splits * (256 + 1) floats, rounded up
     for lt, B, L in ((hyb.FULL, 1, 1 << 20), (hyb.FULL, 16, 131073), (hyb.SLIDING, 16, 512)):
         n = hyb.hyb_attn_decode_workspace_size(lt, B, L)
