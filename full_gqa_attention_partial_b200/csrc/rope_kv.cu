@@ -83,11 +83,15 @@ __device__ __forceinline__ void store_row_fp8(uint4 x, uint8_t* dst, float* dsca
 
 // One block = one token of one sequence, 128 threads; thread i handles
 // 8 consecutive dims (16 bytes) of KV head i / 32.  Rotation partners
-// (k, k + R/2) sit in lanes i and i ^ 16 (R = 256) or i ^ 4 (R = 64).
+// (k, k + R/2) sit in lanes i and i ^ 16 (R = 256) or i ^ 4 (R = 64).  The
+// token's R/2 (cos, sin) pairs are computed once (one per thread) into
+// shared memory and shared by the 4 heads.  Every branch that skips a job
+// depends on the job only, so the whole block takes it.
 template <bool FULL>
 __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
   constexpr int R = RopeCfg<FULL>::R;
   __shared__ double inv_freq[R / 2];
+  __shared__ float2 cs[R / 2];
   for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq(RopeCfg<FULL>::theta, i, R);
   __syncthreads();
 
@@ -125,8 +129,17 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
     const int64_t dst = row_id * kD + d0;
 
     uint4 kx = *reinterpret_cast<const uint4*>(a.k + src);
+    // V's load goes out with K's (independent), not after K's rotation and store
+    const uint4 vx = a.v != nullptr ? *reinterpret_cast<const uint4*>(a.v + src) : make_uint4(0, 0, 0, 0);
     if (!a.src_rotated) {
       const int p = a.pos ? a.pos[(int64_t)b * a.T + t] : L + t;
+      __syncthreads();   // the previous job's pairs have been used
+      if (threadIdx.x < R / 2) {
+        float sn, c;
+        rope_sincos(p, inv_freq[threadIdx.x], &sn, &c);
+        cs[threadIdx.x] = make_float2(c, sn);
+      }
+      __syncthreads();
       const uint32_t xs[4] = {kx.x, kx.y, kx.z, kx.w};
       uint32_t ys[4];
       constexpr int xor_mask = (R == 256) ? 16 : 4;
@@ -143,10 +156,9 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
           for (int e = 0; e < 2; ++e) {
             const float x = e ? bf16hi(xs[w]) : bf16lo(xs[w]);
             const float y = e ? bf16hi(ys[w]) : bf16lo(ys[w]);
-            float s, c;
-            rope_sincos(p, inv_freq[kbase + 2 * w + e], &s, &c);
+            const float2 r = cs[kbase + 2 * w + e];
             // first half: x cos - y sin (y = x[k + R/2]); second half: x cos + y sin (y = x[k])
-            o2[e] = first_half ? fmaf(x, c, -y * s) : fmaf(x, c, y * s);
+            o2[e] = first_half ? fmaf(x, r.x, -y * r.y) : fmaf(x, r.x, y * r.y);
           }
           os[w] = pack_bf16(o2[0], o2[1]);
         }
@@ -156,13 +168,13 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
     if (a.fp8) {
       store_row_fp8(kx, reinterpret_cast<uint8_t*>(a.dk) + dst, a.dks + row_id, lane32);
       if (a.v != nullptr)
-        store_row_fp8(*reinterpret_cast<const uint4*>(a.v + src), reinterpret_cast<uint8_t*>(a.dv) + dst,
+        store_row_fp8(vx, reinterpret_cast<uint8_t*>(a.dv) + dst,
                       a.dvs + row_id, lane32);
       continue;
     }
     *reinterpret_cast<uint4*>(a.dk + dst) = kx;
     if (a.v != nullptr) {
-      *reinterpret_cast<uint4*>(a.dv + dst) = *reinterpret_cast<const uint4*>(a.v + src);
+      *reinterpret_cast<uint4*>(a.dv + dst) = vx;
     }
   }
   if (a.commit) {
