@@ -488,3 +488,61 @@ def test_merged_parts_equal_decode_over_the_union():
     o1, l1 = O.decode_partial(q, qpos, list(k), list(v), O.FULL)
     assert np.abs(o1 - O.decode(q, None, qpos, list(k), list(v), [np.arange(L)] * B, O.FULL)).max() < 1e-12
     assert np.abs(O.merge_partials(o1[None], l1[None], gate) - ref).max() < 1e-12
+
+
+# ---------------------------------------------------------------------------
+# Randomised identities (hypothesis): shapes, positions and partitions drawn
+# at random, each checked against a relation the definition implies.
+# ---------------------------------------------------------------------------
+from hypothesis import given, settings, strategies as st  # noqa: E402
+
+
+@settings(max_examples=25, deadline=None)
+@given(lt=st.sampled_from([O.FULL, O.SLIDING]), p=st.integers(0, 1 << 20), shift=st.integers(-5000, 5000),
+       seed=st.integers(0, 2 ** 31 - 1))
+def test_rope_scores_depend_only_on_the_offset(lt, p, shift, seed):
+    """q(m) . k(n) after rotation depends on m - n only, at any positions."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, 1, 256))
+    k = rng.standard_normal((1, 1, 256))
+    n = max(0, p - 777)
+    a = (O.rope_layer(q, np.array([p]), lt) * O.rope_layer(k, np.array([n]), lt)).sum()
+    p2, n2 = max(0, p + shift), max(0, n + shift)
+    if p2 - n2 != p - n:
+        return
+    b = (O.rope_layer(q, np.array([p2]), lt) * O.rope_layer(k, np.array([n2]), lt)).sum()
+    assert abs(a - b) <= 1e-9 * (1 + abs(a))
+
+
+@settings(max_examples=20, deadline=None)
+@given(L=st.integers(1, 60), n_parts=st.integers(1, 4), seed=st.integers(0, 2 ** 31 - 1))
+def test_any_partition_of_the_history_merges_to_decode(L, n_parts, seed):
+    """The log-sum-exp merge of the parts of any partition equals decode."""
+    rng = np.random.default_rng(seed)
+    q = rng.standard_normal((1, 16, 256))
+    gate = rng.standard_normal((1, 16))
+    k = rng.standard_normal((1, L, 4, 256))
+    v = rng.standard_normal((1, L, 4, 256))
+    owner = rng.integers(0, n_parts, size=L)
+    parts = [O.decode_partial(q, [L - 1], [k[0][owner == p]], [v[0][owner == p]], O.FULL) for p in range(n_parts)]
+    got = O.merge_partials(np.stack([p[0] for p in parts]), np.stack([p[1] for p in parts]), gate)
+    ref = O.decode(q, gate, [L - 1], [k[0]], [v[0]], [np.arange(L)], O.FULL)
+    assert np.abs(got - ref).max() < 1e-12
+
+
+@settings(max_examples=20, deadline=None)
+@given(codes=st.lists(st.integers(0, 255).filter(lambda c: c & 0x7F != 0x7F), min_size=256, max_size=256),
+       scale=st.floats(1e-6, 1e6))
+def test_e4m3_requantizing_a_dequantized_row_is_identity(codes, scale):
+    """quantize(dequantize(codes, s)) gives the codes back (up to the sign of
+    zero) when the row's largest code is 448: the scale is recovered (to the
+    fp32 rounding of 448 s) and every value is on the e4m3 grid."""
+    c = np.array(codes, dtype=np.uint8).reshape(1, 256)
+    c[0, 0] = 0x7E                                  # +448 sets amax
+    vals = O.dequantize_e4m3_rows(c, np.array([scale], dtype=np.float32))
+    c2, s2 = O.quantize_e4m3_rows(vals)
+    s32 = float(np.float32(scale))
+    assert abs(float(s2[0]) - s32) <= 2.0 ** -22 * s32
+    zero = (c & 0x7F) == 0
+    assert np.array_equal(c2[~zero], c[~zero])
+    assert np.all((c2[zero] & 0x7F) == 0)
