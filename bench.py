@@ -267,8 +267,14 @@ def bench_main(hyb, args, dist: Dist, peaks):
     full_ms = statistics.mean(per_layer[3])
     slide_ms = statistics.mean(t for li in range(3) for t in per_layer[li])
     total_s = ms / 1e3
-    peak = peaks["bf16_tflops_sustained"] if total_s >= 1.0 else peaks["bf16_tflops"]
-    peak_kind = "sustained" if total_s >= 1.0 else "burst"
+    # Inside a continuous run of tens of milliseconds the tensor-heavy launches
+    # run under the power cap: back to back, full-layer launches take 6.2 ms for
+    # the first ~30 ms and 7.0 ms after, so a kernel timed inside the step is
+    # compared with the sustained (power-capped, seconds-long) cuBLAS figure;
+    # the burst fraction is reported beside it.
+    sustained = total_s >= 0.05
+    peak = peaks["bf16_tflops_sustained"] if sustained else peaks["bf16_tflops"]
+    peak_kind = "sustained (kernel inside a continuous step run)" if sustained else "burst"
     achieved = flops(T_MAIN, FULL) / (full_ms / 1e3) / 1e12
     kernel_share = sum(kt) / (ms / 1.0) if ms > 0 else None
     res = {
@@ -279,8 +285,10 @@ def bench_main(hyb, args, dist: Dist, peaks):
             "bound": "tensor", "kernel": "prefill_kernel<FULL> (tcgen05)", "achieved": achieved,
             "peak": peak, "unit": "TFLOP/s", "frac": achieved / peak,
             "peak_source": f"{peaks['source']} bf16 {peak_kind}",
+            "frac_of_burst_peak": achieved / peaks["bf16_tflops"], "burst_peak": peaks["bf16_tflops"],
             "algorithmic_flops_per_launch": flops(T_MAIN, FULL),
             "avg_launch_ms": full_ms, "launches": len(per_layer[3]),
+            "first_last_launch_ms": [per_layer[3][0], per_layer[3][-1]],
             "traffic": traffic_of("prefill_full_T32768"),
             "sliding_kernel": {"avg_launch_ms": slide_ms,
                                "achieved": flops(T_MAIN, SLIDING) / (slide_ms / 1e3) / 1e12,
