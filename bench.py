@@ -174,7 +174,10 @@ class Clocks:
 
     def __init__(self):
         self.proc = None
-        self.path = os.path.join(ROOT, "gpurun_out", f"clocks_rank{os.environ.get('RANK', '0')}.csv")
+        # raw samples go to $HYB_BENCH_OUT (default: the system's temporary directory)
+        import tempfile
+        out_dir = os.environ.get("HYB_BENCH_OUT") or tempfile.gettempdir()
+        self.path = os.path.join(out_dir, f"hyb_clocks_rank{os.environ.get('RANK', '0')}.csv")
 
     def start(self):
         try:

@@ -23,7 +23,7 @@ Sources (web pages; titles abbreviated as below):
 [CONFIG]   "读懂Spark-X2.6-4B的config.json：混合注意力与1M上下文的架构入门路线图"
            (sheratonhq.com).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 * window edge: a sliding query at index t sees keys j with 0 <= t - j <= 511
   (512 keys including itself);
 * softmax scale 1/sqrt(256) = 1/16, no soft-cap, no sinks;
