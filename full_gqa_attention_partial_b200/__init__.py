@@ -250,7 +250,7 @@ def hyb_attn_prefill(q, k, v, gate, pos, layer_type: int, out=None, cache: KVCac
     if out is None:
         out = torch.empty(B, T, N_Q_HEADS, HEAD_DIM, dtype=torch.bfloat16, device=q.device)
     need = hyb_attn_prefill_workspace_size(layer_type, B, T, False) if cache is None else \
-        int(load().hyb_attn_prefill_cache_workspace_size(cache.ref, T))
+        hyb_attn_prefill_cache_workspace_size(cache, T)
     if workspace is None and need > 0:
         workspace = alloc_workspace(need, q.device)
     wsz = 0 if workspace is None else workspace.numel() * workspace.element_size()
@@ -261,6 +261,18 @@ def hyb_attn_prefill(q, k, v, gate, pos, layer_type: int, out=None, cache: KVCac
 
 
 HIDDEN = 2560
+
+
+def hyb_attn_layer_decode_workspace_size(layer_type: int, B: int, max_len: int) -> int:
+    return int(load().hyb_attn_layer_decode_workspace_size(layer_type, B, max_len))
+
+
+def hyb_attn_prefill_cache_workspace_size(cache: "KVCache", T: int) -> int:
+    return int(load().hyb_attn_prefill_cache_workspace_size(cache.ref, T))
+
+
+def hyb_attn_layer_prefill_cache_workspace_size(cache: "KVCache", T: int) -> int:
+    return int(load().hyb_attn_layer_prefill_cache_workspace_size(cache.ref, T))
 
 
 def hyb_attn_layer_prefill_workspace_size(layer_type: int, B: int, T: int, with_cache: bool) -> int:
@@ -285,7 +297,7 @@ def hyb_attn_layer_prefill(hidden, w_qkv, w_gate, w_o, pos, layer_type: int, out
     if out is None:
         out = torch.empty(B, T, HIDDEN, dtype=torch.bfloat16, device=hidden.device)
     need = hyb_attn_layer_prefill_workspace_size(layer_type, B, T, False) if cache is None else \
-        int(load().hyb_attn_layer_prefill_cache_workspace_size(cache.ref, T))
+        hyb_attn_layer_prefill_cache_workspace_size(cache, T)
     if workspace is None:
         workspace = alloc_workspace(need, hidden.device)
     wsz = workspace.numel() * workspace.element_size()
@@ -310,7 +322,7 @@ def hyb_attn_layer_decode(hidden, w_qkv, w_gate, w_o, cache: KVCache, max_len: i
     if out is None:
         out = torch.empty(B, HIDDEN, dtype=torch.bfloat16, device=hidden.device)
     lt = cache.layer_type
-    need = int(load().hyb_attn_layer_decode_workspace_size(lt, B, max_len or cache.capacity))
+    need = hyb_attn_layer_decode_workspace_size(lt, B, max_len or cache.capacity)
     if workspace is None:
         workspace = alloc_workspace(need, hidden.device)
     wsz = workspace.numel() * workspace.element_size()

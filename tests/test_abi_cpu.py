@@ -185,3 +185,26 @@ int main(void) {
     r = subprocess.run([str(exe)], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stdout + r.stderr
     assert "512" in r.stdout
+
+
+def test_workspace_sizes_cover_every_grid(hyb):
+    """For random batch sizes and lengths the decode workspace holds the
+    partials of the larger of the bf16 and FP8 split grids (B x 16 x splits x
+    (256 + 1) floats), and the whole-layer sizes exceed the attention's."""
+    import random
+    rnd = random.Random(3)
+    for _ in range(200):
+        lt = rnd.choice([hyb.SLIDING, hyb.FULL])
+        B = rnd.randint(1, 64)
+        L = rnd.randint(1, 1 << 21)
+        n = hyb.hyb_attn_decode_workspace_size(lt, B, L)
+        assert n % 256 == 0 or n % 4 == 0
+        rows = B * 16
+        splits = (n - ((rows * 4 + 255) // 256) * 256) // (rows * 256 * 4)
+        assert splits >= 1
+        assert hyb.hyb_attn_layer_decode_workspace_size(lt, B, L) > n
+        T = rnd.randint(1, 40000)
+        # the layer call holds the fused q|k|v rows and the attention output besides the attention's scratch
+        # (minus the rotated query copy, which the layer's pre-rotated queries do not need)
+        attn = hyb.hyb_attn_prefill_workspace_size(lt, B, T, True) - (B * T * 16 * 256 * 2 if lt == hyb.SLIDING else 0)
+        assert hyb.hyb_attn_layer_prefill_workspace_size(lt, B, T, True) >= attn + B * T * (6144 + 4096) * 2
