@@ -331,15 +331,35 @@ def hyb_attn_layer_decode(hidden, w_qkv, w_gate, w_o, cache: KVCache, max_len: i
     return out
 
 
-def hyb_attn_decode(q, gate, cache: KVCache, pos=None, max_len: int = 0, out=None, workspace=None,
-                    stream=None):
-    """One decode step.  q [B,16,256] contiguous, gate [B,16] or None.  Returns out [B,16,256]."""
-    if q.dtype != torch.bfloat16 or not q.is_contiguous() or tuple(q.shape[1:]) != (N_Q_HEADS, HEAD_DIM):
+
+def _check_decode_args(q, gate, pos, cache: "KVCache", out=None):
+    """Host-side checks of a decode call's tensors against the cache.
+
+    The kernels launch one block row per cache sequence and read q / pos and
+    write out for every one of them, so a q, pos or out with fewer rows than
+    cache.batch would be read or written out of bounds: reject it here."""
+    if q.dtype != torch.bfloat16 or not q.is_contiguous() or q.dim() != 3 \
+            or tuple(q.shape[1:]) != (N_Q_HEADS, HEAD_DIM):
         raise ValueError("q must be contiguous bf16 [B, 16, 256]")
     B = q.shape[0]
+    if B != cache.batch:
+        raise ValueError(f"q has {B} sequences, the cache {cache.batch}")
     if gate is not None and (gate.dtype != torch.bfloat16 or not gate.is_contiguous()
                              or tuple(gate.shape) != (B, N_Q_HEADS)):
         raise ValueError("gate must be contiguous bf16 [B, 16]")
+    if pos is not None and (pos.dtype != torch.int32 or not pos.is_contiguous() or tuple(pos.shape) != (B,)):
+        raise ValueError("pos must be contiguous int32 [B]")
+    if out is not None and (out.dtype != torch.bfloat16 or not out.is_contiguous()
+                            or tuple(out.shape) != (B, N_Q_HEADS, HEAD_DIM)):
+        raise ValueError("out must be contiguous bf16 [B, 16, 256]")
+    return B
+
+
+def hyb_attn_decode(q, gate, cache: KVCache, pos=None, max_len: int = 0, out=None, workspace=None,
+                    stream=None):
+    """One decode step.  q [B,16,256] contiguous (B = cache.batch), gate [B,16] or None,
+    pos int32 [B] or None.  Returns out [B,16,256]."""
+    _check_decode_args(q, gate, pos, cache, out)
     if out is None:
         out = torch.empty_like(q)
     ml = max_len if max_len else cache.capacity
@@ -357,12 +377,7 @@ def hyb_attn_decode_noalloc(q, gate, cache: KVCache, pos=None, max_len: int = 0,
     scratch inside the library, shared by all calls (calls that overlap on
     the GPU race on it).  `out` should be preallocated by such callers; when
     it is None a tensor is allocated here for convenience."""
-    if q.dtype != torch.bfloat16 or not q.is_contiguous() or tuple(q.shape[1:]) != (N_Q_HEADS, HEAD_DIM):
-        raise ValueError("q must be contiguous bf16 [B, 16, 256]")
-    B = q.shape[0]
-    if gate is not None and (gate.dtype != torch.bfloat16 or not gate.is_contiguous()
-                             or tuple(gate.shape) != (B, N_Q_HEADS)):
-        raise ValueError("gate must be contiguous bf16 [B, 16]")
+    _check_decode_args(q, gate, pos, cache, out)
     if out is None:
         out = torch.empty_like(q)
     _check(load().hyb_attn_decode_noalloc(_ptr(q), _ptr(gate), _ptr(pos), cache.ref, cache.layer_type, max_len,
@@ -376,18 +391,21 @@ def hyb_attn_decode_partial(q, cache: KVCache, pos=None, max_len: int = 0, part_
     (part_o fp32 [B,16,256] normalised over these keys, part_lse fp32 [B,16] =
     log2 sum_j exp(q.k_j / 16)).  pos: int32 [B] query positions in the whole
     sequence (None: len - 1 of this cache)."""
-    if q.dtype != torch.bfloat16 or not q.is_contiguous() or tuple(q.shape[1:]) != (N_Q_HEADS, HEAD_DIM):
-        raise ValueError("q must be contiguous bf16 [B, 16, 256]")
-    B = q.shape[0]
+    B = _check_decode_args(q, None, pos, cache)
     if part_o is None:
         part_o = torch.empty(B, N_Q_HEADS, HEAD_DIM, dtype=torch.float32, device=q.device)
     if part_lse is None:
         part_lse = torch.empty(B, N_Q_HEADS, dtype=torch.float32, device=q.device)
+    if part_o.dtype != torch.float32 or not part_o.is_contiguous() or tuple(part_o.shape) != (B, N_Q_HEADS, HEAD_DIM):
+        raise ValueError("part_o must be contiguous fp32 [B, 16, 256]")
+    if part_lse.dtype != torch.float32 or not part_lse.is_contiguous() or tuple(part_lse.shape) != (B, N_Q_HEADS):
+        raise ValueError("part_lse must be contiguous fp32 [B, 16]")
     need = hyb_attn_decode_workspace_size(cache.layer_type, B, max_len or cache.capacity)
     if workspace is None:
         workspace = alloc_workspace(need, q.device)
+    wsz = workspace.numel() * workspace.element_size()
     _check(load().hyb_attn_decode_partial(_ptr(q), _ptr(pos), cache.ref, cache.layer_type, max_len, _ptr(part_o),
-                                          _ptr(part_lse), _ptr(workspace), workspace.numel(), _stream(stream)))
+                                          _ptr(part_lse), _ptr(workspace), wsz, _stream(stream)))
     return part_o, part_lse
 
 

@@ -15,7 +15,12 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libhyb_attn.so")
-SOURCES = ["hyb_attn_lib.cu", "rope_kv.cu", "decode.cu", "prefill.cu", "api.cu", "common.cuh", "launch.h"]
+
+
+def sources() -> list:
+    """Every file under csrc/ (the unity build includes them all)."""
+    return sorted(os.path.join(CSRC, f) for f in os.listdir(CSRC)
+                  if f.endswith((".cu", ".cuh", ".h")))
 
 
 def nvcc() -> str:
@@ -29,7 +34,7 @@ def needs_build() -> bool:
     if not os.path.exists(LIB):
         return True
     t = os.path.getmtime(LIB)
-    deps = [os.path.join(CSRC, s) for s in SOURCES] + [os.path.join(ROOT, "include", "hyb_attn.h")]
+    deps = sources() + [os.path.join(ROOT, "include", "hyb_attn.h")]
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 

@@ -826,10 +826,13 @@ hyb_status hyb_attn_decode_noalloc(const void* q, const void* gate, const int32_
   const size_t need = hyb_attn_decode_workspace_size(layer_type, c->batch, ml);
   if (need > kNoAllocScratchBytes)
     return fail(HYB_EOVERFLOW,
-                "batch %d x 16 heads x %d splits needs %zu bytes of split scratch, more than the %zu-byte fixed "
-                "scratch of hyb_attn_decode_noalloc; use hyb_attn_decode with a workspace",
-                c->batch, decode_num_splits(layer_type == HYB_FULL, c->batch, ml, c->kv_dtype == HYB_KV_FP8), need,
-                kNoAllocScratchBytes);
+                "batch %d x 16 heads x %d splits (the larger of the bf16 and FP8 split grids) needs %zu bytes of "
+                "split scratch, more than the %zu-byte fixed scratch of hyb_attn_decode_noalloc; use "
+                "hyb_attn_decode with a workspace",
+                c->batch,
+                std::max(decode_num_splits(layer_type == HYB_FULL, c->batch, ml, false),
+                         decode_num_splits(layer_type == HYB_FULL, c->batch, ml, true)),
+                need, kNoAllocScratchBytes);
   if ((s = ensure_device()) != HYB_OK) return s;
   void* scratch = nullptr;
   size_t scratch_bytes = 0;

@@ -33,6 +33,8 @@
 // goes onto the split's output.  P then stays below the bf16 maximum for any
 // V row of amax up to 448 * 2^64, and the products P V stay far above the
 // fp32 subnormal range.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -597,23 +599,41 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
 constexpr size_t kNoAllocScratchBytes = size_t(4) << 20;
 static __device__ __align__(256) float g_decode_scratch[kNoAllocScratchBytes / sizeof(float)];
 
-// Device address of g_decode_scratch on the current device.  In host code
-// the array's name is only a host-side stand-in, so the address is looked
-// up with cudaGetSymbolAddress, once per device, the first time a device
-// uses it (with that device current), and cached.
+// Device address of g_decode_scratch in the current context.  In host code
+// the array's name is only a host-side stand-in, so the address is looked up
+// with cudaGetSymbolAddress, once per device, the first time a device uses it
+// (with that device current), and cached together with the CUDA context it
+// was found in.  A different current context on that device (after
+// cudaDeviceReset, or a context the caller created itself) has the module
+// loaded again at another address: the cached entry no longer matches the
+// context, and the address is looked up again.
 cudaError_t decode_noalloc_scratch(void** ptr, size_t* bytes) {
   static std::mutex mu;
   static void* addr[128] = {};
+  static CUcontext ctx_of[128] = {};
+  static PFN_cuCtxGetCurrent_v4000 get_ctx = nullptr;
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   if (dev < 0 || dev >= 128) return cudaErrorInvalidDevice;
   std::lock_guard<std::mutex> lk(mu);
-  if (addr[dev] == nullptr) {
+  if (get_ctx == nullptr) {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    e = cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q);
+    if (e != cudaSuccess) return e;
+    if (q != cudaDriverEntryPointSuccess || fn == nullptr) return cudaErrorNotSupported;
+    get_ctx = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(fn);
+  }
+  // the caller's earlier runtime calls on this device (its set-up) made a context current
+  CUcontext ctx = nullptr;
+  if (get_ctx(&ctx) != CUDA_SUCCESS || ctx == nullptr) return cudaErrorDeviceUninitialized;
+  if (addr[dev] == nullptr || ctx_of[dev] != ctx) {
     void* p = nullptr;
     e = cudaGetSymbolAddress(&p, g_decode_scratch);
     if (e != cudaSuccess) return e;
     addr[dev] = p;
+    ctx_of[dev] = ctx;
   }
   *ptr = addr[dev];
   *bytes = kNoAllocScratchBytes;

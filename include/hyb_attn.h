@@ -208,6 +208,9 @@ hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const v
 /*
  * One decode step: one query token per sequence against its cache, which
  * must already hold the token itself (call hyb_kv_append first).
+ * B is cache->batch: the kernels read q, gate and pos and write out for
+ * every sequence of the cache, so each of them must hold B rows (the call
+ * has no separate batch argument to check them against).
  *   q    : bf16 [B][16][256] contiguous query (not rotated).
  *   gate : bf16 [B][16] or NULL.
  *   pos  : device int32 [B] RoPE position of the query, or NULL (len - 1).
@@ -273,7 +276,9 @@ hyb_status hyb_attn_decode_merge(const float* part_o, const float* part_lse, int
  *   nothing.
  *   Set-up: the first call on a device looks up the scratch's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call
- *   before any stream capture.
+ *   before any stream capture.  The address is cached with the CUDA context
+ *   it belongs to: after cudaDeviceReset, or from another context, the next
+ *   call looks it up again (make that call outside a capture too).
  *   Sharing: every call uses the same scratch, which keeps the previous
  *   call's contents (nothing in it needs to start at zero).  Calls whose
  *   kernels can overlap on the GPU -- e.g. on two streams without ordering

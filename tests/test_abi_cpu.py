@@ -208,3 +208,47 @@ def test_workspace_sizes_cover_every_grid(hyb):
         # (minus the rotated query copy, which the layer's pre-rotated queries do not need)
         attn = hyb.hyb_attn_prefill_workspace_size(lt, B, T, True) - (B * T * 16 * 256 * 2 if lt == hyb.SLIDING else 0)
         assert hyb.hyb_attn_layer_prefill_workspace_size(lt, B, T, True) >= attn + B * T * (6144 + 4096) * 2
+
+
+class _FakeCache:
+    """Stands in for a KVCache in the binding's host-side checks (no device memory)."""
+
+    def __init__(self, batch, layer_type=0, capacity=512):
+        self.batch, self.layer_type, self.capacity = batch, layer_type, capacity
+
+    @property
+    def ref(self):   # reaching the library would mean a check was skipped
+        raise AssertionError("the call got past the binding's checks")
+
+
+@pytest.mark.parametrize("fn", ["hyb_attn_decode", "hyb_attn_decode_noalloc", "hyb_attn_decode_partial"])
+def test_decode_wrappers_reject_shape_mismatches_before_any_launch(hyb, fn):
+    import torch
+    call = getattr(hyb, fn)
+    cache = _FakeCache(batch=3)
+    bf = torch.bfloat16
+
+    def go(q, gate=None, pos=None, out=None):
+        if fn == "hyb_attn_decode_partial":
+            return call(q, cache, pos=pos)
+        return call(q, gate, cache, pos=pos, out=out)
+
+    good_q = torch.zeros(3, 16, 256, dtype=bf)
+    bad = [
+        dict(q=torch.zeros(2, 16, 256, dtype=bf)),                       # fewer sequences than the cache
+        dict(q=torch.zeros(4, 16, 256, dtype=bf)),                       # more sequences than the cache
+        dict(q=torch.zeros(3, 16, 256, dtype=torch.float16)),            # wrong dtype
+        dict(q=torch.zeros(3, 256, 16, dtype=bf).transpose(1, 2)),       # not contiguous
+        dict(q=good_q, pos=torch.zeros(2, dtype=torch.int32)),           # pos too short
+        dict(q=good_q, pos=torch.zeros(3, dtype=torch.int64)),           # pos not int32
+        dict(q=good_q, pos=torch.zeros(6, dtype=torch.int32)[::2]),      # pos not contiguous
+    ]
+    if fn != "hyb_attn_decode_partial":
+        bad += [
+            dict(q=good_q, gate=torch.zeros(2, 16, dtype=bf)),               # gate too short
+            dict(q=good_q, out=torch.zeros(2, 16, 256, dtype=bf)),           # out too short
+            dict(q=good_q, out=torch.zeros(3, 16, 256, dtype=torch.float32)),  # out not bf16
+        ]
+    for kw in bad:
+        with pytest.raises(ValueError):
+            go(**kw)
