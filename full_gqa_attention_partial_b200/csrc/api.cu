@@ -523,8 +523,9 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
     if (layer_type == HYB_FULL && (int64_t)T > cache->capacity)
       return fail(HYB_ESHAPE, "T = %d exceeds the cache capacity %lld", T, (long long)cache->capacity);
   }
-  // sliding layers read a rotated copy of the queries (one pass over them)
-  // instead of rotating every query tile in the attention kernel
+  // sliding layers read a rotated copy of the queries (one pass over them): the
+  // attention kernel rotates query tiles itself on full layers only (64 rotary
+  // dims), where it costs little next to the long key loop of each tile
   const bool rot_q = layer_type == HYB_SLIDING && !qk_rotated;
   const size_t need = prefill_ws(layer_type, B, T, cache, rot_q);
   if (need > 0) {

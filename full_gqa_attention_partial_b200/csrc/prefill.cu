@@ -8,84 +8,112 @@
 // query and the 511 keys before it on sliding layers (same page, §"混合注意力").
 // Key tiles wholly outside the band are never loaded.
 //
-// The pair shares every K/V tile: each CTA loads half of it (32 of the 64
-// keys of a K tile, 128 of the 256 dims of a V tile) and the pair MMAs
-// (cta_group::2, M = 256: 128 rows per CTA) read both halves, so each SM
-// draws 32 KB from L2 per 64-key tile instead of 64 KB.
+// Key tiles hold 128 keys.  The pair shares every K/V tile: each CTA loads
+// half of it (64 of the 128 keys of a K tile, 128 of the 256 dims of a V
+// tile) and the pair MMAs (cta_group::2, M = 256: 128 rows per CTA) read
+// both halves, so each SM draws 64 KB from L2 per 128-key tile instead of
+// 128 KB.  Per 128 keys the pair issues 16 MMAs for S = Q K^T (N = 128) and
+// 8 for O += P V (K = 16 keys each): with 64-key tiles the MMA-issuing
+// warp, at about 40 cycles per MMA and a few hundred per barrier wait, could
+// not keep the tensor pipe fed.
 //
-// Roles in each CTA (192 threads):
-//   warps 0-3  rotate this CTA's query head in place in the shared-memory
-//              query tile (rotate-half RoPE, theta / rotary dim per layer
-//              type); then the online softmax (one TMEM lane = one query row
-//              per thread) and the epilogue (1/l, sigmoid gate, bf16, TMA
-//              store);
-//   warp 4     lane 0: TMA producer for this CTA's halves of the K/V tiles,
-//              into an 8-slot ring of 16 KB, bytes counted on CTA 0's
-//              barriers; lane 1: TMA producer of the query tile;
-//   warp 5     tensor-memory allocation (both CTAs); in CTA 0 the warp runs
+// Roles in each CTA (320 threads):
+//   warps 0-7  two softmax warpgroups.  Both own the tile's 128 query rows
+//              (warp w reads TMEM lanes 32 (w % 4) ..); warpgroup g takes
+//              keys [64 g, 64 g + 64) of every key tile.  A row's maximum
+//              over the tile is exchanged between the two warps of a lane
+//              quarter through shared memory, so both decide the same
+//              softmax base.  At the end of an item the two warpgroups split
+//              the epilogue (1/l, sigmoid gate, bf16, half of the 256 output
+//              dims each) and, on full layers given raw queries, the
+//              rotation of the next item's query tile (rotate-half RoPE over
+//              the first 64 dims, half of the 32 frequencies each).  Sliding
+//              layers rotate all 256 dims of every query, which on the item
+//              boundary cost more than the separate pass over the queries
+//              the host runs first: their queries always arrive rotated;
+//   warp 8     lane 0: TMA producer for this CTA's halves of the K/V tiles,
+//              into a 4-slot ring of 32 KB, bytes counted on CTA 0's
+//              barriers; lane 1: TMA producer of the query tile (with an L2
+//              prefetch of the next item's);
+//   warp 9     tensor-memory allocation (both CTAs); in CTA 0 the warp runs
 //              the MMA loop convergently and one elected lane issues every
 //              MMA of the pair and commits to both CTAs.
-// S = Q K^T reads both operands from shared memory: with N = 64 an MMA whose
-// A operand sits in tensor memory ran at ~40 % of the tensor rate on B200,
-// one reading A from shared memory at ~90 %.
 // Tensor memory, per CTA (512 columns x 128 lanes of 32 bit):
-//   [0,256)   kNS S buffers (fp32, 64 keys each); P of a tile (bf16 pairs)
-//             overwrites the first 32 columns of its S buffer and is the A
-//             operand of O += P V
+//   [0,256)   two S buffers (fp32, 128 keys each); P of a tile (bf16 pairs)
+//             overwrites the first 32 columns of each warpgroup's 64 and is
+//             the A operand of O += P V
 //   [256,512) O accumulator, fp32 128 x 256.
-// The pair's MMAs run kNS - 1 key tiles ahead of the softmax (S of tile
-// j + kNS - 1 is issued before P.V of tile j), so the time the softmax of a
-// tile takes to hand P over is hidden behind tensor-core work.
-// Softmax in the log2 domain with a lazily updated row maximum: the running
-// maximum only moves (and O is only rescaled) when a tile's maximum exceeds
-// it by more than 8, so P stays <= 256.
+// The pair's MMAs run one key tile ahead of the softmax (S of tile j + 1 is
+// issued before P.V of tile j).
+//
+// Softmax in the log2 domain with a lazily updated base: every probability
+// of a row is 2^(s - base), the base only moves (and O is only rescaled)
+// when a tile's maximum exceeds it by more than 8, so P stays <= 256.
+#include <algorithm>
+
 #include "common.cuh"
 #include "launch.h"
 
 namespace hyb {
 
 constexpr int kBM = 128;                  // query rows per CTA
-constexpr int kBN = 64;                   // keys per tile (shared by the pair)
-constexpr int kSlots = 8;                 // K/V ring
-constexpr int kSlotBytes = 16384;         // one CTA's half of a K or V tile
-constexpr int kKBoxRows = kBN / 2;        // K half: 32 keys x 64 dims per box
-constexpr int kKBox = kKBoxRows * 128;    // 4 KB
-constexpr int kVBox = kBN * 128;          // V half: 64 keys x 64 dims per box, 8 KB
-constexpr int kPfThreads = 192;
-constexpr int kNS = 4;                    // S buffers in tensor memory
+constexpr int kBN = 128;                  // keys per tile (shared by the pair)
+constexpr int kHalfKeys = 64;             // keys per TMA box row range (a K half, a V quarter)
+constexpr int kSlots = 4;                 // K/V ring
+constexpr int kSlotBytes = 32768;         // one CTA's half of a K or V tile
+constexpr int kKBox = kHalfKeys * 128;    // K half: 64 keys x 64 dims per box, 8 KB
+constexpr int kVChunk = kBN * 128;        // V: 128 keys x 64 dims (two 64-key boxes), 16 KB
+constexpr int kPfThreads = 320;
+constexpr int kSmWarps = 8;               // softmax warps (two warpgroups)
+constexpr int kProdWarp = 8;
+constexpr int kMmaWarp = 9;
+constexpr int kNS = 2;                    // S buffers in tensor memory
 constexpr int kAhead = kNS - 1;           // key tiles whose S is issued before the P.V of a tile
 constexpr uint32_t kColO = 256;
 constexpr float kRescaleThreshold = 8.0f;
-__device__ __forceinline__ uint32_t col_s(uint32_t sb) { return 64u * sb; }
+constexpr int kStageBytes = 2048;         // epilogue transpose area per softmax warp
+__device__ __forceinline__ uint32_t col_s(uint32_t sb) { return 128u * sb; }
 
+template <bool FULL>
 struct PfSmem {
+  static constexpr int R = RopeCfg<FULL>::R;
   uint8_t slot[kSlots][kSlotBytes];  // 1024-byte aligned
-  uint8_t qo[4][kSlotBytes];         // the query tile in (4 boxes of 64 dims x 128 rows, rotated in place:
-                                     // the A operand of S = Q K^T), the output tile out
-  double inv_freq[128];
-  // rotation tables for the tile's rows (positions p_base + 16 i + j):
+  uint8_t qo[4][16384];              // the query tile (4 boxes of 64 dims x 128 rows), rotated in place:
+                                     // the A operand of S = Q K^T
+  // full layers: rotation tables for the tile's rows (positions p_base + 16 i + j), rebuilt per item:
   //   rot_lo[k / 2][j] = (cos, sin)(j * inv_freq_k), k even then odd,             j < 16
   //   rot_hi[i][k / 2] = (cos, sin)((p_base + 16 i) * inv_freq_k), k even then odd,  i < 8
-  // (two frequencies per 16-byte entry: one shared-memory load per pair of them)
-  float4 rot_lo[64][16];
-  float4 rot_hi[8][64];
-  uint8_t ostage[4][2048];           // per softmax warp: 32 rows x 32 output dims (bf16), transposed on the way out
+  // (two frequencies per 16-byte entry); warpgroup g owns the entries of its
+  // half of the frequencies
+  float4 rot_lo[FULL ? R / 4 : 1][16];
+  float4 rot_hi[8][FULL ? R / 4 : 1];
+  uint8_t ostage[kSmWarps][kStageBytes];   // epilogue transpose area per softmax warp
+  double inv_freq[R / 2];
+  float xmax[2][2][kBM];             // [tile parity][warpgroup][row]: a row's maximum over the warpgroup's keys
+  float xsum[2][2][kBM];             // [item parity][warpgroup][row]: running sum at item end
   uint64_t full[kSlots];   // CTA 0's count both CTAs' bytes
   uint64_t empty[kSlots];  // per CTA, committed by the MMA issuer
-  uint64_t q_ready;        // CTA 0: one arrival per softmax warp of the pair
+  uint64_t q_ready;        // CTA 0: query tile rotated (one arrival per softmax warp of the pair) or
+                           //   landed (one arrival per CTA from its query producer)
   uint64_t s_full[kNS];
   uint64_t p_full[kNS];    // CTA 0: one arrival per softmax warp of the pair
-  uint64_t o_done[kNS];    // P.V of a tile in S buffer i completed (two P.Vs may be in flight)
-  uint64_t o_final;        // the last P.V completed
+  uint64_t o_done[kNS];    // P.V of a tile in S buffer i completed
+  uint64_t o_final;        // the item's last P.V completed
+  uint64_t o_free;         // CTA 0: every softmax warp of the pair has read O out (epilogue done)
   uint64_t mma_done;       // every MMA of the pair completed
   uint64_t q_full;         // this CTA's query tile landed in qo
   uint64_t q_free;         // qo is free again (the item's last S = Q K^T completed)
-  uint64_t sync_sm;        // the 128 softmax threads (bounded waits, unlike bar.sync)
+  uint64_t xmax_full[2][4];  // xmax[parity] of lane quarter q written by both of its warps
+  uint64_t xsum_full;      // both warpgroups' xsum written (one arrival per softmax warp)
+  uint64_t sync_wg[2];     // the 128 threads of a warpgroup (bounded waits, unlike bar.sync)
   uint32_t tmem_base;
 };
 
-size_t prefill_smem_bytes() { return sizeof(PfSmem) + 1024; }
-static_assert(sizeof(PfSmem) + 1024 <= 232448, "prefill shared memory exceeds 227 KB");
+template <bool FULL>
+size_t prefill_smem_bytes_t() { return sizeof(PfSmem<FULL>) + 1024; }
+size_t prefill_smem_bytes() { return std::max(prefill_smem_bytes_t<true>(), prefill_smem_bytes_t<false>()); }
+static_assert(sizeof(PfSmem<true>) + 1024 <= 232448 && sizeof(PfSmem<false>) + 1024 <= 232448,
+              "prefill shared memory exceeds 227 KB");
 
 struct PfArgs {
   const __nv_bfloat16* q;
@@ -95,47 +123,80 @@ struct PfArgs {
   __nv_bfloat16* out;
   const int32_t* qbase;
   int ctx_mode;
-  int q_rotated;   // the queries arrive rotated (by the projection's epilogue)
+  int q_rotated;   // the queries arrive rotated (by the projection's epilogue or a rotation pass)
   int B, T, n_mtiles;
   PageMap pm;      // K/V maps over a paged cache's pool
 };
 
+// ---------------------------------------------------------------------------
+// Packed fp32 pairs (sm_100 f32x2 instructions): one issue slot for two lanes
+// of arithmetic.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float2 ffma2(float2 a, float2 b, float2 c) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rc, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\tmov.b64 rc, {%6, %7};\n\t"
+      "fma.rn.f32x2 rd, ra, rb, rc;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y), "f"(c.x), "f"(c.y));
+  return d;
+}
+__device__ __forceinline__ float2 fadd2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+__device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "mul.rn.f32x2 rd, ra, rb;\n\tmov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+
 // Load order shared by the K/V producer and the MMA issuer: step s (0 <= s
 // < n + kAhead) loads K_s if s < n, then V_{s - kAhead} if 0 <= s - kAhead < n.
 
-// Rotates 32 dims [k0, k0+32) against their partners [k0+R/2, ...) for one
-// query row: x1 / x2 hold 16 packed bf16 words each; results replace them.
-// Pair k turns by p * inv_freq_k.  Table form, for a row at p_base + 16 i + j
-// (the rows of a tile are consecutive positions): the turn is the product of
-// two precomputed unit complex numbers (rot_hi for i, rot_lo for j).
-// General form (any other position): the fp64-reduced full angle.
-__device__ __forceinline__ void rotate32_table(uint32_t (&x1)[16], uint32_t (&x2)[16], int k0, int i_hi,
-                                               int j_lo, const float4 (*rot_lo)[16], const float4 (*rot_hi)[64]) {
+// Rotates 2 NW dims [k0, k0 + 2 NW) against their partners [k0 + R/2, ...)
+// for one query row: x1 / x2 hold NW packed bf16 words each; results replace
+// them.  Pair k turns by p * inv_freq_k.  Table form, for a row at p_base +
+// 16 i + j (the rows of a tile are consecutive positions): the turn is the
+// product of two precomputed unit complex numbers (rot_hi for i, rot_lo for
+// j).  General form (any other position): the fp64-reduced full angle.
+template <int NW, int NKP>
+__device__ __forceinline__ void rotate_table(uint32_t (&x1)[NW], uint32_t (&x2)[NW], int k0, int i_hi, int j_lo,
+                                             const float4 (*rot_lo)[16], const float4 (*rot_hi)[NKP]) {
 #pragma unroll
-  for (int w = 0; w < 16; ++w) {
+  for (int w = 0; w < NW; ++w) {
     const int kp = k0 / 2 + w;   // frequencies 2 kp and 2 kp + 1
     const float4 u4 = rot_hi[i_hi][kp];
     const float4 v4 = rot_lo[kp][j_lo];
-    float a[2], bb[2];
-#pragma unroll
-    for (int e = 0; e < 2; ++e) {
-      const float x = e ? bf16hi(x1[w]) : bf16lo(x1[w]);
-      const float y = e ? bf16hi(x2[w]) : bf16lo(x2[w]);
-      const float2 u = e ? make_float2(u4.z, u4.w) : make_float2(u4.x, u4.y);
-      const float2 v = e ? make_float2(v4.z, v4.w) : make_float2(v4.x, v4.y);
-      const float c = fmaf(u.x, v.x, -u.y * v.y);
-      const float s = fmaf(u.y, v.x, u.x * v.y);
-      a[e] = fmaf(x, c, -y * s);
-      bb[e] = fmaf(y, c, x * s);
-    }
-    x1[w] = pack_bf16(a[0], a[1]);
-    x2[w] = pack_bf16(bb[0], bb[1]);
+    // (c, s) of both frequencies as products of the two unit complex numbers
+    const float2 ux = make_float2(u4.x, u4.z), uy = make_float2(u4.y, u4.w);
+    const float2 vx = make_float2(v4.x, v4.z), vy = make_float2(v4.y, v4.w);
+    const float2 uyvy = fmul2(uy, vy), uxvy = fmul2(ux, vy);
+    const float2 c = ffma2(ux, vx, make_float2(-uyvy.x, -uyvy.y));
+    const float2 s = ffma2(uy, vx, uxvy);
+    const float2 x = make_float2(bf16lo(x1[w]), bf16hi(x1[w]));
+    const float2 y = make_float2(bf16lo(x2[w]), bf16hi(x2[w]));
+    const float2 ys = fmul2(y, s), xs = fmul2(x, s);
+    const float2 a = ffma2(x, c, make_float2(-ys.x, -ys.y));
+    const float2 bb = ffma2(y, c, xs);
+    x1[w] = pack_bf16(a.x, a.y);
+    x2[w] = pack_bf16(bb.x, bb.y);
   }
 }
-__device__ __noinline__ void rotate32_general(uint32_t (&x1)[16], uint32_t (&x2)[16], int k0, int p,
-                                              const double* inv_freq) {
+template <int NW>
+__device__ __noinline__ void rotate_general(uint32_t (&x1)[NW], uint32_t (&x2)[NW], int k0, int p,
+                                            const double* inv_freq) {
 #pragma unroll 4
-  for (int w = 0; w < 16; ++w) {
+  for (int w = 0; w < NW; ++w) {
     float a[2], bb[2];
 #pragma unroll
     for (int e = 0; e < 2; ++e) {
@@ -149,14 +210,6 @@ __device__ __noinline__ void rotate32_general(uint32_t (&x1)[16], uint32_t (&x2)
     x1[w] = pack_bf16(a[0], a[1]);
     x2[w] = pack_bf16(bb[0], bb[1]);
   }
-}
-// in_table: warp-uniform (every row of the warp at p_base + [0, 128))
-__device__ __forceinline__ void rotate32(uint32_t (&x1)[16], uint32_t (&x2)[16], int k0, int p, int delta,
-                                         bool in_table, const PfSmem& sm) {
-  if (in_table)
-    rotate32_table(x1, x2, k0, delta >> 4, delta & 15, sm.rot_lo, sm.rot_hi);
-  else
-    rotate32_general(x1, x2, k0, p, sm.inv_freq);
 }
 
 // One work item: a 128-query tile of the two query heads (2 hp + {0, 1}) of KV
@@ -201,14 +254,18 @@ __device__ __forceinline__ int item_index(int k, int pair, int n_pairs, int n_it
 
 // Persistent: each CTA pair walks its items round by round.
 // Barrier phases run on across items: K/V loads by a global load counter,
-// S / P buffers by a global tile counter, query / output / last-P.V barriers
-// by the item counter.
+// S / P buffers and the maximum exchange by a global tile counter, query /
+// output / sum-exchange barriers by the item counter.
 template <bool FULL>
+// Warps are dealt round-robin to the SM's four sub-partitions (16,384
+// registers each): with 10 warps two sub-partitions hold three, so a thread
+// may use at most 168 registers.
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, PfArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  PfSmem& sm = *reinterpret_cast<PfSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  using Smem = PfSmem<FULL>;
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int R = RopeCfg<FULL>::R;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const uint32_t rank = cluster_ctarank();   // 0 = the CTA that issues the pair's MMAs
@@ -221,38 +278,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
-    mbar_init(&sm.q_ready, 8);
+    mbar_init(&sm.q_ready, a.q_rotated ? 2 : 2 * kSmWarps);
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&sm.s_full[s], 1);
-      mbar_init(&sm.p_full[s], 8);
+      mbar_init(&sm.p_full[s], 2 * kSmWarps);
+      mbar_init(&sm.o_done[s], 1);
     }
-    for (int s = 0; s < kNS; ++s) mbar_init(&sm.o_done[s], 1);
     mbar_init(&sm.o_final, 1);
+    mbar_init(&sm.o_free, 2 * kSmWarps);
     mbar_init(&sm.mma_done, 1);
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_free, 1);
-    mbar_init(&sm.sync_sm, kBM);
+    for (int p = 0; p < 2; ++p)
+      for (int q = 0; q < 4; ++q) mbar_init(&sm.xmax_full[p][q], 2);
+    mbar_init(&sm.xsum_full, kSmWarps);
+    mbar_init(&sm.sync_wg[0], 128);
+    mbar_init(&sm.sync_wg[1], 128);
     fence_barrier_init();
   }
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
   }
-  // frequencies and the position-independent rotation table
   if (threadIdx.x < R / 2) sm.inv_freq[threadIdx.x] = rope_inv_freq(RopeCfg<FULL>::theta, threadIdx.x, R);
-  __syncthreads();
-  for (int t = threadIdx.x; t < (R / 2) * 16; t += kPfThreads) {
-    const int k = t % (R / 2), e = t / (R / 2);
-    float sn, cs;
-    small_angle_sincos(e, (float)sm.inv_freq[k], &sn, &cs);
-    reinterpret_cast<float2*>(&sm.rot_lo[k >> 1][e])[k & 1] = make_float2(cs, sn);
-  }
   tc_fence_before();
   cluster_sync();   // barriers of both CTAs initialised before any cross-CTA arrive
   tc_fence_after();
   const uint32_t tmem = sm.tmem_base;
 
-  if (warp == 4) {
+  if (warp == kProdWarp) {
     if (lane == 0) {
       // ======================= K/V producer (both CTAs) =======================
       prefetch_tmap(&tm_k);
@@ -264,6 +318,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         if (w == -2) break;
         if (w < 0) continue;
         const Item it = item_of<FULL>(w, a);
+        const int last_row = it.q_hi - it.kb;   // key row of the item's last visible key
+        // (row, page) coordinates of the 64 keys from key row r on; a range past the
+        // item's last key is read from an out-of-range page (zeros) instead of
+        // touching a block-table entry the sequence may not have
+        auto coord = [&](int r, int& row, int& page) {
+          if (r > last_row) {
+            row = 0;
+            page = -1;
+          } else {
+            kv_coord(a.pm, it.b, r, row, page);
+          }
+        };
         for (int st = 0; ok && st < it.n + kAhead; ++st) {
 #pragma unroll 1
           for (int part = 0; part < 2; ++part) {
@@ -274,18 +340,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             if (g >= kSlots && !(ok = mbar_wait(&sm.empty[slot], ((g / kSlots) - 1) & 1))) break;
             if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
             const uint32_t dst = smem_u32(sm.slot[slot]);
-            int row, cpage;   // the tile's 64 keys lie within one page
-            kv_coord(a.pm, it.b, (it.j_lo + tile) * kBN, row, cpage);
-            if (is_k) {
+            const int r0 = (it.j_lo + tile) * kBN;   // key row of the tile's first key
+            int row, page;
+            if (is_k) {   // this CTA's 64 keys, 4 boxes of 64 dims
+              coord(r0 + kHalfKeys * (int)rank, row, page);
 #pragma unroll
               for (int box = 0; box < 4; ++box)
-                tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row + kKBoxRows * (int)rank,
-                                 it.kvh, cpage);
-            } else {
+                tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row, it.kvh, page);
+            } else {      // all 128 keys of this CTA's 128 dims: 2 dim chunks x 2 key halves
 #pragma unroll
-              for (int box = 0; box < 2; ++box)
-                tma_load_4d_pair(dst + box * kVBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * box, row, it.kvh,
-                                 cpage);
+              for (int h = 0; h < 2; ++h) {
+                coord(r0 + kHalfKeys * h, row, page);
+#pragma unroll
+                for (int d = 0; d < 2; ++d)
+                  tma_load_4d_pair(dst + d * kVChunk + h * kKBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * d,
+                                   row, it.kvh, page);
+              }
             }
             ++g;
           }
@@ -297,28 +367,43 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       // ======================= query-tile producer (both CTAs) =======================
       prefetch_tmap(&tm_q);
       int item = 0;
-      for (int k = 0;; ++k) {
-        const int w = item_index(k, pair0, n_pairs, n_items);
+      bool ok = true;
+      for (int k = 0; ok;) {
+        int w = item_index(k, pair0, n_pairs, n_items);
+        while (w == -1) w = item_index(++k, pair0, n_pairs, n_items);
         if (w == -2) break;
-        if (w < 0) continue;
         const Item it = item_of<FULL>(w, a);
-        if (item > 0 && !mbar_wait(&sm.q_free, (item - 1) & 1)) break;
-        mbar_arrive_expect_tx(&sm.q_full, 4 * kSlotBytes);
+        if (item > 0 && !(ok = mbar_wait(&sm.q_free, (item - 1) & 1))) break;
+        mbar_arrive_expect_tx(&sm.q_full, 4 * 16384);
 #pragma unroll
         for (int box = 0; box < 4; ++box)
           tma_load_4d(smem_u32(sm.qo[box]), &tm_q, &sm.q_full, box * 64, it.h_pair0 + (int)rank, it.m0, it.b);
+        // the next item's query tile into L2 while this one is in use
+        int k2 = k + 1, w2 = item_index(k2, pair0, n_pairs, n_items);
+        while (w2 == -1) w2 = item_index(++k2, pair0, n_pairs, n_items);
+        if (w2 >= 0) {
+          const Item nx = item_of<FULL>(w2, a);
+#pragma unroll
+          for (int box = 0; box < 4; ++box) tma_prefetch_l2_4d(&tm_q, box * 64, nx.h_pair0 + (int)rank, nx.m0, nx.b);
+        }
+        if (a.q_rotated) {   // nothing to rotate: the tile is ready once it has landed
+          if (!(ok = mbar_wait(&sm.q_full, item & 1))) break;
+          if (rank == 0) mbar_arrive(&sm.q_ready);
+          else mbar_arrive_remote(&sm.q_ready, 0);
+        }
         ++item;
+        k = k2;
       }
       if (item > 0) mbar_wait(&sm.q_full, (item - 1) & 1);   // no copy left landing at exit
     }
-  } else if (warp == 5) {
+  } else if (warp == kMmaWarp) {
     // ======================= MMA issuer (CTA 0, whole warp, one lane issues) =======================
     if (rank == 0) {
       constexpr uint32_t idesc_s = idesc_bf16(2 * kBM, kBN, false);   // S = Q K^T, B K-major
       constexpr uint32_t idesc_o = idesc_bf16(2 * kBM, kD, true);     // O += P V, B MN-major
-      const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.qo[0]), 16, 1024);         // Q, K-major
-      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(sm.slot[0]), 16, 1024);      // K in slot 0, K-major
-      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(sm.slot[0]), kVBox, 1024);   // V in slot 0, MN-major
+      const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.qo[0]), 16, 1024);          // Q, K-major
+      const uint64_t kdesc0 = smem_desc_sw128(smem_u32(sm.slot[0]), 16, 1024);       // K in slot 0, K-major
+      const uint64_t vdesc0 = smem_desc_sw128(smem_u32(sm.slot[0]), kVChunk, 1024);  // V in slot 0, MN-major
       uint32_t g = 0, J = 0;
       int item = 0;
       bool ok = true;
@@ -344,7 +429,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
               const uint64_t kdesc = desc_advance(kdesc0, slot * kSlotBytes);
 #pragma unroll
               for (int s = 0; s < kD / 16; ++s) {
-                const uint64_t adesc = desc_advance(qdesc, (s >> 2) * kSlotBytes + (s & 3) * 32);
+                const uint64_t adesc = desc_advance(qdesc, (s >> 2) * 16384 + (s & 3) * 32);
                 const uint64_t bdesc = desc_advance(kdesc, (s >> 2) * kKBox + (s & 3) * 32);
                 mma_ss_pair_warp(tmem + col_s(sb), adesc, bdesc, idesc_s, s > 0 ? 1u : 0u);
               }
@@ -352,13 +437,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
               mma_commit_pair_warp(&sm.s_full[sb]);
               if (tile == it.n - 1) mma_commit_pair_warp(&sm.q_free);   // qo is no longer read
             } else {
+              // the item's first P.V overwrites O: the previous item's epilogue must have read it
+              if (tile == 0 && item > 0 &&
+                  !(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_free, (item - 1) & 1))))
+                break;
               if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[sb], (jt / kNS) & 1)))) break;
               tc_fence_after();
               const uint64_t vdesc = desc_advance(vdesc0, slot * kSlotBytes);
 #pragma unroll
               for (int s = 0; s < kBN / 16; ++s) {
+                // keys [16 s, 16 s + 16): P of warpgroup s / 4 at its columns 64 (s / 4) + 8 (s % 4)
                 const uint64_t bdesc = desc_advance(vdesc, s * 16 * 128);
-                mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 8 * s, bdesc, idesc_o,
+                mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 64 * (s >> 2) + 8 * (s & 3), bdesc, idesc_o,
                                  (tile > 0 || s > 0) ? 1u : 0u);
               }
               mma_commit_pair_warp(&sm.empty[slot]);
@@ -376,23 +466,33 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       mbar_wait(&sm.mma_done, 0);
     }
   } else {
-    // ======================= softmax / epilogue (warps 0-3) =======================
-    // Per item: the online softmax over its key tiles; then the next item's
-    // query tile is rotated (so the pair's MMAs for it can start), and only
-    // then this item's output leaves, straight from TMEM to global memory.
-    const int r = threadIdx.x;          // query row in the tile = TMEM lane
-    const uint32_t trow = tmem + ((uint32_t)(warp * 32) << 16);
+    // ======================= softmax / epilogue (warps 0-7) =======================
+    const int wg = warp >> 2;            // warpgroup: keys [64 wg, 64 wg + 64) of each tile
+    const int qtr = warp & 3;            // lane quarter of tensor memory
+    const int r = qtr * 32 + lane;       // query row in the tile = TMEM lane
+    const uint32_t trow = tmem + ((uint32_t)(qtr * 32) << 16);
     const float scale_log2 = 0.0625f * 1.4426950408889634f;
-    // barrier among the softmax threads; each thread counts the phases it has
-    // passed (none can get two phases ahead: every phase needs all arrivals)
+    const float2 scale2 = make_float2(scale_log2, scale_log2);
+    // barrier among the 128 threads of this warpgroup; each thread counts the
+    // phases it has passed (none can get two phases ahead: every phase needs
+    // all arrivals)
     uint32_t n_sync = 0;
-    auto sync_softmax = [&]() -> bool {
-      mbar_arrive(&sm.sync_sm);
-      return mbar_wait(&sm.sync_sm, (n_sync++) & 1);
+    auto sync_wg = [&]() -> bool {
+      mbar_arrive(&sm.sync_wg[wg]);
+      return mbar_wait(&sm.sync_wg[wg], (n_sync++) & 1);
     };
-    // rotates the query tile of `it` (the item_no-th of this pair) in qo and
-    // hands it to the MMA issuer
+    auto arrive_cta0 = [&](uint64_t* bar) {   // lane 0, after __syncwarp: one arrival for the warp
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(bar);
+        else mbar_arrive_remote(bar, 0);
+      }
+    };
+    // Rotates this warpgroup's half of the frequencies of the query tile of
+    // `it` (the item_no-th of this pair) in qo and hands it to the MMA issuer.
     auto prepare_q = [&](const Item& it, int item_no) -> bool {
+     if constexpr (!FULL) {
+      return false;   // sliding layers: queries always arrive rotated
+     } else {
       const int row = it.m0 + r;
       const bool valid = row < a.T;
       const int qseq = it.qb + row;
@@ -400,66 +500,69 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       const int p = a.pos ? (valid ? a.pos[(int64_t)it.b * a.T + row] : 0) : qseq;
       const int delta = p - p_base;
       const bool in_table = __all_sync(0xffffffffu, delta >= 0 && delta < kBM);
-
-      // ---- rotation table for this tile's base position ----
-      if (!a.q_rotated) {
-        for (int t = r; t < (R / 2) * 8; t += kBM) {
-          const int k = t % (R / 2), e = t / (R / 2);
-          float sn, cs;
-          rope_sincos(p_base + 16 * e, sm.inv_freq[k], &sn, &cs);
-          reinterpret_cast<float2*>(&sm.rot_hi[e][k >> 1])[k & 1] = make_float2(cs, sn);
-        }
-        if (!__all_sync(0xffffffffu, sync_softmax())) return false;
+      constexpr int NF = R / 4;          // frequencies of this warpgroup
+      const int f0 = wg * NF;
+      // ---- rotation tables of this tile's base position (this warpgroup's frequencies) ----
+      if (!__all_sync(0xffffffffu, sync_wg())) return false;   // the area is no longer read or staged in
+      for (int t = r; t < NF * 8; t += kBM) {
+        const int kf = f0 + t % NF, e = t / NF;
+        float sn, cs;
+        rope_sincos(p_base + 16 * e, sm.inv_freq[kf], &sn, &cs);
+        reinterpret_cast<float2*>(&sm.rot_hi[e][kf >> 1])[kf & 1] = make_float2(cs, sn);
       }
-
-      // ---- this row of the query tile: shared memory (128-byte swizzled boxes) -> registers ----
-      uint4 qv[kD / 8];
+      for (int t = r; t < NF * 16; t += kBM) {
+        const int kf = f0 + t % NF, e = t / NF;
+        float sn, cs;
+        small_angle_sincos(e, (float)sm.inv_freq[kf], &sn, &cs);
+        reinterpret_cast<float2*>(&sm.rot_lo[kf >> 1][e])[kf & 1] = make_float2(cs, sn);
+      }
+      if (!__all_sync(0xffffffffu, sync_wg())) return false;
       if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full, item_no & 1))) return false;
+      // ---- rotate dims [f0, f0 + NF) against [f0 + R/2, ...) in place ----
+      constexpr int NW = 8;   // packed words (16 dims of each half) per pass
 #pragma unroll
-      for (int i = 0; i < kD / 8; ++i) {
-        const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(i & 7) * 16);
-        qv[i] = *reinterpret_cast<const uint4*>(sm.qo[i >> 3] + off);
+      for (int c = 0; c < NF / (2 * NW); ++c) {
+        const int k0 = f0 + 2 * NW * c;
+        uint32_t x1[NW], x2[NW];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int dim0 = k0 + h * (R / 2);
+#pragma unroll
+          for (int i = 0; i < NW / 4; ++i) {
+            const int ci = dim0 / 8 + i;
+            const uint4 v = *reinterpret_cast<const uint4*>(sm.qo[ci >> 3] + sw128_offset((uint32_t)r, (uint32_t)(ci & 7) * 16));
+            uint32_t* xw = h ? x2 : x1;
+            xw[4 * i] = v.x;
+            xw[4 * i + 1] = v.y;
+            xw[4 * i + 2] = v.z;
+            xw[4 * i + 3] = v.w;
+          }
+        }
+        if (in_table)
+          rotate_table<NW, R / 4>(x1, x2, k0, delta >> 4, delta & 15, sm.rot_lo, sm.rot_hi);
+        else
+          rotate_general<NW>(x1, x2, k0, p, sm.inv_freq);
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int dim0 = k0 + h * (R / 2);
+          const uint32_t* xw = h ? x2 : x1;
+#pragma unroll
+          for (int i = 0; i < NW / 4; ++i) {
+            const int ci = dim0 / 8 + i;
+            *reinterpret_cast<uint4*>(sm.qo[ci >> 3] + sw128_offset((uint32_t)r, (uint32_t)(ci & 7) * 16)) =
+                make_uint4(xw[4 * i], xw[4 * i + 1], xw[4 * i + 2], xw[4 * i + 3]);
+          }
+        }
       }
-      // ---- rotate it in place (rotated dims go back to where they were read) ----
-      auto words16 = [&](int dim0, uint32_t (&wd)[16]) {   // 16 packed words = dims [dim0, dim0 + 32)
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const uint4 v = qv[dim0 / 8 + i];
-          wd[4 * i + 0] = v.x;
-          wd[4 * i + 1] = v.y;
-          wd[4 * i + 2] = v.z;
-          wd[4 * i + 3] = v.w;
-        }
-      };
-      auto store16 = [&](int dim0, const uint32_t (&wd)[16]) {   // inverse of words16, into qo
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int ci = dim0 / 8 + i;
-          const uint32_t off = sw128_offset((uint32_t)r, (uint32_t)(ci & 7) * 16);
-          *reinterpret_cast<uint4*>(sm.qo[ci >> 3] + off) = make_uint4(wd[4 * i], wd[4 * i + 1], wd[4 * i + 2], wd[4 * i + 3]);
-        }
-      };
-      if (!a.q_rotated) {
-#pragma unroll
-        for (int c = 0; c < R / 64; ++c) {   // dims [R, 256) are not rotated and stay as loaded
-          uint32_t x1[16], x2[16];
-          words16(32 * c, x1);
-          words16(R / 2 + 32 * c, x2);
-          rotate32(x1, x2, 32 * c, p, delta, in_table, sm);
-          store16(32 * c, x1);
-          store16(R / 2 + 32 * c, x2);
-        }
-        fence_proxy_async();              // qo is read by the tensor core
-        if (rank != 0) fence_cluster();   // ... through MMAs issued from CTA 0
-      }
+      fence_proxy_async();              // qo is read by the tensor core
+      if (rank != 0) fence_cluster();   // ... through MMAs issued from CTA 0
       tc_fence_before();                // TMEM accesses so far precede the MMAs q_ready releases
       __syncwarp();
-      if (lane == 0) {
-        if (rank == 0) mbar_arrive(&sm.q_ready);
-        else mbar_arrive_remote(&sm.q_ready, 0);
-      }
+      arrive_cta0(&sm.q_ready);
       return true;
+     }
     };
+
     auto next_item = [&](int& k, Item& it) -> bool {
       for (;; ++k) {
         const int w = item_index(k, pair0, n_pairs, n_items);
@@ -476,30 +579,31 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     int k = 0, item = 0;
     Item it;
     bool have = next_item(k, it);
-    bool ok = !have || prepare_q(it, 0);
+    bool ok = !have || a.q_rotated || prepare_q(it, 0);
     while (ok && have) {
       const int h = it.h_pair0 + (int)rank;
       const int row = it.m0 + r;
       const bool valid = row < a.T;
       const int qseq = it.qb + row;
 
-      // ---- online softmax over the key tiles ----
-      float m_run = -INFINITY, l_run = 0.f;
+      // ---- online softmax over this warpgroup's keys of each tile ----
+      float l_run = 0.f, b_run = -INFINITY;   // running sum (this warpgroup's keys) and the row's base
       for (int j = 0; ok && j < it.n; ++j) {
         const uint32_t jt = J + j;
         const uint32_t sb = jt % kNS;
+        const uint32_t scol = col_s(sb) + 64 * wg;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.s_full[sb], (jt / kNS) & 1)))) break;
         tc_fence_after();
         uint32_t sraw[64];
-        tmem_ld32(trow + col_s(sb), *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
-        tmem_ld32(trow + col_s(sb) + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
+        tmem_ld32(trow + scol, *reinterpret_cast<uint32_t(*)[32]>(&sraw[0]));
+        tmem_ld32(trow + scol + 32, *reinterpret_cast<uint32_t(*)[32]>(&sraw[32]));
         tmem_wait_ld();
         float s[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sraw[c]);
 
-        const int ks0 = it.kb + (it.j_lo + j) * kBN;   // sequence index of the tile's first key
-        const bool whole = ks0 >= 0 && ks0 + kBN - 1 <= it.q_lo && (FULL || it.q_hi - ks0 <= kWindow - 1);
+        const int ks0 = it.kb + (it.j_lo + j) * kBN + 64 * wg;   // sequence index of this warpgroup's first key
+        const bool whole = ks0 >= 0 && ks0 + 63 <= it.q_lo && (FULL || it.q_hi - ks0 <= kWindow - 1);
         if (!whole) {
 #pragma unroll
           for (int c = 0; c < 64; ++c) {
@@ -508,7 +612,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             if (!vis) s[c] = -INFINITY;
           }
         }
-        // row maximum: pairwise tree (short dependency chains)
+        // row maximum over this warpgroup's keys: pairwise tree (short dependency chains)
         float mx[32];
 #pragma unroll
         for (int c = 0; c < 32; ++c) mx[c] = fmaxf(s[c], s[c + 32]);
@@ -516,83 +620,101 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         for (int wd = 16; wd >= 1; wd >>= 1)
 #pragma unroll
           for (int c = 0; c < wd; ++c) mx[c] = fmaxf(mx[c], mx[c + wd]);
-        const float m_row = mx[0];
-        const float m_tile = m_row * scale_log2;
-        const float m_new = fmaxf(m_run, m_tile);
-        const bool rescale = m_new > m_run + kRescaleThreshold;
-        const float m_use = rescale ? m_new : m_run;
-        const float base = (m_use == -INFINITY) ? 0.f : m_use;
-        const float alpha = rescale ? ex2(m_run - m_use) : 1.f;
+        // ---- the maximum over the whole tile, through the partner warp ----
+        sm.xmax[jt & 1][wg][r] = mx[0];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.xmax_full[jt & 1][qtr]);
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.xmax_full[jt & 1][qtr], (jt >> 1) & 1)))) break;
+        const float m_tile = fmaxf(mx[0], sm.xmax[jt & 1][wg ^ 1][r]) * scale_log2;
+        const bool rescale = m_tile > b_run + kRescaleThreshold;
+        const float b_new = rescale ? m_tile : b_run;
+        const float alpha = rescale ? ex2(b_run - b_new) : 1.f;   // b_run = -inf: O and l are 0
+
+        const float base = (b_new == -INFINITY) ? 0.f : b_new;
+        const float2 nbase2 = make_float2(-base, -base);
         uint32_t pw[32];
-        float ps[8];
-#pragma unroll
-        for (int c = 0; c < 8; ++c) ps[c] = 0.f;
+        float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
 #pragma unroll
         for (int wd = 0; wd < 32; ++wd) {
-          const float p0 = ex2(fmaf(s[2 * wd], scale_log2, -base));
-          const float p1 = ex2(fmaf(s[2 * wd + 1], scale_log2, -base));
-          ps[wd & 7] += p0 + p1;
-          pw[wd] = pack_bf16(p0, p1);
+          const float2 x = ffma2(make_float2(s[2 * wd], s[2 * wd + 1]), scale2, nbase2);
+          const float2 e = make_float2(ex2(x.x), ex2(x.y));
+          ps[wd & 3] = fadd2(ps[wd & 3], e);
+          pw[wd] = pack_bf16(e.x, e.y);
         }
-        const float sum = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-        l_run = l_run * alpha + sum;
-        m_run = m_use;
-        tmem_st32(trow + col_s(sb), pw);
+        const float2 s01 = fadd2(fadd2(ps[0], ps[1]), fadd2(ps[2], ps[3]));
+        l_run = l_run * alpha + (s01.x + s01.y);
+        b_run = b_new;
+        tmem_st32(trow + scol, pw);
         tmem_wait_st();
         if (j > 0 && __any_sync(0xffffffffu, rescale)) {
-          // O may only be touched once the previous tile's P.V has landed
+          // O holds tiles < jt at the old base: once tile jt - 1's P.V has landed,
+          // bring this warpgroup's half of it to the new one
           const uint32_t jp = jt - 1;
           if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_done[jp % kNS], (jp / kNS) & 1)))) break;
           tc_fence_after();
+          const float2 al2 = make_float2(alpha, alpha);
 #pragma unroll 1
-          for (int c8 = 0; c8 < 8; ++c8) {
+          for (int c4 = 0; c4 < 4; ++c4) {
             uint32_t ov[32];
-            tmem_ld32(trow + kColO + 32 * c8, ov);
+            tmem_ld32(trow + kColO + 128 * wg + 32 * c4, ov);
             tmem_wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) ov[e] = __float_as_uint(__uint_as_float(ov[e]) * alpha);
-            tmem_st32(trow + kColO + 32 * c8, ov);
+            for (int e = 0; e < 16; ++e) {
+              const float2 o = fmul2(make_float2(__uint_as_float(ov[2 * e]), __uint_as_float(ov[2 * e + 1])), al2);
+              ov[2 * e] = __float_as_uint(o.x);
+              ov[2 * e + 1] = __float_as_uint(o.y);
+            }
+            tmem_st32(trow + kColO + 128 * wg + 32 * c4, ov);
           }
           tmem_wait_st();
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          if (rank == 0) mbar_arrive(&sm.p_full[sb]);
-          else mbar_arrive_remote(&sm.p_full[sb], 0);
-        }
+        arrive_cta0(&sm.p_full[sb]);
       }
       J += it.n;
       if (!ok) break;
+      // ---- this warpgroup's sum for the other one ----
+      sm.xsum[item & 1][wg][r] = l_run;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sm.xsum_full);
+
       Item nxt{};
       const bool have_next = next_item(k, nxt);
-      if (have_next && !(ok = prepare_q(nxt, item + 1))) break;
+      if (have_next && !a.q_rotated && !(ok = prepare_q(nxt, item + 1))) break;
 
-      // ---- epilogue: O / l * sigmoid(gate) -> bf16 -> global ----
-      // 32 dims at a time through the warp's staging area: each thread writes
+      // ---- epilogue: O / l * sigmoid(gate) -> bf16 -> global, this warpgroup's 128 dims ----
+      // 32 dims at a time through the warp's transpose area: each thread writes
       // its row (16-byte chunks XOR-swizzled by row, so neither phase has bank
       // conflicts), then each store instruction covers 8 rows x 64 bytes.
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.xsum_full, item & 1)))) break;
+      const float l = l_run + sm.xsum[item & 1][wg ^ 1][r];   // both at the row's final base
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, item & 1)))) break;
       tc_fence_after();
-      float f = l_run > 0.f ? 1.f / l_run : 0.f;
+      float f = l > 0.f ? 1.f / l : 0.f;
       if (a.gate != nullptr && valid) {
         const float gs = __bfloat162float(a.gate[((int64_t)it.b * a.T + row) * kHq + h]);
         f *= 1.f / (1.f + __expf(-gs));
       }
+      const float2 f2 = make_float2(f, f);
       uint8_t* stg = sm.ostage[warp];
       const int rr = lane >> 2, ch = lane & 3;   // store phase: rows rr + 8 t, chunk ch
+      uint32_t ov[32], on[32];
+      tmem_ld32(trow + kColO + 128 * wg, on);
 #pragma unroll 1
-      for (int c8 = 0; c8 < 8; ++c8) {
-        uint32_t ov[32];
-        tmem_ld32(trow + kColO + 32 * c8, ov);
+      for (int c = 0; c < 4; ++c) {
         tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] = on[e];
+        if (c < 3) tmem_ld32(trow + kColO + 128 * wg + 32 * (c + 1), on);   // next chunk in flight
 #pragma unroll
         for (int q4 = 0; q4 < 4; ++q4) {
           uint32_t w4[4];
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const int c = 8 * q4 + 2 * e;
-            w4[e] = pack_bf16(__uint_as_float(ov[c]) * f, __uint_as_float(ov[c + 1]) * f);
+            const int cc = 8 * q4 + 2 * e;
+            const float2 o = fmul2(make_float2(__uint_as_float(ov[cc]), __uint_as_float(ov[cc + 1])), f2);
+            w4[e] = pack_bf16(o.x, o.y);
           }
           *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q4 ^ ((lane >> 1) & 3))) =
               make_uint4(w4[0], w4[1], w4[2], w4[3]);
@@ -601,13 +723,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
           const int rw = rr + 8 * t;                   // row within this warp's 32
-          const int grow = it.m0 + 32 * warp + rw;     // query row in the sequence
+          const int grow = it.m0 + 32 * qtr + rw;      // query row in the sequence
           const uint4 v = *reinterpret_cast<const uint4*>(stg + rw * 64 + 16 * (ch ^ ((rw >> 1) & 3)));
           if (grow < a.T)
-            *reinterpret_cast<uint4*>(a.out + (((int64_t)it.b * a.T + grow) * kHq + h) * kD + 32 * c8 + 8 * ch) = v;
+            *reinterpret_cast<uint4*>(a.out + (((int64_t)it.b * a.T + grow) * kHq + h) * kD + 128 * wg + 32 * c +
+                                      8 * ch) = v;
         }
         __syncwarp();
       }
+      tc_fence_before();
+      __syncwarp();
+      arrive_cta0(&sm.o_free);
       it = nxt;
       have = have_next;
       ++item;
@@ -618,7 +744,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
   tc_fence_before();
   __syncthreads();
   cluster_sync();
-  if (warp == 5) {
+  if (warp == kMmaWarp) {
     tc_fence_after();
     tmem_dealloc_pair(tmem, 512);
   }
@@ -640,28 +766,31 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   a.n_mtiles = (h.T + kBM - 1) / kBM;
   const long long n_items = (long long)a.n_mtiles * h.B * (kHq / 2);   // (query tile, head pair)
   if (n_items <= 0 || n_items > 0x3fffffffLL) return cudaErrorInvalidValue;
+  if (!full && !h.q_rotated) return cudaErrorInvalidValue;   // sliding layers take rotated queries
   const long long grid = 2 * (n_items < h.n_pairs ? n_items : h.n_pairs);   // persistent CTA pairs
-  const size_t smem = prefill_smem_bytes();
   profile_before(st);
   if (full)
-    prefill_kernel<true><<<(unsigned)grid, kPfThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_q, h.tm_o, a);
+    prefill_kernel<true><<<(unsigned)grid, kPfThreads, prefill_smem_bytes_t<true>(), st>>>(h.tm_k, h.tm_v, h.tm_q,
+                                                                                            h.tm_o, a);
   else
-    prefill_kernel<false><<<(unsigned)grid, kPfThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_q, h.tm_o, a);
+    prefill_kernel<false><<<(unsigned)grid, kPfThreads, prefill_smem_bytes_t<false>(), st>>>(h.tm_k, h.tm_v, h.tm_q,
+                                                                                             h.tm_o, a);
   profile_after(st);
   count_launch();
   return cudaGetLastError();
 }
 
-// Box rows of the K and V tensor maps this kernel expects (per-CTA halves).
-int prefill_k_box_rows() { return kKBoxRows; }
-int prefill_v_box_rows() { return kBN; }
+// Box rows of the K and V tensor maps this kernel expects.
+int prefill_k_box_rows() { return kHalfKeys; }
+int prefill_v_box_rows() { return kHalfKeys; }
 int prefill_q_box_rows() { return kBM; }
 
 cudaError_t prefill_set_smem_attr() {
-  const int smem = (int)prefill_smem_bytes();
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)prefill_smem_bytes_t<true>());
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  return cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                              (int)prefill_smem_bytes_t<false>());
 }
 
 }  // namespace hyb

@@ -112,3 +112,45 @@ def test_random_cache_path(lib, seed):
     ref = O.decode(f64(xd["q"]), None if gate is None else f64(gate), [start] * B, [h[0] for h in hist],
                    [h[1] for h in hist], [h[2] for h in hist], lt)
     check(out, ref, f"{c} decode")
+
+
+@pytest.mark.parametrize("seed", SEEDS[:8])
+def test_random_cache_path_against_raw_history(lib, seed):
+    """The same kind of random case on bf16 caches, but the oracle never reads
+    the cache: it gets every raw (unrotated) token of the sequence and applies
+    RoPE, masks and the window itself.  A rotation or placement error on the
+    append side, which the stored-history comparison above would carry into
+    its reference, fails here."""
+    c = _case(seed)
+    c["fp8"] = False
+    lt, B = c["lt"], c["B"]
+    cache = _make_cache(lib, c)
+    chunks, start = [], 0
+    for i, T in enumerate((c["T1"], c["T2"])):
+        x = synth.prefill_inputs(B, T, seed=7000 + 10 * seed + i, device="cuda", start=start)
+        gate = x["gate"] if c["gate"] else None
+        out = lib.hyb_attn_prefill(x["q"], x["k"], x["v"], gate, x["pos"], lt, cache=cache)
+        torch.cuda.synchronize()
+        assert lib.hyb_device_error() == 0
+        chunks.append({k: f64(v) if k != "pos" else v.cpu().numpy() for k, v in x.items() if k != "qkv"})
+        whole = {k: np.concatenate([ch[k] for ch in chunks], axis=1) for k in ("q", "k", "v", "gate", "pos")}
+        rows = np.arange(start, start + T)
+        ref = O.prefill(whole["q"], whole["k"], whole["v"], whole["gate"] if c["gate"] else None, whole["pos"], lt,
+                        rows=rows)
+        check(out, ref, f"{c} chunk {i} (raw history)")
+        start += T
+    xd = synth.decode_query(B, seed=8000 + seed, device="cuda")
+    lib.hyb_kv_append(cache, xd["k"], xd["v"])
+    gate = xd["gate"] if c["gate"] else None
+    out = lib.hyb_attn_decode(xd["q"], gate, cache, max_len=cache.capacity)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    n = start + 1
+    idx = np.arange(n)
+    keys, vals = [], []
+    for b in range(B):
+        kb = np.concatenate([whole["k"][b], f64(xd["k"])[b]], axis=0)
+        keys.append(O.rope_layer(kb, idx, lt))
+        vals.append(np.concatenate([whole["v"][b], f64(xd["v"])[b]], axis=0))
+    ref = O.decode(f64(xd["q"]), None if gate is None else f64(gate), [start] * B, keys, vals, [idx] * B, lt)
+    check(out, ref, f"{c} decode (raw history)")

@@ -196,3 +196,40 @@ def test_bad_block_table_entry_raises_page_error(lib):
     assert lib.hyb_device_error() & lib.DEV_ERR_PAGE
     assert torch.isfinite(out.float()).all()
     assert lib.hyb_device_error() == 0                     # the previous read cleared the word
+
+
+def test_paged_chunked_prefill_matches_oracle(lib):
+    """Two prefill chunks and a decode step through a paged cache with pages
+    of 64 keys scattered over the pool, compared with the oracle on the raw
+    tokens (it rotates the keys and builds the history itself)."""
+    B, page, max_pages = 2, 64, 12
+    n_pages = B * max_pages + 3
+    paged = lib.KVCache(O.FULL, B, kv_dtype=lib.KV_BF16, page_size=page, n_pages=n_pages,
+                        block_table=_table(B, max_pages, n_pages, 111))
+    raw, start = [], 0
+    for i, T in enumerate((333, 190)):
+        x = synth.prefill_inputs(B, T, seed=112 + i, device="cuda", start=start)
+        out = lib.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], x["pos"], O.FULL, cache=paged)
+        torch.cuda.synchronize()
+        assert lib.hyb_device_error() == 0
+        raw.append({k: f64(v) if k != "pos" else v.cpu().numpy() for k, v in x.items() if k != "qkv"})
+        w = {k: np.concatenate([r[k] for r in raw], axis=1) for k in ("q", "k", "v", "gate", "pos")}
+        ref = O.prefill(w["q"], w["k"], w["v"], w["gate"], w["pos"], O.FULL, rows=np.arange(start, start + T))
+        got = f64(out)
+        max_abs = float(np.abs(got - ref).max())
+        rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+        assert max_abs <= 2e-2 and rel <= 5e-3, f"chunk {i}: max_abs {max_abs:.3e} rel_l2 {rel:.3e}"
+        start += T
+    xd = synth.decode_query(B, seed=115, device="cuda")
+    lib.hyb_kv_append(paged, xd["k"], xd["v"])
+    out = lib.hyb_attn_decode(xd["q"], xd["gate"], paged, max_len=paged.capacity)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    idx = np.arange(start + 1)
+    keys = [O.rope_layer(np.concatenate([w["k"][b], f64(xd["k"])[b]]), idx, O.FULL) for b in range(B)]
+    vals = [np.concatenate([w["v"][b], f64(xd["v"])[b]]) for b in range(B)]
+    ref = O.decode(f64(xd["q"]), f64(xd["gate"]), [start] * B, keys, vals, [idx] * B, O.FULL)
+    got = f64(out)
+    max_abs = float(np.abs(got - ref).max())
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    assert max_abs <= 2e-2 and rel <= 5e-3, f"decode: max_abs {max_abs:.3e} rel_l2 {rel:.3e}"

@@ -12,6 +12,7 @@ import numpy as np
 import pytest
 import torch
 
+import oracle as O
 from full_gqa_attention_partial_b200 import synth
 
 pytestmark = pytest.mark.gpu
@@ -56,3 +57,32 @@ def test_noalloc_decode_rejects_batches_beyond_the_fixed_scratch(lib):
         lib.hyb_attn_decode_noalloc(q, None, cache, max_len=512, out=torch.empty_like(q))
     assert e.value.status == -4
     assert "fixed scratch" in str(e.value)
+
+
+@pytest.mark.parametrize("lt", [0, 1])
+def test_noalloc_decode_matches_oracle(lib, lt):
+    """The allocation-free entry point against the oracle directly: the
+    oracle gets the raw history and the new token and applies RoPE, the
+    window and the gate itself."""
+    B, n_hist = 2, 900
+    cap = 1024 if lt == lib.FULL else 512
+    cache = lib.KVCache(lt, B, capacity=cap, head0=[5, 400] if lt == lib.SLIDING else None)
+    hist = synth.prefill_inputs(B, n_hist, seed=930 + lt)
+    lib.hyb_kv_append(cache, hist["k"].cuda(), hist["v"].cuda())
+    qd = synth.decode_query(B, seed=940 + lt)
+    lib.hyb_kv_append(cache, qd["k"].cuda(), qd["v"].cuda())
+    out = torch.empty(B, 16, 256, dtype=torch.bfloat16, device="cuda")
+    lib.hyb_attn_decode_noalloc(qd["q"].cuda(), qd["gate"].cuda(), cache, max_len=cap, out=out)
+    torch.cuda.synchronize()
+    assert lib.hyb_device_error() == 0
+    f = lambda t: t.float().double().numpy()
+    n = n_hist + 1
+    lo = 0 if lt == lib.FULL else n - 512
+    idx = np.arange(lo, n)
+    keys = [O.rope_layer(np.concatenate([f(hist["k"][b]), f(qd["k"][b])])[lo:], idx, lt) for b in range(B)]
+    vals = [np.concatenate([f(hist["v"][b]), f(qd["v"][b])])[lo:] for b in range(B)]
+    ref = O.decode(f(qd["q"]), f(qd["gate"]), [n - 1] * B, keys, vals, [idx] * B, lt)
+    got = out.float().cpu().double().numpy()
+    max_abs = float(np.abs(got - ref).max())
+    rel = float(np.linalg.norm(got - ref) / np.linalg.norm(ref))
+    assert max_abs <= MAX_ABS and rel <= REL_L2, f"max_abs {max_abs:.3e} rel_l2 {rel:.3e}"
