@@ -922,17 +922,17 @@ def main():
     main_res, layers = run("step: 4-layer group prefill", bench_main, hyb, args, dist, peaks)
     extras = {}
     if dist.world == 1 and not args.no_extras:
+        extras["prefill_128k"] = run("prefill_128k", bench_prefill_128k, hyb, args, peaks)
         extras["layer_prefill"] = run("layer_prefill", bench_layer, hyb, args, peaks)
         extras["decode"] = run("decode", bench_decode, hyb, args, peaks)
         extras["decode_fp8"] = run("decode_fp8", bench_decode, hyb, args, peaks, fp8=True)
         extras["decode_paged"] = run("decode_paged", bench_decode, hyb, args, peaks, page=64)
-        if args.chunked:
-            extras["chunked_prefill"] = run("chunked_prefill", bench_chunked, hyb, args, peaks)
-        extras["prefill_128k"] = run("prefill_128k", bench_prefill_128k, hyb, args, peaks)
         if args.decode_1m:
             extras["decode_1m"] = run("decode_1m", bench_decode_1m, hyb, args, peaks)
             torch.cuda.empty_cache()
             extras["decode_1m_fp8"] = run("decode_1m_fp8", bench_decode_1m, hyb, args, peaks, fp8=True)
+        if args.chunked:
+            extras["chunked_prefill"] = run("chunked_prefill", bench_chunked, hyb, args, peaks)
     # with several ranks the sequence-sharded 1M decode runs by default (every rank
     # takes part: it has collectives)
     if (args.decode_sharded or dist.world > 1) and not args.no_extras:

@@ -150,6 +150,23 @@ hyb_status make_q_map(CUtensorMap* m, const void* base, uint64_t T, uint64_t bat
   return HYB_OK;
 }
 
+// 4-D map {256 dims, 16 heads, T tokens, batch} over the bf16 output with boxes
+// of 32 dims x 1 head x 32 tokens and 64-byte swizzle: one softmax warp's 32
+// rows x 32 dims of the prefill epilogue per store.
+hyb_status make_out_map(CUtensorMap* m, void* base, uint64_t T, uint64_t batch) {
+  auto enc = encode_fn();
+  if (!enc) return fail(HYB_EUNSUPPORTED, "cuTensorMapEncodeTiled is not available from the driver");
+  const uint64_t token_bytes = (uint64_t)kHq * kD * 2;
+  cuuint64_t dims[4] = {(cuuint64_t)kD, (cuuint64_t)kHq, T, batch};
+  cuuint64_t strides[3] = {(cuuint64_t)kD * 2, token_bytes, T * token_bytes};
+  cuuint32_t box[4] = {32, 1, 32, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, base, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(HYB_ECUDA, "cuTensorMapEncodeTiled(out) failed with CUresult %d", (int)r);
+  return HYB_OK;
+}
+
 // Rows per (page or sequence) and pages (or sequences) of a cache's storage:
 // a contiguous cache is [batch][4][capacity][256], a paged one
 // [n_pages][4][page_size][256].
@@ -551,7 +568,7 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
     q_rot = true;
   }
   if ((s = make_q_map(&ph.tm_q, q, T, B, (uint64_t)q_row_stride * 2, prefill_q_box_rows(), "Q")) != HYB_OK) return s;
-  if ((s = make_q_map(&ph.tm_o, out, T, B, (uint64_t)kHq * kD * 2, prefill_q_box_rows(), "out")) != HYB_OK) return s;
+  if ((s = make_out_map(&ph.tm_o, out, T, B)) != HYB_OK) return s;
   ph.q = q;
   ph.q_stride = q_row_stride;
   ph.gate = gate;

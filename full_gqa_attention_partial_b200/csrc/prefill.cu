@@ -50,6 +50,7 @@
 // of a row is 2^(s - base), the base only moves (and O is only rescaled)
 // when a tile's maximum exceeds it by more than 8, so P stays <= 256.
 #include <algorithm>
+#include <cstddef>
 
 #include "common.cuh"
 #include "launch.h"
@@ -87,7 +88,8 @@ struct PfSmem {
   // half of the frequencies
   float4 rot_lo[FULL ? R / 4 : 1][16];
   float4 rot_hi[8][FULL ? R / 4 : 1];
-  uint8_t ostage[kSmWarps][kStageBytes];   // epilogue transpose area per softmax warp
+  // epilogue staging per softmax warp, the source of its TMA stores (64-byte swizzle: 512-byte periods)
+  alignas(1024) uint8_t ostage[kSmWarps][kStageBytes];
   double inv_freq[R / 2];
   float xmax[2][2][kBM];             // [tile parity][warpgroup][row]: a row's maximum over the warpgroup's keys
   float xsum[2][2][kBM];             // [item parity][warpgroup][row]: running sum at item end
@@ -114,6 +116,8 @@ size_t prefill_smem_bytes_t() { return sizeof(PfSmem<FULL>) + 1024; }
 size_t prefill_smem_bytes() { return std::max(prefill_smem_bytes_t<true>(), prefill_smem_bytes_t<false>()); }
 static_assert(sizeof(PfSmem<true>) + 1024 <= 232448 && sizeof(PfSmem<false>) + 1024 <= 232448,
               "prefill shared memory exceeds 227 KB");
+static_assert(offsetof(PfSmem<true>, ostage) % 1024 == 0 && offsetof(PfSmem<false>, ostage) % 1024 == 0,
+              "staging areas must start on a swizzle period");
 
 struct PfArgs {
   const __nv_bfloat16* q;
@@ -585,6 +589,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       const int row = it.m0 + r;
       const bool valid = row < a.T;
       const int qseq = it.qb + row;
+      // the row's gate score, loaded now so that its latency is not on the epilogue's path
+      const float gscore = (a.gate != nullptr && valid) ? __bfloat162float(a.gate[((int64_t)it.b * a.T + row) * kHq + h]) : 0.f;
 
       // ---- online softmax over this warpgroup's keys of each tile ----
       float l_run = 0.f, b_run = -INFINITY;   // running sum (this warpgroup's keys) and the row's base
@@ -605,12 +611,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         const int ks0 = it.kb + (it.j_lo + j) * kBN + 64 * wg;   // sequence index of this warpgroup's first key
         const bool whole = ks0 >= 0 && ks0 + 63 <= it.q_lo && (FULL || it.q_hi - ks0 <= kWindow - 1);
         if (!whole) {
+          // visible columns of this row: c_lo <= c <= c_hi (the band is contiguous);
+          // none visible: an empty range past the last column
+          int c_lo = max(-ks0, FULL ? 0 : qseq - (kWindow - 1) - ks0);
+          int c_hi = qseq - ks0;
+          if (c_hi < c_lo) c_lo = c_hi = 64;
+          const uint32_t span = (uint32_t)(c_hi - c_lo);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) {
-            const int ks = ks0 + c;
-            const bool vis = ks >= 0 && ks <= qseq && (FULL || qseq - ks <= kWindow - 1);
-            if (!vis) s[c] = -INFINITY;
-          }
+          for (int c = 0; c < 64; ++c)
+            if ((uint32_t)(c - c_lo) > span) s[c] = -INFINITY;
         }
         // row maximum over this warpgroup's keys: pairwise tree (short dependency chains)
         float mx[32];
@@ -684,21 +693,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       if (have_next && !a.q_rotated && !(ok = prepare_q(nxt, item + 1))) break;
 
       // ---- epilogue: O / l * sigmoid(gate) -> bf16 -> global, this warpgroup's 128 dims ----
-      // 32 dims at a time through the warp's transpose area: each thread writes
-      // its row (16-byte chunks XOR-swizzled by row, so neither phase has bank
-      // conflicts), then each store instruction covers 8 rows x 64 bytes.
+      // 32 dims at a time through the warp's staging area: each thread writes
+      // its row of 64 bytes, 16-byte chunk q at chunk q ^ ((row / 2) % 4) (no bank
+      // conflicts, and the layout of a 64-byte-swizzled tensor map), then one
+      // lane issues a TMA store of the 32 rows x 32 dims (rows past T are not
+      // written).
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.xsum_full, item & 1)))) break;
       const float l = l_run + sm.xsum[item & 1][wg ^ 1][r];   // both at the row's final base
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, item & 1)))) break;
       tc_fence_after();
       float f = l > 0.f ? 1.f / l : 0.f;
-      if (a.gate != nullptr && valid) {
-        const float gs = __bfloat162float(a.gate[((int64_t)it.b * a.T + row) * kHq + h]);
-        f *= 1.f / (1.f + __expf(-gs));
-      }
+      if (a.gate != nullptr) f *= 1.f / (1.f + __expf(-gscore));
       const float2 f2 = make_float2(f, f);
       uint8_t* stg = sm.ostage[warp];
-      const int rr = lane >> 2, ch = lane & 3;   // store phase: rows rr + 8 t, chunk ch
       uint32_t ov[32], on[32];
       tmem_ld32(trow + kColO + 128 * wg, on);
 #pragma unroll 1
@@ -719,15 +726,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
           *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q4 ^ ((lane >> 1) & 3))) =
               make_uint4(w4[0], w4[1], w4[2], w4[3]);
         }
+        fence_proxy_async();   // the staging writes, then the TMA engine's read of them
         __syncwarp();
-#pragma unroll
-        for (int t = 0; t < 4; ++t) {
-          const int rw = rr + 8 * t;                   // row within this warp's 32
-          const int grow = it.m0 + 32 * qtr + rw;      // query row in the sequence
-          const uint4 v = *reinterpret_cast<const uint4*>(stg + rw * 64 + 16 * (ch ^ ((rw >> 1) & 3)));
-          if (grow < a.T)
-            *reinterpret_cast<uint4*>(a.out + (((int64_t)it.b * a.T + grow) * kHq + h) * kD + 128 * wg + 32 * c +
-                                      8 * ch) = v;
+        if (lane == 0) {
+          tma_store_4d(&tm_o, smem_u32(stg), 128 * wg + 32 * c, h, it.m0 + 32 * qtr, it.b);
+          tma_store_commit();
+          tma_store_wait_read();   // the staging area is free again
         }
         __syncwarp();
       }
@@ -740,6 +744,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     }
   }
 
+  if (warp < kSmWarps && lane == 0) tma_store_commit_and_wait();   // epilogue stores complete
   // the peer's shared memory and tensor memory stay alive until both CTAs are done
   tc_fence_before();
   __syncthreads();
