@@ -4,6 +4,7 @@
 #include <cudaTypedefs.h>
 
 #include <atomic>
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -94,6 +95,14 @@ hyb_status ensure_device() {
     g_dev_state[dev] = -1;
     return fail(HYB_EUNSUPPORTED, "device %d has compute capability %d.%d; this library is built for sm_100a",
                 dev, major, minor);
+  }
+  {  // rotation frequencies of both layer types, fp64 on the host
+    double f[2][128] = {};
+    for (int k = 0; k < RopeCfg<false>::R / 2; ++k)
+      f[0][k] = std::pow(RopeCfg<false>::theta, -2.0 * k / RopeCfg<false>::R);
+    for (int k = 0; k < RopeCfg<true>::R / 2; ++k)
+      f[1][k] = std::pow(RopeCfg<true>::theta, -2.0 * k / RopeCfg<true>::R);
+    if ((e = cudaMemcpyToSymbol(g_inv_freq, f, sizeof(f))) != cudaSuccess) return cuda_fail(e, "frequency table");
   }
   if ((e = prefill_set_smem_attr()) != cudaSuccess) return cuda_fail(e, "prefill smem attribute");
   cudaDeviceGetAttribute(&g_dev_sms[dev], cudaDevAttrMultiProcessorCount, dev);

@@ -64,8 +64,14 @@ __device__ __forceinline__ void kv_coord(const PageMap& pm, int b, int row, int&
 // [-pi, pi], far below bf16 resolution).  fp32 pos * inv_freq alone would be
 // off by ~0.06 rad at pos ~ 2^20.
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ double rope_inv_freq(double theta, int k, int R) {
-  return pow(theta, -2.0 * (double)k / (double)R);
+// Rotation frequencies inv_freq_k = theta^(-2k/R), k < R/2, of both layer
+// types: [0][k] sliding (R = 256, theta 1e4), [1][k] full (R = 64, theta 5e6).
+// Computed once per device on the host (fp64) and copied in when the device
+// is set up, so that no kernel evaluates pow() itself.
+static __device__ double g_inv_freq[2][128];
+template <bool FULL>
+__device__ __forceinline__ double rope_inv_freq(int k) {
+  return __ldg(&g_inv_freq[FULL ? 1 : 0][k]);
 }
 
 __device__ __forceinline__ void rope_sincos(int pos, double inv_freq, float* s, float* c) {
@@ -95,6 +101,17 @@ __device__ __forceinline__ void small_angle_sincos(int delta, float inv_freq_f, 
   r = fmaf(-n, -1.74845553e-7f, r);       // ... and the rest of 2*pi
   __sincosf(r, s, c);
 }
+
+// ---------------------------------------------------------------------------
+// Programmatic dependent launch.  A kernel launched with programmatic stream
+// serialization may start while the previous kernel of its stream is still
+// running: pdl_wait() blocks until that kernel has completed and its memory
+// is visible, so everything before it must not read what the previous
+// kernel writes.  pdl_launch_dependents() lets the next kernel start its own
+// launch early.  Without the launch attribute both are no-ops.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
 // bf16 packing

@@ -66,6 +66,8 @@ struct DecSmem {
   float merge_l[4][4];
   __nv_bfloat16 qs[4][kD];      // rotated queries of the group
   int32_t tags[kWindow];
+  float cl_o[4][kD];            // cluster merge: this split's normalised output per head ...
+  float cl_lse[4];              // ... and its base-2 log-sum-exp
   uint64_t full[kStages];
   uint64_t empty[kStages];
   __device__ float (&merge_o())[4][4][kD] { return *reinterpret_cast<float(*)[4][4][kD]>(ring); }
@@ -103,7 +105,27 @@ struct DecArgs {
   float* part_lse;
   int n_splits;
   PageMap pm;         // paged cache: maps over the pool {.., page, 4, n_pages}
+  // cluster merge (the splits of one (sequence, KV head) form a thread-block
+  // cluster): CTA 0 of the cluster merges them and writes the result itself
+  int cluster_merge;
+  const __nv_bfloat16* gate;   // [B][16] or null
+  __nv_bfloat16* out;          // [B][16][256] gated bf16, or
+  float* out_o;                // [B][16][256] fp32 and
+  float* out_lse;              // [B][16] base-2 log-sum-exp
 };
+
+// Loads from the shared memory of another CTA of the cluster.
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
+}
 
 template <bool FULL, bool FP8>
 __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
@@ -117,6 +139,17 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
   const int split = blockIdx.x, kvh = blockIdx.y, b = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < NST; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], 4);
+    }
+    fence_barrier_init();
+  }
+  // the append before this launch writes len, tags and the new token's row
+  pdl_wait();
+  pdl_launch_dependents();
+
   const int L = a.len[b];
   const int qseq = L - 1;
   const int n_keys = FULL ? L : kWindow;          // keys (FULL) or ring slots (SLIDING)
@@ -125,14 +158,6 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
   const int k0 = split * kps;
   const int k1 = min(n_keys, k0 + kps);
   const int n_stages = (k1 > k0 && L > 0) ? (k1 - k0 + kDecKeys - 1) / kDecKeys : 0;
-
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < NST; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], 4);
-    }
-    fence_barrier_init();
-  }
   if (!FULL) {
     for (int i = threadIdx.x; i < kWindow; i += blockDim.x) sm.tags[i] = a.tag[(int64_t)b * kWindow + i];
   }
@@ -178,9 +203,7 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
       for (int i = max(0, issued - NST); i < issued; ++i)
         mbar_wait(&sm.full[i % NST], (i / NST) & 1);
     }
-    return;
-  }
-
+  } else {
   // ---------------- consumers: rotate the group's 4 queries ----------------
   {
     const int hh = threadIdx.x >> 5;        // 0..3
@@ -204,7 +227,7 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
           const float x = e ? bf16hi(xs[w]) : bf16lo(xs[w]);
           const float y = e ? bf16hi(ys[w]) : bf16lo(ys[w]);
           float s, c;
-          rope_sincos(p, rope_inv_freq(RopeCfg<FULL>::theta, kb + 2 * w + e, R), &s, &c);
+          rope_sincos(p, rope_inv_freq<FULL>(kb + 2 * w + e), &s, &c);
           o2[e] = first_half ? fmaf(x, c, -y * s) : fmaf(x, c, y * s);
         }
         os[w] = pack_bf16(o2[0], o2[1]);
@@ -440,11 +463,67 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
       lse = den > 0.f ? M + log2f(den) : -INFINITY;
     }
     const int hq = kvh * kGroup + hh;
-    const int64_t row = ((int64_t)b * kHq + hq) * a.n_splits + split;
-    float4* dst = reinterpret_cast<float4*>(a.part_o + row * kD + d0);
-    dst[0] = make_float4(res[0], res[1], res[2], res[3]);
-    dst[1] = make_float4(res[4], res[5], res[6], res[7]);
-    if (lane == 0) a.part_lse[row] = lse;
+    if (a.cluster_merge) {   // for CTA 0 of the cluster
+      *reinterpret_cast<float4*>(&sm.cl_o[hh][d0]) = make_float4(res[0], res[1], res[2], res[3]);
+      *reinterpret_cast<float4*>(&sm.cl_o[hh][d0 + 4]) = make_float4(res[4], res[5], res[6], res[7]);
+      if (lane == 0) sm.cl_lse[hh] = lse;
+    } else {
+      const int64_t row = ((int64_t)b * kHq + hq) * a.n_splits + split;
+      float4* dst = reinterpret_cast<float4*>(a.part_o + row * kD + d0);
+      dst[0] = make_float4(res[0], res[1], res[2], res[3]);
+      dst[1] = make_float4(res[4], res[5], res[6], res[7]);
+      if (lane == 0) a.part_lse[row] = lse;
+    }
+  }
+  }
+
+  if (a.cluster_merge) {
+    // ---------------- merge the cluster's splits in CTA 0 (the log-sum-exp
+    // combination of decode_combine_kernel, same order of operations) ----------------
+    cluster_sync();   // every split's result is in its CTA's shared memory
+    if (cluster_ctarank() == 0 && warp < 4) {
+      const int hh = warp, d0 = lane * 8;
+      const int hq = kvh * kGroup + hh;
+      const int64_t orow = (int64_t)b * kHq + hq;
+      float M = -INFINITY;
+      for (int s2 = 0; s2 < a.n_splits; ++s2) M = fmaxf(M, ld_cluster_f32(mapa_cluster(smem_u32(&sm.cl_lse[hh]), s2)));
+      float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, den = 0.f;
+      if (M != -INFINITY) {
+        for (int s2 = 0; s2 < a.n_splits; ++s2) {
+          const float ls = ld_cluster_f32(mapa_cluster(smem_u32(&sm.cl_lse[hh]), s2));
+          if (ls == -INFINITY) continue;
+          const float w = exp2f(ls - M);
+          den += w;
+          const float4 o0 = ld_cluster_f32x4(mapa_cluster(smem_u32(&sm.cl_o[hh][d0]), s2));
+          const float4 o1 = ld_cluster_f32x4(mapa_cluster(smem_u32(&sm.cl_o[hh][d0 + 4]), s2));
+          acc[0] += w * o0.x; acc[1] += w * o0.y; acc[2] += w * o0.z; acc[3] += w * o0.w;
+          acc[4] += w * o1.x; acc[5] += w * o1.y; acc[6] += w * o1.z; acc[7] += w * o1.w;
+        }
+      }
+      float r8[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) r8[e] = den > 0.f ? acc[e] / den : 0.f;
+      if (a.out_o != nullptr) {
+        float4* dst = reinterpret_cast<float4*>(a.out_o + orow * kD + d0);
+        dst[0] = make_float4(r8[0], r8[1], r8[2], r8[3]);
+        dst[1] = make_float4(r8[4], r8[5], r8[6], r8[7]);
+        if (lane == 0) a.out_lse[orow] = den > 0.f ? M + log2f(den) : -INFINITY;
+      } else {
+        if (a.gate != nullptr) {
+          const float g = 1.f / (1.f + __expf(-__bfloat162float(a.gate[orow])));
+#pragma unroll
+          for (int e = 0; e < 8; ++e) r8[e] *= g;
+        }
+        uint32_t w4[4];
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const __nv_bfloat16 lo = __float2bfloat16_rn(r8[2 * e]), hi = __float2bfloat16_rn(r8[2 * e + 1]);
+          w4[e] = (uint32_t)__bfloat16_as_ushort(lo) | ((uint32_t)__bfloat16_as_ushort(hi) << 16);
+        }
+        *reinterpret_cast<uint4*>(a.out + orow * kD + d0) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
+      }
+    }
+    cluster_sync();   // the other CTAs' shared memory stays until CTA 0 has read it
   }
 }
 
@@ -467,6 +546,8 @@ struct CombineArgs {
 };
 
 __global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
+  pdl_wait();   // the split kernel's partials
+  pdl_launch_dependents();
   const int row = blockIdx.x;  // b * 16 + h
   const int d = threadIdx.x;
   const float* lse = a.lse + (int64_t)row * a.l_rstride;
@@ -550,21 +631,32 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
   a.part_lse = h.part_lse;
   a.n_splits = h.n_splits;
   a.pm = h.pm;
+  // sliding layers (at most 8 splits of a 512-slot ring): the splits of one
+  // (sequence, KV head) run as a cluster and merge in its CTA 0, no second
+  // kernel; full layers write per-split partials for decode_combine_kernel
+  a.cluster_merge = (!full && h.n_splits <= 8) ? 1 : 0;
+  a.gate = reinterpret_cast<const __nv_bfloat16*>(h.gate);
+  a.out = reinterpret_cast<__nv_bfloat16*>(h.out);
+  a.out_o = h.out_o;
+  a.out_lse = h.out_lse;
   const dim3 grid(h.n_splits, kHkv, h.B);
   const size_t smem = decode_smem_bytes(h.fp8);
   profile_before(st);
+  cudaError_t e;
+  const unsigned cl = a.cluster_merge ? (unsigned)h.n_splits : 0u;
+  const dim3 blk(kDecThreads, 1, 1);
   if (full && h.fp8)
-    decode_split_kernel<true, true><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_ks, h.tm_vs, a);
+    e = launch_pdl(decode_split_kernel<true, true>, grid, blk, smem, st, cl, h.tm_k, h.tm_v, h.tm_ks, h.tm_vs, a);
   else if (full)
-    decode_split_kernel<true, false><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_k, h.tm_v, a);
+    e = launch_pdl(decode_split_kernel<true, false>, grid, blk, smem, st, cl, h.tm_k, h.tm_v, h.tm_k, h.tm_v, a);
   else if (h.fp8)
-    decode_split_kernel<false, true><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_ks, h.tm_vs, a);
+    e = launch_pdl(decode_split_kernel<false, true>, grid, blk, smem, st, cl, h.tm_k, h.tm_v, h.tm_ks, h.tm_vs, a);
   else
-    decode_split_kernel<false, false><<<grid, kDecThreads, smem, st>>>(h.tm_k, h.tm_v, h.tm_k, h.tm_v, a);
+    e = launch_pdl(decode_split_kernel<false, false>, grid, blk, smem, st, cl, h.tm_k, h.tm_v, h.tm_k, h.tm_v, a);
   profile_after(st);
   count_launch();
-  cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
+  if (a.cluster_merge) return cudaSuccess;
   CombineArgs c;
   c.o = h.part_o;
   c.lse = h.part_lse;
@@ -577,9 +669,9 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
   c.out = reinterpret_cast<__nv_bfloat16*>(h.out);
   c.out_o = h.out_o;
   c.out_lse = h.out_lse;
-  decode_combine_kernel<<<h.B * kHq, 256, 0, st>>>(c);
+  e = launch_pdl(decode_combine_kernel, dim3(h.B * kHq, 1, 1), dim3(256, 1, 1), 0, st, 0u, c);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 // ---------------------------------------------------------------------------

@@ -304,7 +304,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     tmem_alloc_pair(&sm.tmem_base, 512);
     tmem_relinquish_pair();
   }
-  if (threadIdx.x < R / 2) sm.inv_freq[threadIdx.x] = rope_inv_freq(RopeCfg<FULL>::theta, threadIdx.x, R);
+  if (threadIdx.x < R / 2) sm.inv_freq[threadIdx.x] = rope_inv_freq<FULL>(threadIdx.x);
   tc_fence_before();
   cluster_sync();   // barriers of both CTAs initialised before any cross-CTA arrive
   tc_fence_after();

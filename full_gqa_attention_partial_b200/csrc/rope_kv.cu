@@ -92,8 +92,10 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
   constexpr int R = RopeCfg<FULL>::R;
   __shared__ double inv_freq[R / 2];
   __shared__ float2 cs[R / 2];
-  for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq(RopeCfg<FULL>::theta, i, R);
+  for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq<FULL>(i);
   __syncthreads();
+  pdl_wait();   // earlier kernels write the keys, values and the cache state read below
+  pdl_launch_dependents();
 
   const int n_tok = a.T - a.t_first;
   const int lane32 = threadIdx.x & 31;
@@ -306,7 +308,7 @@ __global__ void __launch_bounds__(128) rope_q_kernel(const __nv_bfloat16* src, i
   constexpr int R = RopeCfg<FULL>::R;
   __shared__ double inv_freq[R / 2];
   __shared__ float2 cs[R / 2];
-  for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq(RopeCfg<FULL>::theta, i, R);
+  for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq<FULL>(i);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int d0 = lane * 8;
   constexpr int xor_mask = (R == 256) ? 16 : 4;
@@ -362,7 +364,7 @@ __global__ void __launch_bounds__(256) rope_table_kernel(const int32_t* pos, con
                                                          float2* tab) {
   constexpr int R = RopeCfg<FULL>::R;
   __shared__ double inv_freq[R / 2];
-  for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq(RopeCfg<FULL>::theta, i, R);
+  for (int i = threadIdx.x; i < R / 2; i += blockDim.x) inv_freq[i] = rope_inv_freq<FULL>(i);
   __syncthreads();
   const int64_t n = (int64_t)M * (R / 2);
   for (int64_t idx = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; idx < n; idx += (int64_t)gridDim.x * blockDim.x) {
@@ -429,12 +431,10 @@ cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st
   a.commit = h.commit;
   a.capacity = h.capacity;
   const int grid = h.commit ? h.B : rope_grid(h.B * (h.T - h.t_first));
-  if (full)
-    rope_store_kernel<true><<<grid, 128, 0, st>>>(a);
-  else
-    rope_store_kernel<false><<<grid, 128, 0, st>>>(a);
+  cudaError_t e = full ? launch_pdl(rope_store_kernel<true>, dim3(grid, 1, 1), dim3(128, 1, 1), 0, st, 0u, a)
+                       : launch_pdl(rope_store_kernel<false>, dim3(grid, 1, 1), dim3(128, 1, 1), 0, st, 0u, a);
   count_launch();
-  return cudaGetLastError();
+  return e;
 }
 
 cudaError_t launch_ring_gather(const void* rk, const void* rv, const float* rks, const float* rvs,
