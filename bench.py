@@ -99,9 +99,9 @@ def layer_seed(base: int, i: int) -> int:
 # capture of the kernel as it was when its sources hashed to `sha`.  Reported as
 # roofline.traffic only while the sources are unchanged; otherwise null.
 TRAFFIC = {
-    "prefill_full_T32768": {"bytes": 2.2349e9, "sha": "f91bf38ce1984b49",
+    "prefill_full_T32768": {"bytes": 2.0848e9, "sha": "7418b33196f3016d",
                             "sources": ["prefill.cu", "common.cuh"]},
-    "prefill_sliding_T32768": {"bytes": 0.6375e9, "sha": "f91bf38ce1984b49",
+    "prefill_sliding_T32768": {"bytes": 0.6417e9, "sha": "7418b33196f3016d",
                                "sources": ["prefill.cu", "common.cuh"]},
     # captured at 16 x 32768 tokens; decode streams each cached byte once, so
     # traffic scales with the tokens: x 8590491648 / 2147483648

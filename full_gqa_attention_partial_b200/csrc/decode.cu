@@ -602,21 +602,24 @@ int decode_num_splits(bool full, int B, int64_t max_len, bool fp8) {
   // full layers: >= 8 stages of 64 keys per split; a 512-slot ring may go down to one
   // stage per split, so that a small batch still spreads its rings over the SMs
   const int64_t s_max = full ? (keys / 512 > 1 ? keys / 512 : 1) : kWindow / kDecKeys;
-  // whole waves of CTA slots: one bf16 CTA per SM, two FP8 CTAs
+  // whole waves of CTA slots (one bf16 CTA per SM, two FP8 CTAs): the smallest split
+  // count that fills its waves exactly, else the smallest within 5 % of that, else
+  // the best fill
   const int sms = fp8 ? 2 * 148 : 148;
-  int best = 1;
+  int best = 1, first95 = 0;
   double best_eff = 0.0;
   for (int64_t s = 1; s <= s_max && s <= 1024; ++s) {
     const int64_t ctas = pairs * s;
     const int64_t waves = (ctas + sms - 1) / sms;
     const double eff = (double)ctas / (double)(waves * sms);
-    if (eff >= 0.95) return (int)s;
+    if (eff >= 0.999) return (int)s;
+    if (eff >= 0.95 && first95 == 0) first95 = (int)s;
     if (eff > best_eff + 1e-9) {
       best_eff = eff;
       best = (int)s;
     }
   }
-  return best;
+  return first95 ? first95 : best;
 }
 
 cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
