@@ -23,7 +23,8 @@ The JSON line also carries:
                 over e4m3 caches);
   decode_1m_sharded (by default with several ranks, else --decode-sharded) the same with the full
                 layers' history spread over the ranks;
-  chunked_prefill 262144 tokens in 8192-token chunks, 36 layers (these two
+  chunked_prefill 262144 tokens in 8192-token chunks, 36 layers (and
+                chunked_prefill_fp8 over e4m3 caches; these and the 1M decode
                 are skipped with --quick);
   cpu_baseline  the fp64 oracle on a bounded sample of the same workload.
 
@@ -684,8 +685,9 @@ def bench_decode_1m_sharded(hyb, args, peaks, d):
             "frac_of_hbm_per_gpu": kv / (ms / 1e3) / 1e9 / HBM_READ_GBS / d.world}
 
 
-def bench_chunked(hyb, args, peaks):
-    """262144 tokens in 8192-token chunks through all 36 layers (9 full, 27 sliding), batch 1.
+def bench_chunked(hyb, args, peaks, fp8: bool = False):
+    """262144 tokens in 8192-token chunks through all 36 layers (9 full, 27 sliding), batch 1
+    (fp8: every cache in e4m3, the full layers read in place by the attention kernel).
 
     Each chunk is appended to its layer's cache and attends over the cached
     context.  The 32 chunk inputs (seed 4 + c) are shared by the layers: the
@@ -695,9 +697,10 @@ def bench_chunked(hyb, args, peaks):
     total, C = 262144, 8192
     n_chunks = total // C
     xs = [synth.prefill_inputs(1, C, seed=4 + c, device="cuda", start=c * C) for c in range(n_chunks)]
-    fulls = [hyb.KVCache(FULL, 1, capacity=total) for _ in range(9)]
-    rings = [hyb.KVCache(SLIDING, 1) for _ in range(27)]
-    ws = hyb.alloc_workspace(hyb.hyb_attn_prefill_workspace_size(SLIDING, 1, C, True))
+    kvd = hyb.KV_FP8 if fp8 else hyb.KV_BF16
+    fulls = [hyb.KVCache(FULL, 1, capacity=total, kv_dtype=kvd) for _ in range(9)]
+    rings = [hyb.KVCache(SLIDING, 1, kv_dtype=kvd) for _ in range(27)]
+    ws = hyb.alloc_workspace(max(hyb.hyb_attn_prefill_cache_workspace_size(c, C) for c in (fulls[0], rings[0])))
     out = torch.empty(1, C, H, D, dtype=torch.bfloat16, device="cuda")
     work = 9 * flops(total, FULL) + 27 * flops(total, SLIDING)
     torch.cuda.synchronize()
@@ -720,7 +723,8 @@ def bench_chunked(hyb, args, peaks):
     ms = ev0.elapsed_time(ev1)
     rate = work / (ms / 1e3) / 1e12
     # a run of seconds under the power cap: compared with the sustained (seconds-long) figure
-    return {"workload": "262144 tokens in 8192-token chunks, 36 layers, B=1", "pflop": work / 1e15, "ms": ms,
+    return {"workload": "262144 tokens in 8192-token chunks, 36 layers, B=1" + (", FP8 caches" if fp8 else ""),
+            "workspace_bytes": int(ws.numel()), "pflop": work / 1e15, "ms": ms,
             "tflops": rate, "frac_of_peak": rate / peaks["bf16_tflops_sustained"],
             "peak_source": "sustained", "frac_of_burst_peak": rate / peaks["bf16_tflops"],
             "prefill_tokens_per_s": total / (ms / 1e3)}
@@ -933,6 +937,8 @@ def main():
             extras["decode_1m_fp8"] = run("decode_1m_fp8", bench_decode_1m, hyb, args, peaks, fp8=True)
         if args.chunked:
             extras["chunked_prefill"] = run("chunked_prefill", bench_chunked, hyb, args, peaks)
+            torch.cuda.empty_cache()
+            extras["chunked_prefill_fp8"] = run("chunked_prefill_fp8", bench_chunked, hyb, args, peaks, fp8=True)
     # with several ranks the sequence-sharded 1M decode runs by default (every rank
     # takes part: it has collectives)
     if (args.decode_sharded or dist.world > 1) and not args.no_extras:

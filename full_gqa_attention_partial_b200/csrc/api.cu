@@ -502,15 +502,10 @@ size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T,
 }
 
 namespace {
-// bf16 copy of one of K / V of an FP8 full-layer cache, whole capacity
-size_t fp8_copy_bytes(const hyb_kv_cache* c) {
-  return ((size_t)c->batch * kHkv * (size_t)c->capacity * kD * 2 + 255) & ~(size_t)255;
-}
-
-// Scratch of a prefill with cache `c` (NULL: standalone).  An FP8 full-layer
-// cache is attended through bf16 copies of its K and V.  rot_q: as attn_ws.
+// Scratch of a prefill with cache `c` (NULL: standalone): full layers read
+// their cache in place, bf16 or FP8 (the attention kernel widens the codes
+// itself).  rot_q: as attn_ws.
 size_t prefill_ws(int32_t layer_type, int32_t B, int32_t T, const hyb_kv_cache* c, bool rot_q) {
-  if (c && c->type == HYB_FULL && c->kv_dtype == HYB_KV_FP8) return 2 * fp8_copy_bytes(c);
   return attn_ws(layer_type, B, T, c != nullptr, rot_q);
 }
 }  // namespace
@@ -619,51 +614,10 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
   }
 
   const bool fp8 = cache->kv_dtype == HYB_KV_FP8;
-  if (full && fp8) {
-    // the chunk goes into the cache (quantized) and, at full precision, into
-    // bf16 copies of K and V whose rows [0, len) are the stored history
-    // dequantized; attend over the copies' [0, len + T), then advance len
-    uint8_t* wk = reinterpret_cast<uint8_t*>(workspace);
-    uint8_t* wv = wk + fp8_copy_bytes(cache);
-    const int64_t cap = cache->capacity;
-    r.v = v;
-    r.dk = cache->k;
-    r.dv = cache->v;
-    r.dst_rows = cap;
-    r.mode = 0;
-    r.len = cache->len;
-    r.pm = page_map(cache);
-    r.fp8 = 1;
-    r.dks = cache->k_scale;
-    r.dvs = cache->v_scale;
-    if ((e = launch_rope_store(true, r, st)) != cudaSuccess) return cuda_fail(e, "append launch");
-    RopeStoreHost c2 = r;   // the chunk into the bf16 copies
-    c2.dk = wk;
-    c2.dv = wv;
-    c2.fp8 = 0;
-    c2.dks = c2.dvs = nullptr;
-    c2.pm = PageMap();
-    if ((e = launch_rope_store(true, c2, st)) != cudaSuccess) return cuda_fail(e, "chunk copy launch");
-    if ((e = launch_dequant_rows(cache->k, cache->v, cache->k_scale, cache->v_scale, page_map(cache), cap,
-                                 cache->len, T, B, wk, wv, cap, st)) != cudaSuccess)
-      return cuda_fail(e, "history dequantize launch");
-    const uint64_t hb = (uint64_t)cap * row_bytes;
-    if ((s = make_kv_map(&ph.tm_k, wk, (uint64_t)cap, B, row_bytes, hb, hb * kHkv, prefill_k_box_rows(),
-                         "FP8 history K")) != HYB_OK)
-      return s;
-    if ((s = make_kv_map(&ph.tm_v, wv, (uint64_t)cap, B, row_bytes, hb, hb * kHkv, prefill_v_box_rows(),
-                         "FP8 history V")) != HYB_OK)
-      return s;
-    ph.qbase = cache->len;
-    ph.ctx_mode = 0;
-    if ((e = launch_prefill(true, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
-    if ((e = launch_kv_commit(cache->len, cache->head, cache->capacity, false, B, T, st)) != cudaSuccess)
-      return cuda_fail(e, "commit launch");
-    return HYB_OK;
-  }
-
   if (full) {
-    // append first (rows len .. len+T-1), attend over [0, len+T), then advance len
+    // append first (rows len .. len+T-1), attend over [0, len+T), then advance len.
+    // FP8 caches: the chunk goes in quantized and, like a decode step, attends to
+    // its own tokens as the cache stores them
     r.v = v;
     r.dk = cache->k;
     r.dv = cache->v;
@@ -671,8 +625,16 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
     r.mode = 0;
     r.len = cache->len;
     r.pm = page_map(cache);
+    r.fp8 = fp8 ? 1 : 0;
+    r.dks = cache->k_scale;
+    r.dvs = cache->v_scale;
     if ((e = launch_rope_store(true, r, st)) != cudaSuccess) return cuda_fail(e, "append launch");
-    if ((s = cache_maps(cache, &ph.tm_k, &ph.tm_v, prefill_k_box_rows(), prefill_v_box_rows())) != HYB_OK) return s;
+    if (fp8) {
+      if ((s = cache_maps_fp8(cache, &ph.tm_k, &ph.tm_v, &ph.tm_ks, &ph.tm_vs)) != HYB_OK) return s;
+      ph.fp8 = 1;
+    } else if ((s = cache_maps(cache, &ph.tm_k, &ph.tm_v, prefill_k_box_rows(), prefill_v_box_rows())) != HYB_OK) {
+      return s;
+    }
     ph.pm = page_map(cache);
     ph.qbase = cache->len;
     ph.ctx_mode = 0;
@@ -698,6 +660,7 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
   r.dst_row_offset = kWindow - 1;
   r.mode = 2;
   r.len = cache->len;  // default positions: len + t
+  r.qdq = fp8 ? 1 : 0;  // FP8 ring: the chunk's rows as the ring will store them
   if ((e = launch_rope_store(false, r, st)) != cudaSuccess) return cuda_fail(e, "context rope launch");
   const uint64_t hb = (uint64_t)rows * row_bytes;
   if ((s = make_kv_map(&ph.tm_k, ck, rows, B, row_bytes, hb, hb * kHkv, prefill_k_box_rows(), "context K")) != HYB_OK)
@@ -708,13 +671,24 @@ hyb_status prefill_impl(const void* q, const void* k, const void* v, const void*
   ph.ctx_mode = 1;
   if ((e = launch_prefill(false, ph, st)) != cudaSuccess) return cuda_fail(e, "prefill launch");
 
-  RopeStoreHost w;  // ring append from the context rows (already rotated)
-  w.k = reinterpret_cast<const uint8_t*>(ck) + (size_t)(kWindow - 1) * row_bytes;
-  w.v = reinterpret_cast<const uint8_t*>(cv) + (size_t)(kWindow - 1) * row_bytes;
-  w.src_bstride = (int64_t)kHkv * (int64_t)rows * kD;
-  w.src_tstride = kD;
-  w.src_hstride = (int64_t)rows * kD;
-  w.src_rotated = 1;
+  RopeStoreHost w;  // ring append: bf16 from the context rows (already rotated); FP8
+                    // quantizes the rotated raw keys, as the context rows were made
+  if (fp8) {
+    w.k = k;
+    w.v = v;
+    w.src_bstride = (int64_t)T * kv_row_stride;
+    w.src_tstride = kv_row_stride;
+    w.src_hstride = kD;
+    w.src_rotated = qk_rotated ? 1 : 0;
+    w.pos = pos;
+  } else {
+    w.k = reinterpret_cast<const uint8_t*>(ck) + (size_t)(kWindow - 1) * row_bytes;
+    w.v = reinterpret_cast<const uint8_t*>(cv) + (size_t)(kWindow - 1) * row_bytes;
+    w.src_bstride = (int64_t)kHkv * (int64_t)rows * kD;
+    w.src_tstride = kD;
+    w.src_hstride = (int64_t)rows * kD;
+    w.src_rotated = 1;
+  }
   w.dk = cache->k;
   w.dv = cache->v;
   w.dst_rows = kWindow;

@@ -219,6 +219,18 @@ __device__ __forceinline__ uint32_t e4m3_b02_bf16x2(uint32_t w) {
 __device__ __forceinline__ uint32_t e4m3_b13_bf16x2(uint32_t w) {
   return (w & 0x80008000u) | ((w >> 4) & 0x07F007F0u);
 }
+// Two floats -> two e4m3 codes (lo in the low byte), round to nearest even, saturating.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
+  uint16_t h;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(hi), "f"(lo));
+  return h;
+}
+// Two e4m3 codes (low byte first) -> their values (exact).
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t c) {
+  uint32_t d;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)c));
+  return __half22float2(*reinterpret_cast<const __half2*>(&d));
+}
 __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   uint32_t d;
   asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
@@ -368,6 +380,18 @@ __device__ __forceinline__ void mma_ss_pair_warp(uint32_t d_tmem, uint64_t a_des
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// As mma_ss_pair_warp on e4m3 operands (kind::f8f6f4, 32 elements of K per MMA:
+// in a 128-byte-swizzled K-major operand the same 32 bytes per step as bf16's 16).
+__device__ __forceinline__ void mma_ss_pair_e4m3_warp(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc,
+                                                      uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Orders this thread's earlier memory writes before its later ones for every
 // thread of the cluster.
 __device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }
@@ -405,6 +429,11 @@ __device__ __forceinline__ void mma_commit(uint64_t* bar) {
                : "memory");
 }
 
+// Instruction descriptor, kind::f8f6f4: e4m3 A and B (format 0), fp32 D, dense
+// (the bit fields of the kind::f16 descriptor below).
+__host__ __device__ constexpr uint32_t idesc_e4m3(int M, int N, bool b_mn_major) {
+  return (1u << 4) | ((b_mn_major ? 1u : 0u) << 16) | ((uint32_t)(N >> 3) << 17) | ((uint32_t)(M >> 4) << 24);
+}
 // Instruction descriptor, kind::f16: bf16 A/B, fp32 D, dense.
 //   bits 4-5 D format (1 = f32), 7-9 A format (1 = bf16), 10-12 B format,
 //   15 A major (0 = K), 16 B major (1 = MN), 17-22 N >> 3, 24-28 M >> 4.

@@ -73,6 +73,7 @@ struct RopeStoreHost {
   float* dvs = nullptr;
   PageMap pm;                  // linear mode: paged destination cache
   int commit = 0;              // 1: advance len / head in the same launch (one block per sequence)
+  int qdq = 0;                 // rows mode: write each bf16 row as its e4m3 quantization dequantized
   int64_t capacity = 0;        // commit, linear mode: cache capacity
 };
 cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st);
@@ -80,11 +81,6 @@ cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st
 cudaError_t launch_ring_gather(const void* rk, const void* rv, const float* rks, const float* rvs,
                                const int32_t* len, const int32_t* head, const int32_t* tag, void* ck, void* cv,
                                int64_t ctx_rows, int B, cudaStream_t st);
-// bf16 [B][4][dst_rows][256] copies of rows [0, len[b]) of an FP8 full-layer cache,
-// rows [len + T, end of their 64-row tile) zero-filled
-cudaError_t launch_dequant_rows(const void* kc, const void* vc, const float* ks, const float* vs, const PageMap& pm,
-                                int64_t cap, const int32_t* len, int T, int B, void* dk, void* dv, int64_t dst_rows,
-                                cudaStream_t st);
 cudaError_t launch_kv_commit(int32_t* len, int32_t* head, int64_t capacity, bool ring, int B, int T,
                              cudaStream_t st);
 cudaError_t launch_selftest_wait(cudaStream_t st);
@@ -120,6 +116,9 @@ int gemm_box_k();      // K elements per TMA box
 // ---- prefill attention (prefill.cu) -----------------------------------------
 struct PrefillHost {
   CUtensorMap tm_k, tm_v;      // 4-D maps {256, rows, 4, B}, 64-dim boxes, 128B swizzle
+                               // (fp8: uint8 maps of the cache's codes, 128-code boxes)
+  CUtensorMap tm_ks, tm_vs;    // fp8: 3-D maps over the row scales {rows, 4, B}, 64-row boxes
+  int fp8 = 0;                 // 1: a full layer's keys and values come from an FP8 cache
   CUtensorMap tm_q, tm_o;      // 4-D maps {256, 16, T, B} over q and out, 64-dim x 128-row boxes
   const void* q = nullptr;     // raw queries
   int64_t q_stride = 0;        // elements between tokens

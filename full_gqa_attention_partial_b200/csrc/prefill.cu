@@ -49,6 +49,26 @@
 // Softmax in the log2 domain with a lazily updated base: every probability
 // of a row is 2^(s - base), the base only moves (and O is only rescaled)
 // when a tile's maximum exceeds it by more than 8, so P stays <= 256.
+//
+// FP8 (e4m3) full-layer caches (one fp32 scale per key row and KV head) are
+// read in place.  S = Q K^T runs on the tensor cores' e4m3 path
+// (kind::f8f6f4) straight from the K codes, which TMA loads into four 16 KB
+// entries: the query tile is split into two e4m3 tiles, Q_hi (each element
+// rounded, after a power-of-two factor per row that puts the row's largest
+// element in [128, 256)) and Q_lo (the remainder, rounded), and S is their
+// two MMA passes into one accumulator -- the tensor time of one bf16 pass, and
+// at most 2^-8 of each query element left out (a single e4m3 query tile, at
+// 2^-4, would not meet the accuracy bound).  V feeds O += P V in bf16: its
+// codes land in the upper half of one of two 32 KB V slots and two converter
+// warps (12 warps in all) widen them in place by integer bit moves (value x
+// 2^-120, exact), which give the dims of each group of four in the order 0,
+// 2, 1, 3; the slot keeps that order, so O's columns come in it too and the
+// epilogue puts them back.  The row scales never touch the operands: TMA
+// loads them into a four-tile ring, the softmax multiplies the scores by the
+// K scale and P by the V scale, the query row's factor and the softmax scale
+// come in with the row maximum and the exponent, P carries 2^64 (added in the
+// exponent's FMA, so O stays far from fp32's subnormals) and the epilogue
+// takes back 2^120.
 #include <algorithm>
 #include <cstddef>
 
@@ -60,14 +80,22 @@ namespace hyb {
 constexpr int kBM = 128;                  // query rows per CTA
 constexpr int kBN = 128;                  // keys per tile (shared by the pair)
 constexpr int kHalfKeys = 64;             // keys per TMA box row range (a K half, a V quarter)
-constexpr int kSlots = 4;                 // K/V ring
-constexpr int kSlotBytes = 32768;         // one CTA's half of a K or V tile
+constexpr int kSlotBytes = 32768;         // one CTA's half of a K or V tile (bf16)
 constexpr int kKBox = kHalfKeys * 128;    // K half: 64 keys x 64 dims per box, 8 KB
 constexpr int kVChunk = kBN * 128;        // V: 128 keys x 64 dims (two 64-key boxes), 16 KB
-constexpr int kPfThreads = 320;
 constexpr int kSmWarps = 8;               // softmax warps (two warpgroups)
 constexpr int kProdWarp = 8;
 constexpr int kMmaWarp = 9;
+constexpr int kConvWarp = 10;             // FP8: converter warps 10 and 11
+constexpr int kSlots = 4;                 // operand ring: 4 x 32 KB
+constexpr int kCodeBytes = 16384;         // FP8: one CTA's codes of a K or V tile
+constexpr int kNKc = 4;                   // FP8: K code entries (16 KB) in slots 0-1
+constexpr int kNV = 2;                    // FP8: V slots (slots 2-3), codes land in the upper half
+constexpr int kNF = 4;                    // FP8: K / V row-scale ring (tiles)
+template <bool FP8> struct PfCfg {
+  static constexpr int kThreads = FP8 ? 384 : 320;
+};
+constexpr float kTwo120 = 1.329227995784916e36f;    // 2^120
 constexpr int kNS = 2;                    // S buffers in tensor memory
 constexpr int kAhead = kNS - 1;           // key tiles whose S is issued before the P.V of a tile
 constexpr uint32_t kColO = 256;
@@ -75,10 +103,11 @@ constexpr float kRescaleThreshold = 8.0f;
 constexpr int kStageBytes = 2048;         // epilogue transpose area per softmax warp
 __device__ __forceinline__ uint32_t col_s(uint32_t sb) { return 128u * sb; }
 
-template <bool FULL>
+template <bool FULL, bool FP8>
 struct PfSmem {
   static constexpr int R = RopeCfg<FULL>::R;
-  uint8_t slot[kSlots][kSlotBytes];  // 1024-byte aligned
+  // 1024-byte aligned; FP8: slots 0-1 hold four 16 KB K code entries, slots 2-3 the V tiles
+  uint8_t slot[kSlots][kSlotBytes];
   uint8_t qo[4][16384];              // the query tile (4 boxes of 64 dims x 128 rows), rotated in place:
                                      // the A operand of S = Q K^T
   // full layers: rotation tables for the tile's rows (positions p_base + 16 i + j), rebuilt per item:
@@ -93,7 +122,17 @@ struct PfSmem {
   double inv_freq[R / 2];
   float xmax[2][2][kBM];             // [tile parity][warpgroup][row]: a row's maximum over the warpgroup's keys
   float xsum[2][2][kBM];             // [item parity][warpgroup][row]: running sum at item end
-  uint64_t full[kSlots];   // CTA 0's count both CTAs' bytes
+  // FP8: the row scales of a tile's 128 keys, by tile % kNF
+  alignas(16) float kf[FP8 ? kNF : 1][kBN];
+  alignas(16) float vf[FP8 ? kNF : 1][kBN];
+  uint64_t f_full[kNF];              // FP8: a tile's scales landed (this CTA's copy)
+  uint64_t f_free[kNF];              // FP8: a tile's scales read by every softmax warp
+  uint64_t vcode[kNV];               // FP8: this CTA's V codes of a tile landed in its slot
+  uint64_t vready[kNV];              // FP8, CTA 0: V widened (one arrival per converter warp of the pair)
+  uint64_t vempty[kNV];              // FP8: the V slot's P.V completed
+  uint64_t qx_full[4];               // FP8: a query row's largest |element| over each warpgroup's
+                                     //   dims (in xsum[item parity]) of lane quarter q written by both warps
+  uint64_t full[kSlots];   // CTA 0's count both CTAs' bytes (bf16 slots; FP8 K code entries)
   uint64_t empty[kSlots];  // per CTA, committed by the MMA issuer
   uint64_t q_ready;        // CTA 0: query tile rotated (one arrival per softmax warp of the pair) or
                            //   landed (one arrival per CTA from its query producer)
@@ -111,12 +150,19 @@ struct PfSmem {
   uint32_t tmem_base;
 };
 
-template <bool FULL>
-size_t prefill_smem_bytes_t() { return sizeof(PfSmem<FULL>) + 1024; }
-size_t prefill_smem_bytes() { return std::max(prefill_smem_bytes_t<true>(), prefill_smem_bytes_t<false>()); }
-static_assert(sizeof(PfSmem<true>) + 1024 <= 232448 && sizeof(PfSmem<false>) + 1024 <= 232448,
+template <bool FULL, bool FP8 = false>
+size_t prefill_smem_bytes_t() { return sizeof(PfSmem<FULL, FP8>) + 1024; }
+size_t prefill_smem_bytes() {
+  return std::max({prefill_smem_bytes_t<true>(), prefill_smem_bytes_t<false>(), prefill_smem_bytes_t<true, true>()});
+}
+static_assert(sizeof(PfSmem<true, false>) + 1024 <= 232448 && sizeof(PfSmem<false, false>) + 1024 <= 232448 &&
+                  sizeof(PfSmem<true, true>) + 1024 <= 232448,
               "prefill shared memory exceeds 227 KB");
-static_assert(offsetof(PfSmem<true>, ostage) % 1024 == 0 && offsetof(PfSmem<false>, ostage) % 1024 == 0,
+using PfSmemFull = PfSmem<true, false>;
+using PfSmemSliding = PfSmem<false, false>;
+using PfSmemFullFp8 = PfSmem<true, true>;
+static_assert(offsetof(PfSmemFull, ostage) % 1024 == 0 && offsetof(PfSmemSliding, ostage) % 1024 == 0 &&
+                  offsetof(PfSmemFullFp8, ostage) % 1024 == 0,
               "staging areas must start on a swizzle period");
 
 struct PfArgs {
@@ -260,15 +306,16 @@ __device__ __forceinline__ int item_index(int k, int pair, int n_pairs, int n_it
 // Barrier phases run on across items: K/V loads by a global load counter,
 // S / P buffers and the maximum exchange by a global tile counter, query /
 // output / sum-exchange barriers by the item counter.
-template <bool FULL>
 // Warps are dealt round-robin to the SM's four sub-partitions (16,384
-// registers each): with 10 warps two sub-partitions hold three, so a thread
-// may use at most 168 registers.
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
+// registers each): with 10 (12 for FP8) warps a sub-partition holds three,
+// so a thread may use at most 168 registers.
+template <bool FULL, bool FP8>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
-                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o, PfArgs a) {
+                   const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
+                   const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs, PfArgs a) {
   extern __shared__ uint8_t smem_raw[];
-  using Smem = PfSmem<FULL>;
+  using Smem = PfSmem<FULL, FP8>;
   Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   constexpr int R = RopeCfg<FULL>::R;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -282,7 +329,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       mbar_init(&sm.full[s], 1);
       mbar_init(&sm.empty[s], 1);
     }
-    mbar_init(&sm.q_ready, a.q_rotated ? 2 : 2 * kSmWarps);
+    if (FP8) {
+      for (int p = 0; p < kNV; ++p) {
+        mbar_init(&sm.vcode[p], 1);
+        mbar_init(&sm.vready[p], 4);
+        mbar_init(&sm.vempty[p], 1);
+      }
+      for (int p = 0; p < kNF; ++p) {
+        mbar_init(&sm.f_full[p], 1);
+        mbar_init(&sm.f_free[p], kSmWarps);
+      }
+      for (int q = 0; q < 4; ++q) mbar_init(&sm.qx_full[q], 2);
+    }
+    mbar_init(&sm.q_ready, (a.q_rotated && !FP8) ? 2 : 2 * kSmWarps);
     for (int s = 0; s < kNS; ++s) {
       mbar_init(&sm.s_full[s], 1);
       mbar_init(&sm.p_full[s], 2 * kSmWarps);
@@ -315,7 +374,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       // ======================= K/V producer (both CTAs) =======================
       prefetch_tmap(&tm_k);
       prefetch_tmap(&tm_v);
-      uint32_t g = 0;   // loads issued so far by this CTA
+      if (FP8) {
+        prefetch_tmap(&tm_ks);
+        prefetch_tmap(&tm_vs);
+      }
+      uint32_t g = 0;   // loads issued so far by this CTA (bf16)
+      uint32_t J = 0;   // tiles of earlier items (FP8 loads are numbered by tile)
+      uint32_t nk = 0, nf = 0, nv = 0;   // FP8: K code, scale and V loads issued (tile index + 1)
       bool ok = true;
       for (int k = 0; ok; ++k) {
         const int w = item_index(k, pair0, n_pairs, n_items);
@@ -340,12 +405,52 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             const bool is_k = part == 0;
             const int tile = is_k ? st : st - kAhead;
             if (tile < 0 || tile >= it.n) continue;
+            const int r0 = (it.j_lo + tile) * kBN;   // key row of the tile's first key
+            int row, page;
+            if constexpr (FP8) {
+              const uint32_t jt = J + tile;
+              if (is_k) {
+                // this CTA's 64 keys (codes, dims [0, 128) and [128, 256)) into K entry
+                // jt % 4, bytes counted on CTA 0's barrier; then the row scales of all
+                // 128 keys (every softmax row needs them) into this CTA's scale ring
+                const int e = jt % kNKc;
+                if (jt >= kNKc && !(ok = mbar_wait(&sm.empty[e], ((jt / kNKc) - 1) & 1))) break;
+                if (rank == 0) mbar_arrive_expect_tx(&sm.full[e], 2 * kCodeBytes);
+                const uint32_t dst = smem_u32(sm.slot[0]) + e * kCodeBytes;
+                coord(r0 + kHalfKeys * (int)rank, row, page);
+#pragma unroll
+                for (int c = 0; c < 2; ++c) tma_load_4d_pair(dst + c * 8192, &tm_k, &sm.full[e], 128 * c, row, it.kvh, page);
+                nk = jt + 1;
+                const int fe = jt % kNF;
+                if (jt >= kNF && !(ok = mbar_wait(&sm.f_free[fe], ((jt / kNF) - 1) & 1))) break;
+                mbar_arrive_expect_tx(&sm.f_full[fe], 2 * kBN * 4);
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  coord(r0 + kHalfKeys * h, row, page);
+                  tma_load_3d(smem_u32(&sm.kf[fe][kHalfKeys * h]), &tm_ks, &sm.f_full[fe], row, it.kvh, page);
+                  tma_load_3d(smem_u32(&sm.vf[fe][kHalfKeys * h]), &tm_vs, &sm.f_full[fe], row, it.kvh, page);
+                }
+                nf = jt + 1;
+              } else {
+                // the tile's 128 keys of this CTA's 128 dims (codes) into the upper half of
+                // V slot jt % 2, once the slot's last P.V has completed
+                const int v = jt % kNV;
+                if (jt >= kNV && !(ok = mbar_wait(&sm.vempty[v], ((jt / kNV) - 1) & 1))) break;
+                mbar_arrive_expect_tx(&sm.vcode[v], kCodeBytes);
+                const uint32_t dst = smem_u32(sm.slot[2 + v]) + kCodeBytes;
+#pragma unroll
+                for (int h = 0; h < 2; ++h) {
+                  coord(r0 + kHalfKeys * h, row, page);
+                  tma_load_4d(dst + h * 8192, &tm_v, &sm.vcode[v], 128 * (int)rank, row, it.kvh, page);
+                }
+                nv = jt + 1;
+              }
+              continue;
+            }
             const int slot = g % kSlots;
             if (g >= kSlots && !(ok = mbar_wait(&sm.empty[slot], ((g / kSlots) - 1) & 1))) break;
             if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
             const uint32_t dst = smem_u32(sm.slot[slot]);
-            const int r0 = (it.j_lo + tile) * kBN;   // key row of the tile's first key
-            int row, page;
             if (is_k) {   // this CTA's 64 keys, 4 boxes of 64 dims
               coord(r0 + kHalfKeys * (int)rank, row, page);
 #pragma unroll
@@ -364,9 +469,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             ++g;
           }
         }
+        J += it.n;
       }
-      if (rank == 0)  // every load of the pair completes on CTA 0's barriers
+      // no copy left landing in shared memory at exit (the pair's loads complete on
+      // CTA 0's barriers)
+      if constexpr (FP8) {
+        for (uint32_t i = (nv > kNV ? nv - kNV : 0); i < nv; ++i) mbar_wait(&sm.vcode[i % kNV], (i / kNV) & 1);
+        for (uint32_t i = (nf > kNF ? nf - kNF : 0); i < nf; ++i) mbar_wait(&sm.f_full[i % kNF], (i / kNF) & 1);
+        if (rank == 0)
+          for (uint32_t i = (nk > kNKc ? nk - kNKc : 0); i < nk; ++i) mbar_wait(&sm.full[i % kNKc], (i / kNKc) & 1);
+      } else if (rank == 0) {
         for (uint32_t i = (g > kSlots ? g - kSlots : 0); i < g; ++i) mbar_wait(&sm.full[i % kSlots], (i / kSlots) & 1);
+      }
     } else if (lane == 1) {
       // ======================= query-tile producer (both CTAs) =======================
       prefetch_tmap(&tm_q);
@@ -390,7 +504,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
 #pragma unroll
           for (int box = 0; box < 4; ++box) tma_prefetch_l2_4d(&tm_q, box * 64, nx.h_pair0 + (int)rank, nx.m0, nx.b);
         }
-        if (a.q_rotated) {   // nothing to rotate: the tile is ready once it has landed
+        if (a.q_rotated && !FP8) {   // nothing to rotate or permute: the tile is ready once it has landed
           if (!(ok = mbar_wait(&sm.q_full, item & 1))) break;
           if (rank == 0) mbar_arrive(&sm.q_ready);
           else mbar_arrive_remote(&sm.q_ready, 0);
@@ -400,10 +514,76 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       }
       if (item > 0) mbar_wait(&sm.q_full, (item - 1) & 1);   // no copy left landing at exit
     }
+  } else if (FP8 && warp >= kConvWarp) {
+    // ======================= FP8 converters (warps 10, 11; both CTAs) =======================
+    // V codes -> bf16 in place, tile by tile: the 128 keys x 128 codes of this
+    // CTA's dims sit in the upper half of the V slot (two 64-key boxes, 128-byte
+    // swizzle) and become the two 16 KB chunks of 64 dims x 128 keys the P.V
+    // MMAs read.  One item is 16 codes (16 dims) of one key: the 8 lanes of a
+    // quarter-warp read one 128-byte row (conflict-free under the swizzle) and
+    // write its 16 bf16 dims as two 16-byte chunks, lanes 4-7 in the other order
+    // so that the 8 lanes' chunks fall in 8 bank groups.  A thread's output in
+    // the upper half (dims 64-127) lands on the code row it read from, which
+    // only lanes of its own warp read: each warp reads all its codes, then
+    // writes, with no wait on the other warp.
+    const int ct = (warp - kConvWarp) * 32 + lane;   // 0..63
+    // item i of this thread: key 4 i + rq of source box sb, 16 codes q; (4 i) & 7
+    // alternates between 0 and 4, so the swizzled chunk indexes take two values
+    const int q = ct & 7, sb = (ct >> 3) & 1, rq = ct >> 4;
+    const int sx0 = (q ^ rq) << 4, sx1 = (q ^ (rq + 4)) << 4;
+    const int c0 = 2 * (q & 3);
+    // lanes 4-7 of a quarter-warp store their two chunks in the other order
+    const int ca = (q < 4) ? c0 : c0 + 1, cb = (q < 4) ? c0 + 1 : c0;
+    const int da0 = (ca ^ rq) << 4, db0 = (cb ^ rq) << 4, da1 = (ca ^ (rq + 4)) << 4, db1 = (cb ^ (rq + 4)) << 4;
+    uint32_t J = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int w = item_index(k, pair0, n_pairs, n_items);
+      if (w == -2) break;
+      if (w < 0) continue;
+      const Item it = item_of<FULL>(w, a);
+      for (int tile = 0; ok && tile < it.n; ++tile) {
+        const uint32_t jt = J + tile;
+        const int v = jt % kNV;
+        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.vcode[v], (jt / kNV) & 1)))) break;
+        uint8_t* dst = sm.slot[2 + v];
+        const uint8_t* sp = dst + kCodeBytes + sb * 8192 + rq * 128;
+        uint4 cw[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) cw[i] = *reinterpret_cast<const uint4*>(sp + i * 512 + ((i & 1) ? sx1 : sx0));
+        __syncwarp();   // every lane's codes read before any lane overwrites them
+        // 64-dim chunk q / 4, key 64 sb + 4 i + rq
+        uint8_t* dp = dst + (q >> 2) * 16384 + (64 * sb + rq) * 128;
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const uint32_t wv[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
+          uint32_t o[8];   // the dims of each group of four in the order 0, 2, 1, 3
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {
+            o[2 * j] = e4m3_b02_bf16x2(wv[j]);
+            o[2 * j + 1] = e4m3_b13_bf16x2(wv[j]);
+          }
+          const uint4 lo = make_uint4(o[0], o[1], o[2], o[3]), hi = make_uint4(o[4], o[5], o[6], o[7]);
+          const uint4 va = (q < 4) ? lo : hi, vb = (q < 4) ? hi : lo;
+          uint8_t* rowp = dp + i * 512;
+          *reinterpret_cast<uint4*>(rowp + ((i & 1) ? da1 : da0)) = va;
+          *reinterpret_cast<uint4*>(rowp + ((i & 1) ? db1 : db0)) = vb;
+        }
+        fence_proxy_async();              // the slot is read by the tensor core
+        if (rank != 0) fence_cluster();   // ... through MMAs issued from CTA 0
+        __syncwarp();
+        if (lane == 0) {
+          if (rank == 0) mbar_arrive(&sm.vready[v]);
+          else mbar_arrive_remote(&sm.vready[v], 0);
+        }
+      }
+      J += it.n;
+    }
   } else if (warp == kMmaWarp) {
     // ======================= MMA issuer (CTA 0, whole warp, one lane issues) =======================
     if (rank == 0) {
-      constexpr uint32_t idesc_s = idesc_bf16(2 * kBM, kBN, false);   // S = Q K^T, B K-major
+      // S = Q K^T, B K-major (FP8 caches: e4m3 operands, kind::f8f6f4)
+      constexpr uint32_t idesc_s = FP8 ? idesc_e4m3(2 * kBM, kBN, false) : idesc_bf16(2 * kBM, kBN, false);
       constexpr uint32_t idesc_o = idesc_bf16(2 * kBM, kD, true);     // O += P V, B MN-major
       const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.qo[0]), 16, 1024);          // Q, K-major
       const uint64_t kdesc0 = smem_desc_sw128(smem_u32(sm.slot[0]), 16, 1024);       // K in slot 0, K-major
@@ -424,18 +604,38 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
             const bool is_k = part == 0;
             const int tile = is_k ? st : st - kAhead;
             if (tile < 0 || tile >= it.n) continue;
-            const int slot = g % kSlots;
-            if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], (g / kSlots) & 1)))) break;
-            tc_fence_after();
             const uint32_t jt = J + tile;   // global tile index
             const uint32_t sb = jt % kNS;
+            // the operand's slot: bf16, the load ring; FP8, K entry jt % 4 or V slot 2 + jt % 2
+            const int slot = !FP8 ? (int)(g % kSlots) : is_k ? (int)(jt % kNKc) : 2 + (int)(jt % kNV);
+            if (FP8 && !is_k) {
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.vready[slot - 2], (jt / kNV) & 1)))) break;
+            } else {
+              const uint32_t ph = FP8 ? (jt / kNKc) & 1 : (g / kSlots) & 1;
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], ph)))) break;
+            }
+            tc_fence_after();
             if (is_k) {
-              const uint64_t kdesc = desc_advance(kdesc0, slot * kSlotBytes);
+              if constexpr (FP8) {
+                // Q_hi K^T then Q_lo K^T into the same accumulator: 32 dims per MMA; the
+                // 128 dims of dim block d are Q_hi in qo[2 d], Q_lo in qo[2 d + 1], and
+                // codes [128 d, 128 d + 128) of the K entry's 64 keys in its box d
+                const uint64_t kdesc = desc_advance(kdesc0, slot * kCodeBytes);
 #pragma unroll
-              for (int s = 0; s < kD / 16; ++s) {
-                const uint64_t adesc = desc_advance(qdesc, (s >> 2) * 16384 + (s & 3) * 32);
-                const uint64_t bdesc = desc_advance(kdesc, (s >> 2) * kKBox + (s & 3) * 32);
-                mma_ss_pair_warp(tmem + col_s(sb), adesc, bdesc, idesc_s, s > 0 ? 1u : 0u);
+                for (int s = 0; s < 2 * kD / 32; ++s) {
+                  const int s2 = s & 7;
+                  const uint64_t adesc = desc_advance(qdesc, (s2 >> 2) * 32768 + (s >> 3) * 16384 + (s2 & 3) * 32);
+                  const uint64_t bdesc = desc_advance(kdesc, (s2 >> 2) * 8192 + (s2 & 3) * 32);
+                  mma_ss_pair_e4m3_warp(tmem + col_s(sb), adesc, bdesc, idesc_s, s > 0 ? 1u : 0u);
+                }
+              } else {
+                const uint64_t kdesc = desc_advance(kdesc0, slot * kSlotBytes);
+#pragma unroll
+                for (int s = 0; s < kD / 16; ++s) {
+                  const uint64_t adesc = desc_advance(qdesc, (s >> 2) * 16384 + (s & 3) * 32);
+                  const uint64_t bdesc = desc_advance(kdesc, (s >> 2) * kKBox + (s & 3) * 32);
+                  mma_ss_pair_warp(tmem + col_s(sb), adesc, bdesc, idesc_s, s > 0 ? 1u : 0u);
+                }
               }
               mma_commit_pair_warp(&sm.empty[slot]);
               mma_commit_pair_warp(&sm.s_full[sb]);
@@ -455,7 +655,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
                 mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 64 * (s >> 2) + 8 * (s & 3), bdesc, idesc_o,
                                  (tile > 0 || s > 0) ? 1u : 0u);
               }
-              mma_commit_pair_warp(&sm.empty[slot]);
+              mma_commit_pair_warp(FP8 ? &sm.vempty[slot - 2] : &sm.empty[slot]);
               mma_commit_pair_warp(&sm.o_done[sb]);
               if (tile == it.n - 1) mma_commit_pair_warp(&sm.o_final);
             }
@@ -491,12 +691,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         else mbar_arrive_remote(bar, 0);
       }
     };
+    float q_row_scale = 1.f;   // FP8: this row's 2^(ex - 7) x the softmax scale (log2) of the last prepared query tile
     // Rotates this warpgroup's half of the frequencies of the query tile of
     // `it` (the item_no-th of this pair) in qo and hands it to the MMA issuer.
     auto prepare_q = [&](const Item& it, int item_no) -> bool {
      if constexpr (!FULL) {
       return false;   // sliding layers: queries always arrive rotated
      } else {
+      if (a.q_rotated) {   // FP8 with rotated queries: only the permutation below
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full, item_no & 1))) return false;
+      } else {
       const int row = it.m0 + r;
       const bool valid = row < a.T;
       const int qseq = it.qb + row;
@@ -558,6 +762,64 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
           }
         }
       }
+      }
+      if constexpr (FP8) {
+        // The row as Q_hi + Q_lo, both e4m3, for the e4m3 keys: every element times
+        // 2^(7 - e), where 2^e <= the row's largest |element| < 2^(e + 1) (found over
+        // both warpgroups' halves of the row), so that the largest lies in [128, 256);
+        // Q_hi is an element rounded to e4m3, Q_lo the remainder rounded to e4m3,
+        // which leaves out at most 2^-8 of the element (bf16 rounding: 2^-9).  This
+        // warpgroup's 16 chunks of 8 dims for the maximum include every dim it rotated.
+        auto chunk_of = [&](int i) { return i < 4 ? 2 * wg + (i & 1) + 4 * (i >> 1) : 8 + 12 * wg + (i - 4); };
+        float am = 0.f;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {
+          const int ci = chunk_of(i);
+          const uint4 v = *reinterpret_cast<const uint4*>(sm.qo[ci >> 3] + sw128_offset((uint32_t)r, (uint32_t)(ci & 7) * 16));
+          const uint32_t wv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+          for (int j = 0; j < 4; ++j) am = fmaxf(am, fmaxf(fabsf(bf16lo(wv[j])), fabsf(bf16hi(wv[j]))));
+        }
+        // xsum of the coming item's parity is free: the other warpgroup read it in the
+        // epilogue before last, and writes it next after reading this value
+        sm.xsum[item_no & 1][wg][r] = am;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&sm.qx_full[qtr]);
+        if (!__all_sync(0xffffffffu, mbar_wait(&sm.qx_full[qtr], item_no & 1))) return false;
+        am = fmaxf(am, sm.xsum[item_no & 1][wg ^ 1][r]);
+        int ex = am > 0.f ? (int)((__float_as_uint(am) >> 23) & 0xFFu) - 127 : 7;   // zero row: factor 1
+        ex = max(ex, -100);                     // a subnormal row is scaled as 2^-100 would be
+        const float down = __uint_as_float((uint32_t)(127 + 7 - ex) << 23);            // 2^(7 - ex)
+        q_row_scale = __uint_as_float((uint32_t)(127 + ex - 7) << 23) * scale_log2;   // 2^(ex - 7), log2 units
+        // this warpgroup's dims [128 wg, 128 wg + 128), bf16 in qo[2 wg] and qo[2 wg + 1],
+        // become Q_hi in qo[2 wg] and Q_lo in qo[2 wg + 1] (16 dims per 16-byte chunk).
+        // Every one is read before any is overwritten; the other warpgroup rotated some
+        // of them, and arrived at the exchange above after that.
+        uint4 x[16];
+#pragma unroll
+        for (int m = 0; m < 16; ++m)
+          x[m] = *reinterpret_cast<const uint4*>(sm.qo[2 * wg + (m >> 3)] + sw128_offset((uint32_t)r, (uint32_t)(m & 7) * 16));
+#pragma unroll
+        for (int c = 0; c < 8; ++c) {
+          const uint32_t wv[8] = {x[2 * c].x, x[2 * c].y, x[2 * c].z, x[2 * c].w,
+                                  x[2 * c + 1].x, x[2 * c + 1].y, x[2 * c + 1].z, x[2 * c + 1].w};
+          uint32_t hw[4], lw[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) {   // dims 4 j .. 4 j + 3 of the chunk
+            const float v0 = bf16lo(wv[2 * j]) * down, v1 = bf16hi(wv[2 * j]) * down;
+            const float v2 = bf16lo(wv[2 * j + 1]) * down, v3 = bf16hi(wv[2 * j + 1]) * down;
+            const uint32_t h01 = f32x2_to_e4m3x2(v0, v1), h23 = f32x2_to_e4m3x2(v2, v3);
+            const float2 b01 = e4m3x2_to_f32x2(h01), b23 = e4m3x2_to_f32x2(h23);
+            const uint32_t l01 = f32x2_to_e4m3x2(v0 - b01.x, v1 - b01.y), l23 = f32x2_to_e4m3x2(v2 - b23.x, v3 - b23.y);
+            hw[j] = h01 | (h23 << 16);
+            lw[j] = l01 | (l23 << 16);
+          }
+          *reinterpret_cast<uint4*>(sm.qo[2 * wg] + sw128_offset((uint32_t)r, (uint32_t)c * 16)) =
+              make_uint4(hw[0], hw[1], hw[2], hw[3]);
+          *reinterpret_cast<uint4*>(sm.qo[2 * wg + 1] + sw128_offset((uint32_t)r, (uint32_t)c * 16)) =
+              make_uint4(lw[0], lw[1], lw[2], lw[3]);
+        }
+      }
       fence_proxy_async();              // qo is read by the tensor core
       if (rank != 0) fence_cluster();   // ... through MMAs issued from CTA 0
       tc_fence_before();                // TMEM accesses so far precede the MMAs q_ready releases
@@ -583,7 +845,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
     int k = 0, item = 0;
     Item it;
     bool have = next_item(k, it);
-    bool ok = !have || a.q_rotated || prepare_q(it, 0);
+    bool ok = !have || (a.q_rotated && !FP8) || prepare_q(it, 0);
+    float rs = q_row_scale;   // the current item's query row factor (FP8)
     while (ok && have) {
       const int h = it.h_pair0 + (int)rank;
       const int row = it.m0 + r;
@@ -607,6 +870,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         float s[64];
 #pragma unroll
         for (int c = 0; c < 64; ++c) s[c] = __uint_as_float(sraw[c]);
+        if constexpr (FP8) {   // x the key row's scale; the query row's factor and the softmax
+                               // scale (rs) come in with the maximum and the exponent
+          if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.f_full[jt % kNF], (jt / kNF) & 1)))) break;
+          const float2* kf2 = reinterpret_cast<const float2*>(&sm.kf[jt % kNF][64 * wg]);
+#pragma unroll
+          for (int c = 0; c < 32; ++c) {
+            const float2 v = fmul2(make_float2(s[2 * c], s[2 * c + 1]), kf2[c]);
+            s[2 * c] = v.x;
+            s[2 * c + 1] = v.y;
+          }
+        }
 
         const int ks0 = it.kb + (it.j_lo + j) * kBN + 64 * wg;   // sequence index of this warpgroup's first key
         const bool whole = ks0 >= 0 && ks0 + 63 <= it.q_lo && (FULL || it.q_hi - ks0 <= kWindow - 1);
@@ -634,21 +908,35 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
         __syncwarp();
         if (lane == 0) mbar_arrive(&sm.xmax_full[jt & 1][qtr]);
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.xmax_full[jt & 1][qtr], (jt >> 1) & 1)))) break;
-        const float m_tile = fmaxf(mx[0], sm.xmax[jt & 1][wg ^ 1][r]) * scale_log2;
+        const float m_tile = fmaxf(mx[0], sm.xmax[jt & 1][wg ^ 1][r]) * (FP8 ? rs : scale_log2);
         const bool rescale = m_tile > b_run + kRescaleThreshold;
         const float b_new = rescale ? m_tile : b_run;
         const float alpha = rescale ? ex2(b_run - b_new) : 1.f;   // b_run = -inf: O and l are 0
 
         const float base = (b_new == -INFINITY) ? 0.f : b_new;
-        const float2 nbase2 = make_float2(-base, -base);
+        // FP8: P x 2^64 (with V's codes widened x 2^-120, O stays far from fp32's subnormals)
+        const float nb = FP8 ? 64.f - base : -base;
+        const float2 nbase2 = make_float2(nb, nb);
+        const float2 rs2 = make_float2(rs, rs);
         uint32_t pw[32];
         float2 ps[4] = {make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f), make_float2(0.f, 0.f)};
+        // FP8: P for the P.V MMA carries the value row's scale too (the sums do not)
+        const float2* vf2 = FP8 ? reinterpret_cast<const float2*>(&sm.vf[jt % kNF][64 * wg]) : nullptr;
 #pragma unroll
         for (int wd = 0; wd < 32; ++wd) {
-          const float2 x = ffma2(make_float2(s[2 * wd], s[2 * wd + 1]), scale2, nbase2);
+          const float2 x = ffma2(make_float2(s[2 * wd], s[2 * wd + 1]), FP8 ? rs2 : scale2, nbase2);
           const float2 e = make_float2(ex2(x.x), ex2(x.y));
           ps[wd & 3] = fadd2(ps[wd & 3], e);
-          pw[wd] = pack_bf16(e.x, e.y);
+          if constexpr (FP8) {
+            const float2 ev = fmul2(e, vf2[wd]);
+            pw[wd] = pack_bf16(ev.x, ev.y);
+          } else {
+            pw[wd] = pack_bf16(e.x, e.y);
+          }
+        }
+        if constexpr (FP8) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sm.f_free[jt % kNF]);   // this warp is done with the tile's factors
         }
         const float2 s01 = fadd2(fadd2(ps[0], ps[1]), fadd2(ps[2], ps[3]));
         l_run = l_run * alpha + (s01.x + s01.y);
@@ -690,7 +978,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
 
       Item nxt{};
       const bool have_next = next_item(k, nxt);
-      if (have_next && !a.q_rotated && !(ok = prepare_q(nxt, item + 1))) break;
+      if (have_next && (!a.q_rotated || FP8) && !(ok = prepare_q(nxt, item + 1))) break;
+      const float rs_next = q_row_scale;
 
       // ---- epilogue: O / l * sigmoid(gate) -> bf16 -> global, this warpgroup's 128 dims ----
       // 32 dims at a time through the warp's staging area: each thread writes
@@ -702,7 +991,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       const float l = l_run + sm.xsum[item & 1][wg ^ 1][r];   // both at the row's final base
       if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, item & 1)))) break;
       tc_fence_after();
-      float f = l > 0.f ? 1.f / l : 0.f;
+      float f = l > 0.f ? (FP8 ? kTwo120 : 1.f) / l : 0.f;   // FP8: O and l carry P x 2^64, O V x 2^-120
       if (a.gate != nullptr) f *= 1.f / (1.f + __expf(-gscore));
       const float2 f2 = make_float2(f, f);
       uint8_t* stg = sm.ostage[warp];
@@ -720,7 +1009,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int cc = 8 * q4 + 2 * e;
-            const float2 o = fmul2(make_float2(__uint_as_float(ov[cc]), __uint_as_float(ov[cc + 1])), f2);
+            // FP8: O's columns hold the dims of each group of four in the order 0, 2, 1, 3
+            const int c0 = FP8 ? (cc & ~3) + ((cc & 2) >> 1) : cc;
+            const int c1 = FP8 ? c0 + 2 : cc + 1;
+            const float2 o = fmul2(make_float2(__uint_as_float(ov[c0]), __uint_as_float(ov[c1])), f2);
             w4[e] = pack_bf16(o.x, o.y);
           }
           *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q4 ^ ((lane >> 1) & 3))) =
@@ -740,6 +1032,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kPfThreads, 1)
       arrive_cta0(&sm.o_free);
       it = nxt;
       have = have_next;
+      rs = rs_next;
       ++item;
     }
   }
@@ -772,14 +1065,18 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   const long long n_items = (long long)a.n_mtiles * h.B * (kHq / 2);   // (query tile, head pair)
   if (n_items <= 0 || n_items > 0x3fffffffLL) return cudaErrorInvalidValue;
   if (!full && !h.q_rotated) return cudaErrorInvalidValue;   // sliding layers take rotated queries
+  if (!full && h.fp8) return cudaErrorInvalidValue;          // FP8 rings are read through a bf16 context
   const long long grid = 2 * (n_items < h.n_pairs ? n_items : h.n_pairs);   // persistent CTA pairs
   profile_before(st);
-  if (full)
-    prefill_kernel<true><<<(unsigned)grid, kPfThreads, prefill_smem_bytes_t<true>(), st>>>(h.tm_k, h.tm_v, h.tm_q,
-                                                                                            h.tm_o, a);
+  if (full && h.fp8)
+    prefill_kernel<true, true><<<(unsigned)grid, PfCfg<true>::kThreads, prefill_smem_bytes_t<true, true>(), st>>>(
+        h.tm_k, h.tm_v, h.tm_q, h.tm_o, h.tm_ks, h.tm_vs, a);
+  else if (full)
+    prefill_kernel<true, false><<<(unsigned)grid, PfCfg<false>::kThreads, prefill_smem_bytes_t<true>(), st>>>(
+        h.tm_k, h.tm_v, h.tm_q, h.tm_o, h.tm_k, h.tm_v, a);
   else
-    prefill_kernel<false><<<(unsigned)grid, kPfThreads, prefill_smem_bytes_t<false>(), st>>>(h.tm_k, h.tm_v, h.tm_q,
-                                                                                             h.tm_o, a);
+    prefill_kernel<false, false><<<(unsigned)grid, PfCfg<false>::kThreads, prefill_smem_bytes_t<false>(), st>>>(
+        h.tm_k, h.tm_v, h.tm_q, h.tm_o, h.tm_k, h.tm_v, a);
   profile_after(st);
   count_launch();
   return cudaGetLastError();
@@ -791,10 +1088,13 @@ int prefill_v_box_rows() { return kHalfKeys; }
 int prefill_q_box_rows() { return kBM; }
 
 cudaError_t prefill_set_smem_attr() {
-  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  cudaError_t e = cudaFuncSetAttribute(prefill_kernel<true, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)prefill_smem_bytes_t<true>());
+  if (e == cudaSuccess)
+    e = cudaFuncSetAttribute(prefill_kernel<true, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)prefill_smem_bytes_t<true, true>());
   if (e != cudaSuccess) return e;
-  return cudaFuncSetAttribute(prefill_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+  return cudaFuncSetAttribute(prefill_kernel<false, false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                               (int)prefill_smem_bytes_t<false>());
 }
 

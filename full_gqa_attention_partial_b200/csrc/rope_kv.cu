@@ -51,12 +51,14 @@ struct RopeStoreArgs {
   int commit;               // 1: grid = B, block b owns sequence b and advances its len (and
                             //    ring head) after its rows, as kv_commit_kernel would
   int64_t capacity;         // commit, linear mode: the cache capacity
+  int qdq;                  // rows mode: each row written as its e4m3 quantization, dequantized
 };
 
 // One 256-dim row (one token, one KV head) held by a warp, 8 bf16 values per
 // lane in `x`: e4m3 codes with scale amax / 448, codes = satfinite round to
 // nearest even of value * (448 / amax) (a zero row: scale 0, codes 0).
-__device__ __forceinline__ void store_row_fp8(uint4 x, uint8_t* dst, float* dscale, int lane) {
+// Returns this lane's 8 codes (lowest byte first) and the row's scale.
+__device__ __forceinline__ uint2 quantize_row_fp8(uint4 x, float* scale) {
   const uint32_t w[4] = {x.x, x.y, x.z, x.w};
   float f[8];
 #pragma unroll
@@ -77,8 +79,32 @@ __device__ __forceinline__ void store_row_fp8(uint4 x, uint8_t* dst, float* dsca
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(h) : "f"(f[2 * i + 1] * inv), "f"(f[2 * i] * inv));
     c[i] = h;
   }
-  *reinterpret_cast<uint2*>(dst) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
-  if (lane == 0) *dscale = amax / 448.f;
+  *scale = amax / 448.f;
+  return make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+}
+__device__ __forceinline__ void store_row_fp8(uint4 x, uint8_t* dst, float* dscale, int lane) {
+  float sc;
+  *reinterpret_cast<uint2*>(dst) = quantize_row_fp8(x, &sc);
+  if (lane == 0) *dscale = sc;
+}
+
+// Eight e4m3 codes (8 bytes, lowest first) times `scale`, rounded to bf16
+// (8 values in 16 bytes, same order).  The codes are widened exactly (value
+// x 2^-120 by bit moves, then x 2^120 in fp32), then scaled in fp32.
+__device__ __forceinline__ uint4 dequant8_bf16(uint2 codes, float scale) {
+  const uint32_t w[2] = {codes.x, codes.y};
+  uint32_t o[4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    const uint32_t a = e4m3_b02_bf16x2(w[i]), c = e4m3_b13_bf16x2(w[i]);   // codes (0, 2) and (1, 3)
+    const float v0 = __uint_as_float(a << 16) * kE4m3WideScale * scale;
+    const float v2 = __uint_as_float(a & 0xFFFF0000u) * kE4m3WideScale * scale;
+    const float v1 = __uint_as_float(c << 16) * kE4m3WideScale * scale;
+    const float v3 = __uint_as_float(c & 0xFFFF0000u) * kE4m3WideScale * scale;
+    o[2 * i] = pack_bf16(v0, v1);
+    o[2 * i + 1] = pack_bf16(v2, v3);
+  }
+  return make_uint4(o[0], o[1], o[2], o[3]);
 }
 
 // One block = one token of one sequence, 128 threads; thread i handles
@@ -167,6 +193,17 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
         kx = make_uint4(os[0], os[1], os[2], os[3]);
       }
     }
+    if (a.qdq) {   // the rows an FP8 ring will hold, as attention reads them back
+      float sc;
+      uint2 c = quantize_row_fp8(kx, &sc);
+      kx = dequant8_bf16(c, sc);
+      if (a.v != nullptr) {
+        c = quantize_row_fp8(vx, &sc);
+        *reinterpret_cast<uint4*>(a.dv + dst) = dequant8_bf16(c, sc);
+      }
+      *reinterpret_cast<uint4*>(a.dk + dst) = kx;
+      continue;
+    }
     if (a.fp8) {
       store_row_fp8(kx, reinterpret_cast<uint8_t*>(a.dk) + dst, a.dks + row_id, lane32);
       if (a.v != nullptr)
@@ -190,69 +227,6 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
         a.len[b] += a.T;
       }
     }
-  }
-}
-
-// Eight e4m3 codes (8 bytes, lowest first) times `scale`, rounded to bf16
-// (8 values in 16 bytes, same order).  The codes are widened exactly (value
-// x 2^-120 by bit moves, then x 2^120 in fp32), then scaled in fp32.
-__device__ __forceinline__ uint4 dequant8_bf16(uint2 codes, float scale) {
-  const uint32_t w[2] = {codes.x, codes.y};
-  uint32_t o[4];
-#pragma unroll
-  for (int i = 0; i < 2; ++i) {
-    const uint32_t a = e4m3_b02_bf16x2(w[i]), c = e4m3_b13_bf16x2(w[i]);   // codes (0, 2) and (1, 3)
-    const float v0 = __uint_as_float(a << 16) * kE4m3WideScale * scale;
-    const float v2 = __uint_as_float(a & 0xFFFF0000u) * kE4m3WideScale * scale;
-    const float v1 = __uint_as_float(c << 16) * kE4m3WideScale * scale;
-    const float v3 = __uint_as_float(c & 0xFFFF0000u) * kE4m3WideScale * scale;
-    o[2 * i] = pack_bf16(v0, v1);
-    o[2 * i + 1] = pack_bf16(v2, v3);
-  }
-  return make_uint4(o[0], o[1], o[2], o[3]);
-}
-
-// bf16 copy of rows [0, len[b]) of an FP8 full-layer cache (contiguous or
-// paged) into dst [B][4][dst_rows][256], K and V: the history a prefill over
-// that cache attends to.  Rows [len + T, ...) up to the end of their 64-row
-// tile are zero-filled: the prefill loads whole tiles and multiplies the
-// masked rows by a zero weight, so they must hold finite values (the T
-// chunk rows in between are written by the chunk's own store).  Block
-// (tile, kvh, b) handles 64 rows.
-__global__ void __launch_bounds__(128) dequant_rows_kernel(const uint8_t* kc, const uint8_t* vc, const float* ks,
-                                                           const float* vs, PageMap pm, int64_t cap,
-                                                           const int32_t* len, int T, __nv_bfloat16* dk,
-                                                           __nv_bfloat16* dv, int64_t dst_rows) {
-  const int b = blockIdx.z, kvh = blockIdx.y;
-  const int row0 = blockIdx.x * 64;
-  const int L = len[b];
-  const int64_t tail_end = min(((int64_t)L + T + 63) / 64 * 64, dst_rows);
-  if (row0 >= tail_end) return;
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  for (int rr = warp; rr < 64; rr += 4) {
-    const int row = row0 + rr;
-    if (row >= tail_end) break;
-    const int64_t did = (((int64_t)b * kHkv + kvh) * dst_rows + row) * kD + lane * 8;
-    if (row >= L) {
-      if (row >= (int64_t)L + T) {
-        *reinterpret_cast<uint4*>(dk + did) = make_uint4(0, 0, 0, 0);
-        *reinterpret_cast<uint4*>(dv + did) = make_uint4(0, 0, 0, 0);
-      }
-      continue;
-    }
-    int64_t sid;   // source row of the [..][4][rows] layout
-    if (pm.page != 0) {
-      int prow, ppage;
-      kv_coord(pm, b, row, prow, ppage);
-      if (ppage < 0) ppage = 0;   // raised; read a valid page, the output is flagged invalid
-      sid = ((int64_t)ppage * kHkv + kvh) * pm.page + prow;
-    } else {
-      sid = ((int64_t)b * kHkv + kvh) * cap + row;
-    }
-    const uint2 kx = *reinterpret_cast<const uint2*>(kc + sid * kD + lane * 8);
-    const uint2 vx = *reinterpret_cast<const uint2*>(vc + sid * kD + lane * 8);
-    *reinterpret_cast<uint4*>(dk + did) = dequant8_bf16(kx, ks[sid]);
-    *reinterpret_cast<uint4*>(dv + did) = dequant8_bf16(vx, vs[sid]);
   }
 }
 
@@ -430,6 +404,7 @@ cudaError_t launch_rope_store(bool full, const RopeStoreHost& h, cudaStream_t st
   a.t_first = h.t_first;
   a.commit = h.commit;
   a.capacity = h.capacity;
+  a.qdq = h.qdq;
   const int grid = h.commit ? h.B : rope_grid(h.B * (h.T - h.t_first));
   cudaError_t e = full ? launch_pdl(rope_store_kernel<true>, dim3(grid, 1, 1), dim3(128, 1, 1), 0, st, 0u, a)
                        : launch_pdl(rope_store_kernel<false>, dim3(grid, 1, 1), dim3(128, 1, 1), 0, st, 0u, a);
@@ -443,17 +418,6 @@ cudaError_t launch_ring_gather(const void* rk, const void* rv, const float* rks,
   ring_gather_kernel<<<rope_grid(B * (kWindow - 1)), 128, 0, st>>>(
       reinterpret_cast<const __nv_bfloat16*>(rk), reinterpret_cast<const __nv_bfloat16*>(rv), rks, rvs, len, head,
       tag, reinterpret_cast<__nv_bfloat16*>(ck), reinterpret_cast<__nv_bfloat16*>(cv), ctx_rows, B);
-  count_launch();
-  return cudaGetLastError();
-}
-
-cudaError_t launch_dequant_rows(const void* kc, const void* vc, const float* ks, const float* vs, const PageMap& pm,
-                                int64_t cap, const int32_t* len, int T, int B, void* dk, void* dv, int64_t dst_rows,
-                                cudaStream_t st) {
-  const dim3 grid((unsigned)((dst_rows + 63) / 64), kHkv, B);
-  dequant_rows_kernel<<<grid, 128, 0, st>>>(reinterpret_cast<const uint8_t*>(kc), reinterpret_cast<const uint8_t*>(vc),
-                                            ks, vs, pm, cap, len, T, reinterpret_cast<__nv_bfloat16*>(dk),
-                                            reinterpret_cast<__nv_bfloat16*>(dv), dst_rows);
   count_launch();
   return cudaGetLastError();
 }

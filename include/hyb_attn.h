@@ -136,12 +136,13 @@ typedef struct hyb_kv_cache {
  *   stored value = code * scale (a zero row has scale 0 and zero codes).
  * Halves the cache bytes that decode streams (the pages' deployments keep
  * the KV cache in 8 bits: "不用高显存卡也能跑！..." q8_0 KV in llama.cpp).
- * FP8 caches need capacity % 4 == 0.  Decode reads every cached row as
- * stored (code value x scale, the current token included).  A prefill over
- * an FP8 cache attends to the cached history as stored (dequantized, rounded
- * to bf16) and to its own chunk at full precision, and appends the chunk
- * quantized; over a full-layer FP8 cache it needs the larger workspace of
- * hyb_attn_prefill_cache_workspace_size (bf16 copies of K and V).
+ * FP8 caches need capacity % 4 == 0.  Every attention over an FP8 cache
+ * reads the keys and values as the cache stores them (code value x scale):
+ * decode, the current token included, and prefill, whose chunk is appended
+ * quantized and attends to its own tokens in that form as well as to the
+ * history.  A full layer's prefill reads the codes in place (no workspace
+ * beyond the bf16 cache's); a sliding layer builds its usual bf16 context
+ * from the ring's rows and the chunk's rows as the ring will store them.
  */
 #define HYB_KV_BF16 0
 #define HYB_KV_FP8 1
@@ -195,9 +196,8 @@ hyb_status hyb_kv_append(const hyb_kv_cache* cache, const void* k, const void* v
  */
 size_t hyb_attn_prefill_workspace_size(int32_t layer_type, int32_t B, int32_t T, int32_t with_cache);
 /* Workspace of hyb_attn_prefill with this cache and chunk length: the value
- * above for bf16 caches, and for a full-layer FP8 cache two bf16 copies of
- * the cache, 2 x batch x 4 x capacity x 512 bytes (each rounded up to 256).
- * 0 for an invalid cache or T <= 0. */
+ * above, for bf16 and FP8 caches alike (it does not grow with the cache's
+ * capacity).  0 for an invalid cache or T <= 0. */
 size_t hyb_attn_prefill_cache_workspace_size(const hyb_kv_cache* cache, int32_t T);
 hyb_status hyb_attn_prefill(const void* q, const void* k, const void* v, const void* gate,
                             const int32_t* pos, int32_t layer_type, int32_t B, int32_t T,

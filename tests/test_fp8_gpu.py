@@ -59,11 +59,36 @@ def test_fp8_append_matches_quantizer(lib, lt):
     _check_rows(lib, cache, x, lt, slots, tokens)
 
 
+def as_stored(k_raw, v_raw, pos, lt):
+    """A chunk's keys and values as an FP8 cache stores them ([T, 4, 256]
+    each): keys rotated, rounded to bf16 and quantized, values quantized; both
+    dequantized, all by the oracle."""
+    k_rot = O.to_bf16(O.rope_layer(k_raw, pos, lt))
+    return (O.dequantize_e4m3_rows(*O.quantize_e4m3_rows(k_rot)),
+            O.dequantize_e4m3_rows(*O.quantize_e4m3_rows(v_raw)))
+
+
+def attend(x, lt, b, start, hist_k=None, hist_v=None, hist_idx=None):
+    """The oracle's attention of chunk x's queries (sequence b, token 0 at
+    sequence index `start`) over an optional stored history and the chunk's
+    own tokens as stored."""
+    q, k, v, g, pos = (f64(x["q"][b]), f64(x["k"][b]), f64(x["v"][b]), f64(x["gate"][b]), x["pos"][b].cpu().numpy())
+    T = q.shape[0]
+    kc, vc = as_stored(k, v, pos, lt)
+    idx = start + np.arange(T)
+    if hist_k is not None:
+        kc, vc, kidx = np.concatenate([hist_k, kc]), np.concatenate([hist_v, vc]), np.concatenate([hist_idx, idx])
+    else:
+        kidx = idx
+    return O.gqa_attention(O.rope_layer(q, pos, lt), kc, vc, idx, kidx, O.window_of(lt), g)
+
+
 @pytest.mark.parametrize("lt", [O.FULL, O.SLIDING])
 def test_fp8_chunked_prefill_matches_oracle(lib, lt):
-    """Two prefill chunks through an FP8 cache: each chunk attends to the
-    cached history as stored (the oracle dequantizes the codes) and to its
-    own tokens at full precision; the chunks are appended quantized."""
+    """Two prefill chunks through an FP8 cache: each chunk is appended
+    quantized and attends to the cached history and to its own tokens as the
+    cache stores them (the oracle quantizes the chunk itself and dequantizes
+    the history's codes)."""
     B, T1, T2 = 2, 700, 300
     r = synth.ring_offset(51)
     cache = lib.KVCache(lt, B, capacity=1024, kv_dtype=lib.KV_FP8, head0=None if lt == O.FULL else [r, (r + 99) % 512])
@@ -71,7 +96,7 @@ def test_fp8_chunked_prefill_matches_oracle(lib, lt):
     out1 = lib.hyb_attn_prefill(x1["q"], x1["k"], x1["v"], x1["gate"], x1["pos"], lt, cache=cache)
     torch.cuda.synchronize()
     assert lib.hyb_device_error() == 0
-    ref1 = O.prefill(f64(x1["q"]), f64(x1["k"]), f64(x1["v"]), f64(x1["gate"]), x1["pos"].cpu().numpy(), lt)
+    ref1 = np.stack([attend(x1, lt, b, 0) for b in range(B)])
     assert_close(out1, ref1, f"chunk 1 lt={lt}")
     # the history chunk 2 sees, as stored
     if lt == O.FULL:
@@ -94,9 +119,19 @@ def test_fp8_chunked_prefill_matches_oracle(lib, lt):
     torch.cuda.synchronize()
     assert lib.hyb_device_error() == 0
     assert cache.len.tolist() == [T1 + T2] * B
-    ref2 = O.prefill(f64(x2["q"]), f64(x2["k"]), f64(x2["v"]), f64(x2["gate"]), x2["pos"].cpu().numpy(), lt,
-                     start=[T1] * B, hist_k=hk, hist_v=hv, hist_idx=idx)
+    ref2 = np.stack([attend(x2, lt, b, T1, hk[b], hv[b], idx[b]) for b in range(B)])
     assert_close(out2, ref2, f"chunk 2 lt={lt}")
+
+
+def test_fp8_prefill_workspace_does_not_grow_with_capacity(lib):
+    """A full-layer FP8 cache is read in place: the prefill workspace is the
+    bf16 cache's (none), whatever the capacity."""
+    for cap in (1024, 1 << 20):
+        for kvd in (lib.KV_BF16, lib.KV_FP8):
+            c = lib.KVCache(O.FULL, 1, capacity=cap, kv_dtype=kvd)
+            assert lib.hyb_attn_prefill_cache_workspace_size(c, 8192) == 0
+            del c
+            torch.cuda.empty_cache()
 
 
 def assert_close(got, ref, what):

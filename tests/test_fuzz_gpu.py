@@ -2,8 +2,9 @@
 decode step on a cache of random kind (layer type, bf16 or FP8, contiguous
 or paged, ring offset), random batch, chunk lengths and gate.  Each call is
 compared with the oracle on the history as the cache stores it (read back
-and, for FP8, dequantized by the oracle), so any mismatch in the tiling,
-masking, paging or append bookkeeping of an odd size shows up."""
+and, for FP8, dequantized by the oracle; an FP8 chunk also attends to its
+own tokens as stored, which the oracle quantizes itself), so any mismatch in
+the tiling, masking, paging or append bookkeeping of an odd size shows up."""
 import numpy as np
 import pytest
 import torch
@@ -82,6 +83,18 @@ def _stored_history(cache, c, b):
     return (np.stack(ks) if ks else np.zeros(shape)), (np.stack(vs) if vs else np.zeros(shape)), np.asarray(idx)
 
 
+def _attend_fp8(x, gate, lt, b, start, hk, hv, hidx):
+    """The oracle's attention of chunk x over a stored history and the chunk's
+    own tokens as an FP8 cache stores them (rotated, rounded to bf16,
+    quantized and dequantized by the oracle)."""
+    q, k, v, pos = f64(x["q"][b]), f64(x["k"][b]), f64(x["v"][b]), x["pos"][b].cpu().numpy()
+    kc = O.dequantize_e4m3_rows(*O.quantize_e4m3_rows(O.to_bf16(O.rope_layer(k, pos, lt))))
+    vc = O.dequantize_e4m3_rows(*O.quantize_e4m3_rows(v))
+    idx = start + np.arange(q.shape[0])
+    return O.gqa_attention(O.rope_layer(q, pos, lt), np.concatenate([hk, kc]), np.concatenate([hv, vc]), idx,
+                           np.concatenate([hidx, idx]), O.window_of(lt), None if gate is None else f64(gate[b]))
+
+
 @pytest.mark.parametrize("seed", SEEDS)
 def test_random_cache_path(lib, seed):
     c = _case(seed)
@@ -95,9 +108,12 @@ def test_random_cache_path(lib, seed):
         out = lib.hyb_attn_prefill(x["q"], x["k"], x["v"], gate, x["pos"], lt, cache=cache)
         torch.cuda.synchronize()
         assert lib.hyb_device_error() == 0
-        ref = O.prefill(f64(x["q"]), f64(x["k"]), f64(x["v"]), None if gate is None else f64(gate),
-                        x["pos"].cpu().numpy(), lt, start=[start] * B, hist_k=[h[0] for h in hist],
-                        hist_v=[h[1] for h in hist], hist_idx=[h[2] for h in hist])
+        if c["fp8"]:   # the chunk attends to its own tokens as the FP8 cache stores them
+            ref = np.stack([_attend_fp8(x, gate, lt, b, start, *hist[b]) for b in range(B)])
+        else:
+            ref = O.prefill(f64(x["q"]), f64(x["k"]), f64(x["v"]), None if gate is None else f64(gate),
+                            x["pos"].cpu().numpy(), lt, start=[start] * B, hist_k=[h[0] for h in hist],
+                            hist_v=[h[1] for h in hist], hist_idx=[h[2] for h in hist])
         check(out, ref, f"{c} chunk {i}")
         start += T
     assert cache.len.tolist() == [start] * B
