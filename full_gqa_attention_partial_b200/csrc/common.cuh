@@ -207,18 +207,28 @@ __device__ __forceinline__ void tma_load_3d(uint32_t smem_dst, const void* tmap,
       "l"(tmap), "r"(c0), "r"(c1), "r"(c2), "r"(smem_u32(bar))
       : "memory");
 }
+__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
+  uint32_t d;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
+  return d;
+}
 // e4m3 -> bf16 by integer bit moves, scaled by 2^-120: the e4m3 sign,
 // exponent and mantissa bits land in the bf16 sign, the low four exponent
 // bits and the top three mantissa bits, so the code 2^(e-7) (1 + m/8) becomes
 // the bf16 2^(e-127) (1 + m/8) and the subnormal code m 2^-9 the bf16
-// subnormal m 2^-129, both exact.  A word of four codes (byte 0 lowest)
-// gives two bf16 pairs: bytes 0 and 2 (low half first), and bytes 1 and 3.
-__device__ __forceinline__ uint32_t e4m3_b02_bf16x2(uint32_t w) {
-  return ((w << 8) & 0x80008000u) | ((w << 4) & 0x07F007F0u);
+// subnormal m 2^-129, both exact.  Three instructions for two codes: a byte
+// permute puts each code in a 16-bit half with its sign bit copied over the
+// high byte, a shift by 4 moves sign and magnitude into place, and a mask
+// clears the copies and what the low half shifted into the high one.
+// A word of four codes (byte 0 lowest) gives two bf16 pairs (low half first).
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t e4m3_pair_bf16x2(uint32_t w) {
+  return (prmt(w, 0u, SEL) << 4) & 0x87F087F0u;
 }
-__device__ __forceinline__ uint32_t e4m3_b13_bf16x2(uint32_t w) {
-  return (w & 0x80008000u) | ((w >> 4) & 0x07F007F0u);
-}
+__device__ __forceinline__ uint32_t e4m3_b01_bf16x2(uint32_t w) { return e4m3_pair_bf16x2<0x9180u>(w); }
+__device__ __forceinline__ uint32_t e4m3_b23_bf16x2(uint32_t w) { return e4m3_pair_bf16x2<0xB3A2u>(w); }
+__device__ __forceinline__ uint32_t e4m3_b02_bf16x2(uint32_t w) { return e4m3_pair_bf16x2<0xA280u>(w); }
+__device__ __forceinline__ uint32_t e4m3_b13_bf16x2(uint32_t w) { return e4m3_pair_bf16x2<0xB391u>(w); }
 // Two floats -> two e4m3 codes (lo in the low byte), round to nearest even, saturating.
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   uint16_t h;
@@ -230,11 +240,6 @@ __device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t c) {
   uint32_t d;
   asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(d) : "h"((uint16_t)c));
   return __half22float2(*reinterpret_cast<const __half2*>(&d));
-}
-__device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
-  uint32_t d;
-  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(d) : "r"(a), "r"(b), "r"(sel));
-  return d;
 }
 constexpr float kE4m3WideScale = 1.329227995784916e36f;   // 2^120
 constexpr float kE4m3PScale = 18446744073709551616.f;      // 2^64

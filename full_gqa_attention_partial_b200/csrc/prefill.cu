@@ -61,9 +61,7 @@
 // 2^-4, would not meet the accuracy bound).  V feeds O += P V in bf16: its
 // codes land in the upper half of one of two 32 KB V slots and two converter
 // warps (12 warps in all) widen them in place by integer bit moves (value x
-// 2^-120, exact), which give the dims of each group of four in the order 0,
-// 2, 1, 3; the slot keeps that order, so O's columns come in it too and the
-// epilogue puts them back.  The row scales never touch the operands: TMA
+// 2^-120, exact; three instructions for two codes).  The row scales never touch the operands: TMA
 // loads them into a four-tile ring, the softmax multiplies the scores by the
 // K scale and P by the V scale, the query row's factor and the softmax scale
 // come in with the row maximum and the exponent, P carries 2^64 (added in the
@@ -524,8 +522,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
     // write its 16 bf16 dims as two 16-byte chunks, lanes 4-7 in the other order
     // so that the 8 lanes' chunks fall in 8 bank groups.  A thread's output in
     // the upper half (dims 64-127) lands on the code row it read from, which
-    // only lanes of its own warp read: each warp reads all its codes, then
-    // writes, with no wait on the other warp.
+    // only lanes of its own warp read, at the same item: each warp reads a
+    // group of four items, then writes them, with no wait on the other warp
+    // (four at a time keeps the loop small next to the softmax warps' code in
+    // the instruction cache).
     const int ct = (warp - kConvWarp) * 32 + lane;   // 0..63
     // item i of this thread: key 4 i + rq of source box sb, 16 codes q; (4 i) & 7
     // alternates between 0 and 4, so the swizzled chunk indexes take two values
@@ -548,26 +548,30 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.vcode[v], (jt / kNV) & 1)))) break;
         uint8_t* dst = sm.slot[2 + v];
         const uint8_t* sp = dst + kCodeBytes + sb * 8192 + rq * 128;
-        uint4 cw[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) cw[i] = *reinterpret_cast<const uint4*>(sp + i * 512 + ((i & 1) ? sx1 : sx0));
-        __syncwarp();   // every lane's codes read before any lane overwrites them
         // 64-dim chunk q / 4, key 64 sb + 4 i + rq
         uint8_t* dp = dst + (q >> 2) * 16384 + (64 * sb + rq) * 128;
+#pragma unroll 1
+        for (int i0 = 0; i0 < 16; i0 += 4) {
+        uint4 cw[4];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const uint32_t wv[4] = {cw[i].x, cw[i].y, cw[i].z, cw[i].w};
-          uint32_t o[8];   // the dims of each group of four in the order 0, 2, 1, 3
+        for (int i = 0; i < 4; ++i) cw[i] = *reinterpret_cast<const uint4*>(sp + (i0 + i) * 512 + ((i & 1) ? sx1 : sx0));
+        __syncwarp();   // the group's codes read by every lane before any lane overwrites them
+#pragma unroll
+        for (int i1 = 0; i1 < 4; ++i1) {
+          const int i = i0 + i1;
+          const uint32_t wv[4] = {cw[i1].x, cw[i1].y, cw[i1].z, cw[i1].w};
+          uint32_t o[8];
 #pragma unroll
           for (int j = 0; j < 4; ++j) {
-            o[2 * j] = e4m3_b02_bf16x2(wv[j]);
-            o[2 * j + 1] = e4m3_b13_bf16x2(wv[j]);
+            o[2 * j] = e4m3_b01_bf16x2(wv[j]);
+            o[2 * j + 1] = e4m3_b23_bf16x2(wv[j]);
           }
           const uint4 lo = make_uint4(o[0], o[1], o[2], o[3]), hi = make_uint4(o[4], o[5], o[6], o[7]);
           const uint4 va = (q < 4) ? lo : hi, vb = (q < 4) ? hi : lo;
           uint8_t* rowp = dp + i * 512;
           *reinterpret_cast<uint4*>(rowp + ((i & 1) ? da1 : da0)) = va;
           *reinterpret_cast<uint4*>(rowp + ((i & 1) ? db1 : db0)) = vb;
+        }
         }
         fence_proxy_async();              // the slot is read by the tensor core
         if (rank != 0) fence_cluster();   // ... through MMAs issued from CTA 0
@@ -698,7 +702,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
      if constexpr (!FULL) {
       return false;   // sliding layers: queries always arrive rotated
      } else {
-      if (a.q_rotated) {   // FP8 with rotated queries: only the permutation below
+      if (a.q_rotated) {   // FP8 with rotated queries: only the split into Q_hi + Q_lo below
         if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_full, item_no & 1))) return false;
       } else {
       const int row = it.m0 + r;
@@ -1009,10 +1013,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             const int cc = 8 * q4 + 2 * e;
-            // FP8: O's columns hold the dims of each group of four in the order 0, 2, 1, 3
-            const int c0 = FP8 ? (cc & ~3) + ((cc & 2) >> 1) : cc;
-            const int c1 = FP8 ? c0 + 2 : cc + 1;
-            const float2 o = fmul2(make_float2(__uint_as_float(ov[c0]), __uint_as_float(ov[c1])), f2);
+            const float2 o = fmul2(make_float2(__uint_as_float(ov[cc]), __uint_as_float(ov[cc + 1])), f2);
             w4[e] = pack_bf16(o.x, o.y);
           }
           *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q4 ^ ((lane >> 1) & 3))) =
