@@ -572,6 +572,95 @@ def bench_decode(hyb, args, peaks, fp8: bool = False, page: int = 0):
     }
 
 
+def bench_layer_decode(hyb, args, peaks):
+    """The 3-sliding + 1-full group as whole decode layers (q_k_v_proj with the
+    gate rows, append, attention, o_proj), B=16 over 131072-token caches:
+    hyb_attn_layer_decode per layer.  The projections' share is the step time
+    minus that of the attention alone (append + decode) on caches in the same
+    state; they read 52.5 MB of weights per layer, so they are HBM-bound."""
+    from full_gqa_attention_partial_b200 import synth
+    B, L = 16, 131072
+    n = args.steps
+    cap = L + 2 * (args.warmup + 1 + n) + 2
+    cap += (-cap) % 4
+    g = torch.Generator(device="cuda").manual_seed(78)
+    w = [((torch.randn(6144, 2560, generator=g, device="cuda") / 2560 ** 0.5).to(torch.bfloat16),
+          (torch.randn(16, 2560, generator=g, device="cuda") / 2560 ** 0.5).to(torch.bfloat16),
+          (torch.randn(2560, 4096, generator=g, device="cuda") / 4096 ** 0.5).to(torch.bfloat16))
+         for _ in GROUP_LAYERS]
+    r = synth.ring_offset(4)
+    caches = [fill_full_cache(hyb, B, L, cap, seed=40 + i) if lt == FULL else
+              fill_ring_cache(hyb, B, L, seed=40 + i, head0=r) for i, lt in enumerate(GROUP_LAYERS)]
+    hid = [(torch.randn(B, 2560, generator=g, device="cuda")).to(torch.bfloat16) for _ in range(args.warmup + 1)]
+    qs = [synth.decode_query(B, seed=2000 + i, device="cuda") for i in range(args.warmup + 1)]
+    ws = hyb.alloc_workspace(max(hyb.hyb_attn_layer_decode_workspace_size(lt, B, cap if lt == FULL else W)
+                                 for lt in GROUP_LAYERS))
+    out = torch.empty(B, 2560, dtype=torch.bfloat16, device="cuda")
+    aout = torch.empty(B, H, D, dtype=torch.bfloat16, device="cuda")
+
+    def layer_step(i):
+        for li, lt in enumerate(GROUP_LAYERS):
+            hyb.hyb_attn_layer_decode(hid[i], *w[li], caches[li], max_len=cap if lt == FULL else W, out=out,
+                                      workspace=ws)
+
+    def attn_step(i):
+        x = qs[i]
+        for li, lt in enumerate(GROUP_LAYERS):
+            hyb.hyb_kv_append(caches[li], x["k"], x["v"])
+            hyb.hyb_attn_decode(x["q"], x["gate"], caches[li], max_len=cap if lt == FULL else W, out=aout,
+                                workspace=ws)
+
+    def timed(fn):
+        # one step captured as a CUDA graph and replayed (the caches' device-side
+        # len / head move the append position), so host time is not in the number
+        for i in range(args.warmup):
+            fn(i)
+        side = torch.cuda.Stream()
+        side.wait_stream(torch.cuda.current_stream())
+        graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(graph, stream=side):
+            fn(args.warmup)
+        torch.cuda.synchronize()
+        ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        ev0.record()
+        for i in range(n):
+            graph.replay()
+        ev1.record()
+        torch.cuda.synchronize()
+        assert hyb.hyb_device_error() == 0
+        del graph
+        return ev0.elapsed_time(ev1) / n
+
+    ms = timed(layer_step)
+    attn_ms = timed(attn_step)
+    proj_ms = max(ms - attn_ms, 1e-6)
+    # the projection kernels alone: q_k_v_proj and o_proj of the 4 layers through hyb_linear
+    pq = torch.empty(B, 6144, dtype=torch.bfloat16, device="cuda")
+    po = torch.empty(B, 2560, dtype=torch.bfloat16, device="cuda")
+    xa = torch.randn(B, 4096, generator=g, device="cuda").to(torch.bfloat16)
+
+    def proj_step(i):
+        for li in range(len(GROUP_LAYERS)):
+            hyb.hyb_linear(hid[0], w[li][0], out=pq)
+            hyb.hyb_linear(xa, w[li][2], out=po)
+
+    pk_ms = timed(proj_step)
+    pk_bytes = len(GROUP_LAYERS) * 2 * (6144 * 2560 + 2560 * 4096)
+    wbytes = len(GROUP_LAYERS) * 2 * 2560 * (6144 + 16 + 4096)
+    kv = B * (L + args.warmup + 1 + n) * KV_TOKEN_BYTES[False] + 3 * B * W * KV_TOKEN_BYTES[False]
+    del caches
+    return {"workload": "3+1 group as whole decode layers (projections, synthetic weights), B=16, caches 131072",
+            "ms_per_step": ms, "tokens_per_s": B / (ms / 1e3),
+            "gb_per_s": (wbytes + kv) / (ms / 1e3) / 1e9, "frac_of_hbm": (wbytes + kv) / (ms / 1e3) / 1e9 / HBM_READ_GBS,
+            "projections": {"ms_per_step": proj_ms, "weight_bytes": wbytes,
+                            "weight_gb_per_s": wbytes / (proj_ms / 1e3) / 1e9,
+                            "frac_of_hbm": wbytes / (proj_ms / 1e3) / 1e9 / HBM_READ_GBS,
+                            "kernels_alone": {"ms_per_step": pk_ms, "weight_bytes": pk_bytes,
+                                              "weight_gb_per_s": pk_bytes / (pk_ms / 1e3) / 1e9,
+                                              "frac_of_hbm": pk_bytes / (pk_ms / 1e3) / 1e9 / HBM_READ_GBS}},
+            "attention_ms_per_step": attn_ms}
+
+
 def bench_decode_1m(hyb, args, peaks, fp8: bool = False):
     """36 layers (27 rings, 9 full caches of ~1M tokens), batch 1, 64 steps of append + decode.
 
@@ -931,6 +1020,7 @@ def main():
         extras["decode"] = run("decode", bench_decode, hyb, args, peaks)
         extras["decode_fp8"] = run("decode_fp8", bench_decode, hyb, args, peaks, fp8=True)
         extras["decode_paged"] = run("decode_paged", bench_decode, hyb, args, peaks, page=64)
+        extras["layer_decode"] = run("layer_decode", bench_layer_decode, hyb, args, peaks)
         if args.decode_1m:
             extras["decode_1m"] = run("decode_1m", bench_decode_1m, hyb, args, peaks)
             torch.cuda.empty_cache()

@@ -31,9 +31,13 @@ KV_FP8 = 1
 DEV_ERR_CAPACITY = 1
 DEV_ERR_TIMEOUT = 2
 DEV_ERR_PAGE = 4
+DEV_ERR_BOUNDS = 8      # debug build only: an index outside its buffer, access skipped
+BUILD_DEBUG_BOUNDS = 1  # hyb_build_flags() bit of the debug build
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_PKG, "_lib", "libhyb_attn.so")
+# the -DHYB_DEBUG_BOUNDS build (device-side index checks); load(DEBUG_LIB_PATH) instead of load()
+DEBUG_LIB_PATH = os.path.join(_PKG, "_lib", "libhyb_attn_debug.so")
 
 EXPORTED = (
     "hyb_kv_cache_init", "hyb_kv_append", "hyb_attn_prefill_workspace_size", "hyb_attn_prefill",
@@ -42,6 +46,7 @@ EXPORTED = (
     "hyb_selftest_wait_timeout", "hyb_linear", "hyb_attn_layer_prefill_workspace_size", "hyb_attn_layer_prefill",
     "hyb_attn_layer_decode_workspace_size", "hyb_attn_layer_decode", "hyb_attn_decode_partial",
     "hyb_attn_decode_merge", "hyb_attn_prefill_cache_workspace_size", "hyb_attn_layer_prefill_cache_workspace_size",
+    "hyb_build_flags",
 )
 
 
@@ -96,6 +101,7 @@ def load(path: str = LIB_PATH):
     lib.hyb_device_error.argtypes = [ctypes.POINTER(i32), i32, vp]
     lib.hyb_last_error.restype = ctypes.c_char_p
     lib.hyb_launch_count.restype = ctypes.c_uint64
+    lib.hyb_build_flags.restype = ctypes.c_int32
     lib.hyb_profile_events.argtypes = [ctypes.POINTER(ctypes.c_void_p), i32]
     lib.hyb_profile_events.restype = ctypes.c_int
     lib.hyb_profile_pairs_used.restype = i32
@@ -491,6 +497,11 @@ def hyb_selftest_wait_timeout(stream=None) -> None:
 
 def hyb_launch_count() -> int:
     return int(load().hyb_launch_count())
+
+
+def hyb_build_flags() -> int:
+    """BUILD_DEBUG_BOUNDS when the loaded library is the index-checking debug build, else 0."""
+    return int(load().hyb_build_flags())
 
 
 class KernelTimer:

@@ -15,6 +15,9 @@ ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB_DIR = os.path.join(PKG, "_lib")
 LIB = os.path.join(LIB_DIR, "libhyb_attn.so")
+# the same library with -DHYB_DEBUG_BOUNDS: device-side index checks that report
+# through the error word (HYB_DEV_ERR_BOUNDS) and skip the access
+DEBUG_LIB = os.path.join(LIB_DIR, "libhyb_attn_debug.so")
 
 
 def sources() -> list:
@@ -30,23 +33,21 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found")
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB):
+def needs_build(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return True
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     deps = sources() + [os.path.join(ROOT, "include", "hyb_attn.h")]
     return any(os.path.getmtime(d) > t for d in deps if os.path.exists(d))
 
 
-def build(verbose: bool = False, force: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB
+def _compile(lib: str, defines: list, verbose: bool) -> None:
     os.makedirs(LIB_DIR, exist_ok=True)
-    tmp = LIB + ".tmp"
+    tmp = lib + ".tmp"
     cmd = [
         nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-lineinfo", "-O3", "-std=c++17",
         "-Xcompiler", "-fPIC", "-shared", "-I", os.path.join(ROOT, "include"),
-        "-Xptxas", "-v" if verbose else "-O3",
+        "-Xptxas", "-v" if verbose else "-O3", *defines,
         "-o", tmp, os.path.join(CSRC, "hyb_attn_lib.cu"),
     ]
     res = subprocess.run(cmd, capture_output=True, text=True)
@@ -54,7 +55,15 @@ def build(verbose: bool = False, force: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + res.stdout + res.stderr)
     if verbose:
         sys.stderr.write(res.stdout + res.stderr)
-    os.replace(tmp, LIB)
+    os.replace(tmp, lib)
+
+
+def build(verbose: bool = False, force: bool = False, debug: bool = True) -> str:
+    """Builds the library (and, with debug, its -DHYB_DEBUG_BOUNDS twin); returns the normal one's path."""
+    if force or needs_build(LIB):
+        _compile(LIB, [], verbose)
+    if debug and (force or needs_build(DEBUG_LIB)):
+        _compile(DEBUG_LIB, ["-DHYB_DEBUG_BOUNDS"], verbose)
     return LIB
 
 

@@ -295,6 +295,8 @@ const char* hyb_last_error(void) { return t_err.c_str(); }
 
 uint64_t hyb_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
+int32_t hyb_build_flags(void) { return hyb::kBuildFlags ? HYB_BUILD_DEBUG_BOUNDS : 0; }
+
 hyb_status hyb_profile_events(void* const* events, int32_t n_pairs) {
   if (n_pairs < 0) return fail(HYB_EINVAL, "n_pairs %d negative", n_pairs);
   hyb::g_prof_events = (n_pairs > 0) ? events : nullptr;
@@ -341,9 +343,13 @@ hyb_status make_rows_map(CUtensorMap* m, const void* base, uint64_t rows, uint64
 // sliding / full layer's heads (see GemmHost)
 // rope != 0: RoPE epilogue on the column tiles below rope_cols, with the
 // (cos, sin) table of the M rows written first into `rot` (float2 [M][R/2])
+// w2 != NULL: a second output group of N2 columns, y2[M][ldy2] = X w2[N2][K]^T,
+// computed in the same launch as columns N .. N + N2 - 1 (N a multiple of 256)
 hyb_status linear_impl(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int32_t M,
                        int32_t N, int32_t K, void* stream, int rope = 0, int rope_cols = 0, int32_t T = 0,
-                       const int32_t* pos = nullptr, const int32_t* len = nullptr, void* rot = nullptr) {
+                       const int32_t* pos = nullptr, const int32_t* len = nullptr, void* rot = nullptr,
+                       const void* w2 = nullptr, int64_t ldw2 = 0, void* y2 = nullptr, int64_t ldy2 = 0,
+                       int32_t N2 = 0, bool w_not_written_by_previous = false) {
   if (!x || !w || !y) return fail(HYB_EINVAL, "x, w and y must not be NULL");
   if (M <= 0 || N <= 0 || K <= 0) return fail(HYB_ESHAPE, "M, N, K must be positive (got %d, %d, %d)", M, N, K);
   if (N % 8 || K % 8) return fail(HYB_ESHAPE, "N and K must be multiples of 8 (got %d, %d)", N, K);
@@ -352,13 +358,46 @@ hyb_status linear_impl(const void* x, int64_t ldx, const void* w, int64_t ldw, v
   if (!aligned16(x) || !aligned16(w) || !aligned16(y)) return fail(HYB_EALIGN, "x, w and y must be 16-byte aligned");
   hyb_status s = ensure_device();
   if (s != HYB_OK) return s;
+  if (w2 != nullptr && (N % 256 || N2 <= 0 || N2 % 8 || ldw2 < K || ldy2 < N2 || ldw2 % 8 || ldy2 % 8 || !y2 ||
+                        !aligned16(w2) || !aligned16(y2)))
+    return fail(HYB_ESHAPE, "second output group: N %% 256, N2 %% 8, strides or alignment");
+  if (rope == 0 && smallm_supported(M, N + (w2 ? N2 : 0), K, N)) {
+    // a few rows (decode steps): stream W over every SM instead of 256-row tiles
+    SmallMHost sh;
+    sh.x = x;
+    sh.ldx = ldx;
+    sh.w = w;
+    sh.ldw = ldw;
+    sh.w2 = w2;
+    sh.ldw2 = ldw2;
+    sh.y = y;
+    sh.ldy = ldy;
+    sh.y2 = y2;
+    sh.ldy2 = ldy2;
+    sh.n_main = w2 ? N : 0;
+    sh.M = M;
+    sh.N = N + (w2 ? N2 : 0);
+    sh.K = K;
+    sh.early_w = w_not_written_by_previous;
+    const cudaError_t e = launch_smallm(sh, as_stream(stream));
+    if (e != cudaSuccess) return cuda_fail(e, "few-row linear launch");
+    return HYB_OK;
+  }
   GemmHost gh;
   if ((s = make_rows_map(&gh.tm_x, x, (uint64_t)M, (uint64_t)K, (uint64_t)ldx, "x")) != HYB_OK) return s;
   if ((s = make_rows_map(&gh.tm_w, w, (uint64_t)N, (uint64_t)K, (uint64_t)ldw, "w")) != HYB_OK) return s;
+  gh.tm_w2 = gh.tm_w;
   gh.y = y;
   gh.ldy = ldy;
   gh.M = M;
   gh.N = N;
+  if (w2 != nullptr) {
+    if ((s = make_rows_map(&gh.tm_w2, w2, (uint64_t)N2, (uint64_t)K, (uint64_t)ldw2, "w2")) != HYB_OK) return s;
+    gh.y2 = y2;
+    gh.ldy2 = ldy2;
+    gh.n_main = N;
+    gh.N = N + N2;
+  }
   gh.K = K;
   gh.n_pairs = device_sms() / 2;
   gh.rope = rope;
@@ -903,14 +942,13 @@ hyb_status hyb_attn_layer_prefill(const void* hidden, const void* w_qkv, const v
   p += round256(n * 128 * 8);
   const size_t attn_ws = prefill_ws(layer_type, B, T, cache, false);
   // q_k_v_proj with RoPE of the q and k heads in the epilogue (positions as
-  // hyb_attn_prefill: pos, else the cache length + t, else t)
+  // hyb_attn_prefill: pos, else the cache length + t, else t); the gate
+  // projection's 16 rows as one more column tile of the same launch
   const int32_t* len = cache ? cache->len : nullptr;
   hyb_status s = linear_impl(hidden, kHidden, w_qkv, kHidden, qkv, kQkv, M, (int32_t)kQkv, (int32_t)kHidden, stream,
-                             layer_type == HYB_FULL ? 2 : 1, (kHq + kHkv) * kD, T, pos, len, rot);
+                             layer_type == HYB_FULL ? 2 : 1, (kHq + kHkv) * kD, T, pos, len, rot, w_gate, kHidden,
+                             w_gate ? gate : nullptr, kHq, w_gate ? kHq : 0);
   if (s != HYB_OK) return s;
-  if (w_gate && (s = hyb_linear(hidden, kHidden, w_gate, kHidden, gate, kHq, M, kHq, (int32_t)kHidden, stream)) !=
-                    HYB_OK)
-    return s;
   s = prefill_impl(qkv, qkv + (int64_t)kHq * kD, qkv + (int64_t)(kHq + kHkv) * kD, w_gate ? gate : nullptr, pos,
                    layer_type, B, T, kQkv, kQkv, attn, cache, attn_ws ? p : nullptr, attn_ws, stream, true);
   if (s != HYB_OK) return s;
@@ -949,19 +987,23 @@ hyb_status hyb_attn_layer_decode(const void* hidden, const void* w_qkv, const vo
   p += round256(n * kHq * kD * 2);
   void* rot = p;
   p += round256(n * 128 * 8);
-  // q_k_v_proj with RoPE at the new token's position (the cache length)
+  // q_k_v_proj and the gate projection in one launch.  Up to 16 sequences the
+  // few-row kernel streams the weights and the append and the decode rotate
+  // k and q at the new token's position (the cache length); beyond, the
+  // tiled GEMM rotates them in its epilogue.
+  const bool few = smallm_supported(B, (int)(kQkv + (w_gate ? kHq : 0)), (int)kHidden, (int)kQkv);
   if ((s = linear_impl(hidden, kHidden, w_qkv, kHidden, qkv, kQkv, B, (int32_t)kQkv, (int32_t)kHidden, stream,
-                       layer_type == HYB_FULL ? 2 : 1, (kHq + kHkv) * kD, 1, nullptr, cache->len, rot)) != HYB_OK)
-    return s;
-  if (w_gate && (s = linear_impl(hidden, kHidden, w_gate, kHidden, gate, kHq, B, kHq, (int32_t)kHidden, stream)) !=
-                    HYB_OK)
+                       few ? 0 : (layer_type == HYB_FULL ? 2 : 1), few ? 0 : (kHq + kHkv) * kD, 1, nullptr,
+                       cache->len, rot, w_gate, kHidden, w_gate ? gate : nullptr, kHq, w_gate ? kHq : 0)) != HYB_OK)
     return s;
   if ((s = append_impl(cache, qkv + (int64_t)kHq * kD, qkv + (int64_t)(kHq + kHkv) * kD, kQkv, nullptr, 1, stream,
-                       true)) != HYB_OK)
+                       !few)) != HYB_OK)
     return s;
-  if ((s = decode_impl(qkv, kQkv, true, w_gate ? gate : nullptr, nullptr, cache, layer_type, max_len, attn, p,
+  if ((s = decode_impl(qkv, kQkv, !few, w_gate ? gate : nullptr, nullptr, cache, layer_type, max_len, attn, p,
                        hyb_attn_decode_workspace_size(layer_type, B, max_len), stream)) != HYB_OK)
     return s;
+  // o_proj right after the library's own attention, which does not write w_o
   return linear_impl(attn, (int64_t)kHq * kD, w_o, (int64_t)kHq * kD, out, kHidden, B, (int32_t)kHidden,
-                     (int32_t)(kHq * kD), stream);
+                     (int32_t)(kHq * kD), stream, 0, 0, 0, nullptr, nullptr, nullptr, nullptr, 0, nullptr, 0, 0,
+                     true);
 }

@@ -31,8 +31,26 @@ static __device__ int g_dev_err = 0;
 constexpr int kErrCapacity = 1;
 constexpr int kErrTimeout = 2;
 constexpr int kErrPage = 4;
+constexpr int kErrBounds = 8;
 
 __device__ __forceinline__ void raise_err(int bit) { atomicOr(&g_dev_err, bit); }
+
+// Index checks of the debug build (-DHYB_DEBUG_BOUNDS): HYB_BOUNDS(i, lo, hi)
+// is true when lo <= i < hi; otherwise it raises kErrBounds and is false, and
+// the caller skips the access (nothing traps, no CTA leaves a barrier early).
+// In the normal build it is the constant true and the check compiles away.
+#ifdef HYB_DEBUG_BOUNDS
+__device__ __forceinline__ bool hyb_in_bounds(int64_t i, int64_t lo, int64_t hi) {
+  if (i >= lo && i < hi) return true;
+  raise_err(kErrBounds);
+  return false;
+}
+#define HYB_BOUNDS(i, lo, hi) (::hyb::hyb_in_bounds((int64_t)(i), (int64_t)(lo), (int64_t)(hi)))
+constexpr int kBuildFlags = 1;
+#else
+#define HYB_BOUNDS(i, lo, hi) true
+constexpr int kBuildFlags = 0;
+#endif
 
 // Row and batch coordinates of key row `row` of sequence b in a cache's TMA
 // map: the identity for contiguous caches; for paged caches the row within
@@ -396,6 +414,18 @@ __device__ __forceinline__ void mma_ss_pair_e4m3_warp(uint32_t d_tmem, uint64_t 
       "@e tcgen05.mma.cta_group::2.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+// Loads from the shared memory of another CTA of the cluster.
+__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
+               : "memory");
+  return v;
 }
 // Orders this thread's earlier memory writes before its later ones for every
 // thread of the cluster.

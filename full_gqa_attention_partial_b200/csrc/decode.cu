@@ -104,6 +104,7 @@ struct DecArgs {
   float* part_o;
   float* part_lse;
   int n_splits;
+  int B;              // sequences (index checks of the debug build)
   PageMap pm;         // paged cache: maps over the pool {.., page, 4, n_pages}
   // cluster merge (the splits of one (sequence, KV head) form a thread-block
   // cluster): CTA 0 of the cluster merges them and writes the result itself
@@ -114,18 +115,6 @@ struct DecArgs {
   float* out_lse;              // [B][16] base-2 log-sum-exp
 };
 
-// Loads from the shared memory of another CTA of the cluster.
-__device__ __forceinline__ float ld_cluster_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
-  return v;
-}
-__device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
-  float4 v;
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];" : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w) : "r"(addr)
-               : "memory");
-  return v;
-}
 
 template <bool FULL, bool FP8>
 __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
@@ -150,7 +139,7 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
   pdl_wait();
   pdl_launch_dependents();
 
-  const int L = a.len[b];
+  const int L = HYB_BOUNDS(b, 0, a.B) ? a.len[b] : 0;
   const int qseq = L - 1;
   const int n_keys = FULL ? L : kWindow;          // keys (FULL) or ring slots (SLIDING)
   int kps = (n_keys + a.n_splits - 1) / a.n_splits;
@@ -159,7 +148,8 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
   const int k1 = min(n_keys, k0 + kps);
   const int n_stages = (k1 > k0 && L > 0) ? (k1 - k0 + kDecKeys - 1) / kDecKeys : 0;
   if (!FULL) {
-    for (int i = threadIdx.x; i < kWindow; i += blockDim.x) sm.tags[i] = a.tag[(int64_t)b * kWindow + i];
+    for (int i = threadIdx.x; i < kWindow; i += blockDim.x)
+      sm.tags[i] = HYB_BOUNDS((int64_t)b * kWindow + i, 0, (int64_t)a.B * kWindow) ? a.tag[(int64_t)b * kWindow + i] : -1;
   }
   __syncthreads();
 
@@ -208,7 +198,7 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
   {
     const int hh = threadIdx.x >> 5;        // 0..3
     const int d0 = lane * 8;
-    const int p = a.pos ? a.pos[b] : qseq;
+    const int p = a.pos ? (HYB_BOUNDS(b, 0, a.B) ? a.pos[b] : 0) : qseq;
     uint4 qx = *reinterpret_cast<const uint4*>(a.q + (int64_t)b * a.q_stride + (int64_t)(kvh * kGroup + hh) * kD + d0);
     const uint32_t xs[4] = {qx.x, qx.y, qx.z, qx.w};
     uint32_t ys[4];
@@ -469,10 +459,12 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
       if (lane == 0) sm.cl_lse[hh] = lse;
     } else {
       const int64_t row = ((int64_t)b * kHq + hq) * a.n_splits + split;
-      float4* dst = reinterpret_cast<float4*>(a.part_o + row * kD + d0);
-      dst[0] = make_float4(res[0], res[1], res[2], res[3]);
-      dst[1] = make_float4(res[4], res[5], res[6], res[7]);
-      if (lane == 0) a.part_lse[row] = lse;
+      if (HYB_BOUNDS(row, 0, (int64_t)a.B * kHq * a.n_splits)) {
+        float4* dst = reinterpret_cast<float4*>(a.part_o + row * kD + d0);
+        dst[0] = make_float4(res[0], res[1], res[2], res[3]);
+        dst[1] = make_float4(res[4], res[5], res[6], res[7]);
+        if (lane == 0) a.part_lse[row] = lse;
+      }
     }
   }
   }
@@ -503,7 +495,9 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
       float r8[8];
 #pragma unroll
       for (int e = 0; e < 8; ++e) r8[e] = den > 0.f ? acc[e] / den : 0.f;
-      if (a.out_o != nullptr) {
+      if (!HYB_BOUNDS(orow, 0, (int64_t)a.B * kHq)) {
+        // debug build: a row outside the output, skipped
+      } else if (a.out_o != nullptr) {
         float4* dst = reinterpret_cast<float4*>(a.out_o + orow * kD + d0);
         dst[0] = make_float4(r8[0], r8[1], r8[2], r8[3]);
         dst[1] = make_float4(r8[4], r8[5], r8[6], r8[7]);
@@ -633,6 +627,7 @@ cudaError_t launch_decode(bool full, const DecodeHost& h, cudaStream_t st) {
   a.part_o = h.part_o;
   a.part_lse = h.part_lse;
   a.n_splits = h.n_splits;
+  a.B = h.B;
   a.pm = h.pm;
   // sliding layers (at most 8 splits of a 512-slot ring): the splits of one
   // (sequence, KV head) run as a cluster and merge in its CTA 0, no second

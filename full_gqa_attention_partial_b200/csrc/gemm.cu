@@ -25,6 +25,13 @@
 // accumulator at the row's position before the single rounding to bf16.
 // The (cos, sin) of each (row, frequency) come from a table computed once
 // per call (rope_table_kernel), shared by the row's 20 q and k heads.
+//
+// Optional second output group: columns n_main .. N - 1 (n_main a multiple
+// of the 256-wide tile) take their W rows from a second matrix (tm_w2, from
+// its row 0) and go to a second output (y2, column 0 on): the gate
+// projection's 16 rows ride in q_k_v_proj's launch as one more column tile
+// (rows past the second matrix read as zeros), instead of a launch of their
+// own.
 #include "common.cuh"
 #include "launch.h"
 
@@ -55,6 +62,9 @@ static_assert(sizeof(GemmSmem) + 1024 <= 232448, "GEMM shared memory exceeds 227
 struct GemmArgs {
   __nv_bfloat16* y;
   int64_t ldy;
+  __nv_bfloat16* y2;   // columns >= n_main (second output group), or unused
+  int64_t ldy2;
+  int n_main;
   int M, N, K;
   int tiles_n, n_tiles;
   // RoPE epilogue: row m is token m % T of sequence m / T, at position
@@ -82,14 +92,19 @@ __device__ __forceinline__ void store_cols32(const float (&v)[32], uint8_t* stg,
     const int rw = rr + 8 * q;
     const int row = row0 + rw, col = col0 + 8 * ch;
     const uint4 val = *reinterpret_cast<const uint4*>(stg + rw * 64 + 16 * (ch ^ ((rw >> 1) & 3)));
-    if (row < g.M && col < g.N) *reinterpret_cast<uint4*>(g.y + (int64_t)row * g.ldy + col) = val;
+    if (row < g.M && col < g.N) {
+      __nv_bfloat16* dst = col < g.n_main ? g.y + (int64_t)row * g.ldy + col
+                                          : g.y2 + (int64_t)row * g.ldy2 + (col - g.n_main);
+      *reinterpret_cast<uint4*>(dst) = val;
+    }
   }
   __syncwarp();
 }
 
 template <int ROPE>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
-    gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w, GemmArgs g) {
+    gemm_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_w,
+                const __grid_constant__ CUtensorMap tm_w2, GemmArgs g) {
   extern __shared__ uint8_t smem_raw[];
   GemmSmem& sm = *reinterpret_cast<GemmSmem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -126,16 +141,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(kGThreads, 1)
       // ======================= TMA producer (both CTAs) =======================
       prefetch_tmap(&tm_x);
       prefetch_tmap(&tm_w);
+      if (g.n_main < g.N) prefetch_tmap(&tm_w2);
       uint32_t it = 0;   // stages filled so far
       bool ok = true;
       for (int t = pair0; ok && t < g.n_tiles; t += n_pairs) {
         const int mt = t / g.tiles_n, nt = t % g.tiles_n;
+        const bool second = nt * kGN >= g.n_main;   // a column tile of the second group
+        const CUtensorMap* wmap = second ? &tm_w2 : &tm_w;
+        const int wrow = (second ? nt * kGN - g.n_main : nt * kGN) + (int)rank * (kGN / 2);
         for (int kb = 0; kb < k_blocks; ++kb, ++it) {
           const int s = it % kGStages;
           if (it >= kGStages && !(ok = mbar_wait(&sm.empty[s], ((it / kGStages) - 1) & 1))) break;
           if (rank == 0) mbar_arrive_expect_tx(&sm.full[s], 4 * kGHalf);
           tma_load_2d_pair(smem_u32(sm.x[s]), &tm_x, &sm.full[s], kb * kGK, mt * 2 * kGM + (int)rank * kGM);
-          tma_load_2d_pair(smem_u32(sm.w[s]), &tm_w, &sm.full[s], kb * kGK, nt * kGN + (int)rank * (kGN / 2));
+          tma_load_2d_pair(smem_u32(sm.w[s]), wmap, &sm.full[s], kb * kGK, wrow);
         }
       }
       if (rank == 0)   // every load of the pair completes on CTA 0's barriers
@@ -248,6 +267,10 @@ cudaError_t launch_gemm(const GemmHost& h, cudaStream_t st) {
   GemmArgs g;
   g.y = reinterpret_cast<__nv_bfloat16*>(h.y);
   g.ldy = h.ldy;
+  g.y2 = reinterpret_cast<__nv_bfloat16*>(h.y2);
+  g.ldy2 = h.ldy2;
+  g.n_main = h.n_main > 0 ? h.n_main : h.N;
+  if (g.n_main < h.N && (g.n_main % kGN != 0 || h.y2 == nullptr)) return cudaErrorInvalidValue;
   g.M = h.M;
   g.N = h.N;
   g.K = h.K;
@@ -262,11 +285,11 @@ cudaError_t launch_gemm(const GemmHost& h, cudaStream_t st) {
   if (h.rope != 0 && h.rot == nullptr) return cudaErrorInvalidValue;
   const long long grid = 2 * (n_tiles < h.n_pairs ? n_tiles : h.n_pairs);
   if (h.rope == 1)
-    gemm_kernel<1><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, g);
+    gemm_kernel<1><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, h.tm_w2, g);
   else if (h.rope == 2)
-    gemm_kernel<2><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, g);
+    gemm_kernel<2><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, h.tm_w2, g);
   else
-    gemm_kernel<0><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, g);
+    gemm_kernel<0><<<(unsigned)grid, kGThreads, gemm_smem_bytes(), st>>>(h.tm_x, h.tm_w, h.tm_w2, g);
   count_launch();
   return cudaGetLastError();
 }

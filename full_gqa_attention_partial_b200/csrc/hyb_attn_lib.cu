@@ -4,4 +4,5 @@
 #include "decode.cu"
 #include "prefill.cu"
 #include "gemm.cu"
+#include "smallm.cu"
 #include "api.cu"

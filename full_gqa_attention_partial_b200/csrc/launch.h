@@ -100,6 +100,12 @@ struct GemmHost {
   CUtensorMap tm_x, tm_w;      // 2-D maps {K, rows}, 64 x 128 boxes, 128B swizzle
   void* y = nullptr;           // bf16 [M][ldy]
   int64_t ldy = 0;
+  // second output group: columns [n_main, N) from tm_w2's rows 0 .. into y2
+  // (n_main a multiple of 256); n_main = 0: none
+  CUtensorMap tm_w2;
+  void* y2 = nullptr;
+  int64_t ldy2 = 0;
+  int n_main = 0;
   int M = 0, N = 0, K = 0;
   int n_pairs = 74;            // persistent CTA pairs (SMs / 2)
   // RoPE epilogue: 0 none, 1 sliding-layer, 2 full-layer rotation of the
@@ -109,6 +115,26 @@ struct GemmHost {
   const void* rot = nullptr;
 };
 cudaError_t launch_gemm(const GemmHost& h, cudaStream_t st);
+
+// ---- few-row projections (smallm.cu) ------------------------------------------
+// y[M][ldy] = x[M][ldx] w[N][ldw]^T for M <= 16, K a multiple of 512 up to
+// 4096; features n_main .. N - 1 (n_main > 0) from w2's rows into y2.
+struct SmallMHost {
+  const void* x = nullptr;
+  int64_t ldx = 0;
+  const void* w = nullptr;
+  int64_t ldw = 0;
+  const void* w2 = nullptr;
+  int64_t ldw2 = 0;
+  void* y = nullptr;
+  int64_t ldy = 0;
+  void* y2 = nullptr;
+  int64_t ldy2 = 0;
+  int n_main = 0, M = 0, N = 0, K = 0;
+  bool early_w = false;   // the kernel launched just before on the stream does not write w / w2
+};
+bool smallm_supported(int M, int N, int K, int n_main);
+cudaError_t launch_smallm(const SmallMHost& h, cudaStream_t st);
 cudaError_t gemm_set_smem_attr();
 int gemm_box_rows();   // rows of X or W per TMA box
 int gemm_box_k();      // K elements per TMA box

@@ -708,7 +708,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
       const int row = it.m0 + r;
       const bool valid = row < a.T;
       const int qseq = it.qb + row;
-      const int p_base = a.pos ? a.pos[(int64_t)it.b * a.T + it.m0] : it.qb + it.m0;
+      const int64_t pidx = (int64_t)it.b * a.T + it.m0;
+      const int p_base = a.pos ? (HYB_BOUNDS(pidx, 0, (int64_t)a.B * a.T) ? a.pos[pidx] : 0) : it.qb + it.m0;
       const int p = a.pos ? (valid ? a.pos[(int64_t)it.b * a.T + row] : 0) : qseq;
       const int delta = p - p_base;
       const bool in_table = __all_sync(0xffffffffu, delta >= 0 && delta < kBM);
@@ -857,7 +858,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
       const bool valid = row < a.T;
       const int qseq = it.qb + row;
       // the row's gate score, loaded now so that its latency is not on the epilogue's path
-      const float gscore = (a.gate != nullptr && valid) ? __bfloat162float(a.gate[((int64_t)it.b * a.T + row) * kHq + h]) : 0.f;
+      const int64_t gidx = ((int64_t)it.b * a.T + row) * kHq + h;
+      const float gscore = (a.gate != nullptr && valid && HYB_BOUNDS(gidx, 0, (int64_t)a.B * a.T * kHq))
+                               ? __bfloat162float(a.gate[gidx]) : 0.f;
 
       // ---- online softmax over this warpgroup's keys of each tile ----
       float l_run = 0.f, b_run = -INFINITY;   // running sum (this warpgroup's keys) and the row's base

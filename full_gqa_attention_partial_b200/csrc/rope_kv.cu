@@ -147,6 +147,7 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
     } else {
       dst_row = a.dst_row_offset + t;
     }
+    if (!HYB_BOUNDS(dst_row, 0, a.dst_rows)) continue;   // debug build: a row outside the destination
     int64_t row_id = ((int64_t)b * kHkv + kvh) * a.dst_rows + dst_row;   // row of the [..][4][rows] layout
     if (a.mode == kDstLinear && a.pm.page != 0) {
       int prow, ppage;
@@ -250,7 +251,8 @@ __global__ void __launch_bounds__(128) ring_gather_kernel(const __nv_bfloat16* r
     const int L = len[b];
     const int seq = L - P + r;
     const int slot = ((head[b] - L + seq) % kWindow + kWindow) % kWindow;
-    const bool ok = seq >= 0 && tag[(int64_t)b * kWindow + slot] == seq;
+    const bool ok = seq >= 0 && HYB_BOUNDS(slot, 0, kWindow) && tag[(int64_t)b * kWindow + slot] == seq;
+    if (!HYB_BOUNDS(r, 0, ctx_rows)) continue;   // debug build: a row outside the context buffer
     const int64_t dst = (((int64_t)b * kHkv + kvh) * ctx_rows + r) * kD + d0;
     uint4 kx = make_uint4(0, 0, 0, 0), vx = make_uint4(0, 0, 0, 0);
     if (ok) {

@@ -74,6 +74,8 @@ typedef enum {
 #define HYB_DEV_ERR_TIMEOUT 2   /* a pipeline wait exceeded its limit: output invalid */
 #define HYB_DEV_ERR_PAGE 4      /* a block-table entry outside [0, n_pages): the write
                                    is skipped, the read gives zero keys and values */
+#define HYB_DEV_ERR_BOUNDS 8    /* debug build only (hyb_build_flags): an index outside
+                                   its buffer; the access is skipped */
 
 /*
  * KV cache of one layer for `batch` sequences.  All buffers are caller-owned
@@ -306,6 +308,10 @@ hyb_status hyb_device_error(int32_t* flags, int32_t clear, void* stream);
  * fp32 accumulation; y is rounded to bf16 once.  N, K, ldx, ldw, ldy must be
  * multiples of 8 and the pointers 16-byte aligned (HYB_ESHAPE / HYB_EALIGN
  * otherwise, checked before any launch).  Asynchronous on `stream`.
+ * A few rows (M <= 16, K a multiple of 512 up to 4096: the projections of a
+ * decode step) run on a kernel that streams W across every SM (split-K in
+ * thread-block clusters) instead of the tiled tensor-core GEMM; the
+ * result is the same up to fp32 summation order.
  */
 hyb_status hyb_linear(const void* x, int64_t ldx, const void* w, int64_t ldw, void* y, int64_t ldy, int32_t M,
                       int32_t N, int32_t K, void* stream);
@@ -372,6 +378,18 @@ const char* hyb_last_error(void);
 
 /* Number of kernels this library has launched in the process so far. */
 uint64_t hyb_launch_count(void);
+
+/*
+ * How this copy of the library was built (host only, needs no device):
+ * bit HYB_BUILD_DEBUG_BOUNDS is set in the debug build (compiled with
+ * -DHYB_DEBUG_BOUNDS, shipped beside the normal one as
+ * libhyb_attn_debug.so), whose kernels check the index of every plain
+ * global load and store against its buffer, raise HYB_DEV_ERR_BOUNDS and
+ * skip the access when it falls outside; they never trap.  The normal build
+ * returns 0.
+ */
+#define HYB_BUILD_DEBUG_BOUNDS 1
+int32_t hyb_build_flags(void);
 
 /*
  * Profiling aid.  `events` is a host array of 2 * n_pairs cudaEvent_t handles

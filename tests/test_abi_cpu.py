@@ -44,6 +44,18 @@ def test_library_exports_every_declared_symbol(hyb):
     assert set(_declared_functions()) <= set(hyb.EXPORTED) | {"hyb_last_error"}
 
 
+def test_debug_bounds_build(hyb):
+    """The -DHYB_DEBUG_BOUNDS twin is built beside the library, exports the
+    same boundary and says what it is; the normal build says it is not."""
+    assert os.path.exists(hyb.DEBUG_LIB_PATH)
+    dbg = ctypes.CDLL(hyb.DEBUG_LIB_PATH)
+    for name in _declared_functions():
+        assert hasattr(dbg, name), name
+    dbg.hyb_build_flags.restype = ctypes.c_int32
+    assert dbg.hyb_build_flags() == hyb.BUILD_DEBUG_BOUNDS
+    assert hyb.hyb_build_flags() == 0
+
+
 def _cache(hyb, lt=0, batch=1, cap=512, null_k=False):
     c = hyb._Cache(lt, batch, cap, 0 if null_k else 0x1000, 0x2000, 0x3000, 0x4000, 0x5000)
     return c

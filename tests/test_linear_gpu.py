@@ -1,6 +1,9 @@
 """The projection GEMM (hyb_linear) against the fp64 oracle: ragged M and N
 tiles, a K that is not a multiple of the 64-wide K block, strided rows, the
-model's q_k_v_proj / gate / o_proj shapes."""
+model's q_k_v_proj / gate / o_proj shapes; and the few-row kernel that takes
+M <= 16 with K a multiple of 512 (decode steps): M = 1 .. 16, every
+split-K cluster size from 1 to 8, an N that leaves a partial 32-feature
+block, strided rows and an output view."""
 import numpy as np
 import pytest
 import torch
@@ -69,3 +72,23 @@ def test_linear_rejects_bad_shapes(lib):
     w = torch.zeros(8, 12, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(lib.HybError):
         lib.hyb_linear(x, w)                               # K = 12 is not a multiple of 8
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 512), (3, 40, 1024), (16, 264, 1536), (7, 6144, 2560), (16, 16, 2560),
+                                   (16, 2560, 4096), (5, 96, 3584), (11, 200, 2048)])
+def test_linear_few_rows(lib, M, N, K):
+    x, w = make(M, N, K, seed=7 * M + N + K)
+    y = lib.hyb_linear(x, w)
+    torch.cuda.synchronize()
+    check(y, x, w, f"few-row linear {M}x{N}x{K}")
+    assert lib.hyb_device_error() == 0
+
+
+def test_linear_few_rows_strided_and_view(lib):
+    M, N, K = 12, 72, 1024
+    x, w = make(M, N, K, seed=5, ldx=K + 40)
+    ybuf = torch.full((M, N + 24), 7.0, dtype=torch.bfloat16, device="cuda")
+    lib.hyb_linear(x, w, out=ybuf[:, :N])
+    torch.cuda.synchronize()
+    check(ybuf[:, :N], x, w, "strided few-row linear")
+    assert torch.all(ybuf[:, N:] == 7.0)
