@@ -427,6 +427,10 @@ __device__ __forceinline__ float4 ld_cluster_f32x4(uint32_t addr) {
                : "memory");
   return v;
 }
+// Stores to the shared memory of another CTA of the cluster.
+__device__ __forceinline__ void st_cluster_f32x2(uint32_t addr, float x, float y) {
+  asm volatile("st.shared::cluster.v2.f32 [%0], {%1, %2};" ::"r"(addr), "f"(x), "f"(y) : "memory");
+}
 // Orders this thread's earlier memory writes before its later ones for every
 // thread of the cluster.
 __device__ __forceinline__ void fence_cluster() { asm volatile("fence.acq_rel.cluster;" ::: "memory"); }

@@ -11,8 +11,10 @@
 // K columns [512 r, 512 r + 512) of those 32 rows of W (32 KB) straight
 // into registers (16-byte loads, 64 contiguous bytes per row per four
 // lanes), multiplies them by X's 16 x 512 slice from shared memory with
-// mma.sync m16n8k16 (each warp 8 features), and CTA 0 of the cluster sums
-// the S partial tiles through distributed shared memory and writes Y.  When
+// mma.sync m16n8k16 (each warp 8 features); every CTA stores its partial
+// tile into CTA 0's shared memory (distributed shared memory, plain stores),
+// and after one cluster barrier CTA 0 sums the S tiles in rank order (the
+// result does not depend on timing) and writes Y.  When
 // the caller knows that the kernel launched just before does not write W
 // (o_proj after the library's own attention), W's loads are issued before
 // the wait for that kernel, so the weight stream overlaps its tail.
@@ -33,6 +35,7 @@ constexpr int kSmmFeat = 8 * kSmmWarps;   // output features per cluster
 constexpr int kSmmK = 512;                // K columns per CTA
 constexpr int kSmmChunks = kSmmK / 32;    // 32-wide K chunks per CTA
 constexpr int kSmmPad = 8;                // X row padding (elements)
+constexpr int kSmmMaxS = 8;               // cluster size limit (portable)
 
 struct SmallMArgs {
   const __nv_bfloat16* x;
@@ -57,9 +60,9 @@ __device__ __forceinline__ uint4 ld_stream_v4(const void* p) {
   return v;
 }
 
-__global__ void __launch_bounds__(32 * kSmmWarps) smallm_kernel(SmallMArgs a) {
+__global__ void __launch_bounds__(32 * kSmmWarps, 5) smallm_kernel(SmallMArgs a) {
   __shared__ __align__(16) __nv_bfloat16 xs[16][kSmmK + kSmmPad];
-  __shared__ float part[16][kSmmFeat];
+  __shared__ __align__(16) float part[kSmmMaxS][16][kSmmFeat];   // CTA 0's: the partial tile of every rank
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int g = lane >> 2, t = lane & 3;
   const int rank = blockIdx.x % a.S;        // the cluster's CTAs are consecutive in x
@@ -81,12 +84,19 @@ __global__ void __launch_bounds__(32 * kSmmWarps) smallm_kernel(SmallMArgs a) {
   if (a.early_w) pdl_wait();   // X comes from the previous kernel
   pdl_launch_dependents();
 
-  // ---- X's 16 x 512 slice (rows past M are zero) ----
-  for (int i = threadIdx.x; i < 16 * (kSmmK / 8); i += blockDim.x) {
+  // ---- X's 16 x 512 slice (rows past M are zero): every load in flight at once ----
+  constexpr int kXPer = 16 * (kSmmK / 8) / (32 * kSmmWarps);
+  uint4 xv[kXPer];
+#pragma unroll
+  for (int j = 0; j < kXPer; ++j) {
+    const int i = threadIdx.x + j * 32 * kSmmWarps;
     const int m = i / (kSmmK / 8), c8 = i % (kSmmK / 8);
-    uint4 v = make_uint4(0, 0, 0, 0);
-    if (m < a.M) v = *reinterpret_cast<const uint4*>(a.x + (int64_t)m * a.ldx + k0 + 8 * c8);
-    *reinterpret_cast<uint4*>(&xs[m][8 * c8]) = v;
+    xv[j] = m < a.M ? *reinterpret_cast<const uint4*>(a.x + (int64_t)m * a.ldx + k0 + 8 * c8) : make_uint4(0, 0, 0, 0);
+  }
+#pragma unroll
+  for (int j = 0; j < kXPer; ++j) {
+    const int i = threadIdx.x + j * 32 * kSmmWarps;
+    *reinterpret_cast<uint4*>(&xs[i / (kSmmK / 8)][8 * (i % (kSmmK / 8))]) = xv[j];
   }
   __syncthreads();
 
@@ -102,31 +112,30 @@ __global__ void __launch_bounds__(32 * kSmmWarps) smallm_kernel(SmallMArgs a) {
       mma_16816(acc, lo.x, hi.x, lo.y, hi.y, b0, b1);
     }
   }
-  // acc: rows g and g + 8, features 8 warp + 2 t, + 1
-  part[g][8 * warp + 2 * t] = acc[0];
-  part[g][8 * warp + 2 * t + 1] = acc[1];
-  part[g + 8][8 * warp + 2 * t] = acc[2];
-  part[g + 8][8 * warp + 2 * t + 1] = acc[3];
-  cluster_sync();   // every CTA's partial tile written
+  // acc: rows g and g + 8, features 8 warp + 2 t, + 1 -> CTA 0's part[rank]
+  st_cluster_f32x2(mapa_cluster(smem_u32(&part[rank][g][8 * warp + 2 * t]), 0), acc[0], acc[1]);
+  st_cluster_f32x2(mapa_cluster(smem_u32(&part[rank][g + 8][8 * warp + 2 * t]), 0), acc[2], acc[3]);
+  cluster_sync();   // every rank's tile is in CTA 0 (release / acquire); CTA 0 alone reads on
   if (rank == 0) {
     for (int i = threadIdx.x; i < 16 * kSmmFeat / 2; i += blockDim.x) {
       const int m = i / (kSmmFeat / 2), f = 2 * (i % (kSmmFeat / 2));
       const int nn = n0 + f;
       if (m >= a.M || nn >= a.N) continue;
       float s0 = 0.f, s1 = 0.f;
-      for (int r = 0; r < a.S; ++r) {
-        s0 += ld_cluster_f32(mapa_cluster(smem_u32(&part[m][f]), (uint32_t)r));
-        s1 += ld_cluster_f32(mapa_cluster(smem_u32(&part[m][f + 1]), (uint32_t)r));
+      for (int r = 0; r < a.S; ++r) {   // rank order
+        const float2 v = *reinterpret_cast<const float2*>(&part[r][m][f]);
+        s0 += v.x;
+        s1 += v.y;
       }
       __nv_bfloat16* dst = nn < a.n_main ? a.y + (int64_t)m * a.ldy + nn : a.y2 + (int64_t)m * a.ldy2 + (nn - a.n_main);
       *reinterpret_cast<uint32_t*>(dst) = pack_bf16(s0, s1);
     }
   }
-  cluster_sync();   // the other CTAs' partials stay until CTA 0 has read them
 }
 
 bool smallm_supported(int M, int N, int K, int n_main) {
-  return M >= 1 && M <= 16 && K % kSmmK == 0 && K / kSmmK >= 1 && K / kSmmK <= 8 && N % 8 == 0 && n_main % 2 == 0;
+  return M >= 1 && M <= 16 && K % kSmmK == 0 && K / kSmmK >= 1 && K / kSmmK <= kSmmMaxS && N % 8 == 0 &&
+         n_main % 2 == 0;
 }
 
 cudaError_t launch_smallm(const SmallMHost& h, cudaStream_t st) {
