@@ -100,15 +100,15 @@ def layer_seed(base: int, i: int) -> int:
 # capture of the kernel as it was when its sources hashed to `sha`.  Reported as
 # roofline.traffic only while the sources are unchanged; otherwise null.
 TRAFFIC = {
-    "prefill_full_T32768": {"bytes": 2.0848e9, "sha": "7418b33196f3016d",
+    "prefill_full_T32768": {"bytes": 2.2168e9, "sha": "9e5b86665813accc",
                             "sources": ["prefill.cu", "common.cuh"]},
-    "prefill_sliding_T32768": {"bytes": 0.6417e9, "sha": "7418b33196f3016d",
+    "prefill_sliding_T32768": {"bytes": 0.6386e9, "sha": "9e5b86665813accc",
                                "sources": ["prefill.cu", "common.cuh"]},
     # captured at 16 x 32768 tokens; decode streams each cached byte once, so
     # traffic scales with the tokens: x 8590491648 / 2147483648
-    "decode_full_B16_L131072": {"bytes": 2.1536e9 * 8590491648 / 2147483648, "sha": "4683e5d0426bd89b",
+    "decode_full_B16_L131072": {"bytes": 2.1608e9 * 8590491648 / 2147483648, "sha": "11dc48abfcd17baa",
                                 "sources": ["decode.cu", "common.cuh"]},
-    "decode_fp8_full_B16_L131072": {"bytes": 1.0961e9 * 8590491648 / 2147483648, "sha": "4683e5d0426bd89b",
+    "decode_fp8_full_B16_L131072": {"bytes": 1.1053e9 * 8590491648 / 2147483648, "sha": "11dc48abfcd17baa",
                                     "sources": ["decode.cu", "common.cuh"]},
 }
 
@@ -908,14 +908,29 @@ def run_case(hyb, args):
     """One kernel on a small configuration, for profiler captures: 1 warm-up + args.steps launches."""
     from full_gqa_attention_partial_b200 import synth
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    if args.case == "linear_qkv":
-        M, N, K = args.seq * args.batch, 6144, 2560
+    if args.case in ("linear_qkv", "linear_decode"):
+        # q_k_v_proj's shape: M = seq x batch rows (tiled GEMM), or M = batch rows (a decode
+        # step: the few-row kernel, rated by the weight bytes it streams)
+        M, N, K = (args.seq * args.batch if args.case == "linear_qkv" else args.batch), 6144, 2560
         g = torch.Generator(device="cuda").manual_seed(5)
         x = torch.randn(M, K, generator=g, device="cuda").to(torch.bfloat16)
         w = (torch.randn(N, K, generator=g, device="cuda") / K ** 0.5).to(torch.bfloat16)
         y = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
         fn = lambda: hyb.hyb_linear(x, w, out=y)
-        work = 2 * M * N * K
+        work, unit = (2 * M * N * K, "TFLOP/s") if args.case == "linear_qkv" else (N * K * 2, "GB/s")
+    elif args.case == "prefill_full_fp8":
+        # a full layer's prefill of seq tokens into an empty FP8 cache (the length is reset
+        # before each call, so every launch does the same work)
+        T, B = args.seq, args.batch
+        x = synth.prefill_inputs(B, T, seed=layer_seed(1, 3), device="cuda")
+        c = hyb.KVCache(FULL, B, capacity=T + (-T) % 4, kv_dtype=hyb.KV_FP8)
+        ws = hyb.alloc_workspace(hyb.hyb_attn_prefill_cache_workspace_size(c, T))
+        out = torch.empty(B, T, H, D, dtype=torch.bfloat16, device="cuda")
+
+        def fn():
+            c.len.zero_()
+            hyb.hyb_attn_prefill(x["q"], x["k"], x["v"], x["gate"], x["pos"], FULL, out=out, cache=c, workspace=ws)
+        work = B * flops(T, FULL)
         unit = "TFLOP/s"
     elif args.case.startswith("prefill"):
         lt = FULL if args.case == "prefill_full" else SLIDING
@@ -942,7 +957,7 @@ def run_case(hyb, args):
         unit = "GB/s"
     fn()
     torch.cuda.synchronize()
-    if args.case == "linear_qkv":   # one kernel per call: events around the calls
+    if args.case.startswith("linear"):   # one kernel per call: events around the calls
         ev0.record()
         for _ in range(args.steps):
             fn()
@@ -978,8 +993,9 @@ def main():
                     help="also run the 1M-token decode with the full layers' history spread over the ranks")
     ap.add_argument("--cpu-rows", type=int, default=24, help="oracle rows per layer for cpu_baseline")
     ap.add_argument("--ref-rows", type=int, default=8, help="oracle rows per layer per reference step")
-    ap.add_argument("--case", choices=["prefill_full", "prefill_sliding", "decode_full", "decode_sliding", "decode_full_fp8",
-                                       "decode_sliding_fp8", "linear_qkv"],
+    ap.add_argument("--case", choices=["prefill_full", "prefill_sliding", "prefill_full_fp8", "decode_full",
+                                       "decode_sliding", "decode_full_fp8", "decode_sliding_fp8", "linear_qkv",
+                                       "linear_decode"],
                     default=None, help="time one kernel on a small configuration (profiling)")
     ap.add_argument("--seq", type=int, default=16384)
     ap.add_argument("--batch", type=int, default=1)

@@ -52,14 +52,14 @@
 //
 // FP8 (e4m3) full-layer caches (one fp32 scale per key row and KV head) are
 // read in place.  S = Q K^T runs on the tensor cores' e4m3 path
-// (kind::f8f6f4) straight from the K codes, which TMA loads into four 16 KB
+// (kind::f8f6f4) straight from the K codes, which TMA loads into a ring of 16 KB
 // entries: the query tile is split into two e4m3 tiles, Q_hi (each element
 // rounded, after a power-of-two factor per row that puts the row's largest
 // element in [128, 256)) and Q_lo (the remainder, rounded), and S is their
 // two MMA passes into one accumulator -- the tensor time of one bf16 pass, and
 // at most 2^-8 of each query element left out (a single e4m3 query tile, at
 // 2^-4, would not meet the accuracy bound).  V feeds O += P V in bf16: its
-// codes land in the upper half of one of two 32 KB V slots and two converter
+// codes land in the upper half of one of the 32 KB V slots and two converter
 // warps (12 warps in all) widen them in place by integer bit moves (value x
 // 2^-120, exact; three instructions for two codes).  The row scales never touch the operands: TMA
 // loads them into a four-tile ring, the softmax multiplies the scores by the
@@ -87,8 +87,9 @@ constexpr int kMmaWarp = 9;
 constexpr int kConvWarp = 10;             // FP8: converter warps 10 and 11
 constexpr int kSlots = 4;                 // operand ring: 4 x 32 KB
 constexpr int kCodeBytes = 16384;         // FP8: one CTA's codes of a K or V tile
-constexpr int kNKc = 4;                   // FP8: K code entries (16 KB) in slots 0-1
-constexpr int kNV = 2;                    // FP8: V slots (slots 2-3), codes land in the upper half
+constexpr int kNKc = 2;                   // FP8: K code entries (16 KB, two per slot) in the first slots
+constexpr int kVSlot0 = kNKc / 2;         // FP8: the V slots follow them ...
+constexpr int kNV = kSlots - kVSlot0;     // ... codes land in a V slot's upper half
 constexpr int kNF = 4;                    // FP8: K / V row-scale ring (tiles)
 template <bool FP8> struct PfCfg {
   static constexpr int kThreads = FP8 ? 384 : 320;
@@ -104,7 +105,7 @@ __device__ __forceinline__ uint32_t col_s(uint32_t sb) { return 128u * sb; }
 template <bool FULL, bool FP8>
 struct PfSmem {
   static constexpr int R = RopeCfg<FULL>::R;
-  // 1024-byte aligned; FP8: slots 0-1 hold four 16 KB K code entries, slots 2-3 the V tiles
+  // 1024-byte aligned; FP8: the first kVSlot0 slots hold the 16 KB K code entries, the rest the V tiles
   uint8_t slot[kSlots][kSlotBytes];
   uint8_t qo[4][16384];              // the query tile (4 boxes of 64 dims x 128 rows), rotated in place:
                                      // the A operand of S = Q K^T
@@ -435,7 +436,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
                 const int v = jt % kNV;
                 if (jt >= kNV && !(ok = mbar_wait(&sm.vempty[v], ((jt / kNV) - 1) & 1))) break;
                 mbar_arrive_expect_tx(&sm.vcode[v], kCodeBytes);
-                const uint32_t dst = smem_u32(sm.slot[2 + v]) + kCodeBytes;
+                const uint32_t dst = smem_u32(sm.slot[kVSlot0 + v]) + kCodeBytes;
 #pragma unroll
                 for (int h = 0; h < 2; ++h) {
                   coord(r0 + kHalfKeys * h, row, page);
@@ -546,7 +547,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
         const uint32_t jt = J + tile;
         const int v = jt % kNV;
         if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.vcode[v], (jt / kNV) & 1)))) break;
-        uint8_t* dst = sm.slot[2 + v];
+        uint8_t* dst = sm.slot[kVSlot0 + v];
         const uint8_t* sp = dst + kCodeBytes + sb * 8192 + rq * 128;
         // 64-dim chunk q / 4, key 64 sb + 4 i + rq
         uint8_t* dp = dst + (q >> 2) * 16384 + (64 * sb + rq) * 128;
@@ -611,9 +612,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
             const uint32_t jt = J + tile;   // global tile index
             const uint32_t sb = jt % kNS;
             // the operand's slot: bf16, the load ring; FP8, K entry jt % 4 or V slot 2 + jt % 2
-            const int slot = !FP8 ? (int)(g % kSlots) : is_k ? (int)(jt % kNKc) : 2 + (int)(jt % kNV);
+            const int slot = !FP8 ? (int)(g % kSlots) : is_k ? (int)(jt % kNKc) : kVSlot0 + (int)(jt % kNV);
             if (FP8 && !is_k) {
-              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.vready[slot - 2], (jt / kNV) & 1)))) break;
+              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.vready[slot - kVSlot0], (jt / kNV) & 1)))) break;
             } else {
               const uint32_t ph = FP8 ? (jt / kNKc) & 1 : (g / kSlots) & 1;
               if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], ph)))) break;
@@ -659,7 +660,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
                 mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 64 * (s >> 2) + 8 * (s & 3), bdesc, idesc_o,
                                  (tile > 0 || s > 0) ? 1u : 0u);
               }
-              mma_commit_pair_warp(FP8 ? &sm.vempty[slot - 2] : &sm.empty[slot]);
+              mma_commit_pair_warp(FP8 ? &sm.vempty[slot - kVSlot0] : &sm.empty[slot]);
               mma_commit_pair_warp(&sm.o_done[sb]);
               if (tile == it.n - 1) mma_commit_pair_warp(&sm.o_final);
             }
