@@ -17,7 +17,7 @@
 // warp, at about 40 cycles per MMA and a few hundred per barrier wait, could
 // not keep the tensor pipe fed.
 //
-// Roles in each CTA (320 threads):
+// Roles in each CTA (320 threads; sliding layers 448, FP8 caches 384):
 //   warps 0-7  two softmax warpgroups.  Both own the tile's 128 query rows
 //              (warp w reads TMEM lanes 32 (w % 4) ..); warpgroup g takes
 //              keys [64 g, 64 g + 64) of every key tile.  A row's maximum
@@ -37,7 +37,12 @@
 //              prefetch of the next item's);
 //   warp 9     tensor-memory allocation (both CTAs); in CTA 0 the warp runs
 //              the MMA loop convergently and one elected lane issues every
-//              MMA of the pair and commits to both CTAs.
+//              MMA of the pair and commits to both CTAs;
+//   warps 10-13 (sliding layers) the epilogue: a sliding item is only ~5 key
+//              tiles, so the softmax warps hand over the row sums and start
+//              the next item while these drain the output (the softmax warps
+//              fit in the 128 registers 14 warps leave);
+//   warps 10-11 (FP8 caches) converters (below).
 // Tensor memory, per CTA (512 columns x 128 lanes of 32 bit):
 //   [0,256)   two S buffers (fp32, 128 keys each); P of a tile (bf16 pairs)
 //             overwrites the first 32 columns of each warpgroup's 64 and is
@@ -91,8 +96,12 @@ constexpr int kNKc = 2;                   // FP8: K code entries (16 KB, two per
 constexpr int kVSlot0 = kNKc / 2;         // FP8: the V slots follow them ...
 constexpr int kNV = kSlots - kVSlot0;     // ... codes land in a V slot's upper half
 constexpr int kNF = 4;                    // FP8: K / V row-scale ring (tiles)
-template <bool FP8> struct PfCfg {
-  static constexpr int kThreads = FP8 ? 384 : 320;
+constexpr int kEpiWarp0 = 10;             // sliding layers: epilogue warps 10-13
+template <bool FULL, bool FP8> struct PfCfg {
+  // sliding layers: four warps of their own take each item's epilogue, so the
+  // softmax warps start the next item at once (an item is only ~5 key tiles)
+  static constexpr bool kEpi = !FULL && !FP8;
+  static constexpr int kThreads = FP8 ? 384 : (kEpi ? 448 : 320);
 };
 constexpr float kTwo120 = 1.329227995784916e36f;    // 2^120
 constexpr int kNS = 2;                    // S buffers in tensor memory
@@ -209,8 +218,11 @@ __device__ __forceinline__ float2 fmul2(float2 a, float2 b) {
   return d;
 }
 
-// Load order shared by the K/V producer and the MMA issuer: step s (0 <= s
-// < n + kAhead) loads K_s if s < n, then V_{s - kAhead} if 0 <= s - kAhead < n.
+// Load order shared by the K/V producer and the MMA issuer, item by item: K of
+// tile t + 1 before V of tile t (S of the next tile is issued before P.V of
+// this one), the item's last V last.  (Taking the next item's first K before
+// the current item's last V was measured slower on sliding layers: the last
+// P.V then waits for the next query tile's load, and the epilogue with it.)
 
 // Rotates 2 NW dims [k0, k0 + 2 NW) against their partners [k0 + R/2, ...)
 // for one query row: x1 / x2 hold NW packed bf16 words each; results replace
@@ -309,7 +321,7 @@ __device__ __forceinline__ int item_index(int k, int pair, int n_pairs, int n_it
 // registers each): with 10 (12 for FP8) warps a sub-partition holds three,
 // so a thread may use at most 168 registers.
 template <bool FULL, bool FP8>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FULL, FP8>::kThreads, 1)
     prefill_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                    const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_o,
                    const __grid_constant__ CUtensorMap tm_ks, const __grid_constant__ CUtensorMap tm_vs, PfArgs a) {
@@ -347,7 +359,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
       mbar_init(&sm.o_done[s], 1);
     }
     mbar_init(&sm.o_final, 1);
-    mbar_init(&sm.o_free, 2 * kSmWarps);
+    mbar_init(&sm.o_free, 2 * (PfCfg<FULL, FP8>::kEpi ? 4 : kSmWarps));
     mbar_init(&sm.mma_done, 1);
     mbar_init(&sm.q_full, 1);
     mbar_init(&sm.q_free, 1);
@@ -378,14 +390,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
         prefetch_tmap(&tm_vs);
       }
       uint32_t g = 0;   // loads issued so far by this CTA (bf16)
-      uint32_t J = 0;   // tiles of earlier items (FP8 loads are numbered by tile)
       uint32_t nk = 0, nf = 0, nv = 0;   // FP8: K code, scale and V loads issued (tile index + 1)
       bool ok = true;
-      for (int k = 0; ok; ++k) {
-        const int w = item_index(k, pair0, n_pairs, n_items);
-        if (w == -2) break;
-        if (w < 0) continue;
-        const Item it = item_of<FULL>(w, a);
+      // One load: K (is_k) or V of key tile `tile` of item `it`, whose first tile has the
+      // global index Jb.
+      auto load = [&](const Item& it, uint32_t Jb, int tile, bool is_k) -> bool {
         const int last_row = it.q_hi - it.kb;   // key row of the item's last visible key
         // (row, page) coordinates of the 64 keys from key row r on; a range past the
         // item's last key is read from an out-of-range page (zeros) instead of
@@ -398,76 +407,82 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
             kv_coord(a.pm, it.b, r, row, page);
           }
         };
-        for (int st = 0; ok && st < it.n + kAhead; ++st) {
-#pragma unroll 1
-          for (int part = 0; part < 2; ++part) {
-            const bool is_k = part == 0;
-            const int tile = is_k ? st : st - kAhead;
-            if (tile < 0 || tile >= it.n) continue;
-            const int r0 = (it.j_lo + tile) * kBN;   // key row of the tile's first key
-            int row, page;
-            if constexpr (FP8) {
-              const uint32_t jt = J + tile;
-              if (is_k) {
-                // this CTA's 64 keys (codes, dims [0, 128) and [128, 256)) into K entry
-                // jt % 4, bytes counted on CTA 0's barrier; then the row scales of all
-                // 128 keys (every softmax row needs them) into this CTA's scale ring
-                const int e = jt % kNKc;
-                if (jt >= kNKc && !(ok = mbar_wait(&sm.empty[e], ((jt / kNKc) - 1) & 1))) break;
-                if (rank == 0) mbar_arrive_expect_tx(&sm.full[e], 2 * kCodeBytes);
-                const uint32_t dst = smem_u32(sm.slot[0]) + e * kCodeBytes;
-                coord(r0 + kHalfKeys * (int)rank, row, page);
+        const int r0 = (it.j_lo + tile) * kBN;   // key row of the tile's first key
+        int row, page;
+        if constexpr (FP8) {
+          const uint32_t jt = Jb + tile;
+          if (is_k) {
+            // this CTA's 64 keys (codes, dims [0, 128) and [128, 256)) into K entry
+            // jt % 4, bytes counted on CTA 0's barrier; then the row scales of all
+            // 128 keys (every softmax row needs them) into this CTA's scale ring
+            const int e = jt % kNKc;
+            if (jt >= kNKc && !(ok = mbar_wait(&sm.empty[e], ((jt / kNKc) - 1) & 1))) return false;
+            if (rank == 0) mbar_arrive_expect_tx(&sm.full[e], 2 * kCodeBytes);
+            const uint32_t dst = smem_u32(sm.slot[0]) + e * kCodeBytes;
+            coord(r0 + kHalfKeys * (int)rank, row, page);
 #pragma unroll
-                for (int c = 0; c < 2; ++c) tma_load_4d_pair(dst + c * 8192, &tm_k, &sm.full[e], 128 * c, row, it.kvh, page);
-                nk = jt + 1;
-                const int fe = jt % kNF;
-                if (jt >= kNF && !(ok = mbar_wait(&sm.f_free[fe], ((jt / kNF) - 1) & 1))) break;
-                mbar_arrive_expect_tx(&sm.f_full[fe], 2 * kBN * 4);
+            for (int c = 0; c < 2; ++c) tma_load_4d_pair(dst + c * 8192, &tm_k, &sm.full[e], 128 * c, row, it.kvh, page);
+            nk = jt + 1;
+            const int fe = jt % kNF;
+            if (jt >= kNF && !(ok = mbar_wait(&sm.f_free[fe], ((jt / kNF) - 1) & 1))) return false;
+            mbar_arrive_expect_tx(&sm.f_full[fe], 2 * kBN * 4);
 #pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                  coord(r0 + kHalfKeys * h, row, page);
-                  tma_load_3d(smem_u32(&sm.kf[fe][kHalfKeys * h]), &tm_ks, &sm.f_full[fe], row, it.kvh, page);
-                  tma_load_3d(smem_u32(&sm.vf[fe][kHalfKeys * h]), &tm_vs, &sm.f_full[fe], row, it.kvh, page);
-                }
-                nf = jt + 1;
-              } else {
-                // the tile's 128 keys of this CTA's 128 dims (codes) into the upper half of
-                // V slot jt % 2, once the slot's last P.V has completed
-                const int v = jt % kNV;
-                if (jt >= kNV && !(ok = mbar_wait(&sm.vempty[v], ((jt / kNV) - 1) & 1))) break;
-                mbar_arrive_expect_tx(&sm.vcode[v], kCodeBytes);
-                const uint32_t dst = smem_u32(sm.slot[kVSlot0 + v]) + kCodeBytes;
-#pragma unroll
-                for (int h = 0; h < 2; ++h) {
-                  coord(r0 + kHalfKeys * h, row, page);
-                  tma_load_4d(dst + h * 8192, &tm_v, &sm.vcode[v], 128 * (int)rank, row, it.kvh, page);
-                }
-                nv = jt + 1;
-              }
-              continue;
+            for (int h = 0; h < 2; ++h) {
+              coord(r0 + kHalfKeys * h, row, page);
+              tma_load_3d(smem_u32(&sm.kf[fe][kHalfKeys * h]), &tm_ks, &sm.f_full[fe], row, it.kvh, page);
+              tma_load_3d(smem_u32(&sm.vf[fe][kHalfKeys * h]), &tm_vs, &sm.f_full[fe], row, it.kvh, page);
             }
-            const int slot = g % kSlots;
-            if (g >= kSlots && !(ok = mbar_wait(&sm.empty[slot], ((g / kSlots) - 1) & 1))) break;
-            if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
-            const uint32_t dst = smem_u32(sm.slot[slot]);
-            if (is_k) {   // this CTA's 64 keys, 4 boxes of 64 dims
-              coord(r0 + kHalfKeys * (int)rank, row, page);
+            nf = jt + 1;
+          } else {
+            // the tile's 128 keys of this CTA's 128 dims (codes) into the upper half of
+            // V slot jt % 2, once the slot's last P.V has completed
+            const int v = jt % kNV;
+            if (jt >= kNV && !(ok = mbar_wait(&sm.vempty[v], ((jt / kNV) - 1) & 1))) return false;
+            mbar_arrive_expect_tx(&sm.vcode[v], kCodeBytes);
+            const uint32_t dst = smem_u32(sm.slot[kVSlot0 + v]) + kCodeBytes;
 #pragma unroll
-              for (int box = 0; box < 4; ++box)
-                tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row, it.kvh, page);
-            } else {      // all 128 keys of this CTA's 128 dims: 2 dim chunks x 2 key halves
-#pragma unroll
-              for (int h = 0; h < 2; ++h) {
-                coord(r0 + kHalfKeys * h, row, page);
-#pragma unroll
-                for (int d = 0; d < 2; ++d)
-                  tma_load_4d_pair(dst + d * kVChunk + h * kKBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * d,
-                                   row, it.kvh, page);
-              }
+            for (int h = 0; h < 2; ++h) {
+              coord(r0 + kHalfKeys * h, row, page);
+              tma_load_4d(dst + h * 8192, &tm_v, &sm.vcode[v], 128 * (int)rank, row, it.kvh, page);
             }
-            ++g;
+            nv = jt + 1;
+          }
+          return true;
+        }
+        const int slot = g % kSlots;
+        if (g >= kSlots && !(ok = mbar_wait(&sm.empty[slot], ((g / kSlots) - 1) & 1))) return false;
+        if (rank == 0) mbar_arrive_expect_tx(&sm.full[slot], 2 * kSlotBytes);
+        const uint32_t dst = smem_u32(sm.slot[slot]);
+        if (is_k) {   // this CTA's 64 keys, 4 boxes of 64 dims
+          coord(r0 + kHalfKeys * (int)rank, row, page);
+#pragma unroll
+          for (int box = 0; box < 4; ++box)
+            tma_load_4d_pair(dst + box * kKBox, &tm_k, &sm.full[slot], box * 64, row, it.kvh, page);
+        } else {      // all 128 keys of this CTA's 128 dims: 2 dim chunks x 2 key halves
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            coord(r0 + kHalfKeys * h, row, page);
+#pragma unroll
+            for (int d = 0; d < 2; ++d)
+              tma_load_4d_pair(dst + d * kVChunk + h * kKBox, &tm_v, &sm.full[slot], 128 * (int)rank + 64 * d,
+                               row, it.kvh, page);
           }
         }
+        ++g;
+        return true;
+      };
+      // in the order the MMA issuer consumes the loads
+      uint32_t J = 0;   // tiles of earlier items
+      for (int k = 0; ok; ++k) {
+        const int w = item_index(k, pair0, n_pairs, n_items);
+        if (w == -2) break;
+        if (w < 0) continue;
+        const Item it = item_of<FULL>(w, a);
+        for (int t = 0; ok && t < it.n; ++t) {
+          if (!(ok = load(it, J, t, true))) break;
+          if (t > 0) ok = load(it, J, t - 1, false);
+        }
+        if (ok) ok = load(it, J, it.n - 1, false);
         J += it.n;
       }
       // no copy left landing in shared memory at exit (the pair's loads complete on
@@ -593,86 +608,161 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
       const uint64_t qdesc = smem_desc_sw128(smem_u32(sm.qo[0]), 16, 1024);          // Q, K-major
       const uint64_t kdesc0 = smem_desc_sw128(smem_u32(sm.slot[0]), 16, 1024);       // K in slot 0, K-major
       const uint64_t vdesc0 = smem_desc_sw128(smem_u32(sm.slot[0]), kVChunk, 1024);  // V in slot 0, MN-major
-      uint32_t g = 0, J = 0;
-      int item = 0;
+      uint32_t g = 0;
       bool ok = true;
+      // One operation: S = Q K^T (is_k) or O += P V of key tile `tile` of item `it`
+      // (the pair's ino-th item, whose first tile has the global index Jb).
+      auto issue = [&](const Item& it, int ino, uint32_t Jb, int tile, bool is_k) -> bool {
+        if (is_k && tile == 0) {   // the item's query tile is ready
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.q_ready, ino & 1))) return false;
+          tc_fence_after();
+        }
+        const uint32_t jt = Jb + tile;   // global tile index
+        const uint32_t sb = jt % kNS;
+        // the operand's slot: bf16, the load ring; FP8, K entry jt % 4 or V slot 2 + jt % 2
+        const int slot = !FP8 ? (int)(g % kSlots) : is_k ? (int)(jt % kNKc) : kVSlot0 + (int)(jt % kNV);
+        if (FP8 && !is_k) {
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.vready[slot - kVSlot0], (jt / kNV) & 1))) return false;
+        } else {
+          const uint32_t ph = FP8 ? (jt / kNKc) & 1 : (g / kSlots) & 1;
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.full[slot], ph))) return false;
+        }
+        tc_fence_after();
+        if (is_k) {
+          if constexpr (FP8) {
+            // Q_hi K^T then Q_lo K^T into the same accumulator: 32 dims per MMA; the
+            // 128 dims of dim block d are Q_hi in qo[2 d], Q_lo in qo[2 d + 1], and
+            // codes [128 d, 128 d + 128) of the K entry's 64 keys in its box d
+            const uint64_t kdesc = desc_advance(kdesc0, slot * kCodeBytes);
+#pragma unroll
+            for (int s = 0; s < 2 * kD / 32; ++s) {
+              const int s2 = s & 7;
+              const uint64_t adesc = desc_advance(qdesc, (s2 >> 2) * 32768 + (s >> 3) * 16384 + (s2 & 3) * 32);
+              const uint64_t bdesc = desc_advance(kdesc, (s2 >> 2) * 8192 + (s2 & 3) * 32);
+              mma_ss_pair_e4m3_warp(tmem + col_s(sb), adesc, bdesc, idesc_s, s > 0 ? 1u : 0u);
+            }
+          } else {
+            const uint64_t kdesc = desc_advance(kdesc0, slot * kSlotBytes);
+#pragma unroll
+            for (int s = 0; s < kD / 16; ++s) {
+              const uint64_t adesc = desc_advance(qdesc, (s >> 2) * 16384 + (s & 3) * 32);
+              const uint64_t bdesc = desc_advance(kdesc, (s >> 2) * kKBox + (s & 3) * 32);
+              mma_ss_pair_warp(tmem + col_s(sb), adesc, bdesc, idesc_s, s > 0 ? 1u : 0u);
+            }
+          }
+          mma_commit_pair_warp(&sm.empty[slot]);
+          mma_commit_pair_warp(&sm.s_full[sb]);
+          if (tile == it.n - 1) mma_commit_pair_warp(&sm.q_free);   // qo is no longer read
+        } else {
+          // the item's first P.V overwrites O: the previous item's epilogue must have read it
+          if (tile == 0 && ino > 0 &&
+              !__all_sync(0xffffffffu, mbar_wait(&sm.o_free, (ino - 1) & 1)))
+            return false;
+          if (!__all_sync(0xffffffffu, mbar_wait(&sm.p_full[sb], (jt / kNS) & 1))) return false;
+          tc_fence_after();
+          const uint64_t vdesc = desc_advance(vdesc0, slot * kSlotBytes);
+#pragma unroll
+          for (int s = 0; s < kBN / 16; ++s) {
+            // keys [16 s, 16 s + 16): P of warpgroup s / 4 at its columns 64 (s / 4) + 8 (s % 4)
+            const uint64_t bdesc = desc_advance(vdesc, s * 16 * 128);
+            mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 64 * (s >> 2) + 8 * (s & 3), bdesc, idesc_o,
+                             (tile > 0 || s > 0) ? 1u : 0u);
+          }
+          mma_commit_pair_warp(FP8 ? &sm.vempty[slot - kVSlot0] : &sm.empty[slot]);
+          mma_commit_pair_warp(&sm.o_done[sb]);
+          if (tile == it.n - 1) mma_commit_pair_warp(&sm.o_final);
+        }
+        ++g;
+        return true;
+      };
+      // in the producer's load order
+      uint32_t J = 0;
+      int item = 0;
       for (int k = 0; ok; ++k) {
         const int w = item_index(k, pair0, n_pairs, n_items);
         if (w == -2) break;
         if (w < 0) continue;
         const Item it = item_of<FULL>(w, a);
-        if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.q_ready, item & 1)))) break;
-        tc_fence_after();
-        for (int st = 0; ok && st < it.n + kAhead; ++st) {
-#pragma unroll 1
-          for (int part = 0; part < 2; ++part) {
-            const bool is_k = part == 0;
-            const int tile = is_k ? st : st - kAhead;
-            if (tile < 0 || tile >= it.n) continue;
-            const uint32_t jt = J + tile;   // global tile index
-            const uint32_t sb = jt % kNS;
-            // the operand's slot: bf16, the load ring; FP8, K entry jt % 4 or V slot 2 + jt % 2
-            const int slot = !FP8 ? (int)(g % kSlots) : is_k ? (int)(jt % kNKc) : kVSlot0 + (int)(jt % kNV);
-            if (FP8 && !is_k) {
-              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.vready[slot - kVSlot0], (jt / kNV) & 1)))) break;
-            } else {
-              const uint32_t ph = FP8 ? (jt / kNKc) & 1 : (g / kSlots) & 1;
-              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.full[slot], ph)))) break;
-            }
-            tc_fence_after();
-            if (is_k) {
-              if constexpr (FP8) {
-                // Q_hi K^T then Q_lo K^T into the same accumulator: 32 dims per MMA; the
-                // 128 dims of dim block d are Q_hi in qo[2 d], Q_lo in qo[2 d + 1], and
-                // codes [128 d, 128 d + 128) of the K entry's 64 keys in its box d
-                const uint64_t kdesc = desc_advance(kdesc0, slot * kCodeBytes);
-#pragma unroll
-                for (int s = 0; s < 2 * kD / 32; ++s) {
-                  const int s2 = s & 7;
-                  const uint64_t adesc = desc_advance(qdesc, (s2 >> 2) * 32768 + (s >> 3) * 16384 + (s2 & 3) * 32);
-                  const uint64_t bdesc = desc_advance(kdesc, (s2 >> 2) * 8192 + (s2 & 3) * 32);
-                  mma_ss_pair_e4m3_warp(tmem + col_s(sb), adesc, bdesc, idesc_s, s > 0 ? 1u : 0u);
-                }
-              } else {
-                const uint64_t kdesc = desc_advance(kdesc0, slot * kSlotBytes);
-#pragma unroll
-                for (int s = 0; s < kD / 16; ++s) {
-                  const uint64_t adesc = desc_advance(qdesc, (s >> 2) * 16384 + (s & 3) * 32);
-                  const uint64_t bdesc = desc_advance(kdesc, (s >> 2) * kKBox + (s & 3) * 32);
-                  mma_ss_pair_warp(tmem + col_s(sb), adesc, bdesc, idesc_s, s > 0 ? 1u : 0u);
-                }
-              }
-              mma_commit_pair_warp(&sm.empty[slot]);
-              mma_commit_pair_warp(&sm.s_full[sb]);
-              if (tile == it.n - 1) mma_commit_pair_warp(&sm.q_free);   // qo is no longer read
-            } else {
-              // the item's first P.V overwrites O: the previous item's epilogue must have read it
-              if (tile == 0 && item > 0 &&
-                  !(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_free, (item - 1) & 1))))
-                break;
-              if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.p_full[sb], (jt / kNS) & 1)))) break;
-              tc_fence_after();
-              const uint64_t vdesc = desc_advance(vdesc0, slot * kSlotBytes);
-#pragma unroll
-              for (int s = 0; s < kBN / 16; ++s) {
-                // keys [16 s, 16 s + 16): P of warpgroup s / 4 at its columns 64 (s / 4) + 8 (s % 4)
-                const uint64_t bdesc = desc_advance(vdesc, s * 16 * 128);
-                mma_ts_pair_warp(tmem + kColO, tmem + col_s(sb) + 64 * (s >> 2) + 8 * (s & 3), bdesc, idesc_o,
-                                 (tile > 0 || s > 0) ? 1u : 0u);
-              }
-              mma_commit_pair_warp(FP8 ? &sm.vempty[slot - kVSlot0] : &sm.empty[slot]);
-              mma_commit_pair_warp(&sm.o_done[sb]);
-              if (tile == it.n - 1) mma_commit_pair_warp(&sm.o_final);
-            }
-            ++g;
-          }
+        for (int t = 0; ok && t < it.n; ++t) {
+          if (!(ok = issue(it, item, J, t, true))) break;
+          if (t > 0) ok = issue(it, item, J, t - 1, false);
         }
+        if (ok) ok = issue(it, item, J, it.n - 1, false);
         J += it.n;
         ++item;
       }
       // also on an early exit: wait until nothing the pair issued is in flight
       mma_commit_pair_warp(&sm.mma_done);
       mbar_wait(&sm.mma_done, 0);
+    }
+  } else if (PfCfg<FULL, FP8>::kEpi && warp >= kEpiWarp0) {
+    // ======================= epilogue warps (sliding layers: warps 10-13, both CTAs) =======================
+    // Warp w reads TMEM lanes 32 (w % 4) ..: O / l * sigmoid(gate) -> bf16 ->
+    // global for its 32 rows, all 256 dims, 32 dims at a time through its
+    // staging area (64-byte swizzle) and a TMA store, then frees O for the
+    // next item's first P.V.  l is the sum of both softmax warpgroups' sums.
+    // Items in the same order as the other roles; xsum and o_final of an item
+    // cannot advance again before this warp has freed O (the next item's
+    // first P.V waits for it, and every later tile of the pair after that).
+    const int qtr = warp & 3;
+    const int r = qtr * 32 + lane;
+    const uint32_t trow = tmem + ((uint32_t)(qtr * 32) << 16);
+    uint8_t* const stg = sm.ostage[warp - kEpiWarp0];
+    int item = 0;
+    bool ok = true;
+    for (int k = 0; ok; ++k) {
+      const int w = item_index(k, pair0, n_pairs, n_items);
+      if (w == -2) break;
+      if (w < 0) continue;
+      const Item it = item_of<FULL>(w, a);
+      const int h = it.h_pair0 + (int)rank;
+      const int row = it.m0 + r;
+      const int64_t gidx = ((int64_t)it.b * a.T + row) * kHq + h;
+      const float gscore = (a.gate != nullptr && row < a.T && HYB_BOUNDS(gidx, 0, (int64_t)a.B * a.T * kHq))
+                               ? __bfloat162float(a.gate[gidx]) : 0.f;
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.xsum_full, item & 1)))) break;
+      const float l = sm.xsum[item & 1][0][r] + sm.xsum[item & 1][1][r];   // both at the row's final base
+      if (!(ok = __all_sync(0xffffffffu, mbar_wait(&sm.o_final, item & 1)))) break;
+      tc_fence_after();
+      float f = l > 0.f ? 1.f / l : 0.f;
+      if (a.gate != nullptr) f *= 1.f / (1.f + __expf(-gscore));
+      const float2 f2 = make_float2(f, f);
+      uint32_t ov[32], on[32];
+      tmem_ld32(trow + kColO, on);
+#pragma unroll 1
+      for (int c = 0; c < kD / 32; ++c) {
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 32; ++e) ov[e] = on[e];
+        if (c < kD / 32 - 1) tmem_ld32(trow + kColO + 32 * (c + 1), on);   // next chunk in flight
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t w4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int cc = 8 * q4 + 2 * e;
+            const float2 o = fmul2(make_float2(__uint_as_float(ov[cc]), __uint_as_float(ov[cc + 1])), f2);
+            w4[e] = pack_bf16(o.x, o.y);
+          }
+          *reinterpret_cast<uint4*>(stg + lane * 64 + 16 * (q4 ^ ((lane >> 1) & 3))) =
+              make_uint4(w4[0], w4[1], w4[2], w4[3]);
+        }
+        fence_proxy_async();   // the staging writes, then the TMA engine's read of them
+        __syncwarp();
+        if (lane == 0) {
+          tma_store_4d(&tm_o, smem_u32(stg), 32 * c, h, it.m0 + 32 * qtr, it.b);
+          tma_store_commit();
+          tma_store_wait_read();   // the staging area is free again
+        }
+        __syncwarp();
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) {
+        if (rank == 0) mbar_arrive(&sm.o_free);
+        else mbar_arrive_remote(&sm.o_free, 0);
+      }
+      ++item;
     }
   } else {
     // ======================= softmax / epilogue (warps 0-7) =======================
@@ -860,7 +950,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
       const int qseq = it.qb + row;
       // the row's gate score, loaded now so that its latency is not on the epilogue's path
       const int64_t gidx = ((int64_t)it.b * a.T + row) * kHq + h;
-      const float gscore = (a.gate != nullptr && valid && HYB_BOUNDS(gidx, 0, (int64_t)a.B * a.T * kHq))
+      const float gscore = (!PfCfg<FULL, FP8>::kEpi && a.gate != nullptr && valid &&
+                            HYB_BOUNDS(gidx, 0, (int64_t)a.B * a.T * kHq))
                                ? __bfloat162float(a.gate[gidx]) : 0.f;
 
       // ---- online softmax over this warpgroup's keys of each tile ----
@@ -989,6 +1080,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
       if (have_next && (!a.q_rotated || FP8) && !(ok = prepare_q(nxt, item + 1))) break;
       const float rs_next = q_row_scale;
 
+      if constexpr (!PfCfg<FULL, FP8>::kEpi) {
       // ---- epilogue: O / l * sigmoid(gate) -> bf16 -> global, this warpgroup's 128 dims ----
       // 32 dims at a time through the warp's staging area: each thread writes
       // its row of 64 bytes, 16-byte chunk q at chunk q ^ ((row / 2) % 4) (no bank
@@ -1035,6 +1127,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
       tc_fence_before();
       __syncwarp();
       arrive_cta0(&sm.o_free);
+      }
       it = nxt;
       have = have_next;
       rs = rs_next;
@@ -1042,7 +1135,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FP8>::kThreads
     }
   }
 
-  if (warp < kSmWarps && lane == 0) tma_store_commit_and_wait();   // epilogue stores complete
+  if ((warp < kSmWarps || (PfCfg<FULL, FP8>::kEpi && warp >= kEpiWarp0)) && lane == 0)
+    tma_store_commit_and_wait();   // epilogue stores complete
   // the peer's shared memory and tensor memory stay alive until both CTAs are done
   tc_fence_before();
   __syncthreads();
@@ -1074,13 +1168,13 @@ cudaError_t launch_prefill(bool full, const PrefillHost& h, cudaStream_t st) {
   const long long grid = 2 * (n_items < h.n_pairs ? n_items : h.n_pairs);   // persistent CTA pairs
   profile_before(st);
   if (full && h.fp8)
-    prefill_kernel<true, true><<<(unsigned)grid, PfCfg<true>::kThreads, prefill_smem_bytes_t<true, true>(), st>>>(
+    prefill_kernel<true, true><<<(unsigned)grid, PfCfg<true, true>::kThreads, prefill_smem_bytes_t<true, true>(), st>>>(
         h.tm_k, h.tm_v, h.tm_q, h.tm_o, h.tm_ks, h.tm_vs, a);
   else if (full)
-    prefill_kernel<true, false><<<(unsigned)grid, PfCfg<false>::kThreads, prefill_smem_bytes_t<true>(), st>>>(
+    prefill_kernel<true, false><<<(unsigned)grid, PfCfg<true, false>::kThreads, prefill_smem_bytes_t<true>(), st>>>(
         h.tm_k, h.tm_v, h.tm_q, h.tm_o, h.tm_k, h.tm_v, a);
   else
-    prefill_kernel<false, false><<<(unsigned)grid, PfCfg<false>::kThreads, prefill_smem_bytes_t<false>(), st>>>(
+    prefill_kernel<false, false><<<(unsigned)grid, PfCfg<false, false>::kThreads, prefill_smem_bytes_t<false>(), st>>>(
         h.tm_k, h.tm_v, h.tm_q, h.tm_o, h.tm_k, h.tm_v, a);
   profile_after(st);
   count_launch();
