@@ -21,7 +21,7 @@ The JSON line also carries:
   layer_prefill the 4-layer group as whole layers (projections + attention);
   decode_1m     36-layer decode at 1M tokens: tokens/s (and decode_1m_fp8
                 over e4m3 caches);
-  decode_1m_sharded (by default with several ranks, else --decode-sharded) the same with the full
+  decode_1m_sharded (by default, every rank; --quick skips it) the same with the full
                 layers' history spread over the ranks;
   chunked_prefill 262144 tokens in 8192-token chunks, 36 layers (and
                 chunked_prefill_fp8 over e4m3 caches; these and the 1M decode
@@ -78,7 +78,11 @@ def targets_summary(extras: dict, roofline: dict) -> dict:
                             "frac_of_hbm": d["frac_of_hbm"], "target": 0.70}
     d8 = extras.get("decode_1m_fp8")
     if d8:
-        out["decode_1m_fp8"] = {"tokens_per_s": d8["tokens_per_s"], "frac_of_hbm": d8["frac_of_hbm"]}
+        out["decode_1m_fp8"] = {"tokens_per_s": d8["tokens_per_s"], "frac_of_hbm": d8["frac_of_hbm"],
+                                "frac_of_measured_copy": d8["frac_of_measured_copy"]}
+    ds = extras.get("decode_1m_sharded")
+    if ds:
+        out["decode_1m_sharded"] = {"tokens_per_s": ds["tokens_per_s"], "frac_of_hbm_per_gpu": ds["frac_of_hbm_per_gpu"]}
     return out
 
 
@@ -769,9 +773,14 @@ def bench_decode_1m_sharded(hyb, args, peaks, d):
     ms = d.max(ev0.elapsed_time(ev1) / n_steps)
     kv = statistics.mean(9 * 4096 * (L0 + i + 1) + d.world * 27 * 4096 * W for i in range(n_steps))
     del fulls, rings, decs
+    per_gpu = kv / (ms / 1e3) / 1e9 / d.world
     return {"workload": f"36 layers, 9 full caches ~1M over {d.world} GPU(s), 27 rings each, B=1, 64 steps",
             "tokens_per_s": 1e3 / ms, "ms_per_step": ms, "kv_gb_per_s": kv / (ms / 1e3) / 1e9,
-            "frac_of_hbm_per_gpu": kv / (ms / 1e3) / 1e9 / HBM_READ_GBS / d.world}
+            "frac_of_hbm_per_gpu": per_gpu / HBM_READ_GBS,
+            # the step is bound by each GPU streaming its share of the caches
+            "roofline": {"bound": "hbm", "achieved": per_gpu, "peak": HBM_READ_GBS, "unit": "GB/s",
+                         "frac": per_gpu / HBM_READ_GBS, "frac_of_measured_copy": per_gpu / peaks["hbm_gbs"],
+                         "bytes_per_step_per_gpu": kv / d.world, "ms_per_step": ms}}
 
 
 def bench_chunked(hyb, args, peaks, fp8: bool = False):
@@ -1045,9 +1054,9 @@ def main():
             extras["chunked_prefill"] = run("chunked_prefill", bench_chunked, hyb, args, peaks)
             torch.cuda.empty_cache()
             extras["chunked_prefill_fp8"] = run("chunked_prefill_fp8", bench_chunked, hyb, args, peaks, fp8=True)
-    # with several ranks the sequence-sharded 1M decode runs by default (every rank
-    # takes part: it has collectives)
-    if (args.decode_sharded or dist.world > 1) and not args.no_extras:
+    # the sequence-sharded 1M decode runs by default (with one rank: the partial + merge
+    # path over the whole history; every rank takes part: it has collectives)
+    if (args.decode_sharded or args.decode_1m or dist.world > 1) and not args.no_extras:
         torch.cuda.empty_cache()
         extras["decode_1m_sharded"] = run("decode_1m_sharded", bench_decode_1m_sharded, hyb, args, peaks, dist)
     clk = clocks.stop()
