@@ -97,14 +97,17 @@ def test_layer_rejects_bad_weight_shape(lib):
         lib.hyb_attn_layer_prefill(h, w_qkv[:, :2048].contiguous(), w_gate, w_o, None, O.FULL)
 
 
+@pytest.mark.parametrize("B", [3, 20])
 @pytest.mark.parametrize("lt", [O.SLIDING, O.FULL])
-def test_layer_decode_steps(lib, lt):
+def test_layer_decode_steps(lib, lt, B):
     """Three decode steps of the layer over a seeded cache (history snapshot
     taken before any library call on it; the oracle projects and rotates the
-    new tokens itself)."""
+    new tokens itself).  Up to 16 sequences the projections run on the
+    few-row kernel and the append / decode rotate k and q; 20 sequences take
+    the tiled GEMM with RoPE in its epilogue."""
     import bench
     from full_gqa_attention_partial_b200 import synth
-    B, L, n_steps = 3, 1500, 3
+    L, n_steps = 1500, 3
     w_qkv, w_gate, w_o = weights(50 + lt)
     if lt == O.FULL:
         cap = L + n_steps
