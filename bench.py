@@ -104,9 +104,9 @@ def layer_seed(base: int, i: int) -> int:
 # capture of the kernel as it was when its sources hashed to `sha`.  Reported as
 # roofline.traffic only while the sources are unchanged; otherwise null.
 TRAFFIC = {
-    "prefill_full_T32768": {"bytes": 2.1617e9, "sha": "812f57e496e4d88a",
+    "prefill_full_T32768": {"bytes": 2.2145e9, "sha": "316cb8c86943c256",
                             "sources": ["prefill.cu", "common.cuh"]},
-    "prefill_sliding_T32768": {"bytes": 0.6418e9, "sha": "812f57e496e4d88a",
+    "prefill_sliding_T32768": {"bytes": 0.6381e9, "sha": "316cb8c86943c256",
                                "sources": ["prefill.cu", "common.cuh"]},
     # captured at 16 x 32768 tokens; decode streams each cached byte once, so
     # traffic scales with the tokens: x 8590491648 / 2147483648
