@@ -61,9 +61,11 @@
 // entries: the query tile is split into two e4m3 tiles, Q_hi (each element
 // rounded, after a power-of-two factor per row that puts the row's largest
 // element in [128, 256)) and Q_lo (the remainder, rounded), and S is their
-// two MMA passes into one accumulator -- the tensor time of one bf16 pass, and
-// at most 2^-8 of each query element left out (a single e4m3 query tile, at
-// 2^-4, would not meet the accuracy bound).  V feeds O += P V in bf16: its
+// two MMA passes into one accumulator -- the tensor time of one bf16 pass.  A
+// bf16 element has 8 significant bits and each part 4, so the split gives back
+// every element of at least 2^-9 of its row's largest exactly and the rest
+// within 2^-17 of the largest (a single e4m3 query tile would not meet the
+// accuracy bound).  V feeds O += P V in bf16: its
 // codes land in the upper half of one of the 32 KB V slots and two converter
 // warps (12 warps in all) widen them in place by integer bit moves (value x
 // 2^-120, exact; three instructions for two codes).  The row scales never touch the operands: TMA
@@ -863,9 +865,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(PfCfg<FULL, FP8>::kT
         // The row as Q_hi + Q_lo, both e4m3, for the e4m3 keys: every element times
         // 2^(7 - e), where 2^e <= the row's largest |element| < 2^(e + 1) (found over
         // both warpgroups' halves of the row), so that the largest lies in [128, 256);
-        // Q_hi is an element rounded to e4m3, Q_lo the remainder rounded to e4m3,
-        // which leaves out at most 2^-8 of the element (bf16 rounding: 2^-9).  This
-        // warpgroup's 16 chunks of 8 dims for the maximum include every dim it rotated.
+        // Q_hi is an element rounded to e4m3, Q_lo the remainder rounded to e4m3:
+        // for the tile's bf16 values that is exact down to 2^-9 of the row's largest
+        // (8 significant bits = 4 + 4), below within 2^-17 of it.  This warpgroup's
+        // 16 chunks of 8 dims for the maximum include every dim it rotated.
         auto chunk_of = [&](int i) { return i < 4 ? 2 * wg + (i & 1) + 4 * (i >> 1) : 8 + 12 * wg + (i - 4); };
         float am = 0.f;
 #pragma unroll 4
