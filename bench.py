@@ -101,27 +101,33 @@ def layer_seed(base: int, i: int) -> int:
 
 
 # DRAM bytes per launch (dram__bytes_read.sum + dram__bytes_write.sum) from one ncu
-# capture of the kernel as it was when its sources hashed to `sha`.  Reported as
-# roofline.traffic only while the sources are unchanged; otherwise null.
+# capture of the kernel as it was when its sources (comments aside) hashed to `sha`.
+# Reported as roofline.traffic only while the sources are unchanged; otherwise null.
 TRAFFIC = {
-    "prefill_full_T32768": {"bytes": 2.2145e9, "sha": "316cb8c86943c256",
+    "prefill_full_T32768": {"bytes": 2.2145e9, "sha": "8161c7d06d6219b4",
                             "sources": ["prefill.cu", "common.cuh"]},
-    "prefill_sliding_T32768": {"bytes": 0.6381e9, "sha": "316cb8c86943c256",
+    "prefill_sliding_T32768": {"bytes": 0.6381e9, "sha": "8161c7d06d6219b4",
                                "sources": ["prefill.cu", "common.cuh"]},
     # captured at 16 x 32768 tokens; decode streams each cached byte once, so
     # traffic scales with the tokens: x 8590491648 / 2147483648
-    "decode_full_B16_L131072": {"bytes": 2.1608e9 * 8590491648 / 2147483648, "sha": "11dc48abfcd17baa",
+    "decode_full_B16_L131072": {"bytes": 2.1608e9 * 8590491648 / 2147483648, "sha": "0f19a04d16f7b81c",
                                 "sources": ["decode.cu", "common.cuh"]},
-    "decode_fp8_full_B16_L131072": {"bytes": 1.1053e9 * 8590491648 / 2147483648, "sha": "11dc48abfcd17baa",
+    "decode_fp8_full_B16_L131072": {"bytes": 1.1053e9 * 8590491648 / 2147483648, "sha": "0f19a04d16f7b81c",
                                     "sources": ["decode.cu", "common.cuh"]},
 }
 
 
 def kernel_sources_sha(files) -> str:
+    """Hash of the kernel sources with comments and whitespace taken out (a comment
+    edit leaves the kernel, and its traffic, as they were)."""
     import hashlib
+    import re
     d = hashlib.sha256()
     for f in files:
-        d.update(open(os.path.join(ROOT, "full_gqa_attention_partial_b200", "csrc", f), "rb").read())
+        src = open(os.path.join(ROOT, "full_gqa_attention_partial_b200", "csrc", f), encoding="utf-8").read()
+        src = re.sub(r"/\*.*?\*/", " ", src, flags=re.S)
+        src = re.sub(r"//[^\n]*", " ", src)
+        d.update(" ".join(src.split()).encode())
     return d.hexdigest()[:16]
 
 
