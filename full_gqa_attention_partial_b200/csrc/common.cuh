@@ -247,6 +247,13 @@ __device__ __forceinline__ uint32_t e4m3_b01_bf16x2(uint32_t w) { return e4m3_pa
 __device__ __forceinline__ uint32_t e4m3_b23_bf16x2(uint32_t w) { return e4m3_pair_bf16x2<0xB3A2u>(w); }
 __device__ __forceinline__ uint32_t e4m3_b02_bf16x2(uint32_t w) { return e4m3_pair_bf16x2<0xA280u>(w); }
 __device__ __forceinline__ uint32_t e4m3_b13_bf16x2(uint32_t w) { return e4m3_pair_bf16x2<0xB391u>(w); }
+// The same for one code of each of two words a and b (the permute numbers
+// a's bytes 0-3 and b's 4-7): e.g. 0xC480 gives (a byte 0, b byte 0), so a
+// pair of codes from two key rows costs no extra permute.
+template <uint32_t SEL>
+__device__ __forceinline__ uint32_t e4m3_pair2_bf16x2(uint32_t a, uint32_t b) {
+  return (prmt(a, b, SEL) << 4) & 0x87F087F0u;
+}
 // Two floats -> two e4m3 codes (lo in the low byte), round to nearest even, saturating.
 __device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float lo, float hi) {
   uint16_t h;

@@ -355,12 +355,17 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
       m_run[e] = m_new;
       l_part[e] = l_part[e] * alpha[e] + (pv[0][e] + pv[1][e]);
     }
+    // O moves only when a head's maximum grew somewhere in the warp (times 1
+    // otherwise, which changes nothing): past the first stages of a long
+    // history that is rare, and the 64 multiplies are a tenth of a stage's work
+    if (__any_sync(0xffffffffu, alpha[0] != 1.f || alpha[1] != 1.f)) {
 #pragma unroll
-    for (int n = 0; n < 16; ++n) {
-      o[n][0] *= alpha[0];
-      o[n][1] *= alpha[1];
-      o[n][2] *= alpha[0];
-      o[n][3] *= alpha[1];
+      for (int n = 0; n < 16; ++n) {
+        o[n][0] *= alpha[0];
+        o[n][1] *= alpha[1];
+        o[n][2] *= alpha[0];
+        o[n][3] *= alpha[1];
+      }
     }
     // P^T (keys x heads, C layout) -> B fragments (k = keys, n = heads)
     const uint32_t pb0 = movmatrix_t(pack_bf16(pv[0][0] * vsc[0], pv[0][1] * vsc[0]));
@@ -375,14 +380,15 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
                                   {vw[3][u].x, vw[3][u].y, vw[3][u].z, vw[3][u].w}};
 #pragma unroll
         for (int wd = 0; wd < 4; ++wd) {
-          // keys (2q, 2q+1) and (2q+8, 2q+9), dims 4 wd .. 4 wd + 3 of the lane's chunk
-          const uint32_t t0 = prmt(w[0][wd], w[1][wd], 0x5410u), t1 = prmt(w[0][wd], w[1][wd], 0x7632u);
-          const uint32_t t2 = prmt(w[2][wd], w[3][wd], 0x5410u), t3 = prmt(w[2][wd], w[3][wd], 0x7632u);
+          // keys (2q, 2q+1) and (2q+8, 2q+9), dims 4 wd .. 4 wd + 3 of the lane's chunk:
+          // block ib takes dims + 0 (rows r) and + 1 (rows r + 8), block ib + 1 dims + 2 and + 3;
+          // each pair of keys is one code from each of two rows' words
+          const uint32_t w0 = w[0][wd], w1 = w[1][wd], w2 = w[2][wd], w3 = w[3][wd];
           const int ib = 8 * u + 2 * wd;
-          mma_16816(o[ib], e4m3_b02_bf16x2(t0), e4m3_b13_bf16x2(t0), e4m3_b02_bf16x2(t2), e4m3_b13_bf16x2(t2), pb0,
-                    pb1);
-          mma_16816(o[ib + 1], e4m3_b02_bf16x2(t1), e4m3_b13_bf16x2(t1), e4m3_b02_bf16x2(t3),
-                    e4m3_b13_bf16x2(t3), pb0, pb1);
+          mma_16816(o[ib], e4m3_pair2_bf16x2<0xC480u>(w0, w1), e4m3_pair2_bf16x2<0xD591u>(w0, w1),
+                    e4m3_pair2_bf16x2<0xC480u>(w2, w3), e4m3_pair2_bf16x2<0xD591u>(w2, w3), pb0, pb1);
+          mma_16816(o[ib + 1], e4m3_pair2_bf16x2<0xE6A2u>(w0, w1), e4m3_pair2_bf16x2<0xF7B3u>(w0, w1),
+                    e4m3_pair2_bf16x2<0xE6A2u>(w2, w3), e4m3_pair2_bf16x2<0xF7B3u>(w2, w3), pb0, pb1);
         }
       }
     } else {
