@@ -55,25 +55,36 @@ constexpr int kDec8TileBytes = kDecKeys * kD;        // 16 KB of codes
 constexpr int kDec8Box = kDecKeys * 128;             // 128 dims x 64 keys
 constexpr int kDec8StageBytes = 2 * kDec8TileBytes + 2 * kDecKeys * 4 + 512;   // padded to 1 KB multiples
 
+constexpr int kDecClusterMax = 8;   // most splits merged inside a cluster
+
 template <bool FP8>
 struct DecSmem {
   static constexpr int kStages = FP8 ? kDec8Stages : kDecStages;
   static constexpr int kRingBytes = FP8 ? kDec8Stages * kDec8StageBytes : kDecStages * kDecStageBytes;
   // stage ring first (1024-byte aligned base); after the last stage it holds
-  // the warps' partial outputs, float [warp][head][dim]
+  // the warps' partial outputs, float [warp][head][dim], and in CTA 0 of a
+  // cluster, after them, every split's normalised output [split][head][dim]
+  // and base-2 log-sum-exp [split][head]
   uint8_t ring[kRingBytes];
   float merge_m[4][4];
   float merge_l[4][4];
   __nv_bfloat16 qs[4][kD];      // rotated queries of the group
   int32_t tags[kWindow];
-  float cl_o[4][kD];            // cluster merge: this split's normalised output per head ...
-  float cl_lse[4];              // ... and its base-2 log-sum-exp
   uint64_t full[kStages];
   uint64_t empty[kStages];
+  static constexpr int kMergeBytes = 4 * 4 * kD * 4;
+  static constexpr int kGatherBytes = kDecClusterMax * 4 * kD * 4;
   __device__ float (&merge_o())[4][4][kD] { return *reinterpret_cast<float(*)[4][4][kD]>(ring); }
+  __device__ float (&gather_o())[kDecClusterMax][4][kD] {
+    return *reinterpret_cast<float(*)[kDecClusterMax][4][kD]>(ring + kMergeBytes);
+  }
+  __device__ float (&gather_lse())[kDecClusterMax][4] {
+    return *reinterpret_cast<float(*)[kDecClusterMax][4]>(ring + kMergeBytes + kGatherBytes);
+  }
 };
-static_assert(DecSmem<true>::kRingBytes >= 4 * 4 * kD * 4 && DecSmem<false>::kRingBytes >= 4 * 4 * kD * 4,
-              "the ring must hold the merge buffer");
+static_assert(DecSmem<true>::kRingBytes >= DecSmem<true>::kMergeBytes + DecSmem<true>::kGatherBytes + 4 * kDecClusterMax * 4 &&
+                  DecSmem<false>::kRingBytes >= DecSmem<false>::kMergeBytes + DecSmem<false>::kGatherBytes + 4 * kDecClusterMax * 4,
+              "the ring must hold the merge and cluster-gather buffers");
 
 size_t decode_smem_bytes(bool fp8) { return (fp8 ? sizeof(DecSmem<true>) : sizeof(DecSmem<false>)) + 1024; }
 static_assert(2 * (sizeof(DecSmem<true>) + 1024 + 1024) <= 228 * 1024, "two FP8 CTAs must share an SM");
@@ -135,6 +146,7 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
     }
     fence_barrier_init();
   }
+  __syncthreads();   // the barriers are initialised (before the wait: overlaps the previous kernel)
   // the append before this launch writes len, tags and the new token's row
   pdl_wait();
   pdl_launch_dependents();
@@ -147,12 +159,13 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
   const int k0 = split * kps;
   const int k1 = min(n_keys, k0 + kps);
   const int n_stages = (k1 > k0 && L > 0) ? (k1 - k0 + kDecKeys - 1) / kDecKeys : 0;
-  if (!FULL) {
-    for (int i = threadIdx.x; i < kWindow; i += blockDim.x)
-      sm.tags[i] = HYB_BOUNDS((int64_t)b * kWindow + i, 0, (int64_t)a.B * kWindow) ? a.tag[(int64_t)b * kWindow + i] : -1;
-  }
-  __syncthreads();
+  // this split's normalised output (dims 8 lane .. + 7 of head `warp`) and
+  // base-2 log-sum-exp, for the merge inside a cluster
+  float cres[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+  float clse = -INFINITY;
 
+  // The producer issues the first stages as soon as len is known; the
+  // consumers meanwhile load the queries and (ring caches) the slot tags.
   if (warp == 4) {
     // ---------------- producer ----------------
     if (lane == 0 && n_stages > 0) {
@@ -193,6 +206,8 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
       for (int i = max(0, issued - NST); i < issued; ++i)
         mbar_wait(&sm.full[i % NST], (i / NST) & 1);
     }
+    __syncwarp();
+    if (a.cluster_merge) cluster_arrive();   // this CTA's ring takes no more copies
   } else {
   // ---------------- consumers: rotate the group's 4 queries ----------------
   {
@@ -200,6 +215,10 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
     const int d0 = lane * 8;
     const int p = a.pos ? (HYB_BOUNDS(b, 0, a.B) ? a.pos[b] : 0) : qseq;
     uint4 qx = *reinterpret_cast<const uint4*>(a.q + (int64_t)b * a.q_stride + (int64_t)(kvh * kGroup + hh) * kD + d0);
+    if (!FULL) {   // in flight with the query's load
+      for (int i = threadIdx.x; i < kWindow; i += 128)
+        sm.tags[i] = HYB_BOUNDS((int64_t)b * kWindow + i, 0, (int64_t)a.B * kWindow) ? a.tag[(int64_t)b * kWindow + i] : -1;
+    }
     const uint32_t xs[4] = {qx.x, qx.y, qx.z, qx.w};
     uint32_t ys[4];
     constexpr int xor_mask = (R == 256) ? 16 : 4;
@@ -226,7 +245,7 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
     }
     *reinterpret_cast<uint4*>(&sm.qs[hh][d0]) = qx;
   }
-  asm volatile("bar.sync 1, 128;" ::: "memory");
+  asm volatile("bar.sync 1, 128;" ::: "memory");   // queries and tags in shared memory
 
   // Lane (r, q) = (lane / 4, lane % 4) in the m16n8k16 fragment layouts.
   const int r = lane >> 2, q = lane & 3;
@@ -408,6 +427,7 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
   // ---------------- merge the 4 warps, write the split's partial ----------------
   // the merge buffer overlays the ring: every consumer warp must be done with its last stage
   asm volatile("bar.sync 1, 128;" ::: "memory");
+  if (a.cluster_merge) cluster_arrive();   // this CTA is done with its ring
 #pragma unroll
   for (int e = 0; e < 2; ++e) {
     l_part[e] += __shfl_xor_sync(0xffffffffu, l_part[e], 4);
@@ -460,9 +480,9 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
     }
     const int hq = kvh * kGroup + hh;
     if (a.cluster_merge) {   // for CTA 0 of the cluster
-      *reinterpret_cast<float4*>(&sm.cl_o[hh][d0]) = make_float4(res[0], res[1], res[2], res[3]);
-      *reinterpret_cast<float4*>(&sm.cl_o[hh][d0 + 4]) = make_float4(res[4], res[5], res[6], res[7]);
-      if (lane == 0) sm.cl_lse[hh] = lse;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) cres[e] = res[e];
+      clse = lse;
     } else {
       const int64_t row = ((int64_t)b * kHq + hq) * a.n_splits + split;
       if (HYB_BOUNDS(row, 0, (int64_t)a.B * kHq * a.n_splits)) {
@@ -478,22 +498,34 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
   if (a.cluster_merge) {
     // ---------------- merge the cluster's splits in CTA 0 (the log-sum-exp
     // combination of decode_combine_kernel, same order of operations) ----------------
-    cluster_sync();   // every split's result is in its CTA's shared memory
+    // Every CTA of the cluster has arrived once it was done with its ring, so
+    // once the wait returns CTA 0's ring can take every split's result: each
+    // CTA stores its own into CTA 0 (remote stores, no round trips), and after
+    // one more barrier CTA 0 merges from its own shared memory.
+    cluster_wait();
+    if (warp < 4 && HYB_BOUNDS(split, 0, kDecClusterMax)) {
+      const int hh = warp, d0 = lane * 8;
+      st_cluster_f32x4(mapa_cluster(smem_u32(&sm.gather_o()[split][hh][d0]), 0), cres[0], cres[1], cres[2], cres[3]);
+      st_cluster_f32x4(mapa_cluster(smem_u32(&sm.gather_o()[split][hh][d0 + 4]), 0), cres[4], cres[5], cres[6], cres[7]);
+      if (lane == 0) st_cluster_f32(mapa_cluster(smem_u32(&sm.gather_lse()[split][hh]), 0), clse);
+    }
+    cluster_sync();   // every split's result is in CTA 0 (release / acquire)
     if (cluster_ctarank() == 0 && warp < 4) {
       const int hh = warp, d0 = lane * 8;
       const int hq = kvh * kGroup + hh;
       const int64_t orow = (int64_t)b * kHq + hq;
+      const int n_parts = min(a.n_splits, kDecClusterMax);
       float M = -INFINITY;
-      for (int s2 = 0; s2 < a.n_splits; ++s2) M = fmaxf(M, ld_cluster_f32(mapa_cluster(smem_u32(&sm.cl_lse[hh]), s2)));
+      for (int s2 = 0; s2 < n_parts; ++s2) M = fmaxf(M, sm.gather_lse()[s2][hh]);
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, den = 0.f;
       if (M != -INFINITY) {
-        for (int s2 = 0; s2 < a.n_splits; ++s2) {
-          const float ls = ld_cluster_f32(mapa_cluster(smem_u32(&sm.cl_lse[hh]), s2));
+        for (int s2 = 0; s2 < n_parts; ++s2) {
+          const float ls = sm.gather_lse()[s2][hh];
           if (ls == -INFINITY) continue;
           const float w = exp2f(ls - M);
           den += w;
-          const float4 o0 = ld_cluster_f32x4(mapa_cluster(smem_u32(&sm.cl_o[hh][d0]), s2));
-          const float4 o1 = ld_cluster_f32x4(mapa_cluster(smem_u32(&sm.cl_o[hh][d0 + 4]), s2));
+          const float4 o0 = *reinterpret_cast<const float4*>(&sm.gather_o()[s2][hh][d0]);
+          const float4 o1 = *reinterpret_cast<const float4*>(&sm.gather_o()[s2][hh][d0 + 4]);
           acc[0] += w * o0.x; acc[1] += w * o0.y; acc[2] += w * o0.z; acc[3] += w * o0.w;
           acc[4] += w * o1.x; acc[5] += w * o1.y; acc[6] += w * o1.z; acc[7] += w * o1.w;
         }
@@ -523,7 +555,6 @@ __global__ void __launch_bounds__(kDecThreads, FP8 ? 2 : 1)
         *reinterpret_cast<uint4*>(a.out + orow * kD + d0) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
       }
     }
-    cluster_sync();   // the other CTAs' shared memory stays until CTA 0 has read it
   }
 }
 

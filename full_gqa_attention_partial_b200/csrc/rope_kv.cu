@@ -128,12 +128,21 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
   const int kvh = threadIdx.x >> 5;
   const int d0 = lane32 * 8;
   // jobs token-major: with grid = B (commit) block b takes exactly sequence b's tokens
+  int seen_len = 0, seen_head = 0;   // the cache state this thread read (commit: sequence blockIdx.x's)
+  bool seen = false;
   for (int job = blockIdx.x; job < a.B * n_tok; job += gridDim.x) {
     const int b = job % a.B;
     const int t = a.t_first + job / a.B;
     const int64_t src = (int64_t)b * a.src_bstride + (int64_t)t * a.src_tstride + (int64_t)kvh * a.src_hstride + d0;
+    // the row's K / V loads go out first, with the cache state's: none depends on another
+    uint4 kx = *reinterpret_cast<const uint4*>(a.k + src);
+    const uint4 vx = a.v != nullptr ? *reinterpret_cast<const uint4*>(a.v + src) : make_uint4(0, 0, 0, 0);
     int64_t dst_row;
     const int L = (a.len != nullptr) ? a.len[b] : 0;
+    const int H = a.mode == kDstRing ? a.head[b] : 0;
+    seen_len = L;
+    seen_head = H;
+    seen = true;
     if (a.mode == kDstLinear) {
       if ((int64_t)L + a.T > a.dst_rows) {  // capacity exceeded: leave the sequence unchanged
         if (t == a.t_first && threadIdx.x == 0) raise_err(kErrCapacity);
@@ -141,7 +150,7 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
       }
       dst_row = L + t;
     } else if (a.mode == kDstRing) {
-      const int slot = (a.head[b] + t) % kWindow;
+      const int slot = (H + t) % kWindow;
       dst_row = slot;
       if (threadIdx.x == 0) a.tag[(int64_t)b * kWindow + slot] = L + t;
     } else {
@@ -157,9 +166,6 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
     }
     const int64_t dst = row_id * kD + d0;
 
-    uint4 kx = *reinterpret_cast<const uint4*>(a.k + src);
-    // V's load goes out with K's (independent), not after K's rotation and store
-    const uint4 vx = a.v != nullptr ? *reinterpret_cast<const uint4*>(a.v + src) : make_uint4(0, 0, 0, 0);
     if (!a.src_rotated) {
       const int p = a.pos ? a.pos[(int64_t)b * a.T + t] : L + t;
       __syncthreads();   // the previous job's pairs have been used
@@ -221,11 +227,13 @@ __global__ void __launch_bounds__(128) rope_store_kernel(RopeStoreArgs a) {
     __syncthreads();   // every row of sequence blockIdx.x has read len / head
     if (threadIdx.x == 0 && blockIdx.x < a.B) {
       const int b = blockIdx.x;
+      // the values this thread read above (nothing in this launch writes them before here)
+      const int L = seen ? seen_len : a.len[b];
       if (a.mode == kDstRing) {
-        a.head[b] = (a.head[b] + a.T) % kWindow;
-        a.len[b] += a.T;
-      } else if ((int64_t)a.len[b] + a.T <= a.capacity) {
-        a.len[b] += a.T;
+        a.head[b] = ((seen ? seen_head : a.head[b]) + a.T) % kWindow;
+        a.len[b] = L + a.T;
+      } else if ((int64_t)L + a.T <= a.capacity) {
+        a.len[b] = L + a.T;
       }
     }
   }
