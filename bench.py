@@ -110,9 +110,9 @@ TRAFFIC = {
                                "sources": ["prefill.cu", "common.cuh"]},
     # captured at 16 x 32768 tokens; decode streams each cached byte once, so
     # traffic scales with the tokens: x 8590491648 / 2147483648
-    "decode_full_B16_L131072": {"bytes": 2.1608e9 * 8590491648 / 2147483648, "sha": "0f19a04d16f7b81c",
+    "decode_full_B16_L131072": {"bytes": 2.1600e9 * 8590491648 / 2147483648, "sha": "5a3b85a75e2593a5",
                                 "sources": ["decode.cu", "common.cuh"]},
-    "decode_fp8_full_B16_L131072": {"bytes": 1.1053e9 * 8590491648 / 2147483648, "sha": "0f19a04d16f7b81c",
+    "decode_fp8_full_B16_L131072": {"bytes": 1.1028e9 * 8590491648 / 2147483648, "sha": "5a3b85a75e2593a5",
                                     "sources": ["decode.cu", "common.cuh"]},
 }
 
