@@ -264,3 +264,52 @@ def test_decode_wrappers_reject_shape_mismatches_before_any_launch(hyb, fn):
     for kw in bad:
         with pytest.raises(ValueError):
             go(**kw)
+
+
+def _wave_fill_splits(full: bool, B: int, max_len: int, fp8: bool) -> int:
+    """The decode grid's split count as documented: the smallest count whose
+    CTAs (B x 4 KV heads x splits) fill whole waves of CTA slots (148 SMs; two
+    FP8 CTAs per SM), else the first within 5 % of the best fill, else the best
+    fill; full layers take at most one split per 512 keys (and 1024), ring
+    layers at most 8 (one 64-key stage each)."""
+    keys = max_len if full else 512
+    s_max = max(keys // 512, 1) if full else 8
+    sms = 2 * 148 if fp8 else 148
+    best, best_eff, first95 = 1, 0.0, 0
+    for s in range(1, min(s_max, 1024) + 1):
+        ctas = B * 4 * s
+        waves = -(-ctas // sms)
+        eff = ctas / (waves * sms)
+        if eff >= 0.999:
+            return s
+        if eff >= 0.95 and first95 == 0:
+            first95 = s
+        if eff > best_eff + 1e-9:
+            best_eff, best = eff, s
+    return first95 or best
+
+
+def test_decode_grid_fills_whole_waves(hyb):
+    """The split count behind hyb_attn_decode_workspace_size (the larger of the
+    bf16 and FP8 grids) is the wave-filling one: 74 FP8 / 37 bf16 splits for a
+    batch-1 1M-token full layer (296 / 148 CTAs, one wave each), and the same
+    rule for random batches and lengths."""
+    import random
+
+    def splits_of(lt, B, L):
+        n = hyb.hyb_attn_decode_workspace_size(lt, B, L)
+        rows = B * 16
+        s = (n - ((rows * 4 + 255) // 256) * 256) // (rows * 256 * 4)
+        assert n == rows * s * 256 * 4 + ((rows * s * 4 + 255) // 256) * 256
+        return s
+
+    assert splits_of(hyb.FULL, 1, 1 << 20) == 74
+    assert _wave_fill_splits(True, 1, 1 << 20, False) == 37
+    rnd = random.Random(11)
+    for _ in range(300):
+        lt = rnd.choice([hyb.SLIDING, hyb.FULL])
+        B = rnd.randint(1, 64)
+        L = rnd.randint(1, 1 << 21)
+        full = lt == hyb.FULL
+        want = max(_wave_fill_splits(full, B, L, False), _wave_fill_splits(full, B, L, True))
+        assert splits_of(lt, B, L) == want, (lt, B, L)
